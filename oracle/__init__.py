@@ -1,0 +1,17 @@
+"""fp64 CPU oracle for the Gated DeltaNet recurrence (test infrastructure).
+
+Only the tests, the package smoke check and the benchmark's CPU-baseline leg
+may import this package.  The product path never does; it shares no code with
+the CUDA library.  See gdn_oracle.c for what each function computes and the
+passages it follows.
+"""
+from .oracle import (  # noqa: F401
+    build,
+    conv1d_silu,
+    decode,
+    log_alpha,
+    beta,
+    max_threads,
+    prefill,
+    prefill_chunked,
+)

@@ -1,0 +1,469 @@
+/*
+ * gdn_oracle.c -- fp64 CPU oracle for the Gated DeltaNet recurrence.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path (the CUDA library and
+ * its Python binding) may include, link, load or call this file.  Only the
+ * tests, the package smoke check and the benchmark's CPU-baseline leg use it.
+ * It shares no code, header, table or helper with the CUDA path.
+ *
+ * What it computes, and where the pages say so:
+ *
+ *  - The delta rule.  The Qwen3.8-27B architecture page (2kiu.com, "From
+ *    parameter race to efficiency revolution: dissecting Qwen3.8-27B's dense
+ *    architecture and long-context hybrid attention"), section 2.2, states the
+ *    update S_t = S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T: the value
+ *    stored under key k_t is erased, then v_t is written, with beta_t as the
+ *    write strength.  Section 2.2 also keeps this state in float32
+ *    (mamba_ssm_dtype).
+ *  - The gate.  The same page names A_log, dt_bias, in_proj_a and in_proj_b
+ *    per linear-attention layer (section 2.1) and calls the layer "Gated"
+ *    (section 2.2) but prints no gate formula.  The reading used here: a decay
+ *    alpha_t = exp(-exp(A_log) * softplus(a_t + dt_bias)) scales the whole
+ *    erased state, S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T)
+ *    + beta_t v_t k_t^T, with beta_t = sigmoid(b_t).  With alpha = 1 this is
+ *    exactly the page's rule.
+ *  - Output o_t = scale * S_t q_t from the state after the update, scale =
+ *    1/sqrt(d_k).
+ *  - Heads.  Section 2.1 gives 16 key heads and 48 value heads of width 128
+ *    (linear_num_key_heads / linear_num_value_heads).  Value head h reads key
+ *    head h / (Hv/Hqk) (contiguous groups of three).
+ *  - Front end.  Section 2.1 gives linear_conv_kernel_dim = 4 and a
+ *    conv1d.weight per layer: a causal depthwise 4-tap convolution over time,
+ *    then SiLU on every channel, then q and k are divided by their L2 norm
+ *    per head: y / sqrt(sum y^2 + 1e-6).
+ *
+ * Every function is a plain loop in the order the method states it; nothing is
+ * blocked, fused or reordered.  The only exception is gdn_oracle_prefill_chunked,
+ * which exists to check the chunked (WY / UT) algebra against the plain
+ * recurrence, and is written out step by step from that algebra:
+ *   A_ij = beta_i e^{G_i-G_j} k_i.k_j (j<i),  T = (I+A)^{-1} by forward
+ *   substitution,  W = T diag(beta e^G) K,  U' = T diag(beta) V,
+ *   U = U' - W S0^T,  o = scale (diag(e^G) Q S0^T + (M o QK^T) U),
+ *   S = e^{G_C} S0 + U^T diag(e^{G_C-G}) K,  with G the running sum of
+ *   log(alpha) inside the chunk.
+ *
+ * Inputs q, k, v may be given either as bf16 bit patterns (uint16) or as
+ * float64; bf16 is widened exactly.  All arithmetic is in double.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ---- element fetch: exact widening of bf16 bits or plain f64 ---------------- */
+
+static double bf16_bits_to_f64(uint16_t bits) {
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* copies n contiguous elements starting at element offset off */
+static void fetch(const void* base, int is_f64, int64_t off, int n, double* dst) {
+    if (is_f64) {
+        const double* p = (const double*)base + off;
+        for (int i = 0; i < n; ++i) dst[i] = p[i];
+    } else {
+        const uint16_t* p = (const uint16_t*)base + off;
+        for (int i = 0; i < n; ++i) dst[i] = bf16_bits_to_f64(p[i]);
+    }
+}
+
+/* ---- gates ------------------------------------------------------------------ */
+
+/* softplus(x) = log(1 + e^x), evaluated without overflow */
+static double softplus(double x) {
+    if (x > 0.0) return x + log1p(exp(-x));
+    return log1p(exp(x));
+}
+
+/* log(alpha) = -exp(A_log) * softplus(a + dt_bias) */
+double gdn_oracle_log_alpha(double a, double A_log, double dt_bias) {
+    return -exp(A_log) * softplus(a + dt_bias);
+}
+
+double gdn_oracle_beta(double b) { return 1.0 / (1.0 + exp(-b)); }
+
+/* ---- one recurrence step on one head --------------------------------------- */
+
+/* S (dv x dk, row-major) <- alpha S (I - beta k k^T) + beta v k^T,
+ * then o = scale * S q.  Written as x = S k, S = alpha S + beta (v - alpha x) k^T,
+ * which is the same product expanded. */
+static void delta_step(double* S, int dv, int dk, const double* q, const double* k,
+                       const double* v, double alpha, double beta, double scale,
+                       double* o /* may be NULL */, double* x /* scratch dv */) {
+    for (int i = 0; i < dv; ++i) {
+        double acc = 0.0;
+        for (int j = 0; j < dk; ++j) acc += S[(int64_t)i * dk + j] * k[j];
+        x[i] = acc;
+    }
+    for (int i = 0; i < dv; ++i) {
+        double u = beta * (v[i] - alpha * x[i]);
+        for (int j = 0; j < dk; ++j)
+            S[(int64_t)i * dk + j] = alpha * S[(int64_t)i * dk + j] + u * k[j];
+    }
+    if (o) {
+        for (int i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) acc += S[(int64_t)i * dk + j] * q[j];
+            o[i] = scale * acc;
+        }
+    }
+}
+
+static int set_threads(int threads) {
+#ifdef _OPENMP
+    if (threads > 0) omp_set_num_threads(threads);
+    return omp_get_max_threads();
+#else
+    (void)threads;
+    return 1;
+#endif
+}
+
+int gdn_oracle_max_threads(int threads) { return set_threads(threads); }
+
+/* ---- prefill: the plain sequential recurrence ------------------------------ */
+
+/*
+ * q [T, Hqk, dk], k [T, Hqk, dk], v [T, Hv, dv]   (bf16 bits or f64, see is_f64)
+ * a, b [T, Hv] float;  A_log, dt_bias [Hv] float
+ * cu_seqlens [n_seq + 1] int32 (NULL: one sequence of length T)
+ * initial_state [n_seq, Hv, dv, dk] float (NULL: zeros)
+ * Only value heads h_begin <= h < h_end are computed; nh = h_end - h_begin.
+ * o [T, nh, dv] double (NULL: not written)
+ * final_state [n_seq, nh, dv, dk] double (NULL: not written)
+ * seq_mask [n_seq] (NULL: all sequences) -- sequences with mask 0 are skipped.
+ * Returns 0, or -1 on bad arguments.
+ */
+int gdn_oracle_prefill(const void* q, const void* k, const void* v, int is_f64,
+                       const float* a, const float* b, const float* A_log, const float* dt_bias,
+                       const int32_t* cu_seqlens, int32_t n_seq, int64_t T,
+                       int32_t Hqk, int32_t Hv, int32_t dk, int32_t dv, double scale,
+                       const float* initial_state, int32_t h_begin, int32_t h_end,
+                       const uint8_t* seq_mask, double* o, double* final_state, int threads) {
+    if (Hqk <= 0 || Hv <= 0 || Hv % Hqk || h_begin < 0 || h_end > Hv || h_begin >= h_end)
+        return -1;
+    if (n_seq <= 0 || T < 0) return -1;
+    if (!cu_seqlens && n_seq != 1) return -1;
+    set_threads(threads);
+    const int nh = h_end - h_begin;
+    const int grp = Hv / Hqk;
+    const int64_t units = (int64_t)n_seq * nh;
+    int bad = 0;
+
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t u = 0; u < units; ++u) {
+        const int n = (int)(u / nh);
+        const int hl = (int)(u % nh);
+        const int h = h_begin + hl;
+        const int g = h / grp;
+        if (seq_mask && !seq_mask[n]) continue;
+        const int64_t bos = cu_seqlens ? cu_seqlens[n] : 0;
+        const int64_t eos = cu_seqlens ? cu_seqlens[n + 1] : T;
+        if (bos < 0 || eos < bos || eos > T) { bad = 1; continue; }
+
+        double* S = (double*)calloc((size_t)dv * dk, sizeof(double));
+        double* qt = (double*)malloc(sizeof(double) * dk);
+        double* kt = (double*)malloc(sizeof(double) * dk);
+        double* vt = (double*)malloc(sizeof(double) * dv);
+        double* x = (double*)malloc(sizeof(double) * dv);
+        double* ot = (double*)malloc(sizeof(double) * dv);
+        if (initial_state) {
+            const float* s0 = initial_state + ((int64_t)n * Hv + h) * dv * dk;
+            for (int64_t i = 0; i < (int64_t)dv * dk; ++i) S[i] = s0[i];
+        }
+        for (int64_t t = bos; t < eos; ++t) {
+            fetch(q, is_f64, (t * Hqk + g) * dk, dk, qt);
+            fetch(k, is_f64, (t * Hqk + g) * dk, dk, kt);
+            fetch(v, is_f64, (t * Hv + h) * dv, dv, vt);
+            const double la = gdn_oracle_log_alpha(a[t * Hv + h], A_log[h], dt_bias[h]);
+            const double alpha = exp(la);
+            const double beta = gdn_oracle_beta(b[t * Hv + h]);
+            delta_step(S, dv, dk, qt, kt, vt, alpha, beta, scale, o ? ot : NULL, x);
+            if (o) {
+                double* dst = o + (t * nh + hl) * dv;
+                for (int i = 0; i < dv; ++i) dst[i] = ot[i];
+            }
+        }
+        if (final_state) {
+            double* dst = final_state + ((int64_t)n * nh + hl) * dv * dk;
+            memcpy(dst, S, sizeof(double) * dv * dk);
+        }
+        free(S); free(qt); free(kt); free(vt); free(x); free(ot);
+    }
+    return bad ? -1 : 0;
+}
+
+/* ---- prefill: chunked WY / UT form (checks the chunk algebra only) --------- */
+
+/*
+ * Same arguments as gdn_oracle_prefill plus the chunk length C >= 1.  Chunks
+ * restart at every sequence start; the last chunk of a sequence may be short.
+ */
+int gdn_oracle_prefill_chunked(const void* q, const void* k, const void* v, int is_f64,
+                               const float* a, const float* b, const float* A_log,
+                               const float* dt_bias, const int32_t* cu_seqlens, int32_t n_seq,
+                               int64_t T, int32_t Hqk, int32_t Hv, int32_t dk, int32_t dv,
+                               double scale, const float* initial_state, int32_t h_begin,
+                               int32_t h_end, int32_t C, double* o, double* final_state,
+                               int threads) {
+    if (Hqk <= 0 || Hv <= 0 || Hv % Hqk || h_begin < 0 || h_end > Hv || h_begin >= h_end)
+        return -1;
+    if (n_seq <= 0 || T < 0 || C < 1) return -1;
+    if (!cu_seqlens && n_seq != 1) return -1;
+    set_threads(threads);
+    const int nh = h_end - h_begin;
+    const int grp = Hv / Hqk;
+    const int64_t units = (int64_t)n_seq * nh;
+    int bad = 0;
+
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t u = 0; u < units; ++u) {
+        const int n = (int)(u / nh);
+        const int hl = (int)(u % nh);
+        const int h = h_begin + hl;
+        const int g = h / grp;
+        const int64_t bos = cu_seqlens ? cu_seqlens[n] : 0;
+        const int64_t eos = cu_seqlens ? cu_seqlens[n + 1] : T;
+        if (bos < 0 || eos < bos || eos > T) { bad = 1; continue; }
+
+        double* S = (double*)calloc((size_t)dv * dk, sizeof(double));   /* dv x dk */
+        double* Q = (double*)malloc(sizeof(double) * C * dk);
+        double* K = (double*)malloc(sizeof(double) * C * dk);
+        double* V = (double*)malloc(sizeof(double) * C * dv);
+        double* G = (double*)malloc(sizeof(double) * C);
+        double* be = (double*)malloc(sizeof(double) * C);
+        double* A = (double*)malloc(sizeof(double) * C * C);
+        double* Tm = (double*)malloc(sizeof(double) * C * C);
+        double* W = (double*)malloc(sizeof(double) * C * dk);
+        double* Up = (double*)malloc(sizeof(double) * C * dv);
+        double* U = (double*)malloc(sizeof(double) * C * dv);
+        double* Sn = (double*)malloc(sizeof(double) * dv * dk);
+        if (initial_state) {
+            const float* s0 = initial_state + ((int64_t)n * Hv + h) * dv * dk;
+            for (int64_t i = 0; i < (int64_t)dv * dk; ++i) S[i] = s0[i];
+        }
+        for (int64_t c0 = bos; c0 < eos; c0 += C) {
+            const int L = (int)((eos - c0) < C ? (eos - c0) : C);
+            /* load the chunk and its gates; G = running sum of log(alpha) */
+            double run = 0.0;
+            for (int t = 0; t < L; ++t) {
+                const int64_t tt = c0 + t;
+                fetch(q, is_f64, (tt * Hqk + g) * dk, dk, Q + (int64_t)t * dk);
+                fetch(k, is_f64, (tt * Hqk + g) * dk, dk, K + (int64_t)t * dk);
+                fetch(v, is_f64, (tt * Hv + h) * dv, dv, V + (int64_t)t * dv);
+                run += gdn_oracle_log_alpha(a[tt * Hv + h], A_log[h], dt_bias[h]);
+                G[t] = run;
+                be[t] = gdn_oracle_beta(b[tt * Hv + h]);
+            }
+            /* A_ij = beta_i e^{G_i - G_j} (k_i . k_j) for j < i, else 0 */
+            for (int i = 0; i < L; ++i)
+                for (int j = 0; j < L; ++j) {
+                    double val = 0.0;
+                    if (j < i) {
+                        double kk = 0.0;
+                        for (int e = 0; e < dk; ++e) kk += K[(int64_t)i * dk + e] * K[(int64_t)j * dk + e];
+                        val = be[i] * exp(G[i] - G[j]) * kk;
+                    }
+                    A[i * C + j] = val;
+                }
+            /* T = (I + A)^{-1}, lower unit triangular, by forward substitution:
+             * row i of T is e_i - sum_{m<i} A_im T_m */
+            for (int i = 0; i < L; ++i)
+                for (int j = 0; j < L; ++j) {
+                    double val = (i == j) ? 1.0 : 0.0;
+                    for (int m = j; m < i; ++m) val -= A[i * C + m] * Tm[m * C + j];
+                    Tm[i * C + j] = (j <= i) ? val : 0.0;
+                }
+            /* W = T diag(beta e^G) K ;  U' = T diag(beta) V */
+            for (int i = 0; i < L; ++i) {
+                for (int e = 0; e < dk; ++e) {
+                    double acc = 0.0;
+                    for (int j = 0; j <= i; ++j)
+                        acc += Tm[i * C + j] * be[j] * exp(G[j]) * K[(int64_t)j * dk + e];
+                    W[(int64_t)i * dk + e] = acc;
+                }
+                for (int e = 0; e < dv; ++e) {
+                    double acc = 0.0;
+                    for (int j = 0; j <= i; ++j) acc += Tm[i * C + j] * be[j] * V[(int64_t)j * dv + e];
+                    Up[(int64_t)i * dv + e] = acc;
+                }
+            }
+            /* U = U' - W S0^T   (S0 is dv x dk, so (W S0^T)_{i,e} = sum_f W_if S0_ef) */
+            for (int i = 0; i < L; ++i)
+                for (int e = 0; e < dv; ++e) {
+                    double acc = 0.0;
+                    for (int f = 0; f < dk; ++f) acc += W[(int64_t)i * dk + f] * S[(int64_t)e * dk + f];
+                    U[(int64_t)i * dv + e] = Up[(int64_t)i * dv + e] - acc;
+                }
+            /* o_i = scale (e^{G_i} S0 q_i + sum_{j<=i} e^{G_i-G_j} (q_i . k_j) u_j) */
+            if (o) {
+                for (int i = 0; i < L; ++i) {
+                    double* dst = o + ((c0 + i) * nh + hl) * dv;
+                    for (int e = 0; e < dv; ++e) {
+                        double inter = 0.0;
+                        for (int f = 0; f < dk; ++f) inter += S[(int64_t)e * dk + f] * Q[(int64_t)i * dk + f];
+                        double intra = 0.0;
+                        for (int j = 0; j <= i; ++j) {
+                            double qk = 0.0;
+                            for (int f = 0; f < dk; ++f) qk += Q[(int64_t)i * dk + f] * K[(int64_t)j * dk + f];
+                            intra += exp(G[i] - G[j]) * qk * U[(int64_t)j * dv + e];
+                        }
+                        dst[e] = scale * (exp(G[i]) * inter + intra);
+                    }
+                }
+            }
+            /* S = e^{G_L} S0 + sum_j e^{G_L - G_j} u_j k_j^T */
+            const double GL = G[L - 1];
+            for (int e = 0; e < dv; ++e)
+                for (int f = 0; f < dk; ++f) {
+                    double acc = exp(GL) * S[(int64_t)e * dk + f];
+                    for (int j = 0; j < L; ++j)
+                        acc += exp(GL - G[j]) * U[(int64_t)j * dv + e] * K[(int64_t)j * dk + f];
+                    Sn[(int64_t)e * dk + f] = acc;
+                }
+            memcpy(S, Sn, sizeof(double) * dv * dk);
+        }
+        if (final_state) {
+            double* dst = final_state + ((int64_t)n * nh + hl) * dv * dk;
+            memcpy(dst, S, sizeof(double) * dv * dk);
+        }
+        free(S); free(Q); free(K); free(V); free(G); free(be); free(A); free(Tm);
+        free(W); free(Up); free(U); free(Sn);
+    }
+    return bad ? -1 : 0;
+}
+
+/* ---- decode: one recurrence step per (sequence, layer) unit ---------------- */
+
+/*
+ * Units u = s * L + l for sequence s < n_seq and layer l < L.
+ * q, k [U, Hqk, dk]; v [U, Hv, dv] (bf16 bits or f64); a, b [U, Hv] float;
+ * A_log, dt_bias [L, Hv] float; state [U, Hv, dv, dk] float (read only here).
+ * units_sel [n_sel] lists the units to compute (NULL: all units, n_sel = U).
+ * o [n_sel, Hv, dv] double; state_out [n_sel, Hv, dv, dk] double (either may be NULL).
+ */
+int gdn_oracle_decode(const void* q, const void* k, const void* v, int is_f64, const float* a,
+                      const float* b, const float* A_log, const float* dt_bias, int32_t n_seq,
+                      int32_t L, int32_t Hqk, int32_t Hv, int32_t dk, int32_t dv, double scale,
+                      const float* state, const int64_t* units_sel, int64_t n_sel, double* o,
+                      double* state_out, int threads) {
+    if (Hqk <= 0 || Hv <= 0 || Hv % Hqk || n_seq <= 0 || L <= 0) return -1;
+    const int64_t U = (int64_t)n_seq * L;
+    if (!units_sel) n_sel = U;
+    set_threads(threads);
+    const int grp = Hv / Hqk;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t w = 0; w < n_sel * Hv; ++w) {
+        const int64_t si = w / Hv;
+        const int h = (int)(w % Hv);
+        const int64_t u = units_sel ? units_sel[si] : si;
+        if (u < 0 || u >= U) { bad = 1; continue; }
+        const int l = (int)(u % L);
+        const int g = h / grp;
+        double* S = (double*)malloc(sizeof(double) * dv * dk);
+        double* qt = (double*)malloc(sizeof(double) * dk);
+        double* kt = (double*)malloc(sizeof(double) * dk);
+        double* vt = (double*)malloc(sizeof(double) * dv);
+        double* x = (double*)malloc(sizeof(double) * dv);
+        double* ot = (double*)malloc(sizeof(double) * dv);
+        const float* s0 = state + (u * Hv + h) * (int64_t)dv * dk;
+        for (int64_t i = 0; i < (int64_t)dv * dk; ++i) S[i] = s0[i];
+        fetch(q, is_f64, (u * Hqk + g) * dk, dk, qt);
+        fetch(k, is_f64, (u * Hqk + g) * dk, dk, kt);
+        fetch(v, is_f64, (u * Hv + h) * dv, dv, vt);
+        const double alpha = exp(gdn_oracle_log_alpha(a[u * Hv + h], A_log[l * Hv + h], dt_bias[l * Hv + h]));
+        const double beta = gdn_oracle_beta(b[u * Hv + h]);
+        delta_step(S, dv, dk, qt, kt, vt, alpha, beta, scale, ot, x);
+        if (o) memcpy(o + (si * Hv + h) * dv, ot, sizeof(double) * dv);
+        if (state_out) memcpy(state_out + (si * Hv + h) * (int64_t)dv * dk, S, sizeof(double) * dv * dk);
+        free(S); free(qt); free(kt); free(vt); free(x); free(ot);
+    }
+    return bad ? -1 : 0;
+}
+
+/* ---- front end: causal depthwise 4-tap conv, SiLU, per-head L2 norm -------- */
+
+/*
+ * x [T, Ctot] bf16 bits, channels ordered [q heads | k heads | v heads], each
+ * head d channels wide, Ctot = (2 Hqk + Hv) d.  w [Ctot, 4] float; tap j
+ * multiplies x[t - 3 + j] (tap 3 is the current token).  History before a
+ * sequence start is conv_state_in[n, c, 0..2] = x[bos-3 .. bos-1] (NULL: zeros);
+ * no history crosses a cu_seqlens boundary.
+ * Outputs (double): q [T, Hqk, d], k [T, Hqk, d], v [T, Hv, d] (any may be NULL),
+ * conv_state_out [n_seq, Ctot, 3] = the last three inputs of each sequence,
+ * oldest first (NULL: not written).
+ */
+int gdn_oracle_conv1d_silu(const uint16_t* x, const float* w, const int32_t* cu_seqlens,
+                           int32_t n_seq, int64_t T, int32_t Hqk, int32_t Hv, int32_t d,
+                           const float* conv_state_in, double* q, double* k, double* v,
+                           double* conv_state_out, int threads) {
+    if (Hqk <= 0 || Hv <= 0 || d <= 0 || n_seq <= 0 || T < 0) return -1;
+    if (!cu_seqlens && n_seq != 1) return -1;
+    set_threads(threads);
+    const int64_t Ctot = (int64_t)(2 * Hqk + Hv) * d;
+    const int64_t n_heads = 2 * Hqk + Hv;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t u = 0; u < (int64_t)n_seq * n_heads; ++u) {
+        const int n = (int)(u / n_heads);
+        const int hh = (int)(u % n_heads);          /* head index in the packed order */
+        const int64_t bos = cu_seqlens ? cu_seqlens[n] : 0;
+        const int64_t eos = cu_seqlens ? cu_seqlens[n + 1] : T;
+        if (bos < 0 || eos < bos || eos > T) { bad = 1; continue; }
+        double* y = (double*)malloc(sizeof(double) * d);
+        for (int64_t t = bos; t < eos; ++t) {
+            double ss = 0.0;
+            for (int e = 0; e < d; ++e) {
+                const int64_t c = (int64_t)hh * d + e;
+                double acc = 0.0;
+                for (int j = 0; j < 4; ++j) {
+                    const int64_t tau = t - 3 + j;
+                    double xv;
+                    if (tau >= bos) xv = bf16_bits_to_f64(x[tau * Ctot + c]);
+                    else {
+                        /* position bos - m (m = 1..3) is history slot 3 - m */
+                        const int64_t m = bos - tau;
+                        xv = conv_state_in ? conv_state_in[((int64_t)n * Ctot + c) * 3 + (3 - m)] : 0.0;
+                    }
+                    acc += (double)w[c * 4 + j] * xv;
+                }
+                const double s = acc / (1.0 + exp(-acc));   /* SiLU */
+                y[e] = s;
+                ss += s * s;
+            }
+            if (hh < 2 * Hqk) {
+                const double inv = 1.0 / sqrt(ss + 1e-6);
+                for (int e = 0; e < d; ++e) y[e] *= inv;
+            }
+            double* dst;
+            if (hh < Hqk) dst = q ? q + (t * Hqk + hh) * d : NULL;
+            else if (hh < 2 * Hqk) dst = k ? k + (t * Hqk + (hh - Hqk)) * d : NULL;
+            else dst = v ? v + (t * Hv + (hh - 2 * Hqk)) * d : NULL;
+            if (dst) memcpy(dst, y, sizeof(double) * d);
+        }
+        if (conv_state_out) {
+            for (int e = 0; e < d; ++e) {
+                const int64_t c = (int64_t)hh * d + e;
+                for (int s = 0; s < 3; ++s) {
+                    const int64_t tau = eos - 3 + s;
+                    double xv;
+                    if (tau >= bos) xv = bf16_bits_to_f64(x[tau * Ctot + c]);
+                    else {
+                        const int64_t m = bos - tau;
+                        xv = conv_state_in ? conv_state_in[((int64_t)n * Ctot + c) * 3 + (3 - m)] : 0.0;
+                    }
+                    conv_state_out[((int64_t)n * Ctot + c) * 3 + s] = xv;
+                }
+            }
+        }
+        free(y);
+    }
+    return bad ? -1 : 0;
+}

@@ -1,0 +1,207 @@
+"""ctypes wrapper of the fp64 oracle (numpy in, numpy out)."""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+_i32p = np.ctypeslib.ndpointer(np.int32, flags="C_CONTIGUOUS")
+
+
+def _ptr(x):
+    return None if x is None else x.ctypes.data_as(C.c_void_p)
+
+
+def build(force: bool = False, path: str | None = None):
+    """Compile and load the oracle library.  `path` loads another build of the
+    same source (used by the tests that plant mistakes in a copy)."""
+    global _lib
+    if path is not None:
+        return _bind(C.CDLL(path))
+    _lib = _bind(C.CDLL(_build.build(force=force)))
+    return _lib
+
+
+def _bind(lib):
+    vp, i32, i64, dbl = C.c_void_p, C.c_int32, C.c_int64, C.c_double
+    lib.gdn_oracle_prefill.restype = C.c_int
+    lib.gdn_oracle_prefill.argtypes = [vp, vp, vp, C.c_int, vp, vp, vp, vp, vp, i32, i64,
+                                       i32, i32, i32, i32, dbl, vp, i32, i32, vp, vp, vp, C.c_int]
+    lib.gdn_oracle_prefill_chunked.restype = C.c_int
+    lib.gdn_oracle_prefill_chunked.argtypes = [vp, vp, vp, C.c_int, vp, vp, vp, vp, vp, i32, i64,
+                                               i32, i32, i32, i32, dbl, vp, i32, i32, i32, vp, vp,
+                                               C.c_int]
+    lib.gdn_oracle_decode.restype = C.c_int
+    lib.gdn_oracle_decode.argtypes = [vp, vp, vp, C.c_int, vp, vp, vp, vp, i32, i32, i32, i32,
+                                      i32, i32, dbl, vp, vp, i64, vp, vp, C.c_int]
+    lib.gdn_oracle_conv1d_silu.restype = C.c_int
+    lib.gdn_oracle_conv1d_silu.argtypes = [vp, vp, vp, i32, i64, i32, i32, i32, vp, vp, vp, vp,
+                                           vp, C.c_int]
+    lib.gdn_oracle_log_alpha.restype = dbl
+    lib.gdn_oracle_log_alpha.argtypes = [dbl, dbl, dbl]
+    lib.gdn_oracle_beta.restype = dbl
+    lib.gdn_oracle_beta.argtypes = [dbl]
+    lib.gdn_oracle_max_threads.restype = C.c_int
+    lib.gdn_oracle_max_threads.argtypes = [C.c_int]
+    return lib
+
+
+def _L(lib=None):
+    global _lib
+    if lib is not None:
+        return lib
+    if _lib is None:
+        build()
+    return _lib
+
+
+def _qkv(x):
+    """bf16 bits (uint16) pass through; anything else becomes float64."""
+    if x.dtype == np.uint16:
+        return np.ascontiguousarray(x), 0
+    return np.ascontiguousarray(x, dtype=np.float64), 1
+
+
+def _f32(x):
+    return None if x is None else np.ascontiguousarray(x, dtype=np.float32)
+
+
+def max_threads(threads: int = 0, lib=None) -> int:
+    return _L(lib).gdn_oracle_max_threads(int(threads))
+
+
+def log_alpha(a, A_log, dt_bias, lib=None) -> float:
+    return _L(lib).gdn_oracle_log_alpha(float(a), float(A_log), float(dt_bias))
+
+
+def beta(b, lib=None) -> float:
+    return _L(lib).gdn_oracle_beta(float(b))
+
+
+def _prefill_common(q, k, v, a, b, A_log, dt_bias, cu_seqlens, initial_state, heads):
+    q, isf = _qkv(q)
+    k, isf2 = _qkv(k)
+    v, isf3 = _qkv(v)
+    if not (isf == isf2 == isf3):
+        raise TypeError("q, k, v must all be bf16 bits or all float")
+    T, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    cu = None if cu_seqlens is None else np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    n_seq = 1 if cu is None else len(cu) - 1
+    h0, h1 = (0, Hv) if heads is None else (int(heads[0]), int(heads[1]))
+    return (q, k, v, isf, _f32(a), _f32(b), _f32(A_log), _f32(dt_bias), cu, n_seq, T, Hqk, Hv,
+            dk, dv, _f32(initial_state), h0, h1)
+
+
+def prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens=None, scale=None, initial_state=None,
+            heads=None, seq_mask=None, want_o=True, want_state=True, threads=0, lib=None):
+    """Sequential fp64 recurrence.  Returns (o [T, nh, dv] or None,
+    final_state [N, nh, dv, dk] or None) for value heads in range `heads`."""
+    (q, k, v, isf, a, b, A_log, dt_bias, cu, n_seq, T, Hqk, Hv, dk, dv, s0, h0, h1) = \
+        _prefill_common(q, k, v, a, b, A_log, dt_bias, cu_seqlens, initial_state, heads)
+    scale = 1.0 / np.sqrt(dk) if scale is None else float(scale)
+    nh = h1 - h0
+    o = np.zeros((T, nh, dv), np.float64) if want_o else None
+    fs = np.zeros((n_seq, nh, dv, dk), np.float64) if want_state else None
+    mask = None if seq_mask is None else np.ascontiguousarray(seq_mask, dtype=np.uint8)
+    rc = _L(lib).gdn_oracle_prefill(_ptr(q), _ptr(k), _ptr(v), isf, _ptr(a), _ptr(b), _ptr(A_log),
+                                    _ptr(dt_bias), _ptr(cu), n_seq, T, Hqk, Hv, dk, dv, scale,
+                                    _ptr(s0), h0, h1, _ptr(mask), _ptr(o), _ptr(fs), int(threads))
+    if rc != 0:
+        raise ValueError("oracle prefill rejected its arguments")
+    return o, fs
+
+
+def prefill_chunked(q, k, v, a, b, A_log, dt_bias, cu_seqlens=None, scale=None,
+                    initial_state=None, heads=None, chunk=64, threads=0, lib=None):
+    """fp64 chunked WY/UT form; same outputs as prefill()."""
+    (q, k, v, isf, a, b, A_log, dt_bias, cu, n_seq, T, Hqk, Hv, dk, dv, s0, h0, h1) = \
+        _prefill_common(q, k, v, a, b, A_log, dt_bias, cu_seqlens, initial_state, heads)
+    scale = 1.0 / np.sqrt(dk) if scale is None else float(scale)
+    nh = h1 - h0
+    o = np.zeros((T, nh, dv), np.float64)
+    fs = np.zeros((n_seq, nh, dv, dk), np.float64)
+    rc = _L(lib).gdn_oracle_prefill_chunked(_ptr(q), _ptr(k), _ptr(v), isf, _ptr(a), _ptr(b),
+                                            _ptr(A_log), _ptr(dt_bias), _ptr(cu), n_seq, T, Hqk,
+                                            Hv, dk, dv, scale, _ptr(s0), h0, h1, int(chunk),
+                                            _ptr(o), _ptr(fs), int(threads))
+    if rc != 0:
+        raise ValueError("oracle chunked prefill rejected its arguments")
+    return o, fs
+
+
+def decode(q, k, v, a, b, A_log, dt_bias, n_seq, layers, state, units=None, scale=None,
+           threads=0, lib=None):
+    """One step for the listed units.  `state` is float32 [len(units) or U, Hv, dv, dk]:
+    when `units` is given, state[i] is the state of unit units[i].
+    Returns (o [n, Hv, dv], state_out [n, Hv, dv, dk]) in float64."""
+    q, isf = _qkv(q)
+    k, _ = _qkv(k)
+    v, _ = _qkv(v)
+    Hqk, dk = q.shape[1], q.shape[2]
+    Hv, dv = v.shape[1], v.shape[2]
+    scale = 1.0 / np.sqrt(dk) if scale is None else float(scale)
+    state = _f32(state)
+    U = n_seq * layers
+    if units is None:
+        sel, n = None, U
+        st_full = state
+    else:
+        sel = np.ascontiguousarray(units, dtype=np.int64)
+        n = len(sel)
+        # the C side indexes state by unit: scatter the given states into a
+        # sparse full-size view is too large, so remap units to 0..n-1 instead
+        st_full = None
+    o = np.zeros((n, Hv, dv), np.float64)
+    so = np.zeros((n, Hv, dv, dk), np.float64)
+    lib_ = _L(lib)
+    if sel is None:
+        rc = lib_.gdn_oracle_decode(_ptr(q), _ptr(k), _ptr(v), isf, _ptr(_f32(a)), _ptr(_f32(b)),
+                                    _ptr(_f32(A_log)), _ptr(_f32(dt_bias)), n_seq, layers, Hqk, Hv,
+                                    dk, dv, scale, _ptr(st_full), None, n, _ptr(o), _ptr(so),
+                                    int(threads))
+    else:
+        # gather the selected units into a compact problem whose unit i has the
+        # same layer as units[i]: one sequence per selected unit, all layers'
+        # gate parameters kept, per-unit inputs gathered.
+        rc = 0
+        a32, b32 = _f32(a), _f32(b)
+        for i, u in enumerate(sel):
+            l = int(u % layers)
+            # a one-unit problem with layers=1 and this layer's parameters
+            r = lib_.gdn_oracle_decode(
+                _ptr(np.ascontiguousarray(q[u:u + 1])), _ptr(np.ascontiguousarray(k[u:u + 1])),
+                _ptr(np.ascontiguousarray(v[u:u + 1])), isf,
+                _ptr(np.ascontiguousarray(a32[u:u + 1])), _ptr(np.ascontiguousarray(b32[u:u + 1])),
+                _ptr(np.ascontiguousarray(_f32(A_log)[l:l + 1])),
+                _ptr(np.ascontiguousarray(_f32(dt_bias)[l:l + 1])), 1, 1, Hqk, Hv, dk, dv, scale,
+                _ptr(np.ascontiguousarray(state[i:i + 1])), None, 1,
+                _ptr(o[i:i + 1]), _ptr(so[i:i + 1]), int(threads))
+            rc |= r
+    if rc != 0:
+        raise ValueError("oracle decode rejected its arguments")
+    return o, so
+
+
+def conv1d_silu(qkv, conv_w, cu_seqlens=None, Hqk=16, Hv=48, d=128, conv_state=None,
+                threads=0, lib=None):
+    """Front end in fp64.  Returns (q [T,Hqk,d], k [T,Hqk,d], v [T,Hv,d], conv_state_out)."""
+    x = np.ascontiguousarray(qkv, dtype=np.uint16)
+    T = x.shape[0]
+    cu = None if cu_seqlens is None else np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    n_seq = 1 if cu is None else len(cu) - 1
+    ctot = (2 * Hqk + Hv) * d
+    q = np.zeros((T, Hqk, d), np.float64)
+    k = np.zeros((T, Hqk, d), np.float64)
+    v = np.zeros((T, Hv, d), np.float64)
+    cso = np.zeros((n_seq, ctot, 3), np.float64)
+    rc = _L(lib).gdn_oracle_conv1d_silu(_ptr(x), _ptr(_f32(conv_w)), _ptr(cu), n_seq, T, Hqk, Hv,
+                                        d, _ptr(_f32(conv_state)), _ptr(q), _ptr(k), _ptr(v),
+                                        _ptr(cso), int(threads))
+    if rc != 0:
+        raise ValueError("oracle conv1d_silu rejected its arguments")
+    return q, k, v, cso

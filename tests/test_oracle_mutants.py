@@ -1,0 +1,90 @@
+"""The pins must catch plausible mistakes in the oracle.
+
+Each case copies the oracle's C source, plants one mistake (a dropped term, a
+wrong sign, index or operand), builds the copy on the CPU and runs every pin of
+test_oracle_pins against it: at least one pin must fail.  The oracle itself is
+never modified.
+"""
+import functools
+import inspect
+import os
+import shutil
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import oracle as _oracle_mod
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "gdn_oracle.c")
+
+MUTANTS = {
+    "decay_not_on_erase": ("beta * (v[i] - alpha * x[i])", "beta * (v[i] - x[i])"),
+    "decay_not_on_state": ("alpha * S[(int64_t)i * dk + j] + u * k[j]", "S[(int64_t)i * dk + j] + u * k[j]"),
+    "write_sign": ("double u = beta * (v[i] - alpha * x[i]);", "double u = beta * (v[i] + alpha * x[i]);"),
+    "key_head_modulo": ("const int g = h / grp;\n        if (seq_mask", "const int g = h % Hqk;\n        if (seq_mask"),
+    "softplus_branch": ("return x + log1p(exp(-x));", "return x + log1p(exp(x));"),
+    "beta_sign": ("return 1.0 / (1.0 + exp(-b));", "return 1.0 / (1.0 + exp(b));"),
+    "gate_rate_not_exp": ("return -exp(A_log) * softplus(a + dt_bias);", "return -A_log * softplus(a + dt_bias);"),
+    "output_unscaled": ("o[i] = scale * acc;", "o[i] = acc;"),
+    "conv_taps_reversed": ("acc += (double)w[c * 4 + j] * xv;", "acc += (double)w[c * 4 + (3 - j)] * xv;"),
+    "l2_no_eps": ("1.0 / sqrt(ss + 1e-6)", "1.0 / sqrt(ss)"),
+    "silu_sign": ("acc / (1.0 + exp(-acc))", "acc / (1.0 + exp(acc))"),
+    "chunk_u_sign": ("Up[(int64_t)i * dv + e] - acc;", "Up[(int64_t)i * dv + e] + acc;"),
+    "chunk_no_decay_in_A": ("val = be[i] * exp(G[i] - G[j]) * kk;", "val = be[i] * kk;"),
+    "chunk_W_no_gamma": ("acc += Tm[i * C + j] * be[j] * exp(G[j]) * K[(int64_t)j * dk + e];",
+                         "acc += Tm[i * C + j] * be[j] * K[(int64_t)j * dk + e];"),
+    "chunk_state_no_decay": ("double acc = exp(GL) * S[(int64_t)e * dk + f];",
+                             "double acc = S[(int64_t)e * dk + f];"),
+    "chunk_inter_no_gamma": ("dst[e] = scale * (exp(G[i]) * inter + intra);",
+                             "dst[e] = scale * (inter + intra);"),
+    "chunk_substitution_sign": ("val -= A[i * C + m] * Tm[m * C + j];", "val += A[i * C + m] * Tm[m * C + j];"),
+}
+
+
+class _Bound:
+    """The oracle module's functions bound to another build of the library."""
+
+    def __init__(self, lib):
+        self._lib = lib
+
+    def __getattr__(self, name):
+        return functools.partial(getattr(_oracle_mod, name), lib=self._lib)
+
+
+def _pin_functions():
+    out = []
+    for name, fn in inspect.getmembers(pins, inspect.isfunction):
+        if not name.startswith("test_"):
+            continue
+        params = inspect.signature(fn).parameters
+        if "C" in params:
+            for C in (1, 16):
+                out.append((f"{name}[{C}]", functools.partial(fn, C=C)))
+        else:
+            out.append((name, fn))
+    return out
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) >= 1, f"mutation site for {name} not found"
+    mutated = src.replace(old, new, 1)
+    csrc = tmp_path / "mut.c"
+    csrc.write_text(mutated)
+    lib_path = str(tmp_path / "libmut.so")
+    subprocess.run(["gcc", "-O1", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-o", lib_path,
+                    str(csrc), "-lm"], check=True)
+    bound = _Bound(oracle.build(path=lib_path))
+    failed = []
+    for pin_name, fn in _pin_functions():
+        try:
+            with np.errstate(all="ignore"):
+                fn(bound)
+        except (AssertionError, ValueError):
+            failed.append(pin_name)
+    assert failed, f"no pin catches the planted mistake {name}"

@@ -1,0 +1,389 @@
+"""Pins for the fp64 oracle: checks against facts that do not come from the
+oracle itself (CPU only).
+
+- The unrolled-product form of the recurrence, evaluated with explicit matrix
+  products (brute force on tiny inputs).
+- Invariants of the delta rule: retrieval (alpha = beta = 1, unit key:
+  S_t k_t = v_t), no write (beta = 0), pure decay, orthonormal keys, alpha = 0,
+  superposition, and the ungated rule of the Qwen3.8-27B architecture page
+  (2kiu.com), section 2.2, when alpha = 1.
+- Closed forms of the gates.
+- The chunked WY/UT algebra against the recurrence.
+- The front end against a library convolution and special tap patterns.
+"""
+import math
+
+import numpy as np
+import pytest
+
+
+def _gates(a, b, A_log, dt_bias):
+    """alpha, beta for per-token a, b [T, Hv] and per-head A_log, dt_bias [Hv]."""
+    x = a + dt_bias[None, :]
+    sp = np.where(x > 0, x + np.log1p(np.exp(-np.abs(x))), np.log1p(np.exp(np.minimum(x, 0))))
+    alpha = np.exp(-np.exp(A_log)[None, :] * sp)
+    beta = 1.0 / (1.0 + np.exp(-b))
+    return alpha, beta
+
+
+def _brute(q, k, v, alpha, beta, S0, scale):
+    """Unrolled product form for one head: S_t = S0 P_1..P_t + sum_j beta_j v_j k_j^T
+    P_{j+1}..P_t with P_s = alpha_s (I - beta_s k_s k_s^T).  Returns (o [T, dv], S_T)."""
+    T, dk = k.shape
+    I = np.eye(dk)
+    P = [alpha[s] * (I - beta[s] * np.outer(k[s], k[s])) for s in range(T)]
+    outs = []
+    S_t = S0
+    for t in range(T):
+        S_t = S0 @ _chain(P, 0, t + 1)
+        for j in range(t + 1):
+            S_t = S_t + beta[j] * np.outer(v[j], k[j]) @ _chain(P, j + 1, t + 1)
+        outs.append(scale * S_t @ q[t])
+    return np.array(outs), S_t
+
+
+def _chain(P, lo, hi):
+    out = np.eye(P[0].shape[0])
+    for s in range(lo, hi):
+        out = out @ P[s]
+    return out
+
+
+def _rand_case(rng, T, Hqk, Hv, dk, dv, unit_keys=False):
+    q = rng.standard_normal((T, Hqk, dk))
+    k = rng.standard_normal((T, Hqk, dk))
+    if unit_keys:
+        k /= np.linalg.norm(k, axis=-1, keepdims=True)
+        q /= np.linalg.norm(q, axis=-1, keepdims=True)
+    v = rng.standard_normal((T, Hv, dv))
+    a = rng.standard_normal((T, Hv)).astype(np.float32)
+    b = rng.standard_normal((T, Hv)).astype(np.float32)
+    A_log = np.log(rng.uniform(1, 16, Hv)).astype(np.float32)
+    dt = np.exp(rng.uniform(np.log(1e-3), np.log(0.1), Hv))
+    dt_bias = np.log(np.expm1(dt)).astype(np.float32)
+    return q, k, v, a, b, A_log, dt_bias
+
+
+def test_brute_force_unrolled_product(orc):
+    """Every prefix output and the final state equal the explicit product form;
+    value head h reads key head h // 3 (6 value heads over 2 key heads)."""
+    rng = np.random.default_rng(11)
+    T, Hqk, Hv, dk, dv = 9, 2, 6, 5, 4
+    q, k, v, a, b, A_log, dt_bias = _rand_case(rng, T, Hqk, Hv, dk, dv)
+    S0 = (0.3 * rng.standard_normal((1, Hv, dv, dk))).astype(np.float32)
+    scale = 0.37
+    o, fs = orc.prefill(q, k, v, a, b, A_log, dt_bias, scale=scale, initial_state=S0)
+    alpha, beta = _gates(a.astype(np.float64), b.astype(np.float64),
+                         A_log.astype(np.float64), dt_bias.astype(np.float64))
+    for h in range(Hv):
+        g = h // 3
+        ob, Sb = _brute(q[:, g], k[:, g], v[:, h], alpha[:, h], beta[:, h],
+                        S0[0, h].astype(np.float64), scale)
+        np.testing.assert_allclose(o[:, h], ob, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(fs[0, h], Sb, rtol=0, atol=1e-12)
+
+
+def test_retrieval_invariant(orc):
+    """alpha = beta = 1 and unit keys: after writing v_t under k_t, reading with
+    q_t = k_t returns v_t exactly (up to fp64 rounding)."""
+    rng = np.random.default_rng(3)
+    T, dk, dv = 40, 16, 8
+    k = rng.standard_normal((T, 1, dk))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    v = rng.standard_normal((T, 1, dv))
+    a = np.full((T, 1), -np.inf, np.float32)          # softplus(-inf) = 0 -> alpha = 1
+    b = np.full((T, 1), np.inf, np.float32)           # sigmoid(inf) = 1
+    S0 = rng.standard_normal((1, 1, dv, dk)).astype(np.float32)
+    o, fs = orc.prefill(k, k, v, a, b, np.zeros(1, np.float32), np.zeros(1, np.float32),
+                        scale=1.0, initial_state=S0)
+    np.testing.assert_allclose(o[:, 0], v[:, 0], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(fs[0, 0] @ k[-1, 0], v[-1, 0], rtol=0, atol=1e-13)
+
+
+def test_no_write_keeps_state(orc):
+    """beta = 0, alpha = 1: the state is unchanged and o_t = scale S0 q_t."""
+    rng = np.random.default_rng(4)
+    T, dk, dv = 17, 8, 6
+    q = rng.standard_normal((T, 1, dk))
+    k = rng.standard_normal((T, 1, dk))
+    v = rng.standard_normal((T, 1, dv))
+    a = np.full((T, 1), -np.inf, np.float32)
+    b = np.full((T, 1), -np.inf, np.float32)
+    S0 = rng.standard_normal((1, 1, dv, dk)).astype(np.float32)
+    o, fs = orc.prefill(q, k, v, a, b, np.zeros(1, np.float32), np.zeros(1, np.float32),
+                        scale=0.5, initial_state=S0)
+    np.testing.assert_array_equal(fs[0, 0], S0[0, 0].astype(np.float64))
+    np.testing.assert_allclose(o[:, 0], 0.5 * q[:, 0] @ S0[0, 0].astype(np.float64).T,
+                               rtol=0, atol=1e-13)
+
+
+def test_pure_decay(orc):
+    """beta = 0 and a + dt_bias = 0, A_log = 0: alpha = exp(-ln 2) = 1/2 per token,
+    so S_T = 2^-T S0."""
+    rng = np.random.default_rng(5)
+    T, dk, dv = 13, 4, 3
+    q = rng.standard_normal((T, 1, dk))
+    k = rng.standard_normal((T, 1, dk))
+    v = rng.standard_normal((T, 1, dv))
+    a = np.zeros((T, 1), np.float32)
+    b = np.full((T, 1), -np.inf, np.float32)
+    S0 = rng.standard_normal((1, 1, dv, dk)).astype(np.float32)
+    _, fs = orc.prefill(q, k, v, a, b, np.zeros(1, np.float32), np.zeros(1, np.float32),
+                        initial_state=S0)
+    np.testing.assert_allclose(fs[0, 0], S0[0, 0] * 2.0 ** -T, rtol=1e-14, atol=0)
+
+
+def test_orthonormal_keys_write_columns(orc):
+    """alpha = beta = 1, zero S0, keys e_1..e_d: column t of S_T is v_t (the
+    textbook associative-memory write)."""
+    rng = np.random.default_rng(6)
+    d = 8
+    k = np.eye(d)[:, None, :]
+    v = rng.standard_normal((d, 1, d))
+    a = np.full((d, 1), -np.inf, np.float32)
+    b = np.full((d, 1), np.inf, np.float32)
+    _, fs = orc.prefill(k, k, v, a, b, np.zeros(1, np.float32), np.zeros(1, np.float32))
+    np.testing.assert_allclose(fs[0, 0], v[:, 0].T, rtol=0, atol=1e-15)
+
+
+def test_alpha_zero_forgets(orc):
+    """alpha = 0 (a = +inf): S_t = beta_t v_t k_t^T, whatever came before."""
+    rng = np.random.default_rng(7)
+    T, dk, dv = 6, 5, 4
+    q = rng.standard_normal((T, 1, dk))
+    k = rng.standard_normal((T, 1, dk))
+    v = rng.standard_normal((T, 1, dv))
+    a = np.full((T, 1), np.inf, np.float32)
+    b = rng.standard_normal((T, 1)).astype(np.float32)
+    S0 = rng.standard_normal((1, 1, dv, dk)).astype(np.float32)
+    o, fs = orc.prefill(q, k, v, a, b, np.zeros(1, np.float32), np.zeros(1, np.float32),
+                        scale=1.0, initial_state=S0)
+    be = 1.0 / (1.0 + np.exp(-b[:, 0].astype(np.float64)))
+    np.testing.assert_allclose(fs[0, 0], be[-1] * np.outer(v[-1, 0], k[-1, 0]), atol=1e-14)
+    for t in range(T):
+        np.testing.assert_allclose(o[t, 0], be[t] * v[t, 0] * (k[t, 0] @ q[t, 0]), atol=1e-13)
+
+
+def test_superposition(orc):
+    """For fixed keys and gates the map (S0, V) -> (o, S_T) is linear:
+    f(S1 + S2, V1 + V2) = f(S1, V1) + f(S2, V2)."""
+    rng = np.random.default_rng(8)
+    T, dk, dv = 11, 6, 5
+    q, k, v1, a, b, A_log, dt_bias = _rand_case(rng, T, 1, 1, dk, dv)
+    v2 = rng.standard_normal(v1.shape)
+    # halves of float32 draws, so that the sum of two states is exact in float32
+    S1 = (0.5 * rng.standard_normal((1, 1, dv, dk))).astype(np.float32)
+    S2 = (0.5 * rng.standard_normal((1, 1, dv, dk))).astype(np.float32)
+    S12 = S1.astype(np.float64) + S2.astype(np.float64)
+    o1, f1 = orc.prefill(q, k, v1, a, b, A_log, dt_bias, initial_state=S1)
+    o2, f2 = orc.prefill(q, k, v2, a, b, A_log, dt_bias, initial_state=S2)
+    # S1 + S2 rounds in float32 by at most 1e-7 relative: compare at that level
+    o12, f12 = orc.prefill(q, k, v1 + v2, a, b, A_log, dt_bias,
+                           initial_state=(S1 + S2).astype(np.float32))
+    assert np.max(np.abs((S1 + S2).astype(np.float64) - S12)) < 1e-6
+    np.testing.assert_allclose(o12, o1 + o2, rtol=0, atol=1e-6)
+    np.testing.assert_allclose(f12, f1 + f2, rtol=0, atol=1e-6)
+    # exact version: zero states, values only
+    z = np.zeros_like(S1)
+    oa, fa = orc.prefill(q, k, v1, a, b, A_log, dt_bias, initial_state=z)
+    ob, fb = orc.prefill(q, k, v2, a, b, A_log, dt_bias, initial_state=z)
+    oab, fab = orc.prefill(q, k, v1 + v2, a, b, A_log, dt_bias, initial_state=z)
+    np.testing.assert_allclose(oab, oa + ob, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(fab, fa + fb, rtol=0, atol=1e-12)
+    # and states only, with zero values: S -> f(S) is linear (scaling by 2 is exact)
+    z_v = np.zeros_like(v1)
+    os1, fs1 = orc.prefill(q, k, z_v, a, b, A_log, dt_bias, initial_state=S1)
+    os2, fs2 = orc.prefill(q, k, z_v, a, b, A_log, dt_bias, initial_state=2 * S1)
+    np.testing.assert_allclose(os2, 2 * os1, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(fs2, 2 * fs1, rtol=0, atol=1e-14)
+
+
+def test_ungated_rule_of_the_page(orc):
+    """alpha = 1: S_t = S_{t-1}(I - beta k k^T) + beta v k^T, evaluated as written
+    (matrix form) on the page."""
+    rng = np.random.default_rng(9)
+    T, dk, dv = 10, 6, 6
+    q, k, v, _, b, _, _ = _rand_case(rng, T, 1, 1, dk, dv)
+    a = np.full((T, 1), -np.inf, np.float32)
+    S0 = rng.standard_normal((1, 1, dv, dk)).astype(np.float32)
+    o, fs = orc.prefill(q, k, v, a, b, np.zeros(1, np.float32), np.zeros(1, np.float32),
+                        scale=1.0, initial_state=S0)
+    S = S0[0, 0].astype(np.float64)
+    be = 1.0 / (1.0 + np.exp(-b[:, 0].astype(np.float64)))
+    for t in range(T):
+        kt = k[t, 0]
+        S = S @ (np.eye(dk) - be[t] * np.outer(kt, kt)) + be[t] * np.outer(v[t, 0], kt)
+        np.testing.assert_allclose(o[t, 0], S @ q[t, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(fs[0, 0], S, rtol=0, atol=1e-12)
+
+
+def test_gate_closed_forms(orc):
+    # a + dt_bias = 0 -> softplus = ln 2; A_log = 0 -> rate 1
+    assert orc.log_alpha(0.0, 0.0, 0.0) == pytest.approx(-math.log(2.0), abs=1e-16)
+    assert orc.log_alpha(1.0, 0.0, -1.0) == pytest.approx(-math.log(2.0), abs=1e-16)
+    # A_log = ln 16 -> rate 16
+    assert orc.log_alpha(0.0, math.log(16.0), 0.0) == pytest.approx(-16 * math.log(2.0), rel=1e-15)
+    # large arguments: softplus(x) -> x, softplus(-x) -> e^{-x}
+    assert orc.log_alpha(60.0, 0.0, 0.0) == pytest.approx(-60.0, rel=1e-15)
+    assert orc.log_alpha(-60.0, 0.0, 0.0) == pytest.approx(-math.exp(-60.0), rel=1e-12)
+    # dt_bias = ln(expm1(dt)) is the inverse of softplus: log_alpha = -exp(A_log) dt at a = 0
+    for dt in (1e-3, 0.02, 0.1):
+        assert orc.log_alpha(0.0, 0.5, math.log(math.expm1(dt))) == pytest.approx(
+            -math.exp(0.5) * dt, rel=1e-12)
+    assert orc.beta(0.0) == 0.5
+    assert orc.beta(40.0) == pytest.approx(1.0, abs=1e-16)
+    assert orc.beta(-40.0) == pytest.approx(math.exp(-40.0), rel=1e-12)
+
+
+@pytest.mark.parametrize("C", [1, 2, 16, 64])
+def test_chunked_equals_recurrent(orc, C):
+    """The chunked WY/UT algebra reproduces the recurrence, with ragged chunks,
+    several packed sequences (one empty, one of length 1), non-zero S0 and
+    decay strong enough that the in-chunk log-decay falls far below -87."""
+    rng = np.random.default_rng(100 + C)
+    lengths = [70, 0, 1, 133, 64]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    T, Hqk, Hv, dk, dv = int(cu[-1]), 2, 6, 16, 12
+    q, k, v, a, b, A_log, dt_bias = _rand_case(rng, T, Hqk, Hv, dk, dv, unit_keys=True)
+    A_log[:2] = np.float32(math.log(16.0))       # strong decay heads
+    a[:, :2] = 3.0
+    S0 = rng.standard_normal((len(lengths), Hv, dv, dk)).astype(np.float32)
+    o_r, s_r = orc.prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens=cu, initial_state=S0)
+    o_c, s_c = orc.prefill_chunked(q, k, v, a, b, A_log, dt_bias, cu_seqlens=cu,
+                                   initial_state=S0, chunk=C)
+    np.testing.assert_allclose(o_c, o_r, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(s_c, s_r, rtol=0, atol=1e-12)
+    # the empty sequence keeps its initial state
+    np.testing.assert_array_equal(s_r[1], S0[1].astype(np.float64))
+
+
+def test_varlen_equals_separate_calls(orc):
+    rng = np.random.default_rng(12)
+    lengths = [5, 9, 3]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    T = int(cu[-1])
+    q, k, v, a, b, A_log, dt_bias = _rand_case(rng, T, 1, 3, 4, 4)
+    S0 = rng.standard_normal((3, 3, 4, 4)).astype(np.float32)
+    o, fs = orc.prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens=cu, initial_state=S0)
+    for n in range(3):
+        s, e = cu[n], cu[n + 1]
+        o1, f1 = orc.prefill(q[s:e], k[s:e], v[s:e], a[s:e], b[s:e], A_log, dt_bias,
+                             initial_state=S0[n:n + 1])
+        np.testing.assert_array_equal(o[s:e], o1)
+        np.testing.assert_array_equal(fs[n], f1[0])
+
+
+def test_head_subset_and_decode_step(orc):
+    """A one-token prefill equals one decode step, per unit and layer."""
+    import synth
+    inp = synth.make_decode(3, 2, seed=21, Hqk=2, Hv=6, d=8)
+    st = inp.full_state()
+    o_d, s_d = orc.decode(inp.q, inp.k, inp.v, inp.a, inp.b, inp.A_log, inp.dt_bias,
+                          inp.n_seq, inp.layers, st)
+    for u in range(inp.U):
+        l = u % inp.layers
+        o_p, s_p = orc.prefill(inp.q[u:u + 1], inp.k[u:u + 1], inp.v[u:u + 1], inp.a[u:u + 1],
+                               inp.b[u:u + 1], inp.A_log[l], inp.dt_bias[l],
+                               initial_state=st[u:u + 1])
+        np.testing.assert_array_equal(o_d[u], o_p[0])
+        np.testing.assert_array_equal(s_d[u], s_p[0])
+    # the unit-list path gives the same numbers
+    sel = [4, 1]
+    o_s, s_s = orc.decode(inp.q, inp.k, inp.v, inp.a, inp.b, inp.A_log, inp.dt_bias,
+                          inp.n_seq, inp.layers, st[sel], units=sel)
+    np.testing.assert_array_equal(o_s, o_d[sel])
+    np.testing.assert_array_equal(s_s, s_d[sel])
+
+
+# ---- front end ------------------------------------------------------------------
+
+def _fe_case(rng, T, Hqk=1, Hv=2, d=8):
+    import synth
+    ctot = (2 * Hqk + Hv) * d
+    x = synth.f32_to_bf16_bits(rng.standard_normal((T, ctot)).astype(np.float32))
+    return x, ctot
+
+
+def _silu(y):
+    return y / (1.0 + np.exp(-y))
+
+
+def test_conv_identity_tap(orc):
+    """w = e_3 (current token only): y = SiLU(x); q, k then have unit norm."""
+    import synth
+    rng = np.random.default_rng(31)
+    Hqk, Hv, d, T = 1, 2, 8, 7
+    x, ctot = _fe_case(rng, T, Hqk, Hv, d)
+    w = np.zeros((ctot, 4), np.float32)
+    w[:, 3] = 1.0
+    q, k, v, _ = orc.conv1d_silu(x, w, None, Hqk, Hv, d)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    y = _silu(xf)
+    np.testing.assert_allclose(v.reshape(T, -1), y[:, 2 * Hqk * d:], rtol=0, atol=1e-15)
+    yq = y[:, :d]
+    np.testing.assert_allclose(q[:, 0], yq / np.sqrt((yq ** 2).sum(1, keepdims=True) + 1e-6),
+                               rtol=0, atol=1e-15)
+    nrm = np.linalg.norm(k[:, 0], axis=-1)
+    assert np.all(np.abs(nrm - 1.0) < 1e-4)
+
+
+def test_conv_oldest_tap_shifts(orc):
+    """w = e_0: y[t] = SiLU(x[t-3]), zero history before the start."""
+    import synth
+    rng = np.random.default_rng(32)
+    Hqk, Hv, d, T = 1, 1, 8, 9
+    x, ctot = _fe_case(rng, T, Hqk, Hv, d)
+    w = np.zeros((ctot, 4), np.float32)
+    w[:, 0] = 1.0
+    _, _, v, _ = orc.conv1d_silu(x, w, None, Hqk, Hv, d)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)[:, 2 * d:]
+    exp = np.zeros_like(xf)
+    exp[3:] = _silu(xf[:-3])
+    np.testing.assert_allclose(v[:, 0], exp, rtol=0, atol=1e-15)
+
+
+def test_conv_matches_library_conv1d(orc):
+    """General weights and several packed sequences against
+    torch.nn.functional.conv1d (depthwise, left padding 3), per sequence."""
+    torch = pytest.importorskip("torch")
+    import synth
+    rng = np.random.default_rng(33)
+    Hqk, Hv, d = 2, 3, 8
+    lengths = [5, 1, 0, 12]
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    T = int(cu[-1])
+    x, ctot = _fe_case(rng, T, Hqk, Hv, d)
+    w = (0.5 * rng.standard_normal((ctot, 4))).astype(np.float32)
+    q, k, v, _ = orc.conv1d_silu(x, w, cu, Hqk, Hv, d)
+    xf = torch.from_numpy(synth.bf16_bits_to_f32(x).astype(np.float64))
+    wt = torch.from_numpy(w.astype(np.float64)).view(ctot, 1, 4)
+    for n in range(len(lengths)):
+        s, e = int(cu[n]), int(cu[n + 1])
+        if e == s:
+            continue
+        seg = xf[s:e].T.unsqueeze(0)                                    # [1, C, L]
+        y = torch.nn.functional.conv1d(seg, wt, padding=3, groups=ctot)[0, :, : e - s].T
+        y = torch.nn.functional.silu(y).numpy()
+        for hh in range(2 * Hqk + Hv):
+            blk = y[:, hh * d:(hh + 1) * d]
+            if hh < 2 * Hqk:
+                blk = blk / np.sqrt((blk ** 2).sum(1, keepdims=True) + 1e-6)
+            got = q[s:e, hh] if hh < Hqk else (k[s:e, hh - Hqk] if hh < 2 * Hqk
+                                              else v[s:e, hh - 2 * Hqk])
+            np.testing.assert_allclose(got, blk, rtol=0, atol=1e-13)
+
+
+def test_conv_state_carries_history(orc):
+    """Running a sequence in two parts, passing the conv state, equals one run."""
+    rng = np.random.default_rng(34)
+    Hqk, Hv, d, T = 1, 1, 8, 11
+    x, ctot = _fe_case(rng, T, Hqk, Hv, d)
+    w = (0.5 * rng.standard_normal((ctot, 4))).astype(np.float32)
+    q, k, v, cs = orc.conv1d_silu(x, w, None, Hqk, Hv, d)
+    for cut in (1, 2, 3, 7):
+        q1, k1, v1, cs1 = orc.conv1d_silu(x[:cut], w, None, Hqk, Hv, d)
+        q2, k2, v2, cs2 = orc.conv1d_silu(x[cut:], w, None, Hqk, Hv, d,
+                                          conv_state=cs1.astype(np.float32))
+        np.testing.assert_array_equal(np.concatenate([v1, v2]), v)
+        np.testing.assert_array_equal(np.concatenate([q1, q2]), q)
+        np.testing.assert_array_equal(cs2, cs)
