@@ -1,0 +1,501 @@
+"""Benchmark of the Gated DeltaNet recurrence path on B200.
+
+One step = one pass of the whole prefill path over one batch of synthetic
+input: the front end (gdn_conv1d_silu: conv1d + SiLU + L2 norm) and the chunked
+prefill (gdn_prefill) of one GDN layer, T = 8192 tokens, 16 key heads, 48 value
+heads, d = 128, zero initial state.  The metric is tokens per second per layer.
+Two secondary lines are measured in the same run and attached under "extra":
+the T = 262144 prefill (non-zero initial state) and one decode step over
+128 sequences x 48 layers with the 19.3 GB float32 state updated in place.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Timing: CUDA events on the launching stream around every step, L2 flushed
+(a 256 MiB buffer written) before each timed step, W >= 3 untimed warm-up
+steps, max over ranks.  With --gpus N > 1 (launched under torchrun) every rank
+runs its own replica of the workload (weak scaling; the path has no exchange
+step).  `--impl reference` times the fp64 CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+T_MAIN = 8192
+T_LONG = 262144
+HQK, HV, D = 16, 48, 128
+# algorithmic work per token per layer (chunked form, C = 64): 48 value heads x
+# (3 x 2Cd + 3 x 2d^2) + 16 key heads x 2 x 2Cd
+FLOP_PER_TOKEN = HV * (3 * 2 * 64 * D + 3 * 2 * D * D) + HQK * 2 * 2 * 64 * D
+# bytes per token the prefill must move: q, k, v bf16 in; a, b f32 in; o f32 out
+PREFILL_BYTES_PER_TOKEN = 2 * (2 * HQK * D + HV * D) + 4 * 2 * HV + 4 * HV * D
+# front end: read (2Hqk + Hv) d bf16, write the same
+FRONTEND_BYTES_PER_TOKEN = 2 * 2 * (2 * HQK + HV) * D
+STATE_BYTES = HV * D * D * 4
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": float(j["hbm_gbs"]), "bf16_tflops": float(j["bf16_tflops"]),
+                "bf16_tflops_sustained": float(j.get("bf16_tflops_sustained", j["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class Clocks:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"gdn_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+                except ValueError:
+                    continue
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v == "Active"})
+        loaded = [r[0] for r in rows if r[2] > 200.0] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------- GPU arm
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def _time_steps(step, warmup, steps, flush, streams_events):
+    """Warm-up, then `steps` timed steps; returns per-step ms (CUDA events on the
+    current stream) and per-kernel ms lists from streams_events()."""
+    import torch
+    for _ in range(warmup):
+        step(None)
+    torch.cuda.synchronize()
+    times = []
+    per_kernel = {}
+    for _ in range(steps):
+        flush.zero_()
+        ev = streams_events()
+        step(ev)
+        torch.cuda.synchronize()
+        times.append(ev["start"].elapsed_time(ev["end"]))
+        for name, (a, b) in ev.get("kernels", {}).items():
+            per_kernel.setdefault(name, []).append(a.elapsed_time(b))
+    return times, per_kernel
+
+
+def bench_main(args, world, rank, local):
+    import numpy as np
+    import torch
+    import gated_deltanet_recurrence_prefill_b200 as gdn
+    import synth
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    peaks = load_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    # ---- inputs of the 8K workload (seeded, synthetic), resident in HBM
+    fe = synth.workload(1)
+    g = fe.gates
+    to16 = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16)
+    h_qkv = to16(fe.qkv).pin_memory()
+    h_a = torch.from_numpy(g.a).pin_memory()
+    h_b = torch.from_numpy(g.b).pin_memory()
+    qkv = h_qkv.to(dev)
+    conv_w = torch.from_numpy(fe.conv_w).to(dev)
+    a = h_a.to(dev)
+    b = h_b.to(dev)
+    A_log = torch.from_numpy(g.A_log).to(dev)
+    dt_bias = torch.from_numpy(g.dt_bias).to(dev)
+    T = T_MAIN
+    q = torch.empty(T, HQK, D, dtype=torch.bfloat16, device=dev)
+    k = torch.empty_like(q)
+    v = torch.empty(T, HV, D, dtype=torch.bfloat16, device=dev)
+    o = torch.empty(T, HV, D, dtype=torch.float32, device=dev)
+    fs = torch.empty(1, HV, D, D, dtype=torch.float32, device=dev)
+    ws = torch.empty(gdn.prefill_workspace_size(1, T, HQK, HV, D), dtype=torch.uint8, device=dev)
+
+    def new_events():
+        mk = lambda: torch.cuda.Event(enable_timing=True)
+        e = {"start": mk(), "end": mk(), "kernels": {"conv1d_silu": (mk(), mk()),
+                                                       "prefill": (mk(), mk())}}
+        return e
+
+    def step(ev):
+        if ev:
+            ev["start"].record()
+            ev["kernels"]["conv1d_silu"][0].record()
+        gdn.conv1d_silu(qkv, conv_w, HQK, HV, out=(q, k, v))
+        if ev:
+            ev["kernels"]["conv1d_silu"][1].record()
+            ev["kernels"]["prefill"][0].record()
+        gdn.prefill(q, k, v, a, b, A_log, dt_bias, o=o, final_state=fs, workspace=ws)
+        if ev:
+            ev["kernels"]["prefill"][1].record()
+            ev["end"].record()
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with Clocks(local if "CUDA_VISIBLE_DEVICES" not in os.environ else _smi_index(local)) as clk:
+        wall0 = time.perf_counter()
+        times, per_kernel = _time_steps(step, args.warmup, args.steps, flush, new_events)
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+    clocks = clk.summary()
+    ms = sum(times) / len(times)
+    ms_max = _max_over_ranks(ms, world)
+    launches_per_step = 2
+
+    # ---- end to end through the public API with host buffers
+    h_o = torch.empty(T, HV, D, dtype=torch.float32).pin_memory()
+    h_fs = torch.empty(1, HV, D, D, dtype=torch.float32).pin_memory()
+
+    def e2e_step(ev):
+        if ev:
+            ev["start"].record()
+        qkv.copy_(h_qkv, non_blocking=True)
+        a.copy_(h_a, non_blocking=True)
+        b.copy_(h_b, non_blocking=True)
+        gdn.conv1d_silu(qkv, conv_w, HQK, HV, out=(q, k, v))
+        gdn.prefill(q, k, v, a, b, A_log, dt_bias, o=o, final_state=fs, workspace=ws)
+        h_o.copy_(o, non_blocking=True)
+        h_fs.copy_(fs, non_blocking=True)
+        if ev:
+            ev["end"].record()
+
+    mk = lambda: {"start": torch.cuda.Event(enable_timing=True),
+                  "end": torch.cuda.Event(enable_timing=True)}
+    e2e_times, _ = _time_steps(e2e_step, args.warmup, args.steps, flush, mk)
+    e2e_ms = _max_over_ranks(sum(e2e_times) / len(e2e_times), world)
+    h2d = h_qkv.numel() * 2 + h_a.numel() * 4 + h_b.numel() * 4
+    d2h = h_o.numel() * 4 + h_fs.numel() * 4
+
+    # ---- roofline of the dominant kernel
+    kern_ms = {name: sum(v) / len(v) for name, v in per_kernel.items()}
+    prefill_ms = kern_ms["prefill"]
+    conv_ms = kern_ms["conv1d_silu"]
+    if prefill_ms >= conv_ms:
+        dom, dom_ms, dom_bytes = "prefill", prefill_ms, PREFILL_BYTES_PER_TOKEN * T
+    else:
+        dom, dom_ms, dom_bytes = "conv1d_silu", conv_ms, FRONTEND_BYTES_PER_TOKEN * T
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "peak_source": peaks["source"], "bytes_per_launch": dom_bytes,
+                "kernel_ms": round(dom_ms, 4)}
+    prefill_tflops = FLOP_PER_TOKEN * T / (prefill_ms * 1e-3) / 1e12
+    kernels = {
+        "conv1d_silu": {"ms": round(conv_ms, 4),
+                        "GB_s": round(FRONTEND_BYTES_PER_TOKEN * T / (conv_ms * 1e-3) / 1e9, 1)},
+        "prefill": {"ms": round(prefill_ms, 4),
+                    "GB_s": round(PREFILL_BYTES_PER_TOKEN * T / (prefill_ms * 1e-3) / 1e9, 1),
+                    "TFLOP_s": round(prefill_tflops, 2),
+                    "tensor_frac": round(prefill_tflops / peaks["bf16_tflops"], 4)},
+    }
+
+    extra = {}
+    if not args.primary_only:
+        extra["prefill_262k"] = bench_long_prefill(args, dev, flush, peaks, world)
+        extra["decode_128seq_48layers"] = bench_decode(args, dev, peaks, world)
+
+    value = world * T / (ms_max * 1e-3)
+    line = {
+        "metric": "GDN prefill tokens/s/layer (front end + chunked prefill, T=8192)",
+        "value": round(value, 1), "unit": "tokens/s/layer", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded: N(0,1) bf16 q|k|v channels, conv w ~ N(0,0.25), gates per recipe)",
+        "config": {"workload": "gdn_conv1d_silu + gdn_prefill, 1 layer, T=8192, N=1, Hqk=16, "
+                               "Hv=48, d=128, zero S0, fp32 o and state",
+                   "T": T, "n_seq": 1, "Hqk": HQK, "Hv": HV, "d": D, "chunk": 64,
+                   "l2": "flushed before every timed step (256 MiB write)",
+                   "parallelism": f"replicas x{world}"},
+        "e2e": {"value": round(world * T / (e2e_ms * 1e-3), 1), "unit": "tokens/s/layer",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": launches_per_step * args.steps,
+        "roofline": roofline,
+        "kernels": kernels,
+        "clocks": clocks,
+        "wall_s_timed_region": round(wall, 3),
+    }
+    if extra:
+        line["extra"] = extra
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def _smi_index(local):
+    """nvidia-smi --id for this rank's GPU (an index or a UUID)."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [x.strip() for x in vis.split(",") if x.strip()]
+    if local < len(ids):
+        return ids[local]
+    return local
+
+
+def _max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def bench_long_prefill(args, dev, flush, peaks, world):
+    """T = 262144, one sequence, S0 ~ N(0, 0.02^2) (inputs drawn on the device)."""
+    import torch
+    import gated_deltanet_recurrence_prefill_b200 as gdn
+    T = T_LONG
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(2)
+
+    def unit(shape):
+        x = torch.randn(*shape, generator=gen, device=dev)
+        x = x / torch.sqrt((x * x).sum(-1, keepdim=True) + 1e-6)
+        return x.to(torch.bfloat16)
+
+    q = unit((T, HQK, D))
+    k = unit((T, HQK, D))
+    v = torch.randn(T, HV, D, generator=gen, device=dev).to(torch.bfloat16)
+    a = torch.randn(T, HV, generator=gen, device=dev)
+    b = torch.randn(T, HV, generator=gen, device=dev)
+    A_log = torch.log(torch.empty(HV, device=dev).uniform_(1, 16, generator=gen))
+    dt = torch.exp(torch.empty(HV, device=dev).uniform_(-6.907755, -2.302585, generator=gen))
+    dt_bias = torch.log(torch.expm1(dt))
+    s0 = 0.02 * torch.randn(1, HV, D, D, generator=gen, device=dev)
+    o = torch.empty(T, HV, D, dtype=torch.float32, device=dev)
+    fs = torch.empty_like(s0)
+    ws = torch.empty(gdn.prefill_workspace_size(1, T, HQK, HV, D), dtype=torch.uint8, device=dev)
+
+    def step(ev):
+        if ev:
+            ev["start"].record()
+        gdn.prefill(q, k, v, a, b, A_log, dt_bias, initial_state=s0, o=o, final_state=fs,
+                    workspace=ws)
+        if ev:
+            ev["end"].record()
+
+    mk = lambda: {"start": torch.cuda.Event(enable_timing=True),
+                  "end": torch.cuda.Event(enable_timing=True)}
+    times, _ = _time_steps(step, max(3, args.warmup), max(3, min(args.steps, 10)), flush, mk)
+    ms = _max_over_ranks(sum(times) / len(times), world)
+    tflops = FLOP_PER_TOKEN * T / (ms * 1e-3) / 1e12
+    gbs = (PREFILL_BYTES_PER_TOKEN * T + 2 * STATE_BYTES) / (ms * 1e-3) / 1e9
+    out = {"workload": "gdn_prefill T=262144 N=1 Hqk=16 Hv=48 d=128 S0~N(0,0.02^2)",
+           "ms": round(ms, 4), "tokens_per_s_layer": round(world * T / (ms * 1e-3), 1),
+           "TFLOP_s": round(tflops, 2), "tensor_frac": round(tflops / peaks["bf16_tflops"], 4),
+           "GB_s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+           "launches_per_step": 1}
+    del q, k, v, a, b, o
+    torch.cuda.empty_cache()
+    return out
+
+
+def bench_decode(args, dev, peaks, world):
+    """One decode step for 128 sequences x 48 layers, 19.3 GB float32 state in
+    place (inputs drawn on the device; the state is far larger than L2)."""
+    import torch
+    import gated_deltanet_recurrence_prefill_b200 as gdn
+    n_seq, L = 128, 48
+    U = n_seq * L
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4)
+
+    def unit(shape):
+        x = torch.randn(*shape, generator=gen, device=dev)
+        x = x / torch.sqrt((x * x).sum(-1, keepdim=True) + 1e-6)
+        return x.to(torch.bfloat16)
+
+    q = unit((U, HQK, D))
+    k = unit((U, HQK, D))
+    v = torch.randn(U, HV, D, generator=gen, device=dev).to(torch.bfloat16)
+    a = torch.randn(U, HV, generator=gen, device=dev)
+    b = torch.randn(U, HV, generator=gen, device=dev)
+    A_log = torch.log(torch.empty(L, HV, device=dev).uniform_(1, 16, generator=gen))
+    dt = torch.exp(torch.empty(L, HV, device=dev).uniform_(-6.907755, -2.302585, generator=gen))
+    dt_bias = torch.log(torch.expm1(dt))
+    state = torch.empty(U, HV, D, D, dtype=torch.float32, device=dev)
+    for i in range(0, U, 512):
+        state[i:i + 512].normal_(0.0, 0.02, generator=gen)
+    o = torch.empty(U, HV, D, dtype=torch.float32, device=dev)
+
+    def step(ev):
+        if ev:
+            ev["start"].record()
+        gdn.decode_step(q, k, v, a, b, A_log, dt_bias, state, n_seq, L, o=o)
+        if ev:
+            ev["end"].record()
+
+    mk = lambda: {"start": torch.cuda.Event(enable_timing=True),
+                  "end": torch.cuda.Event(enable_timing=True)}
+    dummy = torch.empty(1, device=dev)
+    times, _ = _time_steps(step, max(3, args.warmup), max(5, args.steps), dummy, mk)
+    ms = _max_over_ranks(sum(times) / len(times), world)
+    bytes_step = 2 * U * STATE_BYTES + U * (2 * 2 * HQK * D + 2 * HV * D + 2 * 4 * HV + 4 * HV * D)
+    gbs = bytes_step / (ms * 1e-3) / 1e9
+    out = {"workload": "gdn_decode_step 128 seq x 48 layers, fp32 state 19.33 GB in place",
+           "ms": round(ms, 4), "GB_s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+           "bytes_per_step": int(bytes_step), "l2": "state 19.3 GB >> L2, no flush needed",
+           "launches_per_step": 1}
+    del state, q, k, v, o
+    torch.cuda.empty_cache()
+    return out
+
+
+# ---------------------------------------------------------------------------- CPU oracle
+
+def cpu_baseline(seconds: float = 15.0, threads: int = 0):
+    """The fp64 oracle, as it stands, on the host cores: the 8K workload's front
+    end plus recurrence on a sample of value heads, repeated until ~`seconds`."""
+    import numpy as np
+    import oracle
+    import synth
+    oracle.build()
+    cores = oracle.max_threads(threads)
+    fe = synth.workload(1)
+    g = fe.gates
+    t0 = time.perf_counter()
+    q, k, v, _ = oracle.conv1d_silu(fe.qkv, fe.conv_w, None, HQK, HV, D, threads=threads)
+    t_fe = time.perf_counter() - t0
+    # recurrence on value-head groups of `cores` heads until the time budget is used
+    heads_done = 0
+    t_rec = 0.0
+    h = 0
+    while heads_done < HV and (t_fe + t_rec) < seconds:
+        h1 = min(HV, h + max(1, cores))
+        t1 = time.perf_counter()
+        oracle.prefill(q, k, v, g.a, g.b, g.A_log, g.dt_bias, heads=(h, h1), want_o=True,
+                       threads=threads)
+        t_rec += time.perf_counter() - t1
+        heads_done += h1 - h
+        h = h1
+    per_layer_s = t_fe + t_rec * HV / heads_done
+    return {"value": round(T_MAIN / per_layer_s, 2), "unit": "tokens/s/layer", "cores": cores,
+            "kind": "oracle",
+            "sample": f"front end on all T={T_MAIN} tokens x 80 heads ({t_fe:.2f} s) + recurrence "
+                      f"on {heads_done}/48 value heads x {T_MAIN} tokens ({t_rec:.2f} s), "
+                      f"scaled to 48 heads"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    t0 = time.perf_counter()
+    vals = []
+    # each step is a bounded sample, sized so that the whole run stays within minutes
+    per_step = max(1.0, min(args.cpu_seconds / 3, 150.0 / (args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(seconds=per_step)
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(seconds=per_step))
+    value = statistics.median(v["value"] for v in vals)
+    line = {"impl": "reference",
+            "metric": "GDN prefill tokens/s/layer (front end + chunked prefill, T=8192)",
+            "value": value, "unit": "tokens/s/layer", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(T_MAIN / value * 1e3, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)",
+            "config": {"workload": "gdn_conv1d_silu + gdn_prefill, 1 layer, T=8192, N=1, Hqk=16, "
+                                   "Hv=48, d=128, zero S0, fp32 o and state", "T": T_MAIN},
+            "cpu_baseline": {"kind": "oracle", "cores": vals[-1]["cores"], "value": value,
+                             "unit": "tokens/s/layer", "sample": vals[-1]["sample"]},
+            "e2e": {"value": value, "unit": "tokens/s/layer", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "wall_s": round(time.perf_counter() - t0, 2)}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["gdn", "reference"], default="gdn")
+    ap.add_argument("--primary-only", action="store_true", help="skip the 262K and decode lines")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, local = _dist()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    bench_main(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

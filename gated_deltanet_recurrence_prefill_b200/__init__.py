@@ -1,0 +1,18 @@
+"""Gated DeltaNet recurrence on B200 (sm_100a): Python binding of libgdn.
+
+The compute path is the CUDA library libgdn.so (C ABI declared in
+include/gdn.h).  This module only marshals torch tensors into that ABI:
+pointers, sizes and the current CUDA stream.  There is no CPU fallback: if the
+library is missing or no GPU is present, the calls raise.
+"""
+from ._lib import (  # noqa: F401
+    GdnError,
+    STATUS,
+    conv1d_silu,
+    decode_step,
+    lib,
+    lib_path,
+    prefill,
+    prefill_status,
+    prefill_workspace_size,
+)

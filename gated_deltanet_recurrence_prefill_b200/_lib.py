@@ -1,0 +1,196 @@
+"""ctypes binding of libgdn.so: torch tensors in, torch tensors out."""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(HERE, "libgdn.so")
+_lib = None
+
+STATUS = {
+    0: "GDN_OK",
+    1: "GDN_ERR_INVALID_ARG",
+    2: "GDN_ERR_UNSUPPORTED",
+    3: "GDN_ERR_MISALIGNED",
+    4: "GDN_ERR_CUDA",
+    5: "GDN_ERR_TIMEOUT",
+    6: "GDN_ERR_WORKSPACE",
+}
+
+# exported symbol -> (restype, argtypes)
+_vp, _i32, _i64, _f32, _sz = C.c_void_p, C.c_int32, C.c_int64, C.c_float, C.c_size_t
+SIGNATURES = {
+    "gdn_abi_version": (C.c_int, []),
+    "gdn_status_string": (C.c_char_p, [C.c_int]),
+    "gdn_last_cuda_error": (C.c_int, []),
+    "gdn_last_cuda_error_string": (C.c_char_p, []),
+    "gdn_conv1d_silu": (C.c_int, [_vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _vp,
+                                  _vp, _vp]),
+    "gdn_prefill_workspace_size": (_sz, [_i32, _i64, _i32, _i32, _i32]),
+    "gdn_prefill": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32,
+                              _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "gdn_prefill_status": (C.c_int, [_vp, _vp]),
+    "gdn_decode_step": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
+                                  _f32, _vp, _vp, _vp]),
+}
+
+
+class GdnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        msg = f"{fn} failed: {STATUS.get(status, status)}"
+        if status == 4 and _lib is not None:
+            msg += f" ({_lib.gdn_last_cuda_error_string().decode()})"
+        super().__init__(msg)
+        self.status = status
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def lib():
+    """Load libgdn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"libgdn.so not built at {_LIB_PATH}: run "
+                              "`python -m gated_deltanet_recurrence_prefill_b200.build`")
+        L = C.CDLL(_LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return C.c_void_p(s.cuda_stream)
+
+
+def _check(fn, status):
+    if status != 0:
+        raise GdnError(fn, status)
+
+
+def _need(t, dtype, shape, name):
+    import torch
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    del torch
+    return t
+
+
+def conv1d_silu(qkv, conv_w, Hqk, Hv, d=128, cu_seqlens=None, conv_state_in=None,
+                conv_state_out=None, out=None, stream=None):
+    """Front end.  qkv [T, (2Hqk+Hv)d] bf16, conv_w [Ctot, 4] f32.
+    Returns (q [T,Hqk,d], k [T,Hqk,d], v [T,Hv,d]) bf16."""
+    import torch
+    T = qkv.shape[0]
+    ctot = (2 * Hqk + Hv) * d
+    n_seq = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _need(qkv, torch.bfloat16, (T, ctot), "qkv")
+    _need(conv_w, torch.float32, (ctot, 4), "conv_w")
+    if cu_seqlens is not None:
+        _need(cu_seqlens, torch.int32, (n_seq + 1,), "cu_seqlens")
+    for nm, t in (("conv_state_in", conv_state_in), ("conv_state_out", conv_state_out)):
+        if t is not None:
+            _need(t, torch.float32, (n_seq, ctot, 3), nm)
+    if out is None:
+        q = torch.empty(T, Hqk, d, dtype=torch.bfloat16, device=qkv.device)
+        k = torch.empty(T, Hqk, d, dtype=torch.bfloat16, device=qkv.device)
+        v = torch.empty(T, Hv, d, dtype=torch.bfloat16, device=qkv.device)
+    else:
+        q, k, v = out
+    st = lib().gdn_conv1d_silu(_ptr(qkv), _ptr(conv_w), _ptr(cu_seqlens), n_seq, T, Hqk, Hv, d,
+                               _ptr(conv_state_in), _ptr(conv_state_out), _ptr(q), _ptr(k), _ptr(v),
+                               _stream(stream))
+    _check("gdn_conv1d_silu", st)
+    return q, k, v
+
+
+def prefill_workspace_size(n_seq, T, Hqk, Hv, d=128) -> int:
+    return int(lib().gdn_prefill_workspace_size(n_seq, T, Hqk, Hv, d))
+
+
+def prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens=None, scale=None, initial_state=None,
+            final_state=None, o=None, workspace=None, want_final_state=True, stream=None):
+    """Chunked prefill.  Returns (o [T,Hv,d] f32, final_state [N,Hv,d,d] f32 or None)."""
+    import torch
+    T, Hqk, d = q.shape
+    Hv = v.shape[1]
+    n_seq = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _need(q, torch.bfloat16, (T, Hqk, d), "q")
+    _need(k, torch.bfloat16, (T, Hqk, d), "k")
+    _need(v, torch.bfloat16, (T, Hv, d), "v")
+    _need(a, torch.float32, (T, Hv), "a")
+    _need(b, torch.float32, (T, Hv), "b")
+    _need(A_log, torch.float32, (Hv,), "A_log")
+    _need(dt_bias, torch.float32, (Hv,), "dt_bias")
+    if cu_seqlens is not None:
+        _need(cu_seqlens, torch.int32, (n_seq + 1,), "cu_seqlens")
+    if initial_state is not None:
+        _need(initial_state, torch.float32, (n_seq, Hv, d, d), "initial_state")
+    if scale is None:
+        scale = d ** -0.5
+    if o is None:
+        o = torch.empty(T, Hv, d, dtype=torch.float32, device=q.device)
+    if final_state is None and want_final_state:
+        final_state = torch.empty(n_seq, Hv, d, d, dtype=torch.float32, device=q.device)
+    ws_bytes = prefill_workspace_size(n_seq, T, Hqk, Hv, d)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    st = lib().gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias),
+                           _ptr(cu_seqlens), n_seq, T, Hqk, Hv, d, float(scale),
+                           _ptr(initial_state), _ptr(final_state), _ptr(o), _ptr(workspace),
+                           workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("gdn_prefill", st)
+    return o, final_state
+
+
+def prefill_status(workspace, stream=None) -> int:
+    """Error word left by the last prefill on `workspace` (waits for the stream)."""
+    return int(lib().gdn_prefill_status(_ptr(workspace), _stream(stream)))
+
+
+def decode_step(q, k, v, a, b, A_log, dt_bias, state, n_seq, layers, scale=None, o=None,
+                stream=None):
+    """One decode step over U = n_seq*layers units; `state` [U,Hv,d,d] f32 is
+    updated in place.  Returns o [U,Hv,d] f32."""
+    import torch
+    U, Hqk, d = q.shape
+    Hv = v.shape[1]
+    if U != n_seq * layers:
+        raise ValueError("q.shape[0] must equal n_seq * layers")
+    _need(q, torch.bfloat16, (U, Hqk, d), "q")
+    _need(k, torch.bfloat16, (U, Hqk, d), "k")
+    _need(v, torch.bfloat16, (U, Hv, d), "v")
+    _need(a, torch.float32, (U, Hv), "a")
+    _need(b, torch.float32, (U, Hv), "b")
+    _need(A_log, torch.float32, (layers, Hv), "A_log")
+    _need(dt_bias, torch.float32, (layers, Hv), "dt_bias")
+    _need(state, torch.float32, (U, Hv, d, d), "state")
+    if scale is None:
+        scale = d ** -0.5
+    if o is None:
+        o = torch.empty(U, Hv, d, dtype=torch.float32, device=q.device)
+    st = lib().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(A_log),
+                               _ptr(dt_bias), n_seq, layers, Hqk, Hv, d, float(scale), _ptr(state),
+                               _ptr(o), _stream(stream))
+    _check("gdn_decode_step", st)
+    return o

@@ -1,0 +1,197 @@
+// conv1d_silu.cu -- the layer's front end: causal depthwise convolution of
+// width 4 over time (Qwen3.8-27B architecture page, 2kiu.com, section 2.1:
+// linear_conv_kernel_dim = 4, conv1d.weight), SiLU on every channel, then q
+// and k divided per head by sqrt(sum of squares + 1e-6).
+//
+// The work is elementwise in time apart from a 3-token history, so it is bound
+// by HBM bandwidth (read the packed bf16 channels once, write q, k, v once).
+// Mapping: a half-warp covers one head (16 lanes x 8 channels = 128), a warp
+// two heads; each lane moves 16 bytes per token.  A warp walks a run of
+// kRun consecutive tokens, keeping the last three inputs of its 8 channels in
+// registers, so each input is loaded once plus a 3-token halo per run.  At a
+// sequence boundary the history restarts from conv_state_in (or zeros).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace gdn {
+
+namespace {
+
+constexpr int kD = 128;
+constexpr int kRun = 32;              // tokens per warp
+constexpr int kWarps = 8;             // warps per CTA
+constexpr int kChan = 8;              // channels per lane
+
+// index of the sequence containing token t: largest n with cu[n] <= t
+__device__ int find_seq(const int32_t* cu, int n_seq, int64_t t) {
+    int lo = 0, hi = n_seq - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((int64_t)cu[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+GDN_DEVICE void load8(const uint16_t* p, float* x) {
+    const uint4 r = *reinterpret_cast<const uint4*>(p);
+    float2 t;
+    t = bf16x2_to_f32x2(r.x); x[0] = t.x; x[1] = t.y;
+    t = bf16x2_to_f32x2(r.y); x[2] = t.x; x[3] = t.y;
+    t = bf16x2_to_f32x2(r.z); x[4] = t.x; x[5] = t.y;
+    t = bf16x2_to_f32x2(r.w); x[6] = t.x; x[7] = t.y;
+}
+
+__global__ void __launch_bounds__(kWarps * 32)
+conv1d_silu_kernel(const uint16_t* __restrict__ qkv, const float* __restrict__ w,
+                   const int32_t* __restrict__ cu, int32_t n_seq, int64_t T, int32_t Hqk,
+                   int32_t Hv, const float* __restrict__ cs_in, uint16_t* __restrict__ qo,
+                   uint16_t* __restrict__ ko, uint16_t* __restrict__ vo, int64_t n_runs) {
+    const int lane = threadIdx.x & 31;
+    const int64_t gw = (int64_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+    const int n_heads = 2 * Hqk + Hv;
+    const int n_pairs = (n_heads + 1) >> 1;
+    const int64_t run = gw / n_pairs;
+    if (run >= n_runs) return;
+    const int pair = (int)(gw - run * n_pairs);
+    const int head = pair * 2 + (lane >> 4);
+    const bool active = head < n_heads;
+    const int hc = head < n_heads ? head : n_heads - 1;        // clamp for address math
+    const int64_t Ctot = (int64_t)n_heads * kD;
+    const int64_t c0 = (int64_t)hc * kD + (lane & 15) * kChan;  // first channel of this lane
+
+    float wr[kChan][4];
+#pragma unroll
+    for (int i = 0; i < kChan; ++i) {
+        const float4 t = *reinterpret_cast<const float4*>(w + (c0 + i) * 4);
+        wr[i][0] = t.x; wr[i][1] = t.y; wr[i][2] = t.z; wr[i][3] = t.w;
+    }
+
+    const int64_t t0 = run * kRun;
+    const int64_t t1 = t0 + kRun < T ? t0 + kRun : T;
+    int n = cu ? find_seq(cu, n_seq, t0) : 0;
+    // a sequence of length 0 shares its start with the next one: skip to the
+    // sequence that actually contains t0
+    int64_t bos = cu ? cu[n] : 0;
+    int64_t eos = cu ? cu[n + 1] : T;
+
+    // history h[j] = x[t - 3 + j] for j = 0..2, relative to the current t
+    float hist[3][kChan];
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+        const int64_t tau = t0 - 3 + j;
+        if (tau >= bos) {
+            load8(qkv + tau * Ctot + c0, hist[j]);
+        } else if (cs_in) {
+            const int64_t m = bos - tau;             // 1..3 tokens before the start
+#pragma unroll
+            for (int i = 0; i < kChan; ++i) hist[j][i] = cs_in[((int64_t)n * Ctot + c0 + i) * 3 + (3 - m)];
+        } else {
+#pragma unroll
+            for (int i = 0; i < kChan; ++i) hist[j][i] = 0.f;
+        }
+    }
+
+    const bool is_q = head < Hqk;
+    const bool is_k = head >= Hqk && head < 2 * Hqk;
+    uint16_t* dst_base;
+    int64_t dst_stride;
+    if (is_q) { dst_base = qo + (int64_t)head * kD; dst_stride = (int64_t)Hqk * kD; }
+    else if (is_k) { dst_base = ko + (int64_t)(head - Hqk) * kD; dst_stride = (int64_t)Hqk * kD; }
+    else { dst_base = vo + (int64_t)(hc - 2 * Hqk) * kD; dst_stride = (int64_t)Hv * kD; }
+    dst_base += (lane & 15) * kChan;
+
+    for (int64_t t = t0; t < t1; ++t) {
+        if (t >= eos) {
+            // next sequence(s): skip empty ones, restart the history
+            while (n + 1 < n_seq && (int64_t)cu[n + 1] <= t) ++n;
+            bos = cu[n];
+            eos = cu[n + 1];
+#pragma unroll
+            for (int j = 0; j < 3; ++j)
+#pragma unroll
+                for (int i = 0; i < kChan; ++i)
+                    hist[j][i] = cs_in ? cs_in[((int64_t)n * Ctot + c0 + i) * 3 + j] : 0.f;
+        }
+        float x[kChan];
+        load8(qkv + t * Ctot + c0, x);
+        float y[kChan];
+        float ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < kChan; ++i) {
+            float acc = wr[i][0] * hist[0][i];
+            acc = fmaf(wr[i][1], hist[1][i], acc);
+            acc = fmaf(wr[i][2], hist[2][i], acc);
+            acc = fmaf(wr[i][3], x[i], acc);
+            const float s = acc / (1.f + expf(-acc));
+            y[i] = s;
+            ss = fmaf(s, s, ss);
+            hist[0][i] = hist[1][i];
+            hist[1][i] = hist[2][i];
+            hist[2][i] = x[i];
+        }
+        // sum of squares over the 16 lanes of this head
+#pragma unroll
+        for (int m = 8; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+        const float inv = (is_q || is_k) ? rsqrtf(ss + 1e-6f) : 1.f;
+        uint4 out;
+        out.x = pack_bf16x2(y[0] * inv, y[1] * inv);
+        out.y = pack_bf16x2(y[2] * inv, y[3] * inv);
+        out.z = pack_bf16x2(y[4] * inv, y[5] * inv);
+        out.w = pack_bf16x2(y[6] * inv, y[7] * inv);
+        if (active) *reinterpret_cast<uint4*>(dst_base + t * dst_stride) = out;
+    }
+}
+
+// conv_state_out[n, c, s] = x[eos - 3 + s, c], or the incoming history when
+// that position lies before the sequence start.
+__global__ void conv_state_out_kernel(const uint16_t* __restrict__ qkv, const int32_t* __restrict__ cu,
+                                      int32_t n_seq, int64_t T, int64_t Ctot,
+                                      const float* __restrict__ cs_in, float* __restrict__ cs_out) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (int64_t)n_seq * Ctot) return;
+    const int n = (int)(i / Ctot);
+    const int64_t c = i - (int64_t)n * Ctot;
+    const int64_t bos = cu ? cu[n] : 0;
+    const int64_t eos = cu ? cu[n + 1] : T;
+#pragma unroll
+    for (int s = 0; s < 3; ++s) {
+        const int64_t tau = eos - 3 + s;
+        float xv;
+        if (tau >= bos) xv = bf16_to_f32(qkv[tau * Ctot + c]);
+        else xv = cs_in ? cs_in[((int64_t)n * Ctot + c) * 3 + (3 - (bos - tau))] : 0.f;
+        cs_out[i * 3 + s] = xv;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_conv1d_silu(const uint16_t* qkv, const float* w, const int32_t* cu,
+                               int32_t n_seq, int64_t T, int32_t Hqk, int32_t Hv,
+                               const float* cs_in, float* cs_out, uint16_t* q, uint16_t* k,
+                               uint16_t* v, cudaStream_t stream) {
+    const int n_heads = 2 * Hqk + Hv;
+    const int n_pairs = (n_heads + 1) / 2;
+    const int64_t Ctot = (int64_t)n_heads * kD;
+    if (T > 0) {
+        const int64_t n_runs = (T + kRun - 1) / kRun;
+        const int64_t warps = n_runs * n_pairs;
+        const int64_t blocks = (warps + kWarps - 1) / kWarps;
+        if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+        conv1d_silu_kernel<<<(unsigned)blocks, kWarps * 32, 0, stream>>>(
+            qkv, w, cu, n_seq, T, Hqk, Hv, cs_in, q, k, v, n_runs);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    if (cs_out) {
+        const int64_t total = (int64_t)n_seq * Ctot;
+        const int64_t blocks = (total + 255) / 256;
+        if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+        if (blocks > 0)
+            conv_state_out_kernel<<<(unsigned)blocks, 256, 0, stream>>>(qkv, cu, n_seq, T, Ctot,
+                                                                        cs_in, cs_out);
+        return cudaGetLastError();
+    }
+    return cudaSuccess;
+}
+
+}  // namespace gdn

@@ -1,0 +1,119 @@
+// decode.cu -- one token of the gated delta rule for many (sequence, layer)
+// units, state updated in place.
+//
+// Per value head the step is S <- alpha S (I - beta k k^T) + beta v k^T and
+// o = scale S q (Qwen3.8-27B architecture page, 2kiu.com, section 2.2, with
+// the decay alpha on the erased state).  Row i of S (d_k wide) changes as
+//     x_i = S_i . k,   S_i <- alpha S_i + beta (v_i - alpha x_i) k,
+// and the output needs the updated row only through
+//     S_i' . q = alpha (S_i . q) + beta (v_i - alpha x_i) (k . q),
+// so both dot products are taken from the row as loaded and every row is read
+// once and written once.  The state is float32 and dominates the traffic
+// (2 x 64 KiB per value head per token); the kernel is bound by HBM bandwidth.
+//
+// Mapping: one CTA of 128 threads per (unit, value head).  Each warp owns 32
+// rows; a lane holds 4 consecutive d_k elements (one float4) of a row, so a
+// row is one fully coalesced 512-byte access.  Eight rows are in flight per
+// warp to keep enough bytes outstanding.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace gdn {
+
+namespace {
+
+constexpr int kD = 128;
+constexpr int kThreads = 128;
+constexpr int kRowsPerIter = 8;
+
+__global__ void __launch_bounds__(kThreads)
+decode_step_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
+                   const uint16_t* __restrict__ v, const float* __restrict__ a,
+                   const float* __restrict__ b, const float* __restrict__ A_log,
+                   const float* __restrict__ dt_bias, int32_t layers, int32_t Hqk, int32_t Hv,
+                   float scale, float* __restrict__ state, float* __restrict__ o) {
+    const int64_t uh = blockIdx.x;                 // unit * Hv + h
+    const int64_t u = uh / Hv;
+    const int h = (int)(uh - u * Hv);
+    const int g = h / (Hv / Hqk);
+    const int l = (int)(u % layers);
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+
+    // this lane's 4 elements of k and q
+    const uint2 kb = *reinterpret_cast<const uint2*>(k + (u * Hqk + g) * kD + lane * 4);
+    const uint2 qb = *reinterpret_cast<const uint2*>(q + (u * Hqk + g) * kD + lane * 4);
+    const float2 k01 = bf16x2_to_f32x2(kb.x), k23 = bf16x2_to_f32x2(kb.y);
+    const float2 q01 = bf16x2_to_f32x2(qb.x), q23 = bf16x2_to_f32x2(qb.y);
+    const float kq = warp_sum(k01.x * q01.x + k01.y * q01.y + k23.x * q23.x + k23.y * q23.y);
+
+    const float alpha = expf(log_alpha_f32(a[uh], A_log[(int64_t)l * Hv + h], dt_bias[(int64_t)l * Hv + h]));
+    const float beta = sigmoid_f32(b[uh]);
+
+    float* S = state + uh * (int64_t)(kD * kD);
+    const uint16_t* vh = v + uh * kD;
+    float* oh = o + uh * kD;
+
+#pragma unroll 1
+    for (int r0 = warp * 32; r0 < warp * 32 + 32; r0 += kRowsPerIter) {
+        float4 s[kRowsPerIter];
+#pragma unroll
+        for (int j = 0; j < kRowsPerIter; ++j)
+            s[j] = __ldcs(reinterpret_cast<const float4*>(S + (int64_t)(r0 + j) * kD) + lane);
+        // v for these 8 rows: one 16-byte broadcast load
+        const uint4 vb = *reinterpret_cast<const uint4*>(vh + r0);
+        float vr[kRowsPerIter];
+        {
+            float2 t;
+            t = bf16x2_to_f32x2(vb.x); vr[0] = t.x; vr[1] = t.y;
+            t = bf16x2_to_f32x2(vb.y); vr[2] = t.x; vr[3] = t.y;
+            t = bf16x2_to_f32x2(vb.z); vr[4] = t.x; vr[5] = t.y;
+            t = bf16x2_to_f32x2(vb.w); vr[6] = t.x; vr[7] = t.y;
+        }
+        float xk[kRowsPerIter], xq[kRowsPerIter];
+#pragma unroll
+        for (int j = 0; j < kRowsPerIter; ++j) {
+            xk[j] = s[j].x * k01.x + s[j].y * k01.y + s[j].z * k23.x + s[j].w * k23.y;
+            xq[j] = s[j].x * q01.x + s[j].y * q01.y + s[j].z * q23.x + s[j].w * q23.y;
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) {
+#pragma unroll
+            for (int j = 0; j < kRowsPerIter; ++j) {
+                xk[j] += __shfl_xor_sync(0xffffffffu, xk[j], m);
+                xq[j] += __shfl_xor_sync(0xffffffffu, xq[j], m);
+            }
+        }
+        float orow = 0.f;
+#pragma unroll
+        for (int j = 0; j < kRowsPerIter; ++j) {
+            const float w = beta * (vr[j] - alpha * xk[j]);
+            float4 t;
+            t.x = fmaf(alpha, s[j].x, w * k01.x);
+            t.y = fmaf(alpha, s[j].y, w * k01.y);
+            t.z = fmaf(alpha, s[j].z, w * k23.x);
+            t.w = fmaf(alpha, s[j].w, w * k23.y);
+            __stcs(reinterpret_cast<float4*>(S + (int64_t)(r0 + j) * kD) + lane, t);
+            const float oj = scale * fmaf(alpha, xq[j], w * kq);
+            if (lane == j) orow = oj;
+        }
+        if (lane < kRowsPerIter) oh[r0 + lane] = orow;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_decode_step(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                               const float* a, const float* b, const float* A_log,
+                               const float* dt_bias, int32_t n_seq, int32_t layers, int32_t Hqk,
+                               int32_t Hv, float scale, float* state, float* o,
+                               cudaStream_t stream) {
+    const int64_t blocks = (int64_t)n_seq * layers * Hv;
+    if (blocks == 0) return cudaSuccess;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    decode_step_kernel<<<(unsigned)blocks, kThreads, 0, stream>>>(
+        q, k, v, a, b, A_log, dt_bias, layers, Hqk, Hv, scale, state, o);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

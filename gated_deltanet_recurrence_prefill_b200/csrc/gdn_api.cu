@@ -1,0 +1,145 @@
+// gdn_api.cu -- the C ABI of libgdn (see include/gdn.h): argument checks on the
+// host, then kernel launches on the caller's stream.  Nothing here allocates,
+// frees or synchronises, except gdn_prefill_status, which documents that it
+// waits for the stream.
+#include <cuda_runtime.h>
+
+#include "../../include/gdn.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+gdn_status cuda_fail(cudaError_t e) {
+    g_last_cuda_error = (int)e;
+    return GDN_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int32_t kD = 128;
+
+gdn_status check_heads(int32_t Hqk, int32_t Hv, int32_t d) {
+    if (Hqk <= 0 || Hv <= 0 || d <= 0) return GDN_ERR_INVALID_ARG;
+    if (d != kD) return GDN_ERR_UNSUPPORTED;
+    if (Hv % Hqk != 0) return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+gdn_status check_seqs(const int32_t* cu_seqlens, int32_t n_seq, int64_t T) {
+    if (T < 0 || n_seq <= 0) return GDN_ERR_INVALID_ARG;
+    if (!cu_seqlens && n_seq != 1) return GDN_ERR_INVALID_ARG;
+    if (T > (int64_t)0x7fffffff) return GDN_ERR_UNSUPPORTED;   // cu_seqlens are int32
+    return GDN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdn_abi_version(void) { return GDN_ABI_VERSION; }
+
+const char* gdn_status_string(int status) {
+    switch (status) {
+        case GDN_OK: return "ok";
+        case GDN_ERR_INVALID_ARG: return "invalid argument";
+        case GDN_ERR_UNSUPPORTED: return "unsupported shape";
+        case GDN_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case GDN_ERR_CUDA: return "CUDA error";
+        case GDN_ERR_TIMEOUT: return "bounded device wait timed out";
+        case GDN_ERR_WORKSPACE: return "workspace missing or too small";
+        default: return "unknown status";
+    }
+}
+
+int gdn_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char* gdn_last_cuda_error_string(void) {
+    return cudaGetErrorName((cudaError_t)g_last_cuda_error);
+}
+
+gdn_status gdn_conv1d_silu(const uint16_t* qkv, const float* conv_w, const int32_t* cu_seqlens,
+                           int32_t n_seq, int64_t T, int32_t Hqk, int32_t Hv, int32_t d,
+                           const float* conv_state_in, float* conv_state_out, uint16_t* q,
+                           uint16_t* k, uint16_t* v, gdn_stream_t stream) {
+    gdn_status st = check_heads(Hqk, Hv, d);
+    if (st != GDN_OK) return st;
+    if ((st = check_seqs(cu_seqlens, n_seq, T)) != GDN_OK) return st;
+    if (!conv_w || (T > 0 && (!qkv || !q || !k || !v))) return GDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {qkv, conv_w, cu_seqlens, conv_state_in, conv_state_out, q, k, v};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
+    if (conv_state_in && conv_state_in == conv_state_out) return GDN_ERR_INVALID_ARG;
+    cudaError_t e = gdn::launch_conv1d_silu(qkv, conv_w, cu_seqlens, n_seq, T, Hqk, Hv,
+                                            conv_state_in, conv_state_out, q, k, v,
+                                            (cudaStream_t)stream);
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
+size_t gdn_prefill_workspace_size(int32_t n_seq, int64_t T, int32_t Hqk, int32_t Hv, int32_t d) {
+    (void)T; (void)Hqk; (void)d;
+    size_t n = n_seq > 0 ? (size_t)n_seq : 1;
+    size_t hv = Hv > 0 ? (size_t)Hv : 1;
+    // header (error word) + one int32 per (sequence, value head) for the schedule
+    size_t bytes = gdn::kWsHeaderBytes + ((n * hv * sizeof(int32_t) + 255) / 256) * 256;
+    return bytes;
+}
+
+gdn_status gdn_prefill(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* a,
+                       const float* b, const float* A_log, const float* dt_bias,
+                       const int32_t* cu_seqlens, int32_t n_seq, int64_t T, int32_t Hqk,
+                       int32_t Hv, int32_t d, float scale, const float* initial_state,
+                       float* final_state, float* o, void* workspace, size_t workspace_bytes,
+                       gdn_stream_t stream) {
+    gdn_status st = check_heads(Hqk, Hv, d);
+    if (st != GDN_OK) return st;
+    if ((st = check_seqs(cu_seqlens, n_seq, T)) != GDN_OK) return st;
+    if (!A_log || !dt_bias) return GDN_ERR_INVALID_ARG;
+    if (T > 0 && (!q || !k || !v || !a || !b || !o)) return GDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, a, b, A_log, dt_bias, cu_seqlens, initial_state, final_state,
+                          o};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
+    if (!workspace || workspace_bytes < gdn_prefill_workspace_size(n_seq, T, Hqk, Hv, d))
+        return GDN_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_MISALIGNED;
+    gdn::PrefillArgs p{q, k, v, a, b, A_log, dt_bias, cu_seqlens, n_seq, T, Hqk, Hv, scale,
+                       initial_state, final_state, o, workspace, workspace_bytes};
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaMemsetAsync(workspace, 0, gdn::kWsHeaderBytes, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = gdn::launch_prefill_simt(p, s);
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
+gdn_status gdn_prefill_status(const void* workspace, gdn_stream_t stream) {
+    if (!workspace) return GDN_ERR_WORKSPACE;
+    uint32_t word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, (const char*)workspace + gdn::kWsErrorWordOffset,
+                                    sizeof word, cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+    if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return word == 0 ? GDN_OK : GDN_ERR_TIMEOUT;
+}
+
+gdn_status gdn_decode_step(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                           const float* a, const float* b, const float* A_log,
+                           const float* dt_bias, int32_t n_seq, int32_t layers, int32_t Hqk,
+                           int32_t Hv, int32_t d, float scale, float* state, float* o,
+                           gdn_stream_t stream) {
+    gdn_status st = check_heads(Hqk, Hv, d);
+    if (st != GDN_OK) return st;
+    if (n_seq < 0 || layers <= 0) return GDN_ERR_INVALID_ARG;
+    if (n_seq == 0) return GDN_OK;
+    if (!q || !k || !v || !a || !b || !A_log || !dt_bias || !state || !o)
+        return GDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, a, b, A_log, dt_bias, state, o};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return GDN_ERR_MISALIGNED;
+    cudaError_t e = gdn::launch_decode_step(q, k, v, a, b, A_log, dt_bias, n_seq, layers, Hqk,
+                                            Hv, scale, state, o, (cudaStream_t)stream);
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,50 @@
+// kernels.h -- internal launch interface between the C ABI (gdn_api.cu) and
+// the kernels.  Not installed; the public interface is include/gdn.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gdn {
+
+struct PrefillArgs {
+    const uint16_t* q;
+    const uint16_t* k;
+    const uint16_t* v;
+    const float* a;
+    const float* b;
+    const float* A_log;
+    const float* dt_bias;
+    const int32_t* cu_seqlens;     // NULL: one sequence of length T
+    int32_t n_seq;
+    int64_t T;
+    int32_t Hqk;
+    int32_t Hv;
+    float scale;
+    const float* initial_state;    // may be NULL
+    float* final_state;            // may be NULL
+    float* o;
+    void* workspace;
+    size_t workspace_bytes;
+};
+
+cudaError_t launch_decode_step(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                               const float* a, const float* b, const float* A_log,
+                               const float* dt_bias, int32_t n_seq, int32_t layers, int32_t Hqk,
+                               int32_t Hv, float scale, float* state, float* o,
+                               cudaStream_t stream);
+
+cudaError_t launch_conv1d_silu(const uint16_t* qkv, const float* w, const int32_t* cu,
+                               int32_t n_seq, int64_t T, int32_t Hqk, int32_t Hv,
+                               const float* cs_in, float* cs_out, uint16_t* q, uint16_t* k,
+                               uint16_t* v, cudaStream_t stream);
+
+cudaError_t launch_prefill_simt(const PrefillArgs& p, cudaStream_t stream);
+size_t prefill_simt_smem_bytes();
+
+// workspace layout shared by the prefill kernels
+constexpr size_t kWsErrorWordOffset = 0;     // uint32 error word (0 = ok)
+constexpr size_t kWsHeaderBytes = 256;
+
+}  // namespace gdn

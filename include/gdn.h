@@ -1,0 +1,182 @@
+/*
+ * gdn.h -- C ABI of libgdn: the Gated DeltaNet gated delta-rule recurrence on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation.  A Gated DeltaNet layer keeps, per value head, a fixed-size
+ * state S (d_v x d_k, float32) and updates it once per token with the delta
+ * rule of the Qwen3.8-27B architecture page (2kiu.com, "From parameter race to
+ * efficiency revolution: dissecting Qwen3.8-27B's dense architecture and
+ * long-context hybrid attention", section 2.2): the value stored under key k_t
+ * is erased and v_t written with strength beta_t.  The layer is gated: a decay
+ * alpha_t scales the erased state,
+ *
+ *     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *     o_t = scale * S_t q_t,
+ *     alpha_t = exp(-exp(A_log) * softplus(a_t + dt_bias)),  beta_t = sigmoid(b_t),
+ *
+ * with the per-layer parameters A_log, dt_bias and the per-token inputs a, b
+ * named by that page's weight list (A_log, dt_bias, in_proj_a, in_proj_b,
+ * section 2.1; the page gives no gate formula, this is the reading the library
+ * implements).  Section 2.1 fixes the shape this library is built for: 16 key
+ * heads (q, k), 48 value heads, head width 128; value head h reads key head
+ * h / (Hv / Hqk).  Section 2.2 keeps the state in float32.  Before the
+ * recurrence, q, k and v go through a causal depthwise convolution of width 4
+ * (linear_conv_kernel_dim = 4 and conv1d.weight, section 2.1), SiLU, and an L2
+ * normalisation of q and k per head.
+ *
+ * Conventions for every entry point.
+ *  - Memory.  Every pointer argument is a DEVICE pointer unless stated
+ *    otherwise; the caller owns all memory.  The library never allocates,
+ *    frees or synchronises, and enqueues all work on `stream` (NULL = the
+ *    legacy default stream).  Results are ready when the stream reaches them.
+ *  - Types.  bf16 tensors are passed as uint16_t bit patterns.  Layouts are
+ *    dense row-major in the order written; "[T, H, d]" means d is contiguous.
+ *  - Alignment.  Every tensor pointer must be 16-byte aligned
+ *    (GDN_ERR_MISALIGNED otherwise).
+ *  - Aliasing.  Inputs and outputs must not overlap, except where stated.
+ *  - Errors.  Arguments are checked on the host first; on any error nothing is
+ *    launched and the status says why.  A failed launch returns GDN_ERR_CUDA.
+ *    Device code never traps or asserts.
+ *  - Sequences.  cu_seqlens (int32, device, [n_seq + 1], non-decreasing,
+ *    cu_seqlens[0] = 0, cu_seqlens[n_seq] = T) packs n_seq sequences along the
+ *    token axis; NULL means one sequence of length T (n_seq must be 1).  No
+ *    state, history or chunk crosses a sequence boundary.  Sequences of
+ *    length 0 are allowed.  The library trusts cu_seqlens' contents.
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The CUDA stream type (cudaStream_t / CUstream), declared without CUDA headers. */
+struct CUstream_st;
+typedef struct CUstream_st* gdn_stream_t;
+
+typedef enum gdn_status {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,   /* NULL required pointer, negative size, inconsistent sizes */
+    GDN_ERR_UNSUPPORTED = 2,   /* a shape the kernels do not implement (d != 128, Hv % Hqk != 0) */
+    GDN_ERR_MISALIGNED = 3,    /* a tensor pointer that is not 16-byte aligned */
+    GDN_ERR_CUDA = 4,          /* a CUDA call or kernel launch failed (see gdn_last_cuda_error) */
+    GDN_ERR_TIMEOUT = 5,       /* a bounded wait inside a kernel ran out (prefill only) */
+    GDN_ERR_WORKSPACE = 6      /* workspace NULL or smaller than gdn_prefill_workspace_size() */
+} gdn_status;
+
+/* Version of this ABI; bumped when a signature or a layout changes. */
+#define GDN_ABI_VERSION 1
+int gdn_abi_version(void);
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+const char* gdn_status_string(int status);
+
+/* The last CUDA error code seen by a call that returned GDN_ERR_CUDA in this
+ * process (0 if none), and its name.  Informational; not thread-safe. */
+int gdn_last_cuda_error(void);
+const char* gdn_last_cuda_error_string(void);
+
+/*
+ * gdn_conv1d_silu -- the layer's front end: causal depthwise 4-tap convolution
+ * over time for every channel, SiLU on every channel, then q and k divided per
+ * head by sqrt(sum of squares + 1e-6).  Width-4 causal convolution and
+ * conv1d.weight: architecture page section 2.1.
+ *
+ *  qkv            [T, Ctot] bf16, Ctot = (2 Hqk + Hv) d; channels ordered
+ *                 [q heads 0..Hqk-1 | k heads 0..Hqk-1 | v heads 0..Hv-1],
+ *                 each head d channels.
+ *  conv_w         [Ctot, 4] float32; tap j multiplies x[t - 3 + j] (tap 3 is
+ *                 the current token).  No bias.
+ *  conv_state_in  [n_seq, Ctot, 3] float32 or NULL: the three inputs before
+ *                 each sequence's first token, oldest first (NULL: zeros).
+ *  conv_state_out [n_seq, Ctot, 3] float32 or NULL: receives the last three
+ *                 inputs of each sequence, oldest first (positions before the
+ *                 sequence start come from conv_state_in), so that a later
+ *                 call can continue the sequences.  Must not overlap
+ *                 conv_state_in.
+ *  q, k           [T, Hqk, d] bf16 outputs;  v  [T, Hv, d] bf16 output.
+ * Arithmetic is float32; outputs are rounded to bf16 (nearest even).
+ * Supported: d = 128, Hqk >= 1, Hv >= 1.
+ */
+gdn_status gdn_conv1d_silu(const uint16_t* qkv, const float* conv_w, const int32_t* cu_seqlens,
+                           int32_t n_seq, int64_t T, int32_t Hqk, int32_t Hv, int32_t d,
+                           const float* conv_state_in, float* conv_state_out,
+                           uint16_t* q, uint16_t* k, uint16_t* v, gdn_stream_t stream);
+
+/*
+ * gdn_prefill_workspace_size -- bytes of device workspace gdn_prefill needs for
+ * these sizes (a multiple of 256).  Never 0.  Host-only, no CUDA calls.
+ */
+size_t gdn_prefill_workspace_size(int32_t n_seq, int64_t T, int32_t Hqk, int32_t Hv, int32_t d);
+
+/*
+ * gdn_prefill -- the recurrence over packed sequences, computed in chunks of
+ * 64 tokens (WY / UT form: decay-masked beta K K^T, (I + A)^{-1} by forward
+ * substitution, W and U, the intra-chunk output, then the inter-chunk state
+ * scan), with products on the tensor cores in bf16 and float32 accumulation,
+ * and the state carried in float32 (architecture page section 2.2: float32
+ * state).
+ *
+ *  q, k           [T, Hqk, d] bf16 (the recurrence uses them as given; the
+ *                 front end normalises them).
+ *  v              [T, Hv, d] bf16.
+ *  a, b           [T, Hv] float32 per-token gate inputs.
+ *  A_log, dt_bias [Hv] float32 per-head gate parameters.
+ *  scale          output scale (1/sqrt(d) for the layer).
+ *  initial_state  [n_seq, Hv, d_v, d_k] float32 (d_k contiguous) or NULL (zeros).
+ *  final_state    [n_seq, Hv, d_v, d_k] float32 or NULL (not written).  May be
+ *                 the same pointer as initial_state (updated in place).
+ *  o              [T, Hv, d] float32 output.
+ *  workspace      device scratch of at least gdn_prefill_workspace_size()
+ *                 bytes, 256-byte aligned; its contents on entry do not
+ *                 matter.  Calls that share a workspace must be ordered on
+ *                 one stream.
+ * A sequence of length 0 leaves final_state = initial_state (or zeros).
+ * Supported: d = 128, Hv % Hqk == 0.
+ * GDN_ERR_TIMEOUT is not returned here (the kernel does not stop the host):
+ * a kernel that gave up on a bounded wait records it in the workspace, and
+ * gdn_prefill_status() reports it.
+ */
+gdn_status gdn_prefill(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* a,
+                       const float* b, const float* A_log, const float* dt_bias,
+                       const int32_t* cu_seqlens, int32_t n_seq, int64_t T, int32_t Hqk,
+                       int32_t Hv, int32_t d, float scale, const float* initial_state,
+                       float* final_state, float* o, void* workspace, size_t workspace_bytes,
+                       gdn_stream_t stream);
+
+/*
+ * gdn_prefill_status -- waits for `stream`, then reads the error word that the
+ * last gdn_prefill on this workspace left: GDN_OK, or GDN_ERR_TIMEOUT if a
+ * bounded wait inside the kernel ran out (the outputs are then invalid).
+ * Synchronises the stream; not for use inside stream capture.
+ */
+gdn_status gdn_prefill_status(const void* workspace, gdn_stream_t stream);
+
+/*
+ * gdn_decode_step -- one token of the recurrence for many independent units
+ * (sequence s, layer l), unit u = s * layers + l, state updated in place.
+ * This is the constant-memory, O(d^2)-per-token step the pages contrast with a
+ * growing KV cache.
+ *
+ *  q, k           [U, Hqk, d] bf16, U = n_seq * layers.
+ *  v              [U, Hv, d] bf16.
+ *  a, b           [U, Hv] float32.
+ *  A_log, dt_bias [layers, Hv] float32 (unit u uses row u % layers).
+ *  state          [U, Hv, d_v, d_k] float32, read and overwritten in place.
+ *  o              [U, Hv, d] float32 output (o from the updated state).
+ * All arithmetic float32.  Supported: d = 128, Hv % Hqk == 0.
+ */
+gdn_status gdn_decode_step(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                           const float* a, const float* b, const float* A_log,
+                           const float* dt_bias, int32_t n_seq, int32_t layers, int32_t Hqk,
+                           int32_t Hv, int32_t d, float scale, float* state, float* o,
+                           gdn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

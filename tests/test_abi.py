@@ -1,0 +1,116 @@
+"""The C ABI on the CPU: the library exports every symbol include/gdn.h
+declares, and the host-side argument checks reject bad calls before any launch
+(these calls never reach CUDA)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from gated_deltanet_recurrence_prefill_b200 import build, _lib
+    build.build()
+    return _lib.lib()
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for required in ("gdn_conv1d_silu", "gdn_prefill", "gdn_prefill_workspace_size",
+                     "gdn_decode_step", "gdn_prefill_status", "gdn_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    from gated_deltanet_recurrence_prefill_b200 import _lib
+    names = declared_functions()
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in gdn.h but not exported"
+        assert n in _lib.SIGNATURES, f"{n} has no binding signature"
+
+
+def test_status_strings_and_version(L):
+    assert L.gdn_abi_version() == 1
+    for s in range(7):
+        assert L.gdn_status_string(s)
+    assert L.gdn_status_string(99) == b"unknown status"
+
+
+def test_workspace_size_is_positive_and_aligned(L):
+    for n, T in ((1, 256), (16, 270000), (1, 0)):
+        ws = L.gdn_prefill_workspace_size(n, T, 16, 48, 128)
+        assert ws > 0 and ws % 256 == 0
+
+
+FAKE = 0x10000     # 16-byte aligned non-null stand-in; never dereferenced: every call below fails validation
+
+
+def _p(x=FAKE):
+    return C.c_void_p(x)
+
+
+def test_prefill_rejects_bad_arguments(L):
+    ws = L.gdn_prefill_workspace_size(1, 64, 16, 48, 128)
+    good = dict(q=_p(), k=_p(), v=_p(), a=_p(), b=_p(), A_log=_p(), dt=_p(), cu=None, n=1, T=64,
+                Hqk=16, Hv=48, d=128, s0=None, s1=None, o=_p(), ws=_p(0x20000), wsb=ws)
+
+    def call(**kw):
+        a = dict(good, **kw)
+        return L.gdn_prefill(a["q"], a["k"], a["v"], a["a"], a["b"], a["A_log"], a["dt"], a["cu"],
+                             a["n"], a["T"], a["Hqk"], a["Hv"], a["d"], 0.088, a["s0"], a["s1"],
+                             a["o"], a["ws"], a["wsb"], None)
+
+    assert call(d=64) == 2                       # unsupported head width
+    assert call(Hv=40) == 2                      # Hv % Hqk != 0
+    assert call(Hqk=0) == 1
+    assert call(T=-1) == 1
+    assert call(n=2) == 1                        # several sequences need cu_seqlens
+    assert call(q=None) == 1
+    assert call(A_log=None) == 1
+    assert call(o=_p(FAKE + 4)) == 3             # misaligned
+    assert call(ws=None) == 6
+    assert call(wsb=ws - 1) == 6
+    assert call(ws=_p(0x20000 + 16)) == 3        # workspace must be 256-byte aligned
+
+
+def test_decode_rejects_bad_arguments(L):
+    def call(d=128, Hv=48, layers=48, state=_p(), q=_p()):
+        return L.gdn_decode_step(q, _p(), _p(), _p(), _p(), _p(), _p(), 4, layers, 16, Hv, d,
+                                 0.088, state, _p(), None)
+    assert call(d=256) == 2
+    assert call(Hv=47) == 2
+    assert call(layers=0) == 1
+    assert call(state=None) == 1
+    assert call(q=_p(FAKE + 2)) == 3
+    # zero sequences: nothing to do, no launch
+    assert L.gdn_decode_step(None, None, None, None, None, None, None, 0, 48, 16, 48, 128, 0.1,
+                             None, None, None) == 0
+
+
+def test_conv_rejects_bad_arguments(L):
+    def call(d=128, T=16, conv_w=_p(), cs_in=None, cs_out=None, q=_p()):
+        return L.gdn_conv1d_silu(_p(), conv_w, None, 1, T, 16, 48, d, cs_in, cs_out, q, _p(), _p(),
+                                 None)
+    assert call(d=64) == 2
+    assert call(conv_w=None) == 1
+    assert call(q=None) == 1
+    assert call(cs_in=_p(0x30000), cs_out=_p(0x30000)) == 1      # in/out state must differ
+    assert call(q=_p(FAKE + 8)) == 3
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    from gated_deltanet_recurrence_prefill_b200 import _lib
+    monkeypatch.setattr(_lib, "_LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(_lib, "_lib", None)
+    with pytest.raises(ImportError):
+        _lib.lib()
