@@ -109,7 +109,7 @@ gdn_status gdn_prefill(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = cudaMemsetAsync(workspace, 0, gdn::kWsHeaderBytes, s);
     if (e != cudaSuccess) return cuda_fail(e);
-    e = gdn::launch_prefill_simt(p, s);
+    e = gdn::launch_prefill_tc(p, s);
     return e == cudaSuccess ? GDN_OK : cuda_fail(e);
 }
 

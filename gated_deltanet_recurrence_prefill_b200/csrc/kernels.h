@@ -41,6 +41,8 @@ cudaError_t launch_conv1d_silu(const uint16_t* qkv, const float* w, const int32_
                                uint16_t* v, cudaStream_t stream);
 
 cudaError_t launch_prefill_simt(const PrefillArgs& p, cudaStream_t stream);
+cudaError_t launch_prefill_tc(const PrefillArgs& p, cudaStream_t stream);
+size_t prefill_tc_smem_bytes();
 size_t prefill_simt_smem_bytes();
 
 // workspace layout shared by the prefill kernels
