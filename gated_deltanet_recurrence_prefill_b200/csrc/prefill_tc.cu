@@ -23,7 +23,8 @@
 // value head; both solve the chunk's T themselves.  The CTA walks the
 // sequence's chunks in order with 12 warps:
 //   warp 0      TMA producer: [K; Q] tiles (2 stages) and the V slice
-//   warp 1      MMA issuer (one thread; also allocates TMEM)
+//   warp 1      MMA issuer for the state chain (one thread; also allocates TMEM)
+//   warp 2      MMA issuer for the precompute products (one thread)
 //   warps 4-7   chain epilogues (B, U, o, state), one TMEM lane quadrant each
 //   warps 8-11  precompute: gates, D0 -> A and P, T by blocked forward
 //               substitution (16x16 diagonal blocks on CUDA cores, the
@@ -70,8 +71,10 @@ constexpr uint32_t OFF_AF = OFF_ST + 16384;         // A: 64 x 68 f32
 constexpr uint32_t OFF_TF = OFF_AF + 64 * kLdF * 4; // T: 64 x 68 f32
 constexpr uint32_t OFF_XF = OFF_TF + 64 * kLdF * 4; // mma.sync scratch
 constexpr uint32_t XF_BYTES = 32 * 36 * 4;
-constexpr uint32_t OFF_GATES = OFF_XF + XF_BYTES;   // 4 buffers
-constexpr int kGateFloats = 4 * 64 + 4;             // beta, gamma, kappa, G; gC
+constexpr uint32_t OFF_AB = OFF_XF + XF_BYTES;      // 2 stages: a and b, 64 rows x 4 floats each
+constexpr uint32_t AB_STAGE = 2048;
+constexpr uint32_t OFF_GATES = OFF_AB + 2 * AB_STAGE; // 4 buffers
+constexpr int kGateFloats = 5 * 64 + 4;             // beta, gamma, kappa, G (log2 units), 1/gamma; gC, flag
 constexpr uint32_t OFF_MISC = OFF_GATES + 4 * kGateFloats * 4;
 constexpr uint32_t OFF_BARS = (OFF_MISC + 64 + 7) & ~7u;
 constexpr int kNumBars = 24;
@@ -82,7 +85,7 @@ constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // room to align the base
 enum {
     B_KQ_FULL = 0, B_KQ_EMPTY = 2, B_V_FULL = 4, B_V_EMPTY = 6,
     B_D0_FULL = 8, B_D0_EMPTY, B_TP_FULL, B_R_FULL, B_TR_FULL, B_TR_EMPTY,
-    B_Y_FULL, B_B_READY, B_Z_FULL, B_U_READY, B_S_FULL, B_ST_READY, B_S_SCALED, B_DRAIN
+    B_Y_FULL, B_B_READY, B_Z_FULL, B_U_READY, B_S_FULL, B_ST_READY, B_S_SCALED, B_DRAIN, B_DRAIN2
 };
 
 // TMEM columns
@@ -95,16 +98,23 @@ constexpr uint32_t IDESC_Y = idesc_bf16(128, kBV, false, true);
 constexpr uint32_t IDESC_Z = idesc_bf16(128, kBV, false, true);
 constexpr uint32_t IDESC_S = idesc_bf16(128, kBV, true, true);
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;    // 2 s: far beyond any legitimate wait
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr float kLog2e = 1.4426950408889634f;
+// chunks whose total decay stays above 2^-64 form the decay ratios as products
+constexpr float kFastDecayLog2 = 64.f;    // 2 s: far beyond any legitimate wait
 
 struct GateBuf {
     float beta[64];
     float gamma[64];
     float kappa[64];
     float G[64];
+    float igamma[64];      // 2^{-G}; meaningful when `fast`
     float gC;
-    float pad[3];
+    int fast;              // G_C >= -kFastDecayLog2: 2^{G_i - G_j} = gamma_i * igamma_j
+    float pad[2];
 };
+
+static_assert(sizeof(GateBuf) == kGateFloats * 4, "gate buffer layout");
 
 struct TcParams {
     const float* a;
@@ -119,6 +129,7 @@ struct TcParams {
     float* s_out;
     float* o;
     uint32_t* err;
+    int gate_tma;          // a, b staged by TMA (needs Hv % 4 == 0), else read directly
 };
 
 // K-major operand, K extent 128 split in two 16 KB panels of 128 rows
@@ -187,9 +198,12 @@ TC_DEVICE void ld_bf16x8(const uint8_t* tile, int row, int chunk, float* x) {
 
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const TcParams p) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
+                  const __grid_constant__ CUtensorMap tm_b, const TcParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // align to 1024 bytes by pointer arithmetic on the shared array, so that
+    // every access below stays in the shared state space (LDS/STS)
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BARS);
     auto bar = [&](int i) { return smem_u32(bars + i); };
@@ -244,6 +258,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mbar_init(bar(B_ST_READY), 4);
         mbar_init(bar(B_S_SCALED), 4);
         mbar_init(bar(B_DRAIN), 1);
+        mbar_init(bar(B_DRAIN2), 1);
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
@@ -258,12 +273,19 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v);
+            prefetch_tmap(&tm_a); prefetch_tmap(&tm_b);
             for (int c = 0; c < nch; ++c) {
                 const int s = c & 1, u = c >> 1;
                 const int32_t y = (int32_t)(bos + (int64_t)c * kC);
                 if (u >= 1 && !mbar_wait(bar(B_KQ_EMPTY + s), (u - 1) & 1, abort_flag, kWaitLimitNs)) break;
                 const uint32_t kq = sbase + OFF_KQ + s * KQ_STAGE;
-                mbar_arrive_expect_tx(bar(B_KQ_FULL + s), KQ_STAGE);
+                mbar_arrive_expect_tx(bar(B_KQ_FULL + s), KQ_STAGE + (p.gate_tma ? AB_STAGE : 0));
+                if (p.gate_tma) {
+                    // gate inputs: the 4-column group of a and b that holds column h
+                    const uint32_t ab = sbase + OFF_AB + s * AB_STAGE;
+                    tma_load_2d(ab, &tm_a, h & ~3, y, bar(B_KQ_FULL + s));
+                    tma_load_2d(ab + 1024, &tm_b, h & ~3, y, bar(B_KQ_FULL + s));
+                }
                 tma_load_2d(kq, &tm_k, g * kD, y, bar(B_KQ_FULL + s));
                 tma_load_2d(kq + 8192, &tm_q, g * kD, y, bar(B_KQ_FULL + s));
                 tma_load_2d(kq + KQ_PANEL, &tm_k, g * kD + 64, y, bar(B_KQ_FULL + s));
@@ -274,83 +296,64 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
+        // ------------------------------------------------------------ MMA issuer: state chain
+        // Y = [K;Q] S^T, Z = [T;R] B, S += K^T (kappa U), in order, each as soon
+        // as its operands are ready (blocking waits, no polling).
         if (lane == 0) {
-            int cY = 0, step = 0, cP = 0, cR = 0;
-            uint64_t t_progress = globaltimer_ns();
-            uint32_t idle = 0;
-            while (cY < nch) {
-                bool progressed = false;
-                if (step == 0) {
-                    if (mbar_try_wait(bar(B_ST_READY), cY & 1) && mbar_try_wait(bar(B_TR_FULL), cY & 1)) {
-                        tc_fence_after();
-                        const uint32_t kq = sbase + OFF_KQ + (cY & 1) * KQ_STAGE;
-                        for (int kk = 0; kk < 8; ++kk)
-                            mma_bf16(tmem + COL_Y, desc_kmajor_2panel(kq, kk),
-                                     desc_mnmajor(sbase + OFF_ST, kk, 16384), IDESC_Y, kk > 0);
-                        mma_commit(bar(B_Y_FULL));
-                        step = 1;
-                        progressed = true;
-                    }
-                } else if (step == 1) {
-                    if (mbar_try_wait(bar(B_B_READY), cY & 1)) {
-                        tc_fence_after();
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_bf16(tmem + COL_Z, desc_kmajor_1panel(sbase + OFF_PTR + 8192, kk),
-                                     desc_mnmajor(sbase + OFF_BB, kk, 8192), IDESC_Z, kk > 0);
-                        mma_commit(bar(B_Z_FULL));
-                        mma_commit(bar(B_TR_EMPTY));
-                        step = 2;
-                        progressed = true;
-                    }
-                } else {
-                    if (mbar_try_wait(bar(B_U_READY), cY & 1) && mbar_try_wait(bar(B_S_SCALED), cY & 1)) {
-                        tc_fence_after();
-                        const uint32_t kq = sbase + OFF_KQ + (cY & 1) * KQ_STAGE;
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_bf16(tmem + COL_S, desc_mnmajor(kq, kk, KQ_PANEL),
-                                     desc_mnmajor(sbase + OFF_UB, kk, 8192), IDESC_S, 1);
-                        mma_commit(bar(B_S_FULL));
-                        mma_commit(bar(B_KQ_EMPTY + (cY & 1)));
-                        step = 0;
-                        ++cY;
-                        progressed = true;
-                    }
-                }
-                if (cP < nch && mbar_try_wait(bar(B_KQ_FULL + (cP & 1)), (cP >> 1) & 1) &&
-                    (cP == 0 || mbar_try_wait(bar(B_D0_EMPTY), (cP - 1) & 1))) {
-                    tc_fence_after();
-                    const uint32_t kq = sbase + OFF_KQ + (cP & 1) * KQ_STAGE;
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_bf16(tmem + COL_D0, desc_kmajor_2panel(kq, kk), desc_kmajor_2panel(kq, kk),
-                                 IDESC_D0, kk > 0);
-                    mma_commit(bar(B_D0_FULL));
-                    ++cP;
-                    progressed = true;
-                }
-                if (cR < cP && mbar_try_wait(bar(B_TP_FULL), cR & 1)) {
-                    tc_fence_after();
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(tmem + COL_R, desc_kmajor_1panel(sbase + OFF_PTR, kk),
-                                 desc_mnmajor(sbase + OFF_PTR + 8192, kk, 8192), IDESC_R, kk > 0);
-                    mma_commit(bar(B_R_FULL));
-                    ++cR;
-                    progressed = true;
-                }
-                if (progressed) {
-                    idle = 0;
-                } else if ((++idle & 255u) == 0) {
-                    if (*abort_flag) break;
-                    const uint64_t now = globaltimer_ns();
-                    if (idle == 256u) t_progress = now;      // first idle check since progress
-                    else if (now - t_progress > kWaitLimitNs) { *abort_flag = 1; break; }
-                }
+            for (int c = 0; c < nch; ++c) {
+                const uint32_t kq = sbase + OFF_KQ + (c & 1) * KQ_STAGE;
+                if (!mbar_wait(bar(B_ST_READY), c & 1, abort_flag, kWaitLimitNs)) break;
+                if (!mbar_wait(bar(B_TR_FULL), c & 1, abort_flag, kWaitLimitNs)) break;
+                tc_fence_after();
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(tmem + COL_Y, desc_kmajor_2panel(kq, kk),
+                             desc_mnmajor(sbase + OFF_ST, kk, 16384), IDESC_Y, kk > 0);
+                mma_commit(bar(B_Y_FULL));
+                if (!mbar_wait(bar(B_B_READY), c & 1, abort_flag, kWaitLimitNs)) break;
+                tc_fence_after();
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tmem + COL_Z, desc_kmajor_1panel(sbase + OFF_PTR + 8192, kk),
+                             desc_mnmajor(sbase + OFF_BB, kk, 8192), IDESC_Z, kk > 0);
+                mma_commit(bar(B_Z_FULL));
+                mma_commit(bar(B_TR_EMPTY));
+                if (!mbar_wait(bar(B_U_READY), c & 1, abort_flag, kWaitLimitNs)) break;
+                if (!mbar_wait(bar(B_S_SCALED), c & 1, abort_flag, kWaitLimitNs)) break;
+                tc_fence_after();
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tmem + COL_S, desc_mnmajor(kq, kk, KQ_PANEL),
+                             desc_mnmajor(sbase + OFF_UB, kk, 8192), IDESC_S, 1);
+                mma_commit(bar(B_S_FULL));
+                mma_commit(bar(B_KQ_EMPTY + (c & 1)));
             }
-            // drain: every MMA issued so far has completed before TMEM is released
-            // (bounded even when the CTA is aborting)
+            // drain: every MMA issued by this thread has completed before TMEM is
+            // released (bounded even when the CTA is aborting)
             volatile int no_abort = 0;
             mma_commit(bar(B_DRAIN));
             mbar_wait(bar(B_DRAIN), 0, &no_abort, kWaitLimitNs);
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ MMA issuer: precompute
+        // D0 = [K;Q] K^T and R = [P;T] T for each chunk.
+        if (lane == 0) {
+            for (int c = 0; c < nch; ++c) {
+                const uint32_t kq = sbase + OFF_KQ + (c & 1) * KQ_STAGE;
+                if (!mbar_wait(bar(B_KQ_FULL + (c & 1)), (c >> 1) & 1, abort_flag, kWaitLimitNs)) break;
+                if (c > 0 && !mbar_wait(bar(B_D0_EMPTY), (c - 1) & 1, abort_flag, kWaitLimitNs)) break;
+                tc_fence_after();
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(tmem + COL_D0, desc_kmajor_2panel(kq, kk), desc_kmajor_2panel(kq, kk),
+                             IDESC_D0, kk > 0);
+                mma_commit(bar(B_D0_FULL));
+                if (!mbar_wait(bar(B_TP_FULL), c & 1, abort_flag, kWaitLimitNs)) break;
+                tc_fence_after();
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tmem + COL_R, desc_kmajor_1panel(sbase + OFF_PTR, kk),
+                             desc_mnmajor(sbase + OFF_PTR + 8192, kk, 8192), IDESC_R, kk > 0);
+                mma_commit(bar(B_R_FULL));
+            }
+            volatile int no_abort = 0;
+            mma_commit(bar(B_DRAIN2));
+            mbar_wait(bar(B_DRAIN2), 0, &no_abort, kWaitLimitNs);
         }
     } else if (warp >= 4 && warp < 8) {
         // ------------------------------------------------------------ chain epilogues
@@ -490,62 +493,104 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         for (int c = 0; c < nch; ++c) {
             GateBuf& gb = gates[c & 3];
             const int64_t tok0 = bos + (int64_t)c * kC;
-            // ---- gates: G = running sum of log(alpha); beta; gamma = e^G; kappa = e^{G_C - G}
-            if (pw < 2) {
-                const int t = pt;
+            // ---- gates (warps 10, 11): G = running sum of log2(alpha); beta;
+            //      gamma = 2^G; kappa = 2^{G_C - G}
+            if (pw >= 2) {
+                const int t = pt - 64;
                 const int64_t tok = tok0 + t;
+                mbar_wait(bar(B_KQ_FULL + (c & 1)), (c >> 1) & 1, abort_flag, kWaitLimitNs);
+                const float* abt = reinterpret_cast<const float*>(sm + OFF_AB + (c & 1) * AB_STAGE);
                 float lg = 0.f, be = 0.f;
                 if (tok < eos) {
-                    lg = log_alpha_f32(p.a[tok * p.Hv + h], Al, dtb);
-                    be = sigmoid_f32(p.b[tok * p.Hv + h]);
+                    const float av = p.gate_tma ? abt[t * 4 + (h & 3)] : p.a[tok * p.Hv + h];
+                    const float bv = p.gate_tma ? abt[256 + t * 4 + (h & 3)] : p.b[tok * p.Hv + h];
+                    lg = kLog2e * log_alpha_f32(av, Al, dtb);
+                    be = sigmoid_f32(bv);
                 }
                 float run = lg;
                 for (int m = 1; m < 32; m <<= 1) {
                     const float o = __shfl_up_sync(0xffffffffu, run, m);
                     if (lane >= m) run += o;
                 }
-                if (pw == 0 && lane == 31) xchg[0] = run;
+                if (pw == 2 && lane == 31) xchg[0] = run;
                 named_bar_sync(3, 64);
-                if (pw == 1) run += xchg[0];
+                if (pw == 3) run += xchg[0];
                 gb.G[t] = run;
                 gb.beta[t] = be;
-                gb.gamma[t] = expf(run);
-                if (t == 63) { xchg[1] = run; gb.gC = expf(run); }
+                gb.gamma[t] = exp2f(run);
+                if (t == 63) {
+                    xchg[1] = run;
+                    gb.gC = exp2f(run);
+                    gb.fast = run >= -kFastDecayLog2 ? 1 : 0;
+                }
                 named_bar_sync(3, 64);
-                gb.kappa[t] = expf(xchg[1] - run);
+                gb.kappa[t] = exp2f(xchg[1] - run);
+                gb.igamma[t] = xchg[1] >= -kFastDecayLog2 ? exp2f(-run) : 0.f;
             }
             named_bar_sync(1, 128);
             // ---- D0 rows -> A (f32 scratch) and P (bf16 operand)
             mbar_wait(bar(B_D0_FULL), c & 1, abort_flag, kWaitLimitNs);
             tc_fence_after();
+            // decay ratio 2^{G_i - G_j} (j <= i): gamma_i * igamma_j when the chunk's
+            // decay is moderate, else one exp2 per element (never overflows: G_i <= G_j)
+            const bool fast = gb.fast != 0;
             if (pw < 2) {
+                // A_ij = beta_i 2^{G_i - G_j} (k_i . k_j), j < i
                 const int i = pt;
-                const float Gi = gb.G[i], bi = gb.beta[i];
+                const float Gi = gb.G[i];
+                const float ci = fast ? gb.beta[i] * gb.gamma[i] : gb.beta[i];
+                float* arow = Af + i * kLdF;
                 for (int half = 0; half < 2; ++half) {
                     float kk[32];
                     tmem_ld32(tl + COL_D0 + half * 32, kk);
                     tmem_ld_wait();
+#pragma unroll
                     for (int j4 = 0; j4 < 32; j4 += 4) {
+                        const int j = half * 32 + j4;
                         float4 w;
-                        float* wv = &w.x;
-                        for (int e = 0; e < 4; ++e) {
-                            const int j = half * 32 + j4 + e;
-                            wv[e] = j < i ? bi * expf(Gi - gb.G[j]) * kk[j4 + e] : 0.f;
+                        if (fast) {
+                            const float4 ig = *reinterpret_cast<const float4*>(&gb.igamma[j]);
+                            w.x = (j + 0 < i) ? ci * kk[j4 + 0] * ig.x : 0.f;
+                            w.y = (j + 1 < i) ? ci * kk[j4 + 1] * ig.y : 0.f;
+                            w.z = (j + 2 < i) ? ci * kk[j4 + 2] * ig.z : 0.f;
+                            w.w = (j + 3 < i) ? ci * kk[j4 + 3] * ig.w : 0.f;
+                        } else {
+                            const float4 gj = *reinterpret_cast<const float4*>(&gb.G[j]);
+                            w.x = (j + 0 < i) ? ci * kk[j4 + 0] * exp2f(Gi - gj.x) : 0.f;
+                            w.y = (j + 1 < i) ? ci * kk[j4 + 1] * exp2f(Gi - gj.y) : 0.f;
+                            w.z = (j + 2 < i) ? ci * kk[j4 + 2] * exp2f(Gi - gj.z) : 0.f;
+                            w.w = (j + 3 < i) ? ci * kk[j4 + 3] * exp2f(Gi - gj.w) : 0.f;
                         }
-                        *reinterpret_cast<float4*>(Af + i * kLdF + half * 32 + j4) = w;
+                        *reinterpret_cast<float4*>(arow + j) = w;
                     }
                 }
             } else {
+                // P_ij = 2^{G_i - G_j} (q_i . k_j), j <= i
                 const int i = pt - 64;
                 const float Gi = gb.G[i];
+                const float ci = fast ? gb.gamma[i] : 1.f;
                 for (int half = 0; half < 2; ++half) {
                     float qk[32];
                     tmem_ld32(tl + COL_D0 + half * 32, qk);
                     tmem_ld_wait();
-                    for (int j = 0; j < 32; ++j) {
-                        const int jj = half * 32 + j;
-                        qk[j] = jj <= i ? expf(Gi - gb.G[jj]) * qk[j] : 0.f;
+#pragma unroll
+                    for (int j4 = 0; j4 < 32; j4 += 4) {
+                        const int j = half * 32 + j4;
+                        if (fast) {
+                            const float4 ig = *reinterpret_cast<const float4*>(&gb.igamma[j]);
+                            qk[j4 + 0] = (j + 0 <= i) ? ci * qk[j4 + 0] * ig.x : 0.f;
+                            qk[j4 + 1] = (j + 1 <= i) ? ci * qk[j4 + 1] * ig.y : 0.f;
+                            qk[j4 + 2] = (j + 2 <= i) ? ci * qk[j4 + 2] * ig.z : 0.f;
+                            qk[j4 + 3] = (j + 3 <= i) ? ci * qk[j4 + 3] * ig.w : 0.f;
+                        } else {
+                            const float4 gj = *reinterpret_cast<const float4*>(&gb.G[j]);
+                            qk[j4 + 0] = (j + 0 <= i) ? qk[j4 + 0] * exp2f(Gi - gj.x) : 0.f;
+                            qk[j4 + 1] = (j + 1 <= i) ? qk[j4 + 1] * exp2f(Gi - gj.y) : 0.f;
+                            qk[j4 + 2] = (j + 2 <= i) ? qk[j4 + 2] * exp2f(Gi - gj.z) : 0.f;
+                            qk[j4 + 3] = (j + 3 <= i) ? qk[j4 + 3] * exp2f(Gi - gj.w) : 0.f;
+                        }
                     }
+#pragma unroll
                     for (int j = 0; j < 4; ++j) st_bf16x8(sm + OFF_PTR, i, half * 4 + j, qk + 8 * j);
                 }
             }
@@ -561,10 +606,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 float x[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    float acc = (i == col) ? 1.f : 0.f;
+                    // x_i = delta_{i,col} - sum_{m<i} A_im x_m, with four partial sums
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int m = 0; m < i; ++m) acc = fmaf(-Ab[i * kLdF + m], x[m], acc);
-                    x[i] = acc;
+                    for (int m = 0; m < i; ++m) acc[m & 3] = fmaf(Ab[i * kLdF + m], x[m], acc[m & 3]);
+                    x[i] = ((i == col) ? 1.f : 0.f) - ((acc[0] + acc[1]) + (acc[2] + acc[3]));
                 }
                 if (lane < 16) {
 #pragma unroll
@@ -604,8 +650,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (c >= 1) mbar_wait(bar(B_TR_EMPTY), (c - 1) & 1, abort_flag, kWaitLimitNs);
             for (int u = pt; u < 64 * 8; u += 128) {
                 const int row = u >> 3, chunk = u & 7;
-                float x[8];
-                for (int e = 0; e < 8; ++e) x[e] = Tf[row * kLdF + chunk * 8 + e];
+                const float4 t0 = *reinterpret_cast<const float4*>(Tf + row * kLdF + chunk * 8);
+                const float4 t1 = *reinterpret_cast<const float4*>(Tf + row * kLdF + chunk * 8 + 4);
+                const float x[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
                 st_bf16x8(sm + OFF_PTR + 8192, row, chunk, x);
             }
             fence_async_smem();
@@ -671,6 +718,19 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2D float tensor [rows, cols], 4-column x 64-row boxes, no swizzle
+bool make_map_gates(CUtensorMap* m, const float* base, int64_t rows, int64_t cols) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+    cuuint32_t box[2] = {4, 64};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 size_t prefill_tc_smem_bytes() { return SMEM_ALLOC; }
@@ -687,19 +747,29 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
         }
         return cudaSuccess;
     }
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, ma, mb;
     if (!make_map(&mq, a.q, a.T, (int64_t)a.Hqk * kD) || !make_map(&mk, a.k, a.T, (int64_t)a.Hqk * kD) ||
         !make_map(&mv, a.v, a.T, (int64_t)a.Hv * kD))
         return cudaErrorInvalidValue;
+    // a and b rows must be a multiple of 16 bytes for TMA; otherwise they are read directly
+    const int gate_tma = (a.Hv % 4 == 0) ? 1 : 0;
+    if (gate_tma) {
+        if (!make_map_gates(&ma, a.a, a.T, a.Hv) || !make_map_gates(&mb, a.b, a.T, a.Hv))
+            return cudaErrorInvalidValue;
+    } else {
+        ma = mq;
+        mb = mq;       // unused
+    }
     cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     TcParams p{a.a, a.b, a.A_log, a.dt_bias, a.cu_seqlens, a.T, a.Hqk, a.Hv, a.scale,
                a.initial_state, a.final_state, a.o,
-               reinterpret_cast<uint32_t*>(static_cast<char*>(a.workspace) + kWsErrorWordOffset)};
+               reinterpret_cast<uint32_t*>(static_cast<char*>(a.workspace) + kWsErrorWordOffset),
+               gate_tma};
     const int64_t blocks = (int64_t)a.n_seq * a.Hv * (kD / kBV);
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    prefill_tc_kernel<<<(unsigned)blocks, kThreads, SMEM_ALLOC, stream>>>(mq, mk, mv, p);
+    prefill_tc_kernel<<<(unsigned)blocks, kThreads, SMEM_ALLOC, stream>>>(mq, mk, mv, ma, mb, p);
     return cudaGetLastError();
 }
 

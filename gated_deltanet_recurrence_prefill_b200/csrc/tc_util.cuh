@@ -42,11 +42,26 @@ TC_DEVICE void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
                  : "memory");
 }
 
-TC_DEVICE bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+// Waits for the phase with the given parity to complete, suspending the warp
+// (it issues nothing) for up to `hint_ns`; true once the phase has completed.
+TC_DEVICE bool mbar_try_wait(uint32_t bar, uint32_t parity, uint32_t hint_ns = 20000) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// non-blocking test of a phase (for polling several barriers from one thread)
+TC_DEVICE bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(bar), "r"(parity)
@@ -62,7 +77,7 @@ TC_DEVICE bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, uin
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63u) == 0) {
+        if ((it & 3u) == 0) {
             if (*abort) return false;
             if (globaltimer_ns() - t0 > limit_ns) {
                 *abort = 1;
