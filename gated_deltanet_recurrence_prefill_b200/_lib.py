@@ -31,6 +31,8 @@ SIGNATURES = {
     "gdn_prefill": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32,
                               _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "gdn_prefill_status": (C.c_int, [_vp, _vp]),
+    "gdn_prefill_noalloc": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
+                                      _i32, _f32, _vp, _vp, _vp, _vp]),
     "gdn_decode_step": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                   _f32, _vp, _vp, _vp]),
 }
@@ -160,6 +162,42 @@ def prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens=None, scale=None, initial_
                            _ptr(initial_state), _ptr(final_state), _ptr(o), _ptr(workspace),
                            workspace.numel() * workspace.element_size(), _stream(stream))
     _check("gdn_prefill", st)
+    return o, final_state
+
+
+def prefill_noalloc(q, k, v, a, b, A_log, dt_bias, cu_seqlens=None, scale=None,
+                    initial_state=None, final_state=None, o=None, want_final_state=True,
+                    stream=None):
+    """gdn_prefill_noalloc: the chunked prefill without a caller-provided
+    workspace, for callers that cannot allocate device memory (the library
+    uses its own fixed 64 KiB device array; see include/gdn.h).  The output
+    tensors are created here only when not passed in."""
+    import torch
+    T, Hqk, d = q.shape
+    Hv = v.shape[1]
+    n_seq = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _need(q, torch.bfloat16, (T, Hqk, d), "q")
+    _need(k, torch.bfloat16, (T, Hqk, d), "k")
+    _need(v, torch.bfloat16, (T, Hv, d), "v")
+    _need(a, torch.float32, (T, Hv), "a")
+    _need(b, torch.float32, (T, Hv), "b")
+    _need(A_log, torch.float32, (Hv,), "A_log")
+    _need(dt_bias, torch.float32, (Hv,), "dt_bias")
+    if cu_seqlens is not None:
+        _need(cu_seqlens, torch.int32, (n_seq + 1,), "cu_seqlens")
+    if initial_state is not None:
+        _need(initial_state, torch.float32, (n_seq, Hv, d, d), "initial_state")
+    if scale is None:
+        scale = d ** -0.5
+    if o is None:
+        o = torch.empty(T, Hv, d, dtype=torch.float32, device=q.device)
+    if final_state is None and want_final_state:
+        final_state = torch.empty(n_seq, Hv, d, d, dtype=torch.float32, device=q.device)
+    st = lib().gdn_prefill_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(A_log),
+                                   _ptr(dt_bias), _ptr(cu_seqlens), n_seq, T, Hqk, Hv, d,
+                                   float(scale), _ptr(initial_state), _ptr(final_state), _ptr(o),
+                                   _stream(stream))
+    _check("gdn_prefill_noalloc", st)
     return o, final_state
 
 

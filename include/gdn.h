@@ -156,6 +156,37 @@ gdn_status gdn_prefill(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
 gdn_status gdn_prefill_status(const void* workspace, gdn_stream_t stream);
 
 /*
+ * gdn_prefill_noalloc -- gdn_prefill for callers that cannot allocate device
+ * memory (the pages describe no such variant; it has no counterpart there).
+ * Some callers own no allocator for the GPU: a host framework that manages
+ * all device memory in its own arena and passes in only the model's tensors,
+ * a plugin that is handed input and output pointers, or a latency-critical
+ * loop where cudaMalloc (which can synchronise the device) is not allowed.
+ * This entry point takes the same arguments as gdn_prefill minus the
+ * workspace, and calls no cudaMalloc, cudaFree or other allocating routine.
+ *
+ * The workspace lives instead in a fixed array of 64 KiB inside the library's
+ * device image (every GPU that loads the library holds it until the process
+ * exits).  That bounds n_seq * Hv to 16320 (for example 340 sequences of 48
+ * value heads); larger problems are rejected with GDN_ERR_WORKSPACE before
+ * anything touches the GPU.
+ *
+ * The first call on each device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture.  All calls in the process share the one array, which keeps what the
+ * last call left there: calls that overlap on the GPU (different streams,
+ * devices not involved) race on it, so order them on one stream.  A bounded
+ * device wait that times out is recorded in that shared array and is not
+ * reported by this entry point.
+ */
+gdn_status gdn_prefill_noalloc(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                               const float* a, const float* b, const float* A_log,
+                               const float* dt_bias, const int32_t* cu_seqlens, int32_t n_seq,
+                               int64_t T, int32_t Hqk, int32_t Hv, int32_t d, float scale,
+                               const float* initial_state, float* final_state, float* o,
+                               gdn_stream_t stream);
+
+/*
  * gdn_decode_step -- one token of the recurrence for many independent units
  * (sequence s, layer l), unit u = s * layers + l, state updated in place.
  * This is the constant-memory, O(d^2)-per-token step the pages contrast with a
