@@ -21,6 +21,7 @@ constexpr int kD = 128;
 constexpr int kRun = 32;              // tokens per warp
 constexpr int kWarps = 8;             // warps per CTA
 constexpr int kChan = 8;              // channels per lane
+constexpr int kBatch = 8;             // tokens whose loads are in flight together
 
 // index of the sequence containing token t: largest n with cu[n] <= t
 __device__ int find_seq(const int32_t* cu, int n_seq, int64_t t) {
@@ -32,6 +33,17 @@ __device__ int find_seq(const int32_t* cu, int n_seq, int64_t t) {
     return lo;
 }
 
+GDN_DEVICE uint4 ldg_stream(const uint16_t* p) { return __ldcs(reinterpret_cast<const uint4*>(p)); }
+GDN_DEVICE void stg_stream(uint16_t* p, uint4 v) { __stcs(reinterpret_cast<uint4*>(p), v); }
+
+GDN_DEVICE void unpack8(const uint4 r, float* x) {
+    float2 t;
+    t = bf16x2_to_f32x2(r.x); x[0] = t.x; x[1] = t.y;
+    t = bf16x2_to_f32x2(r.y); x[2] = t.x; x[3] = t.y;
+    t = bf16x2_to_f32x2(r.z); x[4] = t.x; x[5] = t.y;
+    t = bf16x2_to_f32x2(r.w); x[6] = t.x; x[7] = t.y;
+}
+
 GDN_DEVICE void load8(const uint16_t* p, float* x) {
     const uint4 r = *reinterpret_cast<const uint4*>(p);
     float2 t;
@@ -41,7 +53,7 @@ GDN_DEVICE void load8(const uint16_t* p, float* x) {
     t = bf16x2_to_f32x2(r.w); x[6] = t.x; x[7] = t.y;
 }
 
-__global__ void __launch_bounds__(kWarps * 32)
+__global__ void __launch_bounds__(kWarps * 32, 2)
 conv1d_silu_kernel(const uint16_t* __restrict__ qkv, const float* __restrict__ w,
                    const int32_t* __restrict__ cu, int32_t n_seq, int64_t T, int32_t Hqk,
                    int32_t Hv, const float* __restrict__ cs_in, uint16_t* __restrict__ qo,
@@ -100,45 +112,58 @@ conv1d_silu_kernel(const uint16_t* __restrict__ qkv, const float* __restrict__ w
     else { dst_base = vo + (int64_t)(hc - 2 * Hqk) * kD; dst_stride = (int64_t)Hv * kD; }
     dst_base += (lane & 15) * kChan;
 
-    for (int64_t t = t0; t < t1; ++t) {
-        if (t >= eos) {
-            // next sequence(s): skip empty ones, restart the history
-            while (n + 1 < n_seq && (int64_t)cu[n + 1] <= t) ++n;
-            bos = cu[n];
-            eos = cu[n + 1];
+    // tokens are processed in batches of kBatch: all loads of a batch are issued
+    // before any is used, so that kBatch x 16 bytes per lane are in flight
+    for (int64_t tb = t0; tb < t1; tb += kBatch) {
+        uint4 raw[kBatch];
 #pragma unroll
-            for (int j = 0; j < 3; ++j)
-#pragma unroll
-                for (int i = 0; i < kChan; ++i)
-                    hist[j][i] = cs_in ? cs_in[((int64_t)n * Ctot + c0 + i) * 3 + j] : 0.f;
+        for (int u = 0; u < kBatch; ++u) {
+            const int64_t t = tb + u;
+            raw[u] = t < t1 ? ldg_stream(qkv + t * Ctot + c0) : make_uint4(0, 0, 0, 0);
         }
-        float x[kChan];
-        load8(qkv + t * Ctot + c0, x);
-        float y[kChan];
-        float ss = 0.f;
 #pragma unroll
-        for (int i = 0; i < kChan; ++i) {
-            float acc = wr[i][0] * hist[0][i];
-            acc = fmaf(wr[i][1], hist[1][i], acc);
-            acc = fmaf(wr[i][2], hist[2][i], acc);
-            acc = fmaf(wr[i][3], x[i], acc);
-            const float s = acc / (1.f + expf(-acc));
-            y[i] = s;
-            ss = fmaf(s, s, ss);
-            hist[0][i] = hist[1][i];
-            hist[1][i] = hist[2][i];
-            hist[2][i] = x[i];
+        for (int u = 0; u < kBatch; ++u) {
+            const int64_t t = tb + u;
+            if (t >= t1) break;
+            if (t >= eos) {
+                // next sequence(s): skip empty ones, restart the history
+                while (n + 1 < n_seq && (int64_t)cu[n + 1] <= t) ++n;
+                bos = cu[n];
+                eos = cu[n + 1];
+#pragma unroll
+                for (int j = 0; j < 3; ++j)
+#pragma unroll
+                    for (int i = 0; i < kChan; ++i)
+                        hist[j][i] = cs_in ? cs_in[((int64_t)n * Ctot + c0 + i) * 3 + j] : 0.f;
+            }
+            float x[kChan];
+            unpack8(raw[u], x);
+            float y[kChan];
+            float ss = 0.f;
+#pragma unroll
+            for (int i = 0; i < kChan; ++i) {
+                float acc = wr[i][0] * hist[0][i];
+                acc = fmaf(wr[i][1], hist[1][i], acc);
+                acc = fmaf(wr[i][2], hist[2][i], acc);
+                acc = fmaf(wr[i][3], x[i], acc);
+                const float s = acc / (1.f + __expf(-acc));
+                y[i] = s;
+                ss = fmaf(s, s, ss);
+                hist[0][i] = hist[1][i];
+                hist[1][i] = hist[2][i];
+                hist[2][i] = x[i];
+            }
+            // sum of squares over the 16 lanes of this head
+#pragma unroll
+            for (int m = 8; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+            const float inv = (is_q || is_k) ? rsqrtf(ss + 1e-6f) : 1.f;
+            uint4 out;
+            out.x = pack_bf16x2(y[0] * inv, y[1] * inv);
+            out.y = pack_bf16x2(y[2] * inv, y[3] * inv);
+            out.z = pack_bf16x2(y[4] * inv, y[5] * inv);
+            out.w = pack_bf16x2(y[6] * inv, y[7] * inv);
+            if (active) stg_stream(dst_base + t * dst_stride, out);
         }
-        // sum of squares over the 16 lanes of this head
-#pragma unroll
-        for (int m = 8; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-        const float inv = (is_q || is_k) ? rsqrtf(ss + 1e-6f) : 1.f;
-        uint4 out;
-        out.x = pack_bf16x2(y[0] * inv, y[1] * inv);
-        out.y = pack_bf16x2(y[2] * inv, y[3] * inv);
-        out.z = pack_bf16x2(y[4] * inv, y[5] * inv);
-        out.w = pack_bf16x2(y[6] * inv, y[7] * inv);
-        if (active) *reinterpret_cast<uint4*>(dst_base + t * dst_stride) = out;
     }
 }
 

@@ -118,7 +118,11 @@ def test_varlen_equals_separate_calls():
 
 def test_split_prefill_equals_whole():
     """prefill(T1) then prefill(T2, initial = final of the first) equals
-    prefill(T1 + T2) when T1 is a whole number of chunks (bit for bit)."""
+    prefill(T1 + T2) when T1 is a whole number of chunks.  The kernel carries
+    the state as Gamma * S~ with a running scale and rounds a bf16 copy of it
+    each chunk, so the two runs round at different points: they agree within
+    the parity bound (a wrong state hand-off would be off by O(1)), and the
+    first part, computed identically, agrees bit for bit."""
     import torch
     inp = synth.make_prefill([384], seed=65, init_state=True, Hqk=4, Hv=12)
     o, s = _run(inp)
@@ -131,8 +135,10 @@ def test_split_prefill_equals_whole():
                                  inp.A_log, inp.dt_bias, np.array([0, 384 - T1], np.int32),
                                  host(s1).astype(np.float32), inp.scale, inp.Hqk, inp.Hv, inp.d)
     o2, s2 = _run(second)
-    assert torch.equal(torch.cat([o1, o2]), o)
-    assert torch.equal(s2, s)
+    assert rel_err(host(torch.cat([o1, o2])), host(o)) <= TOL
+    assert rel_err(host(s2), host(s)) <= TOL
+    # the first part is the same computation on the same inputs: bit for bit
+    assert torch.equal(o1, o[:T1])
 
 
 def test_prefill_one_token_equals_decode_step():
