@@ -42,6 +42,27 @@ FRONTEND_BYTES_PER_TOKEN = 2 * 2 * (2 * HQK + HV) * D
 STATE_BYTES = HV * D * D * 4
 
 
+def kernel_traffic(name):
+    """DRAM bytes per launch of kernel `name` on the bench workload, from the
+    committed ncu record profiles/ncu_traffic.json -- or None when there is no
+    record or the kernel's source has changed since the counters were taken."""
+    import hashlib
+    rec_path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(rec_path):
+        return None
+    with open(rec_path) as f:
+        rec = json.load(f).get(name)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, "gated_deltanet_recurrence_prefill_b200", "csrc", rec["source"])
+    if not os.path.exists(src):
+        return None
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+            return None
+    return int(rec["dram_bytes_per_launch"])
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -244,7 +265,8 @@ def bench_main(args, world, rank, local):
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     roofline = {"kernel": dom, "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": kernel_traffic("prefill" if dom == "prefill" else "conv1d_silu"),
                 "peak_source": peaks["source"], "bytes_per_launch": dom_bytes,
                 "kernel_ms": round(dom_ms, 4)}
     prefill_tflops = FLOP_PER_TOKEN * T / (prefill_ms * 1e-3) / 1e12
@@ -450,6 +472,43 @@ def cpu_baseline(seconds: float = 15.0, threads: int = 0):
                       f"scaled to 48 heads"}
 
 
+def profile_case(args):
+    """Runs one kernel a few times on a small case for an ncu capture (not a
+    benchmark: nothing is timed or printed as a result).
+      prefill8k   gdn_prefill, T=8192, 1 sequence, S0 != 0   (~0.5 GB resident)
+      frontend8k  gdn_conv1d_silu, T=8192                      (~0.4 GB)
+      decode16    gdn_decode_step, 16 sequences x 48 layers    (~2.4 GB of state)
+    """
+    import numpy as np
+    import torch
+    import gated_deltanet_recurrence_prefill_b200 as gdn
+    import synth
+    dev = torch.device("cuda", 0)
+    to16 = lambda x: torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).to(dev)
+    f32 = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(dev)
+    if args.profile_case == "prefill8k":
+        inp = synth.make_prefill([T_MAIN], 1, init_state=True)
+        d = [to16(inp.q), to16(inp.k), to16(inp.v), f32(inp.a), f32(inp.b), f32(inp.A_log), f32(inp.dt_bias)]
+        s0 = f32(inp.initial_state)
+        for _ in range(args.warmup + args.steps):
+            gdn.prefill(*d, initial_state=s0)
+    elif args.profile_case == "frontend8k":
+        fe = synth.workload(1)
+        x, w = to16(fe.qkv), f32(fe.conv_w)
+        for _ in range(args.warmup + args.steps):
+            gdn.conv1d_silu(x, w, HQK, HV)
+    elif args.profile_case == "decode16":
+        inp = synth.make_decode(16, 48, 4)
+        st = torch.empty(inp.U, HV, D, D, dtype=torch.float32, device=dev)
+        st.normal_(0.0, 0.02)
+        args_ = [to16(inp.q), to16(inp.k), to16(inp.v), f32(inp.a), f32(inp.b), f32(inp.A_log),
+                 f32(inp.dt_bias), st, inp.n_seq, inp.layers]
+        for _ in range(args.warmup + args.steps):
+            gdn.decode_step(*args_)
+    torch.cuda.synchronize()
+    print(f"profile case {args.profile_case}: ok")
+
+
 def run_reference(args, world, rank):
     if rank != 0:
         return
@@ -487,10 +546,15 @@ def main():
     ap.add_argument("--primary-only", action="store_true", help="skip the 262K and decode lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--profile-case", choices=["prefill8k", "frontend8k", "decode16"],
+                    help="run one kernel on a small case for an ncu capture; no timing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, local = _dist()
+    if args.profile_case:
+        profile_case(args)
+        return
     if args.impl == "reference":
         run_reference(args, world, rank)
         return
