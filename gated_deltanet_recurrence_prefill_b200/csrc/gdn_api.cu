@@ -3,6 +3,8 @@
 // frees or synchronises, except gdn_prefill_status, which documents that it
 // waits for the stream.
 #include <cuda_runtime.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "../../include/gdn.h"
 #include "kernels.h"
@@ -34,7 +36,34 @@ gdn_status check_seqs(const int32_t* cu_seqlens, int32_t n_seq, int64_t T) {
     return GDN_OK;
 }
 
+// Which prefill kernel runs: the cluster kernel (two producer CTAs and one
+// consumer CTA per sequence and value head) wherever clusters of three fit on
+// the device, else the single-CTA kernel.  GDN_PREFILL_KERNEL=single or
+// =cluster in the environment forces one of them (for comparisons and tests).
+// The cluster kernel also needs the workspace to hold its ring of chunk slots
+// (gdn_prefill_workspace_size); with less, the single-CTA kernel runs.
+enum class PrefillKernel { Cluster, Single, Unavailable };
+
+PrefillKernel pick_prefill_kernel(bool ring_fits) {
+    const char* env = getenv("GDN_PREFILL_KERNEL");
+    if (env && strcmp(env, "single") == 0) return PrefillKernel::Single;
+    const bool cl = ring_fits && gdn::prefill_cl_available();
+    if (env && strcmp(env, "cluster") == 0) return cl ? PrefillKernel::Cluster : PrefillKernel::Unavailable;
+    return cl ? PrefillKernel::Cluster : PrefillKernel::Single;
+}
+
 }  // namespace
+
+namespace gdn {
+
+size_t prefill_min_workspace_bytes(int32_t n_seq, int32_t Hv) {
+    const size_t n = n_seq > 0 ? (size_t)n_seq : 1;
+    const size_t hv = Hv > 0 ? (size_t)Hv : 1;
+    // header (error word) + one int32 per (sequence, value head)
+    return kWsHeaderBytes + ((n * hv * sizeof(int32_t) + 255) / 256) * 256;
+}
+
+}  // namespace gdn
 
 extern "C" {
 
@@ -79,11 +108,9 @@ gdn_status gdn_conv1d_silu(const uint16_t* qkv, const float* conv_w, const int32
 
 size_t gdn_prefill_workspace_size(int32_t n_seq, int64_t T, int32_t Hqk, int32_t Hv, int32_t d) {
     (void)T; (void)Hqk; (void)d;
-    size_t n = n_seq > 0 ? (size_t)n_seq : 1;
-    size_t hv = Hv > 0 ? (size_t)Hv : 1;
-    // header (error word) + one int32 per (sequence, value head) for the schedule
-    size_t bytes = gdn::kWsHeaderBytes + ((n * hv * sizeof(int32_t) + 255) / 256) * 256;
-    return bytes;
+    const size_t lo = gdn::prefill_min_workspace_bytes(n_seq, Hv);
+    const size_t hi = gdn::prefill_cl_workspace_bytes(n_seq, Hv);
+    return hi > lo ? hi : lo;
 }
 
 gdn_status gdn_prefill(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* a,
@@ -101,15 +128,18 @@ gdn_status gdn_prefill(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
                           o};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
-    if (!workspace || workspace_bytes < gdn_prefill_workspace_size(n_seq, T, Hqk, Hv, d))
+    if (!workspace || workspace_bytes < gdn::prefill_min_workspace_bytes(n_seq, Hv))
         return GDN_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_MISALIGNED;
     gdn::PrefillArgs p{q, k, v, a, b, A_log, dt_bias, cu_seqlens, n_seq, T, Hqk, Hv, scale,
                        initial_state, final_state, o, workspace, workspace_bytes};
+    const PrefillKernel which =
+        pick_prefill_kernel(workspace_bytes >= gdn::prefill_cl_workspace_bytes(n_seq, Hv));
+    if (which == PrefillKernel::Unavailable) return GDN_ERR_UNSUPPORTED;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = cudaMemsetAsync(workspace, 0, gdn::kWsHeaderBytes, s);
     if (e != cudaSuccess) return cuda_fail(e);
-    e = gdn::launch_prefill_tc(p, s);
+    e = which == PrefillKernel::Cluster ? gdn::launch_prefill_cl(p, s) : gdn::launch_prefill_tc(p, s);
     return e == cudaSuccess ? GDN_OK : cuda_fail(e);
 }
 

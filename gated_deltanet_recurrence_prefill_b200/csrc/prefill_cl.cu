@@ -1,0 +1,1141 @@
+// prefill_cl.cu -- chunked gated delta-rule prefill on the sm_100a tensor cores,
+// as a thread-block cluster per (sequence, value head): one consumer CTA runs
+// the state chain, one or two producer CTAs the state-independent algebra.
+//
+// The arithmetic is the chunked WY / UT form of the recurrence (Qwen3.8-27B
+// architecture page, 2kiu.com, section 2.2, with the decay alpha on the erased
+// state), chunks of C = 64 tokens, G the running sum of log2(alpha) in the
+// chunk, gamma = 2^G, kappa = 2^{G_C - G}, S the state at the chunk start:
+//     A_ij = beta_i 2^{G_i - G_j} k_i.k_j  (j < i)      T = (I + A)^{-1}
+//     P_ij = 2^{G_i - G_j} q_i.k_j         (j <= i)     R = P T
+//     W  = T diag(beta gamma) K       U' = T diag(beta) V
+//     Qh = diag(gamma) Q - P W        O' = R diag(beta) V
+//     [U; o / scale] = [U'; O'] + [-W; Qh] S^T
+//     S <- gamma_C S + K^T diag(kappa) U
+// Everything up to [-W; Qh] and [T beta; R beta] is independent of the state.
+//
+// Producers (cluster ranks 1..P, P = 1 or 2).  Producer p takes chunks p,
+// p + P, ...; inside it two groups of 8 warps take alternate chunks.  A group
+// computes the gates, D0 = [K; Q] K^T (tcgen05), A and P, T by blocked forward
+// substitution (16x16 diagonal blocks on CUDA cores, off-diagonal blocks with
+// tf32 mma.sync), R = P T (tcgen05), the scaled bf16 copies [R bg; T bg] and
+// [T b; R b], X1 = [R bg; T bg] K (tcgen05) and from it -W and Qh.  It stages
+// the chunk's outgoing bytes where nothing else needs them any more: -W and Qh
+// over the K and Q rows of the chunk's [K; Q] stage, [T b; R b] with kappa and
+// gamma_C over the A scratch.  A publisher warp per group bulk-stores them to
+// the chunk's slot of a ring in global memory (kRing slots per (sequence,
+// value head), normally resident in L2), hands the staging back as soon as the
+// store has read it, and tells the consumer once the bytes are in place.
+// Warp 16 loads [K; Q] and the gate inputs by TMA into three stages.
+//
+// Consumer (rank 0).  A loader thread bulk-loads each chunk from the ring into
+// one of two receive slots and hands ring slots back to the producers.  d_v is
+// split in two halves of 64 that evolve independently (the rows of S do not mix
+// once T is known); each half has its own MMA issuer thread (warps 1 and 3) and
+// four epilogue warps, so one half's products overlap the other's epilogues:
+//   D  = [T b; R b] V_half                 M128 N64 K64   -> [U'; O']
+//   D += [-W; Qh] S_half^T                 M128 N64 K128  -> [U; o / scale]
+//   S~_half += K^T (kappa U / Gamma)        M128 N64 K64   (accumulates in TMEM)
+// The float32 state lives in TMEM as S~ with S = Gamma S~ (the decay gamma_C of
+// each chunk is folded into the running scalar Gamma and the update is added as
+// kappa U / Gamma); S~ is rescaled in place only when Gamma would fall below
+// 2^-80.  A bf16 copy of S is the operand of the next chunk.  o is staged in
+// shared memory and written by TMA (plain stores for a sequence's ragged last
+// chunk).  Warp 0 loads V and K by TMA.
+//
+// Every wait on an mbarrier is bounded; on expiry a CTA records an error in the
+// workspace, raises the abort flag of every CTA of its cluster, stops waiting and
+// drains its own tensor-core work and copies.  Producer group warps never leave
+// their loop early (their named barriers must always complete): after an abort
+// their waits simply fall through.
+#include <cuda.h>
+
+#include <stdlib.h>
+
+#include <atomic>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_util.cuh"
+#include "tile_util.cuh"
+
+namespace gdn {
+
+namespace {
+
+using namespace tc;
+using namespace tile;
+
+constexpr int kD = 128;
+constexpr int kC = 64;
+constexpr int kMaxProducers = 2;
+constexpr int kWarps = 19;
+constexpr int kThreads = kWarps * 32;
+constexpr int kGroupThreads = 256;
+constexpr int kLdF = 68;                       // fp32 solve scratch row stride
+
+struct GateBuf {
+    float beta[64];
+    float gamma[64];
+    float kappa[64];
+    float G[64];
+    float igamma[64];      // 2^{-G}; meaningful when `fast`
+    float gC;
+    int fast;              // G_C >= -kFastDecayLog2: 2^{G_i - G_j} = gamma_i * igamma_j
+    float pad[2];
+};
+static_assert(sizeof(GateBuf) == (5 * 64 + 4) * 4, "gate buffer layout");
+
+// ---- producer shared memory (byte offsets from a 1024-aligned base) ----------
+constexpr uint32_t KQ_STAGE = 2 * KQ_PANEL;    // [K; Q], d = 0..63 | 64..127
+constexpr int kKqStages = 3;
+constexpr uint32_t P_KQ = 0;
+constexpr uint32_t AB_STAGE = 2048;            // a, b: 64 rows x 4 f32 each
+constexpr uint32_t P_AB = P_KQ + kKqStages * KQ_STAGE;
+constexpr uint32_t P_GROUP = P_AB + kKqStages * AB_STAGE;
+constexpr uint32_t G_PT = 0;                               // P | T, later [R bg; T bg]
+constexpr uint32_t G_AF = G_PT + 16384;                    // A: 64 x 68 f32
+constexpr uint32_t G_TF = G_AF + 64 * kLdF * 4;            // T: 64 x 68 f32
+constexpr uint32_t G_XF = G_TF + 64 * kLdF * 4;            // mma.sync scratch 32 x 36
+constexpr uint32_t G_GATES = G_XF + 32 * 36 * 4;           // 2 gate buffers
+constexpr uint32_t G_END = G_GATES + 2 * sizeof(GateBuf);
+constexpr uint32_t GROUP_BYTES = (G_END + 1023) & ~1023u;
+constexpr uint32_t P_END = P_GROUP + 2 * GROUP_BYTES;
+static_assert(P_GROUP % 1024 == 0 && GROUP_BYTES % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+
+// ---- consumer shared memory ----------------------------------------------------
+// receive slot: [-W; Qh] (2 panels of 128 rows x 64 d), [T b; R b] (128 x 64),
+// kappa[64] and gamma_C -- the producer's staged bytes, copied verbatim
+constexpr uint32_t SL_QW = 0;
+constexpr uint32_t SL_RT2 = 2 * KQ_PANEL;
+constexpr uint32_t SL_GATES = SL_RT2 + 16384;
+constexpr uint32_t SLOT_BYTES = (SL_GATES + 512 + 1023) & ~1023u;
+constexpr uint32_t C_RECV = 0;                              // 2 slots
+constexpr uint32_t C_V = C_RECV + 2 * SLOT_BYTES;           // V: 2 panels of 64 x 64 bf16
+constexpr uint32_t C_K = C_V + 16384;                       // K: 2 panels of 64 x 64 bf16
+constexpr uint32_t C_ST = C_K + 16384;                      // S^T bf16: 2 halves of 128 x 64
+constexpr uint32_t C_UK = C_ST + 32768;                     // kappa U / Gamma: 2 halves of 64 x 64
+constexpr uint32_t C_OST = C_UK + 16384;                    // o staging: 2 halves x 2 boxes of 64 x 32 f32
+constexpr uint32_t C_END = C_OST + 32768;
+// what one chunk sends: the [-W; Qh] tile (staged in place of [K; Q]) and the
+// [T b; R b] tile with the gates (staged in the A scratch)
+constexpr uint32_t SEND_QW = 2 * KQ_PANEL;
+constexpr uint32_t SEND_RT = 16384 + 512;
+static_assert(SL_GATES == SL_RT2 + 16384 && SEND_RT <= 64 * kLdF * 4, "staging layout");
+// The chunks travel through a ring of kRing slots per (sequence, value head) in
+// the workspace (global memory, normally resident in L2): the producer's bulk
+// store frees its staging as soon as the bytes have been read, and the consumer
+// bulk-loads a chunk into its shared memory when a receive slot is free.
+constexpr int kRing = 4;
+constexpr uint32_t GSLOT_BYTES = SEND_QW + SEND_RT;
+static_assert(GSLOT_BYTES % 128 == 0 && kRing % 2 == 0, "ring layout");
+
+constexpr uint32_t OFF_MISC = (P_END > C_END ? P_END : C_END);
+constexpr uint32_t OFF_BARS = OFF_MISC + 64;
+
+enum {
+    // producer
+    PB_KQ_FULL = 0, PB_KQ_TAKEN = 2, PB_KQ_EMPTY = 4, PB_D0_FULL = 7, PB_R_FULL = 9,
+    PB_X1_FULL = 11, PB_DRAIN = 13, PB_STAGED = 15, PB_AF_FREE = 17, PB_GFREE = 19,
+    // consumer
+    CB_RECV_FULL = 23, CB_K_FULL = 25, CB_K_EMPTY, CB_V_FULL, CB_V_EMPTY, CB_D_EMPTY = 29,
+    CB_D_FULL = 31, CB_S_OK = 33, CB_S_FULL = 35, CB_ST_READY = 37, CB_DRAIN = 39, CB_GREADY = 41,
+    kNumBars = 45
+};
+constexpr uint32_t SMEM_BYTES = OFF_BARS + kNumBars * 8;
+constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;           // room to align the base
+static_assert(SMEM_ALLOC <= 232448, "shared memory budget of one CTA");
+
+// TMEM columns.  Producer group g: D0 (64), R (64), X1 (128) at 256 g.
+// Consumer: D[buffer][half] at 128 buffer + 64 half, S~[half] at 256 + 64 half.
+constexpr uint32_t PCOL_D0 = 0, PCOL_R = 64, PCOL_X1 = 128;
+constexpr uint32_t CCOL_S = 256;
+constexpr uint32_t TMEM_COLS = 512;
+
+constexpr uint32_t IDESC_D0 = idesc_bf16(128, 64, false, false);
+constexpr uint32_t IDESC_R = idesc_bf16(128, 64, false, true);
+constexpr uint32_t IDESC_X1 = idesc_bf16(128, 128, false, true);
+constexpr uint32_t IDESC_X2 = idesc_bf16(128, 64, false, true);
+constexpr uint32_t IDESC_D1 = idesc_bf16(128, 64, false, true);
+constexpr uint32_t IDESC_S = idesc_bf16(128, 64, true, true);
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;    // 2 s: far beyond any legitimate wait
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kFastDecayLog2 = 64.f;
+constexpr float kMinGamma = 8.271806125530277e-25f;          // 2^-80
+
+struct ClParams {
+    const float* a;
+    const float* b;
+    const float* A_log;
+    const float* dt_bias;
+    const int32_t* cu;
+    int64_t T;
+    int32_t Hqk, Hv;
+    float scale;
+    const float* s_in;
+    float* s_out;
+    float* o;
+    uint32_t* err;
+    uint8_t* ring;         // kRing slots of GSLOT_BYTES per (sequence, value head)
+    int gate_tma;          // a, b staged by TMA (needs Hv % 4 == 0), else read directly
+    int n_prod;            // producer CTAs per cluster (1 or 2); the cluster has n_prod + 1
+};
+
+struct Ctx {
+    uint8_t* sm;
+    uint32_t sbase;
+    uint32_t tmem;
+    volatile int* abort;
+    int warp, lane;
+    int h, g;              // value head, key head
+    uint8_t* ring;         // this cluster's ring slots
+    int64_t bos, eos;
+    int nch;
+    int64_t state_off;
+    uint32_t bar0;         // shared address of barrier 0
+    TC_DEVICE uint32_t bar(int i) const { return bar0 + 8u * (uint32_t)i; }
+};
+
+// S~ <- g S~ for this thread's TMEM lane over 64 columns
+__device__ __forceinline__ void rescale_state(uint32_t taddr, float g) {
+    for (int half = 0; half < 2; ++half) {
+        float s[32];
+        tmem_ld32(taddr + half * 32, s);
+        tmem_ld_wait();
+        for (int j = 0; j < 32; ++j) s[j] *= g;
+        tmem_st32(taddr + half * 32, s);
+    }
+    tmem_st_wait();
+}
+
+// ================================================================ consumer
+__device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
+                                         const CUtensorMap* tm_o, const ClParams& p) {
+    const int warp = x.warp, lane = x.lane;
+    const int nch = x.nch;
+    if (warp == 0) {
+        // ------------------------------------------------ TMA: V and K of each chunk
+        // One buffer each: V(c) is needed by the first product of chunk c and is
+        // free once both halves' first products of chunk c - 1 are done; K(c) by
+        // the state update at the end of chunk c.
+        if (lane == 0) {
+            prefetch_tmap(tm_k);
+            prefetch_tmap(tm_v);
+            int issued = 0;
+            for (int c = 0; c < nch; ++c) {
+                const int32_t y = (int32_t)(x.bos + (int64_t)c * kC);
+                if (c >= 1 && !mbar_wait(x.bar(CB_V_EMPTY), (c - 1) & 1, x.abort, kWaitLimitNs)) break;
+                mbar_arrive_expect_tx(x.bar(CB_V_FULL), 16384);
+                tma_load_2d(x.sbase + C_V, tm_v, x.h * kD, y, x.bar(CB_V_FULL));
+                tma_load_2d(x.sbase + C_V + 8192, tm_v, x.h * kD + 64, y, x.bar(CB_V_FULL));
+                if (c >= 1 && !mbar_wait(x.bar(CB_K_EMPTY), (c - 1) & 1, x.abort, kWaitLimitNs)) {
+                    issued = -(c + 1);           // V of chunk c is in flight, K is not
+                    break;
+                }
+                mbar_arrive_expect_tx(x.bar(CB_K_FULL), 16384);
+                tma_load_2d(x.sbase + C_K, tm_k, x.g * kD, y, x.bar(CB_K_FULL));
+                tma_load_2d(x.sbase + C_K + 8192, tm_k, x.g * kD + 64, y, x.bar(CB_K_FULL));
+                issued = c + 1;
+            }
+            // copies still in flight land before the CTA may exit
+            volatile int no_abort = 0;
+            const int nv = issued >= 0 ? issued : -issued, nk = issued >= 0 ? issued : -issued - 1;
+            if (nv >= 1) mbar_wait(x.bar(CB_V_FULL), (nv - 1) & 1, &no_abort, kWaitLimitNs);
+            if (nk >= 1) mbar_wait(x.bar(CB_K_FULL), (nk - 1) & 1, &no_abort, kWaitLimitNs);
+        }
+    } else if (warp == 1 || warp == 3) {
+        // ------------------------------------------------ MMA issuer of one d_v half
+        const int hh = warp >> 1;
+        if (lane == 0) {
+            for (int c = 0; c < nch; ++c) {
+                const int b = c & 1;
+                const uint32_t slot = x.sbase + C_RECV + b * SLOT_BYTES;
+                const uint32_t dcol = x.tmem + b * 128 + hh * 64;
+                if (!mbar_wait(x.bar(CB_RECV_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs)) break;
+                if (!mbar_wait(x.bar(CB_V_FULL), c & 1, x.abort, kWaitLimitNs)) break;
+                // D[b] was last read by the epilogues of chunk c - 2
+                if (c >= 2 && !mbar_wait(x.bar(CB_D_EMPTY + b), ((c >> 1) - 1) & 1, x.abort, kWaitLimitNs))
+                    break;
+                fence_async_smem();
+                tc_fence_after();
+                // [U'; O'] = [T b; R b] V_half
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(dcol, desc_kmajor_1panel(slot + SL_RT2, kk),
+                             desc_mnmajor(x.sbase + C_V + hh * 8192, kk, 8192), IDESC_X2, kk > 0);
+                mma_commit(x.bar(CB_V_EMPTY));
+                // += [-W; Qh] S_half^T  ->  [U; o / scale]
+                if (!mbar_wait(x.bar(CB_ST_READY + hh), c & 1, x.abort, kWaitLimitNs)) break;
+                tc_fence_after();
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(dcol, desc_kmajor_2panel(slot + SL_QW, kk),
+                             desc_mnmajor(x.sbase + C_ST + hh * 16384, kk, 16384), IDESC_D1, 1);
+                mma_commit(x.bar(CB_D_FULL + hh));
+                // S~_half += K^T (kappa U / Gamma)
+                if (!mbar_wait(x.bar(CB_S_OK + hh), c & 1, x.abort, kWaitLimitNs)) break;
+                if (!mbar_wait(x.bar(CB_K_FULL), c & 1, x.abort, kWaitLimitNs)) break;
+                tc_fence_after();
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(x.tmem + CCOL_S + hh * 64, desc_mnmajor(x.sbase + C_K, kk, 8192),
+                             desc_mnmajor(x.sbase + C_UK + hh * 8192, kk, 8192), IDESC_S, 1);
+                mma_commit(x.bar(CB_S_FULL + hh));
+                mma_commit(x.bar(CB_K_EMPTY));
+            }
+            volatile int no_abort = 0;
+            mma_commit(x.bar(CB_DRAIN + hh));
+            mbar_wait(x.bar(CB_DRAIN + hh), 0, &no_abort, kWaitLimitNs);
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------ loader: ring slot -> receive slot
+        // Chunk c sits in ring slot c % kRing; producer (c % kRing) % P owns that
+        // slot's "free" barrier.  A slot is handed back once its chunk has been
+        // loaded (checked one chunk later, so that loads overlap).
+        if (lane == 0) {
+            auto ring_free = [&](int c) {
+                const int rs = c % kRing;
+                mbar_arrive_cluster(map_to_rank(x.bar(PB_GFREE + rs), 1 + (uint32_t)(rs % p.n_prod)));
+            };
+            int loaded = 0;
+            for (int c = 0; c < nch; ++c) {
+                const int b = c & 1, rs = c % kRing;
+                if (c >= 2 && !mbar_wait(x.bar(CB_D_EMPTY + b), ((c >> 1) - 1) & 1, x.abort, kWaitLimitNs))
+                    break;
+                if (!mbar_wait_cluster(x.bar(CB_GREADY + rs), (c / kRing) & 1, x.abort, kWaitLimitNs)) break;
+                fence_async_global();
+                const uint32_t slot = x.sbase + C_RECV + b * SLOT_BYTES;
+                const uint8_t* g = x.ring + (size_t)rs * GSLOT_BYTES;
+                mbar_arrive_expect_tx(x.bar(CB_RECV_FULL + b), GSLOT_BYTES);
+                bulk_load(slot + SL_QW, g, SEND_QW, x.bar(CB_RECV_FULL + b));
+                bulk_load(slot + SL_RT2, g + SEND_QW, SEND_RT, x.bar(CB_RECV_FULL + b));
+                loaded = c + 1;
+                if (c >= 1) {
+                    if (!mbar_wait(x.bar(CB_RECV_FULL + ((c - 1) & 1)), ((c - 1) >> 1) & 1, x.abort, kWaitLimitNs))
+                        break;
+                    if (c - 1 + kRing < nch) ring_free(c - 1);
+                }
+            }
+            // loads still in flight land before the CTA may exit
+            volatile int no_abort = 0;
+            for (int c = loaded >= 2 ? loaded - 2 : 0; c < loaded; ++c)
+                mbar_wait(x.bar(CB_RECV_FULL + (c & 1)), (c >> 1) & 1, &no_abort, kWaitLimitNs);
+        }
+    } else if (warp >= 4 && warp < 12) {
+        // ------------------------------------------------ epilogues of one d_v half
+        const int q = warp & 3;                    // TMEM lane quadrant
+        const int hh = (warp - 4) >> 2;            // d_v half
+        const int r = q * 32 + lane;               // TMEM lane = row
+        const uint32_t tl = x.tmem + ((uint32_t)(q * 32) << 16);
+        const uint32_t scol = CCOL_S + hh * 64;
+        uint8_t* st_tile = x.sm + C_ST + hh * 16384;
+        uint8_t* uk_tile = x.sm + C_UK + hh * 8192;
+        // initial state: thread r holds d_k row r of S^T over this half's 64 v-columns
+        {
+            float s[32];
+            for (int half = 0; half < 2; ++half) {
+                for (int j = 0; j < 32; ++j) {
+                    const int vcol = hh * 64 + half * 32 + j;
+                    s[j] = p.s_in ? p.s_in[x.state_off + (int64_t)vcol * kD + r] : 0.f;
+                }
+                tmem_st32(tl + scol + half * 32, s);
+                for (int j = 0; j < 4; ++j) st_bf16x8(st_tile, r, half * 4 + j, s + 8 * j);
+            }
+            tmem_st_wait();
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(x.bar(CB_ST_READY + hh));
+        }
+        float Gam = 1.f;                           // S = Gam * S~ (same value in every thread)
+        for (int c = 0; c < nch; ++c) {
+            const int b = c & 1;
+            const float* kap = reinterpret_cast<const float*>(x.sm + C_RECV + b * SLOT_BYTES + SL_GATES);
+            const int64_t tok0 = x.bos + (int64_t)c * kC;
+            const uint32_t dcol = b * 128 + hh * 64;
+            mbar_wait(x.bar(CB_RECV_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs);
+            mbar_wait(x.bar(CB_D_FULL + hh), c & 1, x.abort, kWaitLimitNs);
+            tc_fence_after();
+            const float Gn = Gam * kap[64];        // scale of the state after this chunk
+            const bool resc = !(Gn >= kMinGamma);
+            const float inv = resc ? 1.f : 1.f / Gn;
+            if (q < 2) {
+                // rows 0-63 hold U_t: write kappa_t U_t / Gamma as the update operand
+                const int t = r;
+                const float sc = kap[t] * inv;
+                float u[2][32];
+                tmem_ld32x2(tl + dcol, tl + dcol + 32, u[0], u[1]);
+                for (int half = 0; half < 2; ++half) {
+                    for (int j = 0; j < 32; ++j) u[half][j] *= sc;
+                    for (int j = 0; j < 4; ++j) st_bf16x8(uk_tile, t, half * 4 + j, u[half] + 8 * j);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(x.bar(CB_D_EMPTY + b));
+                if (resc) rescale_state(tl + scol, Gn);
+                fence_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(x.bar(CB_S_OK + hh));
+            } else {
+                // rows 64-127 hold o_t / scale.  The state update does not touch
+                // these columns, so it may start before o is written.
+                if (resc) rescale_state(tl + scol, Gn);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(x.bar(CB_S_OK + hh));
+                const int t = r - 64;
+                float ov[2][32];
+                tmem_ld32x2(tl + dcol, tl + dcol + 32, ov[0], ov[1]);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(x.bar(CB_D_EMPTY + b));
+                if (tok0 + kC <= x.eos) {
+                    // whole chunk: stage the 64 x 64 tile (two 32-column boxes, 128-byte
+                    // swizzle) and store it with TMA.  The staging was last read by the
+                    // previous chunk's store.
+                    const bool elected = (q == 2 && lane == 0);
+                    if (elected) bulk_wait_read();
+                    named_bar_sync(5 + hh, 64);
+                    uint8_t* ost = x.sm + C_OST + hh * 16384;
+                    for (int bx = 0; bx < 2; ++bx) {
+                        for (int j = 0; j < 8; ++j) {
+                            float4 w;
+                            w.x = p.scale * ov[bx][4 * j];
+                            w.y = p.scale * ov[bx][4 * j + 1];
+                            w.z = p.scale * ov[bx][4 * j + 2];
+                            w.w = p.scale * ov[bx][4 * j + 3];
+                            *reinterpret_cast<float4*>(ost + bx * 8192 + sw128_off(t, j)) = w;
+                        }
+                    }
+                    fence_async_smem();
+                    named_bar_sync(5 + hh, 64);
+                    if (elected) {
+                        for (int bx = 0; bx < 2; ++bx)
+                            tma_store_2d(tm_o, x.h * kD + hh * 64 + bx * 32, (int32_t)tok0,
+                                         x.sbase + C_OST + hh * 16384 + bx * 8192);
+                        bulk_commit();
+                    }
+                } else if (tok0 + t < x.eos) {
+                    // the ragged end of a sequence: rows past its end belong to the next one
+                    float* orow = p.o + ((tok0 + t) * p.Hv + x.h) * kD + hh * 64;
+                    for (int bx = 0; bx < 2; ++bx)
+                        for (int j = 0; j < 32; j += 4) {
+                            float4 w;
+                            w.x = p.scale * ov[bx][j];
+                            w.y = p.scale * ov[bx][j + 1];
+                            w.z = p.scale * ov[bx][j + 2];
+                            w.w = p.scale * ov[bx][j + 3];
+                            *reinterpret_cast<float4*>(orow + bx * 32 + j) = w;
+                        }
+                }
+            }
+            Gam = resc ? 1.f : Gn;
+            // new state -> bf16 operand of the next chunk (and the final state)
+            mbar_wait(x.bar(CB_S_FULL + hh), c & 1, x.abort, kWaitLimitNs);
+            tc_fence_after();
+            const bool last = (c == nch - 1);
+            float sv[2][32];
+            tmem_ld32x2(tl + scol, tl + scol + 32, sv[0], sv[1]);
+            for (int half = 0; half < 2; ++half) {
+                float* s = sv[half];
+                for (int j = 0; j < 32; ++j) s[j] *= Gam;
+                if (!last) {
+                    for (int j = 0; j < 4; ++j) st_bf16x8(st_tile, r, half * 4 + j, s + 8 * j);
+                } else if (p.s_out) {
+                    for (int j = 0; j < 32; ++j)
+                        p.s_out[x.state_off + (int64_t)(hh * 64 + half * 32 + j) * kD + r] = s[j];
+                }
+            }
+            if (!last) {
+                fence_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(x.bar(CB_ST_READY + hh));
+            }
+        }
+        if (q == 2 && lane == 0) bulk_wait();      // this half's last o stores are complete
+    }
+}
+
+// ================================================================ producer
+__device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorMap* tm_q,
+                                         const CUtensorMap* tm_k, const CUtensorMap* tm_a,
+                                         const CUtensorMap* tm_b, const ClParams& p) {
+    const int warp = x.warp, lane = x.lane;
+    const int nch = x.nch;
+    const int h = x.h;
+    if (warp == 16) {
+        // ------------------------------------------------ TMA: [K; Q] and gate inputs
+        if (lane == 0) {
+            prefetch_tmap(tm_q);
+            prefetch_tmap(tm_k);
+            if (p.gate_tma) { prefetch_tmap(tm_a); prefetch_tmap(tm_b); }
+            // chunk i of this producer goes to stage i % 3 and to group i & 1.  The
+            // group's full barrier is armed for its next chunk only after the group
+            // has taken the previous one, so each barrier runs at most one phase
+            // ahead of its waiters.
+            int issued = 0;
+            for (int i = 0;; ++i) {
+                const int c = pidx + p.n_prod * i;
+                if (c >= nch) break;
+                const int s = i % kKqStages, grp = i & 1, jj = i >> 1;
+                if (i >= kKqStages &&
+                    !mbar_wait(x.bar(PB_KQ_EMPTY + s), (i / kKqStages - 1) & 1, x.abort, kWaitLimitNs))
+                    break;
+                if (jj >= 1 && !mbar_wait(x.bar(PB_KQ_TAKEN + grp), (jj - 1) & 1, x.abort, kWaitLimitNs))
+                    break;
+                const uint32_t kq = x.sbase + P_KQ + s * KQ_STAGE;
+                const int32_t y = (int32_t)(x.bos + (int64_t)c * kC);
+                const uint32_t fb = x.bar(PB_KQ_FULL + grp);
+                mbar_arrive_expect_tx(fb, KQ_STAGE + (p.gate_tma ? AB_STAGE : 0));
+                tma_load_2d(kq, tm_k, x.g * kD, y, fb);
+                tma_load_2d(kq + 8192, tm_q, x.g * kD, y, fb);
+                tma_load_2d(kq + KQ_PANEL, tm_k, x.g * kD + 64, y, fb);
+                tma_load_2d(kq + KQ_PANEL + 8192, tm_q, x.g * kD + 64, y, fb);
+                if (p.gate_tma) {
+                    // the 4-column group of a and b that holds column h
+                    const uint32_t ab = x.sbase + P_AB + s * AB_STAGE;
+                    tma_load_2d(ab, tm_a, h & ~3, y, fb);
+                    tma_load_2d(ab + 1024, tm_b, h & ~3, y, fb);
+                }
+                issued = i + 1;
+            }
+            // copies still in flight land before the CTA may exit: the last chunk
+            // armed on each group's barrier
+            volatile int no_abort = 0;
+            for (int i = issued >= 2 ? issued - 2 : 0; i < issued; ++i)
+                mbar_wait(x.bar(PB_KQ_FULL + (i & 1)), (i >> 1) & 1, &no_abort, kWaitLimitNs);
+        }
+        return;
+    }
+    if (warp == 17 || warp == 18) {
+        // ------------------------------------------------ publisher of one group
+        // Once the group has staged a chunk and its ring slot is free, two bulk
+        // stores write it to the ring; the staging (the [K; Q] stage and the
+        // group's A scratch) is reusable as soon as they have read it, and the
+        // consumer is told once the bytes are in global memory.
+        const int grp = warp - 17;
+        if (lane == 0) {
+            const uint32_t gready0 = map_to_rank(x.bar(CB_GREADY), 0);
+            const uint32_t stage_rt = x.sbase + P_GROUP + grp * GROUP_BYTES + G_AF;
+            for (int jj = 0;; ++jj) {
+                const int i = grp + 2 * jj;
+                const int c = pidx + p.n_prod * i;
+                if (c >= nch) break;
+                const int rs = c % kRing;
+                if (!mbar_wait(x.bar(PB_STAGED + grp), jj & 1, x.abort, kWaitLimitNs)) break;
+                if (c >= kRing &&
+                    !mbar_wait_cluster(x.bar(PB_GFREE + rs), (c / kRing - 1) & 1, x.abort, kWaitLimitNs))
+                    break;
+                fence_async_global();
+                uint8_t* g = x.ring + (size_t)rs * GSLOT_BYTES;
+                bulk_store(g, x.sbase + P_KQ + (i % kKqStages) * KQ_STAGE, SEND_QW);
+                bulk_store(g + SEND_QW, stage_rt, SEND_RT);
+                bulk_commit();
+                bulk_wait_read();
+                mbar_arrive(x.bar(PB_KQ_EMPTY + i % kKqStages));
+                mbar_arrive(x.bar(PB_AF_FREE + grp));
+                bulk_wait();
+                fence_async_global();
+                mbar_arrive_cluster(gready0 + 8u * (uint32_t)rs);
+            }
+        }
+        return;
+    }
+    if (warp >= 16) return;
+    // ---------------------------------------------------- precompute group
+    const int grp = warp >> 3;                 // 0 or 1
+    const int pw = warp & 7;                   // warp within the group
+    const int q = warp & 3;                    // TMEM lane quadrant
+    const int hh = pw >> 2;                    // column half
+    const int pt = pw * 32 + lane;
+    const int nb = 1 + grp;                    // group-wide named barrier
+    const int nb_gates = 3 + grp;              // the two gate warps
+    uint8_t* gbase = x.sm + P_GROUP + grp * GROUP_BYTES;
+    const uint32_t gsb = x.sbase + P_GROUP + grp * GROUP_BYTES;
+    float* Af = reinterpret_cast<float*>(gbase + G_AF);
+    float* Tf = reinterpret_cast<float*>(gbase + G_TF);
+    float* Xf = reinterpret_cast<float*>(gbase + G_XF);
+    GateBuf* gates = reinterpret_cast<GateBuf*>(gbase + G_GATES);
+    float* xchg = reinterpret_cast<float*>(x.sm + OFF_MISC + 16 + 8 * grp);
+    const uint32_t tg = x.tmem + 256u * grp;
+    const uint32_t tl = tg + ((uint32_t)(q * 32) << 16);
+    const bool issuer = (pw == 0 && lane == 0);
+    const float Al = p.A_log[h], dtb = p.dt_bias[h];
+    uint8_t* stage_rt = gbase + G_AF;          // [T b; R b] and the gates, staged for sending
+
+    int jj = 0;                                // chunks done by this group
+    for (int i = grp;; i += 2, ++jj) {
+        const int c = pidx + p.n_prod * i;
+        if (c >= nch) break;
+        const int s = i % kKqStages;
+        GateBuf& gb = gates[jj & 1];
+        const int64_t tok0 = x.bos + (int64_t)c * kC;
+        const uint32_t kqo = P_KQ + s * KQ_STAGE;
+        const uint32_t kq = x.sbase + kqo;
+        // every warp of the group has seen chunk i land before the TMA warp may
+        // arm this group's barrier again
+        mbar_wait(x.bar(PB_KQ_FULL + grp), jj & 1, x.abort, kWaitLimitNs);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(x.bar(PB_KQ_TAKEN + grp));
+        if (issuer) {
+            // D0 = [K; Q] K^T
+            tc_fence_after();
+            for (int kk = 0; kk < 8; ++kk)
+                mma_bf16(tg + PCOL_D0, desc_kmajor_2panel(kq, kk), desc_kmajor_2panel(kq, kk), IDESC_D0,
+                         kk > 0);
+            mma_commit(x.bar(PB_D0_FULL + grp));
+        }
+        __syncwarp();
+        // ---- gates (warps 6, 7 of the group): G = running sum of log2(alpha);
+        //      beta; gamma = 2^G; kappa = 2^{G_C - G}
+        if (pw >= 6) {
+            const int t = pt - 192;
+            const int64_t tok = tok0 + t;
+            const float* abt = reinterpret_cast<const float*>(x.sm + P_AB + s * AB_STAGE);
+            float lg = 0.f, be = 0.f;
+            if (tok < x.eos) {
+                const float av = p.gate_tma ? abt[t * 4 + (h & 3)] : p.a[tok * p.Hv + h];
+                const float bv = p.gate_tma ? abt[256 + t * 4 + (h & 3)] : p.b[tok * p.Hv + h];
+                lg = kLog2e * log_alpha_f32(av, Al, dtb);
+                be = sigmoid_f32(bv);
+            }
+            float run = lg;
+            for (int m = 1; m < 32; m <<= 1) {
+                const float o = __shfl_up_sync(0xffffffffu, run, m);
+                if (lane >= m) run += o;
+            }
+            if (pw == 6 && lane == 31) xchg[0] = run;
+            named_bar_sync(nb_gates, 64);
+            if (pw == 7) run += xchg[0];
+            gb.G[t] = run;
+            gb.beta[t] = be;
+            gb.gamma[t] = exp2f(run);
+            if (t == 63) {
+                xchg[1] = run;
+                gb.gC = exp2f(run);
+                gb.fast = run >= -kFastDecayLog2 ? 1 : 0;
+            }
+            named_bar_sync(nb_gates, 64);
+            gb.kappa[t] = exp2f(xchg[1] - run);
+            gb.igamma[t] = xchg[1] >= -kFastDecayLog2 ? exp2f(-run) : 0.f;
+        }
+        named_bar_sync(nb, kGroupThreads);
+        // ---- D0 rows -> A (f32 scratch) and P (bf16 operand); each warp 32 columns.
+        //      The A scratch last held the previous chunk's staged bytes.
+        if (jj >= 1) mbar_wait(x.bar(PB_AF_FREE + grp), (jj - 1) & 1, x.abort, kWaitLimitNs);
+        mbar_wait(x.bar(PB_D0_FULL + grp), jj & 1, x.abort, kWaitLimitNs);
+        tc_fence_after();
+        {
+            const bool fast = gb.fast != 0;
+            float dv[32];
+            tmem_ld32(tl + PCOL_D0 + hh * 32, dv);
+            tmem_ld_wait();
+            const int i_ = (q & 1) * 32 + lane;      // row within KK^T (q<2) or QK^T (q>=2)
+            const float Gi = gb.G[i_];
+            if (q < 2) {
+                // A_ij = beta_i 2^{G_i - G_j} (k_i . k_j), j < i
+                const float ci = fast ? gb.beta[i_] * gb.gamma[i_] : gb.beta[i_];
+                float* arow = Af + i_ * kLdF + hh * 32;
+#pragma unroll
+                for (int j4 = 0; j4 < 32; j4 += 4) {
+                    const int j = hh * 32 + j4;
+                    float4 w;
+                    if (fast) {
+                        const float4 ig = *reinterpret_cast<const float4*>(&gb.igamma[j]);
+                        w.x = (j + 0 < i_) ? ci * dv[j4 + 0] * ig.x : 0.f;
+                        w.y = (j + 1 < i_) ? ci * dv[j4 + 1] * ig.y : 0.f;
+                        w.z = (j + 2 < i_) ? ci * dv[j4 + 2] * ig.z : 0.f;
+                        w.w = (j + 3 < i_) ? ci * dv[j4 + 3] * ig.w : 0.f;
+                    } else {
+                        const float4 gj = *reinterpret_cast<const float4*>(&gb.G[j]);
+                        w.x = (j + 0 < i_) ? ci * dv[j4 + 0] * exp2f(Gi - gj.x) : 0.f;
+                        w.y = (j + 1 < i_) ? ci * dv[j4 + 1] * exp2f(Gi - gj.y) : 0.f;
+                        w.z = (j + 2 < i_) ? ci * dv[j4 + 2] * exp2f(Gi - gj.z) : 0.f;
+                        w.w = (j + 3 < i_) ? ci * dv[j4 + 3] * exp2f(Gi - gj.w) : 0.f;
+                    }
+                    *reinterpret_cast<float4*>(arow + j4) = w;
+                }
+            } else {
+                // P_ij = 2^{G_i - G_j} (q_i . k_j), j <= i
+                const float ci = fast ? gb.gamma[i_] : 1.f;
+#pragma unroll
+                for (int j4 = 0; j4 < 32; j4 += 4) {
+                    const int j = hh * 32 + j4;
+                    if (fast) {
+                        const float4 ig = *reinterpret_cast<const float4*>(&gb.igamma[j]);
+                        dv[j4 + 0] = (j + 0 <= i_) ? ci * dv[j4 + 0] * ig.x : 0.f;
+                        dv[j4 + 1] = (j + 1 <= i_) ? ci * dv[j4 + 1] * ig.y : 0.f;
+                        dv[j4 + 2] = (j + 2 <= i_) ? ci * dv[j4 + 2] * ig.z : 0.f;
+                        dv[j4 + 3] = (j + 3 <= i_) ? ci * dv[j4 + 3] * ig.w : 0.f;
+                    } else {
+                        const float4 gj = *reinterpret_cast<const float4*>(&gb.G[j]);
+                        dv[j4 + 0] = (j + 0 <= i_) ? dv[j4 + 0] * exp2f(Gi - gj.x) : 0.f;
+                        dv[j4 + 1] = (j + 1 <= i_) ? dv[j4 + 1] * exp2f(Gi - gj.y) : 0.f;
+                        dv[j4 + 2] = (j + 2 <= i_) ? dv[j4 + 2] * exp2f(Gi - gj.z) : 0.f;
+                        dv[j4 + 3] = (j + 3 <= i_) ? dv[j4 + 3] * exp2f(Gi - gj.w) : 0.f;
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) st_bf16x8(gbase + G_PT, i_, hh * 4 + j, dv + 8 * j);
+            }
+        }
+        tc_fence_before();
+        named_bar_sync(nb, kGroupThreads);
+        // ---- T = (I + A)^{-1}: 16x16 diagonal blocks by forward substitution
+        if (pw < 4) {
+            const int blk = pw;
+            const int col = lane & 15;
+            const float* Ab = Af + (16 * blk) * kLdF + 16 * blk;
+            float xv[16];
+#pragma unroll
+            for (int ii = 0; ii < 16; ++ii) {
+                float arow[16];
+#pragma unroll
+                for (int m4 = 0; m4 < ii; m4 += 4) {
+                    const float4 a4 = *reinterpret_cast<const float4*>(Ab + ii * kLdF + m4);
+                    arow[m4] = a4.x; arow[m4 + 1] = a4.y; arow[m4 + 2] = a4.z; arow[m4 + 3] = a4.w;
+                }
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int m = 0; m < ii; ++m) acc[m & 3] = fmaf(arow[m], xv[m], acc[m & 3]);
+                xv[ii] = ((ii == col) ? 1.f : 0.f) - ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+            }
+            if (lane < 16) {
+#pragma unroll
+                for (int ii = 0; ii < 16; ++ii) Tf[(16 * blk + ii) * kLdF + 16 * blk + col] = xv[ii];
+            }
+        }
+        named_bar_sync(nb, kGroupThreads);
+        // ---- 32x32 blocks: T10 = -T11 A10 T00 (warp: block pair pw>>1, 8 columns)
+        if (pw < 4) {
+            const int pr = pw >> 1, nh = pw & 1;
+            const int R0 = 32 * pr, R1 = R0 + 16;
+            float* Xw = Xf + pw * 128;                 // 16 x 8
+            float cfr[4];
+            mma_tile(cfr, Af, kLdF, R1, R0, Tf, kLdF, R0, R0 + 8 * nh, 0, 2, lane);
+            frag_c_store(Xw, 8, 0, 0, cfr, 1.f, lane);
+            __syncwarp();
+            mma_tile(cfr, Tf, kLdF, R1, R1, Xw, 8, 0, 0, 0, 2, lane);
+            frag_c_store(Tf, kLdF, R1, R0 + 8 * nh, cfr, -1.f, lane);
+        }
+        named_bar_sync(nb, kGroupThreads);
+        // ---- 64x64: T[32:64, 0:32] = -T[32:64, 32:64] A[32:64, 0:32] T[0:32, 0:32]
+        {
+            const int mt = pw >> 2, nt = pw & 3;
+            float cfr[4];
+            mma_tile(cfr, Af, kLdF, 32 + 16 * mt, 0, Tf, kLdF, 0, 8 * nt, nt, 4, lane);
+            frag_c_store(Xf, 36, 16 * mt, 8 * nt, cfr, 1.f, lane);
+            named_bar_sync(nb, kGroupThreads);
+            mma_tile(cfr, Tf, kLdF, 32 + 16 * mt, 32, Xf, 36, 0, 8 * nt, 0, 2 * mt + 2, lane);
+            frag_c_store(Tf, kLdF, 32 + 16 * mt, 8 * nt, cfr, -1.f, lane);
+        }
+        named_bar_sync(nb, kGroupThreads);
+        // ---- T (bf16) as the B operand of R = P T
+        for (int u = pt; u < 64 * 8; u += kGroupThreads) {
+            const int row = u >> 3, chunk = u & 7;
+            const float4 t0 = *reinterpret_cast<const float4*>(Tf + row * kLdF + chunk * 8);
+            const float4 t1 = *reinterpret_cast<const float4*>(Tf + row * kLdF + chunk * 8 + 4);
+            const float xv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+            st_bf16x8(gbase + G_PT + 8192, row, chunk, xv);
+        }
+        fence_async_smem();
+        named_bar_sync(nb, kGroupThreads);
+        if (issuer) {
+            // R = [P; T] T (rows 0-63 used)
+            tc_fence_after();
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(tg + PCOL_R, desc_kmajor_1panel(gsb + G_PT, kk),
+                         desc_mnmajor(gsb + G_PT + 8192, kk, 8192), IDESC_R, kk > 0);
+            mma_commit(x.bar(PB_R_FULL + grp));
+        }
+        __syncwarp();
+        // ---- [R bg; T bg] (over P | T once R is done) and, staged for sending,
+        //      [T b; R b] with the gates (over A, which the solve no longer needs)
+        mbar_wait(x.bar(PB_R_FULL + grp), jj & 1, x.abort, kWaitLimitNs);
+        tc_fence_after();
+        {
+            const int i_ = (q & 1) * 32 + lane;
+            float v[32];
+            if (q < 2) {
+                tmem_ld32(tl + PCOL_R + hh * 32, v);
+                tmem_ld_wait();
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    const float4 t4 = *reinterpret_cast<const float4*>(Tf + i_ * kLdF + hh * 32 + j);
+                    v[j] = t4.x; v[j + 1] = t4.y; v[j + 2] = t4.z; v[j + 3] = t4.w;
+                }
+            }
+            const int row = (q < 2 ? 0 : 64) + i_;     // [R bg; T bg]: R in rows 0-63
+            const int row2 = (q < 2 ? 64 : 0) + i_;    // [T b; R b]: T in rows 0-63
+#pragma unroll
+            for (int j8 = 0; j8 < 4; ++j8) {
+                const int j0 = hh * 32 + j8 * 8;
+                const float4 b0 = *reinterpret_cast<const float4*>(&gb.beta[j0]);
+                const float4 b1 = *reinterpret_cast<const float4*>(&gb.beta[j0 + 4]);
+                const float4 g0 = *reinterpret_cast<const float4*>(&gb.gamma[j0]);
+                const float4 g1 = *reinterpret_cast<const float4*>(&gb.gamma[j0 + 4]);
+                const float bj[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+                const float gj[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+                float wb[8], wg[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    wb[e] = v[j8 * 8 + e] * bj[e];
+                    wg[e] = wb[e] * gj[e];
+                }
+                st_bf16x8(gbase + G_PT, row, hh * 4 + j8, wg);
+                st_bf16x8(stage_rt, row2, hh * 4 + j8, wb);
+            }
+            if (q < 2 && hh == 0) {
+                float* sg = reinterpret_cast<float*>(stage_rt + (SL_GATES - SL_RT2));
+                sg[i_] = gb.kappa[i_];
+                if (i_ == 63) sg[64] = gb.gC;
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        named_bar_sync(nb, kGroupThreads);
+        if (issuer) {
+            // X1 = [R bg; T bg] K  ->  rows 0-63: P W, rows 64-127: W
+            tc_fence_after();
+            for (int kk = 0; kk < 4; ++kk)
+                mma_bf16(tg + PCOL_X1, desc_kmajor_1panel(gsb + G_PT, kk), desc_mnmajor(kq, kk, KQ_PANEL),
+                         IDESC_X1, kk > 0);
+            mma_commit(x.bar(PB_X1_FULL + grp));
+        }
+        __syncwarp();
+        mbar_wait(x.bar(PB_X1_FULL + grp), jj & 1, x.abort, kWaitLimitNs);
+        tc_fence_after();
+        // ---- -W over the K rows and Qh = diag(gamma) Q - P W over the Q rows of the
+        //      [K; Q] stage (each thread rewrites the Q chunks it has just read)
+        {
+            const int i_ = (q & 1) * 32 + lane;
+            const float ga = gb.gamma[i_];
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                const int dcol = hh * 64 + part * 32;          // 32 of the 128 d columns
+                const int panel = dcol >> 6, ch0 = (dcol & 63) >> 3;
+                float xv[32];
+                tmem_ld32(tl + PCOL_X1 + dcol, xv);
+                tmem_ld_wait();
+                if (q < 2) {
+                    const uint8_t* qrow = x.sm + kqo + panel * KQ_PANEL + 8192;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        float qv[8];
+                        ld_bf16x8(qrow, i_, ch0 + j, qv);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) xv[8 * j + e] = ga * qv[e] - xv[8 * j + e];
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) xv[e] = -xv[e];
+                }
+                uint8_t* dst = x.sm + kqo + panel * KQ_PANEL + (q < 2 ? 8192 : 0);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) st_bf16x8(dst, i_, ch0 + j, xv + 8 * j);
+            }
+        }
+        // staged: the publisher may send the chunk
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(x.bar(PB_STAGED + grp));
+    }
+    if (issuer) {
+        volatile int no_abort = 0;
+        mma_commit(x.bar(PB_DRAIN + grp));
+        mbar_wait(x.bar(PB_DRAIN + grp), 0, &no_abort, kWaitLimitNs);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
+                  const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_o,
+                  const ClParams p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // align to 1024 bytes by pointer arithmetic on the shared array, so that
+    // every access below stays in the shared state space; the offset is the same
+    // in every CTA of the cluster, so local offsets name the peers' buffers too
+    uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    Ctx x;
+    x.sm = sm;
+    x.sbase = smem_u32(sm);
+    x.bar0 = x.sbase + OFF_BARS;
+    x.abort = reinterpret_cast<volatile int*>(sm + OFF_MISC);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC + 4);
+    x.warp = threadIdx.x >> 5;
+    x.lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int cl = blockIdx.x / (p.n_prod + 1);
+    x.h = cl % p.Hv;
+    const int n = cl / p.Hv;
+    x.g = x.h / (p.Hv / p.Hqk);
+    x.bos = p.cu ? p.cu[n] : 0;
+    x.eos = p.cu ? p.cu[n + 1] : p.T;
+    x.nch = (int)((x.eos - x.bos + kC - 1) / kC);
+    x.state_off = ((int64_t)n * p.Hv + x.h) * kD * kD;
+    x.ring = p.ring + (size_t)cl * kRing * GSLOT_BYTES;
+
+    if (x.nch == 0) {
+        // empty sequence (the same in every CTA of the cluster): final state = initial state
+        if (rank == 0 && p.s_out && p.s_out != p.s_in) {
+            for (int i = threadIdx.x; i < kD * kD; i += kThreads)
+                p.s_out[x.state_off + i] = p.s_in ? p.s_in[x.state_off + i] : 0.f;
+        }
+        return;
+    }
+
+    if (threadIdx.x == 0) {
+        *x.abort = 0;
+        if (rank == 0) {
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(x.bar(CB_RECV_FULL + b), 1);
+                mbar_init(x.bar(CB_D_EMPTY + b), 8);
+            }
+            mbar_init(x.bar(CB_K_FULL), 1);
+            mbar_init(x.bar(CB_K_EMPTY), 2);
+            mbar_init(x.bar(CB_V_FULL), 1);
+            mbar_init(x.bar(CB_V_EMPTY), 2);
+            for (int hh = 0; hh < 2; ++hh) {
+                mbar_init(x.bar(CB_D_FULL + hh), 1);
+                mbar_init(x.bar(CB_S_OK + hh), 4);
+                mbar_init(x.bar(CB_S_FULL + hh), 1);
+                mbar_init(x.bar(CB_ST_READY + hh), 4);
+                mbar_init(x.bar(CB_DRAIN + hh), 1);
+            }
+            for (int r = 0; r < kRing; ++r) mbar_init(x.bar(CB_GREADY + r), 1);
+        } else {
+            for (int s = 0; s < kKqStages; ++s) mbar_init(x.bar(PB_KQ_EMPTY + s), 1);
+            for (int r = 0; r < kRing; ++r) mbar_init(x.bar(PB_GFREE + r), 1);
+            for (int grp = 0; grp < 2; ++grp) {
+                mbar_init(x.bar(PB_KQ_FULL + grp), 1);
+                mbar_init(x.bar(PB_KQ_TAKEN + grp), 8);
+                mbar_init(x.bar(PB_D0_FULL + grp), 1);
+                mbar_init(x.bar(PB_R_FULL + grp), 1);
+                mbar_init(x.bar(PB_X1_FULL + grp), 1);
+                mbar_init(x.bar(PB_DRAIN + grp), 1);
+                mbar_init(x.bar(PB_STAGED + grp), 8);
+                mbar_init(x.bar(PB_AF_FREE + grp), 1);
+            }
+        }
+        fence_mbar_init();
+    }
+    if (x.warp == 2) tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    if (rank != 0) {
+        // zero the strictly upper blocks of both groups' T scratch (never written again)
+        for (int gi = 0; gi < 2; ++gi) {
+            float* Tf = reinterpret_cast<float*>(sm + P_GROUP + gi * GROUP_BYTES + G_TF);
+            for (int i = threadIdx.x; i < 64 * kLdF; i += kThreads) Tf[i] = 0.f;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();            // every CTA's barriers exist before anyone arrives remotely
+    tc_fence_after();
+    x.tmem = *tmem_slot;
+
+    if (rank == 0)
+        consumer(x, &tm_k, &tm_v, &tm_o, p);
+    else
+        producer(x, (int)rank - 1, &tm_q, &tm_k, &tm_a, &tm_b, p);
+
+    // ---------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0 && *x.abort) {
+        atomicOr(p.err, 1u);
+        // let the other CTAs of the cluster stop waiting for this one
+        for (uint32_t r = 0; r <= (uint32_t)p.n_prod; ++r)
+            if (r != rank) st_cluster_u32(map_to_rank(smem_u32(sm + OFF_MISC), r), 1u);
+    }
+    cluster_sync();            // no CTA leaves while a peer may still touch its shared memory
+    if (x.warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(x.tmem, TMEM_COLS);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult qres;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) ==
+                cudaSuccess &&
+            qres == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// 2D bf16 tensor [rows, cols] (cols contiguous), 64 x 64 boxes, 128-byte swizzle
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {64, 64};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2D float tensor [rows, cols] (cols contiguous), 32-column x 64-row boxes,
+// 128-byte swizzle (the o tiles)
+bool make_map_o(CUtensorMap* m, float* base, int64_t rows, int64_t cols) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+    cuuint32_t box[2] = {32, 64};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2D float tensor [rows, cols], 4-column x 64-row boxes, no swizzle
+bool make_map_gates(CUtensorMap* m, const float* base, int64_t rows, int64_t cols) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+    cuuint32_t box[2] = {4, 64};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t setup_kernel() {
+    return cudaFuncSetAttribute(prefill_cl_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)SMEM_ALLOC);
+}
+
+// clusters of `size` CTAs that can be resident at once on the current device
+// (0 when none fit); cached per device
+std::atomic<int> g_max_clusters[64][2];     // [device][size - 2], stored + 1 (0 = unknown)
+
+int max_active_clusters(int size) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    int v = g_max_clusters[dev][size - 2].load(std::memory_order_relaxed);
+    if (v > 0) return v - 1;
+    int clusters = 0;
+    if (setup_kernel() == cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(size);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = SMEM_ALLOC;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = size;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&clusters, prefill_cl_kernel, &cfg) != cudaSuccess)
+            clusters = 0;
+    }
+    cudaGetLastError();    // a refused query leaves no sticky error behind
+    g_max_clusters[dev][size - 2].store(clusters + 1, std::memory_order_relaxed);
+    return clusters;
+}
+
+// Producer CTAs per cluster for `units` (sequence, value head) pairs.  Two
+// producers keep the consumer's state chain busy (a chunk takes about half as
+// long as with one), so they win unless clusters of three need more than
+// twice as many waves of resident clusters as clusters of two.
+// GDN_PREFILL_PRODUCERS=1 or =2 in the environment forces the choice.
+int pick_producers(int64_t units) {
+    const char* env = getenv("GDN_PREFILL_PRODUCERS");
+    if (env && (env[0] == '1' || env[0] == '2') && env[1] == 0) {
+        const int want = env[0] - '0';
+        return max_active_clusters(want + 1) > 0 ? want : 0;
+    }
+    const int m3 = max_active_clusters(3);
+    const int m2 = max_active_clusters(2);
+    if (m3 <= 0) return m2 > 0 ? 1 : 0;
+    if (m2 <= 0) return 2;
+    const int64_t waves3 = (units + m3 - 1) / m3, waves2 = (units + m2 - 1) / m2;
+    return waves3 <= 2 * waves2 ? 2 : 1;
+}
+
+}  // namespace
+
+size_t prefill_cl_smem_bytes() { return SMEM_ALLOC; }
+
+size_t prefill_cl_workspace_bytes(int32_t n_seq, int32_t Hv) {
+    const size_t units = (size_t)(n_seq > 0 ? n_seq : 1) * (size_t)(Hv > 0 ? Hv : 1);
+    return kWsHeaderBytes + ((units * kRing * GSLOT_BYTES + 255) / 256) * 256;
+}
+
+bool prefill_cl_available() { return max_active_clusters(2) > 0 || max_active_clusters(3) > 0; }
+
+int prefill_cl_max_active_clusters(int size) {
+    if (size != 2 && size != 3) return -1;
+    return max_active_clusters(size);
+}
+
+cudaError_t launch_prefill_cl(const PrefillArgs& a, cudaStream_t stream) {
+    if (a.T == 0) {
+        // every sequence is empty: final state = initial state
+        if (a.final_state && a.final_state != a.initial_state) {
+            const size_t bytes = (size_t)a.n_seq * a.Hv * kD * kD * sizeof(float);
+            return a.initial_state
+                       ? cudaMemcpyAsync(a.final_state, a.initial_state, bytes,
+                                         cudaMemcpyDeviceToDevice, stream)
+                       : cudaMemsetAsync(a.final_state, 0, bytes, stream);
+        }
+        return cudaSuccess;
+    }
+    CUtensorMap mq, mk, mv, ma, mb, mo;
+    if (!make_map(&mq, a.q, a.T, (int64_t)a.Hqk * kD) || !make_map(&mk, a.k, a.T, (int64_t)a.Hqk * kD) ||
+        !make_map(&mv, a.v, a.T, (int64_t)a.Hv * kD) || !make_map_o(&mo, a.o, a.T, (int64_t)a.Hv * kD))
+        return cudaErrorInvalidValue;
+    // a and b rows must be a multiple of 16 bytes for TMA; otherwise they are read directly
+    const int gate_tma = (a.Hv % 4 == 0) ? 1 : 0;
+    if (gate_tma) {
+        if (!make_map_gates(&ma, a.a, a.T, a.Hv) || !make_map_gates(&mb, a.b, a.T, a.Hv))
+            return cudaErrorInvalidValue;
+    } else {
+        ma = mq;
+        mb = mq;       // unused
+    }
+    cudaError_t e = setup_kernel();
+    if (e != cudaSuccess) return e;
+    const int n_prod = pick_producers((int64_t)a.n_seq * a.Hv);
+    if (n_prod == 0) return cudaErrorNotSupported;
+    const int csize = n_prod + 1;
+    ClParams p{a.a, a.b, a.A_log, a.dt_bias, a.cu_seqlens, a.T, a.Hqk, a.Hv, a.scale,
+               a.initial_state, a.final_state, a.o,
+               reinterpret_cast<uint32_t*>(static_cast<char*>(a.workspace) + kWsErrorWordOffset),
+               static_cast<uint8_t*>(a.workspace) + kWsHeaderBytes, gate_tma, n_prod};
+    const int64_t blocks = (int64_t)a.n_seq * a.Hv * csize;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = SMEM_ALLOC;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, prefill_cl_kernel, mq, mk, mv, ma, mb, mo, p);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

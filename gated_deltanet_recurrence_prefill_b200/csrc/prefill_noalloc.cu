@@ -42,8 +42,8 @@ gdn_status gdn_prefill_noalloc(const uint16_t* q, const uint16_t* k, const uint1
                                const float* initial_state, float* final_state, float* o,
                                gdn_stream_t stream) {
     // sizes first: nothing touches the GPU when the scratch array is too small
-    if (gdn_prefill_workspace_size(n_seq, T, Hqk, Hv, d) > kNoAllocScratchBytes)
-        return GDN_ERR_WORKSPACE;
+    (void)T; (void)Hqk; (void)d;
+    if (gdn::prefill_min_workspace_bytes(n_seq, Hv) > kNoAllocScratchBytes) return GDN_ERR_WORKSPACE;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return GDN_ERR_UNSUPPORTED;

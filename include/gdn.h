@@ -64,7 +64,7 @@ typedef enum gdn_status {
     GDN_ERR_MISALIGNED = 3,    /* a tensor pointer that is not 16-byte aligned */
     GDN_ERR_CUDA = 4,          /* a CUDA call or kernel launch failed (see gdn_last_cuda_error) */
     GDN_ERR_TIMEOUT = 5,       /* a bounded wait inside a kernel ran out (prefill only) */
-    GDN_ERR_WORKSPACE = 6      /* workspace NULL or smaller than gdn_prefill_workspace_size() */
+    GDN_ERR_WORKSPACE = 6      /* workspace NULL or below the least size gdn_prefill accepts */
 } gdn_status;
 
 /* Version of this ABI; bumped when a signature or a layout changes. */
@@ -107,8 +107,14 @@ gdn_status gdn_conv1d_silu(const uint16_t* qkv, const float* conv_w, const int32
                            uint16_t* q, uint16_t* k, uint16_t* v, gdn_stream_t stream);
 
 /*
- * gdn_prefill_workspace_size -- bytes of device workspace gdn_prefill needs for
- * these sizes (a multiple of 256).  Never 0.  Host-only, no CUDA calls.
+ * gdn_prefill_workspace_size -- bytes of device workspace with which
+ * gdn_prefill runs its fastest kernel for these sizes (a multiple of 256; never
+ * 0).  Host-only, no CUDA calls.  That kernel passes each chunk's
+ * state-independent operands from producer to consumer CTAs through a ring of
+ * 4 slots of 49664 bytes per (sequence, value head), so the size is
+ * 256 + 198656 * n_seq * Hv bytes (rounded up to 256).  gdn_prefill also
+ * accepts a workspace as small as 256 + 4 * n_seq * Hv bytes (rounded up to
+ * 256) and then runs a single-CTA kernel with the same results up to rounding.
  */
 size_t gdn_prefill_workspace_size(int32_t n_seq, int64_t T, int32_t Hqk, int32_t Hv, int32_t d);
 
@@ -130,12 +136,19 @@ size_t gdn_prefill_workspace_size(int32_t n_seq, int64_t T, int32_t Hqk, int32_t
  *  final_state    [n_seq, Hv, d_v, d_k] float32 or NULL (not written).  May be
  *                 the same pointer as initial_state (updated in place).
  *  o              [T, Hv, d] float32 output.
- *  workspace      device scratch of at least gdn_prefill_workspace_size()
- *                 bytes, 256-byte aligned; its contents on entry do not
- *                 matter.  Calls that share a workspace must be ordered on
- *                 one stream.
+ *  workspace      device scratch, 256-byte aligned, of
+ *                 gdn_prefill_workspace_size() bytes (or at least the smaller
+ *                 size given there, for the single-CTA kernel); its contents
+ *                 on entry do not matter.  Calls that share a workspace must be
+ *                 ordered on one stream.
  * A sequence of length 0 leaves final_state = initial_state (or zeros).
  * Supported: d = 128, Hv % Hqk == 0.
+ * Kernel choice: with the full workspace, a thread-block cluster per (sequence,
+ * value head) of one consumer CTA (the state chain) and two or one producer
+ * CTAs (the state-independent chunk algebra); otherwise one CTA per (sequence,
+ * value head, half of d).  The environment variables GDN_PREFILL_KERNEL
+ * (=cluster or =single) and GDN_PREFILL_PRODUCERS (=1 or =2) force a choice;
+ * a forced cluster kernel that cannot run returns GDN_ERR_UNSUPPORTED.
  * GDN_ERR_TIMEOUT is not returned here (the kernel does not stop the host):
  * a kernel that gave up on a bounded wait records it in the workspace, and
  * gdn_prefill_status() reports it.

@@ -79,7 +79,11 @@ def test_prefill_rejects_bad_arguments(L):
     assert call(A_log=None) == 1
     assert call(o=_p(FAKE + 4)) == 3             # misaligned
     assert call(ws=None) == 6
-    assert call(wsb=ws - 1) == 6
+    # the least workspace accepted: the 256-byte header and 4 bytes per
+    # (sequence, value head), rounded up to 256 bytes
+    min_ws = 256 + ((4 * 1 * 48 + 255) // 256) * 256
+    assert ws >= min_ws
+    assert call(wsb=min_ws - 1) == 6
     assert call(ws=_p(0x20000 + 16)) == 3        # workspace must be 256-byte aligned
 
 

@@ -14,6 +14,20 @@ from tests.helpers import dev_bf16, dev_f32, dev_i32, host, rel_err
 pytestmark = pytest.mark.gpu
 TOL = 1e-2
 
+# the prefill kernels gdn_prefill can run: the cluster kernel with two or one
+# producer CTAs per (sequence, value head), and the single-CTA kernel
+KERNELS = {"cluster2": {"GDN_PREFILL_KERNEL": "cluster", "GDN_PREFILL_PRODUCERS": "2"},
+           "cluster1": {"GDN_PREFILL_KERNEL": "cluster", "GDN_PREFILL_PRODUCERS": "1"},
+           "single": {"GDN_PREFILL_KERNEL": "single"}}
+
+
+@pytest.fixture(params=sorted(KERNELS))
+def kernel(request, monkeypatch):
+    monkeypatch.delenv("GDN_PREFILL_PRODUCERS", raising=False)
+    for k, v in KERNELS[request.param].items():
+        monkeypatch.setenv(k, v)
+    return request.param
+
 
 def _dev(inp):
     return dict(q=dev_bf16(inp.q), k=dev_bf16(inp.k), v=dev_bf16(inp.v), a=dev_f32(inp.a),
@@ -35,7 +49,7 @@ def _oracle(orc, inp, heads=None, seq_mask=None):
                        initial_state=inp.initial_state, heads=heads, seq_mask=seq_mask)
 
 
-def test_prefill_t256(orc):
+def test_prefill_t256(kernel, orc):
     """T = 256, one sequence, zero initial state (the 256-token workload)."""
     inp = synth.workload(0)
     o, s = _run(inp)
@@ -45,7 +59,7 @@ def test_prefill_t256(orc):
 
 
 @pytest.mark.parametrize("Hqk,Hv", [(16, 48), (4, 12), (2, 2)])
-def test_prefill_varlen_edges(orc, Hqk, Hv):
+def test_prefill_varlen_edges(kernel, orc, Hqk, Hv):
     """Lengths 0, 1, 63, 64, 65, 127, 129 and 200 packed together, non-zero
     per-sequence initial states."""
     lengths = [1, 63, 64, 0, 65, 127, 129, 200]
@@ -58,7 +72,7 @@ def test_prefill_varlen_edges(orc, Hqk, Hv):
     np.testing.assert_array_equal(host(s)[3], inp.initial_state[3].astype(np.float64))
 
 
-def test_prefill_strong_decay(orc):
+def test_prefill_strong_decay(kernel, orc):
     """A_log = ln 16 and a = +3 on some heads: the log-decay summed over a chunk
     falls far below -87 (e^G underflows float32); nothing may overflow."""
     inp = synth.make_prefill([300, 77], seed=61, init_state=True, Hqk=2, Hv=6)
@@ -71,7 +85,7 @@ def test_prefill_strong_decay(orc):
     assert rel_err(host(s), s_ref) <= TOL
 
 
-def test_prefill_in_place_state_and_null_final(orc):
+def test_prefill_in_place_state_and_null_final(kernel, orc):
     import torch
     import gated_deltanet_recurrence_prefill_b200 as gdn
     inp = synth.make_prefill([130, 5], seed=62, init_state=True, Hqk=2, Hv=4)
@@ -88,7 +102,7 @@ def test_prefill_in_place_state_and_null_final(orc):
     assert s2 is None and torch.equal(o, o2)
 
 
-def test_prefill_deterministic():
+def test_prefill_deterministic(kernel):
     import torch
     inp = synth.make_prefill([500, 37], seed=63, init_state=True, Hqk=4, Hv=12)
     d = _dev(inp)
@@ -97,7 +111,7 @@ def test_prefill_deterministic():
     assert torch.equal(o1, o2) and torch.equal(s1, s2)
 
 
-def test_varlen_equals_separate_calls():
+def test_varlen_equals_separate_calls(kernel):
     """Packing never mixes sequences: each sequence's outputs equal a call on
     that sequence alone, bit for bit."""
     import torch
@@ -116,7 +130,7 @@ def test_varlen_equals_separate_calls():
         assert torch.equal(s[n], s1[0])
 
 
-def test_split_prefill_equals_whole():
+def test_split_prefill_equals_whole(kernel):
     """prefill(T1) then prefill(T2, initial = final of the first) equals
     prefill(T1 + T2) when T1 is a whole number of chunks.  The kernel carries
     the state as Gamma * S~ with a running scale and rounds a bf16 copy of it
@@ -141,7 +155,7 @@ def test_split_prefill_equals_whole():
     assert torch.equal(o1, o[:T1])
 
 
-def test_prefill_one_token_equals_decode_step():
+def test_prefill_one_token_equals_decode_step(kernel):
     """A one-token prefill per unit is one decode step."""
     import gated_deltanet_recurrence_prefill_b200 as gdn
     dec = synth.make_decode(4, 1, seed=66, Hqk=4, Hv=12)
