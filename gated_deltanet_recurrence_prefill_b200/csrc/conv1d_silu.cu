@@ -21,7 +21,10 @@ constexpr int kD = 128;
 constexpr int kRun = 32;              // tokens per warp
 constexpr int kWarps = 8;             // warps per CTA
 constexpr int kChan = 8;              // channels per lane
-constexpr int kBatch = 8;             // tokens whose loads are in flight together
+#ifndef GDN_CONV_BATCH
+#define GDN_CONV_BATCH 4
+#endif
+constexpr int kBatch = GDN_CONV_BATCH;  // tokens per batch (two batches of loads in flight)
 
 // index of the sequence containing token t: largest n with cu[n] <= t
 __device__ int find_seq(const int32_t* cu, int n_seq, int64_t t) {
@@ -105,6 +108,8 @@ conv1d_silu_kernel(const uint16_t* __restrict__ qkv, const float* __restrict__ w
 
     const bool is_q = head < Hqk;
     const bool is_k = head >= Hqk && head < 2 * Hqk;
+    // does either half-warp hold a q or k head (then both take part in the reduction)
+    const bool warp_norm = __any_sync(0xffffffffu, is_q || is_k);
     uint16_t* dst_base;
     int64_t dst_stride;
     if (is_q) { dst_base = qo + (int64_t)head * kD; dst_stride = (int64_t)Hqk * kD; }
@@ -112,14 +117,21 @@ conv1d_silu_kernel(const uint16_t* __restrict__ qkv, const float* __restrict__ w
     else { dst_base = vo + (int64_t)(hc - 2 * Hqk) * kD; dst_stride = (int64_t)Hv * kD; }
     dst_base += (lane & 15) * kChan;
 
-    // tokens are processed in batches of kBatch: all loads of a batch are issued
-    // before any is used, so that kBatch x 16 bytes per lane are in flight
+    // tokens are processed in batches of kBatch: the loads of the next batch are
+    // issued before the current one is computed, so that up to 2 kBatch x 16
+    // bytes per lane are in flight while the lane does arithmetic
+    uint4 raw[kBatch], nxt[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+        const int64_t t = t0 + u;
+        raw[u] = t < t1 ? ldg_stream(qkv + t * Ctot + c0) : make_uint4(0, 0, 0, 0);
+    }
     for (int64_t tb = t0; tb < t1; tb += kBatch) {
-        uint4 raw[kBatch];
+        const int64_t tn = tb + kBatch;
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
-            const int64_t t = tb + u;
-            raw[u] = t < t1 ? ldg_stream(qkv + t * Ctot + c0) : make_uint4(0, 0, 0, 0);
+            const int64_t t = tn + u;
+            nxt[u] = t < t1 ? ldg_stream(qkv + t * Ctot + c0) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
         for (int u = 0; u < kBatch; ++u) {
@@ -146,17 +158,21 @@ conv1d_silu_kernel(const uint16_t* __restrict__ qkv, const float* __restrict__ w
                 acc = fmaf(wr[i][1], hist[1][i], acc);
                 acc = fmaf(wr[i][2], hist[2][i], acc);
                 acc = fmaf(wr[i][3], x[i], acc);
-                const float s = acc / (1.f + __expf(-acc));
+                // SiLU: acc * sigmoid(acc), with the fast reciprocal division
+                const float s = __fdividef(acc, 1.f + __expf(-acc));
                 y[i] = s;
                 ss = fmaf(s, s, ss);
                 hist[0][i] = hist[1][i];
                 hist[1][i] = hist[2][i];
                 hist[2][i] = x[i];
             }
-            // sum of squares over the 16 lanes of this head
+            // sum of squares over the 16 lanes of this head (value heads need none)
+            float inv = 1.f;
+            if (warp_norm) {        // warp-uniform: the shuffles need all 32 lanes
 #pragma unroll
-            for (int m = 8; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-            const float inv = (is_q || is_k) ? rsqrtf(ss + 1e-6f) : 1.f;
+                for (int m = 8; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+                if (is_q || is_k) inv = rsqrtf(ss + 1e-6f);
+            }
             uint4 out;
             out.x = pack_bf16x2(y[0] * inv, y[1] * inv);
             out.y = pack_bf16x2(y[2] * inv, y[3] * inv);
@@ -164,6 +180,8 @@ conv1d_silu_kernel(const uint16_t* __restrict__ qkv, const float* __restrict__ w
             out.w = pack_bf16x2(y[6] * inv, y[7] * inv);
             if (active) stg_stream(dst_base + t * dst_stride, out);
         }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) raw[u] = nxt[u];
     }
 }
 
