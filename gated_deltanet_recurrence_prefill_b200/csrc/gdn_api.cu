@@ -36,20 +36,19 @@ gdn_status check_seqs(const int32_t* cu_seqlens, int32_t n_seq, int64_t T) {
     return GDN_OK;
 }
 
-// Which prefill kernel runs: the cluster kernel (two producer CTAs and one
-// consumer CTA per sequence and value head) wherever clusters of three fit on
-// the device, else the single-CTA kernel.  GDN_PREFILL_KERNEL=single or
-// =cluster in the environment forces one of them (for comparisons and tests).
-// The cluster kernel also needs the workspace to hold its ring of chunk slots
-// (gdn_prefill_workspace_size); with less, the single-CTA kernel runs.
-enum class PrefillKernel { Cluster, Single, Unavailable };
+// Which prefill kernel runs: the producer / consumer kernel (two or one
+// producer CTAs and one consumer CTA per sequence and value head) when it can
+// run on the device and the workspace holds at least one unit's ring, else the
+// single-CTA kernel.  GDN_PREFILL_KERNEL=single or =pc in the environment
+// forces one of them (for comparisons and tests).
+enum class PrefillKernel { ProducerConsumer, Single, Unavailable };
 
-PrefillKernel pick_prefill_kernel(bool ring_fits) {
+PrefillKernel pick_prefill_kernel(size_t workspace_bytes) {
     const char* env = getenv("GDN_PREFILL_KERNEL");
     if (env && strcmp(env, "single") == 0) return PrefillKernel::Single;
-    const bool cl = ring_fits && gdn::prefill_cl_available();
-    if (env && strcmp(env, "cluster") == 0) return cl ? PrefillKernel::Cluster : PrefillKernel::Unavailable;
-    return cl ? PrefillKernel::Cluster : PrefillKernel::Single;
+    const bool pc = gdn::prefill_pc_available(workspace_bytes);
+    if (env && strcmp(env, "pc") == 0) return pc ? PrefillKernel::ProducerConsumer : PrefillKernel::Unavailable;
+    return pc ? PrefillKernel::ProducerConsumer : PrefillKernel::Single;
 }
 
 }  // namespace
@@ -109,7 +108,7 @@ gdn_status gdn_conv1d_silu(const uint16_t* qkv, const float* conv_w, const int32
 size_t gdn_prefill_workspace_size(int32_t n_seq, int64_t T, int32_t Hqk, int32_t Hv, int32_t d) {
     (void)T; (void)Hqk; (void)d;
     const size_t lo = gdn::prefill_min_workspace_bytes(n_seq, Hv);
-    const size_t hi = gdn::prefill_cl_workspace_bytes(n_seq, Hv);
+    const size_t hi = gdn::prefill_pc_workspace_bytes(n_seq, Hv);
     return hi > lo ? hi : lo;
 }
 
@@ -133,13 +132,12 @@ gdn_status gdn_prefill(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_MISALIGNED;
     gdn::PrefillArgs p{q, k, v, a, b, A_log, dt_bias, cu_seqlens, n_seq, T, Hqk, Hv, scale,
                        initial_state, final_state, o, workspace, workspace_bytes};
-    const PrefillKernel which =
-        pick_prefill_kernel(workspace_bytes >= gdn::prefill_cl_workspace_bytes(n_seq, Hv));
+    const PrefillKernel which = pick_prefill_kernel(workspace_bytes);
     if (which == PrefillKernel::Unavailable) return GDN_ERR_UNSUPPORTED;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = cudaMemsetAsync(workspace, 0, gdn::kWsHeaderBytes, s);
     if (e != cudaSuccess) return cuda_fail(e);
-    e = which == PrefillKernel::Cluster ? gdn::launch_prefill_cl(p, s) : gdn::launch_prefill_tc(p, s);
+    e = which == PrefillKernel::ProducerConsumer ? gdn::launch_prefill_pc(p, s) : gdn::launch_prefill_tc(p, s);
     return e == cudaSuccess ? GDN_OK : cuda_fail(e);
 }
 

@@ -43,14 +43,16 @@ cudaError_t launch_conv1d_silu(const uint16_t* qkv, const float* w, const int32_
 cudaError_t launch_prefill_simt(const PrefillArgs& p, cudaStream_t stream);
 cudaError_t launch_prefill_tc(const PrefillArgs& p, cudaStream_t stream);
 size_t prefill_tc_smem_bytes();
-// cluster (producer / consumer) prefill: needs clusters of two or three CTAs of
-// prefill_cl_smem_bytes() each to be schedulable on the current device
-cudaError_t launch_prefill_cl(const PrefillArgs& p, cudaStream_t stream);
-bool prefill_cl_available();
-int prefill_cl_max_active_clusters(int size);
-size_t prefill_cl_smem_bytes();
-// workspace the cluster kernel needs: the header and its ring of chunk slots
-size_t prefill_cl_workspace_bytes(int32_t n_seq, int32_t Hv);
+// producer / consumer prefill: a cooperative grid of one consumer and one or
+// two producer CTAs per (sequence, value head), handing chunks over through a
+// ring in the workspace; available when at least two of its CTAs can be
+// resident and the workspace holds one unit's ring
+cudaError_t launch_prefill_pc(const PrefillArgs& p, cudaStream_t stream);
+bool prefill_pc_available(size_t workspace_bytes);
+size_t prefill_pc_smem_bytes();
+// workspace with which the producer / consumer kernel runs every unit of a
+// launch that fits on the device (the header, counters and rings)
+size_t prefill_pc_workspace_bytes(int32_t n_seq, int32_t Hv);
 // workspace the single-CTA kernel needs (and the least gdn_prefill accepts)
 size_t prefill_min_workspace_bytes(int32_t n_seq, int32_t Hv);
 size_t prefill_simt_smem_bytes();

@@ -1,6 +1,7 @@
-// prefill_cl.cu -- chunked gated delta-rule prefill on the sm_100a tensor cores,
-// as a thread-block cluster per (sequence, value head): one consumer CTA runs
-// the state chain, one or two producer CTAs the state-independent algebra.
+// prefill_pc.cu -- chunked gated delta-rule prefill on the sm_100a tensor cores,
+// as a co-resident grid of producer and consumer CTAs: per (sequence, value
+// head) one consumer CTA runs the state chain and one or two producer CTAs the
+// state-independent algebra.
 //
 // The arithmetic is the chunked WY / UT form of the recurrence (Qwen3.8-27B
 // architecture page, 2kiu.com, section 2.2, with the decay alpha on the erased
@@ -14,7 +15,7 @@
 //     S <- gamma_C S + K^T diag(kappa) U
 // Everything up to [-W; Qh] and [T beta; R beta] is independent of the state.
 //
-// Producers (cluster ranks 1..P, P = 1 or 2).  Producer p takes chunks p,
+// Producers (roles 1..P, P = 1 or 2).  Producer p takes chunks p,
 // p + P, ...; inside it two groups of 8 warps take alternate chunks.  A group
 // computes the gates, D0 = [K; Q] K^T (tcgen05), A and P, T by blocked forward
 // substitution (16x16 diagonal blocks on CUDA cores, off-diagonal blocks with
@@ -25,11 +26,13 @@
 // gamma_C over the A scratch.  A publisher warp per group bulk-stores them to
 // the chunk's slot of a ring in global memory (kRing slots per (sequence,
 // value head), normally resident in L2), hands the staging back as soon as the
-// store has read it, and tells the consumer once the bytes are in place.
+// store has read it, and tells the consumer once the bytes are in place by
+// raising a counter in global memory (release / acquire at GPU scope).
 // Warp 16 loads [K; Q] and the gate inputs by TMA into three stages.
 //
-// Consumer (rank 0).  A loader thread bulk-loads each chunk from the ring into
-// one of two receive slots and hands ring slots back to the producers.  d_v is
+// Consumer (role 0).  A loader thread bulk-loads each chunk from the ring into
+// one of two receive slots and hands ring slots back to the producers (a
+// second counter per ring slot).  d_v is
 // split in two halves of 64 that evolve independently (the rows of S do not mix
 // once T is known); each half has its own MMA issuer thread (warps 1 and 3) and
 // four epilogue warps, so one half's products overlap the other's epilogues:
@@ -43,9 +46,16 @@
 // shared memory and written by TMA (plain stores for a sequence's ragged last
 // chunk).  Warp 0 loads V and K by TMA.
 //
-// Every wait on an mbarrier is bounded; on expiry a CTA records an error in the
-// workspace, raises the abort flag of every CTA of its cluster, stops waiting and
-// drains its own tensor-core work and copies.  Producer group warps never leave
+// Grid.  For nu units, blocks [0, nu) are the consumers and blocks
+// [nu, (1 + P) nu) the producers (block b serves unit b % nu).  They wait
+// on one another, so the launch is cooperative: the whole grid is resident at
+// once (one CTA per SM), and units beyond one grid's worth run in further
+// launches.  No thread-block cluster is used, so the CTAs of a unit may sit
+// anywhere on the GPU.
+//
+// Every wait is bounded; on expiry a CTA records an error in the workspace
+// (which makes the other CTAs' waits on global counters give up too), stops
+// waiting and drains its own tensor-core work and copies.  Producer group warps never leave
 // their loop early (their named barriers must always complete): after an abort
 // their waits simply fall through.
 #include <cuda.h>
@@ -68,7 +78,6 @@ using namespace tile;
 
 constexpr int kD = 128;
 constexpr int kC = 64;
-constexpr int kMaxProducers = 2;
 constexpr int kWarps = 19;
 constexpr int kThreads = kWarps * 32;
 constexpr int kGroupThreads = 256;
@@ -122,13 +131,21 @@ constexpr uint32_t C_END = C_OST + 32768;
 constexpr uint32_t SEND_QW = 2 * KQ_PANEL;
 constexpr uint32_t SEND_RT = 16384 + 512;
 static_assert(SL_GATES == SL_RT2 + 16384 && SEND_RT <= 64 * kLdF * 4, "staging layout");
-// The chunks travel through a ring of kRing slots per (sequence, value head) in
-// the workspace (global memory, normally resident in L2): the producer's bulk
-// store frees its staging as soon as the bytes have been read, and the consumer
-// bulk-loads a chunk into its shared memory when a receive slot is free.
+// The chunks travel through a ring of kRing slots per unit of a launch in the
+// workspace (global memory, normally resident in L2): the producer's bulk store
+// frees its staging as soon as the bytes have been read, and the consumer
+// bulk-loads a chunk into its shared memory when a receive slot is free.  Two
+// counters per ring slot, in their own 128-byte line per unit, hand the slot
+// back and forth: ready[rs] = chunks written to slot rs, freed[rs] = chunks
+// the consumer has taken out of it (chunk c uses slot c % kRing).
 constexpr int kRing = 4;
 constexpr uint32_t GSLOT_BYTES = SEND_QW + SEND_RT;
 static_assert(GSLOT_BYTES % 128 == 0 && kRing % 2 == 0, "ring layout");
+constexpr uint32_t kFlagWords = 32;            // per unit: ready[kRing] at 0, freed[kRing] at 16
+constexpr uint32_t kFreedAt = 16;
+// units whose rings the workspace is sized for (one launch handles at most
+// this many; more run in further launches)
+constexpr int kMaxSlots = 64;
 
 constexpr uint32_t OFF_MISC = (P_END > C_END ? P_END : C_END);
 constexpr uint32_t OFF_BARS = OFF_MISC + 64;
@@ -136,11 +153,11 @@ constexpr uint32_t OFF_BARS = OFF_MISC + 64;
 enum {
     // producer
     PB_KQ_FULL = 0, PB_KQ_TAKEN = 2, PB_KQ_EMPTY = 4, PB_D0_FULL = 7, PB_R_FULL = 9,
-    PB_X1_FULL = 11, PB_DRAIN = 13, PB_STAGED = 15, PB_AF_FREE = 17, PB_GFREE = 19,
+    PB_X1_FULL = 11, PB_DRAIN = 13, PB_STAGED = 15, PB_AF_FREE = 17,
     // consumer
-    CB_RECV_FULL = 23, CB_K_FULL = 25, CB_K_EMPTY, CB_V_FULL, CB_V_EMPTY, CB_D_EMPTY = 29,
-    CB_D_FULL = 31, CB_S_OK = 33, CB_S_FULL = 35, CB_ST_READY = 37, CB_DRAIN = 39, CB_GREADY = 41,
-    kNumBars = 45
+    CB_RECV_FULL = 19, CB_K_FULL = 21, CB_K_EMPTY, CB_V_FULL, CB_V_EMPTY, CB_D_EMPTY = 25,
+    CB_D_FULL = 27, CB_S_OK = 29, CB_S_FULL = 31, CB_ST_READY = 33, CB_DRAIN = 35,
+    kNumBars = 37
 };
 constexpr uint32_t SMEM_BYTES = OFF_BARS + kNumBars * 8;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;           // room to align the base
@@ -177,9 +194,11 @@ struct ClParams {
     float* s_out;
     float* o;
     uint32_t* err;
-    uint8_t* ring;         // kRing slots of GSLOT_BYTES per (sequence, value head)
+    uint8_t* ring;         // kRing slots of GSLOT_BYTES per unit of this launch
+    uint32_t* flags;       // kFlagWords counters per unit of this launch
     int gate_tma;          // a, b staged by TMA (needs Hv % 4 == 0), else read directly
-    int n_prod;            // producer CTAs per cluster (1 or 2); the cluster has n_prod + 1
+    int n_prod;            // producer CTAs per unit (1 or 2); a unit has n_prod + 1 CTAs
+    int unit0;             // first (sequence, value head) unit of this launch
 };
 
 struct Ctx {
@@ -189,7 +208,10 @@ struct Ctx {
     volatile int* abort;
     int warp, lane;
     int h, g;              // value head, key head
-    uint8_t* ring;         // this cluster's ring slots
+    uint8_t* ring;         // this unit's ring slots
+    uint32_t* ready;       // this unit's counters: chunks written to each ring slot
+    uint32_t* freed;       //   and chunks taken out of each ring slot
+    const uint32_t* err;   // the launch's error word
     int64_t bos, eos;
     int nch;
     int64_t state_off;
@@ -287,20 +309,21 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
         }
     } else if (warp == 2) {
         // ------------------------------------------------ loader: ring slot -> receive slot
-        // Chunk c sits in ring slot c % kRing; producer (c % kRing) % P owns that
-        // slot's "free" barrier.  A slot is handed back once its chunk has been
-        // loaded (checked one chunk later, so that loads overlap).
+        // Chunk c sits in ring slot c % kRing.  A slot is handed back once its
+        // chunk has been loaded (checked one chunk later, so that loads overlap).
         if (lane == 0) {
             auto ring_free = [&](int c) {
-                const int rs = c % kRing;
-                mbar_arrive_cluster(map_to_rank(x.bar(PB_GFREE + rs), 1 + (uint32_t)(rs % p.n_prod)));
+                // the bulk load of chunk c has completed (its barrier was seen)
+                fence_async_global();
+                st_release_gpu(x.freed + c % kRing, (uint32_t)(c / kRing + 1));
             };
             int loaded = 0;
             for (int c = 0; c < nch; ++c) {
                 const int b = c & 1, rs = c % kRing;
                 if (c >= 2 && !mbar_wait(x.bar(CB_D_EMPTY + b), ((c >> 1) - 1) & 1, x.abort, kWaitLimitNs))
                     break;
-                if (!mbar_wait_cluster(x.bar(CB_GREADY + rs), (c / kRing) & 1, x.abort, kWaitLimitNs)) break;
+                if (!gflag_wait_ge(x.ready + rs, (uint32_t)(c / kRing + 1), x.abort, x.err, kWaitLimitNs))
+                    break;
                 fence_async_global();
                 const uint32_t slot = x.sbase + C_RECV + b * SLOT_BYTES;
                 const uint8_t* g = x.ring + (size_t)rs * GSLOT_BYTES;
@@ -311,7 +334,7 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
                 if (c >= 1) {
                     if (!mbar_wait(x.bar(CB_RECV_FULL + ((c - 1) & 1)), ((c - 1) >> 1) & 1, x.abort, kWaitLimitNs))
                         break;
-                    if (c - 1 + kRing < nch) ring_free(c - 1);
+                    ring_free(c - 1);
                 }
             }
             // loads still in flight land before the CTA may exit
@@ -515,7 +538,6 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
         // consumer is told once the bytes are in global memory.
         const int grp = warp - 17;
         if (lane == 0) {
-            const uint32_t gready0 = map_to_rank(x.bar(CB_GREADY), 0);
             const uint32_t stage_rt = x.sbase + P_GROUP + grp * GROUP_BYTES + G_AF;
             for (int jj = 0;; ++jj) {
                 const int i = grp + 2 * jj;
@@ -524,7 +546,7 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
                 const int rs = c % kRing;
                 if (!mbar_wait(x.bar(PB_STAGED + grp), jj & 1, x.abort, kWaitLimitNs)) break;
                 if (c >= kRing &&
-                    !mbar_wait_cluster(x.bar(PB_GFREE + rs), (c / kRing - 1) & 1, x.abort, kWaitLimitNs))
+                    !gflag_wait_ge(x.freed + rs, (uint32_t)(c / kRing), x.abort, x.err, kWaitLimitNs))
                     break;
                 fence_async_global();
                 uint8_t* g = x.ring + (size_t)rs * GSLOT_BYTES;
@@ -536,7 +558,7 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
                 mbar_arrive(x.bar(PB_AF_FREE + grp));
                 bulk_wait();
                 fence_async_global();
-                mbar_arrive_cluster(gready0 + 8u * (uint32_t)rs);
+                st_release_gpu(x.ready + rs, (uint32_t)(c / kRing + 1));
             }
         }
         return;
@@ -850,14 +872,13 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-prefill_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+prefill_pc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
                   const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_o,
                   const ClParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // align to 1024 bytes by pointer arithmetic on the shared array, so that
-    // every access below stays in the shared state space; the offset is the same
-    // in every CTA of the cluster, so local offsets name the peers' buffers too
+    // every access below stays in the shared state space
     uint8_t* sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     Ctx x;
     x.sm = sm;
@@ -867,19 +888,28 @@ prefill_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC + 4);
     x.warp = threadIdx.x >> 5;
     x.lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_ctarank();
-    const int cl = blockIdx.x / (p.n_prod + 1);
-    x.h = cl % p.Hv;
-    const int n = cl / p.Hv;
+    // blocks [0, nu) are the consumers of the launch's nu units, then the first
+    // producers of every unit, then the second ones: consecutive blocks tend to
+    // land on the two SMs of one TPC, and a consumer next to a producer runs its
+    // state chain about half as fast as next to another consumer
+    const uint32_t nu = gridDim.x / (uint32_t)(p.n_prod + 1);
+    const int slot = (int)(blockIdx.x % nu);                        // unit within this launch
+    const uint32_t rank = blockIdx.x / nu;                          // 0 = consumer, 1.. = producers
+    const int unit = p.unit0 + slot;
+    x.h = unit % p.Hv;
+    const int n = unit / p.Hv;
     x.g = x.h / (p.Hv / p.Hqk);
     x.bos = p.cu ? p.cu[n] : 0;
     x.eos = p.cu ? p.cu[n + 1] : p.T;
     x.nch = (int)((x.eos - x.bos + kC - 1) / kC);
     x.state_off = ((int64_t)n * p.Hv + x.h) * kD * kD;
-    x.ring = p.ring + (size_t)cl * kRing * GSLOT_BYTES;
+    x.ring = p.ring + (size_t)slot * kRing * GSLOT_BYTES;
+    x.ready = p.flags + (size_t)slot * kFlagWords;
+    x.freed = x.ready + kFreedAt;
+    x.err = p.err;
 
     if (x.nch == 0) {
-        // empty sequence (the same in every CTA of the cluster): final state = initial state
+        // empty sequence (the same in every CTA of the unit): final state = initial state
         if (rank == 0 && p.s_out && p.s_out != p.s_in) {
             for (int i = threadIdx.x; i < kD * kD; i += kThreads)
                 p.s_out[x.state_off + i] = p.s_in ? p.s_in[x.state_off + i] : 0.f;
@@ -905,10 +935,8 @@ prefill_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 mbar_init(x.bar(CB_ST_READY + hh), 4);
                 mbar_init(x.bar(CB_DRAIN + hh), 1);
             }
-            for (int r = 0; r < kRing; ++r) mbar_init(x.bar(CB_GREADY + r), 1);
         } else {
             for (int s = 0; s < kKqStages; ++s) mbar_init(x.bar(PB_KQ_EMPTY + s), 1);
-            for (int r = 0; r < kRing; ++r) mbar_init(x.bar(PB_GFREE + r), 1);
             for (int grp = 0; grp < 2; ++grp) {
                 mbar_init(x.bar(PB_KQ_FULL + grp), 1);
                 mbar_init(x.bar(PB_KQ_TAKEN + grp), 8);
@@ -932,7 +960,6 @@ prefill_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     tc_fence_before();
     __syncthreads();
-    cluster_sync();            // every CTA's barriers exist before anyone arrives remotely
     tc_fence_after();
     x.tmem = *tmem_slot;
 
@@ -944,13 +971,9 @@ prefill_cl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // ---------------------------------------------------------------- teardown
     tc_fence_before();
     __syncthreads();
-    if (threadIdx.x == 0 && *x.abort) {
-        atomicOr(p.err, 1u);
-        // let the other CTAs of the cluster stop waiting for this one
-        for (uint32_t r = 0; r <= (uint32_t)p.n_prod; ++r)
-            if (r != rank) st_cluster_u32(map_to_rank(smem_u32(sm + OFF_MISC), r), 1u);
-    }
-    cluster_sync();            // no CTA leaves while a peer may still touch its shared memory
+    // a CTA that gave up records it; the other CTAs' waits on global counters
+    // see the error word and give up too
+    if (threadIdx.x == 0 && *x.abort) atomicOr(p.err, 1u);
     if (x.warp == 2) {
         tc_fence_after();
         tmem_dealloc(x.tmem, TMEM_COLS);
@@ -1016,76 +1039,67 @@ bool make_map_gates(CUtensorMap* m, const float* base, int64_t rows, int64_t col
 }
 
 cudaError_t setup_kernel() {
-    return cudaFuncSetAttribute(prefill_cl_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(prefill_pc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)SMEM_ALLOC);
 }
 
-// clusters of `size` CTAs that can be resident at once on the current device
-// (0 when none fit); cached per device
-std::atomic<int> g_max_clusters[64][2];     // [device][size - 2], stored + 1 (0 = unknown)
+// CTAs of this kernel that can be resident at once on the current device (0 if
+// none); cached per device
+std::atomic<int> g_resident[64];           // stored + 1 (0 = unknown)
 
-int max_active_clusters(int size) {
+int resident_ctas() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    int v = g_max_clusters[dev][size - 2].load(std::memory_order_relaxed);
+    int v = g_resident[dev].load(std::memory_order_relaxed);
     if (v > 0) return v - 1;
-    int clusters = 0;
-    if (setup_kernel() == cudaSuccess) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(size);
-        cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = SMEM_ALLOC;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = size;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        if (cudaOccupancyMaxActiveClusters(&clusters, prefill_cl_kernel, &cfg) != cudaSuccess)
-            clusters = 0;
-    }
+    int per_sm = 0, sms = 0, coop = 0;
+    if (setup_kernel() != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, prefill_pc_kernel, kThreads, SMEM_ALLOC) !=
+            cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess || !coop)
+        per_sm = 0;
     cudaGetLastError();    // a refused query leaves no sticky error behind
-    g_max_clusters[dev][size - 2].store(clusters + 1, std::memory_order_relaxed);
-    return clusters;
+    const int total = per_sm * sms;
+    g_resident[dev].store(total + 1, std::memory_order_relaxed);
+    return total;
 }
 
-// Producer CTAs per cluster for `units` (sequence, value head) pairs.  Two
-// producers keep the consumer's state chain busy (a chunk takes about half as
-// long as with one), so they win unless clusters of three need more than
-// twice as many waves of resident clusters as clusters of two.
-// GDN_PREFILL_PRODUCERS=1 or =2 in the environment forces the choice.
-int pick_producers(int64_t units) {
+// Producer CTAs per unit: two keep the consumer's state chain busy; one when
+// fewer than three CTAs are resident.  GDN_PREFILL_PRODUCERS=1 or =2 in the
+// environment forces the choice.
+int pick_producers(int resident) {
     const char* env = getenv("GDN_PREFILL_PRODUCERS");
     if (env && (env[0] == '1' || env[0] == '2') && env[1] == 0) {
         const int want = env[0] - '0';
-        return max_active_clusters(want + 1) > 0 ? want : 0;
+        return resident >= want + 1 ? want : 0;
     }
-    const int m3 = max_active_clusters(3);
-    const int m2 = max_active_clusters(2);
-    if (m3 <= 0) return m2 > 0 ? 1 : 0;
-    if (m2 <= 0) return 2;
-    const int64_t waves3 = (units + m3 - 1) / m3, waves2 = (units + m2 - 1) / m2;
-    return waves3 <= 2 * waves2 ? 2 : 1;
+    return resident >= 3 ? 2 : (resident >= 2 ? 1 : 0);
+}
+
+size_t ring_bytes_per_unit() { return (size_t)kRing * GSLOT_BYTES + kFlagWords * sizeof(uint32_t); }
+
+// units whose ring a workspace of `bytes` holds
+int64_t slots_in(size_t bytes) {
+    if (bytes < kWsHeaderBytes) return 0;
+    return (int64_t)((bytes - kWsHeaderBytes) / ring_bytes_per_unit());
 }
 
 }  // namespace
 
-size_t prefill_cl_smem_bytes() { return SMEM_ALLOC; }
+size_t prefill_pc_smem_bytes() { return SMEM_ALLOC; }
 
-size_t prefill_cl_workspace_bytes(int32_t n_seq, int32_t Hv) {
-    const size_t units = (size_t)(n_seq > 0 ? n_seq : 1) * (size_t)(Hv > 0 ? Hv : 1);
-    return kWsHeaderBytes + ((units * kRing * GSLOT_BYTES + 255) / 256) * 256;
+size_t prefill_pc_workspace_bytes(int32_t n_seq, int32_t Hv) {
+    const int64_t units = (int64_t)(n_seq > 0 ? n_seq : 1) * (Hv > 0 ? Hv : 1);
+    const int64_t slots = units < kMaxSlots ? units : kMaxSlots;
+    return kWsHeaderBytes + (((size_t)slots * ring_bytes_per_unit() + 255) / 256) * 256;
 }
 
-bool prefill_cl_available() { return max_active_clusters(2) > 0 || max_active_clusters(3) > 0; }
-
-int prefill_cl_max_active_clusters(int size) {
-    if (size != 2 && size != 3) return -1;
-    return max_active_clusters(size);
+bool prefill_pc_available(size_t workspace_bytes) {
+    return slots_in(workspace_bytes) >= 1 && resident_ctas() >= 2;
 }
 
-cudaError_t launch_prefill_cl(const PrefillArgs& a, cudaStream_t stream) {
+cudaError_t launch_prefill_pc(const PrefillArgs& a, cudaStream_t stream) {
     if (a.T == 0) {
         // every sequence is empty: final state = initial state
         if (a.final_state && a.final_state != a.initial_state) {
@@ -1112,29 +1126,46 @@ cudaError_t launch_prefill_cl(const PrefillArgs& a, cudaStream_t stream) {
     }
     cudaError_t e = setup_kernel();
     if (e != cudaSuccess) return e;
-    const int n_prod = pick_producers((int64_t)a.n_seq * a.Hv);
+    const int64_t units = (int64_t)a.n_seq * a.Hv;
+    const int resident = resident_ctas();
+    const int n_prod = pick_producers(resident);
     if (n_prod == 0) return cudaErrorNotSupported;
     const int csize = n_prod + 1;
+    int64_t per_launch = resident / csize;
+    const int64_t slots = slots_in(a.workspace_bytes);
+    if (per_launch > slots) per_launch = slots;
+    if (per_launch > kMaxSlots) per_launch = kMaxSlots;
+    if (per_launch < 1) return cudaErrorNotSupported;
+    // whole sequences per launch where they fit, so that a launch's units end
+    // together when the sequences differ in length
+    if (per_launch > a.Hv && units > per_launch) per_launch -= per_launch % a.Hv;
+    uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+    uint32_t* flags = reinterpret_cast<uint32_t*>(ws + kWsHeaderBytes);
+    uint8_t* ring = ws + kWsHeaderBytes + (size_t)per_launch * kFlagWords * sizeof(uint32_t);
     ClParams p{a.a, a.b, a.A_log, a.dt_bias, a.cu_seqlens, a.T, a.Hqk, a.Hv, a.scale,
                a.initial_state, a.final_state, a.o,
-               reinterpret_cast<uint32_t*>(static_cast<char*>(a.workspace) + kWsErrorWordOffset),
-               static_cast<uint8_t*>(a.workspace) + kWsHeaderBytes, gate_tma, n_prod};
-    const int64_t blocks = (int64_t)a.n_seq * a.Hv * csize;
-    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)blocks);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = SMEM_ALLOC;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = csize;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, prefill_cl_kernel, mq, mk, mv, ma, mb, mo, p);
-    if (e != cudaSuccess) return e;
+               reinterpret_cast<uint32_t*>(ws + kWsErrorWordOffset), ring, flags, gate_tma, n_prod, 0};
+    // Units run in launches of at most per_launch units, in order; each launch
+    // starts from cleared counters.  A unit's CTAs wait on one another, so each
+    // launch is cooperative (all of its CTAs resident together).
+    for (int64_t u0 = 0; u0 < units; u0 += per_launch) {
+        const int64_t nu = units - u0 < per_launch ? units - u0 : per_launch;
+        e = cudaMemsetAsync(flags, 0, (size_t)nu * kFlagWords * sizeof(uint32_t), stream);
+        if (e != cudaSuccess) return e;
+        p.unit0 = (int)u0;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(nu * csize));
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = SMEM_ALLOC;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, prefill_pc_kernel, mq, mk, mv, ma, mb, mo, p);
+        if (e != cudaSuccess) return e;
+    }
     return cudaGetLastError();
 }
 

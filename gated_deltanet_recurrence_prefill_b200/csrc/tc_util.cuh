@@ -116,6 +116,38 @@ TC_DEVICE bool mbar_wait_cluster(uint32_t bar, uint32_t parity, volatile int* ab
     }
 }
 
+// ---- counters in global memory shared between CTAs of one grid ---------------
+
+TC_DEVICE uint32_t ld_acquire_gpu(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+TC_DEVICE void st_release_gpu(uint32_t* p, uint32_t v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Bounded wait until the counter at `flag` (written by another CTA with
+// st_release_gpu) reaches `target`.  Gives up, raising *abort, when *abort is
+// set by another thread of this CTA, when the grid's error word `err` is set
+// by another CTA, or when `limit_ns` has passed; returns false then.
+TC_DEVICE bool gflag_wait_ge(const uint32_t* flag, uint32_t target, volatile int* abort,
+                             const uint32_t* err, uint64_t limit_ns) {
+    if (ld_acquire_gpu(flag) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (ld_acquire_gpu(flag) >= target) return true;
+        if ((it & 7u) == 0) {
+            if (*abort) return false;
+            if (*reinterpret_cast<const volatile uint32_t*>(err) != 0u ||
+                globaltimer_ns() - t0 > limit_ns) {
+                *abort = 1;
+                return false;
+            }
+        }
+    }
+}
+
 // ---- thread-block cluster (distributed shared memory) -----------------------
 
 TC_DEVICE uint32_t cluster_ctarank() {

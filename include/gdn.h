@@ -111,10 +111,13 @@ gdn_status gdn_conv1d_silu(const uint16_t* qkv, const float* conv_w, const int32
  * gdn_prefill runs its fastest kernel for these sizes (a multiple of 256; never
  * 0).  Host-only, no CUDA calls.  That kernel passes each chunk's
  * state-independent operands from producer to consumer CTAs through a ring of
- * 4 slots of 49664 bytes per (sequence, value head), so the size is
- * 256 + 198656 * n_seq * Hv bytes (rounded up to 256).  gdn_prefill also
- * accepts a workspace as small as 256 + 4 * n_seq * Hv bytes (rounded up to
- * 256) and then runs a single-CTA kernel with the same results up to rounding.
+ * 4 slots of 49664 bytes plus 128 bytes of counters per (sequence, value head)
+ * of one launch, and a launch holds at most 64 of them, so the size is
+ * 256 + 198784 * min(n_seq * Hv, 64) bytes (rounded up to 256).  A smaller
+ * workspace that holds at least one such ring runs fewer (sequence, value head)
+ * pairs per launch.  gdn_prefill also accepts a workspace as small as
+ * 256 + 4 * n_seq * Hv bytes (rounded up to 256) and then runs a single-CTA
+ * kernel with the same results up to rounding.
  */
 size_t gdn_prefill_workspace_size(int32_t n_seq, int64_t T, int32_t Hqk, int32_t Hv, int32_t d);
 
@@ -143,12 +146,14 @@ size_t gdn_prefill_workspace_size(int32_t n_seq, int64_t T, int32_t Hqk, int32_t
  *                 ordered on one stream.
  * A sequence of length 0 leaves final_state = initial_state (or zeros).
  * Supported: d = 128, Hv % Hqk == 0.
- * Kernel choice: with the full workspace, a thread-block cluster per (sequence,
- * value head) of one consumer CTA (the state chain) and two or one producer
- * CTAs (the state-independent chunk algebra); otherwise one CTA per (sequence,
- * value head, half of d).  The environment variables GDN_PREFILL_KERNEL
- * (=cluster or =single) and GDN_PREFILL_PRODUCERS (=1 or =2) force a choice;
- * a forced cluster kernel that cannot run returns GDN_ERR_UNSUPPORTED.
+ * Kernel choice: with a workspace that holds at least one ring (see
+ * gdn_prefill_workspace_size), a cooperative grid of one consumer CTA (the
+ * state chain) and two or one producer CTAs (the state-independent chunk
+ * algebra) per (sequence, value head), in launches of as many pairs as fit on
+ * the device at once; otherwise one CTA per (sequence, value head, half of d).
+ * The environment variables GDN_PREFILL_KERNEL (=pc or =single) and
+ * GDN_PREFILL_PRODUCERS (=1 or =2) force a choice; a forced producer /
+ * consumer kernel that cannot run returns GDN_ERR_UNSUPPORTED.
  * GDN_ERR_TIMEOUT is not returned here (the kernel does not stop the host):
  * a kernel that gave up on a bounded wait records it in the workspace, and
  * gdn_prefill_status() reports it.

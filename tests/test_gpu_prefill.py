@@ -14,10 +14,10 @@ from tests.helpers import dev_bf16, dev_f32, dev_i32, host, rel_err
 pytestmark = pytest.mark.gpu
 TOL = 1e-2
 
-# the prefill kernels gdn_prefill can run: the cluster kernel with two or one
-# producer CTAs per (sequence, value head), and the single-CTA kernel
-KERNELS = {"cluster2": {"GDN_PREFILL_KERNEL": "cluster", "GDN_PREFILL_PRODUCERS": "2"},
-           "cluster1": {"GDN_PREFILL_KERNEL": "cluster", "GDN_PREFILL_PRODUCERS": "1"},
+# the prefill kernels gdn_prefill can run: the producer / consumer kernel with
+# two or one producer CTAs per (sequence, value head), and the single-CTA kernel
+KERNELS = {"pc2": {"GDN_PREFILL_KERNEL": "pc", "GDN_PREFILL_PRODUCERS": "2"},
+           "pc1": {"GDN_PREFILL_KERNEL": "pc", "GDN_PREFILL_PRODUCERS": "1"},
            "single": {"GDN_PREFILL_KERNEL": "single"}}
 
 
