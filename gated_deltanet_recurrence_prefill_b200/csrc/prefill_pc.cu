@@ -32,19 +32,21 @@
 //
 // Consumer (role 0).  A loader thread bulk-loads each chunk from the ring into
 // one of two receive slots and hands ring slots back to the producers (a
-// second counter per ring slot).  d_v is
-// split in two halves of 64 that evolve independently (the rows of S do not mix
-// once T is known); each half has its own MMA issuer thread (warps 1 and 3) and
-// four epilogue warps, so one half's products overlap the other's epilogues:
-//   D  = [T b; R b] V_half                 M128 N64 K64   -> [U'; O']
-//   D += [-W; Qh] S_half^T                 M128 N64 K128  -> [U; o / scale]
-//   S~_half += K^T (kappa U / Gamma)        M128 N64 K64   (accumulates in TMEM)
-// The float32 state lives in TMEM as S~ with S = Gamma S~ (the decay gamma_C of
-// each chunk is folded into the running scalar Gamma and the update is added as
-// kappa U / Gamma); S~ is rescaled in place only when Gamma would fall below
-// 2^-80.  A bf16 copy of S is the operand of the next chunk.  o is staged in
-// shared memory and written by TMA (plain stores for a sequence's ragged last
-// chunk).  Warp 0 loads V and K by TMA.
+// second counter per ring slot).  Each product spans all 128 columns of d_v
+// (a tcgen05.mma takes about as long to issue at N = 64 as at N = 128, and one
+// thread issues one every ~75 cycles at best):
+//   E  = [T b; R b] V                      M128 N128 K64   (warp 1, ahead of the chain)
+//   D  = [-W; Qh] S^T                      M128 N128 K128  -> [U; o / scale] = D + E
+//   S~ += K^T (kappa U / Gamma)            M128 N128 K64   (accumulates in TMEM)
+// The last two are the state chain; lane 0 of the first epilogue warp issues
+// them right after the epilogue warps' named barrier.  The float32 state lives
+// in TMEM as S~ with S = Gamma S~ (the decay gamma_C of each chunk is folded
+// into the running scalar Gamma and the update is added as kappa U / Gamma);
+// S~ is rescaled in place only when Gamma would fall below 2^-80.  A bf16 copy
+// of S is the operand of the next chunk.  o is staged in shared memory and
+// written by TMA while the state update runs (plain stores for a sequence's
+// ragged last chunk).
+// Warp 0 loads V and K by TMA.
 //
 // Grid.  For nu units, blocks [0, nu) are the consumers and blocks
 // [nu, (1 + P) nu) the producers (block b serves unit b % nu).  They wait
@@ -78,7 +80,7 @@ using namespace tile;
 
 constexpr int kD = 128;
 constexpr int kC = 64;
-constexpr int kWarps = 19;
+constexpr int kWarps = 20;
 constexpr int kThreads = kWarps * 32;
 constexpr int kGroupThreads = 256;
 constexpr int kLdF = 68;                       // fp32 solve scratch row stride
@@ -113,24 +115,27 @@ constexpr uint32_t P_END = P_GROUP + 2 * GROUP_BYTES;
 static_assert(P_GROUP % 1024 == 0 && GROUP_BYTES % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 
 // ---- consumer shared memory ----------------------------------------------------
-// receive slot: [-W; Qh] (2 panels of 128 rows x 64 d), [T b; R b] (128 x 64),
-// kappa[64] and gamma_C -- the producer's staged bytes, copied verbatim
+// receive slot: [-W; Qh] (2 panels of 128 rows x 64 d) and [T b; R b]
+// (128 x 64) -- the producer's staged tiles, copied verbatim; the chunk's
+// kappa[64] and gamma_C go to a small gate buffer per slot
 constexpr uint32_t SL_QW = 0;
 constexpr uint32_t SL_RT2 = 2 * KQ_PANEL;
-constexpr uint32_t SL_GATES = SL_RT2 + 16384;
-constexpr uint32_t SLOT_BYTES = (SL_GATES + 512 + 1023) & ~1023u;
+constexpr uint32_t SLOT_BYTES = SL_RT2 + 16384;             // a multiple of 1024
+constexpr uint32_t GATES_AT = 16384;                        // kappa[64], gamma_C after [T b; R b] when staged
+constexpr uint32_t GATE_BYTES = 512;
 constexpr uint32_t C_RECV = 0;                              // 2 slots
-constexpr uint32_t C_V = C_RECV + 2 * SLOT_BYTES;           // V: 2 panels of 64 x 64 bf16
-constexpr uint32_t C_K = C_V + 16384;                       // K: 2 panels of 64 x 64 bf16
+constexpr uint32_t C_V = C_RECV + 2 * SLOT_BYTES;           // V: 2 buffers of 2 panels of 64 x 64 bf16
+constexpr uint32_t C_K = C_V + 2 * 16384;                   // K: 2 panels of 64 x 64 bf16
 constexpr uint32_t C_ST = C_K + 16384;                      // S^T bf16: 2 halves of 128 x 64
 constexpr uint32_t C_UK = C_ST + 32768;                     // kappa U / Gamma: 2 halves of 64 x 64
-constexpr uint32_t C_OST = C_UK + 16384;                    // o staging: 2 halves x 2 boxes of 64 x 32 f32
-constexpr uint32_t C_END = C_OST + 32768;
+constexpr uint32_t C_OST = C_UK + 16384;                    // o staging: 4 boxes of 64 x 32 f32
+constexpr uint32_t C_GATES = C_OST + 32768;                 // 2 gate buffers
+constexpr uint32_t C_END = C_GATES + 2 * GATE_BYTES;
 // what one chunk sends: the [-W; Qh] tile (staged in place of [K; Q]) and the
 // [T b; R b] tile with the gates (staged in the A scratch)
 constexpr uint32_t SEND_QW = 2 * KQ_PANEL;
-constexpr uint32_t SEND_RT = 16384 + 512;
-static_assert(SL_GATES == SL_RT2 + 16384 && SEND_RT <= 64 * kLdF * 4, "staging layout");
+constexpr uint32_t SEND_RT = GATES_AT + GATE_BYTES;
+static_assert(SEND_RT == GATES_AT + GATE_BYTES && SEND_RT <= 64 * kLdF * 4, "staging layout");
 // The chunks travel through a ring of kRing slots per unit of a launch in the
 // workspace (global memory, normally resident in L2): the producer's bulk store
 // frees its staging as soon as the bytes have been read, and the consumer
@@ -138,11 +143,12 @@ static_assert(SL_GATES == SL_RT2 + 16384 && SEND_RT <= 64 * kLdF * 4, "staging l
 // counters per ring slot, in their own 128-byte line per unit, hand the slot
 // back and forth: ready[rs] = chunks written to slot rs, freed[rs] = chunks
 // the consumer has taken out of it (chunk c uses slot c % kRing).
-constexpr int kRing = 4;
+constexpr int kRing = 8;
 constexpr uint32_t GSLOT_BYTES = SEND_QW + SEND_RT;
 static_assert(GSLOT_BYTES % 128 == 0 && kRing % 2 == 0, "ring layout");
 constexpr uint32_t kFlagWords = 32;            // per unit: ready[kRing] at 0, freed[kRing] at 16
 constexpr uint32_t kFreedAt = 16;
+static_assert(kRing <= (int)kFreedAt, "counter layout");
 // units whose rings the workspace is sized for (one launch handles at most
 // this many; more run in further launches)
 constexpr int kMaxSlots = 64;
@@ -155,8 +161,8 @@ enum {
     PB_KQ_FULL = 0, PB_KQ_TAKEN = 2, PB_KQ_EMPTY = 4, PB_D0_FULL = 7, PB_R_FULL = 9,
     PB_X1_FULL = 11, PB_DRAIN = 13, PB_STAGED = 15, PB_AF_FREE = 17,
     // consumer
-    CB_RECV_FULL = 19, CB_K_FULL = 21, CB_K_EMPTY, CB_V_FULL, CB_V_EMPTY, CB_D_EMPTY = 25,
-    CB_D_FULL = 27, CB_S_OK = 29, CB_S_FULL = 31, CB_ST_READY = 33, CB_DRAIN = 35,
+    CB_RECV_FULL = 19, CB_K_FULL = 21, CB_K_EMPTY, CB_V_FULL = 23, CB_V_EMPTY = 25, CB_SLOT_FREE = 27,
+    CB_D_FULL = 29, CB_S_FULL, CB_DRAIN, CB_E_FULL, CB_E_EMPTY, CB_E_DRAIN, CB_REL_DONE = 35,
     kNumBars = 37
 };
 constexpr uint32_t SMEM_BYTES = OFF_BARS + kNumBars * 8;
@@ -164,17 +170,27 @@ constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;           // room to align th
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget of one CTA");
 
 // TMEM columns.  Producer group g: D0 (64), R (64), X1 (128) at 256 g.
-// Consumer: D[buffer][half] at 128 buffer + 64 half, S~[half] at 256 + 64 half.
+// Consumer: D = [-W; Qh] S^T at 0, E = [U'; O'] at 128 (rows [U; o / scale] =
+// D + E, d_v columns), S~ (d_k x d_v) at 256.
 constexpr uint32_t PCOL_D0 = 0, PCOL_R = 64, PCOL_X1 = 128;
-constexpr uint32_t CCOL_S = 256;
+constexpr uint32_t CCOL_D = 0, CCOL_E = 128, CCOL_S = 256;
 constexpr uint32_t TMEM_COLS = 512;
 
 constexpr uint32_t IDESC_D0 = idesc_bf16(128, 64, false, false);
 constexpr uint32_t IDESC_R = idesc_bf16(128, 64, false, true);
 constexpr uint32_t IDESC_X1 = idesc_bf16(128, 128, false, true);
-constexpr uint32_t IDESC_X2 = idesc_bf16(128, 64, false, true);
-constexpr uint32_t IDESC_D1 = idesc_bf16(128, 64, false, true);
-constexpr uint32_t IDESC_S = idesc_bf16(128, 64, true, true);
+// consumer products over all of d_v: A K-major or MN-major, B MN-major
+constexpr uint32_t IDESC_N128_KM = idesc_bf16(128, 128, false, true);
+constexpr uint32_t IDESC_N128_MM = idesc_bf16(128, 128, true, true);
+// consumer warps: 0 TMA (V, K), 1 the [U'; O'] products, 2 ring loader and
+// TMEM allocation, then sixteen epilogue / chain product warps, then the ring
+// slot release
+constexpr int kEpiWarp0 = 3;
+constexpr int kEpiThreads = 16 * 32;
+constexpr int kRelWarp = kEpiWarp0 + kEpiThreads / 32;     // ring slot release
+static_assert(kRelWarp < kWarps, "consumer warps");
+constexpr int kEpiBar = 1;                     // named barrier of the epilogue warps
+constexpr int kOutBar = 2;                     // named barrier of their o-row half
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;    // 2 s: far beyond any legitimate wait
 constexpr float kLog2e = 1.4426950408889634f;
@@ -219,18 +235,6 @@ struct Ctx {
     TC_DEVICE uint32_t bar(int i) const { return bar0 + 8u * (uint32_t)i; }
 };
 
-// S~ <- g S~ for this thread's TMEM lane over 64 columns
-__device__ __forceinline__ void rescale_state(uint32_t taddr, float g) {
-    for (int half = 0; half < 2; ++half) {
-        float s[32];
-        tmem_ld32(taddr + half * 32, s);
-        tmem_ld_wait();
-        for (int j = 0; j < 32; ++j) s[j] *= g;
-        tmem_st32(taddr + half * 32, s);
-    }
-    tmem_st_wait();
-}
-
 // ================================================================ consumer
 __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
                                          const CUtensorMap* tm_o, const ClParams& p) {
@@ -238,19 +242,21 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
     const int nch = x.nch;
     if (warp == 0) {
         // ------------------------------------------------ TMA: V and K of each chunk
-        // One buffer each: V(c) is needed by the first product of chunk c and is
-        // free once both halves' first products of chunk c - 1 are done; K(c) by
-        // the state update at the end of chunk c.
+        // V(c) goes to buffer c & 1 (free once the [U'; O'] product of chunk
+        // c - 2 has read it), so that it lands well before that product; K(c)
+        // has one buffer, needed by the state update at the end of chunk c.
         if (lane == 0) {
             prefetch_tmap(tm_k);
             prefetch_tmap(tm_v);
             int issued = 0;
             for (int c = 0; c < nch; ++c) {
                 const int32_t y = (int32_t)(x.bos + (int64_t)c * kC);
-                if (c >= 1 && !mbar_wait(x.bar(CB_V_EMPTY), (c - 1) & 1, x.abort, kWaitLimitNs)) break;
-                mbar_arrive_expect_tx(x.bar(CB_V_FULL), 16384);
-                tma_load_2d(x.sbase + C_V, tm_v, x.h * kD, y, x.bar(CB_V_FULL));
-                tma_load_2d(x.sbase + C_V + 8192, tm_v, x.h * kD + 64, y, x.bar(CB_V_FULL));
+                const int vb = c & 1;
+                if (c >= 2 && !mbar_wait(x.bar(CB_V_EMPTY + vb), ((c >> 1) - 1) & 1, x.abort, kWaitLimitNs))
+                    break;
+                mbar_arrive_expect_tx(x.bar(CB_V_FULL + vb), 16384);
+                tma_load_2d(x.sbase + C_V + vb * 16384, tm_v, x.h * kD, y, x.bar(CB_V_FULL + vb));
+                tma_load_2d(x.sbase + C_V + vb * 16384 + 8192, tm_v, x.h * kD + 64, y, x.bar(CB_V_FULL + vb));
                 if (c >= 1 && !mbar_wait(x.bar(CB_K_EMPTY), (c - 1) & 1, x.abort, kWaitLimitNs)) {
                     issued = -(c + 1);           // V of chunk c is in flight, K is not
                     break;
@@ -263,219 +269,248 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
             // copies still in flight land before the CTA may exit
             volatile int no_abort = 0;
             const int nv = issued >= 0 ? issued : -issued, nk = issued >= 0 ? issued : -issued - 1;
-            if (nv >= 1) mbar_wait(x.bar(CB_V_FULL), (nv - 1) & 1, &no_abort, kWaitLimitNs);
+            for (int c = nv >= 2 ? nv - 2 : 0; c < nv; ++c)
+                mbar_wait(x.bar(CB_V_FULL + (c & 1)), (c >> 1) & 1, &no_abort, kWaitLimitNs);
             if (nk >= 1) mbar_wait(x.bar(CB_K_FULL), (nk - 1) & 1, &no_abort, kWaitLimitNs);
         }
-    } else if (warp == 1 || warp == 3) {
-        // ------------------------------------------------ MMA issuer of one d_v half
-        const int hh = warp >> 1;
+    } else if (warp == 1) {
+        // ------------------------------------------------ [U'; O'] = [T b; R b] V per chunk
+        // State-independent, so it runs ahead of the chain into its own
+        // accumulator E, once the epilogues have read the previous chunk's E.
+        if (lane == 0) {
+            const uint64_t dsc_rt0 = sdesc_sw128(x.sbase + C_RECV + SL_RT2, 16, 1024);
+            const uint64_t dsc_v = sdesc_sw128(x.sbase + C_V, 8192, 1024);
+            for (int c = 0; c < nch; ++c) {
+                const int b = c & 1;
+                if (!mbar_wait(x.bar(CB_RECV_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs)) break;
+                if (!mbar_wait(x.bar(CB_V_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs)) break;
+                if (c >= 1 && !mbar_wait(x.bar(CB_E_EMPTY), (c - 1) & 1, x.abort, kWaitLimitNs)) break;
+                tc_fence_after();
+                const uint64_t a = dsc_rt0 + b * (uint64_t)(SLOT_BYTES >> 4);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(x.tmem + CCOL_E, a + kk * 2, dsc_v + b * (16384 >> 4) + kk * 128, IDESC_N128_KM,
+                             kk > 0);
+                mma_commit(x.bar(CB_E_FULL));
+                mma_commit(x.bar(CB_V_EMPTY + b));
+            }
+            volatile int no_abort = 0;
+            mma_commit(x.bar(CB_E_DRAIN));
+            mbar_wait(x.bar(CB_E_DRAIN), 0, &no_abort, kWaitLimitNs);
+        }
+    } else if (warp == kRelWarp) {
+        // ------------------------------------------------ ring slots back to the producers
+        // Chunk c's ring slot is free once its bulk load into the receive slot
+        // has completed.  This thread issues no copies of its own, so its
+        // release store does not wait for the loader's copies in flight (and a
+        // warp of its own keeps its waits from holding up another role).  The
+        // loader reuses receive slot c & 1 for chunk c + 2 only after REL_DONE,
+        // so this wait never falls two phases behind.
         if (lane == 0) {
             for (int c = 0; c < nch; ++c) {
                 const int b = c & 1;
-                const uint32_t slot = x.sbase + C_RECV + b * SLOT_BYTES;
-                const uint32_t dcol = x.tmem + b * 128 + hh * 64;
                 if (!mbar_wait(x.bar(CB_RECV_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs)) break;
-                if (!mbar_wait(x.bar(CB_V_FULL), c & 1, x.abort, kWaitLimitNs)) break;
-                // D[b] was last read by the epilogues of chunk c - 2
-                if (c >= 2 && !mbar_wait(x.bar(CB_D_EMPTY + b), ((c >> 1) - 1) & 1, x.abort, kWaitLimitNs))
-                    break;
-                fence_async_smem();
-                tc_fence_after();
-                // [U'; O'] = [T b; R b] V_half
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(dcol, desc_kmajor_1panel(slot + SL_RT2, kk),
-                             desc_mnmajor(x.sbase + C_V + hh * 8192, kk, 8192), IDESC_X2, kk > 0);
-                mma_commit(x.bar(CB_V_EMPTY));
-                // += [-W; Qh] S_half^T  ->  [U; o / scale]
-                if (!mbar_wait(x.bar(CB_ST_READY + hh), c & 1, x.abort, kWaitLimitNs)) break;
-                tc_fence_after();
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(dcol, desc_kmajor_2panel(slot + SL_QW, kk),
-                             desc_mnmajor(x.sbase + C_ST + hh * 16384, kk, 16384), IDESC_D1, 1);
-                mma_commit(x.bar(CB_D_FULL + hh));
-                // S~_half += K^T (kappa U / Gamma)
-                if (!mbar_wait(x.bar(CB_S_OK + hh), c & 1, x.abort, kWaitLimitNs)) break;
-                if (!mbar_wait(x.bar(CB_K_FULL), c & 1, x.abort, kWaitLimitNs)) break;
-                tc_fence_after();
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(x.tmem + CCOL_S + hh * 64, desc_mnmajor(x.sbase + C_K, kk, 8192),
-                             desc_mnmajor(x.sbase + C_UK + hh * 8192, kk, 8192), IDESC_S, 1);
-                mma_commit(x.bar(CB_S_FULL + hh));
-                mma_commit(x.bar(CB_K_EMPTY));
+                fence_async_global();
+                st_release_gpu(x.freed + c % kRing, (uint32_t)(c / kRing + 1));
+                mbar_arrive(x.bar(CB_REL_DONE + b));
             }
-            volatile int no_abort = 0;
-            mma_commit(x.bar(CB_DRAIN + hh));
-            mbar_wait(x.bar(CB_DRAIN + hh), 0, &no_abort, kWaitLimitNs);
         }
     } else if (warp == 2) {
         // ------------------------------------------------ loader: ring slot -> receive slot
-        // Chunk c sits in ring slot c % kRing.  A slot is handed back once its
-        // chunk has been loaded (checked one chunk later, so that loads overlap).
+        // Chunk c sits in ring slot c % kRing and goes to receive slot c & 1,
+        // which is free once the epilogues of chunk c - 2 are done with it and
+        // its ring slot has been handed back (warp kRelWarp).  The loader never
+        // waits for its own copies.
         if (lane == 0) {
-            auto ring_free = [&](int c) {
-                // the bulk load of chunk c has completed (its barrier was seen)
-                fence_async_global();
-                st_release_gpu(x.freed + c % kRing, (uint32_t)(c / kRing + 1));
-            };
             int loaded = 0;
             for (int c = 0; c < nch; ++c) {
                 const int b = c & 1, rs = c % kRing;
-                if (c >= 2 && !mbar_wait(x.bar(CB_D_EMPTY + b), ((c >> 1) - 1) & 1, x.abort, kWaitLimitNs))
-                    break;
                 if (!gflag_wait_ge(x.ready + rs, (uint32_t)(c / kRing + 1), x.abort, x.err, kWaitLimitNs))
+                    break;
+                if (c >= 2 && (!mbar_wait(x.bar(CB_SLOT_FREE + b), ((c >> 1) - 1) & 1, x.abort, kWaitLimitNs) ||
+                               !mbar_wait(x.bar(CB_REL_DONE + b), ((c >> 1) - 1) & 1, x.abort, kWaitLimitNs)))
                     break;
                 fence_async_global();
                 const uint32_t slot = x.sbase + C_RECV + b * SLOT_BYTES;
                 const uint8_t* g = x.ring + (size_t)rs * GSLOT_BYTES;
                 mbar_arrive_expect_tx(x.bar(CB_RECV_FULL + b), GSLOT_BYTES);
                 bulk_load(slot + SL_QW, g, SEND_QW, x.bar(CB_RECV_FULL + b));
-                bulk_load(slot + SL_RT2, g + SEND_QW, SEND_RT, x.bar(CB_RECV_FULL + b));
+                bulk_load(slot + SL_RT2, g + SEND_QW, GATES_AT, x.bar(CB_RECV_FULL + b));
+                bulk_load(x.sbase + C_GATES + b * GATE_BYTES, g + SEND_QW + GATES_AT, GATE_BYTES,
+                          x.bar(CB_RECV_FULL + b));
                 loaded = c + 1;
-                if (c >= 1) {
-                    if (!mbar_wait(x.bar(CB_RECV_FULL + ((c - 1) & 1)), ((c - 1) >> 1) & 1, x.abort, kWaitLimitNs))
-                        break;
-                    ring_free(c - 1);
-                }
             }
             // loads still in flight land before the CTA may exit
             volatile int no_abort = 0;
             for (int c = loaded >= 2 ? loaded - 2 : 0; c < loaded; ++c)
                 mbar_wait(x.bar(CB_RECV_FULL + (c & 1)), (c >> 1) & 1, &no_abort, kWaitLimitNs);
         }
-    } else if (warp >= 4 && warp < 12) {
-        // ------------------------------------------------ epilogues of one d_v half
+    } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kEpiThreads / 32) {
+        // ------------------------------------------------ products and epilogues
+        // Sixteen warps: warp w reads TMEM lane quadrant w % 4 (the hardware
+        // rule) and columns 32 cb .. 32 cb + 31, cb = (w - kEpiWarp0) / 4, of
+        // the 128-column accumulators; thread = one row.  Lane 0 of one of
+        // them issues every tensor-core product itself, right after the
+        // group's named barrier, so that no other warp sits between an epilogue
+        // and the next product of the state chain.  Each product covers all
+        // 128 columns of d_v in one instruction per 16-deep K step (a
+        // tcgen05.mma costs about the same to issue at N = 64 as at N = 128).
+        // After an abort the waits fall through and the issuer skips its
+        // products, but every thread still passes every named barrier.
         const int q = warp & 3;                    // TMEM lane quadrant
-        const int hh = (warp - 4) >> 2;            // d_v half
+        const int cb = (warp - kEpiWarp0) >> 2;    // 32-column block
         const int r = q * 32 + lane;               // TMEM lane = row
+        // the issuer reads a U row (quadrant 0), so it has no o rows to write out
+        const bool issuer = (warp == kEpiWarp0 + 1 && lane == 0);
         const uint32_t tl = x.tmem + ((uint32_t)(q * 32) << 16);
-        const uint32_t scol = CCOL_S + hh * 64;
+        const uint32_t dcol = CCOL_D + cb * 32, ecol = CCOL_E + cb * 32, scol = CCOL_S + cb * 32;
+        const int hh = cb >> 1, ch0 = (cb & 1) * 4;   // d_v half and first 16-byte chunk in it
         uint8_t* st_tile = x.sm + C_ST + hh * 16384;
         uint8_t* uk_tile = x.sm + C_UK + hh * 8192;
-        // initial state: thread r holds d_k row r of S^T over this half's 64 v-columns
+        // shared-memory descriptors, computed once; a K step adds a byte offset
+        // (>> 4) to the start address field
+        const uint64_t dsc_qw0 = sdesc_sw128(x.sbase + C_RECV + SL_QW, 16, 1024);
+        const uint64_t dsc_st = sdesc_sw128(x.sbase + C_ST, 16384, 1024);
+        const uint64_t dsc_k = sdesc_sw128(x.sbase + C_K, 8192, 1024);
+        const uint64_t dsc_uk = sdesc_sw128(x.sbase + C_UK, 8192, 1024);
+        constexpr uint64_t kSlotStep = SLOT_BYTES >> 4;
+        // initial state: thread r holds d_k row r of S^T over 32 v-columns
         {
-            float s[32];
-            for (int half = 0; half < 2; ++half) {
-                for (int j = 0; j < 32; ++j) {
-                    const int vcol = hh * 64 + half * 32 + j;
-                    s[j] = p.s_in ? p.s_in[x.state_off + (int64_t)vcol * kD + r] : 0.f;
-                }
-                tmem_st32(tl + scol + half * 32, s);
-                for (int j = 0; j < 4; ++j) st_bf16x8(st_tile, r, half * 4 + j, s + 8 * j);
+            float sv[32];
+            for (int j = 0; j < 32; ++j) {
+                const int vcol = cb * 32 + j;
+                sv[j] = p.s_in ? p.s_in[x.state_off + (int64_t)vcol * kD + r] : 0.f;
             }
+            tmem_st32(tl + scol, sv);
+            for (int j = 0; j < 4; ++j) st_bf16x8(st_tile, r, ch0 + j, sv + 8 * j);
             tmem_st_wait();
             fence_async_smem();
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(x.bar(CB_ST_READY + hh));
+            named_bar_sync(kEpiBar, kEpiThreads);
         }
         float Gam = 1.f;                           // S = Gam * S~ (same value in every thread)
         for (int c = 0; c < nch; ++c) {
             const int b = c & 1;
-            const float* kap = reinterpret_cast<const float*>(x.sm + C_RECV + b * SLOT_BYTES + SL_GATES);
+            const float* kap = reinterpret_cast<const float*>(x.sm + C_GATES + b * GATE_BYTES);
             const int64_t tok0 = x.bos + (int64_t)c * kC;
-            const uint32_t dcol = b * 128 + hh * 64;
+            // ---- [U; o / scale] = [U'; O'] + [-W; Qh] S^T: the second term here, the
+            //      first (E) from warp 1
+            if (issuer && !*x.abort &&
+                mbar_wait(x.bar(CB_RECV_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs)) {
+                tc_fence_after();
+                const uint64_t a = dsc_qw0 + b * kSlotStep;
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(x.tmem + CCOL_D, a + (((kk >> 2) * KQ_PANEL + (kk & 3) * 32) >> 4),
+                             dsc_st + kk * 128, IDESC_N128_KM, kk > 0);
+                mma_commit(x.bar(CB_D_FULL));
+            }
             mbar_wait(x.bar(CB_RECV_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs);
-            mbar_wait(x.bar(CB_D_FULL + hh), c & 1, x.abort, kWaitLimitNs);
+            mbar_wait(x.bar(CB_E_FULL), c & 1, x.abort, kWaitLimitNs);
+            mbar_wait(x.bar(CB_D_FULL), c & 1, x.abort, kWaitLimitNs);
             tc_fence_after();
             const float Gn = Gam * kap[64];        // scale of the state after this chunk
             const bool resc = !(Gn >= kMinGamma);
             const float inv = resc ? 1.f : 1.f / Gn;
-            if (q < 2) {
-                // rows 0-63 hold U_t: write kappa_t U_t / Gamma as the update operand
-                const int t = r;
-                const float sc = kap[t] * inv;
-                float u[2][32];
-                tmem_ld32x2(tl + dcol, tl + dcol + 32, u[0], u[1]);
-                for (int half = 0; half < 2; ++half) {
-                    for (int j = 0; j < 32; ++j) u[half][j] *= sc;
-                    for (int j = 0; j < 4; ++j) st_bf16x8(uk_tile, t, half * 4 + j, u[half] + 8 * j);
+            // rows 0-63 (q < 2) hold U_t: kappa_t U_t / Gamma becomes the update
+            // operand, written before the barrier.  Rows 64-127 hold o_t / scale:
+            // kept in registers and written out after the barrier, while the
+            // state update runs.
+            float ov[32];
+            {
+                float e[32];
+                tmem_ld32x2(tl + dcol, tl + ecol, ov, e);
+                for (int j = 0; j < 32; ++j) ov[j] += e[j];
+                if (q < 2) {
+                    const float sc = kap[r] * inv;
+                    for (int j = 0; j < 32; ++j) e[j] = ov[j] * sc;
+                    for (int j = 0; j < 4; ++j) st_bf16x8(uk_tile, r, ch0 + j, e + 8 * j);
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(x.bar(CB_D_EMPTY + b));
-                if (resc) rescale_state(tl + scol, Gn);
-                fence_async_smem();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(x.bar(CB_S_OK + hh));
-            } else {
-                // rows 64-127 hold o_t / scale.  The state update does not touch
-                // these columns, so it may start before o is written.
-                if (resc) rescale_state(tl + scol, Gn);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(x.bar(CB_S_OK + hh));
+            }
+            if (resc) {
+                // S~ <- Gn S~ on this thread's 32 columns (Gamma restarts at 1)
+                float sv[32];
+                tmem_ld32(tl + scol, sv);
+                tmem_ld_wait();
+                for (int j = 0; j < 32; ++j) sv[j] *= Gn;
+                tmem_st32(tl + scol, sv);
+                tmem_st_wait();
+            }
+            fence_async_smem();
+            tc_fence_before();
+            named_bar_sync(kEpiBar, kEpiThreads);
+            if (issuer) {
+                // D, E and the receive slot's gates have been read by every thread
+                mbar_arrive(x.bar(CB_SLOT_FREE + b));
+                // ---- S~ += K^T (kappa U / Gamma)
+                if (!*x.abort && mbar_wait(x.bar(CB_K_FULL), c & 1, x.abort, kWaitLimitNs)) {
+                    tc_fence_after();
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_bf16(x.tmem + CCOL_S, dsc_k + kk * 128, dsc_uk + kk * 128, IDESC_N128_MM, 1);
+                    mma_commit(x.bar(CB_S_FULL));
+                    mma_commit(x.bar(CB_K_EMPTY));
+                }
+                // E may be overwritten now; the next [U'; O'] product is issued (by
+                // warp 1) only after this chunk's state update, so that it does
+                // not slow down the issue of the chain's products
+                mbar_arrive(x.bar(CB_E_EMPTY));
+            }
+            if (q >= 2) {
+                // o rows, while the state update runs.  A whole chunk is staged
+                // (four 32-column boxes, 128-byte swizzle) and written by TMA; the
+                // ragged end of a sequence is stored directly (rows past its end
+                // belong to the next sequence).
                 const int t = r - 64;
-                float ov[2][32];
-                tmem_ld32x2(tl + dcol, tl + dcol + 32, ov[0], ov[1]);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(x.bar(CB_D_EMPTY + b));
+                const bool elected = (warp == kEpiWarp0 + 3 && lane == 0);
                 if (tok0 + kC <= x.eos) {
-                    // whole chunk: stage the 64 x 64 tile (two 32-column boxes, 128-byte
-                    // swizzle) and store it with TMA.  The staging was last read by the
-                    // previous chunk's store.
-                    const bool elected = (q == 2 && lane == 0);
-                    if (elected) bulk_wait_read();
-                    named_bar_sync(5 + hh, 64);
-                    uint8_t* ost = x.sm + C_OST + hh * 16384;
-                    for (int bx = 0; bx < 2; ++bx) {
-                        for (int j = 0; j < 8; ++j) {
-                            float4 w;
-                            w.x = p.scale * ov[bx][4 * j];
-                            w.y = p.scale * ov[bx][4 * j + 1];
-                            w.z = p.scale * ov[bx][4 * j + 2];
-                            w.w = p.scale * ov[bx][4 * j + 3];
-                            *reinterpret_cast<float4*>(ost + bx * 8192 + sw128_off(t, j)) = w;
-                        }
-                    }
+                    uint8_t* ost = x.sm + C_OST + cb * 8192;
+                    if (elected) bulk_wait_read();      // the previous chunk's stores have read the staging
+                    named_bar_sync(kOutBar, kEpiThreads / 2);
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<float4*>(ost + sw128_off(t, j)) =
+                            make_float4(p.scale * ov[4 * j], p.scale * ov[4 * j + 1], p.scale * ov[4 * j + 2],
+                                        p.scale * ov[4 * j + 3]);
                     fence_async_smem();
-                    named_bar_sync(5 + hh, 64);
+                    named_bar_sync(kOutBar, kEpiThreads / 2);
                     if (elected) {
-                        for (int bx = 0; bx < 2; ++bx)
-                            tma_store_2d(tm_o, x.h * kD + hh * 64 + bx * 32, (int32_t)tok0,
-                                         x.sbase + C_OST + hh * 16384 + bx * 8192);
+                        for (int bx = 0; bx < 4; ++bx)
+                            tma_store_2d(tm_o, x.h * kD + bx * 32, (int32_t)tok0, x.sbase + C_OST + bx * 8192);
                         bulk_commit();
                     }
                 } else if (tok0 + t < x.eos) {
-                    // the ragged end of a sequence: rows past its end belong to the next one
-                    float* orow = p.o + ((tok0 + t) * p.Hv + x.h) * kD + hh * 64;
-                    for (int bx = 0; bx < 2; ++bx)
-                        for (int j = 0; j < 32; j += 4) {
-                            float4 w;
-                            w.x = p.scale * ov[bx][j];
-                            w.y = p.scale * ov[bx][j + 1];
-                            w.z = p.scale * ov[bx][j + 2];
-                            w.w = p.scale * ov[bx][j + 3];
-                            *reinterpret_cast<float4*>(orow + bx * 32 + j) = w;
-                        }
+                    float* orow = p.o + ((tok0 + t) * p.Hv + x.h) * kD + cb * 32;
+                    for (int j = 0; j < 32; j += 4)
+                        *reinterpret_cast<float4*>(orow + j) =
+                            make_float4(p.scale * ov[j], p.scale * ov[j + 1], p.scale * ov[j + 2], p.scale * ov[j + 3]);
                 }
             }
             Gam = resc ? 1.f : Gn;
-            // new state -> bf16 operand of the next chunk (and the final state)
-            mbar_wait(x.bar(CB_S_FULL + hh), c & 1, x.abort, kWaitLimitNs);
+            // ---- new state -> bf16 operand of the next chunk (and the final state)
+            mbar_wait(x.bar(CB_S_FULL), c & 1, x.abort, kWaitLimitNs);
             tc_fence_after();
             const bool last = (c == nch - 1);
-            float sv[2][32];
-            tmem_ld32x2(tl + scol, tl + scol + 32, sv[0], sv[1]);
-            for (int half = 0; half < 2; ++half) {
-                float* s = sv[half];
-                for (int j = 0; j < 32; ++j) s[j] *= Gam;
+            {
+                float sv[32];
+                tmem_ld32(tl + scol, sv);
+                tmem_ld_wait();
+                for (int j = 0; j < 32; ++j) sv[j] *= Gam;
                 if (!last) {
-                    for (int j = 0; j < 4; ++j) st_bf16x8(st_tile, r, half * 4 + j, s + 8 * j);
+                    for (int j = 0; j < 4; ++j) st_bf16x8(st_tile, r, ch0 + j, sv + 8 * j);
                 } else if (p.s_out) {
                     for (int j = 0; j < 32; ++j)
-                        p.s_out[x.state_off + (int64_t)(hh * 64 + half * 32 + j) * kD + r] = s[j];
+                        p.s_out[x.state_off + (int64_t)(cb * 32 + j) * kD + r] = sv[j];
                 }
             }
             if (!last) {
                 fence_async_smem();
                 tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(x.bar(CB_ST_READY + hh));
+                named_bar_sync(kEpiBar, kEpiThreads);
             }
         }
-        if (q == 2 && lane == 0) bulk_wait();      // this half's last o stores are complete
+        if (issuer) {
+            volatile int no_abort = 0;
+            mma_commit(x.bar(CB_DRAIN));
+            mbar_wait(x.bar(CB_DRAIN), 0, &no_abort, kWaitLimitNs);
+        }
+        if (warp == kEpiWarp0 + 3 && lane == 0) bulk_wait();     // the last o stores are complete
     }
 }
 
@@ -809,7 +844,7 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
                 st_bf16x8(stage_rt, row2, hh * 4 + j8, wb);
             }
             if (q < 2 && hh == 0) {
-                float* sg = reinterpret_cast<float*>(stage_rt + (SL_GATES - SL_RT2));
+                float* sg = reinterpret_cast<float*>(stage_rt + GATES_AT);
                 sg[i_] = gb.kappa[i_];
                 if (i_ == 63) sg[64] = gb.gC;
             }
@@ -922,19 +957,21 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (rank == 0) {
             for (int b = 0; b < 2; ++b) {
                 mbar_init(x.bar(CB_RECV_FULL + b), 1);
-                mbar_init(x.bar(CB_D_EMPTY + b), 8);
+                mbar_init(x.bar(CB_SLOT_FREE + b), 1);
+                mbar_init(x.bar(CB_REL_DONE + b), 1);
             }
             mbar_init(x.bar(CB_K_FULL), 1);
-            mbar_init(x.bar(CB_K_EMPTY), 2);
-            mbar_init(x.bar(CB_V_FULL), 1);
-            mbar_init(x.bar(CB_V_EMPTY), 2);
-            for (int hh = 0; hh < 2; ++hh) {
-                mbar_init(x.bar(CB_D_FULL + hh), 1);
-                mbar_init(x.bar(CB_S_OK + hh), 4);
-                mbar_init(x.bar(CB_S_FULL + hh), 1);
-                mbar_init(x.bar(CB_ST_READY + hh), 4);
-                mbar_init(x.bar(CB_DRAIN + hh), 1);
+            mbar_init(x.bar(CB_K_EMPTY), 1);
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(x.bar(CB_V_FULL + b), 1);
+                mbar_init(x.bar(CB_V_EMPTY + b), 1);
             }
+            mbar_init(x.bar(CB_D_FULL), 1);
+            mbar_init(x.bar(CB_S_FULL), 1);
+            mbar_init(x.bar(CB_DRAIN), 1);
+            mbar_init(x.bar(CB_E_FULL), 1);
+            mbar_init(x.bar(CB_E_EMPTY), 1);
+            mbar_init(x.bar(CB_E_DRAIN), 1);
         } else {
             for (int s = 0; s < kKqStages; ++s) mbar_init(x.bar(PB_KQ_EMPTY + s), 1);
             for (int grp = 0; grp < 2; ++grp) {
