@@ -73,6 +73,18 @@
 
 namespace gdn {
 
+// Per-chunk timestamps of one (sequence, value head) unit for latency analysis,
+// compiled in only with -DGDN_PREFILL_TRACE (off in every normal build):
+// TRACE_CLK(ev, c) records clock64() of event ev for chunk c.
+#ifdef GDN_PREFILL_TRACE
+__device__ long long g_prefill_trace[40][4096];
+__device__ int g_prefill_trace_unit = -1;
+#define TRACE_CLK(ev, c) \
+    do { if (x.traced) g_prefill_trace[ev][(c) & 4095] = clock64(); } while (0)
+#else
+#define TRACE_CLK(ev, c) do { } while (0)
+#endif
+
 namespace {
 
 using namespace tc;
@@ -232,6 +244,7 @@ struct Ctx {
     int nch;
     int64_t state_off;
     uint32_t bar0;         // shared address of barrier 0
+    int traced;            // this unit's events are recorded (tracing builds only)
     TC_DEVICE uint32_t bar(int i) const { return bar0 + 8u * (uint32_t)i; }
 };
 
@@ -254,6 +267,7 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
                 const int vb = c & 1;
                 if (c >= 2 && !mbar_wait(x.bar(CB_V_EMPTY + vb), ((c >> 1) - 1) & 1, x.abort, kWaitLimitNs))
                     break;
+                TRACE_CLK(28, c);
                 mbar_arrive_expect_tx(x.bar(CB_V_FULL + vb), 16384);
                 tma_load_2d(x.sbase + C_V + vb * 16384, tm_v, x.h * kD, y, x.bar(CB_V_FULL + vb));
                 tma_load_2d(x.sbase + C_V + vb * 16384 + 8192, tm_v, x.h * kD + 64, y, x.bar(CB_V_FULL + vb));
@@ -261,6 +275,7 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
                     issued = -(c + 1);           // V of chunk c is in flight, K is not
                     break;
                 }
+                TRACE_CLK(29, c);
                 mbar_arrive_expect_tx(x.bar(CB_K_FULL), 16384);
                 tma_load_2d(x.sbase + C_K, tm_k, x.g * kD, y, x.bar(CB_K_FULL));
                 tma_load_2d(x.sbase + C_K + 8192, tm_k, x.g * kD + 64, y, x.bar(CB_K_FULL));
@@ -285,6 +300,7 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
                 if (!mbar_wait(x.bar(CB_RECV_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs)) break;
                 if (!mbar_wait(x.bar(CB_V_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs)) break;
                 if (c >= 1 && !mbar_wait(x.bar(CB_E_EMPTY), (c - 1) & 1, x.abort, kWaitLimitNs)) break;
+                TRACE_CLK(14, c);
                 tc_fence_after();
                 const uint64_t a = dsc_rt0 + b * (uint64_t)(SLOT_BYTES >> 4);
                 for (int kk = 0; kk < 4; ++kk)
@@ -292,6 +308,7 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
                              kk > 0);
                 mma_commit(x.bar(CB_E_FULL));
                 mma_commit(x.bar(CB_V_EMPTY + b));
+                TRACE_CLK(15, c);
             }
             volatile int no_abort = 0;
             mma_commit(x.bar(CB_E_DRAIN));
@@ -312,6 +329,7 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
                 fence_async_global();
                 st_release_gpu(x.freed + c % kRing, (uint32_t)(c / kRing + 1));
                 mbar_arrive(x.bar(CB_REL_DONE + b));
+                TRACE_CLK(13, c);
             }
         }
     } else if (warp == 2) {
@@ -324,8 +342,10 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
             int loaded = 0;
             for (int c = 0; c < nch; ++c) {
                 const int b = c & 1, rs = c % kRing;
+                TRACE_CLK(10, c);
                 if (!gflag_wait_ge(x.ready + rs, (uint32_t)(c / kRing + 1), x.abort, x.err, kWaitLimitNs))
                     break;
+                TRACE_CLK(11, c);
                 if (c >= 2 && (!mbar_wait(x.bar(CB_SLOT_FREE + b), ((c >> 1) - 1) & 1, x.abort, kWaitLimitNs) ||
                                !mbar_wait(x.bar(CB_REL_DONE + b), ((c >> 1) - 1) & 1, x.abort, kWaitLimitNs)))
                     break;
@@ -338,6 +358,7 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
                 bulk_load(x.sbase + C_GATES + b * GATE_BYTES, g + SEND_QW + GATES_AT, GATE_BYTES,
                           x.bar(CB_RECV_FULL + b));
                 loaded = c + 1;
+                TRACE_CLK(12, c);
             }
             // loads still in flight land before the CTA may exit
             volatile int no_abort = 0;
@@ -402,10 +423,13 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
                     mma_bf16(x.tmem + CCOL_D, a + (((kk >> 2) * KQ_PANEL + (kk & 3) * 32) >> 4),
                              dsc_st + kk * 128, IDESC_N128_KM, kk > 0);
                 mma_commit(x.bar(CB_D_FULL));
+                TRACE_CLK(0, c);
             }
             mbar_wait(x.bar(CB_RECV_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs);
             mbar_wait(x.bar(CB_E_FULL), c & 1, x.abort, kWaitLimitNs);
+            if (issuer) TRACE_CLK(1, c);
             mbar_wait(x.bar(CB_D_FULL), c & 1, x.abort, kWaitLimitNs);
+            if (issuer) TRACE_CLK(2, c);
             tc_fence_after();
             const float Gn = Gam * kap[64];        // scale of the state after this chunk
             const bool resc = !(Gn >= kMinGamma);
@@ -436,12 +460,15 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
             }
             fence_async_smem();
             tc_fence_before();
+            if (issuer) TRACE_CLK(3, c);
             named_bar_sync(kEpiBar, kEpiThreads);
+            if (issuer) TRACE_CLK(4, c);
             if (issuer) {
                 // D, E and the receive slot's gates have been read by every thread
                 mbar_arrive(x.bar(CB_SLOT_FREE + b));
                 // ---- S~ += K^T (kappa U / Gamma)
                 if (!*x.abort && mbar_wait(x.bar(CB_K_FULL), c & 1, x.abort, kWaitLimitNs)) {
+                    TRACE_CLK(27, c);
                     tc_fence_after();
                     for (int kk = 0; kk < 4; ++kk)
                         mma_bf16(x.tmem + CCOL_S, dsc_k + kk * 128, dsc_uk + kk * 128, IDESC_N128_MM, 1);
@@ -452,6 +479,7 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
                 // warp 1) only after this chunk's state update, so that it does
                 // not slow down the issue of the chain's products
                 mbar_arrive(x.bar(CB_E_EMPTY));
+                TRACE_CLK(5, c);
             }
             if (q >= 2) {
                 // o rows, while the state update runs.  A whole chunk is staged
@@ -484,7 +512,9 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
             }
             Gam = resc ? 1.f : Gn;
             // ---- new state -> bf16 operand of the next chunk (and the final state)
+            if (issuer) TRACE_CLK(6, c);
             mbar_wait(x.bar(CB_S_FULL), c & 1, x.abort, kWaitLimitNs);
+            if (issuer) TRACE_CLK(7, c);
             tc_fence_after();
             const bool last = (c == nch - 1);
             {
@@ -502,7 +532,9 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
             if (!last) {
                 fence_async_smem();
                 tc_fence_before();
+                if (issuer) TRACE_CLK(8, c);
                 named_bar_sync(kEpiBar, kEpiThreads);
+                if (issuer) TRACE_CLK(9, c);
             }
         }
         if (issuer) {
@@ -580,9 +612,11 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
                 if (c >= nch) break;
                 const int rs = c % kRing;
                 if (!mbar_wait(x.bar(PB_STAGED + grp), jj & 1, x.abort, kWaitLimitNs)) break;
+                TRACE_CLK(24, c);
                 if (c >= kRing &&
                     !gflag_wait_ge(x.freed + rs, (uint32_t)(c / kRing), x.abort, x.err, kWaitLimitNs))
                     break;
+                TRACE_CLK(25, c);
                 fence_async_global();
                 uint8_t* g = x.ring + (size_t)rs * GSLOT_BYTES;
                 bulk_store(g, x.sbase + P_KQ + (i % kKqStages) * KQ_STAGE, SEND_QW);
@@ -594,6 +628,7 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
                 bulk_wait();
                 fence_async_global();
                 st_release_gpu(x.ready + rs, (uint32_t)(c / kRing + 1));
+                TRACE_CLK(26, c);
             }
         }
         return;
@@ -631,7 +666,9 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
         const uint32_t kq = x.sbase + kqo;
         // every warp of the group has seen chunk i land before the TMA warp may
         // arm this group's barrier again
+        if (pw == 0 && lane == 0) TRACE_CLK(16, c);
         mbar_wait(x.bar(PB_KQ_FULL + grp), jj & 1, x.abort, kWaitLimitNs);
+        if (pw == 0 && lane == 0) TRACE_CLK(17, c);
         __syncwarp();
         if (lane == 0) mbar_arrive(x.bar(PB_KQ_TAKEN + grp));
         if (issuer) {
@@ -680,7 +717,9 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
         // ---- D0 rows -> A (f32 scratch) and P (bf16 operand); each warp 32 columns.
         //      The A scratch last held the previous chunk's staged bytes.
         if (jj >= 1) mbar_wait(x.bar(PB_AF_FREE + grp), (jj - 1) & 1, x.abort, kWaitLimitNs);
+        if (pw == 0 && lane == 0) TRACE_CLK(18, c);
         mbar_wait(x.bar(PB_D0_FULL + grp), jj & 1, x.abort, kWaitLimitNs);
+        if (pw == 0 && lane == 0) TRACE_CLK(19, c);
         tc_fence_after();
         {
             const bool fast = gb.fast != 0;
@@ -787,6 +826,7 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
             frag_c_store(Tf, kLdF, 32 + 16 * mt, 8 * nt, cfr, -1.f, lane);
         }
         named_bar_sync(nb, kGroupThreads);
+        if (pw == 0 && lane == 0) TRACE_CLK(20, c);
         // ---- T (bf16) as the B operand of R = P T
         for (int u = pt; u < 64 * 8; u += kGroupThreads) {
             const int row = u >> 3, chunk = u & 7;
@@ -809,6 +849,7 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
         // ---- [R bg; T bg] (over P | T once R is done) and, staged for sending,
         //      [T b; R b] with the gates (over A, which the solve no longer needs)
         mbar_wait(x.bar(PB_R_FULL + grp), jj & 1, x.abort, kWaitLimitNs);
+        if (pw == 0 && lane == 0) TRACE_CLK(21, c);
         tc_fence_after();
         {
             const int i_ = (q & 1) * 32 + lane;
@@ -862,6 +903,7 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
         }
         __syncwarp();
         mbar_wait(x.bar(PB_X1_FULL + grp), jj & 1, x.abort, kWaitLimitNs);
+        if (pw == 0 && lane == 0) TRACE_CLK(22, c);
         tc_fence_after();
         // ---- -W over the K rows and Qh = diag(gamma) Q - P W over the Q rows of the
         //      [K; Q] stage (each thread rewrites the Q chunks it has just read)
@@ -898,6 +940,7 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(x.bar(PB_STAGED + grp));
+        if (pw == 0 && lane == 0) TRACE_CLK(23, c);
     }
     if (issuer) {
         volatile int no_abort = 0;
@@ -939,6 +982,11 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     x.nch = (int)((x.eos - x.bos + kC - 1) / kC);
     x.state_off = ((int64_t)n * p.Hv + x.h) * kD * kD;
     x.ring = p.ring + (size_t)slot * kRing * GSLOT_BYTES;
+#ifdef GDN_PREFILL_TRACE
+    x.traced = (unit == g_prefill_trace_unit);
+#else
+    x.traced = 0;
+#endif
     x.ready = p.flags + (size_t)slot * kFlagWords;
     x.freed = x.ready + kFreedAt;
     x.err = p.err;
@@ -1207,3 +1255,12 @@ cudaError_t launch_prefill_pc(const PrefillArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace gdn
+
+#ifdef GDN_PREFILL_TRACE
+// tracing builds only: read the recorded events and choose the unit to record
+extern "C" int gdn_prefill_trace_read(void* host, int next_unit) {
+    int e = (int)cudaMemcpyFromSymbol(host, gdn::g_prefill_trace, sizeof(gdn::g_prefill_trace));
+    if (e) return e;
+    return (int)cudaMemcpyToSymbol(gdn::g_prefill_trace_unit, &next_unit, sizeof(int));
+}
+#endif
