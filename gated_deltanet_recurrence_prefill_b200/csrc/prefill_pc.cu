@@ -35,8 +35,8 @@
 // second counter per ring slot).  Each product spans all 128 columns of d_v
 // (a tcgen05.mma takes about as long to issue at N = 64 as at N = 128, and one
 // thread issues one every ~75 cycles at best):
-//   E  = [T b; R b] V                      M128 N128 K64   (warp 1, ahead of the chain)
-//   D  = [-W; Qh] S^T                      M128 N128 K128  -> [U; o / scale] = D + E
+//   D  = [T b; R b] V                      M128 N128 K64   (warp 1, during the epilogue before)
+//   D += [-W; Qh] S^T                      M128 N128 K128  -> [U; o / scale]
 //   S~ += K^T (kappa U / Gamma)            M128 N128 K64   (accumulates in TMEM)
 // The last two are the state chain; lane 0 of the first epilogue warp issues
 // them right after the epilogue warps' named barrier.  The float32 state lives
@@ -174,18 +174,18 @@ enum {
     PB_X1_FULL = 11, PB_DRAIN = 13, PB_STAGED = 15, PB_AF_FREE = 17,
     // consumer
     CB_RECV_FULL = 19, CB_K_FULL = 21, CB_K_EMPTY, CB_V_FULL = 23, CB_V_EMPTY = 25, CB_SLOT_FREE = 27,
-    CB_D_FULL = 29, CB_S_FULL, CB_DRAIN, CB_E_FULL, CB_E_EMPTY, CB_E_DRAIN, CB_REL_DONE = 35,
-    kNumBars = 37
+    CB_D_FULL = 29, CB_S_FULL, CB_DRAIN, CB_E_FULL, CB_E_DRAIN, CB_REL_DONE = 34,
+    kNumBars = 36
 };
 constexpr uint32_t SMEM_BYTES = OFF_BARS + kNumBars * 8;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;           // room to align the base
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget of one CTA");
 
 // TMEM columns.  Producer group g: D0 (64), R (64), X1 (128) at 256 g.
-// Consumer: D = [-W; Qh] S^T at 0, E = [U'; O'] at 128 (rows [U; o / scale] =
-// D + E, d_v columns), S~ (d_k x d_v) at 256.
+// Consumer: D = [U'; O'] + [-W; Qh] S^T (rows [U; o / scale], d_v columns) at
+// 0, S~ (d_k x d_v) at 256.
 constexpr uint32_t PCOL_D0 = 0, PCOL_R = 64, PCOL_X1 = 128;
-constexpr uint32_t CCOL_D = 0, CCOL_E = 128, CCOL_S = 256;
+constexpr uint32_t CCOL_D = 0, CCOL_S = 256;
 constexpr uint32_t TMEM_COLS = 512;
 
 constexpr uint32_t IDESC_D0 = idesc_bf16(128, 64, false, false);
@@ -234,6 +234,7 @@ struct Ctx {
     uint32_t sbase;
     uint32_t tmem;
     volatile int* abort;
+    volatile int* mma2_issued;   // consumer: chunks whose state update has been issued
     int warp, lane;
     int h, g;              // value head, key head
     uint8_t* ring;         // this unit's ring slots
@@ -247,6 +248,16 @@ struct Ctx {
     int traced;            // this unit's events are recorded (tracing builds only)
     TC_DEVICE uint32_t bar(int i) const { return bar0 + 8u * (uint32_t)i; }
 };
+
+// a counter in shared memory handed between two threads of the CTA
+__device__ __forceinline__ int ld_acquire_cta_s32(volatile int* p) {
+    int v;
+    asm volatile("ld.acquire.cta.shared.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32((const void*)p)) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_cta_s32(volatile int* p, int v) {
+    asm volatile("st.release.cta.shared.b32 [%0], %1;" ::"r"(smem_u32((const void*)p)), "r"(v) : "memory");
+}
 
 // ================================================================ consumer
 __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
@@ -290,8 +301,11 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
         }
     } else if (warp == 1) {
         // ------------------------------------------------ [U'; O'] = [T b; R b] V per chunk
-        // State-independent, so it runs ahead of the chain into its own
-        // accumulator E, once the epilogues have read the previous chunk's E.
+        // State-independent: it starts chunk c's accumulator D (the chain's
+        // [-W; Qh] S^T is added to it), once the state update of chunk c - 1
+        // has been issued (the epilogues are then done with D), so that it runs
+        // while the tensor core would otherwise wait for the second epilogue,
+        // and its issue does not compete with the chain's.
         if (lane == 0) {
             const uint64_t dsc_rt0 = sdesc_sw128(x.sbase + C_RECV + SL_RT2, 16, 1024);
             const uint64_t dsc_v = sdesc_sw128(x.sbase + C_V, 8192, 1024);
@@ -299,12 +313,18 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
                 const int b = c & 1;
                 if (!mbar_wait(x.bar(CB_RECV_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs)) break;
                 if (!mbar_wait(x.bar(CB_V_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs)) break;
-                if (c >= 1 && !mbar_wait(x.bar(CB_E_EMPTY), (c - 1) & 1, x.abort, kWaitLimitNs)) break;
+                if (c >= 1) {
+                    // bounded wait on the issuer's counter (shared memory)
+                    const uint64_t t0 = globaltimer_ns();
+                    while (ld_acquire_cta_s32(x.mma2_issued) < c && !*x.abort)
+                        if (globaltimer_ns() - t0 > kWaitLimitNs) *x.abort = 1;
+                    if (*x.abort) break;
+                }
                 TRACE_CLK(14, c);
                 tc_fence_after();
                 const uint64_t a = dsc_rt0 + b * (uint64_t)(SLOT_BYTES >> 4);
                 for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(x.tmem + CCOL_E, a + kk * 2, dsc_v + b * (16384 >> 4) + kk * 128, IDESC_N128_KM,
+                    mma_bf16(x.tmem + CCOL_D, a + kk * 2, dsc_v + b * (16384 >> 4) + kk * 128, IDESC_N128_KM,
                              kk > 0);
                 mma_commit(x.bar(CB_E_FULL));
                 mma_commit(x.bar(CB_V_EMPTY + b));
@@ -383,7 +403,7 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
         // the issuer reads a U row (quadrant 0), so it has no o rows to write out
         const bool issuer = (warp == kEpiWarp0 + 1 && lane == 0);
         const uint32_t tl = x.tmem + ((uint32_t)(q * 32) << 16);
-        const uint32_t dcol = CCOL_D + cb * 32, ecol = CCOL_E + cb * 32, scol = CCOL_S + cb * 32;
+        const uint32_t dcol = CCOL_D + cb * 32, scol = CCOL_S + cb * 32;
         const int hh = cb >> 1, ch0 = (cb & 1) * 4;   // d_v half and first 16-byte chunk in it
         uint8_t* st_tile = x.sm + C_ST + hh * 16384;
         uint8_t* uk_tile = x.sm + C_UK + hh * 8192;
@@ -416,17 +436,18 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
             // ---- [U; o / scale] = [U'; O'] + [-W; Qh] S^T: the second term here, the
             //      first (E) from warp 1
             if (issuer && !*x.abort &&
-                mbar_wait(x.bar(CB_RECV_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs)) {
+                mbar_wait(x.bar(CB_RECV_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs) &&
+                mbar_wait(x.bar(CB_E_FULL), c & 1, x.abort, kWaitLimitNs)) {
+                // D holds [U'; O'] (complete: its commit was seen); add [-W; Qh] S^T
                 tc_fence_after();
                 const uint64_t a = dsc_qw0 + b * kSlotStep;
                 for (int kk = 0; kk < 8; ++kk)
                     mma_bf16(x.tmem + CCOL_D, a + (((kk >> 2) * KQ_PANEL + (kk & 3) * 32) >> 4),
-                             dsc_st + kk * 128, IDESC_N128_KM, kk > 0);
+                             dsc_st + kk * 128, IDESC_N128_KM, 1);
                 mma_commit(x.bar(CB_D_FULL));
                 TRACE_CLK(0, c);
             }
             mbar_wait(x.bar(CB_RECV_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs);
-            mbar_wait(x.bar(CB_E_FULL), c & 1, x.abort, kWaitLimitNs);
             if (issuer) TRACE_CLK(1, c);
             mbar_wait(x.bar(CB_D_FULL), c & 1, x.abort, kWaitLimitNs);
             if (issuer) TRACE_CLK(2, c);
@@ -439,15 +460,13 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
             // kept in registers and written out after the barrier, while the
             // state update runs.
             float ov[32];
-            {
+            tmem_ld32(tl + dcol, ov);
+            tmem_ld_wait();
+            if (q < 2) {
+                const float sc = kap[r] * inv;
                 float e[32];
-                tmem_ld32x2(tl + dcol, tl + ecol, ov, e);
-                for (int j = 0; j < 32; ++j) ov[j] += e[j];
-                if (q < 2) {
-                    const float sc = kap[r] * inv;
-                    for (int j = 0; j < 32; ++j) e[j] = ov[j] * sc;
-                    for (int j = 0; j < 4; ++j) st_bf16x8(uk_tile, r, ch0 + j, e + 8 * j);
-                }
+                for (int j = 0; j < 32; ++j) e[j] = ov[j] * sc;
+                for (int j = 0; j < 4; ++j) st_bf16x8(uk_tile, r, ch0 + j, e + 8 * j);
             }
             if (resc) {
                 // S~ <- Gn S~ on this thread's 32 columns (Gamma restarts at 1)
@@ -475,10 +494,8 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
                     mma_commit(x.bar(CB_S_FULL));
                     mma_commit(x.bar(CB_K_EMPTY));
                 }
-                // E may be overwritten now; the next [U'; O'] product is issued (by
-                // warp 1) only after this chunk's state update, so that it does
-                // not slow down the issue of the chain's products
-                mbar_arrive(x.bar(CB_E_EMPTY));
+                // D may be restarted now by the next chunk's [U'; O'] product (warp 1)
+                st_release_cta_s32(x.mma2_issued, c + 1);
                 TRACE_CLK(5, c);
             }
             if (q >= 2) {
@@ -964,6 +981,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     x.bar0 = x.sbase + OFF_BARS;
     x.abort = reinterpret_cast<volatile int*>(sm + OFF_MISC);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC + 4);
+    x.mma2_issued = reinterpret_cast<volatile int*>(sm + OFF_MISC + 40);
     x.warp = threadIdx.x >> 5;
     x.lane = threadIdx.x & 31;
     // blocks [0, nu) are the consumers of the launch's nu units, then the first
@@ -1002,6 +1020,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
     if (threadIdx.x == 0) {
         *x.abort = 0;
+        *x.mma2_issued = 0;
         if (rank == 0) {
             for (int b = 0; b < 2; ++b) {
                 mbar_init(x.bar(CB_RECV_FULL + b), 1);
@@ -1018,7 +1037,6 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             mbar_init(x.bar(CB_S_FULL), 1);
             mbar_init(x.bar(CB_DRAIN), 1);
             mbar_init(x.bar(CB_E_FULL), 1);
-            mbar_init(x.bar(CB_E_EMPTY), 1);
             mbar_init(x.bar(CB_E_DRAIN), 1);
         } else {
             for (int s = 0; s < kKqStages; ++s) mbar_init(x.bar(PB_KQ_EMPTY + s), 1);
