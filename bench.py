@@ -294,6 +294,7 @@ def bench_main(args, world, rank, local):
     if not args.primary_only:
         extra["prefill_262k"] = bench_long_prefill(args, dev, flush, peaks, world)
         extra["decode_128seq_48layers"] = bench_decode(args, dev, peaks, world)
+        extra["decode_fused_128seq_48layers"] = bench_decode_fused(args, dev, peaks, world)
 
     value = world * T / (ms_max * 1e-3)
     line = {
@@ -444,6 +445,56 @@ def bench_decode(args, dev, peaks, world):
            "bytes_per_step": int(bytes_step), "l2": "state 19.3 GB >> L2, no flush needed",
            "launches_per_step": 1}
     del state, q, k, v, o
+    torch.cuda.empty_cache()
+    return out
+
+
+def bench_decode_fused(args, dev, peaks, world):
+    """One fused decode step (front end + recurrence) for 128 sequences x 48
+    layers: 19.3 GB float32 state and 0.75 GB of convolution history in place
+    (inputs drawn on the device; far larger than L2)."""
+    import torch
+    import gated_deltanet_recurrence_prefill_b200 as gdn
+    n_seq, L = 128, 48
+    U = n_seq * L
+    ctot = (2 * HQK + HV) * D
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5)
+    qkv = torch.randn(U, ctot, generator=gen, device=dev).to(torch.bfloat16)
+    conv_w = 0.5 * torch.randn(L, ctot, 4, generator=gen, device=dev)
+    conv_state = torch.randn(U, ctot, 3, generator=gen, device=dev)
+    a = torch.randn(U, HV, generator=gen, device=dev)
+    b = torch.randn(U, HV, generator=gen, device=dev)
+    A_log = torch.log(torch.empty(L, HV, device=dev).uniform_(1, 16, generator=gen))
+    dt = torch.exp(torch.empty(L, HV, device=dev).uniform_(-6.907755, -2.302585, generator=gen))
+    dt_bias = torch.log(torch.expm1(dt))
+    state = torch.empty(U, HV, D, D, dtype=torch.float32, device=dev)
+    for i in range(0, U, 512):
+        state[i:i + 512].normal_(0.0, 0.02, generator=gen)
+    slot = torch.randperm(n_seq, generator=gen, device=dev).to(torch.int32)
+    o = torch.empty(U, HV, D, dtype=torch.float32, device=dev)
+
+    def step(ev):
+        if ev:
+            ev["start"].record()
+        gdn.decode_step_fused(qkv, conv_w, conv_state, a, b, A_log, dt_bias, state, n_seq, L, HQK, HV,
+                              slot=slot, o=o)
+        if ev:
+            ev["end"].record()
+
+    mk = lambda: {"start": torch.cuda.Event(enable_timing=True),
+                  "end": torch.cuda.Event(enable_timing=True)}
+    dummy = torch.empty(1, device=dev)
+    times, _ = _time_steps(step, max(3, args.warmup), max(5, min(args.steps, 50)), dummy, mk)
+    ms = _max_over_ranks(sum(times) / len(times), world)
+    bytes_step = (2 * U * STATE_BYTES + 2 * U * ctot * 3 * 4 + U * ctot * 2 + L * ctot * 16
+                  + U * HV * (2 * 4 + 4 * D))
+    gbs = bytes_step / (ms * 1e-3) / 1e9
+    out = {"workload": "gdn_decode_step_fused 128 seq x 48 layers (front end fused), fp32 state "
+                       "19.33 GB + conv history 0.75 GB in place, shuffled slots",
+           "ms": round(ms, 4), "GB_s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+           "bytes_per_step": int(bytes_step), "launches_per_step": 1}
+    del state, conv_state, qkv, o
     torch.cuda.empty_cache()
     return out
 

@@ -10,6 +10,7 @@ from ._lib import (  # noqa: F401
     STATUS,
     conv1d_silu,
     decode_step,
+    decode_step_fused,
     lib,
     lib_path,
     prefill,

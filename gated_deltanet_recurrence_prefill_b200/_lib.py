@@ -35,6 +35,8 @@ SIGNATURES = {
                                       _i32, _f32, _vp, _vp, _vp, _vp]),
     "gdn_decode_step": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                   _f32, _vp, _vp, _vp]),
+    "gdn_decode_step_fused": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
+                                        _i32, _i32, _f32, _i32, _vp, _vp, _vp]),
 }
 
 
@@ -231,4 +233,36 @@ def decode_step(q, k, v, a, b, A_log, dt_bias, state, n_seq, layers, scale=None,
                                _ptr(dt_bias), n_seq, layers, Hqk, Hv, d, float(scale), _ptr(state),
                                _ptr(o), _stream(stream))
     _check("gdn_decode_step", st)
+    return o
+
+
+def decode_step_fused(qkv, conv_w, conv_state, a, b, A_log, dt_bias, state, n_seq, layers, Hqk, Hv,
+                      slot=None, scale=None, o=None, stream=None):
+    """One decode step with the front end fused in, for n_seq sequences x
+    `layers` layers.  qkv [n_seq*layers, Ctot] bf16, conv_w [layers, Ctot, 4],
+    conv_state [n_slots*layers, Ctot, 3] and state [n_slots*layers, Hv, d, d]
+    float32 (both updated in place), slot [n_seq] int32 or None.  Returns
+    o [n_seq*layers, Hv, d] f32."""
+    import torch
+    d = state.shape[-1]
+    U = n_seq * layers
+    ctot = (2 * Hqk + Hv) * d
+    n_slots = state.shape[0] // layers
+    _need(qkv, torch.bfloat16, (U, ctot), "qkv")
+    _need(conv_w, torch.float32, (layers, ctot, 4), "conv_w")
+    _need(conv_state, torch.float32, (n_slots * layers, ctot, 3), "conv_state")
+    _need(state, torch.float32, (n_slots * layers, Hv, d, d), "state")
+    _need(a, torch.float32, (U, Hv), "a")
+    _need(b, torch.float32, (U, Hv), "b")
+    _need(A_log, torch.float32, (layers, Hv), "A_log")
+    _need(dt_bias, torch.float32, (layers, Hv), "dt_bias")
+    if slot is not None:
+        _need(slot, torch.int32, (n_seq,), "slot")
+    if o is None:
+        o = torch.empty(U, Hv, d, dtype=torch.float32, device=state.device)
+    scale = 1.0 / d ** 0.5 if scale is None else float(scale)
+    st = lib().gdn_decode_step_fused(_ptr(qkv), _ptr(conv_w), _ptr(conv_state), _ptr(a), _ptr(b),
+                                     _ptr(A_log), _ptr(dt_bias), _ptr(slot), n_seq, layers, Hqk, Hv,
+                                     d, scale, n_slots, _ptr(state), _ptr(o), _stream(stream))
+    _check("gdn_decode_step_fused", st)
     return o

@@ -224,6 +224,34 @@ gdn_status gdn_decode_step(const uint16_t* q, const uint16_t* k, const uint16_t*
                            int32_t Hv, int32_t d, float scale, float* state, float* o,
                            gdn_stream_t stream);
 
+/*
+ * gdn_decode_step_fused -- one decode step with the layer's front end fused
+ * in: for each (sequence, layer) unit the token's packed projection goes
+ * through the causal width-4 convolution, SiLU and the q / k L2 norm
+ * (gdn_conv1d_silu's arithmetic, architecture page section 2.1), then one step
+ * of the recurrence (as gdn_decode_step, section 2.2).  q, k and v stay in
+ * float32 between the two (no bf16 rounding).  The convolution history and the
+ * state are updated in place.
+ *
+ *  qkv            [n_seq, layers, Ctot] bf16, Ctot = (2 Hqk + Hv) d, channels
+ *                 ordered as in gdn_conv1d_silu.
+ *  conv_w         [layers, Ctot, 4] float32 (tap 3 multiplies the current input).
+ *  conv_state     [n_slots, layers, Ctot, 3] float32 in place: the three previous
+ *                 inputs of each channel, oldest first.
+ *  a, b           [n_seq, layers, Hv] float32;  A_log, dt_bias [layers, Hv] float32.
+ *  slot           [n_seq] int32 (device): the slot holding sequence n's states,
+ *                 or NULL for slot n (then n_slots >= n_seq).  Slots must be
+ *                 distinct and < n_slots; the library trusts them.
+ *  state          [n_slots, layers, Hv, d_v, d_k] float32 in place.
+ *  o              [n_seq, layers, Hv, d] float32 output.
+ * Slots not named by `slot` are not touched.  Supported: d = 128, Hv % Hqk == 0.
+ */
+gdn_status gdn_decode_step_fused(const uint16_t* qkv, const float* conv_w, float* conv_state,
+                                 const float* a, const float* b, const float* A_log,
+                                 const float* dt_bias, const int32_t* slot, int32_t n_seq,
+                                 int32_t layers, int32_t Hqk, int32_t Hv, int32_t d, float scale,
+                                 int32_t n_slots, float* state, float* o, gdn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -33,7 +33,7 @@ import numpy as np
 HQK, HV, D, CONV_K = 16, 48, 128, 4
 
 # stream ids: one per kind of array, so that changing one size leaves the others
-_S_Q, _S_K, _S_V, _S_A, _S_B, _S_ALOG, _S_DT, _S_S0, _S_QKV, _S_W, _S_LEN = range(11)
+_S_Q, _S_K, _S_V, _S_A, _S_B, _S_ALOG, _S_DT, _S_S0, _S_QKV, _S_W, _S_LEN, _S_SLOT, _S_CS = range(13)
 
 _BLOCK_ROWS = 4096          # rows per independently seeded block
 
@@ -273,6 +273,56 @@ def make_decode(n_seq: int, layers: int, seed: int, *, state_std: float = 0.02,
     A_log, dt_bias = gate_params(seed, Hv, layers)
     return DecodeInputs(q, k, v, a, b, A_log, dt_bias, n_seq, layers, seed, state_std,
                         1.0 / math.sqrt(d), Hqk, Hv, d)
+
+
+@dataclass
+class FusedDecodeInputs:
+    """One decode step with the front end fused in: n_seq sequences x `layers`
+    layers (unit u = n * layers + l), states held in n_slots slots."""
+    qkv: np.ndarray          # uint16 [U, Ctot] packed q|k|v channels of the token
+    conv_w: np.ndarray       # float32 [layers, Ctot, 4]
+    conv_state: np.ndarray   # float32 [n_slots * layers, Ctot, 3], oldest input first
+    a: np.ndarray            # float32 [U, Hv]
+    b: np.ndarray
+    A_log: np.ndarray        # float32 [layers, Hv]
+    dt_bias: np.ndarray
+    state: np.ndarray        # float32 [n_slots * layers, Hv, d, d]
+    slot: np.ndarray         # int32 [n_seq], distinct slots
+    n_seq: int
+    layers: int
+    n_slots: int
+    scale: float
+    Hqk: int = HQK
+    Hv: int = HV
+    d: int = D
+
+    @property
+    def U(self) -> int:
+        return self.n_seq * self.layers
+
+
+def make_decode_fused(n_seq: int, layers: int, n_slots: int, seed: int, *, w_std: float = 0.5,
+                      state_std: float = 0.02, Hqk: int = HQK, Hv: int = HV,
+                      d: int = D) -> FusedDecodeInputs:
+    """Packed channels ~ N(0,1) in bf16, conv weights ~ N(0, w_std^2), conv
+    histories ~ N(0,1) rounded to bf16 values, states ~ N(0, state_std^2), gates
+    as for decode, and the sequences placed in a random choice of distinct
+    slots."""
+    U = n_seq * layers
+    ctot = (2 * Hqk + Hv) * d
+    qkv = f32_to_bf16_bits(_normal_rows(seed, _S_QKV, U, ctot))
+    conv_w = _rng(seed, _S_W).standard_normal((layers, ctot, CONV_K), dtype=np.float32)
+    conv_w *= np.float32(w_std)
+    cs = _rng(seed, _S_CS).standard_normal((n_slots * layers, ctot, 3), dtype=np.float32)
+    cs = bf16_bits_to_f32(f32_to_bf16_bits(cs))
+    a = _normal_rows(seed, _S_A, U, Hv)
+    b = _normal_rows(seed, _S_B, U, Hv)
+    A_log, dt_bias = gate_params(seed, Hv, layers)
+    st = _rng(seed, _S_S0).standard_normal((n_slots * layers, Hv, d, d), dtype=np.float32)
+    st *= np.float32(state_std)
+    slot = _rng(seed, _S_SLOT).permutation(n_slots)[:n_seq].astype(np.int32)
+    return FusedDecodeInputs(qkv, conv_w, cs, a, b, A_log, dt_bias, st, slot, n_seq, layers,
+                             n_slots, 1.0 / math.sqrt(d), Hqk, Hv, d)
 
 
 # ---- the five workloads --------------------------------------------------------

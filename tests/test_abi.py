@@ -27,7 +27,8 @@ def L():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for required in ("gdn_conv1d_silu", "gdn_prefill", "gdn_prefill_workspace_size",
-                     "gdn_decode_step", "gdn_prefill_status", "gdn_status_string"):
+                     "gdn_decode_step", "gdn_decode_step_fused", "gdn_prefill_status",
+                     "gdn_status_string"):
         assert required in names
 
 
@@ -118,3 +119,17 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(_lib, "_lib", None)
     with pytest.raises(ImportError):
         _lib.lib()
+
+
+def test_fused_decode_rejects_bad_arguments(L):
+    def call(d=128, Hv=48, layers=48, n_seq=4, n_slots=4, slot=None, state=_p(), qkv=_p()):
+        return L.gdn_decode_step_fused(qkv, _p(), _p(), _p(), _p(), _p(), _p(), slot, n_seq, layers,
+                                       16, Hv, d, 0.088, n_slots, state, _p(), None)
+    assert call(d=64) == 2
+    assert call(Hv=47) == 2
+    assert call(layers=0) == 1
+    assert call(n_slots=0) == 1
+    assert call(n_slots=3) == 1                  # identity slots need n_slots >= n_seq
+    assert call(qkv=None) == 1
+    assert call(state=_p(FAKE + 8)) == 3         # misaligned
+    assert call(n_seq=0) == 0                    # nothing to do
