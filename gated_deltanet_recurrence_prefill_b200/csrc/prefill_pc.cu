@@ -671,6 +671,14 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
     const bool issuer = (pw == 0 && lane == 0);
     const float Al = p.A_log[h], dtb = p.dt_bias[h];
     uint8_t* stage_rt = gbase + G_AF;          // [T b; R b] and the gates, staged for sending
+    // shared-memory descriptors, computed once (a K step or a stage adds a byte
+    // offset >> 4 to the start address field): rebuilding them per instruction
+    // doubles the cost of issuing a tcgen05.mma
+    const uint64_t dsc_kq0 = sdesc_sw128(x.sbase + P_KQ, 16, 1024);             // [K; Q], K-major
+    const uint64_t dsc_kq0_mn = sdesc_sw128(x.sbase + P_KQ, KQ_PANEL, 1024);    // K rows, MN-major
+    const uint64_t dsc_pt = sdesc_sw128(gsb + G_PT, 16, 1024);                  // [P; T] / [R bg; T bg]
+    const uint64_t dsc_t = sdesc_sw128(gsb + G_PT + 8192, 8192, 1024);          // T, MN-major
+    constexpr uint64_t kStageStep = KQ_STAGE >> 4;
 
     int jj = 0;                                // chunks done by this group
     for (int i = grp;; i += 2, ++jj) {
@@ -680,7 +688,6 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
         GateBuf& gb = gates[jj & 1];
         const int64_t tok0 = x.bos + (int64_t)c * kC;
         const uint32_t kqo = P_KQ + s * KQ_STAGE;
-        const uint32_t kq = x.sbase + kqo;
         // every warp of the group has seen chunk i land before the TMA warp may
         // arm this group's barrier again
         if (pw == 0 && lane == 0) TRACE_CLK(16, c);
@@ -691,9 +698,11 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
         if (issuer) {
             // D0 = [K; Q] K^T
             tc_fence_after();
-            for (int kk = 0; kk < 8; ++kk)
-                mma_bf16(tg + PCOL_D0, desc_kmajor_2panel(kq, kk), desc_kmajor_2panel(kq, kk), IDESC_D0,
-                         kk > 0);
+            const uint64_t d = dsc_kq0 + s * kStageStep;
+            for (int kk = 0; kk < 8; ++kk) {
+                const uint64_t off = ((kk >> 2) * KQ_PANEL + (kk & 3) * 32) >> 4;
+                mma_bf16(tg + PCOL_D0, d + off, d + off, IDESC_D0, kk > 0);
+            }
             mma_commit(x.bar(PB_D0_FULL + grp));
         }
         __syncwarp();
@@ -858,8 +867,7 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
             // R = [P; T] T (rows 0-63 used)
             tc_fence_after();
             for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tg + PCOL_R, desc_kmajor_1panel(gsb + G_PT, kk),
-                         desc_mnmajor(gsb + G_PT + 8192, kk, 8192), IDESC_R, kk > 0);
+                mma_bf16(tg + PCOL_R, dsc_pt + kk * 2, dsc_t + kk * 128, IDESC_R, kk > 0);
             mma_commit(x.bar(PB_R_FULL + grp));
         }
         __syncwarp();
@@ -914,8 +922,8 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
             // X1 = [R bg; T bg] K  ->  rows 0-63: P W, rows 64-127: W
             tc_fence_after();
             for (int kk = 0; kk < 4; ++kk)
-                mma_bf16(tg + PCOL_X1, desc_kmajor_1panel(gsb + G_PT, kk), desc_mnmajor(kq, kk, KQ_PANEL),
-                         IDESC_X1, kk > 0);
+                mma_bf16(tg + PCOL_X1, dsc_pt + kk * 2, dsc_kq0_mn + s * kStageStep + kk * 128, IDESC_X1,
+                         kk > 0);
             mma_commit(x.bar(PB_X1_FULL + grp));
         }
         __syncwarp();
