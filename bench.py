@@ -295,6 +295,7 @@ def bench_main(args, world, rank, local):
         extra["prefill_262k"] = bench_long_prefill(args, dev, flush, peaks, world)
         extra["decode_128seq_48layers"] = bench_decode(args, dev, peaks, world)
         extra["decode_fused_128seq_48layers"] = bench_decode_fused(args, dev, peaks, world)
+        extra["decode_bf16state_128seq_48layers"] = bench_decode(args, dev, peaks, world, bf16_state=True)
 
     value = world * T / (ms_max * 1e-3)
     line = {
@@ -398,9 +399,10 @@ def bench_long_prefill(args, dev, flush, peaks, world):
     return out
 
 
-def bench_decode(args, dev, peaks, world):
-    """One decode step for 128 sequences x 48 layers, 19.3 GB float32 state in
-    place (inputs drawn on the device; the state is far larger than L2)."""
+def bench_decode(args, dev, peaks, world, bf16_state=False):
+    """One decode step for 128 sequences x 48 layers, 19.3 GB float32 state (or
+    9.7 GB bf16 state) in place (inputs drawn on the device; the state is far
+    larger than L2)."""
     import torch
     import gated_deltanet_recurrence_prefill_b200 as gdn
     n_seq, L = 128, 48
@@ -421,7 +423,7 @@ def bench_decode(args, dev, peaks, world):
     A_log = torch.log(torch.empty(L, HV, device=dev).uniform_(1, 16, generator=gen))
     dt = torch.exp(torch.empty(L, HV, device=dev).uniform_(-6.907755, -2.302585, generator=gen))
     dt_bias = torch.log(torch.expm1(dt))
-    state = torch.empty(U, HV, D, D, dtype=torch.float32, device=dev)
+    state = torch.empty(U, HV, D, D, dtype=torch.bfloat16 if bf16_state else torch.float32, device=dev)
     for i in range(0, U, 512):
         state[i:i + 512].normal_(0.0, 0.02, generator=gen)
     o = torch.empty(U, HV, D, dtype=torch.float32, device=dev)
@@ -438,9 +440,12 @@ def bench_decode(args, dev, peaks, world):
     dummy = torch.empty(1, device=dev)
     times, _ = _time_steps(step, max(3, args.warmup), max(5, args.steps), dummy, mk)
     ms = _max_over_ranks(sum(times) / len(times), world)
-    bytes_step = 2 * U * STATE_BYTES + U * (2 * 2 * HQK * D + 2 * HV * D + 2 * 4 * HV + 4 * HV * D)
+    state_bytes = STATE_BYTES // 2 if bf16_state else STATE_BYTES
+    bytes_step = 2 * U * state_bytes + U * (2 * 2 * HQK * D + 2 * HV * D + 2 * 4 * HV + 4 * HV * D)
     gbs = bytes_step / (ms * 1e-3) / 1e9
-    out = {"workload": "gdn_decode_step 128 seq x 48 layers, fp32 state 19.33 GB in place",
+    out = {"workload": ("gdn_decode_step_bf16 128 seq x 48 layers, bf16 state 9.66 GB in place"
+                        if bf16_state else
+                        "gdn_decode_step 128 seq x 48 layers, fp32 state 19.33 GB in place"),
            "ms": round(ms, 4), "GB_s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
            "bytes_per_step": int(bytes_step), "l2": "state 19.3 GB >> L2, no flush needed",
            "launches_per_step": 1}

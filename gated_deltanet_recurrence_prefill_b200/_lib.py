@@ -37,6 +37,10 @@ SIGNATURES = {
                                   _f32, _vp, _vp, _vp]),
     "gdn_decode_step_fused": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32,
                                         _i32, _i32, _f32, _i32, _vp, _vp, _vp]),
+    "gdn_decode_step_bf16": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
+                                       _i32, _f32, _vp, _vp, _vp]),
+    "gdn_decode_step_fused_bf16": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
+                                             _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp]),
 }
 
 
@@ -210,8 +214,9 @@ def prefill_status(workspace, stream=None) -> int:
 
 def decode_step(q, k, v, a, b, A_log, dt_bias, state, n_seq, layers, scale=None, o=None,
                 stream=None):
-    """One decode step over U = n_seq*layers units; `state` [U,Hv,d,d] f32 is
-    updated in place.  Returns o [U,Hv,d] f32."""
+    """One decode step over U = n_seq*layers units; `state` [U,Hv,d,d] (float32,
+    or bfloat16 for the bf16-state entry point) is updated in place.  Returns
+    o [U,Hv,d] f32."""
     import torch
     U, Hqk, d = q.shape
     Hv = v.shape[1]
@@ -224,15 +229,17 @@ def decode_step(q, k, v, a, b, A_log, dt_bias, state, n_seq, layers, scale=None,
     _need(b, torch.float32, (U, Hv), "b")
     _need(A_log, torch.float32, (layers, Hv), "A_log")
     _need(dt_bias, torch.float32, (layers, Hv), "dt_bias")
-    _need(state, torch.float32, (U, Hv, d, d), "state")
+    bf16 = state.dtype == torch.bfloat16
+    _need(state, torch.bfloat16 if bf16 else torch.float32, (U, Hv, d, d), "state")
     if scale is None:
         scale = d ** -0.5
     if o is None:
         o = torch.empty(U, Hv, d, dtype=torch.float32, device=q.device)
-    st = lib().gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(A_log),
-                               _ptr(dt_bias), n_seq, layers, Hqk, Hv, d, float(scale), _ptr(state),
-                               _ptr(o), _stream(stream))
-    _check("gdn_decode_step", st)
+    name = "gdn_decode_step_bf16" if bf16 else "gdn_decode_step"
+    st = getattr(lib(), name)(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(A_log),
+                              _ptr(dt_bias), n_seq, layers, Hqk, Hv, d, float(scale), _ptr(state),
+                              _ptr(o), _stream(stream))
+    _check(name, st)
     return o
 
 
@@ -240,9 +247,9 @@ def decode_step_fused(qkv, conv_w, conv_state, a, b, A_log, dt_bias, state, n_se
                       slot=None, scale=None, o=None, stream=None):
     """One decode step with the front end fused in, for n_seq sequences x
     `layers` layers.  qkv [n_seq*layers, Ctot] bf16, conv_w [layers, Ctot, 4],
-    conv_state [n_slots*layers, Ctot, 3] and state [n_slots*layers, Hv, d, d]
-    float32 (both updated in place), slot [n_seq] int32 or None.  Returns
-    o [n_seq*layers, Hv, d] f32."""
+    conv_state [n_slots*layers, Ctot, 3] float32 and state [n_slots*layers, Hv,
+    d, d] (float32, or bfloat16 for the bf16-state entry point), both updated in
+    place, slot [n_seq] int32 or None.  Returns o [n_seq*layers, Hv, d] f32."""
     import torch
     d = state.shape[-1]
     U = n_seq * layers
@@ -251,7 +258,8 @@ def decode_step_fused(qkv, conv_w, conv_state, a, b, A_log, dt_bias, state, n_se
     _need(qkv, torch.bfloat16, (U, ctot), "qkv")
     _need(conv_w, torch.float32, (layers, ctot, 4), "conv_w")
     _need(conv_state, torch.float32, (n_slots * layers, ctot, 3), "conv_state")
-    _need(state, torch.float32, (n_slots * layers, Hv, d, d), "state")
+    bf16 = state.dtype == torch.bfloat16
+    _need(state, torch.bfloat16 if bf16 else torch.float32, (n_slots * layers, Hv, d, d), "state")
     _need(a, torch.float32, (U, Hv), "a")
     _need(b, torch.float32, (U, Hv), "b")
     _need(A_log, torch.float32, (layers, Hv), "A_log")
@@ -261,8 +269,9 @@ def decode_step_fused(qkv, conv_w, conv_state, a, b, A_log, dt_bias, state, n_se
     if o is None:
         o = torch.empty(U, Hv, d, dtype=torch.float32, device=state.device)
     scale = 1.0 / d ** 0.5 if scale is None else float(scale)
-    st = lib().gdn_decode_step_fused(_ptr(qkv), _ptr(conv_w), _ptr(conv_state), _ptr(a), _ptr(b),
-                                     _ptr(A_log), _ptr(dt_bias), _ptr(slot), n_seq, layers, Hqk, Hv,
-                                     d, scale, n_slots, _ptr(state), _ptr(o), _stream(stream))
-    _check("gdn_decode_step_fused", st)
+    name = "gdn_decode_step_fused_bf16" if bf16 else "gdn_decode_step_fused"
+    st = getattr(lib(), name)(_ptr(qkv), _ptr(conv_w), _ptr(conv_state), _ptr(a), _ptr(b),
+                              _ptr(A_log), _ptr(dt_bias), _ptr(slot), n_seq, layers, Hqk, Hv,
+                              d, scale, n_slots, _ptr(state), _ptr(o), _stream(stream))
+    _check(name, st)
     return o

@@ -12,10 +12,16 @@
 // (2 x 64 KiB per value head per token); the kernel is bound by HBM bandwidth.
 //
 // Mapping: one CTA of 128 threads per (unit, value head).  Each warp owns 32
-// rows; a lane holds 4 consecutive d_k elements (one float4) of a row, so a
-// row is one fully coalesced 512-byte access.  Eight rows are in flight per
-// warp to keep enough bytes outstanding.
+// rows; a lane holds 4 consecutive d_k elements of a row (a float4, or 8 bytes
+// for a bf16 state), so a row is one fully coalesced access.  Eight rows are
+// in flight per warp to keep enough bytes outstanding.
+//
+// The state is stored in float32 (the layer's state, architecture page section
+// 2.2) or, in the bf16 variant, as bf16: the arithmetic is float32 either way
+// and the updated row is rounded to bf16 (nearest even) when stored, which
+// halves the bytes of this bandwidth-bound step.
 #include "common.cuh"
+#include "decode_state.cuh"
 #include "kernels.h"
 
 namespace gdn {
@@ -24,14 +30,16 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kThreads = 128;
-constexpr int kRowsPerIter = 8;
+// rows in flight per warp: 8 float32 rows or 16 bf16 rows (4 KB either way)
+template <typename StateT> constexpr int rows_per_iter() { return sizeof(StateT) == 4 ? 8 : 16; }
 
-__global__ void __launch_bounds__(kThreads)
+template <typename StateT>
+__global__ void __launch_bounds__(kThreads, sizeof(StateT) == 2 ? 1 : 5)
 decode_step_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
                    const uint16_t* __restrict__ v, const float* __restrict__ a,
                    const float* __restrict__ b, const float* __restrict__ A_log,
                    const float* __restrict__ dt_bias, int32_t layers, int32_t Hqk, int32_t Hv,
-                   float scale, float* __restrict__ state, float* __restrict__ o) {
+                   float scale, StateT* __restrict__ state, float* __restrict__ o) {
     const int64_t uh = blockIdx.x;                 // unit * Hv + h
     const int64_t u = uh / Hv;
     const int h = (int)(uh - u * Hv);
@@ -50,7 +58,8 @@ decode_step_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ 
     const float alpha = expf(log_alpha_f32(a[uh], A_log[(int64_t)l * Hv + h], dt_bias[(int64_t)l * Hv + h]));
     const float beta = sigmoid_f32(b[uh]);
 
-    float* S = state + uh * (int64_t)(kD * kD);
+    StateT* S = state + uh * (int64_t)(kD * kD);
+    constexpr int kRowsPerIter = rows_per_iter<StateT>();
     const uint16_t* vh = v + uh * kD;
     float* oh = o + uh * kD;
 
@@ -59,16 +68,17 @@ decode_step_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ 
         float4 s[kRowsPerIter];
 #pragma unroll
         for (int j = 0; j < kRowsPerIter; ++j)
-            s[j] = __ldcs(reinterpret_cast<const float4*>(S + (int64_t)(r0 + j) * kD) + lane);
-        // v for these 8 rows: one 16-byte broadcast load
-        const uint4 vb = *reinterpret_cast<const uint4*>(vh + r0);
+            s[j] = state_load4(S + (int64_t)(r0 + j) * kD, lane);
+        // v for these rows: 16-byte broadcast loads of 8 values
         float vr[kRowsPerIter];
-        {
+#pragma unroll
+        for (int j8 = 0; j8 < kRowsPerIter; j8 += 8) {
+            const uint4 vb = *reinterpret_cast<const uint4*>(vh + r0 + j8);
             float2 t;
-            t = bf16x2_to_f32x2(vb.x); vr[0] = t.x; vr[1] = t.y;
-            t = bf16x2_to_f32x2(vb.y); vr[2] = t.x; vr[3] = t.y;
-            t = bf16x2_to_f32x2(vb.z); vr[4] = t.x; vr[5] = t.y;
-            t = bf16x2_to_f32x2(vb.w); vr[6] = t.x; vr[7] = t.y;
+            t = bf16x2_to_f32x2(vb.x); vr[j8 + 0] = t.x; vr[j8 + 1] = t.y;
+            t = bf16x2_to_f32x2(vb.y); vr[j8 + 2] = t.x; vr[j8 + 3] = t.y;
+            t = bf16x2_to_f32x2(vb.z); vr[j8 + 4] = t.x; vr[j8 + 5] = t.y;
+            t = bf16x2_to_f32x2(vb.w); vr[j8 + 6] = t.x; vr[j8 + 7] = t.y;
         }
         float xk[kRowsPerIter], xq[kRowsPerIter];
 #pragma unroll
@@ -93,7 +103,7 @@ decode_step_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ 
             t.y = fmaf(alpha, s[j].y, w * k01.y);
             t.z = fmaf(alpha, s[j].z, w * k23.x);
             t.w = fmaf(alpha, s[j].w, w * k23.y);
-            __stcs(reinterpret_cast<float4*>(S + (int64_t)(r0 + j) * kD) + lane, t);
+            state_store4(S + (int64_t)(r0 + j) * kD, lane, t);
             const float oj = scale * fmaf(alpha, xq[j], w * kq);
             if (lane == j) orow = oj;
         }
@@ -111,7 +121,20 @@ cudaError_t launch_decode_step(const uint16_t* q, const uint16_t* k, const uint1
     const int64_t blocks = (int64_t)n_seq * layers * Hv;
     if (blocks == 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    decode_step_kernel<<<(unsigned)blocks, kThreads, 0, stream>>>(
+    decode_step_kernel<float><<<(unsigned)blocks, kThreads, 0, stream>>>(
+        q, k, v, a, b, A_log, dt_bias, layers, Hqk, Hv, scale, state, o);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_step_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                    const float* a, const float* b, const float* A_log,
+                                    const float* dt_bias, int32_t n_seq, int32_t layers, int32_t Hqk,
+                                    int32_t Hv, float scale, uint16_t* state, float* o,
+                                    cudaStream_t stream) {
+    const int64_t blocks = (int64_t)n_seq * layers * Hv;
+    if (blocks == 0) return cudaSuccess;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    decode_step_kernel<uint16_t><<<(unsigned)blocks, kThreads, 0, stream>>>(
         q, k, v, a, b, A_log, dt_bias, layers, Hqk, Hv, scale, state, o);
     return cudaGetLastError();
 }

@@ -20,6 +20,7 @@
 // rounding between the front end and the recurrence.  The state traffic
 // dominates: the kernel is bound by HBM bandwidth.
 #include "common.cuh"
+#include "decode_state.cuh"
 #include "kernels.h"
 
 namespace gdn {
@@ -28,7 +29,8 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kThreads = 128;
-constexpr int kRowsPerIter = 8;
+// rows in flight per warp: 8 float32 rows or 16 bf16 rows (4 KB either way)
+template <typename StateT> constexpr int rows_per_iter() { return sizeof(StateT) == 4 ? 8 : 16; }
 
 // SiLU(y) = y / (1 + e^-y) with the accurate exponential (decode is checked
 // to 1e-4, so no fast approximation here)
@@ -58,12 +60,13 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
     return red[0] + red[1] + red[2] + red[3];
 }
 
-__global__ void __launch_bounds__(kThreads)
+template <typename StateT>
+__global__ void __launch_bounds__(kThreads, sizeof(StateT) == 2 ? 1 : 5)
 decode_fused_kernel(const uint16_t* __restrict__ qkv, const float* __restrict__ conv_w,
                     float* __restrict__ conv_state, const float* __restrict__ a,
                     const float* __restrict__ b, const float* __restrict__ A_log,
                     const float* __restrict__ dt_bias, const int32_t* __restrict__ slot,
-                    int32_t layers, int32_t Hqk, int32_t Hv, float scale, float* __restrict__ state,
+                    int32_t layers, int32_t Hqk, int32_t Hv, float scale, StateT* __restrict__ state,
                     float* __restrict__ o) {
     __shared__ float qs[kD], ks[kD], vs[kD];
     __shared__ float red[4];
@@ -117,14 +120,15 @@ decode_fused_kernel(const uint16_t* __restrict__ qkv, const float* __restrict__ 
         const int64_t uh = u * Hv + h;
         const float alpha = expf(log_alpha_f32(a[uh], A_log[(int64_t)l * Hv + h], dt_bias[(int64_t)l * Hv + h]));
         const float beta = sigmoid_f32(b[uh]);
-        float* S = state + (su * Hv + h) * (int64_t)(kD * kD);
+        StateT* S = state + (su * Hv + h) * (int64_t)(kD * kD);
+        constexpr int kRowsPerIter = rows_per_iter<StateT>();
         float* oh = o + uh * kD;
 #pragma unroll 1
         for (int r0 = warp * 32; r0 < warp * 32 + 32; r0 += kRowsPerIter) {
             float4 s[kRowsPerIter];
 #pragma unroll
             for (int i = 0; i < kRowsPerIter; ++i)
-                s[i] = __ldcs(reinterpret_cast<const float4*>(S + (int64_t)(r0 + i) * kD) + lane);
+                s[i] = state_load4(S + (int64_t)(r0 + i) * kD, lane);
             float xk[kRowsPerIter], xq[kRowsPerIter];
 #pragma unroll
             for (int i = 0; i < kRowsPerIter; ++i) {
@@ -148,7 +152,7 @@ decode_fused_kernel(const uint16_t* __restrict__ qkv, const float* __restrict__ 
                 nv.y = fmaf(alpha, s[i].y, w * k4.y);
                 nv.z = fmaf(alpha, s[i].z, w * k4.z);
                 nv.w = fmaf(alpha, s[i].w, w * k4.w);
-                __stcs(reinterpret_cast<float4*>(S + (int64_t)(r0 + i) * kD) + lane, nv);
+                state_store4(S + (int64_t)(r0 + i) * kD, lane, nv);
                 const float oi = scale * fmaf(alpha, xq[i], w * kq);
                 if (lane == i) orow = oi;
             }
@@ -167,7 +171,20 @@ cudaError_t launch_decode_fused(const uint16_t* qkv, const float* conv_w, float*
     const int64_t blocks = (int64_t)n_seq * layers * Hqk;
     if (blocks == 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    decode_fused_kernel<<<(unsigned)blocks, kThreads, 0, stream>>>(
+    decode_fused_kernel<float><<<(unsigned)blocks, kThreads, 0, stream>>>(
+        qkv, conv_w, conv_state, a, b, A_log, dt_bias, slot, layers, Hqk, Hv, scale, state, o);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode_fused_bf16(const uint16_t* qkv, const float* conv_w, float* conv_state,
+                                     const float* a, const float* b, const float* A_log,
+                                     const float* dt_bias, const int32_t* slot, int32_t n_seq,
+                                     int32_t layers, int32_t Hqk, int32_t Hv, float scale,
+                                     uint16_t* state, float* o, cudaStream_t stream) {
+    const int64_t blocks = (int64_t)n_seq * layers * Hqk;
+    if (blocks == 0) return cudaSuccess;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    decode_fused_kernel<uint16_t><<<(unsigned)blocks, kThreads, 0, stream>>>(
         qkv, conv_w, conv_state, a, b, A_log, dt_bias, slot, layers, Hqk, Hv, scale, state, o);
     return cudaGetLastError();
 }

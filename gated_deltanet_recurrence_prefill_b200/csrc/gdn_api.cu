@@ -190,4 +190,44 @@ gdn_status gdn_decode_step_fused(const uint16_t* qkv, const float* conv_w, float
     return e == cudaSuccess ? GDN_OK : cuda_fail(e);
 }
 
+gdn_status gdn_decode_step_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                const float* a, const float* b, const float* A_log,
+                                const float* dt_bias, int32_t n_seq, int32_t layers, int32_t Hqk,
+                                int32_t Hv, int32_t d, float scale, uint16_t* state, float* o,
+                                gdn_stream_t stream) {
+    gdn_status st = check_heads(Hqk, Hv, d);
+    if (st != GDN_OK) return st;
+    if (n_seq < 0 || layers <= 0) return GDN_ERR_INVALID_ARG;
+    if (n_seq == 0) return GDN_OK;
+    if (!q || !k || !v || !a || !b || !A_log || !dt_bias || !state || !o)
+        return GDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, a, b, A_log, dt_bias, state, o};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return GDN_ERR_MISALIGNED;
+    cudaError_t e = gdn::launch_decode_step_bf16(q, k, v, a, b, A_log, dt_bias, n_seq, layers, Hqk, Hv,
+                                                 scale, state, o, (cudaStream_t)stream);
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
+gdn_status gdn_decode_step_fused_bf16(const uint16_t* qkv, const float* conv_w, float* conv_state,
+                                      const float* a, const float* b, const float* A_log,
+                                      const float* dt_bias, const int32_t* slot, int32_t n_seq,
+                                      int32_t layers, int32_t Hqk, int32_t Hv, int32_t d, float scale,
+                                      int32_t n_slots, uint16_t* state, float* o, gdn_stream_t stream) {
+    gdn_status st = check_heads(Hqk, Hv, d);
+    if (st != GDN_OK) return st;
+    if (n_seq < 0 || layers <= 0 || n_slots <= 0) return GDN_ERR_INVALID_ARG;
+    if (!slot && n_slots < n_seq) return GDN_ERR_INVALID_ARG;
+    if (n_seq == 0) return GDN_OK;
+    if (!qkv || !conv_w || !conv_state || !a || !b || !A_log || !dt_bias || !state || !o)
+        return GDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {qkv, conv_w, conv_state, a, b, A_log, dt_bias, slot, state, o};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
+    cudaError_t e = gdn::launch_decode_fused_bf16(qkv, conv_w, conv_state, a, b, A_log, dt_bias, slot,
+                                                  n_seq, layers, Hqk, Hv, scale, state, o,
+                                                  (cudaStream_t)stream);
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
 }  // extern "C"

@@ -35,6 +35,18 @@ cudaError_t launch_decode_step(const uint16_t* q, const uint16_t* k, const uint1
                                int32_t Hv, float scale, float* state, float* o,
                                cudaStream_t stream);
 
+cudaError_t launch_decode_step_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                    const float* a, const float* b, const float* A_log,
+                                    const float* dt_bias, int32_t n_seq, int32_t layers, int32_t Hqk,
+                                    int32_t Hv, float scale, uint16_t* state, float* o,
+                                    cudaStream_t stream);
+
+cudaError_t launch_decode_fused_bf16(const uint16_t* qkv, const float* conv_w, float* conv_state,
+                                     const float* a, const float* b, const float* A_log,
+                                     const float* dt_bias, const int32_t* slot, int32_t n_seq,
+                                     int32_t layers, int32_t Hqk, int32_t Hv, float scale,
+                                     uint16_t* state, float* o, cudaStream_t stream);
+
 cudaError_t launch_decode_fused(const uint16_t* qkv, const float* conv_w, float* conv_state,
                                 const float* a, const float* b, const float* A_log,
                                 const float* dt_bias, const int32_t* slot, int32_t n_seq,

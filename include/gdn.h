@@ -252,6 +252,27 @@ gdn_status gdn_decode_step_fused(const uint16_t* qkv, const float* conv_w, float
                                  int32_t layers, int32_t Hqk, int32_t Hv, int32_t d, float scale,
                                  int32_t n_slots, float* state, float* o, gdn_stream_t stream);
 
+/*
+ * gdn_decode_step_bf16, gdn_decode_step_fused_bf16 -- gdn_decode_step and
+ * gdn_decode_step_fused with the state stored as bf16 (uint16_t bit patterns)
+ * instead of float32; every other argument as there.  The page's ~75 MB of
+ * state for 48 layers (architecture page section 2.2) is this 2-byte size.
+ * The arithmetic is float32; each updated state element is rounded to bf16
+ * (nearest even) when stored.  This halves the bytes of the step, which is
+ * bound by HBM bandwidth, at the price of one bf16 rounding of the state per
+ * token.
+ */
+gdn_status gdn_decode_step_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                const float* a, const float* b, const float* A_log,
+                                const float* dt_bias, int32_t n_seq, int32_t layers, int32_t Hqk,
+                                int32_t Hv, int32_t d, float scale, uint16_t* state, float* o,
+                                gdn_stream_t stream);
+gdn_status gdn_decode_step_fused_bf16(const uint16_t* qkv, const float* conv_w, float* conv_state,
+                                      const float* a, const float* b, const float* A_log,
+                                      const float* dt_bias, const int32_t* slot, int32_t n_seq,
+                                      int32_t layers, int32_t Hqk, int32_t Hv, int32_t d, float scale,
+                                      int32_t n_slots, uint16_t* state, float* o, gdn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -133,3 +133,14 @@ def test_fused_decode_rejects_bad_arguments(L):
     assert call(qkv=None) == 1
     assert call(state=_p(FAKE + 8)) == 3         # misaligned
     assert call(n_seq=0) == 0                    # nothing to do
+
+
+def test_bf16_state_decode_rejects_bad_arguments(L):
+    def call(d=128, Hv=48, layers=48, state=_p()):
+        return L.gdn_decode_step_bf16(_p(), _p(), _p(), _p(), _p(), _p(), _p(), 4, layers, 16, Hv, d,
+                                      0.088, state, _p(), None)
+    assert call(d=64) == 2
+    assert call(Hv=47) == 2
+    assert call(layers=0) == 1
+    assert call(state=None) == 1
+    assert call(state=_p(FAKE + 2)) == 3

@@ -72,3 +72,26 @@ def test_decode_full_size_sampled_units(orc):
     idx = torch.tensor(units, device="cuda")
     assert rel_err(host(o[idx]), o_ref) <= TOL
     assert rel_err(host(st_dev[idx]), s_ref) <= TOL
+
+
+def _bf16_state_check(got, ref):
+    """Each stored element within one bf16 rounding of the exact value."""
+    got = np.asarray(got, np.float64)
+    bound = 2.0 ** -8 * np.abs(ref) + 1e-5 * np.max(np.abs(ref))
+    bad = np.abs(got - ref) > bound
+    assert not bad.any(), f"{bad.sum()} state elements beyond one bf16 ulp"
+
+
+@pytest.mark.parametrize("Hqk,Hv", [(16, 48), (4, 8)])
+def test_decode_bf16_state(orc, Hqk, Hv):
+    """bf16-state variant: the oracle starts from the same (bf16) state values;
+    o within 1e-4, every stored state element within one bf16 rounding."""
+    import torch
+    inp = synth.make_decode(2, 3, seed=43, Hqk=Hqk, Hv=Hv)
+    st16 = torch.from_numpy(inp.full_state()).cuda().to(torch.bfloat16)
+    st_in = host(st16).astype(np.float32)
+    o = _run(inp, st16)
+    o_ref, s_ref = orc.decode(inp.q, inp.k, inp.v, inp.a, inp.b, inp.A_log, inp.dt_bias,
+                              inp.n_seq, inp.layers, st_in)
+    assert rel_err(host(o), o_ref) <= TOL
+    _bf16_state_check(host(st16), s_ref)

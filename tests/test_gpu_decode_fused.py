@@ -96,3 +96,25 @@ def test_fused_decode_identity_slots_and_determinism():
         runs.append((o, st_dev, cs_dev))
     for x, y in zip(runs[0], runs[1]):
         assert torch.equal(x, y)
+
+
+def test_fused_decode_bf16_state(orc):
+    """bf16-state variant of the fused step: o within 1e-4 of the oracle started
+    from the same bf16 state values, every stored state element within one bf16
+    rounding, the convolution history bit for bit."""
+    import torch
+    inp = synth.make_decode_fused(3, 2, 4, 75, Hqk=4, Hv=12)
+    st16 = torch.from_numpy(inp.state).cuda().to(torch.bfloat16)
+    st_in = host(st16).astype(np.float32)
+    cs_dev = dev_f32(inp.conv_state)
+    import gated_deltanet_recurrence_prefill_b200 as gdn
+    o = gdn.decode_step_fused(dev_bf16(inp.qkv), dev_f32(inp.conv_w), cs_dev, dev_f32(inp.a),
+                              dev_f32(inp.b), dev_f32(inp.A_log), dev_f32(inp.dt_bias), st16,
+                              inp.n_seq, inp.layers, inp.Hqk, inp.Hv, slot=dev_i32(inp.slot),
+                              scale=inp.scale)
+    o_ref, st_ref, cs_ref = _oracle(orc, inp, inp.qkv, inp.a, inp.b, inp.conv_state, st_in)
+    assert rel_err(host(o), o_ref) <= TOL
+    got = host(st16)
+    bound = 2.0 ** -8 * np.abs(st_ref) + 1e-5 * np.max(np.abs(st_ref))
+    assert not (np.abs(got - st_ref) > bound).any()
+    np.testing.assert_array_equal(host(cs_dev), cs_ref)
