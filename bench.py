@@ -153,13 +153,15 @@ def _dist():
     return world, rank, local
 
 
-def _time_steps(step, warmup, steps, flush, streams_events):
-    """Warm-up, then `steps` timed steps; returns per-step ms (CUDA events on the
-    current stream) and per-kernel ms lists from streams_events()."""
+def _time_steps(step, warmup, steps, flush, streams_events, world=1):
+    """Warm-up, then `steps` timed steps bracketed by a barrier and a device
+    synchronize on both sides; returns per-step ms (CUDA events on the current
+    stream) and per-kernel ms lists from streams_events()."""
     import torch
     for _ in range(warmup):
         step(None)
     torch.cuda.synchronize()
+    _barrier(world)
     times = []
     per_kernel = {}
     for _ in range(steps):
@@ -170,6 +172,7 @@ def _time_steps(step, warmup, steps, flush, streams_events):
         times.append(ev["start"].elapsed_time(ev["end"]))
         for name, (a, b) in ev.get("kernels", {}).items():
             per_kernel.setdefault(name, []).append(a.elapsed_time(b))
+    _barrier(world)
     return times, per_kernel
 
 
@@ -184,7 +187,7 @@ def bench_main(args, world, rank, local):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     peaks = load_peaks()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
@@ -228,12 +231,10 @@ def bench_main(args, world, rank, local):
             ev["kernels"]["prefill"][1].record()
             ev["end"].record()
 
-    if world > 1:
-        torch.distributed.barrier()
     torch.cuda.synchronize()
     with Clocks(local if "CUDA_VISIBLE_DEVICES" not in os.environ else _smi_index(local)) as clk:
         wall0 = time.perf_counter()
-        times, per_kernel = _time_steps(step, args.warmup, args.steps, flush, new_events)
+        times, per_kernel = _time_steps(step, args.warmup, args.steps, flush, new_events, world)
         torch.cuda.synchronize()
         wall = time.perf_counter() - wall0
     clocks = clk.summary()
@@ -260,7 +261,7 @@ def bench_main(args, world, rank, local):
 
     mk = lambda: {"start": torch.cuda.Event(enable_timing=True),
                   "end": torch.cuda.Event(enable_timing=True)}
-    e2e_times, _ = _time_steps(e2e_step, args.warmup, args.steps, flush, mk)
+    e2e_times, _ = _time_steps(e2e_step, args.warmup, args.steps, flush, mk, world)
     e2e_ms = _max_over_ranks(sum(e2e_times) / len(e2e_times), world)
     h2d = h_qkv.numel() * 2 + h_a.numel() * 4 + h_b.numel() * 4
     d2h = h_o.numel() * 4 + h_fs.numel() * 4
@@ -297,7 +298,7 @@ def bench_main(args, world, rank, local):
         extra["decode_fused_128seq_48layers"] = bench_decode_fused(args, dev, peaks, world)
         extra["decode_bf16state_128seq_48layers"] = bench_decode(args, dev, peaks, world, bf16_state=True)
 
-    value = world * T / (ms_max * 1e-3)
+    value = weak_scaling_rate(T, ms_max, world)
     line = {
         "metric": "GDN prefill tokens/s/layer (front end + chunked prefill, T=8192)",
         "value": round(value, 1), "unit": "tokens/s/layer", "n_gpus": world,
@@ -309,7 +310,7 @@ def bench_main(args, world, rank, local):
                    "T": T, "n_seq": 1, "Hqk": HQK, "Hv": HV, "d": D, "chunk": 64,
                    "l2": "flushed before every timed step (256 MiB write)",
                    "parallelism": f"replicas x{world}"},
-        "e2e": {"value": round(world * T / (e2e_ms * 1e-3), 1), "unit": "tokens/s/layer",
+        "e2e": {"value": round(weak_scaling_rate(T, e2e_ms, world), 1), "unit": "tokens/s/layer",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
                 "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": launches_per_step * args.steps,
@@ -320,7 +321,7 @@ def bench_main(args, world, rank, local):
     }
     if extra:
         line["extra"] = extra
-    if rank == 0 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
     if world > 1:
         import torch.distributed as dist
@@ -340,13 +341,28 @@ def _smi_index(local):
 
 
 def _max_over_ranks(x, world):
+    """The largest of every rank's x (a collective: all ranks call it in the same
+    order).  NCCL reduces a CUDA tensor, gloo a host one."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def weak_scaling_rate(units_per_rank, ms_per_step_max, world):
+    """Whole-job rate of `world` replicas that each process `units_per_rank` per
+    step, timed by the slowest rank (units per second)."""
+    return world * units_per_rank / (ms_per_step_max * 1e-3)
 
 
 def bench_long_prefill(args, dev, flush, peaks, world):
@@ -385,12 +401,12 @@ def bench_long_prefill(args, dev, flush, peaks, world):
 
     mk = lambda: {"start": torch.cuda.Event(enable_timing=True),
                   "end": torch.cuda.Event(enable_timing=True)}
-    times, _ = _time_steps(step, max(3, args.warmup), max(3, min(args.steps, 10)), flush, mk)
+    times, _ = _time_steps(step, max(3, args.warmup), max(3, min(args.steps, 10)), flush, mk, world)
     ms = _max_over_ranks(sum(times) / len(times), world)
     tflops = FLOP_PER_TOKEN * T / (ms * 1e-3) / 1e12
     gbs = (PREFILL_BYTES_PER_TOKEN * T + 2 * STATE_BYTES) / (ms * 1e-3) / 1e9
     out = {"workload": "gdn_prefill T=262144 N=1 Hqk=16 Hv=48 d=128 S0~N(0,0.02^2)",
-           "ms": round(ms, 4), "tokens_per_s_layer": round(world * T / (ms * 1e-3), 1),
+           "ms": round(ms, 4), "tokens_per_s_layer": round(weak_scaling_rate(T, ms, world), 1),
            "TFLOP_s": round(tflops, 2), "tensor_frac": round(tflops / peaks["bf16_tflops"], 4),
            "GB_s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
            "launches_per_step": 1}
@@ -438,7 +454,7 @@ def bench_decode(args, dev, peaks, world, bf16_state=False):
     mk = lambda: {"start": torch.cuda.Event(enable_timing=True),
                   "end": torch.cuda.Event(enable_timing=True)}
     dummy = torch.empty(1, device=dev)
-    times, _ = _time_steps(step, max(3, args.warmup), max(5, args.steps), dummy, mk)
+    times, _ = _time_steps(step, max(3, args.warmup), max(5, args.steps), dummy, mk, world)
     ms = _max_over_ranks(sum(times) / len(times), world)
     state_bytes = STATE_BYTES // 2 if bf16_state else STATE_BYTES
     bytes_step = 2 * U * state_bytes + U * (2 * 2 * HQK * D + 2 * HV * D + 2 * 4 * HV + 4 * HV * D)
@@ -490,7 +506,7 @@ def bench_decode_fused(args, dev, peaks, world):
     mk = lambda: {"start": torch.cuda.Event(enable_timing=True),
                   "end": torch.cuda.Event(enable_timing=True)}
     dummy = torch.empty(1, device=dev)
-    times, _ = _time_steps(step, max(3, args.warmup), max(5, min(args.steps, 50)), dummy, mk)
+    times, _ = _time_steps(step, max(3, args.warmup), max(5, min(args.steps, 50)), dummy, mk, world)
     ms = _max_over_ranks(sum(times) / len(times), world)
     bytes_step = (2 * U * STATE_BYTES + 2 * U * ctot * 3 * 4 + U * ctot * 2 + L * ctot * 16
                   + U * HV * (2 * 4 + 4 * D))
@@ -506,15 +522,16 @@ def bench_decode_fused(args, dev, peaks, world):
 
 # ---------------------------------------------------------------------------- CPU oracle
 
-def cpu_baseline(seconds: float = 15.0, threads: int = 0):
+def cpu_baseline(seconds: float = 15.0, threads: int = 0, fe=None):
     """The fp64 oracle, as it stands, on the host cores: the 8K workload's front
-    end plus recurrence on a sample of value heads, repeated until ~`seconds`."""
-    import numpy as np
+    end plus recurrence on a sample of value heads, repeated until ~`seconds`.
+    `fe` is the workload's input (synth.workload(1)), generated here if None."""
     import oracle
     import synth
     oracle.build()
     cores = oracle.max_threads(threads)
-    fe = synth.workload(1)
+    if fe is None:
+        fe = synth.workload(1)
     g = fe.gates
     t0 = time.perf_counter()
     q, k, v, _ = oracle.conv1d_silu(fe.qkv, fe.conv_w, None, HQK, HV, D, threads=threads)
@@ -523,7 +540,8 @@ def cpu_baseline(seconds: float = 15.0, threads: int = 0):
     heads_done = 0
     t_rec = 0.0
     h = 0
-    while heads_done < HV and (t_fe + t_rec) < seconds:
+    # at least one group of heads, however long the front end took
+    while heads_done < HV and (heads_done == 0 or (t_fe + t_rec) < seconds):
         h1 = min(HV, h + max(1, cores))
         t1 = time.perf_counter()
         oracle.prefill(q, k, v, g.a, g.b, g.A_log, g.dt_bias, heads=(h, h1), want_o=True,
@@ -583,10 +601,12 @@ def run_reference(args, world, rank):
     vals = []
     # each step is a bounded sample, sized so that the whole run stays within minutes
     per_step = max(1.0, min(args.cpu_seconds / 3, 150.0 / (args.steps + args.warmup)))
+    import synth
+    fe = synth.workload(1)
     for _ in range(args.warmup):
-        cpu_baseline(seconds=per_step)
+        cpu_baseline(seconds=per_step, fe=fe)
     for _ in range(args.steps):
-        vals.append(cpu_baseline(seconds=per_step))
+        vals.append(cpu_baseline(seconds=per_step, fe=fe))
     value = statistics.median(v["value"] for v in vals)
     line = {"impl": "reference",
             "metric": "GDN prefill tokens/s/layer (front end + chunked prefill, T=8192)",
