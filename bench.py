@@ -4,9 +4,11 @@ One step = one pass of the whole prefill path over one batch of synthetic
 input: the front end (gdn_conv1d_silu: conv1d + SiLU + L2 norm) and the chunked
 prefill (gdn_prefill) of one GDN layer, T = 8192 tokens, 16 key heads, 48 value
 heads, d = 128, zero initial state.  The metric is tokens per second per layer.
-Two secondary lines are measured in the same run and attached under "extra":
-the T = 262144 prefill (non-zero initial state) and one decode step over
-128 sequences x 48 layers with the 19.3 GB float32 state updated in place.
+Secondary lines are measured in the same run and attached under "extra": the
+T = 262144 prefill (non-zero initial state), the 16-sequence varlen prefill
+(lengths U[1024, 32768]), and one decode step over 128 sequences x 48 layers
+with the 19.3 GB float32 state updated in place (plain, with the front end
+fused, and with a bf16 state).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -294,6 +296,8 @@ def bench_main(args, world, rank, local):
     extra = {}
     if not args.primary_only:
         extra["prefill_262k"] = bench_long_prefill(args, dev, flush, peaks, world)
+        extra["prefill_varlen_16seq"] = bench_long_prefill(
+            args, dev, flush, peaks, world, lengths=synth.varlen_lengths(3), seed=3)
         extra["decode_128seq_48layers"] = bench_decode(args, dev, peaks, world)
         extra["decode_fused_128seq_48layers"] = bench_decode_fused(args, dev, peaks, world)
         extra["decode_bf16state_128seq_48layers"] = bench_decode(args, dev, peaks, world, bf16_state=True)
@@ -365,13 +369,16 @@ def weak_scaling_rate(units_per_rank, ms_per_step_max, world):
     return world * units_per_rank / (ms_per_step_max * 1e-3)
 
 
-def bench_long_prefill(args, dev, flush, peaks, world):
-    """T = 262144, one sequence, S0 ~ N(0, 0.02^2) (inputs drawn on the device)."""
+def bench_long_prefill(args, dev, flush, peaks, world, lengths=None, seed=2):
+    """One gdn_prefill launch over `lengths` (default: one sequence of T = 262144),
+    per-sequence S0 ~ N(0, 0.02^2) (inputs drawn on the device)."""
     import torch
     import gated_deltanet_recurrence_prefill_b200 as gdn
-    T = T_LONG
+    lengths = lengths or [T_LONG]
+    N = len(lengths)
+    T = sum(lengths)
     gen = torch.Generator(device=dev)
-    gen.manual_seed(2)
+    gen.manual_seed(seed)
 
     def unit(shape):
         x = torch.randn(*shape, generator=gen, device=dev)
@@ -386,16 +393,22 @@ def bench_long_prefill(args, dev, flush, peaks, world):
     A_log = torch.log(torch.empty(HV, device=dev).uniform_(1, 16, generator=gen))
     dt = torch.exp(torch.empty(HV, device=dev).uniform_(-6.907755, -2.302585, generator=gen))
     dt_bias = torch.log(torch.expm1(dt))
-    s0 = 0.02 * torch.randn(1, HV, D, D, generator=gen, device=dev)
+    s0 = 0.02 * torch.randn(N, HV, D, D, generator=gen, device=dev)
     o = torch.empty(T, HV, D, dtype=torch.float32, device=dev)
     fs = torch.empty_like(s0)
-    ws = torch.empty(gdn.prefill_workspace_size(1, T, HQK, HV, D), dtype=torch.uint8, device=dev)
+    cu = None
+    if N > 1:
+        offs = [0]
+        for n in lengths:
+            offs.append(offs[-1] + n)
+        cu = torch.tensor(offs, dtype=torch.int32, device=dev)
+    ws = torch.empty(gdn.prefill_workspace_size(N, T, HQK, HV, D), dtype=torch.uint8, device=dev)
 
     def step(ev):
         if ev:
             ev["start"].record()
-        gdn.prefill(q, k, v, a, b, A_log, dt_bias, initial_state=s0, o=o, final_state=fs,
-                    workspace=ws)
+        gdn.prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens=cu, initial_state=s0, o=o,
+                    final_state=fs, workspace=ws)
         if ev:
             ev["end"].record()
 
@@ -404,12 +417,19 @@ def bench_long_prefill(args, dev, flush, peaks, world):
     times, _ = _time_steps(step, max(3, args.warmup), max(3, min(args.steps, 10)), flush, mk, world)
     ms = _max_over_ranks(sum(times) / len(times), world)
     tflops = FLOP_PER_TOKEN * T / (ms * 1e-3) / 1e12
-    gbs = (PREFILL_BYTES_PER_TOKEN * T + 2 * STATE_BYTES) / (ms * 1e-3) / 1e9
-    out = {"workload": "gdn_prefill T=262144 N=1 Hqk=16 Hv=48 d=128 S0~N(0,0.02^2)",
+    gbs = (PREFILL_BYTES_PER_TOKEN * T + 2 * N * STATE_BYTES) / (ms * 1e-3) / 1e9
+    if N == 1:
+        wl = f"gdn_prefill T={T} N=1 Hqk=16 Hv=48 d=128 S0~N(0,0.02^2)"
+    else:
+        wl = (f"gdn_prefill varlen N={N} (lengths U[1024,32768], T={T}, longest {max(lengths)}) "
+              f"Hqk=16 Hv=48 d=128 per-sequence S0~N(0,0.02^2)")
+    out = {"workload": wl,
            "ms": round(ms, 4), "tokens_per_s_layer": round(weak_scaling_rate(T, ms, world), 1),
            "TFLOP_s": round(tflops, 2), "tensor_frac": round(tflops / peaks["bf16_tflops"], 4),
            "GB_s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
-           "launches_per_step": 1}
+           # the producer/consumer kernel runs whole sequences (48 value heads, 144
+           # CTAs) per cooperative launch when more units exist than fit at once
+           "launches_per_step": 1 if N == 1 else -(-N * HV // HV)}
     del q, k, v, a, b, o
     torch.cuda.empty_cache()
     return out
