@@ -429,7 +429,7 @@ def bench_long_prefill(args, dev, flush, peaks, world, lengths=None, seed=2):
            "GB_s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
            # the producer/consumer kernel runs whole sequences (48 value heads, 144
            # CTAs) per cooperative launch when more units exist than fit at once
-           "launches_per_step": 1 if N == 1 else -(-N * HV // HV)}
+           "launches_per_step": N}
     del q, k, v, a, b, o
     torch.cuda.empty_cache()
     return out
