@@ -32,21 +32,29 @@
 //
 // Consumer (role 0).  A loader thread bulk-loads each chunk from the ring into
 // one of two receive slots and hands ring slots back to the producers (a
-// second counter per ring slot).  Each product spans all 128 columns of d_v
-// (a tcgen05.mma takes about as long to issue at N = 64 as at N = 128, and one
-// thread issues one every ~75 cycles at best):
-//   D  = [T b; R b] V                      M128 N128 K64   (warp 1, during the epilogue before)
-//   D += [-W; Qh] S^T                      M128 N128 K128  -> [U; o / scale]
-//   S~ += K^T (kappa U / Gamma)            M128 N128 K64   (accumulates in TMEM)
-// The last two are the state chain; lane 0 of the first epilogue warp issues
-// them right after the epilogue warps' named barrier.  The float32 state lives
-// in TMEM as S~ with S = Gamma S~ (the decay gamma_C of each chunk is folded
-// into the running scalar Gamma and the update is added as kappa U / Gamma);
-// S~ is rescaled in place only when Gamma would fall below 2^-80.  A bf16 copy
-// of S is the operand of the next chunk.  o is staged in shared memory and
-// written by TMA while the state update runs (plain stores for a sequence's
-// ragged last chunk).
-// Warp 0 loads V and K by TMA.
+// second counter per ring slot).  Every product has d_v as its M dimension
+// (TMEM lane = v row) and spans 128 columns (a tcgen05.mma with M = 128 and
+// K = 16 occupies the tensor core for about the same ~150 cycles whatever N
+// is, up to 256):
+//   D^T  = V^T [T b; R b]^T                M128 N128 K64   (in the chain's gaps)
+//   D^T += S [-W; Qh]^T                    M128 N128 K128  -> [U^T | o^T / scale]
+//   S~  += (kappa U / Gamma)^T K           M128 N128 K64   (accumulates in TMEM)
+// The last two are the state chain, issued by one thread; the first by another
+// thread, in two halves placed so that they run while the chain's epilogues
+// would leave the tensor core idle (a thread that issues a tcgen05.mma is held
+// until the tensor core takes it, so each issuer has a thread of its own).  The
+// chain's A operands, S and (kappa U / Gamma)^T in bf16, are written by the
+// epilogue threads straight into TMEM, so the chain keeps off shared memory;
+// S is converted in four column blocks, each reported on its own mbarrier, so
+// that the chain's first K steps start while the rest is converted.  The
+// float32 state lives in TMEM as S~ with S = Gamma S~ (the decay gamma_C of
+// each chunk is folded into the running scalar Gamma and the update is added
+// as kappa U / Gamma); S~ is rescaled in place only when Gamma would fall
+// below 2^-80.  o^T / scale is read back while the state update runs and
+// stored straight to global memory (for each token a warp writes 32
+// consecutive floats).  D has two buffers so that the next chunk's [U'; O']
+// product can start before this chunk's epilogues are done.
+// Warp 0 loads V and K by TMA (two buffers each).
 //
 // Grid.  For nu units, blocks [0, nu) are the consumers and blocks
 // [nu, (1 + P) nu) the producers (block b serves unit b % nu).  They wait
@@ -92,7 +100,7 @@ using namespace tile;
 
 constexpr int kD = 128;
 constexpr int kC = 64;
-constexpr int kWarps = 20;
+constexpr int kWarps = 21;
 constexpr int kThreads = kWarps * 32;
 constexpr int kGroupThreads = 256;
 constexpr int kLdF = 68;                       // fp32 solve scratch row stride
@@ -137,11 +145,8 @@ constexpr uint32_t GATES_AT = 16384;                        // kappa[64], gamma_
 constexpr uint32_t GATE_BYTES = 512;
 constexpr uint32_t C_RECV = 0;                              // 2 slots
 constexpr uint32_t C_V = C_RECV + 2 * SLOT_BYTES;           // V: 2 buffers of 2 panels of 64 x 64 bf16
-constexpr uint32_t C_K = C_V + 2 * 16384;                   // K: 2 panels of 64 x 64 bf16
-constexpr uint32_t C_ST = C_K + 16384;                      // S^T bf16: 2 halves of 128 x 64
-constexpr uint32_t C_UK = C_ST + 32768;                     // kappa U / Gamma: 2 halves of 64 x 64
-constexpr uint32_t C_OST = C_UK + 16384;                    // o staging: 4 boxes of 64 x 32 f32
-constexpr uint32_t C_GATES = C_OST + 32768;                 // 2 gate buffers
+constexpr uint32_t C_K = C_V + 2 * 16384;                   // K: 2 buffers of 2 panels of 64 x 64 bf16
+constexpr uint32_t C_GATES = C_K + 2 * 16384;               // 2 gate buffers
 constexpr uint32_t C_END = C_GATES + 2 * GATE_BYTES;
 // what one chunk sends: the [-W; Qh] tile (staged in place of [K; Q]) and the
 // [T b; R b] tile with the gates (staged in the A scratch)
@@ -173,36 +178,42 @@ enum {
     PB_KQ_FULL = 0, PB_KQ_TAKEN = 2, PB_KQ_EMPTY = 4, PB_D0_FULL = 7, PB_R_FULL = 9,
     PB_X1_FULL = 11, PB_DRAIN = 13, PB_STAGED = 15, PB_AF_FREE = 17,
     // consumer
-    CB_RECV_FULL = 19, CB_K_FULL = 21, CB_K_EMPTY, CB_V_FULL = 23, CB_V_EMPTY = 25, CB_SLOT_FREE = 27,
-    CB_D_FULL = 29, CB_S_FULL, CB_DRAIN, CB_E_FULL, CB_E_DRAIN, CB_REL_DONE = 34,
-    kNumBars = 36
+    CB_RECV_FULL = 19, CB_K_FULL = 21, CB_V_FULL = 23, CB_V_EMPTY = 25, CB_SLOT_FREE = 27,
+    CB_D_FULL = 29, CB_S_FULL = 30, CB_DRAIN = 31, CB_REL_DONE = 32, CB_K_EMPTY = 34,
+    CB_EPI1_DONE = 36, CB_EPI2_BLK = 37, CB_E_FULL = 41, CB_E_DRAIN, CB_CHAIN_ISSUED, CB_SUPD_ISSUED,
+    kNumBars = 45
 };
 constexpr uint32_t SMEM_BYTES = OFF_BARS + kNumBars * 8;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;           // room to align the base
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget of one CTA");
 
 // TMEM columns.  Producer group g: D0 (64), R (64), X1 (128) at 256 g.
-// Consumer: D = [U'; O'] + [-W; Qh] S^T (rows [U; o / scale], d_v columns) at
-// 0, S~ (d_k x d_v) at 256.
+// Consumer (lane = d_v row everywhere): D^T = [U'; O']^T + S [-W; Qh]^T
+// (columns U^T | o^T / scale) at 0 and 128 (alternate chunks), S~ (d_v x d_k)
+// at 256, the bf16 A operands S (64 columns of pairs) at 384 and
+// (kappa U / Gamma)^T (32 columns) at 448.
 constexpr uint32_t PCOL_D0 = 0, PCOL_R = 64, PCOL_X1 = 128;
-constexpr uint32_t CCOL_D = 0, CCOL_S = 256;
+constexpr uint32_t CCOL_D = 0, CCOL_S = 256, CCOL_AS = 384, CCOL_AU = 448;
+constexpr uint32_t kDCols = 128;               // D has two buffers: chunk c uses CCOL_D + (c & 1) kDCols
 constexpr uint32_t TMEM_COLS = 512;
 
 constexpr uint32_t IDESC_D0 = idesc_bf16(128, 64, false, false);
 constexpr uint32_t IDESC_R = idesc_bf16(128, 64, false, true);
 constexpr uint32_t IDESC_X1 = idesc_bf16(128, 128, false, true);
-// consumer products over all of d_v: A K-major or MN-major, B MN-major
-constexpr uint32_t IDESC_N128_KM = idesc_bf16(128, 128, false, true);
-constexpr uint32_t IDESC_N128_MM = idesc_bf16(128, 128, true, true);
-// consumer warps: 0 TMA (V, K), 1 the [U'; O'] products, 2 ring loader and
-// TMEM allocation, then sixteen epilogue / chain product warps, then the ring
-// slot release
+// consumer products, M = d_v: [U'; O']^T = V^T [T b; R b]^T (A = V^T MN-major,
+// B K-major), S [-W; Qh]^T (A in TMEM, B K-major), (kappa U / Gamma)^T K (A in
+// TMEM, B = K MN-major)
+constexpr uint32_t IDESC_UO = idesc_bf16(128, 128, true, false);
+constexpr uint32_t IDESC_CHAIN = idesc_bf16(128, 128, false, false);
+constexpr uint32_t IDESC_SUPD = idesc_bf16(128, 128, false, true);
+// consumer warps: 0 TMA (V, K), 1 the state chain's products, 2 ring loader and
+// TMEM allocation, then sixteen epilogue warps, then the ring slot release and
+// the [U'; O'] products
 constexpr int kEpiWarp0 = 3;
 constexpr int kEpiThreads = 16 * 32;
 constexpr int kRelWarp = kEpiWarp0 + kEpiThreads / 32;     // ring slot release
-static_assert(kRelWarp < kWarps, "consumer warps");
-constexpr int kEpiBar = 1;                     // named barrier of the epilogue warps
-constexpr int kOutBar = 2;                     // named barrier of their o-row half
+constexpr int kUoWarp = kRelWarp + 1;                      // [U'; O'] products
+static_assert(kUoWarp < kWarps, "consumer warps");
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;    // 2 s: far beyond any legitimate wait
 constexpr float kLog2e = 1.4426950408889634f;
@@ -234,7 +245,6 @@ struct Ctx {
     uint32_t sbase;
     uint32_t tmem;
     volatile int* abort;
-    volatile int* mma2_issued;   // consumer: chunks whose state update has been issued
     int warp, lane;
     int h, g;              // value head, key head
     uint8_t* ring;         // this unit's ring slots
@@ -249,30 +259,20 @@ struct Ctx {
     TC_DEVICE uint32_t bar(int i) const { return bar0 + 8u * (uint32_t)i; }
 };
 
-// a counter in shared memory handed between two threads of the CTA
-__device__ __forceinline__ int ld_acquire_cta_s32(volatile int* p) {
-    int v;
-    asm volatile("ld.acquire.cta.shared.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32((const void*)p)) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_release_cta_s32(volatile int* p, int v) {
-    asm volatile("st.release.cta.shared.b32 [%0], %1;" ::"r"(smem_u32((const void*)p)), "r"(v) : "memory");
-}
-
 // ================================================================ consumer
 __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                                         const CUtensorMap* tm_o, const ClParams& p) {
+                                         const ClParams& p) {
     const int warp = x.warp, lane = x.lane;
     const int nch = x.nch;
     if (warp == 0) {
         // ------------------------------------------------ TMA: V and K of each chunk
-        // V(c) goes to buffer c & 1 (free once the [U'; O'] product of chunk
-        // c - 2 has read it), so that it lands well before that product; K(c)
-        // has one buffer, needed by the state update at the end of chunk c.
+        // V(c) and K(c) go to buffers c & 1; V is free once the [U'; O'] product
+        // of chunk c - 2 has read it, K once the state update of chunk c - 2 has,
+        // so that both land well before they are needed.
         if (lane == 0) {
             prefetch_tmap(tm_k);
             prefetch_tmap(tm_v);
-            int issued = 0;
+            int nv = 0, nk = 0;
             for (int c = 0; c < nch; ++c) {
                 const int32_t y = (int32_t)(x.bos + (int64_t)c * kC);
                 const int vb = c & 1;
@@ -282,57 +282,21 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
                 mbar_arrive_expect_tx(x.bar(CB_V_FULL + vb), 16384);
                 tma_load_2d(x.sbase + C_V + vb * 16384, tm_v, x.h * kD, y, x.bar(CB_V_FULL + vb));
                 tma_load_2d(x.sbase + C_V + vb * 16384 + 8192, tm_v, x.h * kD + 64, y, x.bar(CB_V_FULL + vb));
-                if (c >= 1 && !mbar_wait(x.bar(CB_K_EMPTY), (c - 1) & 1, x.abort, kWaitLimitNs)) {
-                    issued = -(c + 1);           // V of chunk c is in flight, K is not
+                nv = c + 1;
+                if (c >= 2 && !mbar_wait(x.bar(CB_K_EMPTY + vb), ((c >> 1) - 1) & 1, x.abort, kWaitLimitNs))
                     break;
-                }
                 TRACE_CLK(29, c);
-                mbar_arrive_expect_tx(x.bar(CB_K_FULL), 16384);
-                tma_load_2d(x.sbase + C_K, tm_k, x.g * kD, y, x.bar(CB_K_FULL));
-                tma_load_2d(x.sbase + C_K + 8192, tm_k, x.g * kD + 64, y, x.bar(CB_K_FULL));
-                issued = c + 1;
+                mbar_arrive_expect_tx(x.bar(CB_K_FULL + vb), 16384);
+                tma_load_2d(x.sbase + C_K + vb * 16384, tm_k, x.g * kD, y, x.bar(CB_K_FULL + vb));
+                tma_load_2d(x.sbase + C_K + vb * 16384 + 8192, tm_k, x.g * kD + 64, y, x.bar(CB_K_FULL + vb));
+                nk = c + 1;
             }
             // copies still in flight land before the CTA may exit
             volatile int no_abort = 0;
-            const int nv = issued >= 0 ? issued : -issued, nk = issued >= 0 ? issued : -issued - 1;
             for (int c = nv >= 2 ? nv - 2 : 0; c < nv; ++c)
                 mbar_wait(x.bar(CB_V_FULL + (c & 1)), (c >> 1) & 1, &no_abort, kWaitLimitNs);
-            if (nk >= 1) mbar_wait(x.bar(CB_K_FULL), (nk - 1) & 1, &no_abort, kWaitLimitNs);
-        }
-    } else if (warp == 1) {
-        // ------------------------------------------------ [U'; O'] = [T b; R b] V per chunk
-        // State-independent: it starts chunk c's accumulator D (the chain's
-        // [-W; Qh] S^T is added to it), once the state update of chunk c - 1
-        // has been issued (the epilogues are then done with D), so that it runs
-        // while the tensor core would otherwise wait for the second epilogue,
-        // and its issue does not compete with the chain's.
-        if (lane == 0) {
-            const uint64_t dsc_rt0 = sdesc_sw128(x.sbase + C_RECV + SL_RT2, 16, 1024);
-            const uint64_t dsc_v = sdesc_sw128(x.sbase + C_V, 8192, 1024);
-            for (int c = 0; c < nch; ++c) {
-                const int b = c & 1;
-                if (!mbar_wait(x.bar(CB_RECV_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs)) break;
-                if (!mbar_wait(x.bar(CB_V_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs)) break;
-                if (c >= 1) {
-                    // bounded wait on the issuer's counter (shared memory)
-                    const uint64_t t0 = globaltimer_ns();
-                    while (ld_acquire_cta_s32(x.mma2_issued) < c && !*x.abort)
-                        if (globaltimer_ns() - t0 > kWaitLimitNs) *x.abort = 1;
-                    if (*x.abort) break;
-                }
-                TRACE_CLK(14, c);
-                tc_fence_after();
-                const uint64_t a = dsc_rt0 + b * (uint64_t)(SLOT_BYTES >> 4);
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_bf16(x.tmem + CCOL_D, a + kk * 2, dsc_v + b * (16384 >> 4) + kk * 128, IDESC_N128_KM,
-                             kk > 0);
-                mma_commit(x.bar(CB_E_FULL));
-                mma_commit(x.bar(CB_V_EMPTY + b));
-                TRACE_CLK(15, c);
-            }
-            volatile int no_abort = 0;
-            mma_commit(x.bar(CB_E_DRAIN));
-            mbar_wait(x.bar(CB_E_DRAIN), 0, &no_abort, kWaitLimitNs);
+            for (int c = nk >= 2 ? nk - 2 : 0; c < nk; ++c)
+                mbar_wait(x.bar(CB_K_FULL + (c & 1)), (c >> 1) & 1, &no_abort, kWaitLimitNs);
         }
     } else if (warp == kRelWarp) {
         // ------------------------------------------------ ring slots back to the producers
@@ -385,181 +349,241 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
             for (int c = loaded >= 2 ? loaded - 2 : 0; c < loaded; ++c)
                 mbar_wait(x.bar(CB_RECV_FULL + (c & 1)), (c >> 1) & 1, &no_abort, kWaitLimitNs);
         }
+    } else if (warp == 1) {
+        // ------------------------------------------------ the state chain's products
+        // Per chunk c: D(c) += S [-W; Qh]^T, its K steps issued block by block as
+        // the second epilogue of chunk c - 1 turns S into the bf16 operand (so
+        // the tensor core starts on S's first 32 columns while the others are
+        // converted); then, once the first epilogue of c is done,
+        // S~ += (kappa U / Gamma)^T K.  A thread is held up while the tensor core
+        // works through the products it has issued, so the [U'; O'] products
+        // have a thread of their own (warp kUoWarp).
+        if (lane == 0) {
+            const uint64_t dsc_qw0 = sdesc_sw128(x.sbase + C_RECV + SL_QW, 16, 1024);
+            const uint64_t dsc_k = sdesc_sw128(x.sbase + C_K, 8192, 1024);
+            constexpr uint64_t kSlotStep = SLOT_BYTES >> 4;
+            for (int c = 0; c < nch && !*x.abort; ++c) {
+                const int b = c & 1;
+                if (!mbar_wait(x.bar(CB_RECV_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs) ||
+                    !mbar_wait(x.bar(CB_E_FULL), c & 1, x.abort, kWaitLimitNs))
+                    break;
+                const uint64_t bq = dsc_qw0 + b * kSlotStep;
+                bool ok = true;
+                for (int j = 0; j < 4 && ok; ++j) {
+                    // columns 32 j .. 32 j + 31 of the bf16 S: K steps 2 j, 2 j + 1
+                    ok = mbar_wait(x.bar(CB_EPI2_BLK + j), c & 1, x.abort, kWaitLimitNs);
+                    if (!ok) break;
+                    tc_fence_after();
+                    for (int kk = 2 * j; kk < 2 * j + 2; ++kk)
+                        mma_bf16_ta(x.tmem + CCOL_D + b * kDCols, x.tmem + CCOL_AS + kk * 8,
+                                    bq + (((kk >> 2) * KQ_PANEL + (kk & 3) * 32) >> 4), IDESC_CHAIN, 1);
+                }
+                if (!ok) break;
+                mma_commit(x.bar(CB_D_FULL));
+                mbar_arrive(x.bar(CB_CHAIN_ISSUED));
+                TRACE_CLK(0, c);
+                if (!mbar_wait(x.bar(CB_EPI1_DONE), c & 1, x.abort, kWaitLimitNs)) break;
+                TRACE_CLK(4, c);
+                if (!mbar_wait(x.bar(CB_K_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs)) break;
+                tc_fence_after();
+                const uint64_t bk = dsc_k + b * (16384 >> 4);
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16_ta(x.tmem + CCOL_S, x.tmem + CCOL_AU + kk * 8, bk + kk * 128, IDESC_SUPD, 1);
+                mma_commit(x.bar(CB_S_FULL));
+                mma_commit(x.bar(CB_K_EMPTY + b));
+                mbar_arrive(x.bar(CB_SUPD_ISSUED));
+                TRACE_CLK(5, c);
+                // receive slot b has been read: its products are complete (the
+                // first epilogue waited for them) and so are the epilogues' reads
+                // of its gates
+                mbar_arrive(x.bar(CB_SLOT_FREE + b));
+            }
+            volatile int no_abort = 0;
+            mma_commit(x.bar(CB_DRAIN));
+            mbar_wait(x.bar(CB_DRAIN), 0, &no_abort, kWaitLimitNs);
+        }
+    } else if (warp == kUoWarp) {
+        // ------------------------------------------------ [U'; O']^T = V^T [T b; R b]^T per chunk
+        // State-independent: it starts chunk c's accumulator D (buffer c & 1).
+        // Its K steps fill the two gaps the chain leaves on the tensor core:
+        // tokens 0-31 once chunk c - 1's chain product is issued (they run during
+        // its first epilogue), tokens 32-63 once chunk c - 1's state update is
+        // issued (they run during its second epilogue).  By the first point the
+        // epilogues of chunk c - 2 are done with buffer c & 1.
+        if (lane == 0) {
+            const uint64_t dsc_rt0 = sdesc_sw128(x.sbase + C_RECV + SL_RT2, 16, 1024);
+            const uint64_t dsc_v = sdesc_sw128(x.sbase + C_V, 8192, 1024);
+            for (int c = 0; c < nch; ++c) {
+                const int b = c & 1;
+                if (!mbar_wait(x.bar(CB_RECV_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs) ||
+                    !mbar_wait(x.bar(CB_V_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs))
+                    break;
+                const uint64_t bt = dsc_rt0 + b * (uint64_t)(SLOT_BYTES >> 4);
+                const uint64_t av = dsc_v + b * (16384 >> 4);
+                bool ok = true;
+                for (int half = 0; half < 2 && ok; ++half) {
+                    if (c >= 1)
+                        ok = mbar_wait(x.bar(half == 0 ? CB_CHAIN_ISSUED : CB_SUPD_ISSUED), (c - 1) & 1, x.abort,
+                                       kWaitLimitNs);
+                    if (!ok) break;
+                    tc_fence_after();
+                    for (int kk = 2 * half; kk < 2 * half + 2; ++kk)
+                        mma_bf16(x.tmem + CCOL_D + b * kDCols, av + kk * 128, bt + kk * 2, IDESC_UO, kk > 0);
+                }
+                if (!ok) break;
+                mma_commit(x.bar(CB_E_FULL));
+                mma_commit(x.bar(CB_V_EMPTY + b));
+                TRACE_CLK(15, c);
+            }
+            volatile int no_abort = 0;
+            mma_commit(x.bar(CB_E_DRAIN));
+            mbar_wait(x.bar(CB_E_DRAIN), 0, &no_abort, kWaitLimitNs);
+        }
     } else if (warp >= kEpiWarp0 && warp < kEpiWarp0 + kEpiThreads / 32) {
-        // ------------------------------------------------ products and epilogues
-        // Sixteen warps: warp w reads TMEM lane quadrant w % 4 (the hardware
-        // rule) and columns 32 cb .. 32 cb + 31, cb = (w - kEpiWarp0) / 4, of
-        // the 128-column accumulators; thread = one row.  Lane 0 of one of
-        // them issues every tensor-core product itself, right after the
-        // group's named barrier, so that no other warp sits between an epilogue
-        // and the next product of the state chain.  Each product covers all
-        // 128 columns of d_v in one instruction per 16-deep K step (a
-        // tcgen05.mma costs about the same to issue at N = 64 as at N = 128).
-        // After an abort the waits fall through and the issuer skips its
-        // products, but every thread still passes every named barrier.
+        // ------------------------------------------------ epilogues
+        // Every product has d_v as its M dimension, so TMEM lane = v row: warp w
+        // reads lane quadrant q = w % 4 (the hardware rule); thread = one v row.
+        // The four warps of a quadrant split the columns: warp (q, cb), cb =
+        // (w - kEpiWarp0) / 4, takes tokens 16 cb .. 16 cb + 15 of U^T and of
+        // o^T, state columns 32 cb .. 32 cb + 31 for the rescale and the final
+        // state, and columns 32 j + 8 cb .. + 7 of block j when S is turned
+        // into the bf16 operand.  The bf16 operands of the chain, S and
+        // (kappa U / Gamma)^T, go straight to TMEM, where the tensor core reads
+        // them (A operand):
+        //   D^T  = [U'; O']^T + S [-W; Qh]^T      columns U^T (0-63), o^T / scale (64-127)
+        //   S~  += (kappa U / Gamma)^T K
+        // Each warp reports each finished part to the issuing thread on an
+        // mbarrier (one arrival per warp).  After an abort the waits fall
+        // through; every warp still makes every arrival.
         const int q = warp & 3;                    // TMEM lane quadrant
-        const int cb = (warp - kEpiWarp0) >> 2;    // 32-column block
-        const int r = q * 32 + lane;               // TMEM lane = row
-        // the issuer reads a U row (quadrant 0), so it has no o rows to write out
-        const bool issuer = (warp == kEpiWarp0 + 1 && lane == 0);
+        const int cb = (warp - kEpiWarp0) >> 2;    // column share
+        const int v = q * 32 + lane;               // d_v row
+        const bool tracer = (warp == kEpiWarp0 + 1 && lane == 0);
         const uint32_t tl = x.tmem + ((uint32_t)(q * 32) << 16);
-        const uint32_t dcol = CCOL_D + cb * 32, scol = CCOL_S + cb * 32;
-        const int hh = cb >> 1, ch0 = (cb & 1) * 4;   // d_v half and first 16-byte chunk in it
-        uint8_t* st_tile = x.sm + C_ST + hh * 16384;
-        uint8_t* uk_tile = x.sm + C_UK + hh * 8192;
-        // shared-memory descriptors, computed once; a K step adds a byte offset
-        // (>> 4) to the start address field
-        const uint64_t dsc_qw0 = sdesc_sw128(x.sbase + C_RECV + SL_QW, 16, 1024);
-        const uint64_t dsc_st = sdesc_sw128(x.sbase + C_ST, 16384, 1024);
-        const uint64_t dsc_k = sdesc_sw128(x.sbase + C_K, 8192, 1024);
-        const uint64_t dsc_uk = sdesc_sw128(x.sbase + C_UK, 8192, 1024);
-        constexpr uint64_t kSlotStep = SLOT_BYTES >> 4;
-        // initial state: thread r holds d_k row r of S^T over 32 v-columns
+        const int64_t o_stride = (int64_t)p.Hv * kD;
+        auto report = [&](int bar) {
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(x.bar(bar));
+        };
+        // initial state: S~ = S0 (Gamma = 1) on columns 32 cb .. + 31, and its
+        // bf16 copy (all four blocks reported at once)
         {
             float sv[32];
-            for (int j = 0; j < 32; ++j) {
-                const int vcol = cb * 32 + j;
-                sv[j] = p.s_in ? p.s_in[x.state_off + (int64_t)vcol * kD + r] : 0.f;
+            if (p.s_in) {
+                const float4* src = reinterpret_cast<const float4*>(p.s_in + x.state_off + (int64_t)v * kD + cb * 32);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float4 t4 = src[j];
+                    sv[4 * j] = t4.x; sv[4 * j + 1] = t4.y; sv[4 * j + 2] = t4.z; sv[4 * j + 3] = t4.w;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) sv[j] = 0.f;
             }
-            tmem_st32(tl + scol, sv);
-            for (int j = 0; j < 4; ++j) st_bf16x8(st_tile, r, ch0 + j, sv + 8 * j);
+            tmem_st32(tl + CCOL_S + cb * 32, sv);
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(sv[2 * j], sv[2 * j + 1]);
+            tmem_st16u(tl + CCOL_AS + cb * 16, pk);
             tmem_st_wait();
-            fence_async_smem();
             tc_fence_before();
-            named_bar_sync(kEpiBar, kEpiThreads);
+            __syncwarp();
+            if (lane == 0)
+                for (int j = 0; j < 4; ++j) mbar_arrive(x.bar(CB_EPI2_BLK + j));
         }
         float Gam = 1.f;                           // S = Gam * S~ (same value in every thread)
         for (int c = 0; c < nch; ++c) {
             const int b = c & 1;
             const float* kap = reinterpret_cast<const float*>(x.sm + C_GATES + b * GATE_BYTES);
             const int64_t tok0 = x.bos + (int64_t)c * kC;
-            // ---- [U; o / scale] = [U'; O'] + [-W; Qh] S^T: the second term here, the
-            //      first (E) from warp 1
-            if (issuer && !*x.abort &&
-                mbar_wait(x.bar(CB_RECV_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs) &&
-                mbar_wait(x.bar(CB_E_FULL), c & 1, x.abort, kWaitLimitNs)) {
-                // D holds [U'; O'] (complete: its commit was seen); add [-W; Qh] S^T
-                tc_fence_after();
-                const uint64_t a = dsc_qw0 + b * kSlotStep;
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_bf16(x.tmem + CCOL_D, a + (((kk >> 2) * KQ_PANEL + (kk & 3) * 32) >> 4),
-                             dsc_st + kk * 128, IDESC_N128_KM, 1);
-                mma_commit(x.bar(CB_D_FULL));
-                TRACE_CLK(0, c);
-            }
+            const uint32_t dbuf = CCOL_D + b * kDCols;
             mbar_wait(x.bar(CB_RECV_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs);
-            if (issuer) TRACE_CLK(1, c);
-            mbar_wait(x.bar(CB_D_FULL), c & 1, x.abort, kWaitLimitNs);
-            if (issuer) TRACE_CLK(2, c);
-            tc_fence_after();
             const float Gn = Gam * kap[64];        // scale of the state after this chunk
             const bool resc = !(Gn >= kMinGamma);
-            const float inv = resc ? 1.f : 1.f / Gn;
-            // rows 0-63 (q < 2) hold U_t: kappa_t U_t / Gamma becomes the update
-            // operand, written before the barrier.  Rows 64-127 hold o_t / scale:
-            // kept in registers and written out after the barrier, while the
-            // state update runs.
-            float ov[32];
-            tmem_ld32(tl + dcol, ov);
-            tmem_ld_wait();
-            if (q < 2) {
-                const float sc = kap[r] * inv;
-                float e[32];
-                for (int j = 0; j < 32; ++j) e[j] = ov[j] * sc;
-                for (int j = 0; j < 4; ++j) st_bf16x8(uk_tile, r, ch0 + j, e + 8 * j);
+            const float inv = resc ? 1.f : __frcp_rn(Gn);
+            if (tracer) TRACE_CLK(1, c);
+            mbar_wait(x.bar(CB_D_FULL), c & 1, x.abort, kWaitLimitNs);
+            if (tracer) TRACE_CLK(2, c);
+            tc_fence_after();
+            {
+                // U^T, tokens t = 16 cb .. 16 cb + 15 -> (kappa_t U_t / Gamma)^T in bf16
+                float uv[16];
+                tmem_ld16(tl + dbuf + cb * 16, uv);
+                tmem_ld_wait();
+                const float4* k4 = reinterpret_cast<const float4*>(kap + cb * 16);
+                uint32_t pk[8];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float4 kv = k4[j];
+                    pk[2 * j] = pack_bf16x2(uv[4 * j] * (kv.x * inv), uv[4 * j + 1] * (kv.y * inv));
+                    pk[2 * j + 1] = pack_bf16x2(uv[4 * j + 2] * (kv.z * inv), uv[4 * j + 3] * (kv.w * inv));
+                }
+                tmem_st8u(tl + CCOL_AU + cb * 8, pk);
             }
             if (resc) {
                 // S~ <- Gn S~ on this thread's 32 columns (Gamma restarts at 1)
                 float sv[32];
-                tmem_ld32(tl + scol, sv);
+                tmem_ld32(tl + CCOL_S + cb * 32, sv);
                 tmem_ld_wait();
+#pragma unroll
                 for (int j = 0; j < 32; ++j) sv[j] *= Gn;
-                tmem_st32(tl + scol, sv);
-                tmem_st_wait();
+                tmem_st32(tl + CCOL_S + cb * 32, sv);
             }
-            fence_async_smem();
-            tc_fence_before();
-            if (issuer) TRACE_CLK(3, c);
-            named_bar_sync(kEpiBar, kEpiThreads);
-            if (issuer) TRACE_CLK(4, c);
-            if (issuer) {
-                // D, E and the receive slot's gates have been read by every thread
-                mbar_arrive(x.bar(CB_SLOT_FREE + b));
-                // ---- S~ += K^T (kappa U / Gamma)
-                if (!*x.abort && mbar_wait(x.bar(CB_K_FULL), c & 1, x.abort, kWaitLimitNs)) {
-                    TRACE_CLK(27, c);
-                    tc_fence_after();
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16(x.tmem + CCOL_S, dsc_k + kk * 128, dsc_uk + kk * 128, IDESC_N128_MM, 1);
-                    mma_commit(x.bar(CB_S_FULL));
-                    mma_commit(x.bar(CB_K_EMPTY));
-                }
-                // D may be restarted now by the next chunk's [U'; O'] product (warp 1)
-                st_release_cta_s32(x.mma2_issued, c + 1);
-                TRACE_CLK(5, c);
-            }
-            if (q >= 2) {
-                // o rows, while the state update runs.  A whole chunk is staged
-                // (four 32-column boxes, 128-byte swizzle) and written by TMA; the
-                // ragged end of a sequence is stored directly (rows past its end
-                // belong to the next sequence).
-                const int t = r - 64;
-                const bool elected = (warp == kEpiWarp0 + 3 && lane == 0);
-                if (tok0 + kC <= x.eos) {
-                    uint8_t* ost = x.sm + C_OST + cb * 8192;
-                    if (elected) bulk_wait_read();      // the previous chunk's stores have read the staging
-                    named_bar_sync(kOutBar, kEpiThreads / 2);
-                    for (int j = 0; j < 8; ++j)
-                        *reinterpret_cast<float4*>(ost + sw128_off(t, j)) =
-                            make_float4(p.scale * ov[4 * j], p.scale * ov[4 * j + 1], p.scale * ov[4 * j + 2],
-                                        p.scale * ov[4 * j + 3]);
-                    fence_async_smem();
-                    named_bar_sync(kOutBar, kEpiThreads / 2);
-                    if (elected) {
-                        for (int bx = 0; bx < 4; ++bx)
-                            tma_store_2d(tm_o, x.h * kD + bx * 32, (int32_t)tok0, x.sbase + C_OST + bx * 8192);
-                        bulk_commit();
-                    }
-                } else if (tok0 + t < x.eos) {
-                    float* orow = p.o + ((tok0 + t) * p.Hv + x.h) * kD + cb * 32;
-                    for (int j = 0; j < 32; j += 4)
-                        *reinterpret_cast<float4*>(orow + j) =
-                            make_float4(p.scale * ov[j], p.scale * ov[j + 1], p.scale * ov[j + 2], p.scale * ov[j + 3]);
+            if (tracer) TRACE_CLK(3, c);
+            report(CB_EPI1_DONE);
+            {
+                // o^T / scale, tokens t = 16 cb .. 16 cb + 15, written while the state
+                // update runs; for each t a warp stores 32 consecutive floats of o.
+                // Rows past the sequence's end belong to the next sequence.
+                float ov[16];
+                tmem_ld16(tl + dbuf + 64 + cb * 16, ov);
+                tmem_ld_wait();
+                const int64_t t0 = tok0 + cb * 16;
+                float* ocol = p.o + t0 * o_stride + x.h * kD + v;
+                const int64_t nvalid = x.eos - t0;
+                if (nvalid >= 16) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) ocol[j * o_stride] = p.scale * ov[j];
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (j < nvalid) ocol[j * o_stride] = p.scale * ov[j];
                 }
             }
             Gam = resc ? 1.f : Gn;
             // ---- new state -> bf16 operand of the next chunk (and the final state)
-            if (issuer) TRACE_CLK(6, c);
+            if (tracer) TRACE_CLK(6, c);
             mbar_wait(x.bar(CB_S_FULL), c & 1, x.abort, kWaitLimitNs);
-            if (issuer) TRACE_CLK(7, c);
+            if (tracer) TRACE_CLK(7, c);
             tc_fence_after();
-            const bool last = (c == nch - 1);
-            {
-                float sv[32];
-                tmem_ld32(tl + scol, sv);
-                tmem_ld_wait();
-                for (int j = 0; j < 32; ++j) sv[j] *= Gam;
-                if (!last) {
-                    for (int j = 0; j < 4; ++j) st_bf16x8(st_tile, r, ch0 + j, sv + 8 * j);
-                } else if (p.s_out) {
-                    for (int j = 0; j < 32; ++j)
-                        p.s_out[x.state_off + (int64_t)(cb * 32 + j) * kD + r] = sv[j];
+            if (c == nch - 1) {
+                if (p.s_out) {
+                    float sv[32];
+                    tmem_ld32(tl + CCOL_S + cb * 32, sv);
+                    tmem_ld_wait();
+                    float4* dst = reinterpret_cast<float4*>(p.s_out + x.state_off + (int64_t)v * kD + cb * 32);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j)
+                        dst[j] = make_float4(Gam * sv[4 * j], Gam * sv[4 * j + 1], Gam * sv[4 * j + 2],
+                                             Gam * sv[4 * j + 3]);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float sv[8];
+                    tmem_ld8(tl + CCOL_S + 32 * j + 8 * cb, sv);
+                    tmem_ld_wait();
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) pk[e] = pack_bf16x2(Gam * sv[2 * e], Gam * sv[2 * e + 1]);
+                    tmem_st4u(tl + CCOL_AS + 16 * j + 4 * cb, pk);
+                    report(CB_EPI2_BLK + j);
                 }
             }
-            if (!last) {
-                fence_async_smem();
-                tc_fence_before();
-                if (issuer) TRACE_CLK(8, c);
-                named_bar_sync(kEpiBar, kEpiThreads);
-                if (issuer) TRACE_CLK(9, c);
-            }
+            if (tracer) TRACE_CLK(8, c);
         }
-        if (issuer) {
-            volatile int no_abort = 0;
-            mma_commit(x.bar(CB_DRAIN));
-            mbar_wait(x.bar(CB_DRAIN), 0, &no_abort, kWaitLimitNs);
-        }
-        if (warp == kEpiWarp0 + 3 && lane == 0) bulk_wait();     // the last o stores are complete
     }
 }
 
@@ -977,8 +1001,7 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_pc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
-                  const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_o,
-                  const ClParams p) {
+                  const __grid_constant__ CUtensorMap tm_b, const ClParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // align to 1024 bytes by pointer arithmetic on the shared array, so that
     // every access below stays in the shared state space
@@ -989,7 +1012,6 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     x.bar0 = x.sbase + OFF_BARS;
     x.abort = reinterpret_cast<volatile int*>(sm + OFF_MISC);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC + 4);
-    x.mma2_issued = reinterpret_cast<volatile int*>(sm + OFF_MISC + 40);
     x.warp = threadIdx.x >> 5;
     x.lane = threadIdx.x & 31;
     // blocks [0, nu) are the consumers of the launch's nu units, then the first
@@ -1028,24 +1050,27 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
     if (threadIdx.x == 0) {
         *x.abort = 0;
-        *x.mma2_issued = 0;
         if (rank == 0) {
             for (int b = 0; b < 2; ++b) {
                 mbar_init(x.bar(CB_RECV_FULL + b), 1);
                 mbar_init(x.bar(CB_SLOT_FREE + b), 1);
                 mbar_init(x.bar(CB_REL_DONE + b), 1);
             }
-            mbar_init(x.bar(CB_K_FULL), 1);
-            mbar_init(x.bar(CB_K_EMPTY), 1);
             for (int b = 0; b < 2; ++b) {
+                mbar_init(x.bar(CB_K_FULL + b), 1);
+                mbar_init(x.bar(CB_K_EMPTY + b), 1);
                 mbar_init(x.bar(CB_V_FULL + b), 1);
                 mbar_init(x.bar(CB_V_EMPTY + b), 1);
             }
             mbar_init(x.bar(CB_D_FULL), 1);
-            mbar_init(x.bar(CB_S_FULL), 1);
-            mbar_init(x.bar(CB_DRAIN), 1);
+            mbar_init(x.bar(CB_EPI1_DONE), kEpiThreads / 32);
+            for (int j = 0; j < 4; ++j) mbar_init(x.bar(CB_EPI2_BLK + j), kEpiThreads / 32);
             mbar_init(x.bar(CB_E_FULL), 1);
             mbar_init(x.bar(CB_E_DRAIN), 1);
+            mbar_init(x.bar(CB_CHAIN_ISSUED), 1);
+            mbar_init(x.bar(CB_SUPD_ISSUED), 1);
+            mbar_init(x.bar(CB_S_FULL), 1);
+            mbar_init(x.bar(CB_DRAIN), 1);
         } else {
             for (int s = 0; s < kKqStages; ++s) mbar_init(x.bar(PB_KQ_EMPTY + s), 1);
             for (int grp = 0; grp < 2; ++grp) {
@@ -1075,7 +1100,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     x.tmem = *tmem_slot;
 
     if (rank == 0)
-        consumer(x, &tm_k, &tm_v, &tm_o, p);
+        consumer(x, &tm_k, &tm_v, p);
     else
         producer(x, (int)rank - 1, &tm_q, &tm_k, &tm_a, &tm_b, p);
 
@@ -1120,20 +1145,6 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// 2D float tensor [rows, cols] (cols contiguous), 32-column x 64-row boxes,
-// 128-byte swizzle (the o tiles)
-bool make_map_o(CUtensorMap* m, float* base, int64_t rows, int64_t cols) {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
-    cuuint32_t box[2] = {32, 64};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // 2D float tensor [rows, cols], 4-column x 64-row boxes, no swizzle
@@ -1222,9 +1233,9 @@ cudaError_t launch_prefill_pc(const PrefillArgs& a, cudaStream_t stream) {
         }
         return cudaSuccess;
     }
-    CUtensorMap mq, mk, mv, ma, mb, mo;
+    CUtensorMap mq, mk, mv, ma, mb;
     if (!make_map(&mq, a.q, a.T, (int64_t)a.Hqk * kD) || !make_map(&mk, a.k, a.T, (int64_t)a.Hqk * kD) ||
-        !make_map(&mv, a.v, a.T, (int64_t)a.Hv * kD) || !make_map_o(&mo, a.o, a.T, (int64_t)a.Hv * kD))
+        !make_map(&mv, a.v, a.T, (int64_t)a.Hv * kD))
         return cudaErrorInvalidValue;
     // a and b rows must be a multiple of 16 bytes for TMA; otherwise they are read directly
     const int gate_tma = (a.Hv % 4 == 0) ? 1 : 0;
@@ -1274,7 +1285,7 @@ cudaError_t launch_prefill_pc(const PrefillArgs& a, cudaStream_t stream) {
         attr[0].val.cooperative = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, prefill_pc_kernel, mq, mk, mv, ma, mb, mo, p);
+        e = cudaLaunchKernelEx(&cfg, prefill_pc_kernel, mq, mk, mv, ma, mb, p);
         if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
