@@ -111,9 +111,9 @@ gdn_status gdn_conv1d_silu(const uint16_t* qkv, const float* conv_w, const int32
  * gdn_prefill runs its fastest kernel for these sizes (a multiple of 256; never
  * 0).  Host-only, no CUDA calls.  That kernel passes each chunk's
  * state-independent operands from producer to consumer CTAs through a ring of
- * 4 slots of 49664 bytes plus 128 bytes of counters per (sequence, value head)
+ * 8 slots of 49664 bytes plus 128 bytes of counters per (sequence, value head)
  * of one launch, and a launch holds at most 64 of them, so the size is
- * 256 + 198784 * min(n_seq * Hv, 64) bytes (rounded up to 256).  A smaller
+ * 256 + 397440 * min(n_seq * Hv, 64) bytes (rounded up to 256).  A smaller
  * workspace that holds at least one such ring runs fewer (sequence, value head)
  * pairs per launch.  gdn_prefill also accepts a workspace as small as
  * 256 + 4 * n_seq * Hv bytes (rounded up to 256) and then runs a single-CTA

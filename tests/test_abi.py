@@ -53,6 +53,14 @@ def test_workspace_size_is_positive_and_aligned(L):
         assert ws > 0 and ws % 256 == 0
 
 
+def test_workspace_size_matches_the_documented_formula(L):
+    # gdn.h: 256 + 397440 * min(n_seq * Hv, 64), rounded up to 256
+    for n, Hqk, Hv in ((1, 16, 48), (2, 16, 48), (1, 4, 12), (3, 1, 1), (16, 16, 48)):
+        units = min(n * Hv, 64)
+        want = 256 + ((397440 * units + 255) // 256) * 256
+        assert L.gdn_prefill_workspace_size(n, 1000, Hqk, Hv, 128) == want
+
+
 FAKE = 0x10000     # 16-byte aligned non-null stand-in; never dereferenced: every call below fails validation
 
 
