@@ -9,6 +9,7 @@ from .oracle import (  # noqa: F401
     build,
     conv1d_silu,
     decode,
+    gated_norm,
     log_alpha,
     beta,
     max_threads,

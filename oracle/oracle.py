@@ -205,3 +205,31 @@ def conv1d_silu(qkv, conv_w, cu_seqlens=None, Hqk=16, Hv=48, d=128, conv_state=N
     if rc != 0:
         raise ValueError("oracle conv1d_silu rejected its arguments")
     return q, k, v, cso
+
+
+def gated_norm(o, z, norm_w, eps=1e-6):
+    """Gated output norm of the linear-attention layer, in fp64:
+        y[t, h, :] = norm_w * o[t, h, :] / sqrt(mean_v o[t, h, v]^2 + eps) * silu(z[t, h, :])
+    with silu(x) = x / (1 + e^{-x}).
+
+    The Qwen3.8-27B architecture page (2kiu.com), section 2.1, lists `norm` and
+    `in_proj_z` among the weights of every linear-attention layer but prints no
+    formula.  Reading used: `norm` is an RMS norm over the d_v channels of each
+    value head (one weight vector of length d_v shared by all heads, eps = 1e-6,
+    the epsilon of the layer's other norms), and z = in_proj_z(x), one value per
+    output channel, gates it through SiLU, the same activation the layer's
+    front end uses.  parity pinned by tests/test_oracle_pins.py (closed forms of
+    silu, unit RMS, scale invariance, per-head independence).
+
+    o: [T, Hv, d] (any float); z: [T, Hv, d] float or bf16 bits (uint16);
+    norm_w: [d].  Returns y [T, Hv, d] float64.
+    """
+    o = np.asarray(o, dtype=np.float64)
+    z = np.asarray(z)
+    if z.dtype == np.uint16:
+        z = (z.astype(np.uint32) << 16).view(np.float32)
+    z = z.astype(np.float64)
+    w = np.asarray(norm_w, dtype=np.float64)
+    ms = np.mean(o * o, axis=-1, keepdims=True)
+    gate = z / (1.0 + np.exp(-z))
+    return w * (o / np.sqrt(ms + eps)) * gate

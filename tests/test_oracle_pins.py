@@ -387,3 +387,75 @@ def test_conv_state_carries_history(orc):
         np.testing.assert_array_equal(np.concatenate([v1, v2]), v)
         np.testing.assert_array_equal(np.concatenate([q1, q2]), q)
         np.testing.assert_array_equal(cs2, cs)
+
+
+# ---- gated output norm -------------------------------------------------------
+
+def _gn_inputs(T=5, Hv=3, d=16, seed=3):
+    rng = np.random.default_rng(seed)
+    o = rng.standard_normal((T, Hv, d))
+    z = rng.standard_normal((T, Hv, d))
+    w = rng.uniform(0.5, 1.5, d)
+    return o, z, w
+
+
+def test_gated_norm_silu_closed_forms(orc):
+    # with o a constant row and w = 1, eps = 0 the norm is exactly 1 per channel, so y is silu(z):
+    # silu(0) = 0, silu(1) = 1 / (1 + 1/e), silu(-1) = -1 / (1 + e), silu(2) = 2 / (1 + e^-2)
+    o = np.full((1, 1, 4), 3.0)
+    z = np.array([[[0.0, 1.0, -1.0, 2.0]]])
+    y = orc.gated_norm(o, z, np.ones(4), eps=0.0)
+    e = np.e
+    want = [0.0, 1.0 / (1.0 + 1.0 / e), -1.0 / (1.0 + e), 2.0 / (1.0 + e ** -2)]
+    assert np.allclose(y[0, 0], want, rtol=0, atol=1e-15)
+
+
+def test_gated_norm_unit_rms(orc):
+    # constant gate c per row, w = 1, eps = 0: the mean square of y over d_v is silu(c)^2
+    o, _, _ = _gn_inputs(T=7, Hv=4, d=32)
+    c = 1.0
+    z = np.full_like(o, c)
+    y = orc.gated_norm(o, z, np.ones(32), eps=0.0)
+    s = c / (1.0 + np.exp(-c))
+    assert np.allclose(np.mean(y * y, axis=-1), s * s, rtol=1e-13)
+
+
+def test_gated_norm_scale_invariance_and_eps(orc):
+    o, z, w = _gn_inputs()
+    y = orc.gated_norm(o, z, w, eps=0.0)
+    assert np.allclose(orc.gated_norm(37.5 * o, z, w, eps=0.0), y, rtol=1e-13, atol=0)
+    assert np.allclose(orc.gated_norm(-o, z, w, eps=0.0), -y, rtol=1e-13, atol=0)
+    # eps only matters against the row's mean square: a tiny row is shrunk, not blown up
+    tiny = 1e-6 * o
+    yt = orc.gated_norm(tiny, z, w, eps=1e-6)
+    ms = np.mean(tiny * tiny, axis=-1, keepdims=True)
+    assert np.allclose(yt, y * np.sqrt(ms / (ms + 1e-6)), rtol=1e-12)
+    # o = 0 gives 0
+    assert np.all(orc.gated_norm(np.zeros_like(o), z, w) == 0.0)
+
+
+def test_gated_norm_heads_and_tokens_independent(orc):
+    # the norm runs over d_v within one (token, head): changing another head or token
+    # changes nothing else; the weight scales channel v alone
+    o, z, w = _gn_inputs(T=4, Hv=3, d=8)
+    y = orc.gated_norm(o, z, w)
+    o2 = o.copy()
+    o2[1, 2] *= 5.0
+    o2[3, 0] += 1.0
+    y2 = orc.gated_norm(o2, z, w)
+    mask = np.ones(y.shape[:2], bool)
+    mask[1, 2] = mask[3, 0] = False
+    assert np.array_equal(y[mask], y2[mask])
+    w2 = w.copy()
+    w2[5] *= 3.0
+    y3 = orc.gated_norm(o, z, w2)
+    assert np.allclose(y3[..., 5], 3.0 * y[..., 5], rtol=1e-14)
+    assert np.array_equal(np.delete(y3, 5, axis=-1), np.delete(y, 5, axis=-1))
+
+
+def test_gated_norm_bf16_gate_bits(orc):
+    # z given as bf16 bit patterns is widened exactly
+    o, z, w = _gn_inputs()
+    zb = (z.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    zw = (zb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert np.array_equal(orc.gated_norm(o, zb, w), orc.gated_norm(o, zw, w))
