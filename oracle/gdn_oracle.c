@@ -467,3 +467,33 @@ int gdn_oracle_conv1d_silu(const uint16_t* x, const float* w, const int32_t* cu_
     }
     return bad ? -1 : 0;
 }
+
+/*
+ * Gated output norm of the linear-attention layer.  The architecture page
+ * (section 2.1) lists the weights `norm` and `in_proj_z` of every
+ * linear-attention layer and prints no formula.  Reading used: per (token t,
+ * value head h) an RMS norm over the d_v channels, one weight vector per layer
+ * shared by the heads (row t uses layer t % layers), eps as given (the layer's
+ * other norms use 1e-6), gated by SiLU of z:
+ *     y[t,h,e] = w[l][e] * o[t,h,e] / sqrt(mean_e' o[t,h,e']^2 + eps)
+ *                * z[t,h,e] / (1 + exp(-z[t,h,e])).
+ * o, z, w, y in double; z may carry bf16 values widened exactly by the caller.
+ */
+int gdn_oracle_gated_norm(const double* o, const double* z, const double* w, int64_t T, int Hv, int d,
+                          int layers, double eps, double* y) {
+    if (T < 0 || Hv <= 0 || d <= 0 || layers <= 0 || !(eps >= 0.0)) return -1;
+    for (int64_t t = 0; t < T; ++t) {
+        const double* wl = w + (int64_t)(t % layers) * d;
+        for (int h = 0; h < Hv; ++h) {
+            const int64_t row = (t * Hv + h) * (int64_t)d;
+            double ss = 0.0;
+            for (int e = 0; e < d; ++e) ss += o[row + e] * o[row + e];
+            const double inv = 1.0 / sqrt(ss / d + eps);
+            for (int e = 0; e < d; ++e) {
+                const double g = z[row + e] / (1.0 + exp(-z[row + e]));
+                y[row + e] = wl[e] * (o[row + e] * inv) * g;
+            }
+        }
+    }
+    return 0;
+}

@@ -45,6 +45,8 @@ def _bind(lib):
     lib.gdn_oracle_log_alpha.argtypes = [dbl, dbl, dbl]
     lib.gdn_oracle_beta.restype = dbl
     lib.gdn_oracle_beta.argtypes = [dbl]
+    lib.gdn_oracle_gated_norm.restype = C.c_int
+    lib.gdn_oracle_gated_norm.argtypes = [vp, vp, vp, i64, C.c_int, C.c_int, C.c_int, dbl, vp]
     lib.gdn_oracle_max_threads.restype = C.c_int
     lib.gdn_oracle_max_threads.argtypes = [C.c_int]
     return lib
@@ -207,29 +209,27 @@ def conv1d_silu(qkv, conv_w, cu_seqlens=None, Hqk=16, Hv=48, d=128, conv_state=N
     return q, k, v, cso
 
 
-def gated_norm(o, z, norm_w, eps=1e-6):
-    """Gated output norm of the linear-attention layer, in fp64:
-        y[t, h, :] = norm_w * o[t, h, :] / sqrt(mean_v o[t, h, v]^2 + eps) * silu(z[t, h, :])
-    with silu(x) = x / (1 + e^{-x}).
 
-    The Qwen3.8-27B architecture page (2kiu.com), section 2.1, lists `norm` and
-    `in_proj_z` among the weights of every linear-attention layer but prints no
-    formula.  Reading used: `norm` is an RMS norm over the d_v channels of each
-    value head (one weight vector of length d_v shared by all heads, eps = 1e-6,
-    the epsilon of the layer's other norms), and z = in_proj_z(x), one value per
-    output channel, gates it through SiLU, the same activation the layer's
-    front end uses.  parity pinned by tests/test_oracle_pins.py (closed forms of
-    silu, unit RMS, scale invariance, per-head independence).
+def gated_norm(o, z, norm_w, eps=1e-6, lib=None):
+    """Gated output norm in fp64 (gdn_oracle_gated_norm in gdn_oracle.c, which
+    states the formula and the reading of the pages it follows).
 
     o: [T, Hv, d] (any float); z: [T, Hv, d] float or bf16 bits (uint16);
-    norm_w: [d].  Returns y [T, Hv, d] float64.
+    norm_w: [d] or [layers, d] (row t uses layer t % layers).
+    Returns y [T, Hv, d] float64.
     """
-    o = np.asarray(o, dtype=np.float64)
+    o = np.ascontiguousarray(o, dtype=np.float64)
     z = np.asarray(z)
     if z.dtype == np.uint16:
         z = (z.astype(np.uint32) << 16).view(np.float32)
-    z = z.astype(np.float64)
-    w = np.asarray(norm_w, dtype=np.float64)
-    ms = np.mean(o * o, axis=-1, keepdims=True)
-    gate = z / (1.0 + np.exp(-z))
-    return w * (o / np.sqrt(ms + eps)) * gate
+    z = np.ascontiguousarray(z, dtype=np.float64)
+    w = np.ascontiguousarray(norm_w, dtype=np.float64)
+    if w.ndim == 1:
+        w = w[None, :]
+    T, Hv, d = o.shape
+    y = np.zeros_like(o)
+    rc = _L(lib).gdn_oracle_gated_norm(_ptr(o), _ptr(z), _ptr(w), T, Hv, d, w.shape[0], float(eps),
+                                       _ptr(y))
+    if rc != 0:
+        raise ValueError("oracle gated_norm rejected its arguments")
+    return y

@@ -41,6 +41,13 @@ MUTANTS = {
     "chunk_inter_no_gamma": ("dst[e] = scale * (exp(G[i]) * inter + intra);",
                              "dst[e] = scale * (inter + intra);"),
     "chunk_substitution_sign": ("val -= A[i * C + m] * Tm[m * C + j];", "val += A[i * C + m] * Tm[m * C + j];"),
+    "norm_sum_not_mean": ("1.0 / sqrt(ss / d + eps)", "1.0 / sqrt(ss + eps)"),
+    "norm_no_eps": ("1.0 / sqrt(ss / d + eps)", "1.0 / sqrt(ss / d)"),
+    "gate_sigmoid_only": ("const double g = z[row + e] / (1.0 + exp(-z[row + e]));",
+                          "const double g = 1.0 / (1.0 + exp(-z[row + e]));"),
+    "norm_weight_wrong_layer": ("const double* wl = w + (int64_t)(t % layers) * d;", "const double* wl = w;"),
+    "norm_over_heads": ("const int64_t row = (t * Hv + h) * (int64_t)d;\n            double ss = 0.0;\n            for (int e = 0; e < d; ++e) ss += o[row + e] * o[row + e];",
+                        "const int64_t row = (t * Hv + h) * (int64_t)d;\n            double ss = 0.0;\n            for (int e = 0; e < d; ++e) ss += o[t * Hv * (int64_t)d + e] * o[t * Hv * (int64_t)d + e];"),
 }
 
 

@@ -459,3 +459,16 @@ def test_gated_norm_bf16_gate_bits(orc):
     zb = (z.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
     zw = (zb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     assert np.array_equal(orc.gated_norm(o, zb, w), orc.gated_norm(o, zw, w))
+
+
+def test_gated_norm_layer_of_each_row(orc):
+    # rows are units s * layers + l: row t takes the weight of layer t % layers.  With the same
+    # o and z in every row and w[l] = (l + 1), row t is (t % layers + 1) times row 0.
+    layers, T = 3, 7
+    o1, z1, _ = _gn_inputs(T=1, Hv=2, d=8)
+    o = np.repeat(o1, T, axis=0)
+    z = np.repeat(z1, T, axis=0)
+    w = np.array([[l + 1.0] * 8 for l in range(layers)])
+    y = orc.gated_norm(o, z, w)
+    for t in range(T):
+        assert np.allclose(y[t], (t % layers + 1) * y[0], rtol=1e-14, atol=0)
