@@ -298,6 +298,7 @@ def bench_main(args, world, rank, local):
         extra["prefill_262k"] = bench_long_prefill(args, dev, flush, peaks, world)
         extra["prefill_varlen_16seq"] = bench_long_prefill(
             args, dev, flush, peaks, world, lengths=synth.varlen_lengths(3), seed=3)
+        extra["gated_norm_T8192"] = bench_gated_norm(args, dev, flush, peaks, world)
         extra["decode_128seq_48layers"] = bench_decode(args, dev, peaks, world)
         extra["decode_fused_128seq_48layers"] = bench_decode_fused(args, dev, peaks, world)
         extra["decode_bf16state_128seq_48layers"] = bench_decode(args, dev, peaks, world, bf16_state=True)
@@ -431,6 +432,41 @@ def bench_long_prefill(args, dev, flush, peaks, world, lengths=None, seed=2):
            # CTAs) per cooperative launch when more units exist than fit at once
            "launches_per_step": N}
     del q, k, v, a, b, o
+    torch.cuda.empty_cache()
+    return out
+
+
+def bench_gated_norm(args, dev, flush, peaks, world):
+    """gdn_gated_norm over the T = 8192 output of one layer (48 heads): o
+    float32 in, z bf16 in, y bf16 out, 1024 bytes per (token, head)."""
+    import torch
+    import gated_deltanet_recurrence_prefill_b200 as gdn
+    T = T_MAIN
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(5)
+    o = torch.randn(T, HV, D, generator=gen, device=dev)
+    z = torch.randn(T, HV, D, generator=gen, device=dev).to(torch.bfloat16)
+    w = torch.empty(D, device=dev).uniform_(0.5, 1.5, generator=gen)
+    y = torch.empty(T, HV, D, dtype=torch.bfloat16, device=dev)
+
+    def step(ev):
+        if ev:
+            ev["start"].record()
+        gdn.gated_norm(o, z, w, y=y)
+        if ev:
+            ev["end"].record()
+
+    mk = lambda: {"start": torch.cuda.Event(enable_timing=True),
+                  "end": torch.cuda.Event(enable_timing=True)}
+    times, _ = _time_steps(step, max(3, args.warmup), max(5, min(args.steps, 50)), flush, mk, world)
+    ms = _max_over_ranks(sum(times) / len(times), world)
+    bytes_step = T * HV * D * (4 + 2 + 2)
+    gbs = bytes_step / (ms * 1e-3) / 1e9
+    out = {"workload": f"gdn_gated_norm T={T} Hv=48 d=128 (o f32, z bf16 -> y bf16)",
+           "ms": round(ms, 4), "GB_s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+           "bytes_per_step": int(bytes_step), "l2": "flushed before every timed step",
+           "launches_per_step": 1}
+    del o, z, y
     torch.cuda.empty_cache()
     return out
 

@@ -41,6 +41,7 @@ SIGNATURES = {
                                        _i32, _f32, _vp, _vp, _vp]),
     "gdn_decode_step_fused_bf16": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
                                              _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp]),
+    "gdn_gated_norm": (C.c_int, [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _f32, _vp, _vp]),
 }
 
 
@@ -275,3 +276,23 @@ def decode_step_fused(qkv, conv_w, conv_state, a, b, A_log, dt_bias, state, n_se
                               d, scale, n_slots, _ptr(state), _ptr(o), _stream(stream))
     _check(name, st)
     return o
+
+
+def gated_norm(o, z, norm_w, eps=1e-6, y=None, stream=None):
+    """Gated output norm: y = norm_w * o / sqrt(mean_v o^2 + eps) * silu(z) per
+    (token, value head).  o [T, Hv, d] float32, z [T, Hv, d] bf16, norm_w [d]
+    or [layers, d] float32 (row t uses layer t % layers).  Returns y [T, Hv, d]
+    bf16."""
+    import torch
+    T, Hv, d = o.shape
+    w = norm_w if norm_w.dim() == 2 else norm_w.view(1, -1)
+    layers = w.shape[0]
+    _need(o, torch.float32, (T, Hv, d), "o")
+    _need(z, torch.bfloat16, (T, Hv, d), "z")
+    _need(w, torch.float32, (layers, d), "norm_w")
+    if y is None:
+        y = torch.empty(T, Hv, d, dtype=torch.bfloat16, device=o.device)
+    st = lib().gdn_gated_norm(_ptr(o), _ptr(z), _ptr(w), T, Hv, d, layers, float(eps), _ptr(y),
+                              _stream(stream))
+    _check("gdn_gated_norm", st)
+    return y

@@ -230,4 +230,17 @@ gdn_status gdn_decode_step_fused_bf16(const uint16_t* qkv, const float* conv_w, 
     return e == cudaSuccess ? GDN_OK : cuda_fail(e);
 }
 
+gdn_status gdn_gated_norm(const float* o, const uint16_t* z, const float* norm_w, int64_t T, int32_t Hv,
+                          int32_t d, int32_t layers, float eps, uint16_t* y, gdn_stream_t stream) {
+    if (T < 0 || Hv <= 0 || d <= 0 || layers <= 0 || !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+    if (d != kD) return GDN_ERR_UNSUPPORTED;
+    if (T == 0) return GDN_OK;
+    if (!o || !z || !norm_w || !y) return GDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {o, z, norm_w, y};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return GDN_ERR_MISALIGNED;
+    cudaError_t e = gdn::launch_gated_norm(o, z, norm_w, T, Hv, layers, eps, y, (cudaStream_t)stream);
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
 }  // extern "C"

@@ -58,6 +58,8 @@ cudaError_t launch_conv1d_silu(const uint16_t* qkv, const float* w, const int32_
                                const float* cs_in, float* cs_out, uint16_t* q, uint16_t* k,
                                uint16_t* v, cudaStream_t stream);
 
+cudaError_t launch_gated_norm(const float* o, const uint16_t* z, const float* w, int64_t T, int32_t Hv,
+                              int32_t layers, float eps, uint16_t* y, cudaStream_t stream);
 cudaError_t launch_prefill_simt(const PrefillArgs& p, cudaStream_t stream);
 cudaError_t launch_prefill_tc(const PrefillArgs& p, cudaStream_t stream);
 size_t prefill_tc_smem_bytes();

@@ -273,6 +273,29 @@ gdn_status gdn_decode_step_fused_bf16(const uint16_t* qkv, const float* conv_w, 
                                       int32_t layers, int32_t Hqk, int32_t Hv, int32_t d, float scale,
                                       int32_t n_slots, uint16_t* state, float* o, gdn_stream_t stream);
 
+/*
+ * gdn_gated_norm -- the gated output norm that follows the recurrence in a
+ * linear-attention layer:
+ *     y[t, h, :] = norm_w[l] * o[t, h, :] / sqrt(mean_v o[t, h, v]^2 + eps)
+ *                  * silu(z[t, h, :]),      silu(x) = x / (1 + e^{-x}).
+ * The architecture page (section 2.1) lists `norm` and `in_proj_z` among each
+ * linear-attention layer's weights but prints no formula; this is the reading
+ * used: an RMS norm over the d_v channels of each value head, one weight
+ * vector per layer shared by all heads, gated by SiLU of z = in_proj_z(x).
+ *
+ *  o       [T, Hv, d] float32 (the output of gdn_prefill or of a decode step).
+ *  z       [T, Hv, d] bf16.
+ *  norm_w  [layers, d] float32; row t uses layer t % layers (1 for a prefill;
+ *          for a decode batch, rows are units s * layers + l).
+ *  eps     >= 0 (the layer uses 1e-6).
+ *  y       [T, Hv, d] bf16 output (round to nearest even); must not overlap o
+ *          or z.
+ * Supported: d = 128.  T = 0 does nothing.  All pointers 16-byte aligned.
+ * One launch, bound by HBM bandwidth (1024 bytes per (token, head)).
+ */
+gdn_status gdn_gated_norm(const float* o, const uint16_t* z, const float* norm_w, int64_t T, int32_t Hv,
+                          int32_t d, int32_t layers, float eps, uint16_t* y, gdn_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

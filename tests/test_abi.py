@@ -28,7 +28,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for required in ("gdn_conv1d_silu", "gdn_prefill", "gdn_prefill_workspace_size",
                      "gdn_decode_step", "gdn_decode_step_fused", "gdn_prefill_status",
-                     "gdn_status_string"):
+                     "gdn_gated_norm", "gdn_status_string"):
         assert required in names
 
 
@@ -152,3 +152,18 @@ def test_bf16_state_decode_rejects_bad_arguments(L):
     assert call(layers=0) == 1
     assert call(state=None) == 1
     assert call(state=_p(FAKE + 2)) == 3
+
+
+def test_gated_norm_rejects_bad_arguments(L):
+    def call(o=_p(), z=_p(), w=_p(), T=8, Hv=48, d=128, layers=1, eps=1e-6, y=_p()):
+        return L.gdn_gated_norm(o, z, w, T, Hv, d, layers, eps, y, None)
+    assert call(d=64) == 2                        # unsupported head width
+    assert call(T=-1) == 1
+    assert call(Hv=0) == 1
+    assert call(layers=0) == 1
+    assert call(eps=-1.0) == 1
+    assert call(eps=float("nan")) == 1
+    assert call(z=None) == 1
+    assert call(y=None) == 1
+    assert call(o=_p(FAKE + 4)) == 3              # misaligned
+    assert call(T=0, o=None, z=None, w=None, y=None) == 0   # nothing to do, nothing read
