@@ -21,6 +21,10 @@ namespace {
 constexpr int kD = 128;
 constexpr int kRowsPerBlock = 8;
 
+// silu(x) = x / (1 + e^{-x}), as x * rcp(1 + e^{-x}): for x -> -inf the
+// reciprocal of +inf is 0 and the result -0, for x -> +inf it is x
+__device__ __forceinline__ float silu(float x) { return x * __frcp_rn(1.f + __expf(-x)); }
+
 __global__ void __launch_bounds__(kRowsPerBlock * 32)
 gated_norm_kernel(const float* __restrict__ o, const uint16_t* __restrict__ z, const float* __restrict__ w,
                   int64_t rows, int32_t Hv, int32_t layers, float eps, uint16_t* __restrict__ y) {
@@ -39,9 +43,7 @@ gated_norm_kernel(const float* __restrict__ o, const uint16_t* __restrict__ z, c
     for (int m = 16; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
     const float r = rsqrtf(ss * (1.f / kD) + eps);
     const float2 z01 = bf16x2_to_f32x2(zv.x), z23 = bf16x2_to_f32x2(zv.y);
-    // silu(x) = x / (1 + e^{-x}); for x -> -inf the quotient is -0
-    const float g0 = z01.x / (1.f + expf(-z01.x)), g1 = z01.y / (1.f + expf(-z01.y));
-    const float g2 = z23.x / (1.f + expf(-z23.x)), g3 = z23.y / (1.f + expf(-z23.y));
+    const float g0 = silu(z01.x), g1 = silu(z01.y), g2 = silu(z23.x), g3 = silu(z23.y);
     uint2 out;
     out.x = pack_bf16x2(wv.x * (ov.x * r) * g0, wv.y * (ov.y * r) * g1);
     out.y = pack_bf16x2(wv.z * (ov.z * r) * g2, wv.w * (ov.w * r) * g3);
