@@ -15,6 +15,7 @@ from ._lib import (  # noqa: F401
     lib,
     lib_path,
     prefill,
+    prefill_gated,
     prefill_noalloc,
     prefill_status,
     prefill_workspace_size,

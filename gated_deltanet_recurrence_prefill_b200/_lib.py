@@ -42,6 +42,8 @@ SIGNATURES = {
     "gdn_decode_step_fused_bf16": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
                                              _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp]),
     "gdn_gated_norm": (C.c_int, [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _f32, _vp, _vp]),
+    "gdn_prefill_gated": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
+                                    _i32, _f32, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _sz, _vp]),
 }
 
 
@@ -296,3 +298,47 @@ def gated_norm(o, z, norm_w, eps=1e-6, y=None, stream=None):
                               _stream(stream))
     _check("gdn_gated_norm", st)
     return y
+
+
+def prefill_gated(q, k, v, a, b, A_log, dt_bias, z, norm_w, eps=1e-6, cu_seqlens=None, scale=None,
+                  initial_state=None, final_state=None, y=None, o=None, want_o=False,
+                  workspace=None, want_final_state=True, stream=None):
+    """gdn_prefill_gated: the chunked prefill with the gated output norm fused
+    in.  z [T, Hv, d] bf16, norm_w [d] float32.  Returns (y [T, Hv, d] bf16,
+    o [T, Hv, d] f32 or None, final_state or None); o is written only when
+    passed in or want_o is set."""
+    import torch
+    T, Hqk, d = q.shape
+    Hv = v.shape[1]
+    n_seq = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _need(q, torch.bfloat16, (T, Hqk, d), "q")
+    _need(k, torch.bfloat16, (T, Hqk, d), "k")
+    _need(v, torch.bfloat16, (T, Hv, d), "v")
+    _need(a, torch.float32, (T, Hv), "a")
+    _need(b, torch.float32, (T, Hv), "b")
+    _need(A_log, torch.float32, (Hv,), "A_log")
+    _need(dt_bias, torch.float32, (Hv,), "dt_bias")
+    _need(z, torch.bfloat16, (T, Hv, d), "z")
+    _need(norm_w, torch.float32, (d,), "norm_w")
+    if cu_seqlens is not None:
+        _need(cu_seqlens, torch.int32, (n_seq + 1,), "cu_seqlens")
+    if initial_state is not None:
+        _need(initial_state, torch.float32, (n_seq, Hv, d, d), "initial_state")
+    if scale is None:
+        scale = d ** -0.5
+    if y is None:
+        y = torch.empty(T, Hv, d, dtype=torch.bfloat16, device=q.device)
+    if o is None and want_o:
+        o = torch.empty(T, Hv, d, dtype=torch.float32, device=q.device)
+    if final_state is None and want_final_state:
+        final_state = torch.empty(n_seq, Hv, d, d, dtype=torch.float32, device=q.device)
+    ws_bytes = prefill_workspace_size(n_seq, T, Hqk, Hv, d)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    st = lib().gdn_prefill_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(A_log),
+                                 _ptr(dt_bias), _ptr(cu_seqlens), n_seq, T, Hqk, Hv, d, float(scale),
+                                 _ptr(initial_state), _ptr(final_state), _ptr(o), _ptr(z),
+                                 _ptr(norm_w), float(eps), _ptr(y), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("gdn_prefill_gated", st)
+    return y, o, final_state

@@ -24,9 +24,15 @@ struct PrefillArgs {
     float scale;
     const float* initial_state;    // may be NULL
     float* final_state;            // may be NULL
-    float* o;
+    float* o;                      // may be NULL when y is given
     void* workspace;
     size_t workspace_bytes;
+    // fused gated output norm (producer / consumer kernel only): y = norm_w * o /
+    // sqrt(mean_v o^2 + eps) * silu(z), bf16, when y != NULL
+    const uint16_t* z = nullptr;
+    const float* norm_w = nullptr;
+    float eps = 0.f;
+    uint16_t* y = nullptr;
 };
 
 cudaError_t launch_decode_step(const uint16_t* q, const uint16_t* k, const uint16_t* v,

@@ -147,7 +147,8 @@ constexpr uint32_t C_RECV = 0;                              // 2 slots
 constexpr uint32_t C_V = C_RECV + 2 * SLOT_BYTES;           // V: 2 buffers of 2 panels of 64 x 64 bf16
 constexpr uint32_t C_K = C_V + 2 * 16384;                   // K: 2 buffers of 2 panels of 64 x 64 bf16
 constexpr uint32_t C_GATES = C_K + 2 * 16384;               // 2 gate buffers
-constexpr uint32_t C_END = C_GATES + 2 * GATE_BYTES;
+constexpr uint32_t C_NORM = C_GATES + 2 * GATE_BYTES;      // output norm: 2 x [4 cb][16 t][4 q] f32
+constexpr uint32_t C_END = C_NORM + 2 * 1024;
 // what one chunk sends: the [-W; Qh] tile (staged in place of [K; Q]) and the
 // [T b; R b] tile with the gates (staged in the A scratch)
 constexpr uint32_t SEND_QW = 2 * KQ_PANEL;
@@ -213,6 +214,7 @@ constexpr int kEpiWarp0 = 3;
 constexpr int kEpiThreads = 16 * 32;
 constexpr int kRelWarp = kEpiWarp0 + kEpiThreads / 32;     // ring slot release
 constexpr int kUoWarp = kRelWarp + 1;                      // [U'; O'] products
+constexpr int kNormBar0 = 1;                   // named barriers 1-4: the output norm of column share cb
 static_assert(kUoWarp < kWarps, "consumer warps");
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;    // 2 s: far beyond any legitimate wait
@@ -238,6 +240,12 @@ struct ClParams {
     int gate_tma;          // a, b staged by TMA (needs Hv % 4 == 0), else read directly
     int n_prod;            // producer CTAs per unit (1 or 2); a unit has n_prod + 1 CTAs
     int unit0;             // first (sequence, value head) unit of this launch
+    // fused gated output norm (y = norm_w * o / rms(o) * silu(z) per token and
+    // head, written as bf16) when y != NULL; o may then be NULL
+    const uint16_t* z;
+    const float* norm_w;
+    float eps;
+    uint16_t* y;
 };
 
 struct Ctx {
@@ -539,17 +547,77 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
                 // Rows past the sequence's end belong to the next sequence.
                 float ov[16];
                 tmem_ld16(tl + dbuf + 64 + cb * 16, ov);
-                tmem_ld_wait();
                 const int64_t t0 = tok0 + cb * 16;
-                float* ocol = p.o + t0 * o_stride + x.h * kD + v;
                 const int64_t nvalid = x.eos - t0;
-                if (nvalid >= 16) {
+                const int64_t col = x.h * kD + v;
+                uint16_t zr[16];
+                if (p.y) {
+                    // the output norm's gate inputs, in flight during the TMEM load
+                    const uint16_t* zc = p.z + t0 * o_stride + col;
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) ocol[j * o_stride] = p.scale * ov[j];
-                } else {
+                    for (int j = 0; j < 16; ++j) zr[j] = j < nvalid ? zc[j * o_stride] : (uint16_t)0;
+                }
+                tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        if (j < nvalid) ocol[j * o_stride] = p.scale * ov[j];
+                for (int j = 0; j < 16; ++j) ov[j] *= p.scale;
+                if (p.o) {
+                    float* ocol = p.o + t0 * o_stride + col;
+                    if (nvalid >= 16) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) ocol[j * o_stride] = ov[j];
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (j < nvalid) ocol[j * o_stride] = ov[j];
+                    }
+                }
+                if (p.y) {
+                    // gated output norm: the mean square of o over the 128 rows v of
+                    // a token is spread over the four warps of this column share
+                    // (lane quadrants 0-3).  Each warp sums its 32 rows for its 16
+                    // tokens by a reduce-scatter (lanes 2i and 2i + 1 end with one
+                    // token's sum), the four partial sums meet in shared memory (two
+                    // buffers: a warp is at most one chunk ahead of the others here).
+                    float sq[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) sq[j] = ov[j] * ov[j];
+                    float a8[8], a4[4], a2[2];
+                    const unsigned full = 0xffffffffu;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const bool hi = lane & 16;
+                        a8[i] = (hi ? sq[i + 8] : sq[i]) + __shfl_xor_sync(full, hi ? sq[i] : sq[i + 8], 16);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const bool hi = lane & 8;
+                        a4[i] = (hi ? a8[i + 4] : a8[i]) + __shfl_xor_sync(full, hi ? a8[i] : a8[i + 4], 8);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) {
+                        const bool hi = lane & 4;
+                        a2[i] = (hi ? a4[i + 2] : a4[i]) + __shfl_xor_sync(full, hi ? a4[i] : a4[i + 2], 4);
+                    }
+                    const bool hi2 = lane & 2;
+                    float a1 = (hi2 ? a2[1] : a2[0]) + __shfl_xor_sync(full, hi2 ? a2[0] : a2[1], 2);
+                    a1 += __shfl_xor_sync(full, a1, 1);
+                    const int tau = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
+                                    ((lane >> 1) & 1);
+                    float* part = reinterpret_cast<float*>(x.sm + C_NORM + (c & 1) * 1024 + cb * 256);
+                    if ((lane & 1) == 0) part[tau * 4 + q] = a1;
+                    named_bar_sync(kNormBar0 + cb, 128);
+                    const float wv = p.norm_w[v];
+                    uint16_t* ycol = p.y + t0 * o_stride + col;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        if (j < nvalid) {
+                            const float4 pp = reinterpret_cast<const float4*>(part)[j];
+                            const float r = rsqrtf(((pp.x + pp.y) + (pp.z + pp.w)) * (1.f / kD) + p.eps);
+                            const float zf = __uint_as_float((uint32_t)zr[j] << 16);
+                            const float g = zf * __frcp_rn(1.f + __expf(-zf));
+                            ycol[j * o_stride] = (uint16_t)f32_to_bf16_bits(wv * (ov[j] * r) * g);
+                        }
+                    }
                 }
             }
             Gam = resc ? 1.f : Gn;
@@ -1266,7 +1334,8 @@ cudaError_t launch_prefill_pc(const PrefillArgs& a, cudaStream_t stream) {
     uint8_t* ring = ws + kWsHeaderBytes + (size_t)per_launch * kFlagWords * sizeof(uint32_t);
     ClParams p{a.a, a.b, a.A_log, a.dt_bias, a.cu_seqlens, a.T, a.Hqk, a.Hv, a.scale,
                a.initial_state, a.final_state, a.o,
-               reinterpret_cast<uint32_t*>(ws + kWsErrorWordOffset), ring, flags, gate_tma, n_prod, 0};
+               reinterpret_cast<uint32_t*>(ws + kWsErrorWordOffset), ring, flags, gate_tma, n_prod, 0,
+               a.z, a.norm_w, a.eps, a.y};
     // Units run in launches of at most per_launch units, in order; each launch
     // starts from cleared counters.  A unit's CTAs wait on one another, so each
     // launch is cooperative (all of its CTAs resident together).

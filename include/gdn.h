@@ -274,6 +274,27 @@ gdn_status gdn_decode_step_fused_bf16(const uint16_t* qkv, const float* conv_w, 
                                       int32_t n_slots, uint16_t* state, float* o, gdn_stream_t stream);
 
 /*
+ * gdn_prefill_gated -- gdn_prefill followed by gdn_gated_norm on its output, in
+ * one pass: y = norm_w * o / sqrt(mean_v o^2 + eps) * silu(z) per token and
+ * value head (see gdn_gated_norm for the formula and the reading of the pages),
+ * written as bf16 by the same kernel that computes o, so that o need not go
+ * through memory.  Arguments as for gdn_prefill, plus
+ *  z       [T, Hv, d] bf16, norm_w [d] float32, eps >= 0, y [T, Hv, d] bf16.
+ *  o       may be NULL (o is then not written); if given, o is written too.
+ * With a workspace that holds the producer / consumer kernel's ring (see
+ * gdn_prefill_workspace_size) the norm is fused into that kernel; otherwise the
+ * single-CTA kernel writes o, which must then be given (else
+ * GDN_ERR_WORKSPACE), and gdn_gated_norm runs on it.
+ */
+gdn_status gdn_prefill_gated(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* a,
+                             const float* b, const float* A_log, const float* dt_bias,
+                             const int32_t* cu_seqlens, int32_t n_seq, int64_t T, int32_t Hqk,
+                             int32_t Hv, int32_t d, float scale, const float* initial_state,
+                             float* final_state, float* o, const uint16_t* z, const float* norm_w,
+                             float eps, uint16_t* y, void* workspace, size_t workspace_bytes,
+                             gdn_stream_t stream);
+
+/*
  * gdn_gated_norm -- the gated output norm that follows the recurrence in a
  * linear-attention layer:
  *     y[t, h, :] = norm_w[l] * o[t, h, :] / sqrt(mean_v o[t, h, v]^2 + eps)

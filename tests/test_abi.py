@@ -28,7 +28,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for required in ("gdn_conv1d_silu", "gdn_prefill", "gdn_prefill_workspace_size",
                      "gdn_decode_step", "gdn_decode_step_fused", "gdn_prefill_status",
-                     "gdn_gated_norm", "gdn_status_string"):
+                     "gdn_gated_norm", "gdn_prefill_gated", "gdn_status_string"):
         assert required in names
 
 
@@ -167,3 +167,19 @@ def test_gated_norm_rejects_bad_arguments(L):
     assert call(y=None) == 1
     assert call(o=_p(FAKE + 4)) == 3              # misaligned
     assert call(T=0, o=None, z=None, w=None, y=None) == 0   # nothing to do, nothing read
+
+
+def test_prefill_gated_rejects_bad_arguments(L):
+    ws = L.gdn_prefill_workspace_size(1, 64, 16, 48, 128)
+
+    def call(z=_p(), w=_p(), y=_p(), o=None, eps=1e-6, d=128, wsp=_p(0x20000), wsb=ws):
+        return L.gdn_prefill_gated(_p(), _p(), _p(), _p(), _p(), _p(), _p(), None, 1, 64, 16, 48, d, 0.088,
+                                   None, None, o, z, w, eps, y, wsp, wsb, None)
+    assert call(d=64) == 2
+    assert call(z=None) == 1
+    assert call(w=None) == 1
+    assert call(y=None) == 1
+    assert call(eps=-1.0) == 1
+    assert call(y=_p(FAKE + 8)) == 3
+    assert call(wsp=None) == 6
+    assert call(wsb=16) == 6
