@@ -299,6 +299,7 @@ def bench_main(args, world, rank, local):
         extra["prefill_varlen_16seq"] = bench_long_prefill(
             args, dev, flush, peaks, world, lengths=synth.varlen_lengths(3), seed=3)
         extra["gated_norm_T8192"] = bench_gated_norm(args, dev, flush, peaks, world)
+        extra["layer_tail_T8192"] = bench_layer_tail(args, dev, flush, peaks, world)
         extra["decode_128seq_48layers"] = bench_decode(args, dev, peaks, world)
         extra["decode_fused_128seq_48layers"] = bench_decode_fused(args, dev, peaks, world)
         extra["decode_bf16state_128seq_48layers"] = bench_decode(args, dev, peaks, world, bf16_state=True)
@@ -467,6 +468,68 @@ def bench_gated_norm(args, dev, flush, peaks, world):
            "bytes_per_step": int(bytes_step), "l2": "flushed before every timed step",
            "launches_per_step": 1}
     del o, z, y
+    torch.cuda.empty_cache()
+    return out
+
+
+def bench_layer_tail(args, dev, flush, peaks, world):
+    """The recurrence plus the gated output norm at T = 8192 (one sequence, zero
+    S0): gdn_prefill_gated (norm fused, bf16 y only) against gdn_prefill followed
+    by gdn_gated_norm (o written and read back)."""
+    import torch
+    import gated_deltanet_recurrence_prefill_b200 as gdn
+    T = T_MAIN
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(6)
+
+    def unit(shape):
+        x = torch.randn(*shape, generator=gen, device=dev)
+        return (x / torch.sqrt((x * x).sum(-1, keepdim=True) + 1e-6)).to(torch.bfloat16)
+
+    q, k = unit((T, HQK, D)), unit((T, HQK, D))
+    v = torch.randn(T, HV, D, generator=gen, device=dev).to(torch.bfloat16)
+    a = torch.randn(T, HV, generator=gen, device=dev)
+    b = torch.randn(T, HV, generator=gen, device=dev)
+    A_log = torch.log(torch.empty(HV, device=dev).uniform_(1, 16, generator=gen))
+    dt = torch.exp(torch.empty(HV, device=dev).uniform_(-6.907755, -2.302585, generator=gen))
+    dt_bias = torch.log(torch.expm1(dt))
+    z = torch.randn(T, HV, D, generator=gen, device=dev).to(torch.bfloat16)
+    w = torch.empty(D, device=dev).uniform_(0.5, 1.5, generator=gen)
+    o = torch.empty(T, HV, D, device=dev)
+    y = torch.empty(T, HV, D, dtype=torch.bfloat16, device=dev)
+    fs = torch.empty(1, HV, D, D, device=dev)
+    ws = torch.empty(gdn.prefill_workspace_size(1, T, HQK, HV, D), dtype=torch.uint8, device=dev)
+    mk = lambda: {"start": torch.cuda.Event(enable_timing=True),
+                  "end": torch.cuda.Event(enable_timing=True)}
+
+    def fused(ev):
+        if ev:
+            ev["start"].record()
+        gdn.prefill_gated(q, k, v, a, b, A_log, dt_bias, z, w, y=y, final_state=fs, workspace=ws)
+        if ev:
+            ev["end"].record()
+
+    def unfused(ev):
+        if ev:
+            ev["start"].record()
+        gdn.prefill(q, k, v, a, b, A_log, dt_bias, o=o, final_state=fs, workspace=ws)
+        gdn.gated_norm(o, z, w, y=y)
+        if ev:
+            ev["end"].record()
+
+    n = max(5, min(args.steps, 50))
+    tf, _ = _time_steps(fused, max(3, args.warmup), n, flush, mk, world)
+    tu, _ = _time_steps(unfused, max(3, args.warmup), n, flush, mk, world)
+    ms_f = _max_over_ranks(sum(tf) / len(tf), world)
+    ms_u = _max_over_ranks(sum(tu) / len(tu), world)
+    # algorithmic bytes of the fused pass: q, k, v, a, b and z in, y out (o never stored)
+    bytes_f = T * (2 * (2 * HQK * D + HV * D) + 4 * 2 * HV + 2 * HV * D + 2 * HV * D)
+    out = {"workload": f"gdn_prefill_gated T={T} N=1 Hqk=16 Hv=48 d=128 zero S0, bf16 y (o not stored)",
+           "fused_ms": round(ms_f, 4), "prefill_then_norm_ms": round(ms_u, 4),
+           "tokens_per_s_layer": round(weak_scaling_rate(T, ms_f, world), 1),
+           "GB_s": round(bytes_f / (ms_f * 1e-3) / 1e9, 1), "bytes_per_step": int(bytes_f),
+           "launches_per_step": 1}
+    del q, k, v, a, b, z, o, y
     torch.cuda.empty_cache()
     return out
 

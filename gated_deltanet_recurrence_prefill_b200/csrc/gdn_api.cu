@@ -173,14 +173,22 @@ gdn_status gdn_prefill_gated(const uint16_t* q, const uint16_t* k, const uint16_
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = cudaMemsetAsync(workspace, 0, gdn::kWsHeaderBytes, s);
     if (e != cudaSuccess) return cuda_fail(e);
-    if (which == PrefillKernel::ProducerConsumer) {
+    // Without o the norm runs inside the producer / consumer kernel (o never goes
+    // through memory).  With o, the prefill writes o and gdn_gated_norm runs on
+    // it: two launches, and the faster of the two on B200, where the fused norm's
+    // exponentials on the consumer's SM lengthen the state chain more than the
+    // second pass costs.  GDN_PREFILL_NORM=fused forces the fused kernel.
+    const char* env = getenv("GDN_PREFILL_NORM");
+    const bool fused = which == PrefillKernel::ProducerConsumer &&
+                       (!o || (env && strcmp(env, "fused") == 0));
+    if (fused) {
         e = gdn::launch_prefill_pc(p, s);
     } else {
         p.z = nullptr;
         p.norm_w = nullptr;
         p.y = nullptr;
-        e = gdn::launch_prefill_tc(p, s);
-        if (e == cudaSuccess) e = gdn::launch_gated_norm(o, z, norm_w, T, Hv, 1, eps, y, s);
+        e = which == PrefillKernel::ProducerConsumer ? gdn::launch_prefill_pc(p, s) : gdn::launch_prefill_tc(p, s);
+        if (e == cudaSuccess && T > 0) e = gdn::launch_gated_norm(o, z, norm_w, T, Hv, 1, eps, y, s);
     }
     return e == cudaSuccess ? GDN_OK : cuda_fail(e);
 }

@@ -148,7 +148,8 @@ constexpr uint32_t C_V = C_RECV + 2 * SLOT_BYTES;           // V: 2 buffers of 2
 constexpr uint32_t C_K = C_V + 2 * 16384;                   // K: 2 buffers of 2 panels of 64 x 64 bf16
 constexpr uint32_t C_GATES = C_K + 2 * 16384;               // 2 gate buffers
 constexpr uint32_t C_NORM = C_GATES + 2 * GATE_BYTES;      // output norm: 2 x [4 cb][16 t][4 q] f32
-constexpr uint32_t C_END = C_NORM + 2 * 1024;
+constexpr uint32_t C_Z = C_NORM + 2 * 1024;                 // output norm gate z: 2 x [64 t][128 v] bf16
+constexpr uint32_t C_END = C_Z + 2 * 16384;
 // what one chunk sends: the [-W; Qh] tile (staged in place of [K; Q]) and the
 // [T b; R b] tile with the gates (staged in the A scratch)
 constexpr uint32_t SEND_QW = 2 * KQ_PANEL;
@@ -182,7 +183,7 @@ enum {
     CB_RECV_FULL = 19, CB_K_FULL = 21, CB_V_FULL = 23, CB_V_EMPTY = 25, CB_SLOT_FREE = 27,
     CB_D_FULL = 29, CB_S_FULL = 30, CB_DRAIN = 31, CB_REL_DONE = 32, CB_K_EMPTY = 34,
     CB_EPI1_DONE = 36, CB_EPI2_BLK = 37, CB_E_FULL = 41, CB_E_DRAIN, CB_CHAIN_ISSUED, CB_SUPD_ISSUED,
-    kNumBars = 45
+    CB_Z_FULL = 45, CB_Z_EMPTY = 47, kNumBars = 49
 };
 constexpr uint32_t SMEM_BYTES = OFF_BARS + kNumBars * 8;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;           // room to align the base
@@ -269,7 +270,7 @@ struct Ctx {
 
 // ================================================================ consumer
 __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, const CUtensorMap* tm_v,
-                                         const ClParams& p) {
+                                         const CUtensorMap* tm_z, const ClParams& p) {
     const int warp = x.warp, lane = x.lane;
     const int nch = x.nch;
     if (warp == 0) {
@@ -280,7 +281,8 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
         if (lane == 0) {
             prefetch_tmap(tm_k);
             prefetch_tmap(tm_v);
-            int nv = 0, nk = 0;
+            if (p.y) prefetch_tmap(tm_z);
+            int nv = 0, nk = 0, nz = 0;
             for (int c = 0; c < nch; ++c) {
                 const int32_t y = (int32_t)(x.bos + (int64_t)c * kC);
                 const int vb = c & 1;
@@ -298,6 +300,15 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
                 tma_load_2d(x.sbase + C_K + vb * 16384, tm_k, x.g * kD, y, x.bar(CB_K_FULL + vb));
                 tma_load_2d(x.sbase + C_K + vb * 16384 + 8192, tm_k, x.g * kD + 64, y, x.bar(CB_K_FULL + vb));
                 nk = c + 1;
+                if (p.y) {
+                    // the output norm's gate z of this chunk (free once the epilogues
+                    // of chunk c - 2 have read it)
+                    if (c >= 2 && !mbar_wait(x.bar(CB_Z_EMPTY + vb), ((c >> 1) - 1) & 1, x.abort, kWaitLimitNs))
+                        break;
+                    mbar_arrive_expect_tx(x.bar(CB_Z_FULL + vb), 16384);
+                    tma_load_2d(x.sbase + C_Z + vb * 16384, tm_z, x.h * kD, y, x.bar(CB_Z_FULL + vb));
+                    nz = c + 1;
+                }
             }
             // copies still in flight land before the CTA may exit
             volatile int no_abort = 0;
@@ -305,6 +316,8 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
                 mbar_wait(x.bar(CB_V_FULL + (c & 1)), (c >> 1) & 1, &no_abort, kWaitLimitNs);
             for (int c = nk >= 2 ? nk - 2 : 0; c < nk; ++c)
                 mbar_wait(x.bar(CB_K_FULL + (c & 1)), (c >> 1) & 1, &no_abort, kWaitLimitNs);
+            for (int c = nz >= 2 ? nz - 2 : 0; c < nz; ++c)
+                mbar_wait(x.bar(CB_Z_FULL + (c & 1)), (c >> 1) & 1, &no_abort, kWaitLimitNs);
         }
     } else if (warp == kRelWarp) {
         // ------------------------------------------------ ring slots back to the producers
@@ -541,83 +554,26 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
             }
             if (tracer) TRACE_CLK(3, c);
             report(CB_EPI1_DONE);
-            {
-                // o^T / scale, tokens t = 16 cb .. 16 cb + 15, written while the state
-                // update runs; for each t a warp stores 32 consecutive floats of o.
-                // Rows past the sequence's end belong to the next sequence.
-                float ov[16];
-                tmem_ld16(tl + dbuf + 64 + cb * 16, ov);
-                const int64_t t0 = tok0 + cb * 16;
-                const int64_t nvalid = x.eos - t0;
-                const int64_t col = x.h * kD + v;
-                uint16_t zr[16];
-                if (p.y) {
-                    // the output norm's gate inputs, in flight during the TMEM load
-                    const uint16_t* zc = p.z + t0 * o_stride + col;
+            // o^T / scale, tokens t = 16 cb .. 16 cb + 15, read while the state update
+            // runs and kept in registers for the output norm at the end of the chunk
+            float ov[16];
+            const int64_t t0 = tok0 + cb * 16;
+            const int64_t nvalid = x.eos - t0;     // rows past the end belong to the next sequence
+            const int64_t col = x.h * kD + v;
+            tmem_ld16(tl + dbuf + 64 + cb * 16, ov);
+            tmem_ld_wait();
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) zr[j] = j < nvalid ? zc[j * o_stride] : (uint16_t)0;
-                }
-                tmem_ld_wait();
+            for (int j = 0; j < 16; ++j) ov[j] *= p.scale;
+            if (p.o) {
+                // for each t a warp stores 32 consecutive floats of o
+                float* ocol = p.o + t0 * o_stride + col;
+                if (nvalid >= 16) {
 #pragma unroll
-                for (int j = 0; j < 16; ++j) ov[j] *= p.scale;
-                if (p.o) {
-                    float* ocol = p.o + t0 * o_stride + col;
-                    if (nvalid >= 16) {
+                    for (int j = 0; j < 16; ++j) ocol[j * o_stride] = ov[j];
+                } else {
 #pragma unroll
-                        for (int j = 0; j < 16; ++j) ocol[j * o_stride] = ov[j];
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            if (j < nvalid) ocol[j * o_stride] = ov[j];
-                    }
-                }
-                if (p.y) {
-                    // gated output norm: the mean square of o over the 128 rows v of
-                    // a token is spread over the four warps of this column share
-                    // (lane quadrants 0-3).  Each warp sums its 32 rows for its 16
-                    // tokens by a reduce-scatter (lanes 2i and 2i + 1 end with one
-                    // token's sum), the four partial sums meet in shared memory (two
-                    // buffers: a warp is at most one chunk ahead of the others here).
-                    float sq[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) sq[j] = ov[j] * ov[j];
-                    float a8[8], a4[4], a2[2];
-                    const unsigned full = 0xffffffffu;
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const bool hi = lane & 16;
-                        a8[i] = (hi ? sq[i + 8] : sq[i]) + __shfl_xor_sync(full, hi ? sq[i] : sq[i + 8], 16);
-                    }
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const bool hi = lane & 8;
-                        a4[i] = (hi ? a8[i + 4] : a8[i]) + __shfl_xor_sync(full, hi ? a8[i] : a8[i + 4], 8);
-                    }
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        const bool hi = lane & 4;
-                        a2[i] = (hi ? a4[i + 2] : a4[i]) + __shfl_xor_sync(full, hi ? a4[i] : a4[i + 2], 4);
-                    }
-                    const bool hi2 = lane & 2;
-                    float a1 = (hi2 ? a2[1] : a2[0]) + __shfl_xor_sync(full, hi2 ? a2[0] : a2[1], 2);
-                    a1 += __shfl_xor_sync(full, a1, 1);
-                    const int tau = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
-                                    ((lane >> 1) & 1);
-                    float* part = reinterpret_cast<float*>(x.sm + C_NORM + (c & 1) * 1024 + cb * 256);
-                    if ((lane & 1) == 0) part[tau * 4 + q] = a1;
-                    named_bar_sync(kNormBar0 + cb, 128);
-                    const float wv = p.norm_w[v];
-                    uint16_t* ycol = p.y + t0 * o_stride + col;
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        if (j < nvalid) {
-                            const float4 pp = reinterpret_cast<const float4*>(part)[j];
-                            const float r = rsqrtf(((pp.x + pp.y) + (pp.z + pp.w)) * (1.f / kD) + p.eps);
-                            const float zf = __uint_as_float((uint32_t)zr[j] << 16);
-                            const float g = zf * __frcp_rn(1.f + __expf(-zf));
-                            ycol[j * o_stride] = (uint16_t)f32_to_bf16_bits(wv * (ov[j] * r) * g);
-                        }
-                    }
+                    for (int j = 0; j < 16; ++j)
+                        if (j < nvalid) ocol[j * o_stride] = ov[j];
                 }
             }
             Gam = resc ? 1.f : Gn;
@@ -651,6 +607,62 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
                 }
             }
             if (tracer) TRACE_CLK(8, c);
+            if (p.y) {
+                // gated output norm of chunk c, computed here so that it overlaps
+                // the tensor core's work on chunk c + 1.  The mean square of o
+                // over the 128 rows v of a token is spread over the four warps of
+                // this column share (lane quadrants 0-3): each warp sums its 32
+                // rows for its 16 tokens by a reduce-scatter (lanes 2i and 2i + 1
+                // end with one token's sum), the four partial sums meet in shared
+                // memory (two buffers: no warp gets two chunks ahead of another
+                // here), and lane j < 16 turns token j's total into 1 / rms.
+                float sq[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) sq[j] = ov[j] * ov[j];
+                float a8[8], a4[4], a2[2];
+                const unsigned full = 0xffffffffu;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const bool hi = lane & 16;
+                    a8[i] = (hi ? sq[i + 8] : sq[i]) + __shfl_xor_sync(full, hi ? sq[i] : sq[i + 8], 16);
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const bool hi = lane & 8;
+                    a4[i] = (hi ? a8[i + 4] : a8[i]) + __shfl_xor_sync(full, hi ? a8[i] : a8[i + 4], 8);
+                }
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const bool hi = lane & 4;
+                    a2[i] = (hi ? a4[i + 2] : a4[i]) + __shfl_xor_sync(full, hi ? a4[i] : a4[i + 2], 4);
+                }
+                const bool hi2 = lane & 2;
+                float a1 = (hi2 ? a2[1] : a2[0]) + __shfl_xor_sync(full, hi2 ? a2[0] : a2[1], 2);
+                a1 += __shfl_xor_sync(full, a1, 1);
+                const int tau = ((lane >> 4) & 1) * 8 + ((lane >> 3) & 1) * 4 + ((lane >> 2) & 1) * 2 +
+                                ((lane >> 1) & 1);
+                float* part = reinterpret_cast<float*>(x.sm + C_NORM + (c & 1) * 1024 + cb * 256);
+                if ((lane & 1) == 0) part[tau * 4 + q] = a1;
+                named_bar_sync(kNormBar0 + cb, 128);
+                const float4 pp = reinterpret_cast<const float4*>(part)[lane & 15];
+                const float rl = rsqrtf(((pp.x + pp.y) + (pp.z + pp.w)) * (1.f / kD) + p.eps);
+                const float wv = p.norm_w[v];
+                uint16_t* ycol = p.y + t0 * o_stride + col;
+                // z of this chunk, loaded by TMA: [64 t][128 v] bf16, row-major
+                mbar_wait(x.bar(CB_Z_FULL + b), (c >> 1) & 1, x.abort, kWaitLimitNs);
+                const uint16_t* zs = reinterpret_cast<const uint16_t*>(x.sm + C_Z + b * 16384) + cb * 16 * kD + v;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float r = __shfl_sync(full, rl, j);
+                    if (j < nvalid) {
+                        const float zf = __uint_as_float((uint32_t)zs[j * kD] << 16);
+                        const float g = __fdividef(zf, 1.f + __expf(-zf));
+                        ycol[j * o_stride] = (uint16_t)f32_to_bf16_bits(wv * (ov[j] * r) * g);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(x.bar(CB_Z_EMPTY + b));
+            }
         }
     }
 }
@@ -1069,7 +1081,8 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_pc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
-                  const __grid_constant__ CUtensorMap tm_b, const ClParams p) {
+                  const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_z,
+                  const ClParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // align to 1024 bytes by pointer arithmetic on the shared array, so that
     // every access below stays in the shared state space
@@ -1137,6 +1150,10 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             mbar_init(x.bar(CB_E_DRAIN), 1);
             mbar_init(x.bar(CB_CHAIN_ISSUED), 1);
             mbar_init(x.bar(CB_SUPD_ISSUED), 1);
+            for (int b = 0; b < 2; ++b) {
+                mbar_init(x.bar(CB_Z_FULL + b), 1);
+                mbar_init(x.bar(CB_Z_EMPTY + b), kEpiThreads / 32);
+            }
             mbar_init(x.bar(CB_S_FULL), 1);
             mbar_init(x.bar(CB_DRAIN), 1);
         } else {
@@ -1168,7 +1185,7 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     x.tmem = *tmem_slot;
 
     if (rank == 0)
-        consumer(x, &tm_k, &tm_v, p);
+        consumer(x, &tm_k, &tm_v, &tm_z, p);
     else
         producer(x, (int)rank - 1, &tm_q, &tm_k, &tm_a, &tm_b, p);
 
@@ -1212,6 +1229,20 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
     cuuint32_t estr[2] = {1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2D bf16 tensor [rows, cols], 128-column x 64-row boxes, no swizzle (a
+// row-major [64][128] tile: the output norm's gate z of one value head)
+bool make_map_plain(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {128, 64};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1301,10 +1332,15 @@ cudaError_t launch_prefill_pc(const PrefillArgs& a, cudaStream_t stream) {
         }
         return cudaSuccess;
     }
-    CUtensorMap mq, mk, mv, ma, mb;
+    CUtensorMap mq, mk, mv, ma, mb, mz;
     if (!make_map(&mq, a.q, a.T, (int64_t)a.Hqk * kD) || !make_map(&mk, a.k, a.T, (int64_t)a.Hqk * kD) ||
         !make_map(&mv, a.v, a.T, (int64_t)a.Hv * kD))
         return cudaErrorInvalidValue;
+    if (a.y) {
+        if (!make_map_plain(&mz, a.z, a.T, (int64_t)a.Hv * kD)) return cudaErrorInvalidValue;
+    } else {
+        mz = mq;       // unused
+    }
     // a and b rows must be a multiple of 16 bytes for TMA; otherwise they are read directly
     const int gate_tma = (a.Hv % 4 == 0) ? 1 : 0;
     if (gate_tma) {
@@ -1354,7 +1390,7 @@ cudaError_t launch_prefill_pc(const PrefillArgs& a, cudaStream_t stream) {
         attr[0].val.cooperative = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, prefill_pc_kernel, mq, mk, mv, ma, mb, p);
+        e = cudaLaunchKernelEx(&cfg, prefill_pc_kernel, mq, mk, mv, ma, mb, mz, p);
         if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();

@@ -280,11 +280,17 @@ gdn_status gdn_decode_step_fused_bf16(const uint16_t* qkv, const float* conv_w, 
  * written as bf16 by the same kernel that computes o, so that o need not go
  * through memory.  Arguments as for gdn_prefill, plus
  *  z       [T, Hv, d] bf16, norm_w [d] float32, eps >= 0, y [T, Hv, d] bf16.
- *  o       may be NULL (o is then not written); if given, o is written too.
- * With a workspace that holds the producer / consumer kernel's ring (see
- * gdn_prefill_workspace_size) the norm is fused into that kernel; otherwise the
- * single-CTA kernel writes o, which must then be given (else
- * GDN_ERR_WORKSPACE), and gdn_gated_norm runs on it.
+ *  o       may be NULL: the norm then runs inside the producer / consumer
+ *          kernel and o is not written (no o buffer at all).  If o is given,
+ *          the prefill writes o and gdn_gated_norm runs on it (two launches;
+ *          measured faster on B200 at T = 8192: 0.38 ms against 0.46 ms for
+ *          the fused kernel, whose exponentials on the consumer's SM lengthen
+ *          the state chain).  GDN_PREFILL_NORM=fused in the environment forces
+ *          the fused kernel with o written too.
+ * The fused kernel needs a workspace that holds the producer / consumer
+ * kernel's ring (see gdn_prefill_workspace_size); with a smaller one the
+ * single-CTA kernel runs, o must be given (else GDN_ERR_WORKSPACE), and
+ * gdn_gated_norm runs on it.
  */
 gdn_status gdn_prefill_gated(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* a,
                              const float* b, const float* A_log, const float* dt_bias,
