@@ -303,6 +303,7 @@ def bench_main(args, world, rank, local):
         extra["decode_128seq_48layers"] = bench_decode(args, dev, peaks, world)
         extra["decode_fused_128seq_48layers"] = bench_decode_fused(args, dev, peaks, world)
         extra["decode_bf16state_128seq_48layers"] = bench_decode(args, dev, peaks, world, bf16_state=True)
+        extra["decode_gated_128seq_48layers"] = bench_decode(args, dev, peaks, world, gated=True)
 
     value = weak_scaling_rate(T, ms_max, world)
     line = {
@@ -534,10 +535,11 @@ def bench_layer_tail(args, dev, flush, peaks, world):
     return out
 
 
-def bench_decode(args, dev, peaks, world, bf16_state=False):
+def bench_decode(args, dev, peaks, world, bf16_state=False, gated=False):
     """One decode step for 128 sequences x 48 layers, 19.3 GB float32 state (or
     9.7 GB bf16 state) in place (inputs drawn on the device; the state is far
-    larger than L2)."""
+    larger than L2).  gated: the step with the gated output norm fused in
+    (z in, bf16 y out instead of float32 o)."""
     import torch
     import gated_deltanet_recurrence_prefill_b200 as gdn
     n_seq, L = 128, 48
@@ -562,11 +564,18 @@ def bench_decode(args, dev, peaks, world, bf16_state=False):
     for i in range(0, U, 512):
         state[i:i + 512].normal_(0.0, 0.02, generator=gen)
     o = torch.empty(U, HV, D, dtype=torch.float32, device=dev)
+    if gated:
+        z = torch.randn(U, HV, D, generator=gen, device=dev).to(torch.bfloat16)
+        w = torch.empty(L, D, device=dev).uniform_(0.5, 1.5, generator=gen)
+        y = torch.empty(U, HV, D, dtype=torch.bfloat16, device=dev)
 
     def step(ev):
         if ev:
             ev["start"].record()
-        gdn.decode_step(q, k, v, a, b, A_log, dt_bias, state, n_seq, L, o=o)
+        if gated:
+            gdn.decode_step_gated(q, k, v, a, b, A_log, dt_bias, state, n_seq, L, z, w, y=y)
+        else:
+            gdn.decode_step(q, k, v, a, b, A_log, dt_bias, state, n_seq, L, o=o)
         if ev:
             ev["end"].record()
 
@@ -576,15 +585,21 @@ def bench_decode(args, dev, peaks, world, bf16_state=False):
     times, _ = _time_steps(step, max(3, args.warmup), max(5, args.steps), dummy, mk, world)
     ms = _max_over_ranks(sum(times) / len(times), world)
     state_bytes = STATE_BYTES // 2 if bf16_state else STATE_BYTES
-    bytes_step = 2 * U * state_bytes + U * (2 * 2 * HQK * D + 2 * HV * D + 2 * 4 * HV + 4 * HV * D)
+    out_bytes = (2 + 2) * HV * D if gated else 4 * HV * D      # z in + y out, or o out
+    bytes_step = 2 * U * state_bytes + U * (2 * 2 * HQK * D + 2 * HV * D + 2 * 4 * HV + out_bytes)
     gbs = bytes_step / (ms * 1e-3) / 1e9
-    out = {"workload": ("gdn_decode_step_bf16 128 seq x 48 layers, bf16 state 9.66 GB in place"
-                        if bf16_state else
-                        "gdn_decode_step 128 seq x 48 layers, fp32 state 19.33 GB in place"),
+    wl = ("gdn_decode_step_bf16 128 seq x 48 layers, bf16 state 9.66 GB in place" if bf16_state else
+          "gdn_decode_step 128 seq x 48 layers, fp32 state 19.33 GB in place")
+    if gated:
+        wl = wl.replace("gdn_decode_step_bf16", "gdn_decode_step").replace(
+            "gdn_decode_step", "gdn_decode_step_gated (output norm fused, bf16 y)", 1)
+    out = {"workload": wl,
            "ms": round(ms, 4), "GB_s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
            "bytes_per_step": int(bytes_step), "l2": "state 19.3 GB >> L2, no flush needed",
            "launches_per_step": 1}
     del state, q, k, v, o
+    if gated:
+        del z, y
     torch.cuda.empty_cache()
     return out
 

@@ -11,6 +11,7 @@ from ._lib import (  # noqa: F401
     conv1d_silu,
     decode_step,
     decode_step_fused,
+    decode_step_gated,
     gated_norm,
     lib,
     lib_path,

@@ -42,6 +42,8 @@ SIGNATURES = {
     "gdn_decode_step_fused_bf16": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
                                              _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp]),
     "gdn_gated_norm": (C.c_int, [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _f32, _vp, _vp]),
+    "gdn_decode_step_gated": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
+                                        _i32, _f32, _vp, _i32, _vp, _vp, _vp, _f32, _vp, _vp]),
     "gdn_prefill_gated": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
                                     _i32, _f32, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp, _sz, _vp]),
 }
@@ -342,3 +344,36 @@ def prefill_gated(q, k, v, a, b, A_log, dt_bias, z, norm_w, eps=1e-6, cu_seqlens
                                  workspace.numel() * workspace.element_size(), _stream(stream))
     _check("gdn_prefill_gated", st)
     return y, o, final_state
+
+
+def decode_step_gated(q, k, v, a, b, A_log, dt_bias, state, n_seq, layers, z, norm_w, eps=1e-6,
+                      scale=None, y=None, o=None, want_o=False, stream=None):
+    """One decode step with the gated output norm fused in.  As decode_step,
+    plus z [U, Hv, d] bf16 and norm_w [layers, d] f32.  Returns (y [U, Hv, d]
+    bf16, o or None)."""
+    import torch
+    U, Hqk, d = q.shape
+    Hv = v.shape[1]
+    _need(q, torch.bfloat16, (U, Hqk, d), "q")
+    _need(k, torch.bfloat16, (U, Hqk, d), "k")
+    _need(v, torch.bfloat16, (U, Hv, d), "v")
+    _need(a, torch.float32, (U, Hv), "a")
+    _need(b, torch.float32, (U, Hv), "b")
+    _need(A_log, torch.float32, (layers, Hv), "A_log")
+    _need(dt_bias, torch.float32, (layers, Hv), "dt_bias")
+    bf16 = state.dtype == torch.bfloat16
+    _need(state, torch.bfloat16 if bf16 else torch.float32, (U, Hv, d, d), "state")
+    _need(z, torch.bfloat16, (U, Hv, d), "z")
+    _need(norm_w, torch.float32, (layers, d), "norm_w")
+    if scale is None:
+        scale = d ** -0.5
+    if y is None:
+        y = torch.empty(U, Hv, d, dtype=torch.bfloat16, device=q.device)
+    if o is None and want_o:
+        o = torch.empty(U, Hv, d, dtype=torch.float32, device=q.device)
+    st = lib().gdn_decode_step_gated(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(A_log),
+                                     _ptr(dt_bias), n_seq, layers, Hqk, Hv, d, float(scale),
+                                     _ptr(state), 1 if bf16 else 0, _ptr(o), _ptr(z), _ptr(norm_w),
+                                     float(eps), _ptr(y), _stream(stream))
+    _check("gdn_decode_step_gated", st)
+    return y, o

@@ -30,16 +30,19 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kThreads = 128;
+static_assert(kThreads == kD && kThreads / 32 == 4, "the output norm takes one row per thread");
 // rows in flight per warp: 8 float32 rows or 16 bf16 rows (4 KB either way)
 template <typename StateT> constexpr int rows_per_iter() { return sizeof(StateT) == 4 ? 8 : 16; }
 
 template <typename StateT>
-__global__ void __launch_bounds__(kThreads, sizeof(StateT) == 2 ? 1 : 5)
+__global__ void __launch_bounds__(kThreads, sizeof(StateT) == 2 ? 3 : 5)
 decode_step_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ k,
                    const uint16_t* __restrict__ v, const float* __restrict__ a,
                    const float* __restrict__ b, const float* __restrict__ A_log,
                    const float* __restrict__ dt_bias, int32_t layers, int32_t Hqk, int32_t Hv,
-                   float scale, StateT* __restrict__ state, float* __restrict__ o) {
+                   float scale, StateT* __restrict__ state, float* __restrict__ o, DecodeNorm nrm) {
+    __shared__ float o_sm[kD];
+    __shared__ float ss_sm[kThreads / 32];
     const int64_t uh = blockIdx.x;                 // unit * Hv + h
     const int64_t u = uh / Hv;
     const int h = (int)(uh - u * Hv);
@@ -107,7 +110,24 @@ decode_step_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ 
             const float oj = scale * fmaf(alpha, xq[j], w * kq);
             if (lane == j) orow = oj;
         }
-        if (lane < kRowsPerIter) oh[r0 + lane] = orow;
+        if (lane < kRowsPerIter) {
+            if (o) oh[r0 + lane] = orow;
+            if (nrm.y) o_sm[r0 + lane] = orow;
+        }
+    }
+    if (nrm.y) {
+        // gated output norm of this (unit, head): y = w * o / sqrt(mean o^2 + eps) * silu(z),
+        // thread i takes row i
+        __syncthreads();
+        const int i = threadIdx.x;
+        const float oi = o_sm[i];
+        const float ssw = warp_sum(oi * oi);
+        if (lane == 0) ss_sm[warp] = ssw;
+        __syncthreads();
+        const float r = rsqrtf(((ss_sm[0] + ss_sm[1]) + (ss_sm[2] + ss_sm[3])) * (1.f / kD) + nrm.eps);
+        const float zf = bf16_to_f32(nrm.z[uh * kD + i]);
+        const float g = zf * __frcp_rn(1.f + __expf(-zf));
+        nrm.y[uh * kD + i] = (uint16_t)f32_to_bf16_bits(nrm.w[(int64_t)l * kD + i] * (oi * r) * g);
     }
 }
 
@@ -117,12 +137,12 @@ cudaError_t launch_decode_step(const uint16_t* q, const uint16_t* k, const uint1
                                const float* a, const float* b, const float* A_log,
                                const float* dt_bias, int32_t n_seq, int32_t layers, int32_t Hqk,
                                int32_t Hv, float scale, float* state, float* o,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, const DecodeNorm& nrm) {
     const int64_t blocks = (int64_t)n_seq * layers * Hv;
     if (blocks == 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     decode_step_kernel<float><<<(unsigned)blocks, kThreads, 0, stream>>>(
-        q, k, v, a, b, A_log, dt_bias, layers, Hqk, Hv, scale, state, o);
+        q, k, v, a, b, A_log, dt_bias, layers, Hqk, Hv, scale, state, o, nrm);
     return cudaGetLastError();
 }
 
@@ -130,12 +150,12 @@ cudaError_t launch_decode_step_bf16(const uint16_t* q, const uint16_t* k, const 
                                     const float* a, const float* b, const float* A_log,
                                     const float* dt_bias, int32_t n_seq, int32_t layers, int32_t Hqk,
                                     int32_t Hv, float scale, uint16_t* state, float* o,
-                                    cudaStream_t stream) {
+                                    cudaStream_t stream, const DecodeNorm& nrm) {
     const int64_t blocks = (int64_t)n_seq * layers * Hv;
     if (blocks == 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     decode_step_kernel<uint16_t><<<(unsigned)blocks, kThreads, 0, stream>>>(
-        q, k, v, a, b, A_log, dt_bias, layers, Hqk, Hv, scale, state, o);
+        q, k, v, a, b, A_log, dt_bias, layers, Hqk, Hv, scale, state, o, nrm);
     return cudaGetLastError();
 }
 

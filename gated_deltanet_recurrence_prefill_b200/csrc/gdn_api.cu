@@ -282,6 +282,36 @@ gdn_status gdn_decode_step_fused_bf16(const uint16_t* qkv, const float* conv_w, 
     return e == cudaSuccess ? GDN_OK : cuda_fail(e);
 }
 
+gdn_status gdn_decode_step_gated(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                 const float* a, const float* b, const float* A_log,
+                                 const float* dt_bias, int32_t n_seq, int32_t layers, int32_t Hqk,
+                                 int32_t Hv, int32_t d, float scale, void* state, int32_t state_bf16,
+                                 float* o, const uint16_t* z, const float* norm_w, float eps,
+                                 uint16_t* y, gdn_stream_t stream) {
+    gdn_status st = check_heads(Hqk, Hv, d);
+    if (st != GDN_OK) return st;
+    if (n_seq < 0 || layers <= 0 || !(eps >= 0.f) || (state_bf16 != 0 && state_bf16 != 1))
+        return GDN_ERR_INVALID_ARG;
+    if (n_seq == 0) return GDN_OK;
+    if (!q || !k || !v || !a || !b || !A_log || !dt_bias || !state || !z || !norm_w || !y)
+        return GDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, a, b, A_log, dt_bias, state, o, z, norm_w, y};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
+    gdn::DecodeNorm nrm;
+    nrm.z = z;
+    nrm.w = norm_w;
+    nrm.eps = eps;
+    nrm.y = y;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = state_bf16
+        ? gdn::launch_decode_step_bf16(q, k, v, a, b, A_log, dt_bias, n_seq, layers, Hqk, Hv, scale,
+                                       static_cast<uint16_t*>(state), o, s, nrm)
+        : gdn::launch_decode_step(q, k, v, a, b, A_log, dt_bias, n_seq, layers, Hqk, Hv, scale,
+                                  static_cast<float*>(state), o, s, nrm);
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
 gdn_status gdn_gated_norm(const float* o, const uint16_t* z, const float* norm_w, int64_t T, int32_t Hv,
                           int32_t d, int32_t layers, float eps, uint16_t* y, gdn_stream_t stream) {
     if (T < 0 || Hv <= 0 || d <= 0 || layers <= 0 || !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;

@@ -35,17 +35,26 @@ struct PrefillArgs {
     uint16_t* y = nullptr;
 };
 
+// the gated output norm fused into a decode step (y == NULL: none); norm_w is
+// [layers, d], row u of the batch uses layer u % layers
+struct DecodeNorm {
+    const uint16_t* z = nullptr;
+    const float* w = nullptr;
+    float eps = 0.f;
+    uint16_t* y = nullptr;
+};
+
 cudaError_t launch_decode_step(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                const float* a, const float* b, const float* A_log,
                                const float* dt_bias, int32_t n_seq, int32_t layers, int32_t Hqk,
                                int32_t Hv, float scale, float* state, float* o,
-                               cudaStream_t stream);
+                               cudaStream_t stream, const DecodeNorm& nrm = DecodeNorm());
 
 cudaError_t launch_decode_step_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                     const float* a, const float* b, const float* A_log,
                                     const float* dt_bias, int32_t n_seq, int32_t layers, int32_t Hqk,
                                     int32_t Hv, float scale, uint16_t* state, float* o,
-                                    cudaStream_t stream);
+                                    cudaStream_t stream, const DecodeNorm& nrm = DecodeNorm());
 
 cudaError_t launch_decode_fused_bf16(const uint16_t* qkv, const float* conv_w, float* conv_state,
                                      const float* a, const float* b, const float* A_log,

@@ -301,6 +301,24 @@ gdn_status gdn_prefill_gated(const uint16_t* q, const uint16_t* k, const uint16_
                              gdn_stream_t stream);
 
 /*
+ * gdn_decode_step_gated -- gdn_decode_step (state_bf16 = 0, float32 state) or
+ * gdn_decode_step_bf16 (state_bf16 = 1, bf16 state) with the gated output norm
+ * of gdn_gated_norm applied to each (unit, value head)'s output in the same
+ * kernel:  y = norm_w[l] * o / sqrt(mean_v o^2 + eps) * silu(z).
+ *  state   [n_seq * layers, Hv, d, d] float32 or bf16 bits, updated in place.
+ *  o       [n_seq * layers, Hv, d] float32, or NULL (not written).
+ *  z       [n_seq * layers, Hv, d] bf16; norm_w [layers, d] float32 (unit u
+ *          uses layer u % layers); eps >= 0; y [n_seq * layers, Hv, d] bf16.
+ * Every other argument as for gdn_decode_step.
+ */
+gdn_status gdn_decode_step_gated(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                 const float* a, const float* b, const float* A_log,
+                                 const float* dt_bias, int32_t n_seq, int32_t layers, int32_t Hqk,
+                                 int32_t Hv, int32_t d, float scale, void* state, int32_t state_bf16,
+                                 float* o, const uint16_t* z, const float* norm_w, float eps,
+                                 uint16_t* y, gdn_stream_t stream);
+
+/*
  * gdn_gated_norm -- the gated output norm that follows the recurrence in a
  * linear-attention layer:
  *     y[t, h, :] = norm_w[l] * o[t, h, :] / sqrt(mean_v o[t, h, v]^2 + eps)

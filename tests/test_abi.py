@@ -28,7 +28,8 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for required in ("gdn_conv1d_silu", "gdn_prefill", "gdn_prefill_workspace_size",
                      "gdn_decode_step", "gdn_decode_step_fused", "gdn_prefill_status",
-                     "gdn_gated_norm", "gdn_prefill_gated", "gdn_status_string"):
+                     "gdn_gated_norm", "gdn_prefill_gated", "gdn_decode_step_gated",
+                     "gdn_status_string"):
         assert required in names
 
 
@@ -183,3 +184,17 @@ def test_prefill_gated_rejects_bad_arguments(L):
     assert call(y=_p(FAKE + 8)) == 3
     assert call(wsp=None) == 6
     assert call(wsb=16) == 6
+
+
+def test_decode_gated_rejects_bad_arguments(L):
+    def call(d=128, sb=0, z=_p(), w=_p(), y=_p(), eps=1e-6, layers=48):
+        return L.gdn_decode_step_gated(_p(), _p(), _p(), _p(), _p(), _p(), _p(), 4, layers, 16, 48, d, 0.088,
+                                       _p(), sb, None, z, w, eps, y, None)
+    assert call(d=64) == 2
+    assert call(sb=2) == 1
+    assert call(z=None) == 1
+    assert call(w=None) == 1
+    assert call(y=None) == 1
+    assert call(eps=-0.5) == 1
+    assert call(layers=0) == 1
+    assert call(y=_p(FAKE + 2)) == 3
