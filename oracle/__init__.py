@@ -14,5 +14,7 @@ from .oracle import (  # noqa: F401
     beta,
     max_threads,
     prefill,
+    prefill_backward,
     prefill_chunked,
+    prefill_f64,
 )

@@ -497,3 +497,174 @@ int gdn_oracle_gated_norm(const double* o, const double* z, const double* w, int
     }
     return 0;
 }
+
+/* ---- everything in double: forward and its gradient ------------------------ */
+
+/*
+ * gdn_oracle_prefill_f64 -- the same sequential recurrence as
+ * gdn_oracle_prefill with every input in double (q, k, v, gates, initial
+ * state), for the finite-difference checks of the gradient below.  One call
+ * covers all value heads; o [T, Hv, dv] and final_state [n_seq, Hv, dv, dk]
+ * may be NULL.
+ */
+int gdn_oracle_prefill_f64(const double* q, const double* k, const double* v, const double* a,
+                           const double* b, const double* A_log, const double* dt_bias,
+                           const int32_t* cu_seqlens, int32_t n_seq, int64_t T, int32_t Hqk,
+                           int32_t Hv, int32_t dk, int32_t dv, double scale,
+                           const double* initial_state, double* o, double* final_state) {
+    if (Hqk <= 0 || Hv <= 0 || Hv % Hqk || n_seq <= 0 || T < 0) return -1;
+    if (!cu_seqlens && n_seq != 1) return -1;
+    const int grp = Hv / Hqk;
+    double* S = (double*)malloc(sizeof(double) * dv * dk);
+    double* x = (double*)malloc(sizeof(double) * dv);
+    double* ot = (double*)malloc(sizeof(double) * dv);
+    for (int n = 0; n < n_seq; ++n) {
+        const int64_t bos = cu_seqlens ? cu_seqlens[n] : 0;
+        const int64_t eos = cu_seqlens ? cu_seqlens[n + 1] : T;
+        for (int h = 0; h < Hv; ++h) {
+            const int g = h / grp;
+            for (int64_t i = 0; i < (int64_t)dv * dk; ++i)
+                S[i] = initial_state ? initial_state[((int64_t)n * Hv + h) * dv * dk + i] : 0.0;
+            for (int64_t t = bos; t < eos; ++t) {
+                const double alpha = exp(gdn_oracle_log_alpha(a[t * Hv + h], A_log[h], dt_bias[h]));
+                const double beta = gdn_oracle_beta(b[t * Hv + h]);
+                delta_step(S, dv, dk, q + (t * Hqk + g) * dk, k + (t * Hqk + g) * dk, v + (t * Hv + h) * dv,
+                           alpha, beta, scale, o ? ot : NULL, x);
+                if (o)
+                    for (int i = 0; i < dv; ++i) o[(t * Hv + h) * dv + i] = ot[i];
+            }
+            if (final_state) memcpy(final_state + ((int64_t)n * Hv + h) * dv * dk, S, sizeof(double) * dv * dk);
+        }
+    }
+    free(S); free(x); free(ot);
+    return 0;
+}
+
+/*
+ * gdn_oracle_prefill_backward -- the gradient of a scalar loss through the
+ * recurrence, by reverse-mode differentiation of each step in turn (the step
+ * of the architecture page, section 2.2, with the gate reading of
+ * gdn_oracle_log_alpha):
+ *     S_t = alpha_t S (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   S = S_{t-1},
+ *     o_t = scale S_t q_t.
+ * Given d_o = dL/do [T, Hv, dv] and d_final = dL/dS_T [n_seq, Hv, dv, dk]
+ * (NULL: 0), with G = dL/dS_t collected from the later steps plus the
+ * output's scale d_o_t q_t^T, one step back gives
+ *     dq_t += scale S_t^T d_o_t
+ *     dv_t  = beta G k                       (G k written g)
+ *     dk_t += -alpha beta (S^T g + G^T S k) + beta G^T v
+ *     dalpha = <G, S> - beta (S k).g          dbeta = -alpha (S k).g + v.g
+ *     dL/dS_{t-1} = alpha (G - beta g k^T)
+ * and through the gates (log alpha = -exp(A_log) softplus(a + dt_bias),
+ * beta = sigmoid(b)):
+ *     da_t = dalpha alpha (-exp(A_log) sigmoid(a_t + dt_bias)),
+ *     ddt_bias += da_t,  dA_log += dalpha alpha log(alpha_t),
+ *     db_t = dbeta beta (1 - beta).
+ * dq and dk sum over the value heads that share a key head.  The states S_t
+ * are kept for the whole sequence (small inputs only).  All inputs double;
+ * outputs dq, dk [T, Hqk, dk], dv [T, Hv, dv], da, db [T, Hv], dA_log,
+ * ddt_bias [Hv], d_initial [n_seq, Hv, dv, dk] (NULL: not written).
+ */
+int gdn_oracle_prefill_backward(const double* q, const double* k, const double* v, const double* a,
+                                const double* b, const double* A_log, const double* dt_bias,
+                                const int32_t* cu_seqlens, int32_t n_seq, int64_t T, int32_t Hqk,
+                                int32_t Hv, int32_t dk, int32_t dv, double scale,
+                                const double* initial_state, const double* d_o, const double* d_final,
+                                double* dq, double* dkk, double* dvv, double* da, double* db,
+                                double* dA_log, double* ddt_bias, double* d_initial) {
+    if (Hqk <= 0 || Hv <= 0 || Hv % Hqk || n_seq <= 0 || T < 0) return -1;
+    if (!cu_seqlens && n_seq != 1) return -1;
+    const int grp = Hv / Hqk;
+    const int64_t sz = (int64_t)dv * dk;
+    memset(dq, 0, sizeof(double) * T * Hqk * dk);
+    memset(dkk, 0, sizeof(double) * T * Hqk * dk);
+    memset(dA_log, 0, sizeof(double) * Hv);
+    memset(ddt_bias, 0, sizeof(double) * Hv);
+    double* G = (double*)malloc(sizeof(double) * sz);
+    double* Sk = (double*)malloc(sizeof(double) * dv);
+    double* g = (double*)malloc(sizeof(double) * dv);
+    double* x = (double*)malloc(sizeof(double) * dv);
+    for (int n = 0; n < n_seq; ++n) {
+        const int64_t bos = cu_seqlens ? cu_seqlens[n] : 0;
+        const int64_t eos = cu_seqlens ? cu_seqlens[n + 1] : T;
+        const int64_t len = eos - bos;
+        for (int h = 0; h < Hv; ++h) {
+            const int gk = h / grp;
+            /* states S_{bos-1} .. S_{eos-1}: hist[j] is the state before token bos + j */
+            double* hist = (double*)malloc(sizeof(double) * sz * (len + 1));
+            for (int64_t i = 0; i < sz; ++i)
+                hist[i] = initial_state ? initial_state[((int64_t)n * Hv + h) * sz + i] : 0.0;
+            for (int64_t j = 0; j < len; ++j) {
+                const int64_t t = bos + j;
+                memcpy(hist + (j + 1) * sz, hist + j * sz, sizeof(double) * sz);
+                const double alpha = exp(gdn_oracle_log_alpha(a[t * Hv + h], A_log[h], dt_bias[h]));
+                const double beta = gdn_oracle_beta(b[t * Hv + h]);
+                delta_step(hist + (j + 1) * sz, dv, dk, q + (t * Hqk + gk) * dk, k + (t * Hqk + gk) * dk,
+                           v + (t * Hv + h) * dv, alpha, beta, scale, NULL, x);
+            }
+            for (int64_t i = 0; i < sz; ++i) G[i] = d_final ? d_final[((int64_t)n * Hv + h) * sz + i] : 0.0;
+            for (int64_t j = len - 1; j >= 0; --j) {
+                const int64_t t = bos + j;
+                const double* S = hist + j * sz;          /* S_{t-1} */
+                const double* St = hist + (j + 1) * sz;   /* S_t */
+                const double* qt = q + (t * Hqk + gk) * dk;
+                const double* kt = k + (t * Hqk + gk) * dk;
+                const double* vt = v + (t * Hv + h) * dv;
+                const double* dot = d_o + (t * Hv + h) * dv;
+                const double la = gdn_oracle_log_alpha(a[t * Hv + h], A_log[h], dt_bias[h]);
+                const double alpha = exp(la);
+                const double beta = gdn_oracle_beta(b[t * Hv + h]);
+                /* the output of step t: o_t = scale S_t q_t */
+                for (int e = 0; e < dk; ++e) {
+                    double acc = 0.0;
+                    for (int i = 0; i < dv; ++i) acc += St[(int64_t)i * dk + e] * dot[i];
+                    dq[(t * Hqk + gk) * dk + e] += scale * acc;
+                }
+                for (int i = 0; i < dv; ++i)
+                    for (int e = 0; e < dk; ++e) G[(int64_t)i * dk + e] += scale * dot[i] * qt[e];
+                /* back through the update */
+                double GS = 0.0;
+                for (int64_t i = 0; i < sz; ++i) GS += G[i] * S[i];
+                for (int i = 0; i < dv; ++i) {
+                    double s1 = 0.0, s2 = 0.0;
+                    for (int e = 0; e < dk; ++e) {
+                        s1 += S[(int64_t)i * dk + e] * kt[e];
+                        s2 += G[(int64_t)i * dk + e] * kt[e];
+                    }
+                    Sk[i] = s1;
+                    g[i] = s2;
+                }
+                double Skg = 0.0, vg = 0.0;
+                for (int i = 0; i < dv; ++i) { Skg += Sk[i] * g[i]; vg += vt[i] * g[i]; }
+                const double dalpha = GS - beta * Skg;
+                const double dbeta = -alpha * Skg + vg;
+                for (int i = 0; i < dv; ++i) dvv[(t * Hv + h) * dv + i] = beta * g[i];
+                for (int e = 0; e < dk; ++e) {
+                    double sg = 0.0, gs = 0.0, gv = 0.0;
+                    for (int i = 0; i < dv; ++i) {
+                        sg += S[(int64_t)i * dk + e] * g[i];
+                        gs += G[(int64_t)i * dk + e] * Sk[i];
+                        gv += G[(int64_t)i * dk + e] * vt[i];
+                    }
+                    dkk[(t * Hqk + gk) * dk + e] += -alpha * beta * (sg + gs) + beta * gv;
+                }
+                const double xg = a[t * Hv + h] + dt_bias[h];
+                const double sig = 1.0 / (1.0 + exp(-xg));
+                const double dla = dalpha * alpha;
+                const double dat = dla * (-exp(A_log[h]) * sig);
+                da[t * Hv + h] = dat;
+                ddt_bias[h] += dat;
+                dA_log[h] += dla * la;
+                db[t * Hv + h] = dbeta * beta * (1.0 - beta);
+                /* dL/dS_{t-1} = alpha (G - beta g k^T) */
+                for (int i = 0; i < dv; ++i)
+                    for (int e = 0; e < dk; ++e)
+                        G[(int64_t)i * dk + e] = alpha * (G[(int64_t)i * dk + e] - beta * g[i] * kt[e]);
+            }
+            if (d_initial) memcpy(d_initial + ((int64_t)n * Hv + h) * sz, G, sizeof(double) * sz);
+            free(hist);
+        }
+    }
+    free(G); free(Sk); free(g); free(x);
+    return 0;
+}

@@ -47,6 +47,12 @@ def _bind(lib):
     lib.gdn_oracle_beta.argtypes = [dbl]
     lib.gdn_oracle_gated_norm.restype = C.c_int
     lib.gdn_oracle_gated_norm.argtypes = [vp, vp, vp, i64, C.c_int, C.c_int, C.c_int, dbl, vp]
+    lib.gdn_oracle_prefill_f64.restype = C.c_int
+    lib.gdn_oracle_prefill_f64.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32,
+                                           dbl, vp, vp, vp]
+    lib.gdn_oracle_prefill_backward.restype = C.c_int
+    lib.gdn_oracle_prefill_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32,
+                                                i32, dbl, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.gdn_oracle_max_threads.restype = C.c_int
     lib.gdn_oracle_max_threads.argtypes = [C.c_int]
     return lib
@@ -233,3 +239,61 @@ def gated_norm(o, z, norm_w, eps=1e-6, lib=None):
     if rc != 0:
         raise ValueError("oracle gated_norm rejected its arguments")
     return y
+
+
+
+def _f64(x):
+    return None if x is None else np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _widen(x):
+    """bf16 bits (uint16) -> float64 exactly; anything else -> float64."""
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        return (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def prefill_f64(q, k, v, a, b, A_log, dt_bias, cu_seqlens=None, scale=None, initial_state=None,
+                lib=None):
+    """The sequential recurrence with every input in float64 (gdn_oracle_prefill_f64).
+    Returns (o [T, Hv, dv], final_state [N, Hv, dv, dk])."""
+    q, k, v = _widen(q), _widen(k), _widen(v)
+    T, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    cu = None if cu_seqlens is None else np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    n_seq = 1 if cu is None else len(cu) - 1
+    scale = 1.0 / np.sqrt(dk) if scale is None else float(scale)
+    o = np.zeros((T, Hv, dv))
+    fs = np.zeros((n_seq, Hv, dv, dk))
+    rc = _L(lib).gdn_oracle_prefill_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(_f64(a)), _ptr(_f64(b)),
+                                        _ptr(_f64(A_log)), _ptr(_f64(dt_bias)), _ptr(cu), n_seq, T, Hqk,
+                                        Hv, dk, dv, scale, _ptr(_f64(initial_state)), _ptr(o), _ptr(fs))
+    if rc != 0:
+        raise ValueError("oracle prefill_f64 rejected its arguments")
+    return o, fs
+
+
+def prefill_backward(q, k, v, a, b, A_log, dt_bias, d_o, d_final=None, cu_seqlens=None, scale=None,
+                     initial_state=None, lib=None):
+    """Gradient of <d_o, o> + <d_final, S_T> through the recurrence, in float64
+    (gdn_oracle_prefill_backward).  Returns a dict with dq, dk [T, Hqk, dk],
+    dv [T, Hv, dv], da, db [T, Hv], dA_log, ddt_bias [Hv] and d_initial
+    [N, Hv, dv, dk]."""
+    q, k, v = _widen(q), _widen(k), _widen(v)
+    T, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    cu = None if cu_seqlens is None else np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    n_seq = 1 if cu is None else len(cu) - 1
+    scale = 1.0 / np.sqrt(dk) if scale is None else float(scale)
+    out = dict(dq=np.zeros((T, Hqk, dk)), dk=np.zeros((T, Hqk, dk)), dv=np.zeros((T, Hv, dv)),
+               da=np.zeros((T, Hv)), db=np.zeros((T, Hv)), dA_log=np.zeros(Hv), ddt_bias=np.zeros(Hv),
+               d_initial=np.zeros((n_seq, Hv, dv, dk)))
+    rc = _L(lib).gdn_oracle_prefill_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(_f64(a)), _ptr(_f64(b)), _ptr(_f64(A_log)), _ptr(_f64(dt_bias)),
+        _ptr(cu), n_seq, T, Hqk, Hv, dk, dv, scale, _ptr(_f64(initial_state)), _ptr(_f64(d_o)),
+        _ptr(_f64(d_final)), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["da"]),
+        _ptr(out["db"]), _ptr(out["dA_log"]), _ptr(out["ddt_bias"]), _ptr(out["d_initial"]))
+    if rc != 0:
+        raise ValueError("oracle prefill_backward rejected its arguments")
+    return out

@@ -42,6 +42,12 @@ MUTANTS = {
                              "dst[e] = scale * (inter + intra);"),
     "chunk_substitution_sign": ("val -= A[i * C + m] * Tm[m * C + j];", "val += A[i * C + m] * Tm[m * C + j];"),
     "norm_sum_not_mean": ("1.0 / sqrt(ss / d + eps)", "1.0 / sqrt(ss + eps)"),
+    "bw_dk_one_sided": ("-alpha * beta * (sg + gs) + beta * gv", "-alpha * beta * (2.0 * sg) + beta * gv"),
+    "bw_dalpha_no_erase": ("const double dalpha = GS - beta * Skg;", "const double dalpha = GS;"),
+    "bw_state_no_decay": ("G[(int64_t)i * dk + e] = alpha * (G[(int64_t)i * dk + e] - beta * g[i] * kt[e]);",
+                          "G[(int64_t)i * dk + e] = G[(int64_t)i * dk + e] - beta * g[i] * kt[e];"),
+    "bw_output_from_old_state": ("acc += St[(int64_t)i * dk + e] * dot[i];", "acc += S[(int64_t)i * dk + e] * dot[i];"),
+    "bw_gate_sign": ("const double dat = dla * (-exp(A_log[h]) * sig);", "const double dat = dla * (exp(A_log[h]) * sig);"),
     "norm_no_eps": ("1.0 / sqrt(ss / d + eps)", "1.0 / sqrt(ss / d)"),
     "gate_sigmoid_only": ("const double g = z[row + e] / (1.0 + exp(-z[row + e]));",
                           "const double g = 1.0 / (1.0 + exp(-z[row + e]));"),

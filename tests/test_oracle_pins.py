@@ -472,3 +472,83 @@ def test_gated_norm_layer_of_each_row(orc):
     y = orc.gated_norm(o, z, w)
     for t in range(T):
         assert np.allclose(y[t], (t % layers + 1) * y[0], rtol=1e-14, atol=0)
+
+
+# ---- the backward pass: gradients pinned by central finite differences ----------
+
+def _bw_case(seed=0, lengths=(5, 3), Hqk=1, Hv=2, d=4):
+    rng = np.random.default_rng(seed)
+    T = sum(lengths)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    q = rng.standard_normal((T, Hqk, d)) / np.sqrt(d)
+    k = rng.standard_normal((T, Hqk, d))
+    k /= np.linalg.norm(k, axis=-1, keepdims=True)
+    return dict(q=q, k=k, v=rng.standard_normal((T, Hv, d)), a=rng.standard_normal((T, Hv)),
+                b=rng.standard_normal((T, Hv)), A_log=np.log(rng.uniform(1, 4, Hv)),
+                dt_bias=rng.uniform(-3, 0, Hv), cu_seqlens=cu,
+                initial_state=0.3 * rng.standard_normal((len(lengths), Hv, d, d))), \
+        rng.standard_normal((T, Hv, d)), rng.standard_normal((len(lengths), Hv, d, d))
+
+
+def test_prefill_f64_equals_prefill(orc):
+    # float-representable gates: the all-double forward is the forward
+    inp, _, _ = _bw_case(1)
+    f32 = {n: inp[n].astype(np.float32) for n in ("a", "b", "A_log", "dt_bias", "initial_state")}
+    o1, s1 = orc.prefill_f64(inp["q"], inp["k"], inp["v"], f32["a"], f32["b"], f32["A_log"], f32["dt_bias"],
+                             cu_seqlens=inp["cu_seqlens"], initial_state=f32["initial_state"])
+    o2, s2 = orc.prefill(inp["q"], inp["k"], inp["v"], f32["a"], f32["b"], f32["A_log"], f32["dt_bias"],
+                         cu_seqlens=inp["cu_seqlens"], initial_state=f32["initial_state"])
+    assert np.allclose(o1, o2, rtol=0, atol=1e-14) and np.allclose(s1, s2, rtol=0, atol=1e-14)
+
+
+def test_backward_matches_finite_differences(orc):
+    for seed in (0, 3):
+        _backward_vs_finite_differences(orc, seed)
+
+
+def _backward_vs_finite_differences(orc, seed):
+    inp, d_o, d_fin = _bw_case(seed)
+
+    def loss(**over):
+        x = dict(inp, **over)
+        o, s = orc.prefill_f64(x["q"], x["k"], x["v"], x["a"], x["b"], x["A_log"], x["dt_bias"],
+                               cu_seqlens=x["cu_seqlens"], initial_state=x["initial_state"])
+        return float(np.sum(d_o * o) + np.sum(d_fin * s))
+
+    g = orc.prefill_backward(inp["q"], inp["k"], inp["v"], inp["a"], inp["b"], inp["A_log"], inp["dt_bias"],
+                             d_o, d_final=d_fin, cu_seqlens=inp["cu_seqlens"],
+                             initial_state=inp["initial_state"])
+    names = {"q": "dq", "k": "dk", "v": "dv", "a": "da", "b": "db", "A_log": "dA_log",
+             "dt_bias": "ddt_bias", "initial_state": "d_initial"}
+    h = 1e-6
+    for name, gname in names.items():
+        base = inp[name]
+        fd = np.zeros_like(base)
+        for idx in np.ndindex(base.shape):
+            xp, xm = base.copy(), base.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            fd[idx] = (loss(**{name: xp}) - loss(**{name: xm})) / (2 * h)
+        scale_ = max(1.0, np.max(np.abs(fd)))
+        assert np.max(np.abs(g[gname] - fd)) <= 2e-7 * scale_, name
+
+
+def test_backward_of_a_sum_over_heads(orc):
+    # dq and dk collect every value head of the key group: with two key heads of two
+    # value heads each, the gradient equals the sum of the per-head gradients taken alone
+    inp, d_o, d_fin = _bw_case(5, lengths=(6,), Hqk=2, Hv=4)
+    g = orc.prefill_backward(**{n: inp[n] for n in ("q", "k", "v", "a", "b", "A_log", "dt_bias")},
+                             d_o=d_o, d_final=d_fin, cu_seqlens=inp["cu_seqlens"], initial_state=inp["initial_state"])
+    for gk in range(2):
+        acc_q = np.zeros_like(g["dq"][:, gk])
+        acc_k = np.zeros_like(g["dk"][:, gk])
+        for h in (2 * gk, 2 * gk + 1):
+            sub = dict(q=inp["q"][:, gk:gk + 1], k=inp["k"][:, gk:gk + 1], v=inp["v"][:, h:h + 1],
+                       a=inp["a"][:, h:h + 1], b=inp["b"][:, h:h + 1], A_log=inp["A_log"][h:h + 1],
+                       dt_bias=inp["dt_bias"][h:h + 1])
+            gh = orc.prefill_backward(**sub, d_o=d_o[:, h:h + 1], d_final=d_fin[:, h:h + 1],
+                                      cu_seqlens=inp["cu_seqlens"], initial_state=inp["initial_state"][:, h:h + 1])
+            acc_q += gh["dq"][:, 0]
+            acc_k += gh["dk"][:, 0]
+        assert np.allclose(g["dq"][:, gk], acc_q, rtol=1e-13, atol=1e-15)
+        assert np.allclose(g["dk"][:, gk], acc_k, rtol=1e-13, atol=1e-15)
