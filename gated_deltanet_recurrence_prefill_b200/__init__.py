@@ -16,6 +16,7 @@ from ._lib import (  # noqa: F401
     lib,
     lib_path,
     prefill,
+    prefill_backward,
     prefill_gated,
     prefill_noalloc,
     prefill_status,

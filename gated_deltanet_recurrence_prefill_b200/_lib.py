@@ -42,6 +42,10 @@ SIGNATURES = {
     "gdn_decode_step_fused_bf16": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
                                              _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp]),
     "gdn_gated_norm": (C.c_int, [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _f32, _vp, _vp]),
+    "gdn_prefill_backward_workspace_size": (_sz, [_i32, _i64, _i32, _i32]),
+    "gdn_prefill_backward": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
+                                       _i32, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                       _vp, _vp, _sz, _vp]),
     "gdn_decode_step_gated": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
                                         _i32, _f32, _vp, _i32, _vp, _vp, _vp, _f32, _vp, _vp]),
     "gdn_prefill_gated": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
@@ -377,3 +381,47 @@ def decode_step_gated(q, k, v, a, b, A_log, dt_bias, state, n_seq, layers, z, no
                                      float(eps), _ptr(y), _stream(stream))
     _check("gdn_decode_step_gated", st)
     return y, o
+
+
+def prefill_backward(q, k, v, a, b, A_log, dt_bias, d_o, d_final_state=None, cu_seqlens=None,
+                     scale=None, initial_state=None, want_d_initial=True, workspace=None, stream=None):
+    """gdn_prefill_backward: gradients of a loss with dL/do = d_o [T, Hv, d] and
+    dL/dS_T = d_final_state [N, Hv, d, d] (or zero).  Returns a dict of float32
+    tensors dq, dk [T, Hqk, d], dv [T, Hv, d], da, db [T, Hv], dA_log,
+    ddt_bias [Hv] and d_initial_state [N, Hv, d, d] (or None)."""
+    import torch
+    T, Hqk, d = q.shape
+    Hv = v.shape[1]
+    n_seq = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _need(q, torch.bfloat16, (T, Hqk, d), "q")
+    _need(k, torch.bfloat16, (T, Hqk, d), "k")
+    _need(v, torch.bfloat16, (T, Hv, d), "v")
+    _need(a, torch.float32, (T, Hv), "a")
+    _need(b, torch.float32, (T, Hv), "b")
+    _need(A_log, torch.float32, (Hv,), "A_log")
+    _need(dt_bias, torch.float32, (Hv,), "dt_bias")
+    _need(d_o, torch.float32, (T, Hv, d), "d_o")
+    if cu_seqlens is not None:
+        _need(cu_seqlens, torch.int32, (n_seq + 1,), "cu_seqlens")
+    if initial_state is not None:
+        _need(initial_state, torch.float32, (n_seq, Hv, d, d), "initial_state")
+    if d_final_state is not None:
+        _need(d_final_state, torch.float32, (n_seq, Hv, d, d), "d_final_state")
+    if scale is None:
+        scale = d ** -0.5
+    dev = q.device
+    f = lambda *shape: torch.empty(*shape, dtype=torch.float32, device=dev)
+    out = dict(dq=f(T, Hqk, d), dk=f(T, Hqk, d), dv=f(T, Hv, d), da=f(T, Hv), db=f(T, Hv),
+               dA_log=f(Hv), ddt_bias=f(Hv),
+               d_initial_state=f(n_seq, Hv, d, d) if want_d_initial else None)
+    ws_bytes = lib().gdn_prefill_backward_workspace_size(n_seq, T, Hv, d)
+    if workspace is None:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    st = lib().gdn_prefill_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias), _ptr(cu_seqlens), n_seq, T,
+        Hqk, Hv, d, float(scale), _ptr(initial_state), _ptr(d_o), _ptr(d_final_state), _ptr(out["dq"]),
+        _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["da"]), _ptr(out["db"]), _ptr(out["dA_log"]),
+        _ptr(out["ddt_bias"]), _ptr(out["d_initial_state"]), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("gdn_prefill_backward", st)
+    return out

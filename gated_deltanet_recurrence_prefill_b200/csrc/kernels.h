@@ -73,6 +73,36 @@ cudaError_t launch_conv1d_silu(const uint16_t* qkv, const float* w, const int32_
                                const float* cs_in, float* cs_out, uint16_t* q, uint16_t* k,
                                uint16_t* v, cudaStream_t stream);
 
+struct BackwardArgs {
+    const uint16_t* q;
+    const uint16_t* k;
+    const uint16_t* v;
+    const float* a;
+    const float* b;
+    const float* A_log;
+    const float* dt_bias;
+    const int32_t* cu_seqlens;     // NULL: one sequence of length T
+    int32_t n_seq;
+    int64_t T;
+    int32_t Hqk;
+    int32_t Hv;
+    float scale;
+    const float* initial_state;    // may be NULL
+    const float* d_o;
+    const float* d_final_state;    // may be NULL
+    float* dq;
+    float* dk;
+    float* dv;
+    float* da;
+    float* db;
+    float* dA_log;
+    float* ddt_bias;
+    float* d_initial_state;        // may be NULL
+    void* workspace;
+};
+size_t backward_workspace_bytes(int32_t n_seq, int64_t T, int32_t Hv);
+cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t stream);
+
 cudaError_t launch_gated_norm(const float* o, const uint16_t* z, const float* w, int64_t T, int32_t Hv,
                               int32_t layers, float eps, uint16_t* y, cudaStream_t stream);
 cudaError_t launch_prefill_simt(const PrefillArgs& p, cudaStream_t stream);

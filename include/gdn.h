@@ -319,6 +319,42 @@ gdn_status gdn_decode_step_gated(const uint16_t* q, const uint16_t* k, const uin
                                  uint16_t* y, gdn_stream_t stream);
 
 /*
+ * gdn_prefill_backward_workspace_size -- bytes of device workspace
+ * gdn_prefill_backward needs (a multiple of 256): a float32 state checkpoint per
+ * 64-token chunk ((T / 64 + n_seq + 1) * Hv * d * d * 4), the 64 states of one
+ * chunk per (sequence, value head) (n_seq * Hv * 64 * d * d * 4), dq and dk per
+ * value head (2 * T * Hv * d * 4) and the gate-parameter sums.  Host-only.
+ */
+size_t gdn_prefill_backward_workspace_size(int32_t n_seq, int64_t T, int32_t Hv, int32_t d);
+
+/*
+ * gdn_prefill_backward -- the gradient of a scalar loss L through the
+ * recurrence of gdn_prefill (reverse-mode, one token at a time):
+ *     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *     o_t = scale S_t q_t,  alpha = exp(-exp(A_log) softplus(a + dt_bias)),
+ *     beta = sigmoid(b)   (architecture page section 2.2, gate reading as for
+ *     gdn_prefill).
+ * Inputs as for gdn_prefill, plus
+ *  d_o            [T, Hv, d] float32: dL/do.
+ *  d_final_state  [n_seq, Hv, d_v, d_k] float32 or NULL (zero): dL/dS_T.
+ * Outputs (float32, written in full; caller-owned):
+ *  dq, dk         [T, Hqk, d] (summed over the value heads of each key head)
+ *  dv             [T, Hv, d];  da, db [T, Hv];  dA_log, ddt_bias [Hv]
+ *  d_initial_state [n_seq, Hv, d_v, d_k] or NULL (not written).
+ * workspace: gdn_prefill_backward_workspace_size() bytes, 256-byte aligned.
+ * The kernel runs on CUDA cores (one CTA per (sequence, value head), every
+ * token in turn, float32 arithmetic); the result is deterministic.
+ */
+gdn_status gdn_prefill_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* a,
+                                const float* b, const float* A_log, const float* dt_bias,
+                                const int32_t* cu_seqlens, int32_t n_seq, int64_t T, int32_t Hqk,
+                                int32_t Hv, int32_t d, float scale, const float* initial_state,
+                                const float* d_o, const float* d_final_state, float* dq, float* dk,
+                                float* dv, float* da, float* db, float* dA_log, float* ddt_bias,
+                                float* d_initial_state, void* workspace, size_t workspace_bytes,
+                                gdn_stream_t stream);
+
+/*
  * gdn_gated_norm -- the gated output norm that follows the recurrence in a
  * linear-attention layer:
  *     y[t, h, :] = norm_w[l] * o[t, h, :] / sqrt(mean_v o[t, h, v]^2 + eps)

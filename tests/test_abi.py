@@ -29,7 +29,7 @@ def test_header_declares_the_entry_points():
     for required in ("gdn_conv1d_silu", "gdn_prefill", "gdn_prefill_workspace_size",
                      "gdn_decode_step", "gdn_decode_step_fused", "gdn_prefill_status",
                      "gdn_gated_norm", "gdn_prefill_gated", "gdn_decode_step_gated",
-                     "gdn_status_string"):
+                     "gdn_prefill_backward", "gdn_prefill_backward_workspace_size", "gdn_status_string"):
         assert required in names
 
 
@@ -198,3 +198,28 @@ def test_decode_gated_rejects_bad_arguments(L):
     assert call(eps=-0.5) == 1
     assert call(layers=0) == 1
     assert call(y=_p(FAKE + 2)) == 3
+
+
+def test_backward_workspace_formula(L):
+    # gdn.h: checkpoints + one chunk of states per unit + dq, dk per value head + gate sums
+    for n, T, Hv in ((1, 8192, 48), (16, 241567, 48), (3, 100, 6)):
+        d = 128
+        want = ((T // 64 + n + 1) * Hv * d * d * 4 + n * Hv * 64 * d * d * 4 + 2 * T * Hv * d * 4
+                + n * Hv * 2 * 4)
+        want = (want + 255) // 256 * 256
+        assert L.gdn_prefill_backward_workspace_size(n, T, Hv, d) == want
+
+
+def test_backward_rejects_bad_arguments(L):
+    ws = L.gdn_prefill_backward_workspace_size(1, 64, 48, 128)
+
+    def call(d=128, d_o=_p(), dq=_p(), dA=_p(), wsp=_p(0x20000), wsb=ws):
+        return L.gdn_prefill_backward(_p(), _p(), _p(), _p(), _p(), _p(), _p(), None, 1, 64, 16, 48, d, 0.088,
+                                      None, d_o, None, dq, _p(), _p(), _p(), _p(), dA, _p(), None, wsp, wsb, None)
+    assert call(d=64) == 2
+    assert call(d_o=None) == 1
+    assert call(dq=None) == 1
+    assert call(dA=None) == 1
+    assert call(dq=_p(FAKE + 4)) == 3
+    assert call(wsb=ws - 256) == 6
+    assert call(wsp=_p(0x20000 + 16)) == 3
