@@ -300,6 +300,7 @@ def bench_main(args, world, rank, local):
             args, dev, flush, peaks, world, lengths=synth.varlen_lengths(3), seed=3)
         extra["gated_norm_T8192"] = bench_gated_norm(args, dev, flush, peaks, world)
         extra["layer_tail_T8192"] = bench_layer_tail(args, dev, flush, peaks, world)
+        extra["backward_T8192"] = bench_backward(args, dev, flush, peaks, world)
         extra["decode_128seq_48layers"] = bench_decode(args, dev, peaks, world)
         extra["decode_fused_128seq_48layers"] = bench_decode_fused(args, dev, peaks, world)
         extra["decode_bf16state_128seq_48layers"] = bench_decode(args, dev, peaks, world, bf16_state=True)
@@ -531,6 +532,52 @@ def bench_layer_tail(args, dev, flush, peaks, world):
            "GB_s": round(bytes_f / (ms_f * 1e-3) / 1e9, 1), "bytes_per_step": int(bytes_f),
            "launches_per_step": 1}
     del q, k, v, a, b, z, o, y
+    torch.cuda.empty_cache()
+    return out
+
+
+def bench_backward(args, dev, flush, peaks, world):
+    """gdn_prefill_backward at T = 8192 (one sequence, 16 / 48 heads, S0 and
+    dL/dS_T given): all gradients of the recurrence."""
+    import torch
+    import gated_deltanet_recurrence_prefill_b200 as gdn
+    T = T_MAIN
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(8)
+
+    def unit(shape):
+        x = torch.randn(*shape, generator=gen, device=dev)
+        return (x / torch.sqrt((x * x).sum(-1, keepdim=True) + 1e-6)).to(torch.bfloat16)
+
+    q, k = unit((T, HQK, D)), unit((T, HQK, D))
+    v = torch.randn(T, HV, D, generator=gen, device=dev).to(torch.bfloat16)
+    a = torch.randn(T, HV, generator=gen, device=dev)
+    b = torch.randn(T, HV, generator=gen, device=dev)
+    A_log = torch.log(torch.empty(HV, device=dev).uniform_(1, 16, generator=gen))
+    dt = torch.exp(torch.empty(HV, device=dev).uniform_(-6.907755, -2.302585, generator=gen))
+    dt_bias = torch.log(torch.expm1(dt))
+    s0 = 0.02 * torch.randn(1, HV, D, D, generator=gen, device=dev)
+    d_o = torch.randn(T, HV, D, generator=gen, device=dev)
+    d_fin = 0.1 * torch.randn(1, HV, D, D, generator=gen, device=dev)
+    ws = torch.empty(gdn.lib().gdn_prefill_backward_workspace_size(1, T, HV, D), dtype=torch.uint8, device=dev)
+
+    def step(ev):
+        if ev:
+            ev["start"].record()
+        gdn.prefill_backward(q, k, v, a, b, A_log, dt_bias, d_o, d_final_state=d_fin, initial_state=s0,
+                             workspace=ws)
+        if ev:
+            ev["end"].record()
+
+    mk = lambda: {"start": torch.cuda.Event(enable_timing=True),
+                  "end": torch.cuda.Event(enable_timing=True)}
+    times, _ = _time_steps(step, 3, 3, flush, mk, world)
+    ms = _max_over_ranks(sum(times) / len(times), world)
+    out = {"workload": f"gdn_prefill_backward T={T} N=1 Hqk=16 Hv=48 d=128, S0 and dL/dS_T given "
+                       "(CUDA cores, one CTA per value head, token by token)",
+           "ms": round(ms, 3), "tokens_per_s_layer": round(weak_scaling_rate(T, ms, world), 1),
+           "launches_per_step": 3}
+    del q, k, v, d_o, ws
     torch.cuda.empty_cache()
     return out
 
