@@ -16,8 +16,10 @@
 // Everything up to [-W; Qh] and [T beta; R beta] is independent of the state.
 //
 // Producers (roles 1..P, P = 1 or 2).  Producer p takes chunks p,
-// p + P, ...; inside it two groups of 8 warps take alternate chunks.  A group
-// computes the gates, D0 = [K; Q] K^T (tcgen05), A and P, T by blocked forward
+// p + P, ...; inside it two groups of 8 warps take alternate chunks.  A thread
+// per group (warps 19, 20) issues D0 = [K; Q] K^T (tcgen05) as soon as the
+// chunk's [K; Q] lands and the group has read the previous D0.  A group
+// computes the gates, A and P from D0, T by blocked forward
 // substitution (16x16 diagonal blocks on CUDA cores, off-diagonal blocks with
 // tf32 mma.sync), R = P T (tcgen05), the scaled bf16 copies [R bg; T bg] and
 // [T b; R b], X1 = [R bg; T bg] K (tcgen05) and from it -W and Qh.  It stages
@@ -179,6 +181,8 @@ enum {
     // producer
     PB_KQ_FULL = 0, PB_KQ_TAKEN = 2, PB_KQ_EMPTY = 4, PB_D0_FULL = 7, PB_R_FULL = 9,
     PB_X1_FULL = 11, PB_DRAIN = 13, PB_STAGED = 15, PB_AF_FREE = 17,
+    // (producer and consumer CTAs use the slots from 19 on for different barriers)
+    PB_D0_FREE = 19, PB_D0_DRAIN = 21,
     // consumer
     CB_RECV_FULL = 19, CB_K_FULL = 21, CB_V_FULL = 23, CB_V_EMPTY = 25, CB_SLOT_FREE = 27,
     CB_D_FULL = 29, CB_S_FULL = 30, CB_DRAIN = 31, CB_REL_DONE = 32, CB_K_EMPTY = 34,
@@ -754,6 +758,39 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
         }
         return;
     }
+    if (warp == 19 || warp == 20) {
+        // ------------------------------------------------ D0 = [K; Q] K^T of one group
+        // Issued as soon as the chunk's [K; Q] has landed and the group has read
+        // the previous D0, by a thread of its own (a thread that issues
+        // tcgen05.mma is held until the tensor core takes them), so that D0 is
+        // ready when the group turns to the chunk.
+        const int grp = warp - 19;
+        if (lane == 0) {
+            const uint64_t dsc_kq0 = sdesc_sw128(x.sbase + P_KQ, 16, 1024);
+            constexpr uint64_t kStageStep = KQ_STAGE >> 4;
+            const uint32_t tg = x.tmem + 256u * grp;
+            for (int jj = 0;; ++jj) {
+                const int i = grp + 2 * jj;
+                const int c = pidx + p.n_prod * i;
+                if (c >= nch) break;
+                const int s = i % kKqStages;
+                if (!mbar_wait(x.bar(PB_KQ_FULL + grp), jj & 1, x.abort, kWaitLimitNs)) break;
+                mbar_arrive(x.bar(PB_KQ_TAKEN + grp));
+                if (jj >= 1 && !mbar_wait(x.bar(PB_D0_FREE + grp), (jj - 1) & 1, x.abort, kWaitLimitNs)) break;
+                tc_fence_after();
+                const uint64_t d = dsc_kq0 + s * kStageStep;
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t off = ((kk >> 2) * KQ_PANEL + (kk & 3) * 32) >> 4;
+                    mma_bf16(tg + PCOL_D0, d + off, d + off, IDESC_D0, kk > 0);
+                }
+                mma_commit(x.bar(PB_D0_FULL + grp));
+            }
+            volatile int no_abort = 0;
+            mma_commit(x.bar(PB_D0_DRAIN + grp));
+            mbar_wait(x.bar(PB_D0_DRAIN + grp), 0, &no_abort, kWaitLimitNs);
+        }
+        return;
+    }
     if (warp >= 16) return;
     // ---------------------------------------------------- precompute group
     const int grp = warp >> 3;                 // 0 or 1
@@ -799,17 +836,6 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
         if (pw == 0 && lane == 0) TRACE_CLK(17, c);
         __syncwarp();
         if (lane == 0) mbar_arrive(x.bar(PB_KQ_TAKEN + grp));
-        if (issuer) {
-            // D0 = [K; Q] K^T
-            tc_fence_after();
-            const uint64_t d = dsc_kq0 + s * kStageStep;
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint64_t off = ((kk >> 2) * KQ_PANEL + (kk & 3) * 32) >> 4;
-                mma_bf16(tg + PCOL_D0, d + off, d + off, IDESC_D0, kk > 0);
-            }
-            mma_commit(x.bar(PB_D0_FULL + grp));
-        }
-        __syncwarp();
         // ---- gates (warps 6, 7 of the group): G = running sum of log2(alpha);
         //      beta; gamma = 2^G; kappa = 2^{G_C - G}
         if (pw >= 6) {
@@ -907,6 +933,8 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
         }
         tc_fence_before();
         named_bar_sync(nb, kGroupThreads);
+        // D0 has been read: the next chunk's D0 may be issued into it
+        if (pw == 0 && lane == 0) mbar_arrive(x.bar(PB_D0_FREE + grp));
         // ---- T = (I + A)^{-1}: 16x16 diagonal blocks by forward substitution
         if (pw < 4) {
             const int blk = pw;
@@ -1160,13 +1188,15 @@ prefill_pc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             for (int s = 0; s < kKqStages; ++s) mbar_init(x.bar(PB_KQ_EMPTY + s), 1);
             for (int grp = 0; grp < 2; ++grp) {
                 mbar_init(x.bar(PB_KQ_FULL + grp), 1);
-                mbar_init(x.bar(PB_KQ_TAKEN + grp), 8);
+                mbar_init(x.bar(PB_KQ_TAKEN + grp), 9);     // the group's 8 warps and its D0 issuer
                 mbar_init(x.bar(PB_D0_FULL + grp), 1);
                 mbar_init(x.bar(PB_R_FULL + grp), 1);
                 mbar_init(x.bar(PB_X1_FULL + grp), 1);
                 mbar_init(x.bar(PB_DRAIN + grp), 1);
                 mbar_init(x.bar(PB_STAGED + grp), 8);
                 mbar_init(x.bar(PB_AF_FREE + grp), 1);
+                mbar_init(x.bar(PB_D0_FREE + grp), 1);
+                mbar_init(x.bar(PB_D0_DRAIN + grp), 1);
             }
         }
         fence_mbar_init();
