@@ -42,6 +42,7 @@ SIGNATURES = {
     "gdn_decode_step_fused_bf16": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32,
                                              _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp]),
     "gdn_gated_norm": (C.c_int, [_vp, _vp, _vp, _i64, _i32, _i32, _i32, _f32, _vp, _vp]),
+    "gdn_selftest_bounded_wait": (C.c_int, [_i32, _i64, _vp, _vp]),
     "gdn_prefill_backward_workspace_size": (_sz, [_i32, _i64, _i32, _i32]),
     "gdn_prefill_backward": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
                                        _i32, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,

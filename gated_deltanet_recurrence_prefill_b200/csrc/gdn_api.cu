@@ -344,6 +344,16 @@ gdn_status gdn_prefill_backward(const uint16_t* q, const uint16_t* k, const uint
     return e == cudaSuccess ? GDN_OK : cuda_fail(e);
 }
 
+gdn_status gdn_selftest_bounded_wait(int32_t which, int64_t limit_us, void* workspace, gdn_stream_t stream) {
+    if ((which != 0 && which != 1) || limit_us < 1000 || limit_us > 2000000) return GDN_ERR_INVALID_ARG;
+    if (!workspace) return GDN_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_MISALIGNED;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaMemsetAsync(workspace, 0, gdn::kWsHeaderBytes, s);
+    if (e == cudaSuccess) e = gdn::launch_selftest_wait(which, (uint64_t)limit_us * 1000ull, workspace, s);
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
 gdn_status gdn_gated_norm(const float* o, const uint16_t* z, const float* norm_w, int64_t T, int32_t Hv,
                           int32_t d, int32_t layers, float eps, uint16_t* y, gdn_stream_t stream) {
     if (T < 0 || Hv <= 0 || d <= 0 || layers <= 0 || !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;

@@ -101,6 +101,7 @@ struct BackwardArgs {
     void* workspace;
 };
 size_t backward_workspace_bytes(int32_t n_seq, int64_t T, int32_t Hv);
+cudaError_t launch_selftest_wait(int which, uint64_t limit_ns, void* workspace, cudaStream_t stream);
 cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t stream);
 
 cudaError_t launch_gated_norm(const float* o, const uint16_t* z, const float* w, int64_t T, int32_t Hv,

@@ -355,6 +355,19 @@ gdn_status gdn_prefill_backward(const uint16_t* q, const uint16_t* k, const uint
                                 gdn_stream_t stream);
 
 /*
+ * gdn_selftest_bounded_wait -- failure detection check.  Runs, in one small
+ * kernel, one of the bounded waits the prefill's CTAs use, on something that
+ * never happens: which = 0 waits for a counter in global memory (as on the
+ * producer / consumer ring) that no thread raises, which = 1 for an mbarrier
+ * phase that never completes.  After limit_us microseconds (1 ms .. 2 s) the
+ * wait gives up and the kernel records the error in the workspace's error word
+ * as the prefill does, so that gdn_prefill_status(workspace) then returns
+ * GDN_ERR_TIMEOUT.  Nothing faults or hangs; the context stays usable.
+ * workspace: at least 256 bytes, 256-byte aligned (its header is cleared).
+ */
+gdn_status gdn_selftest_bounded_wait(int32_t which, int64_t limit_us, void* workspace, gdn_stream_t stream);
+
+/*
  * gdn_gated_norm -- the gated output norm that follows the recurrence in a
  * linear-attention layer:
  *     y[t, h, :] = norm_w[l] * o[t, h, :] / sqrt(mean_v o[t, h, v]^2 + eps)

@@ -29,7 +29,8 @@ def test_header_declares_the_entry_points():
     for required in ("gdn_conv1d_silu", "gdn_prefill", "gdn_prefill_workspace_size",
                      "gdn_decode_step", "gdn_decode_step_fused", "gdn_prefill_status",
                      "gdn_gated_norm", "gdn_prefill_gated", "gdn_decode_step_gated",
-                     "gdn_prefill_backward", "gdn_prefill_backward_workspace_size", "gdn_status_string"):
+                     "gdn_prefill_backward", "gdn_prefill_backward_workspace_size",
+                     "gdn_selftest_bounded_wait", "gdn_status_string"):
         assert required in names
 
 
@@ -223,3 +224,11 @@ def test_backward_rejects_bad_arguments(L):
     assert call(dq=_p(FAKE + 4)) == 3
     assert call(wsb=ws - 256) == 6
     assert call(wsp=_p(0x20000 + 16)) == 3
+
+
+def test_selftest_rejects_bad_arguments(L):
+    assert L.gdn_selftest_bounded_wait(2, 20000, _p(0x20000), None) == 1     # unknown wait
+    assert L.gdn_selftest_bounded_wait(0, 10, _p(0x20000), None) == 1        # below 1 ms
+    assert L.gdn_selftest_bounded_wait(0, 10_000_000, _p(0x20000), None) == 1   # above 2 s
+    assert L.gdn_selftest_bounded_wait(0, 20000, None, None) == 6
+    assert L.gdn_selftest_bounded_wait(0, 20000, _p(0x20000 + 16), None) == 3
