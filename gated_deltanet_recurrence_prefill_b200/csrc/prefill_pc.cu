@@ -55,7 +55,12 @@
 // below 2^-80.  o^T / scale is read back while the state update runs and
 // stored straight to global memory (for each token a warp writes 32
 // consecutive floats).  D has two buffers so that the next chunk's [U'; O']
-// product can start before this chunk's epilogues are done.
+// product can start before this chunk's epilogues are done.  With the fused
+// output norm (y requested), the TMA warp also stages the gate z of each
+// chunk, and after the second epilogue (while the tensor core works on the
+// next chunk) the epilogue warps turn their o rows into
+// y = norm_w * o / rms(o) * silu(z), bf16, summing each token's squares over
+// the four warps of a column share in shared memory.
 // Warp 0 loads V and K by TMA (two buffers each).
 //
 // Grid.  For nu units, blocks [0, nu) are the consumers and blocks
