@@ -64,7 +64,7 @@ decode_step_kernel(const uint16_t* __restrict__ q, const uint16_t* __restrict__ 
     StateT* S = state + uh * (int64_t)(kD * kD);
     constexpr int kRowsPerIter = rows_per_iter<StateT>();
     const uint16_t* vh = v + uh * kD;
-    float* oh = o + uh * kD;
+    float* oh = o ? o + uh * kD : nullptr;
 
 #pragma unroll 1
     for (int r0 = warp * 32; r0 < warp * 32 + 32; r0 += kRowsPerIter) {

@@ -106,7 +106,6 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t stream);
 
 cudaError_t launch_gated_norm(const float* o, const uint16_t* z, const float* w, int64_t T, int32_t Hv,
                               int32_t layers, float eps, uint16_t* y, cudaStream_t stream);
-cudaError_t launch_prefill_simt(const PrefillArgs& p, cudaStream_t stream);
 cudaError_t launch_prefill_tc(const PrefillArgs& p, cudaStream_t stream);
 size_t prefill_tc_smem_bytes();
 // producer / consumer prefill: a cooperative grid of one consumer and one or
@@ -121,7 +120,6 @@ size_t prefill_pc_smem_bytes();
 size_t prefill_pc_workspace_bytes(int32_t n_seq, int32_t Hv);
 // workspace the single-CTA kernel needs (and the least gdn_prefill accepts)
 size_t prefill_min_workspace_bytes(int32_t n_seq, int32_t Hv);
-size_t prefill_simt_smem_bytes();
 
 // workspace layout shared by the prefill kernels
 constexpr size_t kWsErrorWordOffset = 0;     // uint32 error word (0 = ok)
