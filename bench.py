@@ -6,9 +6,11 @@ prefill (gdn_prefill) of one GDN layer, T = 8192 tokens, 16 key heads, 48 value
 heads, d = 128, zero initial state.  The metric is tokens per second per layer.
 Secondary lines are measured in the same run and attached under "extra": the
 T = 262144 prefill (non-zero initial state), the 16-sequence varlen prefill
-(lengths U[1024, 32768]), and one decode step over 128 sequences x 48 layers
-with the 19.3 GB float32 state updated in place (plain, with the front end
-fused, and with a bf16 state).
+(lengths U[1024, 32768]), the gated output norm at T = 8192, the layer tail
+(recurrence + gated norm, fused and in two passes), the backward pass at
+T = 8192, and one decode step over 128 sequences x 48 layers with the 19.3 GB
+float32 state updated in place (plain, with the front end fused, with a bf16
+state, and with the gated norm fused).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
