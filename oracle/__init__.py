@@ -15,6 +15,7 @@ from .oracle import (  # noqa: F401
     max_threads,
     prefill,
     prefill_backward,
+    prefill_backward_chunked,
     prefill_chunked,
     prefill_f64,
 )

@@ -668,3 +668,304 @@ int gdn_oracle_prefill_backward(const double* q, const double* k, const double* 
     free(G); free(Sk); free(g); free(x);
     return 0;
 }
+
+/*
+ * gdn_oracle_prefill_backward_chunked -- the same gradient as
+ * gdn_oracle_prefill_backward, taken through the chunked (WY / UT) form of
+ * gdn_oracle_prefill_chunked, chunk by chunk from the last: the algebra a
+ * tensor-core backward follows.  Within a chunk of L tokens with start state S
+ * (G the running sum of log alpha, gam_i = e^{G_i}, Gam_ij = e^{G_i - G_j},
+ * kap_j = e^{G_{L-1} - G_j}):
+ *     A = strict_lower(diag(beta) Gam o K K^T),  T = (I + A)^{-1},
+ *     W = T diag(beta gam) K,  U' = T diag(beta) V,  U = U' - W S^T,
+ *     P = lower(Gam o Q K^T),  O = scale (diag(gam) Q S^T + P U),
+ *     S_end = gam_{L-1} S + U^T diag(kap) K.
+ * Each of these is differentiated in reverse order: S_end, O, P, U, U', W, then
+ * T (dA = -T^T dT T^T on the strictly lower part), A, and the decays through
+ * G (dG_i collects gam, Gam and kap terms; d log alpha_m = sum_{i >= m} dG_i).
+ * The gradient at the chunk start becomes dL/dS_end of the chunk before.
+ * Arguments and outputs as for gdn_oracle_prefill_backward, plus the chunk
+ * length C >= 1.
+ */
+int gdn_oracle_prefill_backward_chunked(const double* q, const double* k, const double* v, const double* a,
+                                        const double* b, const double* A_log, const double* dt_bias,
+                                        const int32_t* cu_seqlens, int32_t n_seq, int64_t T, int32_t Hqk,
+                                        int32_t Hv, int32_t dk, int32_t dv, double scale,
+                                        const double* initial_state, const double* d_o, const double* d_final,
+                                        int32_t C, double* dq, double* dkk, double* dvv, double* da, double* db,
+                                        double* dA_log, double* ddt_bias, double* d_initial) {
+    if (Hqk <= 0 || Hv <= 0 || Hv % Hqk || n_seq <= 0 || T < 0 || C < 1) return -1;
+    if (!cu_seqlens && n_seq != 1) return -1;
+    const int grp = Hv / Hqk;
+    const int64_t sz = (int64_t)dv * dk;
+    memset(dq, 0, sizeof(double) * T * Hqk * dk);
+    memset(dkk, 0, sizeof(double) * T * Hqk * dk);
+    memset(dA_log, 0, sizeof(double) * Hv);
+    memset(ddt_bias, 0, sizeof(double) * Hv);
+    /* chunk scratch */
+    double *Q = malloc(sizeof(double) * C * dk), *K = malloc(sizeof(double) * C * dk), *V = malloc(sizeof(double) * C * dv);
+    double *G = malloc(sizeof(double) * C), *lg = malloc(sizeof(double) * C), *be = malloc(sizeof(double) * C);
+    double *gam = malloc(sizeof(double) * C), *kap = malloc(sizeof(double) * C);
+    double *KK = malloc(sizeof(double) * C * C), *QK = malloc(sizeof(double) * C * C), *Gm = malloc(sizeof(double) * C * C);
+    double *A = malloc(sizeof(double) * C * C), *Tm = malloc(sizeof(double) * C * C), *P = malloc(sizeof(double) * C * C);
+    double *W = malloc(sizeof(double) * C * dk), *Up = malloc(sizeof(double) * C * dv), *U = malloc(sizeof(double) * C * dv);
+    double *dU = malloc(sizeof(double) * C * dv), *dK = malloc(sizeof(double) * C * dk), *dQ = malloc(sizeof(double) * C * dk);
+    double *dV = malloc(sizeof(double) * C * dv), *dW = malloc(sizeof(double) * C * dk);
+    double *dbe = malloc(sizeof(double) * C), *dgam = malloc(sizeof(double) * C), *dkap = malloc(sizeof(double) * C);
+    double *dGm = malloc(sizeof(double) * C * C), *dT = malloc(sizeof(double) * C * C), *dA = malloc(sizeof(double) * C * C);
+    double *tmp = malloc(sizeof(double) * C * C), *dG = malloc(sizeof(double) * C);
+    double *TtdUp = malloc(sizeof(double) * C * dv), *TtdW = malloc(sizeof(double) * C * dk);
+    double *dS = malloc(sizeof(double) * sz), *dSn = malloc(sizeof(double) * sz);
+    for (int n = 0; n < n_seq; ++n) {
+        const int64_t bos = cu_seqlens ? cu_seqlens[n] : 0;
+        const int64_t eos = cu_seqlens ? cu_seqlens[n + 1] : T;
+        const int64_t nch = (eos - bos + C - 1) / C;
+        for (int h = 0; h < Hv; ++h) {
+            const int gk = h / grp;
+            /* chunk-start states by the chunked forward: starts[c] */
+            double* starts = malloc(sizeof(double) * sz * (nch + 1));
+            for (int64_t i = 0; i < sz; ++i)
+                starts[i] = initial_state ? initial_state[((int64_t)n * Hv + h) * sz + i] : 0.0;
+            /* one chunk's forward quantities (shared by the forward sweep and the backward one) */
+#define GDN_CHUNK_FORWARD(c0, L, S)                                                                          \
+    do {                                                                                                     \
+        double run_ = 0.0;                                                                                   \
+        for (int t_ = 0; t_ < (L); ++t_) {                                                                   \
+            const int64_t tt_ = (c0) + t_;                                                                   \
+            memcpy(Q + (int64_t)t_ * dk, q + (tt_ * Hqk + gk) * dk, sizeof(double) * dk);                    \
+            memcpy(K + (int64_t)t_ * dk, k + (tt_ * Hqk + gk) * dk, sizeof(double) * dk);                    \
+            memcpy(V + (int64_t)t_ * dv, v + (tt_ * Hv + h) * dv, sizeof(double) * dv);                      \
+            lg[t_] = gdn_oracle_log_alpha(a[tt_ * Hv + h], A_log[h], dt_bias[h]);                            \
+            run_ += lg[t_];                                                                                  \
+            G[t_] = run_;                                                                                    \
+            be[t_] = gdn_oracle_beta(b[tt_ * Hv + h]);                                                       \
+        }                                                                                                    \
+        for (int i_ = 0; i_ < (L); ++i_) {                                                                   \
+            gam[i_] = exp(G[i_]);                                                                            \
+            kap[i_] = exp(G[(L) - 1] - G[i_]);                                                               \
+            for (int j_ = 0; j_ < (L); ++j_) {                                                               \
+                double kk_ = 0.0, qk_ = 0.0;                                                                 \
+                for (int e_ = 0; e_ < dk; ++e_) {                                                            \
+                    kk_ += K[(int64_t)i_ * dk + e_] * K[(int64_t)j_ * dk + e_];                              \
+                    qk_ += Q[(int64_t)i_ * dk + e_] * K[(int64_t)j_ * dk + e_];                              \
+                }                                                                                            \
+                KK[i_ * C + j_] = kk_;                                                                       \
+                QK[i_ * C + j_] = qk_;                                                                       \
+                Gm[i_ * C + j_] = j_ <= i_ ? exp(G[i_] - G[j_]) : 0.0;                                       \
+                A[i_ * C + j_] = j_ < i_ ? be[i_] * Gm[i_ * C + j_] * kk_ : 0.0;                             \
+                P[i_ * C + j_] = j_ <= i_ ? Gm[i_ * C + j_] * qk_ : 0.0;                                     \
+            }                                                                                                \
+        }                                                                                                    \
+        for (int i_ = 0; i_ < (L); ++i_)                                                                     \
+            for (int j_ = 0; j_ < (L); ++j_) {                                                               \
+                double val_ = (i_ == j_) ? 1.0 : 0.0;                                                        \
+                for (int m_ = j_; m_ < i_; ++m_) val_ -= A[i_ * C + m_] * Tm[m_ * C + j_];                   \
+                Tm[i_ * C + j_] = (j_ <= i_) ? val_ : 0.0;                                                   \
+            }                                                                                                \
+        for (int i_ = 0; i_ < (L); ++i_) {                                                                   \
+            for (int e_ = 0; e_ < dk; ++e_) {                                                                \
+                double acc_ = 0.0;                                                                           \
+                for (int j_ = 0; j_ <= i_; ++j_) acc_ += Tm[i_ * C + j_] * be[j_] * gam[j_] * K[(int64_t)j_ * dk + e_]; \
+                W[(int64_t)i_ * dk + e_] = acc_;                                                             \
+            }                                                                                                \
+            for (int e_ = 0; e_ < dv; ++e_) {                                                                \
+                double acc_ = 0.0;                                                                           \
+                for (int j_ = 0; j_ <= i_; ++j_) acc_ += Tm[i_ * C + j_] * be[j_] * V[(int64_t)j_ * dv + e_]; \
+                Up[(int64_t)i_ * dv + e_] = acc_;                                                            \
+            }                                                                                                \
+            for (int e_ = 0; e_ < dv; ++e_) {                                                                \
+                double acc_ = 0.0;                                                                           \
+                for (int f_ = 0; f_ < dk; ++f_) acc_ += W[(int64_t)i_ * dk + f_] * (S)[(int64_t)e_ * dk + f_]; \
+                U[(int64_t)i_ * dv + e_] = Up[(int64_t)i_ * dv + e_] - acc_;                                 \
+            }                                                                                                \
+        }                                                                                                    \
+    } while (0)
+            for (int64_t c = 0; c < nch; ++c) {
+                const int64_t c0 = bos + c * C;
+                const int L = (int)((eos - c0) < C ? (eos - c0) : C);
+                const double* S = starts + c * sz;
+                double* Sn = starts + (c + 1) * sz;
+                GDN_CHUNK_FORWARD(c0, L, S);
+                for (int e = 0; e < dv; ++e)
+                    for (int f = 0; f < dk; ++f) {
+                        double acc = gam[L - 1] * S[(int64_t)e * dk + f];
+                        for (int j = 0; j < L; ++j) acc += kap[j] * U[(int64_t)j * dv + e] * K[(int64_t)j * dk + f];
+                        Sn[(int64_t)e * dk + f] = acc;
+                    }
+            }
+            for (int64_t i = 0; i < sz; ++i) dSn[i] = d_final ? d_final[((int64_t)n * Hv + h) * sz + i] : 0.0;
+            for (int64_t c = nch - 1; c >= 0; --c) {
+                const int64_t c0 = bos + c * C;
+                const int L = (int)((eos - c0) < C ? (eos - c0) : C);
+                const double* S = starts + c * sz;
+                GDN_CHUNK_FORWARD(c0, L, S);
+                memset(dU, 0, sizeof(double) * C * dv);
+                memset(dK, 0, sizeof(double) * C * dk);
+                memset(dQ, 0, sizeof(double) * C * dk);
+                memset(dV, 0, sizeof(double) * C * dv);
+                memset(dbe, 0, sizeof(double) * C);
+                memset(dgam, 0, sizeof(double) * C);
+                memset(dkap, 0, sizeof(double) * C);
+                memset(dGm, 0, sizeof(double) * C * C);
+                memset(dT, 0, sizeof(double) * C * C);
+                memset(dS, 0, sizeof(double) * sz);
+                /* 1. S_end = gam_{L-1} S + U^T diag(kap) K */
+                double dSS = 0.0;
+                for (int64_t i = 0; i < sz; ++i) { dS[i] += gam[L - 1] * dSn[i]; dSS += dSn[i] * S[i]; }
+                dgam[L - 1] += dSS;
+                for (int j = 0; j < L; ++j) {
+                    double s_ = 0.0;
+                    for (int e = 0; e < dv; ++e) {
+                        double dk_ = 0.0;
+                        for (int f = 0; f < dk; ++f) dk_ += dSn[(int64_t)e * dk + f] * K[(int64_t)j * dk + f];
+                        dU[(int64_t)j * dv + e] += kap[j] * dk_;
+                        s_ += U[(int64_t)j * dv + e] * dk_;
+                    }
+                    dkap[j] = s_;
+                    for (int f = 0; f < dk; ++f) {
+                        double acc = 0.0;
+                        for (int e = 0; e < dv; ++e) acc += U[(int64_t)j * dv + e] * dSn[(int64_t)e * dk + f];
+                        dK[(int64_t)j * dk + f] += kap[j] * acc;
+                    }
+                }
+                /* 2. O = scale (diag(gam) Q S^T + P U);  3. P = lower(Gam o Q K^T) */
+                for (int i = 0; i < L; ++i) {
+                    const double* doi = d_o + ((c0 + i) * Hv + h) * dv;
+                    double sqd = 0.0;
+                    for (int e = 0; e < dv; ++e) {
+                        double sq = 0.0;
+                        for (int f = 0; f < dk; ++f) sq += S[(int64_t)e * dk + f] * Q[(int64_t)i * dk + f];
+                        sqd += doi[e] * sq;
+                    }
+                    dgam[i] += scale * sqd;
+                    for (int f = 0; f < dk; ++f) {
+                        double acc = 0.0;
+                        for (int e = 0; e < dv; ++e) acc += doi[e] * S[(int64_t)e * dk + f];
+                        dQ[(int64_t)i * dk + f] += scale * gam[i] * acc;
+                    }
+                    for (int e = 0; e < dv; ++e)
+                        for (int f = 0; f < dk; ++f) dS[(int64_t)e * dk + f] += scale * gam[i] * doi[e] * Q[(int64_t)i * dk + f];
+                    for (int j = 0; j <= i; ++j) {
+                        double dP = 0.0;
+                        for (int e = 0; e < dv; ++e) {
+                            dP += doi[e] * U[(int64_t)j * dv + e];
+                            dU[(int64_t)j * dv + e] += scale * P[i * C + j] * doi[e];
+                        }
+                        dP *= scale;
+                        for (int f = 0; f < dk; ++f) {
+                            dQ[(int64_t)i * dk + f] += dP * Gm[i * C + j] * K[(int64_t)j * dk + f];
+                            dK[(int64_t)j * dk + f] += dP * Gm[i * C + j] * Q[(int64_t)i * dk + f];
+                        }
+                        dGm[i * C + j] += dP * QK[i * C + j];
+                    }
+                }
+                /* 4. U = U' - W S^T */
+                for (int i = 0; i < L; ++i)
+                    for (int f = 0; f < dk; ++f) {
+                        double acc = 0.0;
+                        for (int e = 0; e < dv; ++e) acc += dU[(int64_t)i * dv + e] * S[(int64_t)e * dk + f];
+                        dW[(int64_t)i * dk + f] = -acc;
+                    }
+                for (int e = 0; e < dv; ++e)
+                    for (int f = 0; f < dk; ++f) {
+                        double acc = 0.0;
+                        for (int i = 0; i < L; ++i) acc += dU[(int64_t)i * dv + e] * W[(int64_t)i * dk + f];
+                        dS[(int64_t)e * dk + f] -= acc;
+                    }
+                /* 5. U' = T diag(beta) V  (dU' = dU);  6. W = T diag(beta gam) K */
+                for (int i = 0; i < L; ++i)
+                    for (int j = 0; j <= i; ++j) {
+                        double a1 = 0.0, a2 = 0.0;
+                        for (int e = 0; e < dv; ++e) a1 += dU[(int64_t)i * dv + e] * V[(int64_t)j * dv + e];
+                        for (int f = 0; f < dk; ++f) a2 += dW[(int64_t)i * dk + f] * K[(int64_t)j * dk + f];
+                        dT[i * C + j] += be[j] * a1 + be[j] * gam[j] * a2;
+                    }
+                for (int j = 0; j < L; ++j) {
+                    for (int e = 0; e < dv; ++e) {
+                        double acc = 0.0;
+                        for (int i = j; i < L; ++i) acc += Tm[i * C + j] * dU[(int64_t)i * dv + e];
+                        TtdUp[(int64_t)j * dv + e] = acc;
+                    }
+                    for (int f = 0; f < dk; ++f) {
+                        double acc = 0.0;
+                        for (int i = j; i < L; ++i) acc += Tm[i * C + j] * dW[(int64_t)i * dk + f];
+                        TtdW[(int64_t)j * dk + f] = acc;
+                    }
+                    double sv = 0.0, sk = 0.0;
+                    for (int e = 0; e < dv; ++e) {
+                        dV[(int64_t)j * dv + e] += be[j] * TtdUp[(int64_t)j * dv + e];
+                        sv += TtdUp[(int64_t)j * dv + e] * V[(int64_t)j * dv + e];
+                    }
+                    for (int f = 0; f < dk; ++f) {
+                        dK[(int64_t)j * dk + f] += be[j] * gam[j] * TtdW[(int64_t)j * dk + f];
+                        sk += TtdW[(int64_t)j * dk + f] * K[(int64_t)j * dk + f];
+                    }
+                    dbe[j] += sv + gam[j] * sk;
+                    dgam[j] += be[j] * sk;
+                }
+                /* 7. T = (I + A)^{-1}: dA = -T^T dT T^T on the strictly lower part */
+                for (int i = 0; i < L; ++i)
+                    for (int j = 0; j < L; ++j) {
+                        double acc = 0.0;
+                        for (int m = 0; m < L; ++m) acc += Tm[m * C + i] * dT[m * C + j];   /* (T^T dT)_ij */
+                        tmp[i * C + j] = acc;
+                    }
+                for (int i = 0; i < L; ++i)
+                    for (int j = 0; j < L; ++j) {
+                        double acc = 0.0;
+                        for (int m = 0; m < L; ++m) acc += tmp[i * C + m] * Tm[j * C + m];   /* (. T^T)_ij */
+                        dA[i * C + j] = j < i ? -acc : 0.0;
+                    }
+                /* 8. A_ij = beta_i Gam_ij (k_i . k_j), j < i */
+                for (int i = 0; i < L; ++i)
+                    for (int j = 0; j < i; ++j) {
+                        const double dAij = dA[i * C + j];
+                        dbe[i] += dAij * Gm[i * C + j] * KK[i * C + j];
+                        dGm[i * C + j] += dAij * be[i] * KK[i * C + j];
+                        const double E = dAij * be[i] * Gm[i * C + j];
+                        for (int f = 0; f < dk; ++f) {
+                            dK[(int64_t)i * dk + f] += E * K[(int64_t)j * dk + f];
+                            dK[(int64_t)j * dk + f] += E * K[(int64_t)i * dk + f];
+                        }
+                    }
+                /* 9. decays: G_i = sum_{m <= i} log alpha_m */
+                double kk_sum = 0.0;
+                for (int i = 0; i < L; ++i) kk_sum += kap[i] * dkap[i];
+                for (int i = 0; i < L; ++i) {
+                    double acc = gam[i] * dgam[i] - kap[i] * dkap[i];
+                    for (int j = 0; j <= i; ++j) acc += Gm[i * C + j] * dGm[i * C + j];
+                    for (int i2 = i; i2 < L; ++i2) acc -= Gm[i2 * C + i] * dGm[i2 * C + i];
+                    dG[i] = acc;
+                }
+                dG[L - 1] += kk_sum;
+                double suffix = 0.0;
+                for (int m = L - 1; m >= 0; --m) {
+                    suffix += dG[m];
+                    const int64_t tt = c0 + m;
+                    const double la = lg[m];
+                    const double xg = a[tt * Hv + h] + dt_bias[h];
+                    const double sig = 1.0 / (1.0 + exp(-xg));
+                    const double dat = suffix * (-exp(A_log[h]) * sig);
+                    da[tt * Hv + h] = dat;
+                    ddt_bias[h] += dat;
+                    dA_log[h] += suffix * la;
+                    db[tt * Hv + h] = dbe[m] * be[m] * (1.0 - be[m]);
+                    for (int e = 0; e < dv; ++e) dvv[(tt * Hv + h) * dv + e] = dV[(int64_t)m * dv + e];
+                    for (int f = 0; f < dk; ++f) {
+                        dq[(tt * Hqk + gk) * dk + f] += dQ[(int64_t)m * dk + f];
+                        dkk[(tt * Hqk + gk) * dk + f] += dK[(int64_t)m * dk + f];
+                    }
+                }
+                memcpy(dSn, dS, sizeof(double) * sz);
+            }
+#undef GDN_CHUNK_FORWARD
+            if (d_initial) memcpy(d_initial + ((int64_t)n * Hv + h) * sz, dSn, sizeof(double) * sz);
+            free(starts);
+        }
+    }
+    free(Q); free(K); free(V); free(G); free(lg); free(be); free(gam); free(kap); free(KK); free(QK); free(Gm);
+    free(A); free(Tm); free(P); free(W); free(Up); free(U); free(dU); free(dK); free(dQ); free(dV); free(dW);
+    free(dbe); free(dgam); free(dkap); free(dGm); free(dT); free(dA); free(tmp); free(dG); free(TtdUp);
+    free(TtdW); free(dS); free(dSn);
+    return 0;
+}

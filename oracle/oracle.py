@@ -53,6 +53,10 @@ def _bind(lib):
     lib.gdn_oracle_prefill_backward.restype = C.c_int
     lib.gdn_oracle_prefill_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32,
                                                 i32, dbl, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.gdn_oracle_prefill_backward_chunked.restype = C.c_int
+    lib.gdn_oracle_prefill_backward_chunked.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
+                                                        i32, i32, dbl, vp, vp, vp, i32, vp, vp, vp, vp, vp,
+                                                        vp, vp, vp]
     lib.gdn_oracle_max_threads.restype = C.c_int
     lib.gdn_oracle_max_threads.argtypes = [C.c_int]
     return lib
@@ -296,4 +300,28 @@ def prefill_backward(q, k, v, a, b, A_log, dt_bias, d_o, d_final=None, cu_seqlen
         _ptr(out["db"]), _ptr(out["dA_log"]), _ptr(out["ddt_bias"]), _ptr(out["d_initial"]))
     if rc != 0:
         raise ValueError("oracle prefill_backward rejected its arguments")
+    return out
+
+
+def prefill_backward_chunked(q, k, v, a, b, A_log, dt_bias, d_o, d_final=None, cu_seqlens=None, scale=None,
+                             initial_state=None, C=64, lib=None):
+    """The gradient of prefill_backward taken through the chunked (WY / UT) form
+    with chunks of C tokens (gdn_oracle_prefill_backward_chunked).  Same
+    arguments and outputs as prefill_backward."""
+    q, k, v = _widen(q), _widen(k), _widen(v)
+    T, Hqk, dk = q.shape
+    Hv, dv = v.shape[1], v.shape[2]
+    cu = None if cu_seqlens is None else np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    n_seq = 1 if cu is None else len(cu) - 1
+    scale = 1.0 / np.sqrt(dk) if scale is None else float(scale)
+    out = dict(dq=np.zeros((T, Hqk, dk)), dk=np.zeros((T, Hqk, dk)), dv=np.zeros((T, Hv, dv)),
+               da=np.zeros((T, Hv)), db=np.zeros((T, Hv)), dA_log=np.zeros(Hv), ddt_bias=np.zeros(Hv),
+               d_initial=np.zeros((n_seq, Hv, dv, dk)))
+    rc = _L(lib).gdn_oracle_prefill_backward_chunked(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(_f64(a)), _ptr(_f64(b)), _ptr(_f64(A_log)), _ptr(_f64(dt_bias)),
+        _ptr(cu), n_seq, T, Hqk, Hv, dk, dv, scale, _ptr(_f64(initial_state)), _ptr(_f64(d_o)),
+        _ptr(_f64(d_final)), int(C), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["da"]),
+        _ptr(out["db"]), _ptr(out["dA_log"]), _ptr(out["ddt_bias"]), _ptr(out["d_initial"]))
+    if rc != 0:
+        raise ValueError("oracle prefill_backward_chunked rejected its arguments")
     return out

@@ -54,6 +54,13 @@ MUTANTS = {
     "norm_weight_wrong_layer": ("const double* wl = w + (int64_t)(t % layers) * d;", "const double* wl = w;"),
     "norm_over_heads": ("const int64_t row = (t * Hv + h) * (int64_t)d;\n            double ss = 0.0;\n            for (int e = 0; e < d; ++e) ss += o[row + e] * o[row + e];",
                         "const int64_t row = (t * Hv + h) * (int64_t)d;\n            double ss = 0.0;\n            for (int e = 0; e < d; ++e) ss += o[t * Hv * (int64_t)d + e] * o[t * Hv * (int64_t)d + e];"),
+    "cbw_inverse_sign": ("dA[i * C + j] = j < i ? -acc : 0.0;", "dA[i * C + j] = j < i ? acc : 0.0;"),
+    "cbw_inverse_transposed": ("acc += Tm[m * C + i] * dT[m * C + j];", "acc += Tm[i * C + m] * dT[m * C + j];"),
+    "cbw_kk_one_sided": ("dK[(int64_t)j * dk + f] += E * K[(int64_t)i * dk + f];",
+                         "dK[(int64_t)j * dk + f] += 0.0 * E;"),
+    "cbw_no_kappa_sum": ("dG[L - 1] += kk_sum;", "dG[L - 1] += 0.0 * kk_sum;"),
+    "cbw_no_W_gamma_grad": ("dgam[j] += be[j] * sk;", "dgam[j] += 0.0 * sk;"),
+    "cbw_carry_no_decay": ("dS[i] += gam[L - 1] * dSn[i];", "dS[i] += dSn[i];"),
 }
 
 

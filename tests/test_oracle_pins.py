@@ -552,3 +552,28 @@ def test_backward_of_a_sum_over_heads(orc):
             acc_k += gh["dk"][:, 0]
         assert np.allclose(g["dq"][:, gk], acc_q, rtol=1e-13, atol=1e-15)
         assert np.allclose(g["dk"][:, gk], acc_k, rtol=1e-13, atol=1e-15)
+
+
+def test_chunked_backward_equals_sequential_backward(orc):
+    # the chunked (WY) gradient is the same function as the token-by-token one: for
+    # any chunk length, with chunks that span several tokens, a ragged tail and a
+    # one-token sequence
+    inp, d_o, d_fin = _bw_case(7, lengths=(37, 5, 1), Hqk=2, Hv=4, d=6)
+    args = {n: inp[n] for n in ("q", "k", "v", "a", "b", "A_log", "dt_bias")}
+    ref = orc.prefill_backward(**args, d_o=d_o, d_final=d_fin, cu_seqlens=inp["cu_seqlens"],
+                               initial_state=inp["initial_state"])
+    for C in (1, 2, 3, 8, 16, 64):
+        got = orc.prefill_backward_chunked(**args, d_o=d_o, d_final=d_fin, cu_seqlens=inp["cu_seqlens"],
+                                           initial_state=inp["initial_state"], C=C)
+        for name, x in ref.items():
+            s = max(1.0, np.max(np.abs(x)))
+            assert np.max(np.abs(got[name] - x)) <= 1e-11 * s, (C, name)
+
+
+def test_chunked_backward_without_initial_or_final_state(orc):
+    inp, d_o, _ = _bw_case(8, lengths=(20,), Hqk=1, Hv=1, d=4)
+    args = {n: inp[n] for n in ("q", "k", "v", "a", "b", "A_log", "dt_bias")}
+    ref = orc.prefill_backward(**args, d_o=d_o, cu_seqlens=inp["cu_seqlens"])
+    got = orc.prefill_backward_chunked(**args, d_o=d_o, cu_seqlens=inp["cu_seqlens"], C=8)
+    for name, x in ref.items():
+        assert np.max(np.abs(got[name] - x)) <= 1e-11 * max(1.0, np.max(np.abs(x))), name
