@@ -235,7 +235,7 @@ def test_gate_closed_forms(orc):
     assert orc.beta(-40.0) == pytest.approx(math.exp(-40.0), rel=1e-12)
 
 
-@pytest.mark.parametrize("C", [1, 2, 16, 64])
+@pytest.mark.parametrize("C", [1, 2, 16, 64, 128])
 def test_chunked_equals_recurrent(orc, C):
     """The chunked WY/UT algebra reproduces the recurrence, with ragged chunks,
     several packed sequences (one empty, one of length 1), non-zero S0 and
