@@ -17,6 +17,7 @@ from ._lib import (  # noqa: F401
     lib_path,
     prefill,
     prefill_backward,
+    prefill_backward_chunked,
     prefill_gated,
     prefill_noalloc,
     prefill_status,

@@ -47,6 +47,10 @@ SIGNATURES = {
     "gdn_prefill_backward": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
                                        _i32, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                        _vp, _vp, _sz, _vp]),
+    "gdn_prefill_backward_chunked_workspace_size": (_sz, [_i32, _i64, _i32, _i32]),
+    "gdn_prefill_backward_chunked": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
+                                               _i32, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                               _vp, _vp, _sz, _vp]),
     "gdn_decode_step_gated": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32,
                                         _i32, _f32, _vp, _i32, _vp, _vp, _vp, _f32, _vp, _vp]),
     "gdn_prefill_gated": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
@@ -390,6 +394,21 @@ def prefill_backward(q, k, v, a, b, A_log, dt_bias, d_o, d_final_state=None, cu_
     dL/dS_T = d_final_state [N, Hv, d, d] (or zero).  Returns a dict of float32
     tensors dq, dk [T, Hqk, d], dv [T, Hv, d], da, db [T, Hv], dA_log,
     ddt_bias [Hv] and d_initial_state [N, Hv, d, d] (or None)."""
+    return _backward("gdn_prefill_backward", q, k, v, a, b, A_log, dt_bias, d_o, d_final_state, cu_seqlens,
+                     scale, initial_state, want_d_initial, workspace, stream)
+
+
+def prefill_backward_chunked(q, k, v, a, b, A_log, dt_bias, d_o, d_final_state=None, cu_seqlens=None,
+                             scale=None, initial_state=None, want_d_initial=True, workspace=None, stream=None):
+    """gdn_prefill_backward_chunked: the same gradients through the chunked
+    form (two chains over 64-token chunks, the rest chunk-parallel).  Arguments
+    and result as for prefill_backward."""
+    return _backward("gdn_prefill_backward_chunked", q, k, v, a, b, A_log, dt_bias, d_o, d_final_state,
+                     cu_seqlens, scale, initial_state, want_d_initial, workspace, stream)
+
+
+def _backward(entry, q, k, v, a, b, A_log, dt_bias, d_o, d_final_state, cu_seqlens, scale, initial_state,
+              want_d_initial, workspace, stream):
     import torch
     T, Hqk, d = q.shape
     Hv = v.shape[1]
@@ -415,14 +434,14 @@ def prefill_backward(q, k, v, a, b, A_log, dt_bias, d_o, d_final_state=None, cu_
     out = dict(dq=f(T, Hqk, d), dk=f(T, Hqk, d), dv=f(T, Hv, d), da=f(T, Hv), db=f(T, Hv),
                dA_log=f(Hv), ddt_bias=f(Hv),
                d_initial_state=f(n_seq, Hv, d, d) if want_d_initial else None)
-    ws_bytes = lib().gdn_prefill_backward_workspace_size(n_seq, T, Hv, d)
+    ws_bytes = getattr(lib(), entry + "_workspace_size")(n_seq, T, Hv, d)
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    st = lib().gdn_prefill_backward(
+    st = getattr(lib(), entry)(
         _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias), _ptr(cu_seqlens), n_seq, T,
         Hqk, Hv, d, float(scale), _ptr(initial_state), _ptr(d_o), _ptr(d_final_state), _ptr(out["dq"]),
         _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["da"]), _ptr(out["db"]), _ptr(out["dA_log"]),
         _ptr(out["ddt_bias"]), _ptr(out["d_initial_state"]), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream))
-    _check("gdn_prefill_backward", st)
+    _check(entry, st)
     return out

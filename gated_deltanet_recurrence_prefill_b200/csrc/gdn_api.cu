@@ -317,14 +317,24 @@ size_t gdn_prefill_backward_workspace_size(int32_t n_seq, int64_t T, int32_t Hv,
     return gdn::backward_workspace_bytes(n_seq > 0 ? n_seq : 1, T > 0 ? T : 0, Hv > 0 ? Hv : 1);
 }
 
-gdn_status gdn_prefill_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* a,
-                                const float* b, const float* A_log, const float* dt_bias,
-                                const int32_t* cu_seqlens, int32_t n_seq, int64_t T, int32_t Hqk,
-                                int32_t Hv, int32_t d, float scale, const float* initial_state,
-                                const float* d_o, const float* d_final_state, float* dq, float* dk,
-                                float* dv, float* da, float* db, float* dA_log, float* ddt_bias,
-                                float* d_initial_state, void* workspace, size_t workspace_bytes,
-                                gdn_stream_t stream) {
+size_t gdn_prefill_backward_chunked_workspace_size(int32_t n_seq, int64_t T, int32_t Hv, int32_t d) {
+    (void)d;
+    return gdn::backward_chunked_workspace_bytes(n_seq > 0 ? n_seq : 1, T > 0 ? T : 0, Hv > 0 ? Hv : 1);
+}
+
+}  // extern "C"
+
+namespace {
+
+// the arguments both backward entry points take, checked; runs the token-by-token
+// kernel or the chunked one
+gdn_status prefill_backward_common(bool chunked, const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                   const float* a, const float* b, const float* A_log, const float* dt_bias,
+                                   const int32_t* cu_seqlens, int32_t n_seq, int64_t T, int32_t Hqk, int32_t Hv,
+                                   int32_t d, float scale, const float* initial_state, const float* d_o,
+                                   const float* d_final_state, float* dq, float* dk, float* dv, float* da,
+                                   float* db, float* dA_log, float* ddt_bias, float* d_initial_state,
+                                   void* workspace, size_t workspace_bytes, gdn_stream_t stream) {
     gdn_status st = check_heads(Hqk, Hv, d);
     if (st != GDN_OK) return st;
     if ((st = check_seqs(cu_seqlens, n_seq, T)) != GDN_OK) return st;
@@ -335,13 +345,46 @@ gdn_status gdn_prefill_backward(const uint16_t* q, const uint16_t* k, const uint
                           dq, dk, dv, da, db, dA_log, ddt_bias, d_initial_state};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
-    if (!workspace || workspace_bytes < gdn::backward_workspace_bytes(n_seq, T, Hv)) return GDN_ERR_WORKSPACE;
+    const size_t need = chunked ? gdn::backward_chunked_workspace_bytes(n_seq, T, Hv)
+                                : gdn::backward_workspace_bytes(n_seq, T, Hv);
+    if (!workspace || workspace_bytes < need) return GDN_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_MISALIGNED;
     gdn::BackwardArgs ba{q, k, v, a, b, A_log, dt_bias, cu_seqlens, n_seq, T, Hqk, Hv, scale,
                          initial_state, d_o, d_final_state, dq, dk, dv, da, db, dA_log, ddt_bias,
                          d_initial_state, workspace};
-    cudaError_t e = gdn::launch_backward(ba, (cudaStream_t)stream);
+    cudaError_t e = chunked ? gdn::launch_backward_chunked(ba, (cudaStream_t)stream)
+                            : gdn::launch_backward(ba, (cudaStream_t)stream);
     return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+gdn_status gdn_prefill_backward(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* a,
+                                const float* b, const float* A_log, const float* dt_bias,
+                                const int32_t* cu_seqlens, int32_t n_seq, int64_t T, int32_t Hqk,
+                                int32_t Hv, int32_t d, float scale, const float* initial_state,
+                                const float* d_o, const float* d_final_state, float* dq, float* dk,
+                                float* dv, float* da, float* db, float* dA_log, float* ddt_bias,
+                                float* d_initial_state, void* workspace, size_t workspace_bytes,
+                                gdn_stream_t stream) {
+    return prefill_backward_common(false, q, k, v, a, b, A_log, dt_bias, cu_seqlens, n_seq, T, Hqk, Hv, d, scale,
+                                   initial_state, d_o, d_final_state, dq, dk, dv, da, db, dA_log, ddt_bias,
+                                   d_initial_state, workspace, workspace_bytes, stream);
+}
+
+gdn_status gdn_prefill_backward_chunked(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* a,
+                                        const float* b, const float* A_log, const float* dt_bias,
+                                        const int32_t* cu_seqlens, int32_t n_seq, int64_t T, int32_t Hqk,
+                                        int32_t Hv, int32_t d, float scale, const float* initial_state,
+                                        const float* d_o, const float* d_final_state, float* dq, float* dk,
+                                        float* dv, float* da, float* db, float* dA_log, float* ddt_bias,
+                                        float* d_initial_state, void* workspace, size_t workspace_bytes,
+                                        gdn_stream_t stream) {
+    return prefill_backward_common(true, q, k, v, a, b, A_log, dt_bias, cu_seqlens, n_seq, T, Hqk, Hv, d, scale,
+                                   initial_state, d_o, d_final_state, dq, dk, dv, da, db, dA_log, ddt_bias,
+                                   d_initial_state, workspace, workspace_bytes, stream);
 }
 
 gdn_status gdn_selftest_bounded_wait(int32_t which, int64_t limit_us, void* workspace, gdn_stream_t stream) {

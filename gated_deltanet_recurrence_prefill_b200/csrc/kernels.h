@@ -103,6 +103,10 @@ struct BackwardArgs {
 size_t backward_workspace_bytes(int32_t n_seq, int64_t T, int32_t Hv);
 cudaError_t launch_selftest_wait(int which, uint64_t limit_ns, void* workspace, cudaStream_t stream);
 cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t stream);
+// the same gradient through the chunked form (backward_chunked.cu): two chains
+// over chunks and chunk-parallel work; workspace of backward_chunked_workspace_bytes
+size_t backward_chunked_workspace_bytes(int32_t n_seq, int64_t T, int32_t Hv);
+cudaError_t launch_backward_chunked(const BackwardArgs& a, cudaStream_t stream);
 
 cudaError_t launch_gated_norm(const float* o, const uint16_t* z, const float* w, int64_t T, int32_t Hv,
                               int32_t layers, float eps, uint16_t* y, cudaStream_t stream);

@@ -355,6 +355,39 @@ gdn_status gdn_prefill_backward(const uint16_t* q, const uint16_t* k, const uint
                                 gdn_stream_t stream);
 
 /*
+ * gdn_prefill_backward_chunked_workspace_size -- bytes of device workspace
+ * gdn_prefill_backward_chunked needs (a multiple of 256).  With
+ * slots = T / 64 + n_seq + 1: per (slot, value head) W and U' (2 * 64 * d
+ * floats), T (64 * 64), Y, the chunk-start state and the chunk-end gradient
+ * (3 * d * d) and 65 decay floats; dq and dk per value head (2 * T * Hv * d
+ * floats); the chunk list and the gate-parameter sums.  About 256 KiB per
+ * (chunk, value head).  Host-only.
+ */
+size_t gdn_prefill_backward_chunked_workspace_size(int32_t n_seq, int64_t T, int32_t Hv, int32_t d);
+
+/*
+ * gdn_prefill_backward_chunked -- the same gradient as gdn_prefill_backward,
+ * taken through the chunked (WY / UT) form of the recurrence with 64-token
+ * chunks (architecture page section 2.2 for the recurrence; the chunk algebra
+ * is that of gdn_prefill).  The sequential work is two chains over chunks
+ * instead of one over tokens: the chunk-start states, and the gradient at each
+ * chunk end, dS_{c-1} = gam dS_c - (diag(kap) K dS_c^T)^T W + Y_c, whose
+ * state-free term Y_c is computed for all chunks at once; everything else (dq,
+ * dk, dv, the gates) is computed per (chunk, value head) in parallel.  Float32
+ * arithmetic on CUDA cores, no atomics: the result is deterministic.
+ * Arguments, layouts, outputs and errors as for gdn_prefill_backward, with the
+ * workspace sized by gdn_prefill_backward_chunked_workspace_size().
+ */
+gdn_status gdn_prefill_backward_chunked(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* a,
+                                        const float* b, const float* A_log, const float* dt_bias,
+                                        const int32_t* cu_seqlens, int32_t n_seq, int64_t T, int32_t Hqk,
+                                        int32_t Hv, int32_t d, float scale, const float* initial_state,
+                                        const float* d_o, const float* d_final_state, float* dq, float* dk,
+                                        float* dv, float* da, float* db, float* dA_log, float* ddt_bias,
+                                        float* d_initial_state, void* workspace, size_t workspace_bytes,
+                                        gdn_stream_t stream);
+
+/*
  * gdn_selftest_bounded_wait -- failure detection check.  Runs, in one small
  * kernel, one of the bounded waits the prefill's CTAs use, on something that
  * never happens: which = 0 waits for a counter in global memory (as on the

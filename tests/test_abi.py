@@ -30,6 +30,7 @@ def test_header_declares_the_entry_points():
                      "gdn_decode_step", "gdn_decode_step_fused", "gdn_prefill_status",
                      "gdn_gated_norm", "gdn_prefill_gated", "gdn_decode_step_gated",
                      "gdn_prefill_backward", "gdn_prefill_backward_workspace_size",
+                     "gdn_prefill_backward_chunked", "gdn_prefill_backward_chunked_workspace_size",
                      "gdn_selftest_bounded_wait", "gdn_status_string"):
         assert required in names
 
@@ -217,6 +218,34 @@ def test_backward_rejects_bad_arguments(L):
     def call(d=128, d_o=_p(), dq=_p(), dA=_p(), wsp=_p(0x20000), wsb=ws):
         return L.gdn_prefill_backward(_p(), _p(), _p(), _p(), _p(), _p(), _p(), None, 1, 64, 16, 48, d, 0.088,
                                       None, d_o, None, dq, _p(), _p(), _p(), _p(), dA, _p(), None, wsp, wsb, None)
+    assert call(d=64) == 2
+    assert call(d_o=None) == 1
+    assert call(dq=None) == 1
+    assert call(dA=None) == 1
+    assert call(dq=_p(FAKE + 4)) == 3
+    assert call(wsb=ws - 256) == 6
+    assert call(wsp=_p(0x20000 + 16)) == 3
+
+
+def test_chunked_backward_workspace_formula(L):
+    # gdn.h: per (slot, value head) W, U', T, Y, S, dS and the decays; dq, dk per
+    # value head; the chunk list and gate sums, each region rounded to 256 bytes
+    r = lambda x: (x + 255) // 256 * 256
+    for n, T, Hv in ((1, 8192, 48), (16, 241567, 48), (3, 100, 6)):
+        d = 128
+        sh = (T // 64 + n + 1) * Hv
+        want = (r((T // 64 + n + 1) * 2 * 4) + 2 * r(sh * 64 * d * 4) + r(sh * 64 * 64 * 4)
+                + 3 * r(sh * d * d * 4) + r(sh * 65 * 4) + 2 * r(T * Hv * d * 4) + r(sh * 2 * 4))
+        assert L.gdn_prefill_backward_chunked_workspace_size(n, T, Hv, d) == want
+
+
+def test_chunked_backward_rejects_bad_arguments(L):
+    ws = L.gdn_prefill_backward_chunked_workspace_size(1, 64, 48, 128)
+
+    def call(d=128, d_o=_p(), dq=_p(), dA=_p(), wsp=_p(0x20000), wsb=ws):
+        return L.gdn_prefill_backward_chunked(_p(), _p(), _p(), _p(), _p(), _p(), _p(), None, 1, 64, 16, 48, d,
+                                              0.088, None, d_o, None, dq, _p(), _p(), _p(), _p(), dA, _p(), None,
+                                              wsp, wsb, None)
     assert call(d=64) == 2
     assert call(d_o=None) == 1
     assert call(dq=None) == 1
