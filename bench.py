@@ -10,7 +10,8 @@ T = 262144 prefill (non-zero initial state), the 16-sequence varlen prefill
 (recurrence + gated norm, fused and in two passes), the backward pass at
 T = 8192, and one decode step over 128 sequences x 48 layers with the 19.3 GB
 float32 state updated in place (plain, with the front end fused, with a bf16
-state, and with the gated norm fused).
+state, and with the gated norm fused); last, at N = 1 only, the backward pass
+through the chunked form at T = 8192 (an error there is recorded in its entry).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -307,6 +308,13 @@ def bench_main(args, world, rank, local):
         extra["decode_fused_128seq_48layers"] = bench_decode_fused(args, dev, peaks, world)
         extra["decode_bf16state_128seq_48layers"] = bench_decode(args, dev, peaks, world, bf16_state=True)
         extra["decode_gated_128seq_48layers"] = bench_decode(args, dev, peaks, world, gated=True)
+        if world == 1:
+            # the chunked backward is the newest path: last, and an error is
+            # recorded in its entry rather than ending the run
+            try:
+                extra["backward_chunked_T8192"] = bench_backward(args, dev, flush, peaks, world, chunked=True)
+            except Exception as exc:     # noqa: BLE001
+                extra["backward_chunked_T8192"] = {"error": str(exc)[:300]}
 
     value = weak_scaling_rate(T, ms_max, world)
     line = {
@@ -538,9 +546,10 @@ def bench_layer_tail(args, dev, flush, peaks, world):
     return out
 
 
-def bench_backward(args, dev, flush, peaks, world):
-    """gdn_prefill_backward at T = 8192 (one sequence, 16 / 48 heads, S0 and
-    dL/dS_T given): all gradients of the recurrence."""
+def bench_backward(args, dev, flush, peaks, world, chunked=False):
+    """gdn_prefill_backward (or, chunked, gdn_prefill_backward_chunked) at
+    T = 8192 (one sequence, 16 / 48 heads, S0 and dL/dS_T given): all gradients
+    of the recurrence."""
     import torch
     import gated_deltanet_recurrence_prefill_b200 as gdn
     T = T_MAIN
@@ -561,13 +570,15 @@ def bench_backward(args, dev, flush, peaks, world):
     s0 = 0.02 * torch.randn(1, HV, D, D, generator=gen, device=dev)
     d_o = torch.randn(T, HV, D, generator=gen, device=dev)
     d_fin = 0.1 * torch.randn(1, HV, D, D, generator=gen, device=dev)
-    ws = torch.empty(gdn.lib().gdn_prefill_backward_workspace_size(1, T, HV, D), dtype=torch.uint8, device=dev)
+    entry = "gdn_prefill_backward_chunked" if chunked else "gdn_prefill_backward"
+    ws_bytes = getattr(gdn.lib(), entry + "_workspace_size")(1, T, HV, D)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    fn = gdn.prefill_backward_chunked if chunked else gdn.prefill_backward
 
     def step(ev):
         if ev:
             ev["start"].record()
-        gdn.prefill_backward(q, k, v, a, b, A_log, dt_bias, d_o, d_final_state=d_fin, initial_state=s0,
-                             workspace=ws)
+        fn(q, k, v, a, b, A_log, dt_bias, d_o, d_final_state=d_fin, initial_state=s0, workspace=ws)
         if ev:
             ev["end"].record()
 
@@ -575,10 +586,11 @@ def bench_backward(args, dev, flush, peaks, world):
                   "end": torch.cuda.Event(enable_timing=True)}
     times, _ = _time_steps(step, 3, 3, flush, mk, world)
     ms = _max_over_ranks(sum(times) / len(times), world)
-    out = {"workload": f"gdn_prefill_backward T={T} N=1 Hqk=16 Hv=48 d=128, S0 and dL/dS_T given "
-                       "(CUDA cores, one CTA per value head, token by token)",
+    how = ("CUDA cores, chunk-parallel prep and gradients, two state chains over chunks" if chunked
+           else "CUDA cores, one CTA per value head, token by token")
+    out = {"workload": f"{entry} T={T} N=1 Hqk=16 Hv=48 d=128, S0 and dL/dS_T given ({how})",
            "ms": round(ms, 3), "tokens_per_s_layer": round(weak_scaling_rate(T, ms, world), 1),
-           "launches_per_step": 3}
+           "launches_per_step": 7 if chunked else 3}
     del q, k, v, d_o, ws
     torch.cuda.empty_cache()
     return out
