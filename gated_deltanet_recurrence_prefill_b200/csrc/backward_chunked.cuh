@@ -32,6 +32,7 @@
 
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 #ifndef BWC_FN
@@ -42,6 +43,9 @@
 #endif
 #ifndef BWC_SYNC
 #define BWC_SYNC() __syncthreads()
+#endif
+#ifndef BWC_MISALIGNED
+#define BWC_MISALIGNED(ptr) abort()
 #endif
 
 namespace gdn {
@@ -54,8 +58,11 @@ constexpr int kRowSplit = 4;             // chain CTAs per (sequence, value head
 constexpr int kRows = kD / kRowSplit;    // state rows per chain CTA
 constexpr int kEB = 16;                  // v columns per step of the gradient kernel
 constexpr int kLd = kD + 1;              // padded row strides of shared-memory matrices
-constexpr int kLc = kC + 1;
+constexpr int kLc = kC + 1;               // (scalar access: consecutive rows on different banks)
 constexpr int kLe = kEB + 1;
+constexpr int kL4 = kD + 4;              // row strides for float4 access (16-byte rows)
+constexpr int kLt = kC + 4;
+constexpr int kLu = kRows + 4;
 
 // ---- workspace plan ----------------------------------------------------------------
 // Per (chunk slot, value head): W, U' [64 x 128], T [64 x 64], Y, S_c, dS_c
@@ -132,7 +139,9 @@ BWC_HD void bind_workspace(Params& p, void* ws, const Plan& plan) {
 
 // Shared-memory floats each block function needs.
 constexpr int kPrepFloats = 5 * kC * kLd + 3 * kC * kLc + 5 * kC;
-constexpr int kChainFloats = 2 * kC * kLd + kRows * kLd + kC * (kRows + 1) + kRows * kLc + kC + 4;
+constexpr int kFwdChainFloats = 2 * kC * kL4 + kRows * kLd + kC * kLu + kC + 4;
+constexpr int kBwdChainFloats = kC * kL4 + kD * kLt + kRows * kLd + kRows * kLt + kC + 4;
+constexpr int kChainFloats = kFwdChainFloats > kBwdChainFloats ? kFwdChainFloats : kBwdChainFloats;
 constexpr int kGradFloats = 3 * kC * kLd + 5 * kC * kLc + 2 * kEB * kLd + 6 * kC * kLe + 9 * kC + kThreads;
 
 // ---- small helpers ----------------------------------------------------------------------
@@ -145,6 +154,23 @@ BWC_FN float bf16f(uint16_t h) {
     memcpy(&f, &u, sizeof f);
     return f;
 #endif
+}
+
+// four consecutive floats from a 16-byte aligned address (the host build checks
+// the alignment, so that the CPU tests catch a misaligned vector access)
+struct F4 {
+    float v[4];
+};
+BWC_FN F4 ld4(const float* ptr) {
+    F4 r;
+#ifdef __CUDA_ARCH__
+    const float4 x = *reinterpret_cast<const float4*>(ptr);
+    r.v[0] = x.x; r.v[1] = x.y; r.v[2] = x.z; r.v[3] = x.w;
+#else
+    if (reinterpret_cast<uintptr_t>(ptr) & 15u) BWC_MISALIGNED(ptr);
+    memcpy(r.v, ptr, sizeof r.v);
+#endif
+    return r;
 }
 
 // softplus(x) = log(1 + e^x) without overflow; log alpha and beta as in the forward
@@ -192,12 +218,13 @@ BWC_FN void chunk_gates(const Params& p, int h, int64_t t0, int L, int tid, floa
     BWC_SYNC();
 }
 
-// Rows t0 .. t0 + 63 of a bf16 [T, H, 128] tensor (head hh) into a [64][kLd]
+// Rows t0 .. t0 + 63 of a bf16 [T, H, 128] tensor (head hh) into a [64][ld]
 // float matrix; rows >= L are zero.
-BWC_FN void load_rows_bf16(const uint16_t* x, int H, int hh, int64_t t0, int L, int tid, float* dst) {
+BWC_FN void load_rows_bf16(const uint16_t* x, int H, int hh, int64_t t0, int L, int tid, float* dst,
+                           int ld = kLd) {
     for (int idx = tid; idx < kC * kD; idx += kThreads) {
         const int i = idx >> 7, e = idx & (kD - 1);
-        dst[i * kLd + e] = i < L ? bf16f(x[((t0 + i) * H + hh) * kD + e]) : 0.f;
+        dst[i * ld + e] = i < L ? bf16f(x[((t0 + i) * H + hh) * kD + e]) : 0.f;
     }
 }
 
@@ -336,7 +363,8 @@ BWC_FN void prep_block(const Params& p, int64_t slot, int h, int tid, float* sm)
 }
 
 // ---- the chains: per (sequence, value head, quarter of the state rows) -----------------
-// Thread tid owns state row r0 + tid / 8 and its 16 columns from 16 (tid % 8).
+// Thread tid owns rows 4 (tid / 32) .. + 4 of the CTA's 32 state rows and
+// columns 4 (tid % 32) .. + 4.
 
 // Forward: S_c for every chunk of sequence n into the workspace.
 BWC_FN void fwd_chain_block(const Params& p, int n, int h, int rq, int tid, float* sm) {
@@ -344,53 +372,64 @@ BWC_FN void fwd_chain_block(const Params& p, int n, int h, int rq, int tid, floa
     seq_bounds(p, n, bos, eos);
     const int g = h / (p.Hv / p.Hqk);
     const int r0 = rq * kRows;
-    const int er = tid >> 3, c0 = (tid & 7) * 16;
-    float* Ws = sm;
-    float* Ks = Ws + kC * kLd;
-    float* Ss = Ks + kC * kLd;                 // my rows of S   [kRows][kLd]
-    float* Us = Ss + kRows * kLd;              // U' then kap U  [kC][kRows + 1]
-    float* kap = Us + kC * (kRows + 1) + kRows * kLc;
+    const int w4 = (tid >> 5) * 4, l4 = (tid & 31) * 4;     // my 4 x 4 block of the state rows
+    const int i2 = (tid >> 3) * 2, e4 = (tid & 7) * 4;      // my 2 x 4 block of U [64 x 32]
+    float* Ws = sm;                            // W             [kC][kL4]
+    float* Ks = Ws + kC * kL4;                 // K             [kC][kL4]
+    float* Ss = Ks + kC * kL4;                 // my rows of S  [kRows][kLd]
+    float* Us = Ss + kRows * kLd;              // U', then kap U for my rows  [kC][kLu]
+    float* kap = Us + kC * kLu;
     float* gl = kap + kC;
-    float s[16];
-    for (int x = 0; x < 16; ++x)
-        s[x] = p.s0 ? p.s0[(((size_t)n * p.Hv + h) * kD + r0 + er) * kD + c0 + x] : 0.f;
+    float s[4][4];
+    const size_t unit = ((size_t)n * p.Hv + h) * kD * kD + (size_t)(r0 + w4) * kD + l4;
+    for (int r = 0; r < 4; ++r)
+        for (int c = 0; c < 4; ++c) s[r][c] = p.s0 ? p.s0[unit + (size_t)r * kD + c] : 0.f;
     const int64_t nch = (eos - bos + kC - 1) / kC;
     for (int64_t j = 0; j < nch; ++j) {
         const int64_t t0 = bos + j * kC;
         const int L = (int)((eos - t0) < kC ? (eos - t0) : kC);
         const size_t sh = sh_index(p, t0 / kC + n, h);
-        float* Sg = p.S + sh * kD * kD + (size_t)(r0 + er) * kD + c0;
-        for (int x = 0; x < 16; ++x) {
-            Sg[x] = s[x];
-            Ss[er * kLd + c0 + x] = s[x];
-        }
+        float* Sg = p.S + sh * kD * kD + (size_t)(r0 + w4) * kD + l4;
+        for (int r = 0; r < 4; ++r)
+            for (int c = 0; c < 4; ++c) {
+                Sg[(size_t)r * kD + c] = s[r][c];
+                Ss[(w4 + r) * kLd + l4 + c] = s[r][c];
+            }
         const float* Wg = p.W + sh * kC * kD;
         const float* Ug = p.Up + sh * kC * kD;
-        for (int idx = tid; idx < kC * kD; idx += kThreads) {
-            const int i = idx >> 7, f = idx & (kD - 1);
-            Ws[i * kLd + f] = Wg[idx];
-        }
-        load_rows_bf16(p.k, p.Hqk, g, t0, L, tid, Ks);
+        for (int idx = tid; idx < kC * kD; idx += kThreads) Ws[(idx >> 7) * kL4 + (idx & (kD - 1))] = Wg[idx];
+        load_rows_bf16(p.k, p.Hqk, g, t0, L, tid, Ks, kL4);
         for (int idx = tid; idx < kC * kRows; idx += kThreads) {
             const int i = idx / kRows, e = idx % kRows;
-            Us[i * (kRows + 1) + e] = Ug[i * kD + r0 + e];
+            Us[i * kLu + e] = Ug[(size_t)i * kD + r0 + e];
         }
         if (tid < kC) kap[tid] = p.G[sh * (kC + 1) + tid];
         if (tid == 0) gl[0] = p.G[sh * (kC + 1) + kC];
         BWC_SYNC();
-        // kap_i (U'_ie - sum_f W_if S_ef) for my rows e
-        for (int idx = tid; idx < kC * kRows; idx += kThreads) {
-            const int i = idx / kRows, e = idx % kRows;
-            float u = Us[i * (kRows + 1) + e];
-            for (int f = 0; f < kD; ++f) u = fmaf(-Ws[i * kLd + f], Ss[e * kLd + f], u);
-            Us[i * (kRows + 1) + e] = kap[i] * u;
+        // kap_i (U'_ie - sum_f W_if S_ef) for rows i2, i2 + 1 and my rows e4 .. e4 + 3
+        {
+            float u[2][4];
+            for (int a = 0; a < 2; ++a)
+                for (int x = 0; x < 4; ++x) u[a][x] = Us[(i2 + a) * kLu + e4 + x];
+            for (int f = 0; f < kD; ++f) {
+                const float w0 = Ws[i2 * kL4 + f], w1 = Ws[(i2 + 1) * kL4 + f];
+                for (int x = 0; x < 4; ++x) {
+                    const float sv = Ss[(e4 + x) * kLd + f];
+                    u[0][x] = fmaf(-w0, sv, u[0][x]);
+                    u[1][x] = fmaf(-w1, sv, u[1][x]);
+                }
+            }
+            for (int a = 0; a < 2; ++a)
+                for (int x = 0; x < 4; ++x) Us[(i2 + a) * kLu + e4 + x] = kap[i2 + a] * u[a][x];
         }
         BWC_SYNC();
         const float gL = gl[0];
-        for (int x = 0; x < 16; ++x) {
-            float acc = gL * s[x];
-            for (int i = 0; i < L; ++i) acc = fmaf(Us[i * (kRows + 1) + er], Ks[i * kLd + c0 + x], acc);
-            s[x] = acc;
+        for (int r = 0; r < 4; ++r)
+            for (int c = 0; c < 4; ++c) s[r][c] *= gL;
+        for (int i = 0; i < L; ++i) {
+            const F4 u = ld4(Us + i * kLu + w4), kv = ld4(Ks + i * kL4 + l4);
+            for (int r = 0; r < 4; ++r)
+                for (int c = 0; c < 4; ++c) s[r][c] = fmaf(u.v[r], kv.v[c], s[r][c]);
         }
         BWC_SYNC();
     }
@@ -403,53 +442,70 @@ BWC_FN void bwd_chain_block(const Params& p, int n, int h, int rq, int tid, floa
     seq_bounds(p, n, bos, eos);
     const int g = h / (p.Hv / p.Hqk);
     const int r0 = rq * kRows;
-    const int er = tid >> 3, c0 = (tid & 7) * 16;
-    float* Ws = sm;
-    float* Ks = Ws + kC * kLd;
-    float* Ss = Ks + kC * kLd;                 // my rows of dS  [kRows][kLd]
-    float* Xs = Ss + kRows * kLd + kC * (kRows + 1);   // kap_i (dS K^T)_{e,i}  [kRows][kLc]
-    float* kap = Xs + kRows * kLc;
+    const int w4 = (tid >> 5) * 4, l4 = (tid & 31) * 4;     // my 4 x 4 block of the state rows
+    const int e2 = (tid >> 4) * 2, i4 = (tid & 15) * 4;     // my 2 x 4 block of X [32 x 64]
+    float* Ws = sm;                            // W              [kC][kL4]
+    float* KT = Ws + kC * kL4;                 // K transposed   [kD][kLt]
+    float* Ss = KT + kD * kLt;                 // my rows of dS  [kRows][kLd]
+    float* Xs = Ss + kRows * kLd;              // kap_i (dS K^T)_{e,i}  [kRows][kLt]
+    float* kap = Xs + kRows * kLt;
     float* gl = kap + kC;
-    float s[16];
-    const size_t unit = ((size_t)n * p.Hv + h) * kD * kD + (size_t)(r0 + er) * kD + c0;
-    for (int x = 0; x < 16; ++x) s[x] = p.d_fin ? p.d_fin[unit + x] : 0.f;
+    float s[4][4];
+    const size_t unit = ((size_t)n * p.Hv + h) * kD * kD + (size_t)(r0 + w4) * kD + l4;
+    for (int r = 0; r < 4; ++r)
+        for (int c = 0; c < 4; ++c) s[r][c] = p.d_fin ? p.d_fin[unit + (size_t)r * kD + c] : 0.f;
     const int64_t nch = (eos - bos + kC - 1) / kC;
     for (int64_t j = nch - 1; j >= 0; --j) {
         const int64_t t0 = bos + j * kC;
         const int L = (int)((eos - t0) < kC ? (eos - t0) : kC);
         const size_t sh = sh_index(p, t0 / kC + n, h);
-        float* dSg = p.dS + sh * kD * kD + (size_t)(r0 + er) * kD + c0;
-        for (int x = 0; x < 16; ++x) {
-            dSg[x] = s[x];
-            Ss[er * kLd + c0 + x] = s[x];
-        }
+        float* dSg = p.dS + sh * kD * kD + (size_t)(r0 + w4) * kD + l4;
+        for (int r = 0; r < 4; ++r)
+            for (int c = 0; c < 4; ++c) {
+                dSg[(size_t)r * kD + c] = s[r][c];
+                Ss[(w4 + r) * kLd + l4 + c] = s[r][c];
+            }
         const float* Wg = p.W + sh * kC * kD;
+        for (int idx = tid; idx < kC * kD; idx += kThreads) Ws[(idx >> 7) * kL4 + (idx & (kD - 1))] = Wg[idx];
         for (int idx = tid; idx < kC * kD; idx += kThreads) {
             const int i = idx >> 7, f = idx & (kD - 1);
-            Ws[i * kLd + f] = Wg[idx];
+            KT[f * kLt + i] = i < L ? bf16f(p.k[((t0 + i) * p.Hqk + g) * kD + f]) : 0.f;
         }
-        load_rows_bf16(p.k, p.Hqk, g, t0, L, tid, Ks);
         if (tid < kC) kap[tid] = p.G[sh * (kC + 1) + tid];
         if (tid == 0) gl[0] = p.G[sh * (kC + 1) + kC];
         BWC_SYNC();
-        for (int idx = tid; idx < kRows * kC; idx += kThreads) {
-            const int e = idx / kC, i = idx % kC;
-            float x = 0.f;
-            for (int f = 0; f < kD; ++f) x = fmaf(Ss[e * kLd + f], Ks[i * kLd + f], x);
-            Xs[e * kLc + i] = kap[i] * x;
+        {
+            float x[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            for (int f = 0; f < kD; ++f) {
+                const float d0 = Ss[e2 * kLd + f], d1 = Ss[(e2 + 1) * kLd + f];
+                const F4 kv = ld4(KT + f * kLt + i4);
+                for (int c = 0; c < 4; ++c) {
+                    x[0][c] = fmaf(d0, kv.v[c], x[0][c]);
+                    x[1][c] = fmaf(d1, kv.v[c], x[1][c]);
+                }
+            }
+            for (int a = 0; a < 2; ++a)
+                for (int c = 0; c < 4; ++c) Xs[(e2 + a) * kLt + i4 + c] = kap[i4 + c] * x[a][c];
         }
         BWC_SYNC();
         const float gL = gl[0];
-        const float* Yg = p.Y + sh * kD * kD + (size_t)(r0 + er) * kD + c0;
-        for (int x = 0; x < 16; ++x) {
-            float acc = gL * s[x] + Yg[x];
-            for (int i = 0; i < L; ++i) acc = fmaf(-Xs[er * kLc + i], Ws[i * kLd + c0 + x], acc);
-            s[x] = acc;
+        const float* Yg = p.Y + sh * kD * kD + (size_t)(r0 + w4) * kD + l4;
+        for (int r = 0; r < 4; ++r) {
+            const F4 y = ld4(Yg + (size_t)r * kD);
+            for (int c = 0; c < 4; ++c) s[r][c] = fmaf(gL, s[r][c], y.v[c]);
+        }
+        for (int i = 0; i < L; ++i) {
+            const F4 wv = ld4(Ws + i * kL4 + l4);
+            float xv[4];
+            for (int r = 0; r < 4; ++r) xv[r] = Xs[(w4 + r) * kLt + i];
+            for (int r = 0; r < 4; ++r)
+                for (int c = 0; c < 4; ++c) s[r][c] = fmaf(-xv[r], wv.v[c], s[r][c]);
         }
         BWC_SYNC();
     }
     if (p.d_init)
-        for (int x = 0; x < 16; ++x) p.d_init[unit + x] = s[x];
+        for (int r = 0; r < 4; ++r)
+            for (int c = 0; c < 4; ++c) p.d_init[unit + (size_t)r * kD + c] = s[r][c];
 }
 
 // ---- gradients of one (chunk, value head) -------------------------------------------------
@@ -539,20 +595,32 @@ BWC_FN void grad_block(const Params& p, int64_t slot, int h, int tid, float* sm)
             Vb[i * kLe + e] = ok ? bf16f(p.v[((t0 + i) * p.Hv + h) * kD + e0 + e]) : 0.f;
         }
         BWC_SYNC();
-        // U = U' - W S^T; K dS^T; Q S^T; P^T dO  (element (i, e) per thread)
-        for (int idx = tid; idx < kC * kEB; idx += kThreads) {
-            const int i = idx / kEB, e = idx % kEB;
-            float u = Ub[i * kLe + e], kds = 0.f, qs = 0.f, pdo = 0.f;
+        // U = U' - W S^T; K dS^T; Q S^T; P^T dO  (row i, columns eg .. eg + 3 per thread)
+        {
+            static_assert(kC * kEB == 4 * kThreads, "one row and four v columns per thread");
+            const int i = tid >> 2, eg = (tid & 3) * 4;
+            float u[4], kds[4] = {0.f, 0.f, 0.f, 0.f}, qs[4] = {0.f, 0.f, 0.f, 0.f}, pdo[4] = {0.f, 0.f, 0.f, 0.f};
+            for (int x = 0; x < 4; ++x) u[x] = Ub[i * kLe + eg + x];
             for (int f = 0; f < kD; ++f) {
-                u = fmaf(-Ws[i * kLd + f], Sb[e * kLd + f], u);
-                kds = fmaf(Ks[i * kLd + f], dSb[e * kLd + f], kds);
-                qs = fmaf(Qs[i * kLd + f], Sb[e * kLd + f], qs);
+                const float wv = Ws[i * kLd + f], kv = Ks[i * kLd + f], qv = Qs[i * kLd + f];
+                for (int x = 0; x < 4; ++x) {
+                    const float sv = Sb[(eg + x) * kLd + f], dsv = dSb[(eg + x) * kLd + f];
+                    u[x] = fmaf(-wv, sv, u[x]);
+                    kds[x] = fmaf(kv, dsv, kds[x]);
+                    qs[x] = fmaf(qv, sv, qs[x]);
+                }
             }
-            for (int m = i; m < L; ++m) pdo = fmaf(Pm[m * kLc + i], dOb[m * kLe + e], pdo);
-            Ub[i * kLe + e] = u;
-            dUb[i * kLe + e] = kap[i] * kds + p.scale * pdo;
-            R1[i * kLe + e] = u * kds;
-            R2[i * kLe + e] = dOb[i * kLe + e] * qs;
+            for (int m = i; m < L; ++m) {
+                const float pm = Pm[m * kLc + i];
+                for (int x = 0; x < 4; ++x) pdo[x] = fmaf(pm, dOb[m * kLe + eg + x], pdo[x]);
+            }
+            for (int x = 0; x < 4; ++x) {
+                const int e = eg + x;
+                Ub[i * kLe + e] = u[x];
+                dUb[i * kLe + e] = kap[i] * kds[x] + p.scale * pdo[x];
+                R1[i * kLe + e] = u[x] * kds[x];
+                R2[i * kLe + e] = dOb[i * kLe + e] * qs[x];
+            }
         }
         BWC_SYNC();
         if (tid < kC) {
