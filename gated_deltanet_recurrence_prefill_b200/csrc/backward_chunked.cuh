@@ -229,21 +229,33 @@ BWC_FN void load_rows_bf16(const uint16_t* x, int H, int hh, int64_t t0, int L, 
 }
 
 // A' = strict_lower(Gam o K K^T) and P = lower(Gam o Q K^T), rows and columns
-// >= L zero.  K and Q are [64][kLd]; A' and P [64][kLc].
+// >= L zero.  K and Q are [64][kLd]; A' and P [64][kLc].  Thread tid takes rows
+// tid / 16 + 16 x and columns tid % 16 + 16 y (x, y < 4).
 BWC_FN void build_ap(const float* Ks, const float* Qs, const float* G, int L, int tid, float* Ap, float* Pm) {
-    for (int idx = tid; idx < kC * kC; idx += kThreads) {
-        const int i = idx >> 6, j = idx & (kC - 1);
-        float kk = 0.f, qk = 0.f;
-        if (j <= i && i < L) {
-            for (int f = 0; f < kD; ++f) {
-                kk = fmaf(Ks[i * kLd + f], Ks[j * kLd + f], kk);
-                qk = fmaf(Qs[i * kLd + f], Ks[j * kLd + f], qk);
-            }
+    const int ib = tid >> 4, jb = tid & 15;
+    float kk[4][4], qk[4][4];
+    for (int x = 0; x < 4; ++x)
+        for (int y = 0; y < 4; ++y) kk[x][y] = qk[x][y] = 0.f;
+    for (int f = 0; f < kD; ++f) {
+        float ki[4], qi[4], kj[4];
+        for (int x = 0; x < 4; ++x) {
+            ki[x] = Ks[(ib + 16 * x) * kLd + f];
+            qi[x] = Qs[(ib + 16 * x) * kLd + f];
+            kj[x] = Ks[(jb + 16 * x) * kLd + f];
         }
-        const float gm = (j <= i && i < L) ? expf(G[i] - G[j]) : 0.f;
-        Ap[i * kLc + j] = j < i ? gm * kk : 0.f;
-        Pm[i * kLc + j] = j <= i ? gm * qk : 0.f;
+        for (int x = 0; x < 4; ++x)
+            for (int y = 0; y < 4; ++y) {
+                kk[x][y] = fmaf(ki[x], kj[y], kk[x][y]);
+                qk[x][y] = fmaf(qi[x], kj[y], qk[x][y]);
+            }
     }
+    for (int x = 0; x < 4; ++x)
+        for (int y = 0; y < 4; ++y) {
+            const int i = ib + 16 * x, j = jb + 16 * y;
+            const float gm = (j <= i && i < L) ? expf(G[i] - G[j]) : 0.f;
+            Ap[i * kLc + j] = j < i ? gm * kk[x][y] : 0.f;
+            Pm[i * kLc + j] = j <= i ? gm * qk[x][y] : 0.f;
+        }
 }
 
 // ---- chunk list --------------------------------------------------------------------------
@@ -314,20 +326,35 @@ BWC_FN void prep_block(const Params& p, int64_t slot, int h, int tid, float* sm)
         }
     }
     BWC_SYNC();
-    // U' = T diag(beta) V and W = T diag(beta gam) K
+    // U' = T diag(beta) V and W = T diag(beta gam) K: thread tid takes rows
+    // 4 (tid / 16) .. + 4 and columns tid % 16 + 16 c (c < 8)
     float* Wg = p.W + sh * kC * kD;
     float* Ug = p.Up + sh * kC * kD;
-    for (int idx = tid; idx < kC * kD; idx += kThreads) {
-        const int i = idx >> 7, e = idx & (kD - 1);
-        float up = 0.f, w = 0.f;
-        for (int m = 0; m <= i; ++m) {
-            const float tb = Tm[i * kLc + m] * be[m];
-            up = fmaf(tb, Vs[m * kLd + e], up);
-            w = fmaf(tb * gam[m], Ks[m * kLd + e], w);
+    {
+        const int i4 = (tid >> 4) * 4, eb = tid & 15;
+        float up[4][8], w[4][8];
+        for (int r = 0; r < 4; ++r)
+            for (int c = 0; c < 8; ++c) up[r][c] = w[r][c] = 0.f;
+        for (int m = 0; m <= i4 + 3; ++m) {     // T is lower triangular (zeros above)
+            float tb[4], vv[8], kv[8];
+            for (int r = 0; r < 4; ++r) tb[r] = Tm[(i4 + r) * kLc + m] * be[m];
+            for (int c = 0; c < 8; ++c) {
+                vv[c] = Vs[m * kLd + eb + 16 * c];
+                kv[c] = gam[m] * Ks[m * kLd + eb + 16 * c];
+            }
+            for (int r = 0; r < 4; ++r)
+                for (int c = 0; c < 8; ++c) {
+                    up[r][c] = fmaf(tb[r], vv[c], up[r][c]);
+                    w[r][c] = fmaf(tb[r], kv[c], w[r][c]);
+                }
         }
-        Ug[idx] = up;
-        Wg[idx] = w;
-        Ws[i * kLd + e] = w;
+        for (int r = 0; r < 4; ++r)
+            for (int c = 0; c < 8; ++c) {
+                const int i = i4 + r, e = eb + 16 * c;
+                Ug[i * kD + e] = up[r][c];
+                Wg[i * kD + e] = w[r][c];
+                Ws[i * kLd + e] = w[r][c];
+            }
     }
     float* Tg = p.Tm + sh * kC * kC;
     for (int idx = tid; idx < kC * kC; idx += kThreads) Tg[idx] = Tm[(idx >> 6) * kLc + (idx & (kC - 1))];
@@ -341,24 +368,46 @@ BWC_FN void prep_block(const Params& p, int64_t slot, int h, int tid, float* sm)
         Vs[i * kLd + e] = i < L ? p.d_o[((t0 + i) * p.Hv + h) * kD + e] : 0.f;
     }
     BWC_SYNC();
-    // Z = P^T dO
-    for (int idx = tid; idx < kC * kD; idx += kThreads) {
-        const int j = idx >> 7, e = idx & (kD - 1);
-        float z = 0.f;
-        for (int i = j; i < L; ++i) z = fmaf(Pm[i * kLc + j], Vs[i * kLd + e], z);
-        Zs[j * kLd + e] = z;
+    // Z = P^T dO: thread tid takes rows 4 (tid / 16) .. + 4, columns tid % 16 + 16 c
+    {
+        const int j4 = (tid >> 4) * 4, eb = tid & 15;
+        float z[4][8];
+        for (int r = 0; r < 4; ++r)
+            for (int c = 0; c < 8; ++c) z[r][c] = 0.f;
+        for (int i = j4; i < L; ++i) {          // P is lower triangular (zeros above)
+            float pv[4], dv[8];
+            for (int r = 0; r < 4; ++r) pv[r] = Pm[i * kLc + j4 + r];
+            for (int c = 0; c < 8; ++c) dv[c] = Vs[i * kLd + eb + 16 * c];
+            for (int r = 0; r < 4; ++r)
+                for (int c = 0; c < 8; ++c) z[r][c] = fmaf(pv[r], dv[c], z[r][c]);
+        }
+        for (int r = 0; r < 4; ++r)
+            for (int c = 0; c < 8; ++c) Zs[(j4 + r) * kLd + eb + 16 * c] = z[r][c];
     }
     BWC_SYNC();
-    // Y = scale (dO^T diag(gam) Q - Z^T W)
+    // Y = scale (dO^T diag(gam) Q - Z^T W): thread tid takes rows tid / 16 + 16 x
+    // and columns tid % 16 + 16 c (x, c < 8)
     float* Yg = p.Y + sh * kD * kD;
-    for (int idx = tid; idx < kD * kD; idx += kThreads) {
-        const int e = idx >> 7, f = idx & (kD - 1);
-        float y = 0.f;
+    {
+        const int eb = tid >> 4, fb = tid & 15;
+        float y[8][8];
+        for (int x = 0; x < 8; ++x)
+            for (int c = 0; c < 8; ++c) y[x][c] = 0.f;
         for (int i = 0; i < L; ++i) {
-            y = fmaf(Vs[i * kLd + e] * gam[i], Qs[i * kLd + f], y);
-            y = fmaf(-Zs[i * kLd + e], Ws[i * kLd + f], y);
+            float dg[8], zv[8], qv[8], wv[8];
+            for (int x = 0; x < 8; ++x) {
+                dg[x] = gam[i] * Vs[i * kLd + eb + 16 * x];
+                zv[x] = Zs[i * kLd + eb + 16 * x];
+            }
+            for (int c = 0; c < 8; ++c) {
+                qv[c] = Qs[i * kLd + fb + 16 * c];
+                wv[c] = Ws[i * kLd + fb + 16 * c];
+            }
+            for (int x = 0; x < 8; ++x)
+                for (int c = 0; c < 8; ++c) y[x][c] = fmaf(dg[x], qv[c], fmaf(-zv[x], wv[c], y[x][c]));
         }
-        Yg[idx] = p.scale * y;
+        for (int x = 0; x < 8; ++x)
+            for (int c = 0; c < 8; ++c) Yg[(size_t)(eb + 16 * x) * kD + fb + 16 * c] = p.scale * y[x][c];
     }
 }
 
