@@ -8,6 +8,8 @@ passages it follows.
 from .oracle import (  # noqa: F401
     build,
     conv1d_silu,
+    conv1d_silu_backward,
+    conv1d_silu_f64,
     decode,
     gated_norm,
     log_alpha,

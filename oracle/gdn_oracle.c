@@ -969,3 +969,115 @@ int gdn_oracle_prefill_backward_chunked(const double* q, const double* k, const 
     free(TtdW); free(dS); free(dSn);
     return 0;
 }
+
+/*
+ * Front end with every input in double (x [T, Ctot], w [Ctot, 4], conv_state
+ * [n_seq, Ctot, 3] or NULL): the same arithmetic as gdn_oracle_conv1d_silu,
+ * for finite differences of the front end's gradient.  Outputs as there
+ * (q, k, v; no conv_state_out).
+ */
+static double gdn_oracle_front_x(const double* x, const double* cs, int64_t Ctot, int n, int64_t bos,
+                                 int64_t tau, int64_t c) {
+    if (tau >= bos) return x[tau * Ctot + c];
+    const int64_t m = bos - tau;                       /* position bos - m is history slot 3 - m */
+    return cs ? cs[((int64_t)n * Ctot + c) * 3 + (3 - m)] : 0.0;
+}
+
+int gdn_oracle_conv1d_silu_f64(const double* x, const double* w, const int32_t* cu_seqlens, int32_t n_seq,
+                               int64_t T, int32_t Hqk, int32_t Hv, int32_t d, const double* conv_state_in,
+                               double* q, double* k, double* v) {
+    if (Hqk <= 0 || Hv <= 0 || d <= 0 || n_seq <= 0 || T < 0) return -1;
+    if (!cu_seqlens && n_seq != 1) return -1;
+    const int64_t n_heads = 2 * Hqk + Hv, Ctot = n_heads * d;
+    double* y = malloc(sizeof(double) * d);
+    for (int n = 0; n < n_seq; ++n) {
+        const int64_t bos = cu_seqlens ? cu_seqlens[n] : 0, eos = cu_seqlens ? cu_seqlens[n + 1] : T;
+        for (int64_t hh = 0; hh < n_heads; ++hh)
+            for (int64_t t = bos; t < eos; ++t) {
+                double ss = 0.0;
+                for (int e = 0; e < d; ++e) {
+                    const int64_t c = hh * d + e;
+                    double acc = 0.0;
+                    for (int j = 0; j < 4; ++j)
+                        acc += w[c * 4 + j] * gdn_oracle_front_x(x, conv_state_in, Ctot, n, bos, t - 3 + j, c);
+                    y[e] = acc / (1.0 + exp(-acc));
+                    ss += y[e] * y[e];
+                }
+                const double inv = hh < 2 * Hqk ? 1.0 / sqrt(ss + 1e-6) : 1.0;
+                double* dst = hh < Hqk ? q + (t * Hqk + hh) * d
+                            : hh < 2 * Hqk ? k + (t * Hqk + (hh - Hqk)) * d : v + (t * Hv + (hh - 2 * Hqk)) * d;
+                for (int e = 0; e < d; ++e) dst[e] = y[e] * inv;
+            }
+    }
+    free(y);
+    return 0;
+}
+
+/*
+ * gdn_oracle_conv1d_silu_backward -- the gradient of the front end (conv1d,
+ * SiLU, per-head L2 norm of q and k) given dL/dq, dL/dk [T, Hqk, d] and dL/dv
+ * [T, Hv, d].  Reverse mode through each step of the forward:
+ *   out = a / n with n = sqrt(sum a^2 + 1e-6) (q, k heads; out = a for v):
+ *       da = (dout - out <dout, out>) / n;
+ *   a = silu(y) = y sigma(y):  dy = da sigma(y) (1 + y (1 - sigma(y)));
+ *   y[t, c] = sum_j w[c, j] x~[t - 3 + j, c]:  dx~ += w dy, dw += dy x~,
+ * where x~ before a sequence's first token is its conv_state history (or
+ * zero).  Outputs (all overwritten): dx [T, Ctot], dw [Ctot, 4] (summed over
+ * every token of every sequence), dconv_state [n_seq, Ctot, 3] or NULL.
+ * Parallel over heads only, so each sum has a fixed order.
+ */
+int gdn_oracle_conv1d_silu_backward(const double* x, const double* w, const int32_t* cu_seqlens, int32_t n_seq,
+                                    int64_t T, int32_t Hqk, int32_t Hv, int32_t d, const double* conv_state_in,
+                                    const double* dq, const double* dk, const double* dv, double* dx, double* dw,
+                                    double* dconv_state, int threads) {
+    if (Hqk <= 0 || Hv <= 0 || d <= 0 || n_seq <= 0 || T < 0) return -1;
+    if (!cu_seqlens && n_seq != 1) return -1;
+    set_threads(threads);
+    const int64_t n_heads = 2 * Hqk + Hv, Ctot = n_heads * d;
+    memset(dx, 0, sizeof(double) * T * Ctot);
+    memset(dw, 0, sizeof(double) * Ctot * 4);
+    if (dconv_state) memset(dconv_state, 0, sizeof(double) * n_seq * Ctot * 3);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t hh = 0; hh < n_heads; ++hh) {
+        double* yv = malloc(sizeof(double) * d);
+        double* av = malloc(sizeof(double) * d);
+        for (int n = 0; n < n_seq; ++n) {
+            const int64_t bos = cu_seqlens ? cu_seqlens[n] : 0, eos = cu_seqlens ? cu_seqlens[n + 1] : T;
+            for (int64_t t = bos; t < eos; ++t) {
+                double ss = 0.0;
+                for (int e = 0; e < d; ++e) {
+                    const int64_t c = hh * d + e;
+                    double acc = 0.0;
+                    for (int j = 0; j < 4; ++j)
+                        acc += w[c * 4 + j] * gdn_oracle_front_x(x, conv_state_in, Ctot, n, bos, t - 3 + j, c);
+                    yv[e] = acc;
+                    av[e] = acc / (1.0 + exp(-acc));
+                    ss += av[e] * av[e];
+                }
+                const double* dout = hh < Hqk ? dq + (t * Hqk + hh) * d
+                                   : hh < 2 * Hqk ? dk + (t * Hqk + (hh - Hqk)) * d
+                                                  : dv + (t * Hv + (hh - 2 * Hqk)) * d;
+                const int normed = hh < 2 * Hqk;
+                const double nrm = normed ? sqrt(ss + 1e-6) : 1.0;
+                double dot = 0.0;
+                if (normed)
+                    for (int e = 0; e < d; ++e) dot += dout[e] * av[e] / nrm;
+                for (int e = 0; e < d; ++e) {
+                    const int64_t c = hh * d + e;
+                    const double da = normed ? (dout[e] - av[e] / nrm * dot) / nrm : dout[e];
+                    const double sg = 1.0 / (1.0 + exp(-yv[e]));
+                    const double dy = da * sg * (1.0 + yv[e] * (1.0 - sg));
+                    for (int j = 0; j < 4; ++j) {
+                        const int64_t tau = t - 3 + j;
+                        dw[c * 4 + j] += dy * gdn_oracle_front_x(x, conv_state_in, Ctot, n, bos, tau, c);
+                        if (tau >= bos) dx[tau * Ctot + c] += w[c * 4 + j] * dy;
+                        else if (dconv_state) dconv_state[((int64_t)n * Ctot + c) * 3 + (3 - (bos - tau))] += w[c * 4 + j] * dy;
+                    }
+                }
+            }
+        }
+        free(yv);
+        free(av);
+    }
+    return 0;
+}

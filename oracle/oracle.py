@@ -57,6 +57,11 @@ def _bind(lib):
     lib.gdn_oracle_prefill_backward_chunked.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i32, i64, i32, i32,
                                                         i32, i32, dbl, vp, vp, vp, i32, vp, vp, vp, vp, vp,
                                                         vp, vp, vp]
+    lib.gdn_oracle_conv1d_silu_f64.restype = C.c_int
+    lib.gdn_oracle_conv1d_silu_f64.argtypes = [vp, vp, vp, i32, i64, i32, i32, i32, vp, vp, vp, vp]
+    lib.gdn_oracle_conv1d_silu_backward.restype = C.c_int
+    lib.gdn_oracle_conv1d_silu_backward.argtypes = [vp, vp, vp, i32, i64, i32, i32, i32, vp, vp, vp, vp, vp, vp,
+                                                    vp, C.c_int]
     lib.gdn_oracle_max_threads.restype = C.c_int
     lib.gdn_oracle_max_threads.argtypes = [C.c_int]
     return lib
@@ -324,4 +329,48 @@ def prefill_backward_chunked(q, k, v, a, b, A_log, dt_bias, d_o, d_final=None, c
         _ptr(out["db"]), _ptr(out["dA_log"]), _ptr(out["ddt_bias"]), _ptr(out["d_initial"]))
     if rc != 0:
         raise ValueError("oracle prefill_backward_chunked rejected its arguments")
+    return out
+
+
+def _front_x64(qkv):
+    """bf16 bits (uint16) or real values -> float64"""
+    x = np.asarray(qkv)
+    if x.dtype == np.uint16:
+        return (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def conv1d_silu_f64(qkv, conv_w, cu_seqlens=None, Hqk=16, Hv=48, d=128, conv_state=None, lib=None):
+    """The front end with every input in float64 (gdn_oracle_conv1d_silu_f64):
+    qkv [T, Ctot] (bf16 bits or values), conv_w [Ctot, 4], conv_state
+    [N, Ctot, 3] or None.  Returns (q, k, v)."""
+    x = _front_x64(qkv)
+    T = x.shape[0]
+    cu = None if cu_seqlens is None else np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    n_seq = 1 if cu is None else len(cu) - 1
+    q, k, v = np.zeros((T, Hqk, d)), np.zeros((T, Hqk, d)), np.zeros((T, Hv, d))
+    rc = _L(lib).gdn_oracle_conv1d_silu_f64(_ptr(x), _ptr(_f64(conv_w)), _ptr(cu), n_seq, T, Hqk, Hv, d,
+                                            _ptr(_f64(conv_state)), _ptr(q), _ptr(k), _ptr(v))
+    if rc != 0:
+        raise ValueError("oracle conv1d_silu_f64 rejected its arguments")
+    return q, k, v
+
+
+def conv1d_silu_backward(qkv, conv_w, dq, dk, dv, cu_seqlens=None, Hqk=16, Hv=48, d=128, conv_state=None,
+                         threads=0, lib=None):
+    """Gradient of the front end (gdn_oracle_conv1d_silu_backward) given dL/dq,
+    dL/dk [T, Hqk, d] and dL/dv [T, Hv, d].  Returns a dict with d_qkv
+    [T, Ctot], d_conv_w [Ctot, 4] and d_conv_state [N, Ctot, 3]."""
+    x = _front_x64(qkv)
+    T = x.shape[0]
+    cu = None if cu_seqlens is None else np.ascontiguousarray(cu_seqlens, dtype=np.int32)
+    n_seq = 1 if cu is None else len(cu) - 1
+    ctot = (2 * Hqk + Hv) * d
+    out = dict(d_qkv=np.zeros((T, ctot)), d_conv_w=np.zeros((ctot, 4)), d_conv_state=np.zeros((n_seq, ctot, 3)))
+    rc = _L(lib).gdn_oracle_conv1d_silu_backward(
+        _ptr(x), _ptr(_f64(conv_w)), _ptr(cu), n_seq, T, Hqk, Hv, d, _ptr(_f64(conv_state)), _ptr(_f64(dq)),
+        _ptr(_f64(dk)), _ptr(_f64(dv)), _ptr(out["d_qkv"]), _ptr(out["d_conv_w"]), _ptr(out["d_conv_state"]),
+        int(threads))
+    if rc != 0:
+        raise ValueError("oracle conv1d_silu_backward rejected its arguments")
     return out

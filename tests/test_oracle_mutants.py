@@ -61,6 +61,18 @@ MUTANTS = {
     "cbw_no_kappa_sum": ("dG[L - 1] += kk_sum;", "dG[L - 1] += 0.0 * kk_sum;"),
     "cbw_no_W_gamma_grad": ("dgam[j] += be[j] * sk;", "dgam[j] += 0.0 * sk;"),
     "cbw_carry_no_decay": ("dS[i] += gam[L - 1] * dSn[i];", "dS[i] += dSn[i];"),
+    "fbw_no_norm_projection": ("const double da = normed ? (dout[e] - av[e] / nrm * dot) / nrm : dout[e];",
+                               "const double da = normed ? dout[e] / nrm : dout[e];"),
+    "fbw_silu_derivative": ("const double dy = da * sg * (1.0 + yv[e] * (1.0 - sg));",
+                            "const double dy = da * sg * (1.0 + yv[e] * sg);"),
+    "fbw_weight_tap_reversed": ("dw[c * 4 + j] += dy * gdn_oracle_front_x(x, conv_state_in, Ctot, n, bos, tau, c);",
+                                "dw[c * 4 + (3 - j)] += dy * gdn_oracle_front_x(x, conv_state_in, Ctot, n, bos, tau, c);"),
+    "fbw_history_slot": ("else if (dconv_state) dconv_state[((int64_t)n * Ctot + c) * 3 + (3 - (bos - tau))] += w[c * 4 + j] * dy;",
+                         "else if (dconv_state) dconv_state[((int64_t)n * Ctot + c) * 3 + (bos - tau - 1)] += w[c * 4 + j] * dy;"),
+    "f64_front_history_slot": ("return cs ? cs[((int64_t)n * Ctot + c) * 3 + (3 - m)] : 0.0;",
+                               "return cs ? cs[((int64_t)n * Ctot + c) * 3 + (m - 1)] : 0.0;"),
+    "f64_front_norm_on_v": ("const double inv = hh < 2 * Hqk ? 1.0 / sqrt(ss + 1e-6) : 1.0;",
+                            "const double inv = 1.0 / sqrt(ss + 1e-6);"),
 }
 
 

@@ -577,3 +577,80 @@ def test_chunked_backward_without_initial_or_final_state(orc):
     got = orc.prefill_backward_chunked(**args, d_o=d_o, cu_seqlens=inp["cu_seqlens"], C=8)
     for name, x in ref.items():
         assert np.max(np.abs(got[name] - x)) <= 1e-11 * max(1.0, np.max(np.abs(x))), name
+
+
+# ---- the front end's backward: pinned by central finite differences ---------------------
+
+def _front_case(seed, lengths=(5, 2), Hqk=1, Hv=1, d=4):
+    rng = np.random.default_rng(seed)
+    T = sum(lengths)
+    ctot = (2 * Hqk + Hv) * d
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    bits = lambda x: (x.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    return dict(qkv=bits(rng.standard_normal((T, ctot))), conv_w=(0.5 * rng.standard_normal((ctot, 4))).astype(np.float32),
+                conv_state=rng.standard_normal((len(lengths), ctot, 3)).astype(np.float32), cu=cu,
+                Hqk=Hqk, Hv=Hv, d=d)
+
+
+def test_front_f64_equals_front_end(orc):
+    c = _front_case(11)
+    q1, k1, v1 = orc.conv1d_silu_f64(c["qkv"], c["conv_w"], c["cu"], c["Hqk"], c["Hv"], c["d"], c["conv_state"])
+    q2, k2, v2, _ = orc.conv1d_silu(c["qkv"], c["conv_w"], c["cu"], c["Hqk"], c["Hv"], c["d"], c["conv_state"])
+    for x, y in ((q1, q2), (k1, k2), (v1, v2)):
+        assert np.max(np.abs(x - y)) <= 1e-14
+
+
+def test_front_backward_matches_finite_differences(orc):
+    for seed in (12, 13):
+        c = _front_case(seed)
+        rng = np.random.default_rng(seed + 100)
+        T, Hqk, Hv, d = c["qkv"].shape[0], c["Hqk"], c["Hv"], c["d"]
+        gq, gk, gv = rng.standard_normal((T, Hqk, d)), rng.standard_normal((T, Hqk, d)), rng.standard_normal((T, Hv, d))
+        x0 = (c["qkv"].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        w0, s0 = c["conv_w"].astype(np.float64), c["conv_state"].astype(np.float64)
+
+        def loss(x, w, s):
+            q, k, v = orc.conv1d_silu_f64(x, w, c["cu"], Hqk, Hv, d, s)
+            return float(np.sum(gq * q) + np.sum(gk * k) + np.sum(gv * v))
+
+        g = orc.conv1d_silu_backward(x0, w0, gq, gk, gv, c["cu"], Hqk, Hv, d, s0)
+        h = 1e-6
+        for name, base, gname in (("x", x0, "d_qkv"), ("w", w0, "d_conv_w"), ("s", s0, "d_conv_state")):
+            fd = np.zeros_like(base)
+            for idx in np.ndindex(base.shape):
+                p_, m_ = base.copy(), base.copy()
+                p_[idx] += h
+                m_[idx] -= h
+                args_p = dict(x=x0, w=w0, s=s0)
+                args_m = dict(x=x0, w=w0, s=s0)
+                args_p[name], args_m[name] = p_, m_
+                fd[idx] = (loss(**args_p) - loss(**args_m)) / (2 * h)
+            assert np.max(np.abs(g[gname] - fd)) <= 2e-7 * max(1.0, np.max(np.abs(fd))), (seed, gname)
+
+
+def test_front_backward_without_history_and_one_sequence(orc):
+    # no conv_state: the history is zero; the gradient with respect to it is the
+    # one taken at an explicit zero history
+    c = _front_case(14, lengths=(6,))
+    rng = np.random.default_rng(114)
+    T = c["qkv"].shape[0]
+    gq, gk, gv = rng.standard_normal((T, 1, 4)), rng.standard_normal((T, 1, 4)), rng.standard_normal((T, 1, 4))
+    g = orc.conv1d_silu_backward(c["qkv"], c["conv_w"], gq, gk, gv, None, 1, 1, 4, None)
+    x0 = (c["qkv"].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    w0 = c["conv_w"].astype(np.float64)
+    h = 1e-6
+    base = orc.conv1d_silu_f64(x0, w0, None, 1, 1, 4, None)
+    fd = np.zeros_like(x0)
+    for idx in np.ndindex(x0.shape):
+        p_ = x0.copy()
+        p_[idx] += h
+        m_ = x0.copy()
+        m_[idx] -= h
+        lp = sum(float(np.sum(gg * o)) for gg, o in zip((gq, gk, gv), orc.conv1d_silu_f64(p_, w0, None, 1, 1, 4, None)))
+        lm = sum(float(np.sum(gg * o)) for gg, o in zip((gq, gk, gv), orc.conv1d_silu_f64(m_, w0, None, 1, 1, 4, None)))
+        fd[idx] = (lp - lm) / (2 * h)
+    assert base[0].shape == (T, 1, 4)
+    assert np.max(np.abs(g["d_qkv"] - fd)) <= 2e-7 * max(1.0, np.max(np.abs(fd)))
+    g0 = orc.conv1d_silu_backward(c["qkv"], c["conv_w"], gq, gk, gv, None, 1, 1, 4, np.zeros((1, 12, 3)))
+    assert np.array_equal(g["d_conv_state"], g0["d_conv_state"])
+    assert np.array_equal(g["d_qkv"], g0["d_qkv"])
