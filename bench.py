@@ -11,7 +11,8 @@ T = 262144 prefill (non-zero initial state), the 16-sequence varlen prefill
 T = 8192, and one decode step over 128 sequences x 48 layers with the 19.3 GB
 float32 state updated in place (plain, with the front end fused, with a bf16
 state, and with the gated norm fused); last, at N = 1 only, the backward pass
-through the chunked form at T = 8192 (an error there is recorded in its entry).
+through the chunked form and the front end's backward at T = 8192 (an error
+there is recorded in its entry).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -315,6 +316,10 @@ def bench_main(args, world, rank, local):
                 extra["backward_chunked_T8192"] = bench_backward(args, dev, flush, peaks, world, chunked=True)
             except Exception as exc:     # noqa: BLE001
                 extra["backward_chunked_T8192"] = {"error": str(exc)[:300]}
+            try:
+                extra["front_backward_T8192"] = bench_front_backward(args, dev, flush, peaks, world)
+            except Exception as exc:     # noqa: BLE001
+                extra["front_backward_T8192"] = {"error": str(exc)[:300]}
 
     value = weak_scaling_rate(T, ms_max, world)
     line = {
@@ -592,6 +597,47 @@ def bench_backward(args, dev, flush, peaks, world, chunked=False):
            "ms": round(ms, 3), "tokens_per_s_layer": round(weak_scaling_rate(T, ms, world), 1),
            "launches_per_step": 7 if chunked else 3}
     del q, k, v, d_o, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def bench_front_backward(args, dev, flush, peaks, world):
+    """gdn_conv1d_silu_backward at T = 8192 (one sequence, 16 / 48 heads, a
+    conv history given): d qkv, d conv_w and d conv_state.  Algorithmic bytes
+    per token: the bf16 input and the float32 dq, dk, dv read, the float32
+    d qkv written (2 + 4 + 4 bytes per channel)."""
+    import torch
+    import gated_deltanet_recurrence_prefill_b200 as gdn
+    T = T_MAIN
+    ctot = (2 * HQK + HV) * D
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(9)
+    qkv = torch.randn(T, ctot, generator=gen, device=dev).to(torch.bfloat16)
+    w = 0.5 * torch.randn(ctot, 4, generator=gen, device=dev)
+    cs = torch.randn(1, ctot, 3, generator=gen, device=dev)
+    dq = torch.randn(T, HQK, D, generator=gen, device=dev)
+    dk = torch.randn(T, HQK, D, generator=gen, device=dev)
+    dv = torch.randn(T, HV, D, generator=gen, device=dev)
+    ws = torch.empty(gdn.lib().gdn_conv1d_silu_backward_workspace_size(T, HQK, HV, D), dtype=torch.uint8,
+                     device=dev)
+
+    def step(ev):
+        if ev:
+            ev["start"].record()
+        gdn.conv1d_silu_backward(qkv, w, dq, dk, dv, HQK, HV, conv_state=cs, workspace=ws)
+        if ev:
+            ev["end"].record()
+
+    mk = lambda: {"start": torch.cuda.Event(enable_timing=True),
+                  "end": torch.cuda.Event(enable_timing=True)}
+    times, _ = _time_steps(step, 3, 5, flush, mk, world)
+    ms = _max_over_ranks(sum(times) / len(times), world)
+    nbytes = T * ctot * (2 + 4 + 4)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    out = {"workload": f"gdn_conv1d_silu_backward T={T} N=1 Hqk=16 Hv=48 d=128, conv history given",
+           "ms": round(ms, 4), "GB_s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+           "bytes_per_step": nbytes, "launches_per_step": 2}
+    del qkv, dq, dk, dv, ws
     torch.cuda.empty_cache()
     return out
 

@@ -9,6 +9,7 @@ from ._lib import (  # noqa: F401
     GdnError,
     STATUS,
     conv1d_silu,
+    conv1d_silu_backward,
     decode_step,
     decode_step_fused,
     decode_step_gated,

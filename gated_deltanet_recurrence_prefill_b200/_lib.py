@@ -47,6 +47,9 @@ SIGNATURES = {
     "gdn_prefill_backward": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
                                        _i32, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                        _vp, _vp, _sz, _vp]),
+    "gdn_conv1d_silu_backward_workspace_size": (_sz, [_i64, _i32, _i32, _i32]),
+    "gdn_conv1d_silu_backward": (C.c_int, [_vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _vp,
+                                           _vp, _vp, _vp, _vp, _sz, _vp]),
     "gdn_prefill_backward_chunked_workspace_size": (_sz, [_i32, _i64, _i32, _i32]),
     "gdn_prefill_backward_chunked": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
                                                _i32, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -144,6 +147,41 @@ def conv1d_silu(qkv, conv_w, Hqk, Hv, d=128, cu_seqlens=None, conv_state_in=None
                                _stream(stream))
     _check("gdn_conv1d_silu", st)
     return q, k, v
+
+
+def conv1d_silu_backward(qkv, conv_w, dq, dk, dv, Hqk, Hv, d=128, cu_seqlens=None, conv_state=None,
+                         want_d_conv_state=True, workspace=None, stream=None):
+    """gdn_conv1d_silu_backward: the front end's gradient given dL/dq, dL/dk
+    [T, Hqk, d] and dL/dv [T, Hv, d] (float32).  Returns a dict of float32
+    tensors d_qkv [T, Ctot], d_conv_w [Ctot, 4] and d_conv_state [N, Ctot, 3]
+    (or None)."""
+    import torch
+    T = qkv.shape[0]
+    ctot = (2 * Hqk + Hv) * d
+    n_seq = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    _need(qkv, torch.bfloat16, (T, ctot), "qkv")
+    _need(conv_w, torch.float32, (ctot, 4), "conv_w")
+    _need(dq, torch.float32, (T, Hqk, d), "dq")
+    _need(dk, torch.float32, (T, Hqk, d), "dk")
+    _need(dv, torch.float32, (T, Hv, d), "dv")
+    if cu_seqlens is not None:
+        _need(cu_seqlens, torch.int32, (n_seq + 1,), "cu_seqlens")
+    if conv_state is not None:
+        _need(conv_state, torch.float32, (n_seq, ctot, 3), "conv_state")
+    dev = qkv.device
+    out = dict(d_qkv=torch.empty(T, ctot, dtype=torch.float32, device=dev),
+               d_conv_w=torch.empty(ctot, 4, dtype=torch.float32, device=dev),
+               d_conv_state=torch.empty(n_seq, ctot, 3, dtype=torch.float32, device=dev)
+               if want_d_conv_state else None)
+    ws_bytes = int(lib().gdn_conv1d_silu_backward_workspace_size(T, Hqk, Hv, d))
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    st = lib().gdn_conv1d_silu_backward(
+        _ptr(qkv), _ptr(conv_w), _ptr(cu_seqlens), n_seq, T, Hqk, Hv, d, _ptr(conv_state), _ptr(dq), _ptr(dk),
+        _ptr(dv), _ptr(out["d_qkv"]), _ptr(out["d_conv_w"]), _ptr(out["d_conv_state"]), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("gdn_conv1d_silu_backward", st)
+    return out
 
 
 def prefill_workspace_size(n_seq, T, Hqk, Hv, d=128) -> int:

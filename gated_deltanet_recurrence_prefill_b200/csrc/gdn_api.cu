@@ -105,6 +105,33 @@ gdn_status gdn_conv1d_silu(const uint16_t* qkv, const float* conv_w, const int32
     return e == cudaSuccess ? GDN_OK : cuda_fail(e);
 }
 
+size_t gdn_conv1d_silu_backward_workspace_size(int64_t T, int32_t Hqk, int32_t Hv, int32_t d) {
+    (void)d;
+    if (T <= 0 || Hqk <= 0 || Hv <= 0) return 0;
+    return gdn::conv1d_silu_backward_workspace_bytes(T, Hqk, Hv);
+}
+
+gdn_status gdn_conv1d_silu_backward(const uint16_t* qkv, const float* conv_w, const int32_t* cu_seqlens,
+                                    int32_t n_seq, int64_t T, int32_t Hqk, int32_t Hv, int32_t d,
+                                    const float* conv_state, const float* dq, const float* dk, const float* dv,
+                                    float* d_qkv, float* d_conv_w, float* d_conv_state, void* workspace,
+                                    size_t workspace_bytes, gdn_stream_t stream) {
+    gdn_status st = check_heads(Hqk, Hv, d);
+    if (st != GDN_OK) return st;
+    if ((st = check_seqs(cu_seqlens, n_seq, T)) != GDN_OK) return st;
+    if (!conv_w || !d_conv_w || (T > 0 && (!qkv || !dq || !dk || !dv || !d_qkv))) return GDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {qkv, conv_w, cu_seqlens, conv_state, dq, dk, dv, d_qkv, d_conv_w, d_conv_state};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
+    const size_t need = T > 0 ? gdn::conv1d_silu_backward_workspace_bytes(T, Hqk, Hv) : 0;
+    if (need > 0 && (!workspace || workspace_bytes < need)) return GDN_ERR_WORKSPACE;
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_MISALIGNED;
+    gdn::ConvBackwardArgs a{qkv, conv_w, cu_seqlens, n_seq, T, Hqk, Hv, conv_state, dq, dk, dv,
+                            d_qkv, d_conv_w, d_conv_state, workspace};
+    cudaError_t e = gdn::launch_conv1d_silu_backward(a, (cudaStream_t)stream);
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
 size_t gdn_prefill_workspace_size(int32_t n_seq, int64_t T, int32_t Hqk, int32_t Hv, int32_t d) {
     (void)T; (void)Hqk; (void)d;
     const size_t lo = gdn::prefill_min_workspace_bytes(n_seq, Hv);

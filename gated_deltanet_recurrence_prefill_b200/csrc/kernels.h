@@ -106,6 +106,27 @@ cudaError_t launch_backward(const BackwardArgs& a, cudaStream_t stream);
 // the same gradient through the chunked form (backward_chunked.cu): two chains
 // over chunks and chunk-parallel work; workspace of backward_chunked_workspace_bytes
 size_t backward_chunked_workspace_bytes(int32_t n_seq, int64_t T, int32_t Hv);
+
+// the front end's gradient (conv1d_silu_backward.cu)
+struct ConvBackwardArgs {
+    const uint16_t* qkv;
+    const float* conv_w;
+    const int32_t* cu_seqlens;     // NULL: one sequence of length T
+    int32_t n_seq;
+    int64_t T;
+    int32_t Hqk;
+    int32_t Hv;
+    const float* conv_state;       // may be NULL
+    const float* dq;
+    const float* dk;
+    const float* dv;
+    float* d_qkv;
+    float* d_conv_w;
+    float* d_conv_state;           // may be NULL
+    void* workspace;
+};
+size_t conv1d_silu_backward_workspace_bytes(int64_t T, int32_t Hqk, int32_t Hv);
+cudaError_t launch_conv1d_silu_backward(const ConvBackwardArgs& a, cudaStream_t stream);
 cudaError_t launch_backward_chunked(const BackwardArgs& a, cudaStream_t stream);
 
 cudaError_t launch_gated_norm(const float* o, const uint16_t* z, const float* w, int64_t T, int32_t Hv,

@@ -107,6 +107,44 @@ gdn_status gdn_conv1d_silu(const uint16_t* qkv, const float* conv_w, const int32
                            uint16_t* q, uint16_t* k, uint16_t* v, gdn_stream_t stream);
 
 /*
+ * gdn_conv1d_silu_backward_workspace_size -- bytes of device workspace
+ * gdn_conv1d_silu_backward needs: per-tile sums of the weight gradient,
+ * ceil(T / 32) * (2 Hqk + Hv) * d * 4 floats, rounded up to 256 bytes (0 for
+ * T = 0).  Host-only.
+ */
+size_t gdn_conv1d_silu_backward_workspace_size(int64_t T, int32_t Hqk, int32_t Hv, int32_t d);
+
+/*
+ * gdn_conv1d_silu_backward -- the gradient of gdn_conv1d_silu (the front end:
+ * 4-tap causal depthwise conv1d, SiLU, L2 norm of each q and k head; the
+ * architecture page, section 2.1, gives the conv width) given dL/dq, dL/dk and
+ * dL/dv.  Reverse mode, recomputing the forward from qkv:
+ *     da = (dout - out <dout, out>) / n  for q and k heads (n the head's norm),
+ *     da = dout for v;  dy = da (sigma(y) + a (1 - sigma(y))) with a = silu(y);
+ *     d qkv[t] = sum_j w[c, j] dy[t + 3 - j] over tokens of t's sequence;
+ *     d conv_w[c, j] = sum over all tokens of dy[t] x~[t - 3 + j];
+ *     d conv_state: the taps of a sequence's first three tokens that read its
+ *     history (x~ is the history, or zero, before the first token).
+ * Inputs as for gdn_conv1d_silu (qkv [T, Ctot] bf16, conv_w [Ctot, 4],
+ * cu_seqlens, conv_state [n_seq, Ctot, 3] or NULL for a zero history), plus
+ *  dq, dk  [T, Hqk, d] float32,  dv [T, Hv, d] float32.
+ * Outputs (float32, overwritten; caller-owned):
+ *  d_qkv        [T, Ctot]
+ *  d_conv_w     [Ctot, 4]
+ *  d_conv_state [n_seq, Ctot, 3] or NULL (not written); with conv_state NULL
+ *               it is the gradient at a zero history.
+ * workspace: gdn_conv1d_silu_backward_workspace_size() bytes, 256-byte aligned
+ * (may be NULL when that is 0).  Supported: d = 128.  CUDA cores, float32, one
+ * CTA per (32-token tile, head); sums in a fixed order, so the result is
+ * deterministic.  Errors as for gdn_conv1d_silu, plus GDN_ERR_WORKSPACE.
+ */
+gdn_status gdn_conv1d_silu_backward(const uint16_t* qkv, const float* conv_w, const int32_t* cu_seqlens,
+                                    int32_t n_seq, int64_t T, int32_t Hqk, int32_t Hv, int32_t d,
+                                    const float* conv_state, const float* dq, const float* dk, const float* dv,
+                                    float* d_qkv, float* d_conv_w, float* d_conv_state, void* workspace,
+                                    size_t workspace_bytes, gdn_stream_t stream);
+
+/*
  * gdn_prefill_workspace_size -- bytes of device workspace with which
  * gdn_prefill runs its fastest kernel for these sizes (a multiple of 256; never
  * 0).  Host-only, no CUDA calls.  That kernel passes each chunk's

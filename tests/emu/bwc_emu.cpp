@@ -10,90 +10,22 @@
 //
 // usage: bwc_emu <dir>   reads <dir>/meta.txt and the raw input files the test
 // writes, runs the backward, writes the gradients as raw float32 files.
-#include <barrier>
-#include <cmath>
-#include <cstdio>
-#include <cstdlib>
-#include <cstring>
-#include <functional>
-#include <string>
-#include <thread>
-#include <vector>
+#include "emu_common.h"
 
-namespace emu {
-std::barrier<>* g_bar = nullptr;
-}
 #define BWC_FN inline
 #define BWC_HD inline
 #define BWC_SYNC() ::emu::g_bar->arrive_and_wait()
 #include "../../gated_deltanet_recurrence_prefill_b200/csrc/backward_chunked.cuh"
 
 using namespace gdn::bwc;
+using emu::load;
+using emu::save;
 
-// 256 worker threads, one per CUDA thread, kept for the whole run: each block
-// is handed to all of them between two barriers shared with the main thread
-class Pool {
-  public:
-    Pool() : start_(kThreads + 1), end_(kThreads + 1), sync_(kThreads) {
-        emu::g_bar = &sync_;
-        for (int t = 0; t < kThreads; ++t)
-            th_.emplace_back([this, t] {
-                for (;;) {
-                    start_.arrive_and_wait();
-                    if (stop_) return;
-                    job_(t, sm_);
-                    end_.arrive_and_wait();
-                }
-            });
-    }
-    ~Pool() {
-        stop_ = true;
-        start_.arrive_and_wait();
-        for (auto& x : th_) x.join();
-    }
-    template <class F>
-    void run(size_t smem_floats, F f) {
-        std::vector<float> sm(smem_floats ? smem_floats : 1, NAN);
-        sm_ = sm.data();
-        job_ = f;
-        start_.arrive_and_wait();
-        end_.arrive_and_wait();
-    }
-
-  private:
-    std::barrier<> start_, end_, sync_;
-    std::vector<std::thread> th_;
-    std::function<void(int, float*)> job_;
-    float* sm_ = nullptr;
-    bool stop_ = false;
-};
-
-static Pool* g_pool = nullptr;
+static emu::Pool* g_pool = nullptr;
 
 template <class F>
 static void run_block(size_t smem_floats, F f) {
     g_pool->run(smem_floats, f);
-}
-
-template <class T>
-static std::vector<T> load(const std::string& path, size_t n) {
-    std::vector<T> v(n);
-    FILE* f = fopen(path.c_str(), "rb");
-    if (!f || fread(v.data(), sizeof(T), n, f) != n) {
-        fprintf(stderr, "cannot read %s\n", path.c_str());
-        exit(2);
-    }
-    fclose(f);
-    return v;
-}
-
-static void save(const std::string& path, const float* x, size_t n) {
-    FILE* f = fopen(path.c_str(), "wb");
-    if (!f || fwrite(x, sizeof(float), n, f) != n) {
-        fprintf(stderr, "cannot write %s\n", path.c_str());
-        exit(2);
-    }
-    fclose(f);
 }
 
 int main(int argc, char** argv) {
@@ -124,7 +56,7 @@ int main(int argc, char** argv) {
     std::vector<float> dq((size_t)T * Hqk * kD, NAN), dk((size_t)T * Hqk * kD, NAN), dv((size_t)T * Hv * kD, NAN),
         da((size_t)T * Hv, NAN), db((size_t)T * Hv, NAN), dA_log(Hv, NAN), ddt(Hv, NAN), dinit(st, NAN);
 
-    Pool pool;
+    emu::Pool pool(kThreads);
     g_pool = &pool;
     const Plan plan = make_plan(n_seq, T, Hv);
     std::vector<float> ws(plan.bytes / sizeof(float), NAN);

@@ -31,6 +31,7 @@ def test_header_declares_the_entry_points():
                      "gdn_gated_norm", "gdn_prefill_gated", "gdn_decode_step_gated",
                      "gdn_prefill_backward", "gdn_prefill_backward_workspace_size",
                      "gdn_prefill_backward_chunked", "gdn_prefill_backward_chunked_workspace_size",
+                     "gdn_conv1d_silu_backward", "gdn_conv1d_silu_backward_workspace_size",
                      "gdn_selftest_bounded_wait", "gdn_status_string"):
         assert required in names
 
@@ -252,6 +253,32 @@ def test_chunked_backward_rejects_bad_arguments(L):
     assert call(dA=None) == 1
     assert call(dq=_p(FAKE + 4)) == 3
     assert call(wsb=ws - 256) == 6
+    assert call(wsp=_p(0x20000 + 16)) == 3
+
+
+def test_front_backward_workspace_formula(L):
+    # gdn.h: ceil(T / 32) * Ctot * 4 floats, rounded up to 256 bytes; 0 for T = 0
+    for T, Hqk, Hv in ((8192, 16, 48), (100, 2, 6), (1, 1, 1)):
+        want = -(-T // 32) * (2 * Hqk + Hv) * 128 * 4 * 4
+        assert L.gdn_conv1d_silu_backward_workspace_size(T, Hqk, Hv, 128) == (want + 255) // 256 * 256
+    assert L.gdn_conv1d_silu_backward_workspace_size(0, 16, 48, 128) == 0
+
+
+def test_front_backward_rejects_bad_arguments(L):
+    ws = L.gdn_conv1d_silu_backward_workspace_size(64, 16, 48, 128)
+
+    def call(d=128, w=_p(), dq=_p(), dw=_p(), dx=_p(), wsp=_p(0x20000), wsb=ws, n_seq=1, cu=None):
+        return L.gdn_conv1d_silu_backward(_p(), w, cu, n_seq, 64, 16, 48, d, None, dq, _p(), _p(), dx, dw, None,
+                                          wsp, wsb, None)
+    assert call(d=64) == 2
+    assert call(w=None) == 1
+    assert call(dw=None) == 1
+    assert call(dq=None) == 1
+    assert call(dx=None) == 1
+    assert call(n_seq=2) == 1          # several sequences need cu_seqlens
+    assert call(dx=_p(FAKE + 4)) == 3
+    assert call(wsb=ws - 256) == 6
+    assert call(wsp=None) == 6
     assert call(wsp=_p(0x20000 + 16)) == 3
 
 
