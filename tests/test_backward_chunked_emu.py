@@ -108,3 +108,16 @@ def test_emulated_chunked_backward_two_key_heads(orc, emu, tmp_path):
     d_o, d_fin = _grads(inp, 3)
     got = _run(emu, tmp_path, inp, d_o, d_fin, with_s0=True, with_cu=True)
     _check(orc, got, inp, d_o, d_fin, with_s0=True, with_cu=True)
+
+
+def test_emulated_chunked_backward_strong_decay(orc, emu, tmp_path):
+    # one head decays by ~e^-48 per token, so gam = e^G underflows to zero inside
+    # a chunk; the other is almost undecayed
+    inp = synth.make_prefill([100, 30], seed=93, init_state=True, init_std=0.05, Hqk=1, Hv=2)
+    inp.A_log[0] = np.float32(np.log(16.0))
+    inp.a[:, 0] = 3.0
+    inp.A_log[1] = np.float32(np.log(1.0))
+    inp.dt_bias[1] = np.float32(-9.0)
+    d_o, d_fin = _grads(inp, 4)
+    got = _run(emu, tmp_path, inp, d_o, d_fin, with_s0=True, with_cu=True)
+    _check(orc, got, inp, d_o, d_fin, with_s0=True, with_cu=True)
