@@ -562,7 +562,7 @@ def test_chunked_backward_equals_sequential_backward(orc):
     args = {n: inp[n] for n in ("q", "k", "v", "a", "b", "A_log", "dt_bias")}
     ref = orc.prefill_backward(**args, d_o=d_o, d_final=d_fin, cu_seqlens=inp["cu_seqlens"],
                                initial_state=inp["initial_state"])
-    for C in (1, 2, 3, 8, 16, 64):
+    for C in (1, 2, 3, 8, 16, 64, 128):
         got = orc.prefill_backward_chunked(**args, d_o=d_o, d_final=d_fin, cu_seqlens=inp["cu_seqlens"],
                                            initial_state=inp["initial_state"], C=C)
         for name, x in ref.items():
