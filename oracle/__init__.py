@@ -12,6 +12,7 @@ from .oracle import (  # noqa: F401
     conv1d_silu_f64,
     decode,
     gated_norm,
+    gated_norm_backward,
     log_alpha,
     beta,
     max_threads,

@@ -1081,3 +1081,41 @@ int gdn_oracle_conv1d_silu_backward(const double* x, const double* w, const int3
     }
     return 0;
 }
+
+/*
+ * gdn_oracle_gated_norm_backward -- the gradient of gdn_oracle_gated_norm
+ * (y = w[l] * o * r * silu(z), r = 1 / sqrt(mean(o^2) + eps), l = t % layers)
+ * given dL/dy.  With u = w g dy (g = silu(z)):
+ *     do = r u - (r^3 / d) o <o, u>,
+ *     dz = dy w r o silu'(z),  silu'(z) = sigma(z) (1 + z (1 - sigma(z))),
+ *     dw[l] = sum over the rows of layer l of dy r o g.
+ * Rows are summed in order (t, then h).  Outputs overwritten.
+ */
+int gdn_oracle_gated_norm_backward(const double* o, const double* z, const double* w, int64_t T, int Hv, int d,
+                                   int layers, double eps, const double* dy, double* d_o, double* dz, double* dw) {
+    if (T < 0 || Hv <= 0 || d <= 0 || layers <= 0 || !(eps >= 0.0)) return -1;
+    memset(dw, 0, sizeof(double) * (size_t)layers * d);
+    for (int64_t t = 0; t < T; ++t) {
+        const int l = (int)(t % layers);
+        const double* wl = w + (int64_t)l * d;
+        for (int h = 0; h < Hv; ++h) {
+            const int64_t row = (t * Hv + h) * (int64_t)d;
+            double ss = 0.0, ou = 0.0;
+            for (int e = 0; e < d; ++e) ss += o[row + e] * o[row + e];
+            const double r = 1.0 / sqrt(ss / d + eps);
+            for (int e = 0; e < d; ++e) {
+                const double sg = 1.0 / (1.0 + exp(-z[row + e]));
+                ou += o[row + e] * wl[e] * z[row + e] * sg * dy[row + e];
+            }
+            for (int e = 0; e < d; ++e) {
+                const double sg = 1.0 / (1.0 + exp(-z[row + e]));
+                const double g = z[row + e] * sg;
+                const double u = wl[e] * g * dy[row + e];
+                d_o[row + e] = r * u - r * r * r / d * o[row + e] * ou;
+                dz[row + e] = dy[row + e] * wl[e] * r * o[row + e] * sg * (1.0 + z[row + e] * (1.0 - sg));
+                dw[(int64_t)l * d + e] += dy[row + e] * r * o[row + e] * g;
+            }
+        }
+    }
+    return 0;
+}

@@ -62,6 +62,8 @@ def _bind(lib):
     lib.gdn_oracle_conv1d_silu_backward.restype = C.c_int
     lib.gdn_oracle_conv1d_silu_backward.argtypes = [vp, vp, vp, i32, i64, i32, i32, i32, vp, vp, vp, vp, vp, vp,
                                                     vp, C.c_int]
+    lib.gdn_oracle_gated_norm_backward.restype = C.c_int
+    lib.gdn_oracle_gated_norm_backward.argtypes = [vp, vp, vp, i64, C.c_int, C.c_int, C.c_int, dbl, vp, vp, vp, vp]
     lib.gdn_oracle_max_threads.restype = C.c_int
     lib.gdn_oracle_max_threads.argtypes = [C.c_int]
     return lib
@@ -373,4 +375,26 @@ def conv1d_silu_backward(qkv, conv_w, dq, dk, dv, cu_seqlens=None, Hqk=16, Hv=48
         int(threads))
     if rc != 0:
         raise ValueError("oracle conv1d_silu_backward rejected its arguments")
+    return out
+
+
+def gated_norm_backward(o, z, norm_w, dy, eps=1e-6, lib=None):
+    """Gradient of gated_norm given dL/dy (gdn_oracle_gated_norm_backward).
+    Arguments as for gated_norm; returns a dict with d_o, d_z [T, Hv, d] and
+    d_norm_w [layers, d] (float64)."""
+    o = np.ascontiguousarray(o, dtype=np.float64)
+    z = np.asarray(z)
+    if z.dtype == np.uint16:
+        z = (z.astype(np.uint32) << 16).view(np.float32)
+    z = np.ascontiguousarray(z, dtype=np.float64)
+    w = np.ascontiguousarray(norm_w, dtype=np.float64)
+    if w.ndim == 1:
+        w = w[None, :]
+    T, Hv, d = o.shape
+    out = dict(d_o=np.zeros_like(o), d_z=np.zeros_like(o), d_norm_w=np.zeros_like(w))
+    rc = _L(lib).gdn_oracle_gated_norm_backward(_ptr(o), _ptr(z), _ptr(w), T, Hv, d, w.shape[0], float(eps),
+                                                _ptr(_f64(dy)), _ptr(out["d_o"]), _ptr(out["d_z"]),
+                                                _ptr(out["d_norm_w"]))
+    if rc != 0:
+        raise ValueError("oracle gated_norm_backward rejected its arguments")
     return out

@@ -73,6 +73,11 @@ MUTANTS = {
                                "return cs ? cs[((int64_t)n * Ctot + c) * 3 + (m - 1)] : 0.0;"),
     "f64_front_norm_on_v": ("const double inv = hh < 2 * Hqk ? 1.0 / sqrt(ss + 1e-6) : 1.0;",
                             "const double inv = 1.0 / sqrt(ss + 1e-6);"),
+    "nbw_no_norm_term": ("d_o[row + e] = r * u - r * r * r / d * o[row + e] * ou;", "d_o[row + e] = r * u;"),
+    "nbw_silu_derivative": ("dz[row + e] = dy[row + e] * wl[e] * r * o[row + e] * sg * (1.0 + z[row + e] * (1.0 - sg));",
+                            "dz[row + e] = dy[row + e] * wl[e] * r * o[row + e] * sg;"),
+    "nbw_weight_one_layer": ("dw[(int64_t)l * d + e] += dy[row + e] * r * o[row + e] * g;",
+                             "dw[e] += dy[row + e] * r * o[row + e] * g;"),
 }
 
 

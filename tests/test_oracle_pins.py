@@ -654,3 +654,28 @@ def test_front_backward_without_history_and_one_sequence(orc):
     g0 = orc.conv1d_silu_backward(c["qkv"], c["conv_w"], gq, gk, gv, None, 1, 1, 4, np.zeros((1, 12, 3)))
     assert np.array_equal(g["d_conv_state"], g0["d_conv_state"])
     assert np.array_equal(g["d_qkv"], g0["d_qkv"])
+
+
+def test_gated_norm_backward_matches_finite_differences(orc):
+    # two layers, so that the weight gradient's rows collect the right tokens
+    rng = np.random.default_rng(21)
+    T, Hv, d, layers = 5, 2, 6, 2
+    o = rng.standard_normal((T, Hv, d))
+    z = rng.standard_normal((T, Hv, d))
+    w = rng.standard_normal((layers, d))
+    dy = rng.standard_normal((T, Hv, d))
+    g = orc.gated_norm_backward(o, z, w, dy, eps=1e-3)
+    h = 1e-6
+    for name, base, gname in (("o", o, "d_o"), ("z", z, "d_z"), ("w", w, "d_norm_w")):
+        fd = np.zeros_like(base)
+        for idx in np.ndindex(base.shape):
+            xp, xm = base.copy(), base.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = dict(o=o, z=z, norm_w=w)
+            args_m = dict(o=o, z=z, norm_w=w)
+            key = {"o": "o", "z": "z", "w": "norm_w"}[name]
+            args_p[key], args_m[key] = xp, xm
+            fd[idx] = (np.sum(dy * orc.gated_norm(eps=1e-3, **args_p))
+                       - np.sum(dy * orc.gated_norm(eps=1e-3, **args_m))) / (2 * h)
+        assert np.max(np.abs(g[gname] - fd)) <= 2e-7 * max(1.0, np.max(np.abs(fd))), gname
