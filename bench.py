@@ -11,8 +11,8 @@ T = 262144 prefill (non-zero initial state), the 16-sequence varlen prefill
 T = 8192, and one decode step over 128 sequences x 48 layers with the 19.3 GB
 float32 state updated in place (plain, with the front end fused, with a bf16
 state, and with the gated norm fused); last, at N = 1 only, the backward pass
-through the chunked form and the front end's backward at T = 8192 (an error
-there is recorded in its entry).
+through the chunked form, the front end's backward and the gated norm's
+backward at T = 8192 (an error there is recorded in its entry).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -320,6 +320,10 @@ def bench_main(args, world, rank, local):
                 extra["front_backward_T8192"] = bench_front_backward(args, dev, flush, peaks, world)
             except Exception as exc:     # noqa: BLE001
                 extra["front_backward_T8192"] = {"error": str(exc)[:300]}
+            try:
+                extra["gated_norm_backward_T8192"] = bench_norm_backward(args, dev, flush, peaks, world)
+            except Exception as exc:     # noqa: BLE001
+                extra["gated_norm_backward_T8192"] = {"error": str(exc)[:300]}
 
     value = weak_scaling_rate(T, ms_max, world)
     line = {
@@ -638,6 +642,42 @@ def bench_front_backward(args, dev, flush, peaks, world):
            "ms": round(ms, 4), "GB_s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
            "bytes_per_step": nbytes, "launches_per_step": 2}
     del qkv, dq, dk, dv, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def bench_norm_backward(args, dev, flush, peaks, world):
+    """gdn_gated_norm_backward at T = 8192 x 48 heads, one layer: d o, d z and
+    d norm_w.  Algorithmic bytes per (token, head): o, dy float32 and z bf16
+    read, d o and d z float32 written (4 + 4 + 2 + 4 + 4 bytes per element)."""
+    import torch
+    import gated_deltanet_recurrence_prefill_b200 as gdn
+    T = T_MAIN
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(10)
+    o = torch.randn(T, HV, D, generator=gen, device=dev)
+    z = torch.randn(T, HV, D, generator=gen, device=dev).to(torch.bfloat16)
+    w = 1.0 + 0.1 * torch.randn(1, D, generator=gen, device=dev)
+    dy = torch.randn(T, HV, D, generator=gen, device=dev)
+    ws = torch.empty(gdn.lib().gdn_gated_norm_backward_workspace_size(T, HV, D, 1), dtype=torch.uint8, device=dev)
+
+    def step(ev):
+        if ev:
+            ev["start"].record()
+        gdn.gated_norm_backward(o, z, w, dy, workspace=ws)
+        if ev:
+            ev["end"].record()
+
+    mk = lambda: {"start": torch.cuda.Event(enable_timing=True),
+                  "end": torch.cuda.Event(enable_timing=True)}
+    times, _ = _time_steps(step, 3, 5, flush, mk, world)
+    ms = _max_over_ranks(sum(times) / len(times), world)
+    nbytes = T * HV * D * (4 + 4 + 2 + 4 + 4)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    out = {"workload": f"gdn_gated_norm_backward T={T} Hv=48 d=128, one layer",
+           "ms": round(ms, 4), "GB_s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+           "bytes_per_step": nbytes, "launches_per_step": 3}
+    del o, z, dy, ws
     torch.cuda.empty_cache()
     return out
 

@@ -14,6 +14,7 @@ from ._lib import (  # noqa: F401
     decode_step_fused,
     decode_step_gated,
     gated_norm,
+    gated_norm_backward,
     lib,
     lib_path,
     prefill,

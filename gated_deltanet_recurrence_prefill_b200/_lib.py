@@ -47,6 +47,9 @@ SIGNATURES = {
     "gdn_prefill_backward": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
                                        _i32, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                        _vp, _vp, _sz, _vp]),
+    "gdn_gated_norm_backward_workspace_size": (_sz, [_i64, _i32, _i32, _i32]),
+    "gdn_gated_norm_backward": (C.c_int, [_vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _f32, _vp, _vp, _vp,
+                                          _vp, _sz, _vp]),
     "gdn_conv1d_silu_backward_workspace_size": (_sz, [_i64, _i32, _i32, _i32]),
     "gdn_conv1d_silu_backward": (C.c_int, [_vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _vp,
                                            _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -181,6 +184,35 @@ def conv1d_silu_backward(qkv, conv_w, dq, dk, dv, Hqk, Hv, d=128, cu_seqlens=Non
         _ptr(dv), _ptr(out["d_qkv"]), _ptr(out["d_conv_w"]), _ptr(out["d_conv_state"]), _ptr(workspace),
         0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream))
     _check("gdn_conv1d_silu_backward", st)
+    return out
+
+
+def gated_norm_backward(o, z, norm_w, dy, eps=1e-6, workspace=None, stream=None):
+    """gdn_gated_norm_backward: the gated norm's gradient given dL/dy [T, Hv, d]
+    (float32).  o [T, Hv, d] float32, z [T, Hv, d] bf16, norm_w [layers, d] or
+    [d] float32.  Returns a dict of float32 tensors d_o, d_z [T, Hv, d] and
+    d_norm_w (shaped as norm_w)."""
+    import torch
+    T, Hv, d = o.shape
+    w2 = norm_w if norm_w.dim() == 2 else norm_w.view(1, -1)
+    layers = w2.shape[0]
+    _need(o, torch.float32, (T, Hv, d), "o")
+    _need(z, torch.bfloat16, (T, Hv, d), "z")
+    _need(w2, torch.float32, (layers, d), "norm_w")
+    _need(dy, torch.float32, (T, Hv, d), "dy")
+    dev = o.device
+    out = dict(d_o=torch.empty_like(o), d_z=torch.empty(T, Hv, d, dtype=torch.float32, device=dev),
+               d_norm_w=torch.empty(layers, d, dtype=torch.float32, device=dev))
+    ws_bytes = int(lib().gdn_gated_norm_backward_workspace_size(T, Hv, d, layers))
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    st = lib().gdn_gated_norm_backward(
+        _ptr(o), _ptr(z), _ptr(w2), _ptr(dy), T, Hv, d, layers, float(eps), _ptr(out["d_o"]), _ptr(out["d_z"]),
+        _ptr(out["d_norm_w"]), _ptr(workspace),
+        0 if workspace is None else workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("gdn_gated_norm_backward", st)
+    if norm_w.dim() == 1:
+        out["d_norm_w"] = out["d_norm_w"].view(-1)
     return out
 
 

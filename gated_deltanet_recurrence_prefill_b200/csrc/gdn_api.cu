@@ -424,6 +424,31 @@ gdn_status gdn_selftest_bounded_wait(int32_t which, int64_t limit_us, void* work
     return e == cudaSuccess ? GDN_OK : cuda_fail(e);
 }
 
+size_t gdn_gated_norm_backward_workspace_size(int64_t T, int32_t Hv, int32_t d, int32_t layers) {
+    (void)d;
+    if (T <= 0 || Hv <= 0 || layers <= 0) return 0;
+    return gdn::gated_norm_backward_workspace_bytes(T, Hv, layers);
+}
+
+gdn_status gdn_gated_norm_backward(const float* o, const uint16_t* z, const float* norm_w, const float* dy,
+                                   int64_t T, int32_t Hv, int32_t d, int32_t layers, float eps, float* d_o,
+                                   float* d_z, float* d_norm_w, void* workspace, size_t workspace_bytes,
+                                   gdn_stream_t stream) {
+    if (T < 0 || Hv <= 0 || d <= 0 || layers <= 0 || !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;
+    if (d != kD) return GDN_ERR_UNSUPPORTED;
+    if (T > (int64_t)0x7fffffff) return GDN_ERR_UNSUPPORTED;
+    if (!norm_w || !d_norm_w || (T > 0 && (!o || !z || !dy || !d_o || !d_z))) return GDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {o, z, norm_w, dy, d_o, d_z, d_norm_w};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
+    const size_t need = T > 0 ? gdn::gated_norm_backward_workspace_bytes(T, Hv, layers) : 0;
+    if (need > 0 && (!workspace || workspace_bytes < need)) return GDN_ERR_WORKSPACE;
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_MISALIGNED;
+    cudaError_t e = gdn::launch_gated_norm_backward(o, z, norm_w, dy, T, Hv, layers, eps, d_o, d_z, d_norm_w,
+                                                    workspace, (cudaStream_t)stream);
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
 gdn_status gdn_gated_norm(const float* o, const uint16_t* z, const float* norm_w, int64_t T, int32_t Hv,
                           int32_t d, int32_t layers, float eps, uint16_t* y, gdn_stream_t stream) {
     if (T < 0 || Hv <= 0 || d <= 0 || layers <= 0 || !(eps >= 0.f)) return GDN_ERR_INVALID_ARG;

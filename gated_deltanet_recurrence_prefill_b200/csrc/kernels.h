@@ -126,6 +126,11 @@ struct ConvBackwardArgs {
     void* workspace;
 };
 size_t conv1d_silu_backward_workspace_bytes(int64_t T, int32_t Hqk, int32_t Hv);
+// the gated output norm's gradient (gated_norm_backward.cu)
+size_t gated_norm_backward_workspace_bytes(int64_t T, int32_t Hv, int32_t layers);
+cudaError_t launch_gated_norm_backward(const float* o, const uint16_t* z, const float* w, const float* dy,
+                                       int64_t T, int32_t Hv, int32_t layers, float eps, float* d_o, float* d_z,
+                                       float* d_w, void* workspace, cudaStream_t stream);
 cudaError_t launch_conv1d_silu_backward(const ConvBackwardArgs& a, cudaStream_t stream);
 cudaError_t launch_backward_chunked(const BackwardArgs& a, cudaStream_t stream);
 

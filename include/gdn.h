@@ -426,6 +426,35 @@ gdn_status gdn_prefill_backward_chunked(const uint16_t* q, const uint16_t* k, co
                                         gdn_stream_t stream);
 
 /*
+ * gdn_gated_norm_backward_workspace_size -- bytes of device workspace
+ * gdn_gated_norm_backward needs: per-tile partial sums of the weight gradient
+ * (ceil(T / 8) * ceil(Hv / 8) * 8 * d floats) and per-chunk sums
+ * (layers * ceil(ceil(T / layers) / 64) * d floats), each rounded up to 256
+ * bytes; 0 for T = 0.  Host-only.
+ */
+size_t gdn_gated_norm_backward_workspace_size(int64_t T, int32_t Hv, int32_t d, int32_t layers);
+
+/*
+ * gdn_gated_norm_backward -- the gradient of gdn_gated_norm
+ *     y = norm_w[l] * o * r * silu(z),  r = 1 / sqrt(mean_v o^2 + eps),  l = t % layers
+ * given dL/dy (the same reading of the architecture page, section 2.1):
+ *     d_o = r u - (r^3 / d) o <o, u>  with u = norm_w silu(z) dy,
+ *     d_z = dy norm_w r o sigma(z) (1 + z (1 - sigma(z))),
+ *     d_norm_w[l] = sum over the rows of layer l of dy r o silu(z).
+ *  o, z, norm_w, T, Hv, d, layers, eps as for gdn_gated_norm;
+ *  dy          [T, Hv, d] float32.
+ * Outputs (float32, overwritten; caller-owned): d_o, d_z [T, Hv, d],
+ * d_norm_w [layers, d].  workspace: gdn_gated_norm_backward_workspace_size()
+ * bytes, 256-byte aligned (may be NULL when that is 0).  Supported: d = 128.
+ * CUDA cores, float32, sums in a fixed order (deterministic).  Errors as for
+ * gdn_gated_norm, plus GDN_ERR_WORKSPACE.
+ */
+gdn_status gdn_gated_norm_backward(const float* o, const uint16_t* z, const float* norm_w, const float* dy,
+                                   int64_t T, int32_t Hv, int32_t d, int32_t layers, float eps, float* d_o,
+                                   float* d_z, float* d_norm_w, void* workspace, size_t workspace_bytes,
+                                   gdn_stream_t stream);
+
+/*
  * gdn_selftest_bounded_wait -- failure detection check.  Runs, in one small
  * kernel, one of the bounded waits the prefill's CTAs use, on something that
  * never happens: which = 0 waits for a counter in global memory (as on the

@@ -32,6 +32,7 @@ def test_header_declares_the_entry_points():
                      "gdn_prefill_backward", "gdn_prefill_backward_workspace_size",
                      "gdn_prefill_backward_chunked", "gdn_prefill_backward_chunked_workspace_size",
                      "gdn_conv1d_silu_backward", "gdn_conv1d_silu_backward_workspace_size",
+                     "gdn_gated_norm_backward", "gdn_gated_norm_backward_workspace_size",
                      "gdn_selftest_bounded_wait", "gdn_status_string"):
         assert required in names
 
@@ -279,6 +280,33 @@ def test_front_backward_rejects_bad_arguments(L):
     assert call(dx=_p(FAKE + 4)) == 3
     assert call(wsb=ws - 256) == 6
     assert call(wsp=None) == 6
+    assert call(wsp=_p(0x20000 + 16)) == 3
+
+
+def test_norm_backward_workspace_formula(L):
+    # gdn.h: per-tile partials ceil(T/8) * ceil(Hv/8) * 8 * d and per-chunk sums
+    # layers * ceil(ceil(T/layers)/64) * d floats, each rounded to 256 bytes
+    r = lambda x: (x + 255) // 256 * 256
+    for T, Hv, layers in ((8192, 48, 1), (6144, 48, 48), (100, 6, 3)):
+        want = r(-(-T // 8) * -(-Hv // 8) * 8 * 128 * 4) + r(layers * -(-(-(-T // layers)) // 64) * 128 * 4)
+        assert L.gdn_gated_norm_backward_workspace_size(T, Hv, 128, layers) == want
+    assert L.gdn_gated_norm_backward_workspace_size(0, 48, 128, 1) == 0
+
+
+def test_norm_backward_rejects_bad_arguments(L):
+    ws = L.gdn_gated_norm_backward_workspace_size(64, 48, 128, 1)
+
+    def call(d=128, layers=1, eps=1e-6, o=_p(), dy=_p(), dw=_p(), wsp=_p(0x20000), wsb=ws):
+        return L.gdn_gated_norm_backward(o, _p(), _p(), dy, 64, 48, d, layers, eps, _p(), _p(), dw, wsp, wsb,
+                                         None)
+    assert call(d=64) == 2
+    assert call(layers=0) == 1
+    assert call(eps=-1.0) == 1
+    assert call(o=None) == 1
+    assert call(dy=None) == 1
+    assert call(dw=None) == 1
+    assert call(o=_p(FAKE + 4)) == 3
+    assert call(wsb=ws - 256) == 6
     assert call(wsp=_p(0x20000 + 16)) == 3
 
 
