@@ -152,12 +152,28 @@ def conv1d_silu(qkv, conv_w, Hqk, Hv, d=128, cu_seqlens=None, conv_state_in=None
     return q, k, v
 
 
+def _outputs(given, shapes, dev):
+    """float32 output tensors of the given shapes (None: not wanted), taken from
+    the caller's dict `given` where it has them (checked), else allocated."""
+    import torch
+    out = {}
+    for name, shape in shapes.items():
+        if shape is None:
+            out[name] = None
+        elif given is not None and given.get(name) is not None:
+            _need(given[name], torch.float32, shape, name)
+            out[name] = given[name]
+        else:
+            out[name] = torch.empty(*shape, dtype=torch.float32, device=dev)
+    return out
+
+
 def conv1d_silu_backward(qkv, conv_w, dq, dk, dv, Hqk, Hv, d=128, cu_seqlens=None, conv_state=None,
-                         want_d_conv_state=True, workspace=None, stream=None):
+                         want_d_conv_state=True, workspace=None, stream=None, out=None):
     """gdn_conv1d_silu_backward: the front end's gradient given dL/dq, dL/dk
     [T, Hqk, d] and dL/dv [T, Hv, d] (float32).  Returns a dict of float32
     tensors d_qkv [T, Ctot], d_conv_w [Ctot, 4] and d_conv_state [N, Ctot, 3]
-    (or None)."""
+    (or None).  out: an optional dict of preallocated tensors under those names."""
     import torch
     T = qkv.shape[0]
     ctot = (2 * Hqk + Hv) * d
@@ -172,10 +188,8 @@ def conv1d_silu_backward(qkv, conv_w, dq, dk, dv, Hqk, Hv, d=128, cu_seqlens=Non
     if conv_state is not None:
         _need(conv_state, torch.float32, (n_seq, ctot, 3), "conv_state")
     dev = qkv.device
-    out = dict(d_qkv=torch.empty(T, ctot, dtype=torch.float32, device=dev),
-               d_conv_w=torch.empty(ctot, 4, dtype=torch.float32, device=dev),
-               d_conv_state=torch.empty(n_seq, ctot, 3, dtype=torch.float32, device=dev)
-               if want_d_conv_state else None)
+    out = _outputs(out, dict(d_qkv=(T, ctot), d_conv_w=(ctot, 4),
+                             d_conv_state=(n_seq, ctot, 3) if want_d_conv_state else None), dev)
     ws_bytes = int(lib().gdn_conv1d_silu_backward_workspace_size(T, Hqk, Hv, d))
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
@@ -187,11 +201,12 @@ def conv1d_silu_backward(qkv, conv_w, dq, dk, dv, Hqk, Hv, d=128, cu_seqlens=Non
     return out
 
 
-def gated_norm_backward(o, z, norm_w, dy, eps=1e-6, workspace=None, stream=None):
+def gated_norm_backward(o, z, norm_w, dy, eps=1e-6, workspace=None, stream=None, out=None):
     """gdn_gated_norm_backward: the gated norm's gradient given dL/dy [T, Hv, d]
     (float32).  o [T, Hv, d] float32, z [T, Hv, d] bf16, norm_w [layers, d] or
     [d] float32.  Returns a dict of float32 tensors d_o, d_z [T, Hv, d] and
-    d_norm_w (shaped as norm_w)."""
+    d_norm_w (shaped as norm_w).  out: an optional dict of preallocated tensors
+    under those names (d_norm_w as [layers, d])."""
     import torch
     T, Hv, d = o.shape
     w2 = norm_w if norm_w.dim() == 2 else norm_w.view(1, -1)
@@ -201,8 +216,7 @@ def gated_norm_backward(o, z, norm_w, dy, eps=1e-6, workspace=None, stream=None)
     _need(w2, torch.float32, (layers, d), "norm_w")
     _need(dy, torch.float32, (T, Hv, d), "dy")
     dev = o.device
-    out = dict(d_o=torch.empty_like(o), d_z=torch.empty(T, Hv, d, dtype=torch.float32, device=dev),
-               d_norm_w=torch.empty(layers, d, dtype=torch.float32, device=dev))
+    out = _outputs(out, dict(d_o=(T, Hv, d), d_z=(T, Hv, d), d_norm_w=(layers, d)), dev)
     ws_bytes = int(lib().gdn_gated_norm_backward_workspace_size(T, Hv, d, layers))
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
@@ -459,26 +473,28 @@ def decode_step_gated(q, k, v, a, b, A_log, dt_bias, state, n_seq, layers, z, no
 
 
 def prefill_backward(q, k, v, a, b, A_log, dt_bias, d_o, d_final_state=None, cu_seqlens=None,
-                     scale=None, initial_state=None, want_d_initial=True, workspace=None, stream=None):
+                     scale=None, initial_state=None, want_d_initial=True, workspace=None, stream=None, out=None):
     """gdn_prefill_backward: gradients of a loss with dL/do = d_o [T, Hv, d] and
     dL/dS_T = d_final_state [N, Hv, d, d] (or zero).  Returns a dict of float32
     tensors dq, dk [T, Hqk, d], dv [T, Hv, d], da, db [T, Hv], dA_log,
-    ddt_bias [Hv] and d_initial_state [N, Hv, d, d] (or None)."""
+    ddt_bias [Hv] and d_initial_state [N, Hv, d, d] (or None).  out: an optional
+    dict of preallocated tensors under those names (float32, contiguous)."""
     return _backward("gdn_prefill_backward", q, k, v, a, b, A_log, dt_bias, d_o, d_final_state, cu_seqlens,
-                     scale, initial_state, want_d_initial, workspace, stream)
+                     scale, initial_state, want_d_initial, workspace, stream, out)
 
 
 def prefill_backward_chunked(q, k, v, a, b, A_log, dt_bias, d_o, d_final_state=None, cu_seqlens=None,
-                             scale=None, initial_state=None, want_d_initial=True, workspace=None, stream=None):
+                             scale=None, initial_state=None, want_d_initial=True, workspace=None, stream=None,
+                             out=None):
     """gdn_prefill_backward_chunked: the same gradients through the chunked
     form (two chains over 64-token chunks, the rest chunk-parallel).  Arguments
     and result as for prefill_backward."""
     return _backward("gdn_prefill_backward_chunked", q, k, v, a, b, A_log, dt_bias, d_o, d_final_state,
-                     cu_seqlens, scale, initial_state, want_d_initial, workspace, stream)
+                     cu_seqlens, scale, initial_state, want_d_initial, workspace, stream, out)
 
 
 def _backward(entry, q, k, v, a, b, A_log, dt_bias, d_o, d_final_state, cu_seqlens, scale, initial_state,
-              want_d_initial, workspace, stream):
+              want_d_initial, workspace, stream, given=None):
     import torch
     T, Hqk, d = q.shape
     Hv = v.shape[1]
@@ -500,10 +516,9 @@ def _backward(entry, q, k, v, a, b, A_log, dt_bias, d_o, d_final_state, cu_seqle
     if scale is None:
         scale = d ** -0.5
     dev = q.device
-    f = lambda *shape: torch.empty(*shape, dtype=torch.float32, device=dev)
-    out = dict(dq=f(T, Hqk, d), dk=f(T, Hqk, d), dv=f(T, Hv, d), da=f(T, Hv), db=f(T, Hv),
-               dA_log=f(Hv), ddt_bias=f(Hv),
-               d_initial_state=f(n_seq, Hv, d, d) if want_d_initial else None)
+    shapes = dict(dq=(T, Hqk, d), dk=(T, Hqk, d), dv=(T, Hv, d), da=(T, Hv), db=(T, Hv), dA_log=(Hv,),
+                  ddt_bias=(Hv,), d_initial_state=(n_seq, Hv, d, d) if want_d_initial else None)
+    out = _outputs(given, shapes, dev)
     ws_bytes = getattr(lib(), entry + "_workspace_size")(n_seq, T, Hv, d)
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
