@@ -8,7 +8,7 @@ namespace {
 
 using namespace nbw;
 
-__global__ void __launch_bounds__(kThreads) nbw_rows_kernel(Params p, int ng) {
+__global__ void __launch_bounds__(kRowThreads) nbw_rows_kernel(Params p, int ng) {
     __shared__ float smem[kRowsFloats];
     rows_block(p, blockIdx.x / ng, blockIdx.x % ng, threadIdx.x, smem);
 }
@@ -41,7 +41,7 @@ cudaError_t launch_gated_norm_backward(const float* o, const uint16_t* z, const 
     const int64_t nc = n_chunks(T, layers);
     const int64_t rows_blocks = n_tiles(T) * ng, chunk_blocks = (int64_t)layers * nc;
     if (rows_blocks > 0x7fffffff || chunk_blocks > 0x7fffffff) return cudaErrorInvalidValue;
-    nbw_rows_kernel<<<(unsigned)rows_blocks, kThreads, 0, s>>>(p, ng);
+    nbw_rows_kernel<<<(unsigned)rows_blocks, kRowThreads, 0, s>>>(p, ng);
     cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) {
         nbw_chunk_kernel<<<(unsigned)chunk_blocks, kThreads, 0, s>>>(p, nc);

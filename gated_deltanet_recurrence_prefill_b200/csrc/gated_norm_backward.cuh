@@ -7,11 +7,13 @@
 //     do = r u - (r^3 / d) o <o, u>,
 //     dz = dy w r o sigma(z) (1 + z (1 - sigma(z))),
 //     dw[l] = sum over the rows of layer l of dy r o g.
-// Three block functions: rows (a CTA of 128 threads, one per element, over 8
-// tokens x 8 heads, keeping the weight gradient of each token of its tile), a
-// sum over chunks of 64 of each layer's tokens, and a sum over those chunks --
-// every sum in a fixed order.  As in backward_chunked.cuh, the CUDA kernels
-// and the CPU tests' emulation run the same source.
+// Three block functions: rows (a CTA of 8 warps over 8 tokens x 8 heads: warp
+// w takes head h0 + w for the 8 tokens, a lane 4 elements of each row, the
+// row sums by warp shuffles; the weight gradient of each token of the tile is
+// then summed over the warps in order), a sum over chunks of 64 of each
+// layer's tokens, and a sum over those chunks -- every sum in a fixed order.
+// As in backward_chunked.cuh, the CUDA kernels and the CPU tests' emulation
+// run the same source (shuffles included).
 #pragma once
 
 #include <math.h>
@@ -27,16 +29,20 @@
 #ifndef BWC_SYNC
 #define BWC_SYNC() __syncthreads()
 #endif
+#ifndef BWC_SHFL_XOR
+#define BWC_SHFL_XOR(v, m) __shfl_xor_sync(0xffffffffu, (v), (m))
+#endif
 
 namespace gdn {
 namespace nbw {
 
 constexpr int kD = 128;
-constexpr int kThreads = 128;            // one thread per element of a row
+constexpr int kThreads = 128;            // the sums: one thread per element
+constexpr int kRowThreads = 256;         // rows: 8 warps, one head each
 constexpr int kTok = 8;                  // tokens per rows job
-constexpr int kHeads = 8;                // heads per rows job
+constexpr int kHeads = kRowThreads / 32; // heads per rows job
 constexpr int kChunk = 64;               // tokens of one layer per first-stage sum
-constexpr int kRowsFloats = 2 * kD + 2 * 8;
+constexpr int kRowsFloats = kHeads * kTok * kD;
 
 struct Params {
     const float* o;             // [T, Hv, 128]
@@ -73,50 +79,51 @@ BWC_FN float bf16f(uint16_t h) {
 }
 
 BWC_FN void rows_block(const Params& p, int64_t tile, int hg, int tid, float* sm) {
-    float* red = sm;                  // [2][128]: o^2 and o u of this thread's element
-    float* part = red + 2 * kD;       // [2][8]: sums of 16 elements each
-    const int e = tid;
-    const int h0 = hg * kHeads;
-    const int h1 = (h0 + kHeads) < p.Hv ? h0 + kHeads : p.Hv;
-    float acc[kTok];
-    for (int j = 0; j < kTok; ++j) {
-        acc[j] = 0.f;
-        const int64_t t = tile * kTok + j;
-        if (t >= p.T) continue;                           // the same for every thread
-        const float w = p.w[(int64_t)(t % p.layers) * kD + e];
-        for (int h = h0; h < h1; ++h) {
-            const int64_t row = (t * p.Hv + h) * kD;
-            const float o = p.o[row + e], z = bf16f(p.z[row + e]), dy = p.dy[row + e];
-            const float sg = 1.f / (1.f + expf(-z));
-            const float g = z * sg;
-            const float u = w * g * dy;
-            red[e] = o * o;
-            red[kD + e] = o * u;
-            BWC_SYNC();
-            if (tid < 8) {
-                float s0 = 0.f, s1 = 0.f;
-                for (int i = 0; i < 16; ++i) {
-                    s0 += red[16 * tid + i];
-                    s1 += red[kD + 16 * tid + i];
-                }
-                part[tid] = s0;
-                part[8 + tid] = s1;
-            }
-            BWC_SYNC();
+    float* red = sm;                  // [warp][token][element]: each warp's weight gradient
+    const int warp = tid >> 5, lane = tid & 31;
+    const int h = hg * kHeads + warp;
+    float acc[kTok][4];
+    for (int j = 0; j < kTok; ++j)
+        for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
+    if (h < p.Hv) {                                       // the same for every lane of the warp
+        for (int j = 0; j < kTok; ++j) {
+            const int64_t t = tile * kTok + j;
+            if (t >= p.T) break;
+            const int64_t row = (t * p.Hv + h) * kD + lane * 4;
+            const float* wl = p.w + (int64_t)(t % p.layers) * kD + lane * 4;
+            float o[4], z[4], dy[4], w[4], sg[4], u[4];
             float ss = 0.f, ou = 0.f;
-            for (int i = 0; i < 8; ++i) {
-                ss += part[i];
-                ou += part[8 + i];
+            for (int i = 0; i < 4; ++i) {
+                o[i] = p.o[row + i];
+                z[i] = bf16f(p.z[row + i]);
+                dy[i] = p.dy[row + i];
+                w[i] = wl[i];
+                sg[i] = 1.f / (1.f + expf(-z[i]));
+                u[i] = w[i] * z[i] * sg[i] * dy[i];
+                ss = fmaf(o[i], o[i], ss);
+                ou = fmaf(o[i], u[i], ou);
+            }
+            for (int m = 16; m >= 1; m >>= 1) {
+                ss += BWC_SHFL_XOR(ss, m);
+                ou += BWC_SHFL_XOR(ou, m);
             }
             const float r = 1.f / sqrtf(ss / kD + p.eps);
-            p.d_o[row + e] = r * u - r * r * r / kD * o * ou;
-            p.d_z[row + e] = dy * w * r * o * sg * (1.f + z * (1.f - sg));
-            acc[j] = fmaf(dy * r, o * g, acc[j]);
-            BWC_SYNC();
+            for (int i = 0; i < 4; ++i) {
+                p.d_o[row + i] = r * u[i] - r * r * r / kD * o[i] * ou;
+                p.d_z[row + i] = dy[i] * w[i] * r * o[i] * sg[i] * (1.f + z[i] * (1.f - sg[i]));
+                acc[j][i] = dy[i] * r * o[i] * (z[i] * sg[i]);
+            }
         }
     }
+    for (int j = 0; j < kTok; ++j)
+        for (int i = 0; i < 4; ++i) red[(warp * kTok + j) * kD + lane * 4 + i] = acc[j][i];
+    BWC_SYNC();
     const int ng = n_groups(p.Hv);
-    for (int j = 0; j < kTok; ++j) p.part1[((tile * ng + hg) * kTok + j) * kD + e] = acc[j];
+    for (int x = tid; x < kTok * kD; x += kRowThreads) {
+        float s = 0.f;
+        for (int w = 0; w < kHeads; ++w) s += red[w * kTok * kD + x];
+        p.part1[(tile * ng + hg) * kTok * kD + x] = s;
+    }
 }
 
 // first stage: tokens l + layers m, m in [kChunk k, kChunk (k + 1)), all head groups

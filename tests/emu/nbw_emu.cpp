@@ -12,6 +12,7 @@
 #define BWC_FN inline
 #define BWC_HD inline
 #define BWC_SYNC() ::emu::g_bar->arrive_and_wait()
+#define BWC_SHFL_XOR(v, m) ::emu::shfl_xor((v), (m))
 #include "../../gated_deltanet_recurrence_prefill_b200/csrc/gated_norm_backward.cuh"
 
 using namespace gdn::nbw;
@@ -39,13 +40,16 @@ int main(int argc, char** argv) {
     p.o = o.data(); p.z = z.data(); p.w = w.data(); p.dy = dy.data(); p.T = T; p.Hv = Hv; p.layers = layers;
     p.eps = eps; p.d_o = d_o.data(); p.d_z = d_z.data(); p.dw = dw.data(); p.part1 = p1.data(); p.part2 = p2.data();
 
+    emu::Pool rows_pool(kRowThreads);
+    if (T > 0) {
+        const int ng = n_groups(Hv);
+        for (int64_t b = 0; b < n_tiles(T) * ng; ++b)
+            rows_pool.run(kRowsFloats, [&](int tid, float* sm) { rows_block(p, b / ng, (int)(b % ng), tid, sm); });
+    }
     emu::Pool pool(kThreads);
     if (T == 0) {
         std::fill(dw.begin(), dw.end(), 0.f);
     } else {
-        const int ng = n_groups(Hv);
-        for (int64_t b = 0; b < n_tiles(T) * ng; ++b)
-            pool.run(kRowsFloats, [&](int tid, float* sm) { rows_block(p, b / ng, (int)(b % ng), tid, sm); });
         const int64_t nc = n_chunks(T, layers);
         for (int64_t b = 0; b < (int64_t)layers * nc; ++b)
             pool.run(0, [&](int tid, float*) { sum_chunk_block(p, (int)(b / nc), b % nc, tid); });
