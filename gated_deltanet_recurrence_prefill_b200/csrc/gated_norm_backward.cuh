@@ -83,12 +83,15 @@ BWC_FN void rows_block(const Params& p, int64_t tile, int hg, int tid, float* sm
     const int warp = tid >> 5, lane = tid & 31;
     const int h = hg * kHeads + warp;
     float acc[kTok][4];
+#pragma unroll
     for (int j = 0; j < kTok; ++j)
+#pragma unroll
         for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
     if (h < p.Hv) {                                       // the same for every lane of the warp
+#pragma unroll
         for (int j = 0; j < kTok; ++j) {
             const int64_t t = tile * kTok + j;
-            if (t >= p.T) break;
+            if (t >= p.T) continue;                       // the same for every lane
             const int64_t row = (t * p.Hv + h) * kD + lane * 4;
             const float* wl = p.w + (int64_t)(t % p.layers) * kD + lane * 4;
             float o[4], z[4], dy[4], w[4], sg[4], u[4];
@@ -115,7 +118,9 @@ BWC_FN void rows_block(const Params& p, int64_t tile, int hg, int tid, float* sm
             }
         }
     }
+#pragma unroll
     for (int j = 0; j < kTok; ++j)
+#pragma unroll
         for (int i = 0; i < 4; ++i) red[(warp * kTok + j) * kD + lane * 4 + i] = acc[j][i];
     BWC_SYNC();
     const int ng = n_groups(p.Hv);
