@@ -19,7 +19,7 @@
 // history gradient of a sequence is written by the job whose tile holds the
 // sequence's first token.  Block functions as in backward_chunked.cuh: the
 // CUDA kernels and the CPU tests' emulation run the same source; threads meet
-// only at block barriers, sums have a fixed order.
+// at block barriers and in warp shuffles, and every sum has a fixed order.
 #pragma once
 
 #include <math.h>
@@ -34,6 +34,9 @@
 #endif
 #ifndef BWC_SYNC
 #define BWC_SYNC() __syncthreads()
+#endif
+#ifndef BWC_SHFL_XOR
+#define BWC_SHFL_XOR(v, m) __shfl_xor_sync(0xffffffffu, (v), (m))
 #endif
 
 namespace gdn {
@@ -134,16 +137,27 @@ BWC_FN void tile_block(const Params& p, int64_t tile, int hh, int tid, float* sm
         gs[tau * kLd + tid] = dsrc[t * dstride + tid];
     }
     BWC_SYNC();
-    if (tid < ntok) {
-        float ss = 0.f, gd = 0.f;
-        for (int e = 0; e < kD; ++e) {
-            const float a = as[tid * kLd + e];
-            ss = fmaf(a, a, ss);
-            gd = fmaf(gs[tid * kLd + e], a, gd);
+    // per token: the norm and <dout, out> / n, one warp per token (a lane sums 4
+    // channels, then 5 xor shuffles)
+    {
+        const int warp = tid >> 5, lane = tid & 31;
+        for (int tau = warp; tau < ntok; tau += kThreads / 32) {
+            float ss = 0.f, gd = 0.f;
+            for (int x = 0; x < kD / 32; ++x) {
+                const float a = as[tau * kLd + lane + 32 * x];
+                ss = fmaf(a, a, ss);
+                gd = fmaf(gs[tau * kLd + lane + 32 * x], a, gd);
+            }
+            for (int m = 16; m >= 1; m >>= 1) {
+                ss += BWC_SHFL_XOR(ss, m);
+                gd += BWC_SHFL_XOR(gd, m);
+            }
+            if (lane == 0) {
+                const float nv = normed ? sqrtf(ss + 1e-6f) : 1.f;
+                nrm[tau] = nv;
+                dot[tau] = normed ? gd / (nv * nv) : 0.f;     // <dout, out> / n
+            }
         }
-        const float nv = normed ? sqrtf(ss + 1e-6f) : 1.f;
-        nrm[tid] = nv;
-        dot[tid] = normed ? gd / (nv * nv) : 0.f;     // <dout, out> / n
     }
     BWC_SYNC();
     // dy in place of dout (each thread its own channel)

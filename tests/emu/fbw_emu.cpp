@@ -12,6 +12,7 @@
 #define BWC_FN inline
 #define BWC_HD inline
 #define BWC_SYNC() ::emu::g_bar->arrive_and_wait()
+#define BWC_SHFL_XOR(v, m) ::emu::shfl_xor((v), (m))
 #include "../../gated_deltanet_recurrence_prefill_b200/csrc/conv1d_silu_backward.cuh"
 
 using namespace gdn::fbw;
