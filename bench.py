@@ -346,16 +346,45 @@ def bench_main(args, world, rank, local):
         "clocks": clocks,
         "wall_s_timed_region": round(wall, 3),
     }
-    if extra:
-        line["extra"] = extra
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+    if extra:
+        # the secondary lines go last, the long-context prefill at the very end,
+        # so that a reader that keeps only the tail of the line still has them
+        last = ["decode_bf16state_128seq_48layers", "decode_fused_128seq_48layers",
+                "decode_128seq_48layers", "prefill_varlen_16seq", "prefill_262k"]
+        ordered = {k: v for k, v in extra.items() if k not in last}
+        ordered.update({k: extra[k] for k in last if k in extra})
+        line["extra"] = ordered
+        line["summary"] = _summary(line)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def _summary(line):
+    """The headline numbers of the run in one small object (the JSON line's last key)."""
+    ex = line.get("extra", {})
+    out = {"prefill_T8192_ms": line["kernels"]["prefill"]["ms"],
+           "prefill_T8192_hbm_frac": line["roofline"]["frac"]}
+    lp = ex.get("prefill_262k")
+    if isinstance(lp, dict) and "ms" in lp:
+        out.update({"prefill_262k_ms": lp["ms"], "prefill_262k_tokens_per_s_layer": lp["tokens_per_s_layer"],
+                    "prefill_262k_tensor_frac": lp["tensor_frac"], "prefill_262k_hbm_frac": lp["hbm_frac"]})
+    vl = ex.get("prefill_varlen_16seq")
+    if isinstance(vl, dict) and "ms" in vl:
+        out.update({"prefill_varlen_ms": vl["ms"], "prefill_varlen_tensor_frac": vl["tensor_frac"],
+                    "prefill_varlen_hbm_frac": vl["hbm_frac"],
+                    "prefill_varlen_launches_per_step": vl["launches_per_step"]})
+    for key, name in (("decode_128seq_48layers", "decode_fp32_state"),
+                      ("decode_bf16state_128seq_48layers", "decode_bf16_state")):
+        d = ex.get(key)
+        if isinstance(d, dict) and "ms" in d:
+            out.update({name + "_ms": d["ms"], name + "_hbm_frac": d["hbm_frac"]})
+    return out
 
 
 def _smi_index(local):
@@ -450,6 +479,17 @@ def bench_long_prefill(args, dev, flush, peaks, world, lengths=None, seed=2):
            "ms": round(ms, 4), "tokens_per_s_layer": round(weak_scaling_rate(T, ms, world), 1),
            "TFLOP_s": round(tflops, 2), "tensor_frac": round(tflops / peaks["bf16_tflops"], 4),
            "GB_s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
+           # both roofs of the launch: algorithmic FLOPs (C = 64 chunked form) over
+           # the measured dense bf16 peak, algorithmic bytes over the measured copy
+           # bandwidth (the path is HBM-bound by arithmetic intensity)
+           "roofline": {
+               "tensor": {"achieved": round(tflops, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                          "frac": round(tflops / peaks["bf16_tflops"], 4),
+                          "flop_per_launch": int(FLOP_PER_TOKEN * T)},
+               "hbm": {"achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                       "frac": round(gbs / peaks["hbm_gbs"], 4),
+                       "bytes_per_launch": int(PREFILL_BYTES_PER_TOKEN * T + 2 * N * STATE_BYTES)},
+               "peak_source": peaks["source"]},
            # the producer/consumer kernel runs whole sequences (48 value heads, 144
            # CTAs) per cooperative launch when more units exist than fit at once
            "launches_per_step": N}

@@ -8,6 +8,7 @@ library is missing or no GPU is present, the calls raise.
 from ._lib import (  # noqa: F401
     GdnError,
     STATUS,
+    check_async,
     conv1d_silu,
     conv1d_silu_backward,
     decode_step,

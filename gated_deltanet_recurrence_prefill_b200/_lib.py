@@ -31,6 +31,7 @@ SIGNATURES = {
     "gdn_prefill": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32,
                               _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "gdn_prefill_status": (C.c_int, [_vp, _vp]),
+    "gdn_check_async": (C.c_int, [_vp, _vp, _vp]),
     "gdn_prefill_noalloc": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
                                       _i32, _f32, _vp, _vp, _vp, _vp]),
     "gdn_decode_step": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
@@ -306,8 +307,21 @@ def prefill_noalloc(q, k, v, a, b, A_log, dt_bias, cu_seqlens=None, scale=None,
 
 
 def prefill_status(workspace, stream=None) -> int:
-    """Error word left by the last prefill on `workspace` (waits for the stream)."""
+    """Error word left by the last prefill on `workspace` (waits for the stream);
+    workspace None: the array of gdn_prefill_noalloc on the current device."""
     return int(lib().gdn_prefill_status(_ptr(workspace), _stream(stream)))
+
+
+def check_async(workspace, status_word, stream=None) -> None:
+    """gdn_check_async: enqueue a copy of the workspace's error word (None: the
+    array of gdn_prefill_noalloc) into `status_word`, a one-element int32 tensor
+    on the device or in pinned host memory; returns without waiting."""
+    import torch
+    if status_word.numel() < 1 or status_word.dtype not in (torch.int32, torch.uint32):
+        raise ValueError("status_word must be a one-element int32 tensor")
+    if not status_word.is_cuda and not status_word.is_pinned():
+        raise ValueError("status_word must be on the device or in pinned host memory")
+    _check("gdn_check_async", lib().gdn_check_async(_ptr(workspace), _ptr(status_word), _stream(stream)))
 
 
 def decode_step(q, k, v, a, b, A_log, dt_bias, state, n_seq, layers, scale=None, o=None,

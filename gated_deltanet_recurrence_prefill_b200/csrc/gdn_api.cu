@@ -1,7 +1,7 @@
 // gdn_api.cu -- the C ABI of libgdn (see include/gdn.h): argument checks on the
 // host, then kernel launches on the caller's stream.  Nothing here allocates,
 // frees or synchronises, except gdn_prefill_status, which documents that it
-// waits for the stream.
+// waits for the stream (gdn_check_async is its non-waiting form).
 #include <cuda_runtime.h>
 #include <stdlib.h>
 #include <string.h>
@@ -221,13 +221,26 @@ gdn_status gdn_prefill_gated(const uint16_t* q, const uint16_t* k, const uint16_
 }
 
 gdn_status gdn_prefill_status(const void* workspace, gdn_stream_t stream) {
-    if (!workspace) return GDN_ERR_WORKSPACE;
+    if (!workspace) workspace = gdn::noalloc_scratch();
+    if (!workspace) return GDN_ERR_CUDA;
     uint32_t word = 0;
     cudaError_t e = cudaMemcpyAsync(&word, (const char*)workspace + gdn::kWsErrorWordOffset,
                                     sizeof word, cudaMemcpyDeviceToHost, (cudaStream_t)stream);
     if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e);
     return word == 0 ? GDN_OK : GDN_ERR_TIMEOUT;
+}
+
+gdn_status gdn_check_async(const void* workspace, uint32_t* status_word, gdn_stream_t stream) {
+    if (!status_word) return GDN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(status_word) & 3u) != 0) return GDN_ERR_MISALIGNED;
+    if (!workspace) workspace = gdn::noalloc_scratch();
+    if (!workspace) return GDN_ERR_CUDA;
+    // a 4-byte copy enqueued behind the prefill; the host does not wait
+    cudaError_t e = cudaMemcpyAsync(status_word, (const char*)workspace + gdn::kWsErrorWordOffset,
+                                    sizeof(uint32_t), cudaMemcpyDefault, (cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return GDN_OK;
 }
 
 gdn_status gdn_decode_step(const uint16_t* q, const uint16_t* k, const uint16_t* v,
@@ -416,7 +429,8 @@ gdn_status gdn_prefill_backward_chunked(const uint16_t* q, const uint16_t* k, co
 
 gdn_status gdn_selftest_bounded_wait(int32_t which, int64_t limit_us, void* workspace, gdn_stream_t stream) {
     if ((which != 0 && which != 1) || limit_us < 1000 || limit_us > 2000000) return GDN_ERR_INVALID_ARG;
-    if (!workspace) return GDN_ERR_WORKSPACE;
+    if (!workspace) workspace = gdn::noalloc_scratch();      // the array of gdn_prefill_noalloc
+    if (!workspace) return GDN_ERR_CUDA;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_MISALIGNED;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = cudaMemsetAsync(workspace, 0, gdn::kWsHeaderBytes, s);

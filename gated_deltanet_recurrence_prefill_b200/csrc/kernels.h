@@ -155,4 +155,10 @@ size_t prefill_min_workspace_bytes(int32_t n_seq, int32_t Hv);
 constexpr size_t kWsErrorWordOffset = 0;     // uint32 error word (0 = ok)
 constexpr size_t kWsHeaderBytes = 256;
 
+// device address of the library-owned prefill scratch array (the workspace of
+// gdn_prefill_noalloc) on the current device, looked up once per device and
+// cached; null if the lookup fails.  Allocates nothing.
+void* noalloc_scratch();
+size_t noalloc_scratch_bytes();
+
 }  // namespace gdn

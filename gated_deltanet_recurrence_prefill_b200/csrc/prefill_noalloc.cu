@@ -14,7 +14,15 @@
 // library holds kNoAllocScratchBytes of it until the process exits.  Host code
 // cannot pass its name to a kernel (on the host the name is only a stand-in for
 // the symbol), so the first call on each device looks up its device address
-// with cudaGetSymbolAddress while that device is current, and caches it.
+// with cudaGetSymbolAddress while that device is current, and caches it.  The
+// cache is per device number and lives as long as the process: a
+// cudaDeviceReset destroys the module and with it the array, so a process that
+// resets a device must not call gdn_prefill_noalloc on it again.
+//
+// The array holds 64 KiB, less than one producer / consumer ring (397,440
+// bytes), so this entry point always runs the single-CTA prefill kernel
+// (about 2.5x slower than gdn_prefill with a full workspace at T = 8192), and
+// GDN_PREFILL_KERNEL=pc makes it return GDN_ERR_UNSUPPORTED.
 #include <atomic>
 
 #include <cuda_runtime.h>
@@ -33,6 +41,30 @@ std::atomic<void*> g_scratch_addr[kMaxDevices];
 
 }  // namespace
 
+namespace gdn {
+
+void* noalloc_scratch() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    void* scratch = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (!scratch) {
+        // one-time set-up on this device (with the device current)
+        if (cudaGetSymbolAddress(&scratch, g_prefill_scratch) != cudaSuccess || !scratch) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        g_scratch_addr[dev].store(scratch, std::memory_order_release);
+    }
+    return scratch;
+}
+
+size_t noalloc_scratch_bytes() { return kNoAllocScratchBytes; }
+
+}  // namespace gdn
+
 extern "C" {
 
 gdn_status gdn_prefill_noalloc(const uint16_t* q, const uint16_t* k, const uint16_t* v,
@@ -44,16 +76,8 @@ gdn_status gdn_prefill_noalloc(const uint16_t* q, const uint16_t* k, const uint1
     // sizes first: nothing touches the GPU when the scratch array is too small
     (void)T; (void)Hqk; (void)d;
     if (gdn::prefill_min_workspace_bytes(n_seq, Hv) > kNoAllocScratchBytes) return GDN_ERR_WORKSPACE;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return GDN_ERR_UNSUPPORTED;
-    void* scratch = g_scratch_addr[dev].load(std::memory_order_acquire);
-    if (!scratch) {
-        // one-time set-up on this device (with the device current)
-        if (cudaGetSymbolAddress(&scratch, g_prefill_scratch) != cudaSuccess || !scratch)
-            return GDN_ERR_CUDA;
-        g_scratch_addr[dev].store(scratch, std::memory_order_release);
-    }
+    void* scratch = gdn::noalloc_scratch();
+    if (!scratch) return GDN_ERR_CUDA;
     // gdn_prefill clears the error word at the start of the scratch on `stream`
     // before its kernel runs; everything else in the scratch is written before
     // it is read within one call.

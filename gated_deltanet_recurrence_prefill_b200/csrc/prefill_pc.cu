@@ -35,9 +35,10 @@
 // Consumer (role 0).  A loader thread bulk-loads each chunk from the ring into
 // one of two receive slots and hands ring slots back to the producers (a
 // second counter per ring slot).  Every product has d_v as its M dimension
-// (TMEM lane = v row) and spans 128 columns (a tcgen05.mma with M = 128 and
-// K = 16 occupies the tensor core for about the same ~150 cycles whatever N
-// is, up to 256):
+// (TMEM lane = v row) and spans 128 columns (measured on B200: a bf16
+// tcgen05.mma with M = 128 and K = 16 takes about 50 cycles at N = 64, 66 at
+// N = 128 and 130 at N = 256, and M = 64 costs as much as M = 128, so
+// N = 128 is the cheapest width per column that keeps the issue rate up):
 //   D^T  = V^T [T b; R b]^T                M128 N128 K64   (in the chain's gaps)
 //   D^T += S [-W; Qh]^T                    M128 N128 K128  -> [U^T | o^T / scale]
 //   S~  += (kappa U / Gamma)^T K           M128 N128 K64   (accumulates in TMEM)

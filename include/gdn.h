@@ -207,9 +207,29 @@ gdn_status gdn_prefill(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
  * gdn_prefill_status -- waits for `stream`, then reads the error word that the
  * last gdn_prefill on this workspace left: GDN_OK, or GDN_ERR_TIMEOUT if a
  * bounded wait inside the kernel ran out (the outputs are then invalid).
- * Synchronises the stream; not for use inside stream capture.
+ * workspace NULL: the library-owned array that gdn_prefill_noalloc uses on the
+ * current device.  Synchronises the stream; not for use inside stream capture
+ * (gdn_check_async is the form that does not wait).
  */
 gdn_status gdn_prefill_status(const void* workspace, gdn_stream_t stream);
+
+/*
+ * gdn_check_async -- the non-waiting error check (library error reporting; the
+ * pages define no interface).  Enqueues on `stream` a copy of the workspace's
+ * error word into *status_word and returns at once: nothing is synchronised,
+ * so it may follow gdn_prefill inside a stream capture.  Once the stream has
+ * passed that point, *status_word is 0 if every bounded wait of the prefills
+ * that used this workspace before it succeeded, nonzero if one ran out (their
+ * outputs are then invalid; gdn_prefill_status would report GDN_ERR_TIMEOUT).
+ *  workspace    the prefill's workspace, or NULL for the library-owned array
+ *               of gdn_prefill_noalloc on the current device.
+ *  status_word  4-byte aligned uint32 in device memory or in page-locked host
+ *               memory (with pageable host memory the copy may wait for the
+ *               stream); owned by the caller.
+ * Errors: GDN_ERR_INVALID_ARG (status_word NULL), GDN_ERR_MISALIGNED,
+ * GDN_ERR_CUDA (the copy could not be enqueued).
+ */
+gdn_status gdn_check_async(const void* workspace, uint32_t* status_word, gdn_stream_t stream);
 
 /*
  * gdn_prefill_noalloc -- gdn_prefill for callers that cannot allocate device
@@ -227,13 +247,20 @@ gdn_status gdn_prefill_status(const void* workspace, gdn_stream_t stream);
  * value heads); larger problems are rejected with GDN_ERR_WORKSPACE before
  * anything touches the GPU.
  *
+ * The array holds less than one producer / consumer ring, so this entry point
+ * always runs the single-CTA prefill kernel: about 0.77 ms at T = 8192 (16 / 48
+ * heads) against 0.30 ms for gdn_prefill with a full workspace.  With
+ * GDN_PREFILL_KERNEL=pc set it returns GDN_ERR_UNSUPPORTED.
+ *
  * The first call on each device looks up the array's device address (with that
  * device current) and caches it; make that first call before any stream
- * capture.  All calls in the process share the one array, which keeps what the
- * last call left there: calls that overlap on the GPU (different streams,
- * devices not involved) race on it, so order them on one stream.  A bounded
- * device wait that times out is recorded in that shared array and is not
- * reported by this entry point.
+ * capture.  The cache lasts as long as the process: after a cudaDeviceReset of
+ * a device, do not call this entry point on that device again.  All calls in
+ * the process share the one array, which keeps what the last call left there:
+ * calls that overlap on the GPU (different streams, devices not involved) race
+ * on it, so order them on one stream.  A bounded device wait that times out is
+ * recorded in that shared array: gdn_prefill_status(NULL, stream) and
+ * gdn_check_async(NULL, word, stream) read it.
  */
 gdn_status gdn_prefill_noalloc(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                const float* a, const float* b, const float* A_log,
@@ -463,7 +490,8 @@ gdn_status gdn_gated_norm_backward(const float* o, const uint16_t* z, const floa
  * wait gives up and the kernel records the error in the workspace's error word
  * as the prefill does, so that gdn_prefill_status(workspace) then returns
  * GDN_ERR_TIMEOUT.  Nothing faults or hangs; the context stays usable.
- * workspace: at least 256 bytes, 256-byte aligned (its header is cleared).
+ * workspace: at least 256 bytes, 256-byte aligned (its header is cleared), or
+ * NULL for the library-owned array of gdn_prefill_noalloc.
  */
 gdn_status gdn_selftest_bounded_wait(int32_t which, int64_t limit_us, void* workspace, gdn_stream_t stream);
 

@@ -27,7 +27,7 @@ def L():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for required in ("gdn_conv1d_silu", "gdn_prefill", "gdn_prefill_workspace_size",
-                     "gdn_decode_step", "gdn_decode_step_fused", "gdn_prefill_status",
+                     "gdn_decode_step", "gdn_decode_step_fused", "gdn_prefill_status", "gdn_check_async",
                      "gdn_gated_norm", "gdn_prefill_gated", "gdn_decode_step_gated",
                      "gdn_prefill_backward", "gdn_prefill_backward_workspace_size",
                      "gdn_prefill_backward_chunked", "gdn_prefill_backward_chunked_workspace_size",
@@ -314,5 +314,10 @@ def test_selftest_rejects_bad_arguments(L):
     assert L.gdn_selftest_bounded_wait(2, 20000, _p(0x20000), None) == 1     # unknown wait
     assert L.gdn_selftest_bounded_wait(0, 10, _p(0x20000), None) == 1        # below 1 ms
     assert L.gdn_selftest_bounded_wait(0, 10_000_000, _p(0x20000), None) == 1   # above 2 s
-    assert L.gdn_selftest_bounded_wait(0, 20000, None, None) == 6
     assert L.gdn_selftest_bounded_wait(0, 20000, _p(0x20000 + 16), None) == 3
+
+
+def test_check_async_rejects_bad_arguments(L):
+    """gdn_check_async validates its output word before enqueueing anything."""
+    assert L.gdn_check_async(_p(0x20000), None, None) == 1          # no status word
+    assert L.gdn_check_async(_p(0x20000), _p(0x30002), None) == 3   # not 4-byte aligned
