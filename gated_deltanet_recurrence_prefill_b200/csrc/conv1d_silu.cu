@@ -17,6 +17,15 @@
 // sequence boundary the history restarts from conv_state_in
 // (or zeros).  (A variant that staged 64-token tiles in shared memory by TMA
 // measured slower: with one tile's arithmetic per barrier the SMs sat idle.)
+//
+// The kernel is bound as much by instruction issue as by HBM (about 130
+// instructions per lane and token for 16 bytes in and 16 out), so a run that
+// lies inside one sequence and is a full kRun tokens long takes a fast path:
+// the arithmetic on pairs of channels with the packed f32x2 FMA of sm_100a,
+// tokens in unrolled steps of three (the width of the history, so the history
+// rotates by register renaming instead of copies), and pointers advanced
+// instead of recomputed.  Runs that hold a sequence boundary, and the last
+// partial run, take the general per-token path.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -25,7 +34,7 @@ namespace gdn {
 namespace {
 
 constexpr int kD = 128;
-constexpr int kRun = 32;              // tokens per warp
+constexpr int kRun = 48;              // tokens per warp (a multiple of kStep)
 constexpr int kWarps = 8;             // warps per CTA
 constexpr int kChan = 8;              // channels per lane
 #ifndef GDN_CONV_BATCH
@@ -38,6 +47,10 @@ constexpr int kBatch = GDN_CONV_BATCH;  // tokens per batch
 // in flight); kDepth / kBatch batches are outstanding at once.
 constexpr int kDepth = 16;
 static_assert(kDepth % kBatch == 0 && kRun % kBatch == 0, "ring of whole batches");
+// fast path: steps of three tokens, four steps in flight in the first 12 ring slots
+constexpr int kStep = 3;
+constexpr int kFastSteps = 4;
+static_assert(kRun % kStep == 0 && kStep * kFastSteps <= kDepth, "fast path ring");
 constexpr int kRingBytesPerWarp = kDepth * 32 * 16;
 
 // index of the sequence containing token t: largest n with cu[n] <= t
@@ -69,6 +82,21 @@ GDN_DEVICE void cp_async16(void* sdst, const void* gsrc) {
 GDN_DEVICE void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N> GDN_DEVICE void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 GDN_DEVICE void stg_stream(uint16_t* p, uint4 v) { __stcs(reinterpret_cast<uint4*>(p), v); }
+
+GDN_DEVICE float2 silu2(float2 x) {
+    const float2 h = __fmul2_rn(x, make_float2(0.5f, 0.5f));
+    float tx, ty;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(tx) : "f"(h.x));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(ty) : "f"(h.y));
+    return __ffma2_rn(h, make_float2(tx, ty), h);
+}
+
+GDN_DEVICE void unpack4x2(const uint4 r, float2* x) {
+    x[0] = bf16x2_to_f32x2(r.x);
+    x[1] = bf16x2_to_f32x2(r.y);
+    x[2] = bf16x2_to_f32x2(r.z);
+    x[3] = bf16x2_to_f32x2(r.w);
+}
 
 GDN_DEVICE void unpack8(const uint4 r, float* x) {
     float2 t;
@@ -148,11 +176,91 @@ conv1d_silu_kernel(const uint16_t* __restrict__ qkv, const float* __restrict__ w
     else { dst_base = vo + (int64_t)(hc - 2 * Hqk) * kD; dst_stride = (int64_t)Hv * kD; }
     dst_base += (lane & 15) * kChan;
 
+    extern __shared__ __align__(16) uint8_t ring_all[];
+    uint8_t* ring = ring_all + (threadIdx.x >> 5) * kRingBytesPerWarp + lane * 16;
+
+    if (t1 - t0 == kRun && eos >= t1) {
+        // ---- fast path: a full run inside one sequence.  Step j covers tokens
+        // t0 + 3 j .. + 2, whose inputs sit in ring slots 3 (j % 4) .. + 2,
+        // requested four steps ahead (one commit group per step).
+        float2 w2[4][4], h[3][4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) w2[p][j] = make_float2(wr[2 * p][j], wr[2 * p + 1][j]);
+#pragma unroll
+            for (int j = 0; j < 3; ++j) h[j][p] = make_float2(hist[j][2 * p], hist[j][2 * p + 1]);
+        }
+        const uint16_t* src = qkv + t0 * Ctot + c0;
+#pragma unroll
+        for (int st = 0; st < kFastSteps; ++st) {
+#pragma unroll
+            for (int u = 0; u < kStep; ++u) cp_async16(ring + (st * kStep + u) * 512, src + (st * kStep + u) * Ctot);
+            cp_async_commit();
+        }
+        uint16_t* dst = dst_base + t0 * dst_stride;
+#pragma unroll 1
+        for (int st = 0; st < kRun / kStep; ++st) {
+            cp_async_wait<kFastSteps - 1>();
+            const int slot0 = (st % kFastSteps) * kStep;
+            float2 x[kStep][4];
+#pragma unroll
+            for (int u = 0; u < kStep; ++u) unpack4x2(*reinterpret_cast<const uint4*>(ring + (slot0 + u) * 512), x[u]);
+            // the slots just read take the step kFastSteps ahead (its group may be empty)
+            if (st + kFastSteps < kRun / kStep) {
+#pragma unroll
+                for (int u = 0; u < kStep; ++u)
+                    cp_async16(ring + (slot0 + u) * 512, src + ((st + kFastSteps) * kStep + u) * Ctot);
+            }
+            cp_async_commit();
+#pragma unroll
+            for (int u = 0; u < kStep; ++u) {
+                // inputs x[t-3], x[t-2], x[t-1], x[t] of token u of this step
+                float2 y[4];
+                float2 ss2 = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    const float2 a0 = u == 0 ? h[0][p] : (u == 1 ? h[1][p] : h[2][p]);
+                    const float2 a1 = u == 0 ? h[1][p] : (u == 1 ? h[2][p] : x[0][p]);
+                    const float2 a2 = u == 0 ? h[2][p] : (u == 1 ? x[0][p] : x[1][p]);
+                    float2 acc = __fmul2_rn(w2[p][0], a0);
+                    acc = __ffma2_rn(w2[p][1], a1, acc);
+                    acc = __ffma2_rn(w2[p][2], a2, acc);
+                    acc = __ffma2_rn(w2[p][3], x[u][p], acc);
+                    y[p] = silu2(acc);
+                    ss2 = __ffma2_rn(y[p], y[p], ss2);
+                }
+                if (warp_norm) {       // warp-uniform: the shuffles need all 32 lanes
+                    float ss = ss2.x + ss2.y;
+#pragma unroll
+                    for (int m = 8; m >= 1; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
+                    const float inv = (is_q || is_k) ? rsqrtf(ss + 1e-6f) : 1.f;
+                    const float2 iv = make_float2(inv, inv);
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) y[p] = __fmul2_rn(y[p], iv);
+                }
+                uint4 out;
+                out.x = pack_bf16x2(y[0].x, y[0].y);
+                out.y = pack_bf16x2(y[1].x, y[1].y);
+                out.z = pack_bf16x2(y[2].x, y[2].y);
+                out.w = pack_bf16x2(y[3].x, y[3].y);
+                if (active) stg_stream(dst, out);
+                dst += dst_stride;
+            }
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                h[0][p] = x[0][p];
+                h[1][p] = x[1][p];
+                h[2][p] = x[2][p];
+            }
+        }
+        cp_async_wait<0>();
+        return;
+    }
+
     // tokens are processed in batches of kBatch; token t's 16 bytes of this lane
     // sit in ring slot (t - t0) % kDepth, requested kDepth tokens ahead, one
     // commit group per batch
-    extern __shared__ __align__(16) uint8_t ring_all[];
-    uint8_t* ring = ring_all + (threadIdx.x >> 5) * kRingBytesPerWarp + lane * 16;
 #pragma unroll
     for (int bq = 0; bq < kDepth / kBatch; ++bq) {
 #pragma unroll
