@@ -680,7 +680,7 @@ def bench_front_backward(args, dev, flush, peaks, world):
     gbs = nbytes / (ms * 1e-3) / 1e9
     out = {"workload": f"gdn_conv1d_silu_backward T={T} N=1 Hqk=16 Hv=48 d=128, conv history given",
            "ms": round(ms, 4), "GB_s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
-           "bytes_per_step": nbytes, "launches_per_step": 2}
+           "bytes_per_step": nbytes, "launches_per_step": 3}
     del qkv, dq, dk, dv, ws
     torch.cuda.empty_cache()
     return out
@@ -884,6 +884,8 @@ def profile_case(args):
       prefill8k   gdn_prefill, T=8192, 1 sequence, S0 != 0   (~0.5 GB resident)
       frontend8k  gdn_conv1d_silu, T=8192                      (~0.4 GB)
       decode16    gdn_decode_step, 16 sequences x 48 layers    (~2.4 GB of state)
+      decode16bf  gdn_decode_step_bf16, the same units         (~1.2 GB of state)
+      frontbw8k   gdn_conv1d_silu_backward, T=8192, history    (~1.3 GB)
     """
     import numpy as np
     import torch
@@ -911,6 +913,25 @@ def profile_case(args):
                  f32(inp.dt_bias), st, inp.n_seq, inp.layers]
         for _ in range(args.warmup + args.steps):
             gdn.decode_step(*args_)
+    elif args.profile_case == "decode16bf":
+        inp = synth.make_decode(16, 48, 4)
+        st = torch.empty(inp.U, HV, D, D, dtype=torch.bfloat16, device=dev)
+        st.normal_(0.0, 0.02)
+        args_ = [to16(inp.q), to16(inp.k), to16(inp.v), f32(inp.a), f32(inp.b), f32(inp.A_log),
+                 f32(inp.dt_bias), st, inp.n_seq, inp.layers]
+        for _ in range(args.warmup + args.steps):
+            gdn.decode_step(*args_)
+    elif args.profile_case == "frontbw8k":
+        fe = synth.workload(1)
+        x, w = to16(fe.qkv), f32(fe.conv_w)
+        cs = torch.randn(1, (2 * HQK + HV) * D, 3, device=dev)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(9)
+        dq = torch.randn(T_MAIN, HQK, D, generator=gen, device=dev)
+        dk = torch.randn(T_MAIN, HQK, D, generator=gen, device=dev)
+        dv = torch.randn(T_MAIN, HV, D, generator=gen, device=dev)
+        for _ in range(args.warmup + args.steps):
+            gdn.conv1d_silu_backward(x, w, dq, dk, dv, HQK, HV, conv_state=cs)
     torch.cuda.synchronize()
     print(f"profile case {args.profile_case}: ok")
 
@@ -954,7 +975,7 @@ def main():
     ap.add_argument("--primary-only", action="store_true", help="skip the 262K and decode lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--profile-case", choices=["prefill8k", "frontend8k", "decode16"],
+    ap.add_argument("--profile-case", choices=["prefill8k", "frontend8k", "decode16", "decode16bf", "frontbw8k"],
                     help="run one kernel on a small case for an ncu capture; no timing")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -67,7 +67,7 @@ struct Params {
 BWC_HD int64_t n_tiles(int64_t T) { return (T + kTile - 1) / kTile; }
 
 // shared-memory floats of one job
-constexpr int kTileFloats = 3 * kSpan * kLd + 4 * kSpan;
+constexpr int kTileFloats = 3 * kSpan * kLd + 4 * kSpan + (kSpan + 3) * kD;
 
 BWC_FN float bf16f(uint16_t h) {
 #ifdef __CUDA_ARCH__
@@ -92,9 +92,24 @@ BWC_FN int seq_of(const Params& p, int64_t t) {
     return lo;
 }
 
-// x~ at position pos for a token of sequence n starting at bos, channel c
-BWC_FN float xt(const Params& p, int64_t Ctot, int n, int64_t bos, int64_t pos, int64_t c) {
-    if (pos >= bos) return bf16f(p.x[pos * Ctot + c]);
+
+// A tile whose tokens, their three-token history and the three tokens after it
+// all lie in one sequence takes the streaming kernel (conv1d_silu_backward.cu);
+// tile_block handles every other tile.  Both kernels decide with this test.
+BWC_FN bool stream_tile(const Params& p, int64_t tile) {
+    const int64_t t0 = tile * kTile;
+    if (t0 < 3 || t0 + kSpan > p.T) return false;
+    if (!p.cu) return true;
+    const int n = seq_of(p, t0);
+    return (int64_t)p.cu[n] + 3 <= t0 && t0 + kSpan <= (int64_t)p.cu[n + 1];
+}
+
+// x~ at position pos for a token of sequence n starting at bos, channel c:
+// x from the tile's staged copy (xr holds positions t0 - 3 ..), or the
+// sequence's conv_state history (or zero) before its first token
+BWC_FN float xts(const Params& p, int64_t Ctot, int n, int64_t bos, int64_t pos, int64_t c, const float* xr,
+                 int64_t t0, int tid) {
+    if (pos >= bos) return xr[(pos - (t0 - 3)) * kD + tid];
     return p.cs ? p.cs[((int64_t)n * Ctot + c) * 3 + (3 - (bos - pos))] : 0.f;
 }
 
@@ -113,11 +128,18 @@ BWC_FN void tile_block(const Params& p, int64_t tile, int hh, int tid, float* sm
     float* dot = nrm + kSpan;
     int32_t* sq = reinterpret_cast<int32_t*>(dot + kSpan);    // per token: sequence
     int32_t* eo = sq + kSpan;                                 // per token: sequence end
+    float* xr = reinterpret_cast<float*>(eo + kSpan);         // x at positions t0 - 3 ..  [kSpan + 3][kD]
 
     if (tid < ntok) {
         const int n = seq_of(p, t0 + tid);
         sq[tid] = n;
         eo[tid] = p.cu ? p.cu[n + 1] : (int32_t)p.T;
+    }
+    // this channel's inputs at every position the tile reads, loaded up front so
+    // that the loads overlap (positions before 0 are never read from here)
+    for (int r = 0; r < ntok + 3; ++r) {
+        const int64_t pos = t0 - 3 + r;
+        xr[r * kD + tid] = pos >= 0 ? bf16f(p.x[pos * Ctot + c]) : 0.f;
     }
     BWC_SYNC();
     float w[4];
@@ -125,16 +147,17 @@ BWC_FN void tile_block(const Params& p, int64_t tile, int hh, int tid, float* sm
     const float* dsrc = hh < p.Hqk ? p.dq + (int64_t)hh * kD
                       : normed ? p.dk + (int64_t)(hh - p.Hqk) * kD : p.dv + (int64_t)(hh - 2 * p.Hqk) * kD;
     const int64_t dstride = (normed ? (int64_t)p.Hqk : (int64_t)p.Hv) * kD;
+    // the output gradient of every token, loaded up front (independent loads)
+    for (int tau = 0; tau < ntok; ++tau) gs[tau * kLd + tid] = dsrc[(t0 + tau) * dstride + tid];
     for (int tau = 0; tau < ntok; ++tau) {
         const int64_t t = t0 + tau;
         const int n = sq[tau];
         const int64_t bos = p.cu ? p.cu[n] : 0;
         float y = 0.f;
-        for (int j = 0; j < 4; ++j) y = fmaf(w[j], xt(p, Ctot, n, bos, t - 3 + j, c), y);
+        for (int j = 0; j < 4; ++j) y = fmaf(w[j], xts(p, Ctot, n, bos, t - 3 + j, c, xr, t0, tid), y);
         const float s = 1.f / (1.f + expf(-y));
         as[tau * kLd + tid] = y * s;
         sg[tau * kLd + tid] = s;
-        gs[tau * kLd + tid] = dsrc[t * dstride + tid];
     }
     BWC_SYNC();
     // per token: the norm and <dout, out> / n, one warp per token (a lane sums 4
@@ -180,7 +203,7 @@ BWC_FN void tile_block(const Params& p, int64_t tile, int hh, int tid, float* sm
         const int n = sq[tau];
         const int64_t bos = p.cu ? p.cu[n] : 0;
         const float dy = gs[tau * kLd + tid];
-        for (int j = 0; j < 4; ++j) dwa[j] = fmaf(dy, xt(p, Ctot, n, bos, t - 3 + j, c), dwa[j]);
+        for (int j = 0; j < 4; ++j) dwa[j] = fmaf(dy, xts(p, Ctot, n, bos, t - 3 + j, c, xr, t0, tid), dwa[j]);
     }
     for (int j = 0; j < 4; ++j) p.dwp[(tile * Ctot + c) * 4 + j] = dwa[j];
     // the history gradient of every sequence that starts in this tile
@@ -214,8 +237,19 @@ BWC_FN void reduce_w_block(const Params& p, int64_t blk, int tid) {
     const int64_t Ctot = (int64_t)(2 * p.Hqk + p.Hv) * kD;
     const int64_t i = blk * kThreads + tid;
     if (i >= Ctot * 4) return;
+    // the partial sums are added in tile order; eight are loaded ahead of their
+    // additions so that the loads overlap (the order of the additions, and so
+    // the result, is the same)
     float s = 0.f;
-    for (int64_t tl = 0; tl < p.n_tiles; ++tl) s += p.dwp[tl * Ctot * 4 + i];
+    const float* src = p.dwp + i;
+    const int64_t stride = Ctot * 4;
+    int64_t tl = 0;
+    for (; tl + 8 <= p.n_tiles; tl += 8) {
+        float v[8];
+        for (int r = 0; r < 8; ++r) v[r] = src[(tl + r) * stride];
+        for (int r = 0; r < 8; ++r) s += v[r];
+    }
+    for (; tl < p.n_tiles; ++tl) s += src[tl * stride];
     p.dw[i] = s;
 }
 
