@@ -302,6 +302,7 @@ def bench_main(args, world, rank, local):
         extra["prefill_262k"] = bench_long_prefill(args, dev, flush, peaks, world)
         extra["prefill_varlen_16seq"] = bench_long_prefill(
             args, dev, flush, peaks, world, lengths=synth.varlen_lengths(3), seed=3)
+        extra["prefill_262k_bf16o"] = bench_long_prefill(args, dev, flush, peaks, world, o_bf16=True)
         extra["gated_norm_T8192"] = bench_gated_norm(args, dev, flush, peaks, world)
         extra["layer_tail_T8192"] = bench_layer_tail(args, dev, flush, peaks, world)
         extra["backward_T8192"] = bench_backward(args, dev, flush, peaks, world)
@@ -352,7 +353,7 @@ def bench_main(args, world, rank, local):
         # the secondary lines go last, the long-context prefill at the very end,
         # so that a reader that keeps only the tail of the line still has them
         last = ["decode_bf16state_128seq_48layers", "decode_fused_128seq_48layers",
-                "decode_128seq_48layers", "prefill_varlen_16seq", "prefill_262k"]
+                "decode_128seq_48layers", "prefill_varlen_16seq", "prefill_262k_bf16o", "prefill_262k"]
         ordered = {k: v for k, v in extra.items() if k not in last}
         ordered.update({k: extra[k] for k in last if k in extra})
         line["extra"] = ordered
@@ -374,6 +375,9 @@ def _summary(line):
     if isinstance(lp, dict) and "ms" in lp:
         out.update({"prefill_262k_ms": lp["ms"], "prefill_262k_tokens_per_s_layer": lp["tokens_per_s_layer"],
                     "prefill_262k_tensor_frac": lp["tensor_frac"], "prefill_262k_hbm_frac": lp["hbm_frac"]})
+    lb = ex.get("prefill_262k_bf16o")
+    if isinstance(lb, dict) and "ms" in lb:
+        out.update({"prefill_262k_bf16o_ms": lb["ms"], "prefill_262k_bf16o_hbm_frac": lb["hbm_frac"]})
     vl = ex.get("prefill_varlen_16seq")
     if isinstance(vl, dict) and "ms" in vl:
         out.update({"prefill_varlen_ms": vl["ms"], "prefill_varlen_tensor_frac": vl["tensor_frac"],
@@ -421,9 +425,10 @@ def weak_scaling_rate(units_per_rank, ms_per_step_max, world):
     return world * units_per_rank / (ms_per_step_max * 1e-3)
 
 
-def bench_long_prefill(args, dev, flush, peaks, world, lengths=None, seed=2):
+def bench_long_prefill(args, dev, flush, peaks, world, lengths=None, seed=2, o_bf16=False):
     """One gdn_prefill launch over `lengths` (default: one sequence of T = 262144),
-    per-sequence S0 ~ N(0, 0.02^2) (inputs drawn on the device)."""
+    per-sequence S0 ~ N(0, 0.02^2) (inputs drawn on the device).  o_bf16: the
+    bf16-output variant gdn_prefill_bf16 (o is 2 bytes per element)."""
     import torch
     import gated_deltanet_recurrence_prefill_b200 as gdn
     lengths = lengths or [T_LONG]
@@ -446,7 +451,7 @@ def bench_long_prefill(args, dev, flush, peaks, world, lengths=None, seed=2):
     dt = torch.exp(torch.empty(HV, device=dev).uniform_(-6.907755, -2.302585, generator=gen))
     dt_bias = torch.log(torch.expm1(dt))
     s0 = 0.02 * torch.randn(N, HV, D, D, generator=gen, device=dev)
-    o = torch.empty(T, HV, D, dtype=torch.float32, device=dev)
+    o = torch.empty(T, HV, D, dtype=torch.bfloat16 if o_bf16 else torch.float32, device=dev)
     fs = torch.empty_like(s0)
     cu = None
     if N > 1:
@@ -469,9 +474,12 @@ def bench_long_prefill(args, dev, flush, peaks, world, lengths=None, seed=2):
     times, _ = _time_steps(step, max(3, args.warmup), max(3, min(args.steps, 10)), flush, mk, world)
     ms = _max_over_ranks(sum(times) / len(times), world)
     tflops = FLOP_PER_TOKEN * T / (ms * 1e-3) / 1e12
-    gbs = (PREFILL_BYTES_PER_TOKEN * T + 2 * N * STATE_BYTES) / (ms * 1e-3) / 1e9
+    bytes_per_token = PREFILL_BYTES_PER_TOKEN - (2 * HV * D if o_bf16 else 0)
+    gbs = (bytes_per_token * T + 2 * N * STATE_BYTES) / (ms * 1e-3) / 1e9
     if N == 1:
         wl = f"gdn_prefill T={T} N=1 Hqk=16 Hv=48 d=128 S0~N(0,0.02^2)"
+        if o_bf16:
+            wl = wl.replace("gdn_prefill", "gdn_prefill_bf16 (bf16 o)")
     else:
         wl = (f"gdn_prefill varlen N={N} (lengths U[1024,32768], T={T}, longest {max(lengths)}) "
               f"Hqk=16 Hv=48 d=128 per-sequence S0~N(0,0.02^2)")
@@ -488,7 +496,7 @@ def bench_long_prefill(args, dev, flush, peaks, world, lengths=None, seed=2):
                           "flop_per_launch": int(FLOP_PER_TOKEN * T)},
                "hbm": {"achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                        "frac": round(gbs / peaks["hbm_gbs"], 4),
-                       "bytes_per_launch": int(PREFILL_BYTES_PER_TOKEN * T + 2 * N * STATE_BYTES)},
+                       "bytes_per_launch": int(bytes_per_token * T + 2 * N * STATE_BYTES)},
                "peak_source": peaks["source"]},
            # the producer/consumer kernel runs whole sequences (48 value heads, 144
            # CTAs) per cooperative launch when more units exist than fit at once

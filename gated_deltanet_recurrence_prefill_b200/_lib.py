@@ -31,6 +31,8 @@ SIGNATURES = {
     "gdn_prefill": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32,
                               _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "gdn_prefill_status": (C.c_int, [_vp, _vp]),
+    "gdn_prefill_bf16": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32,
+                                   _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "gdn_check_async": (C.c_int, [_vp, _vp, _vp]),
     "gdn_prefill_noalloc": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
                                       _i32, _f32, _vp, _vp, _vp, _vp]),
@@ -236,9 +238,16 @@ def prefill_workspace_size(n_seq, T, Hqk, Hv, d=128) -> int:
 
 
 def prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens=None, scale=None, initial_state=None,
-            final_state=None, o=None, workspace=None, want_final_state=True, stream=None):
-    """Chunked prefill.  Returns (o [T,Hv,d] f32, final_state [N,Hv,d,d] f32 or None)."""
+            final_state=None, o=None, workspace=None, want_final_state=True, stream=None,
+            o_dtype=None):
+    """Chunked prefill.  Returns (o [T,Hv,d], final_state [N,Hv,d,d] f32 or None).
+    o is float32 (gdn_prefill), or bf16 (gdn_prefill_bf16) when o_dtype is
+    torch.bfloat16 or a bf16 `o` is passed."""
     import torch
+    if o_dtype is None:
+        o_dtype = o.dtype if o is not None else torch.float32
+    if o_dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("o must be float32 or bfloat16")
     T, Hqk, d = q.shape
     Hv = v.shape[1]
     n_seq = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
@@ -256,17 +265,20 @@ def prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens=None, scale=None, initial_
     if scale is None:
         scale = d ** -0.5
     if o is None:
-        o = torch.empty(T, Hv, d, dtype=torch.float32, device=q.device)
+        o = torch.empty(T, Hv, d, dtype=o_dtype, device=q.device)
+    _need(o, o_dtype, (T, Hv, d), "o")
     if final_state is None and want_final_state:
         final_state = torch.empty(n_seq, Hv, d, d, dtype=torch.float32, device=q.device)
     ws_bytes = prefill_workspace_size(n_seq, T, Hqk, Hv, d)
     if workspace is None:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
-    st = lib().gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias),
-                           _ptr(cu_seqlens), n_seq, T, Hqk, Hv, d, float(scale),
-                           _ptr(initial_state), _ptr(final_state), _ptr(o), _ptr(workspace),
-                           workspace.numel() * workspace.element_size(), _stream(stream))
-    _check("gdn_prefill", st)
+    fn, name = ((lib().gdn_prefill_bf16, "gdn_prefill_bf16") if o_dtype == torch.bfloat16
+                else (lib().gdn_prefill, "gdn_prefill"))
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(A_log), _ptr(dt_bias),
+            _ptr(cu_seqlens), n_seq, T, Hqk, Hv, d, float(scale),
+            _ptr(initial_state), _ptr(final_state), _ptr(o), _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(name, st)
     return o, final_state
 
 

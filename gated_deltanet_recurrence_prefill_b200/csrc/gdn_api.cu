@@ -168,6 +168,36 @@ gdn_status gdn_prefill(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
     return e == cudaSuccess ? GDN_OK : cuda_fail(e);
 }
 
+gdn_status gdn_prefill_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* a,
+                            const float* b, const float* A_log, const float* dt_bias,
+                            const int32_t* cu_seqlens, int32_t n_seq, int64_t T, int32_t Hqk,
+                            int32_t Hv, int32_t d, float scale, const float* initial_state,
+                            float* final_state, uint16_t* o, void* workspace, size_t workspace_bytes,
+                            gdn_stream_t stream) {
+    gdn_status st = check_heads(Hqk, Hv, d);
+    if (st != GDN_OK) return st;
+    if ((st = check_seqs(cu_seqlens, n_seq, T)) != GDN_OK) return st;
+    if (!A_log || !dt_bias) return GDN_ERR_INVALID_ARG;
+    if (T > 0 && (!q || !k || !v || !a || !b || !o)) return GDN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, a, b, A_log, dt_bias, cu_seqlens, initial_state, final_state,
+                          o};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return GDN_ERR_MISALIGNED;
+    if (!workspace || workspace_bytes < gdn::prefill_min_workspace_bytes(n_seq, Hv))
+        return GDN_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GDN_ERR_MISALIGNED;
+    gdn::PrefillArgs p{q, k, v, a, b, A_log, dt_bias, cu_seqlens, n_seq, T, Hqk, Hv, scale,
+                       initial_state, final_state, nullptr, workspace, workspace_bytes};
+    p.o16 = o;
+    const PrefillKernel which = pick_prefill_kernel(workspace_bytes);
+    if (which == PrefillKernel::Unavailable) return GDN_ERR_UNSUPPORTED;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaMemsetAsync(workspace, 0, gdn::kWsHeaderBytes, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = which == PrefillKernel::ProducerConsumer ? gdn::launch_prefill_pc(p, s) : gdn::launch_prefill_tc(p, s);
+    return e == cudaSuccess ? GDN_OK : cuda_fail(e);
+}
+
 gdn_status gdn_prefill_gated(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* a,
                              const float* b, const float* A_log, const float* dt_bias,
                              const int32_t* cu_seqlens, int32_t n_seq, int64_t T, int32_t Hqk,

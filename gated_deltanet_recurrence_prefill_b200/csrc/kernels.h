@@ -24,7 +24,7 @@ struct PrefillArgs {
     float scale;
     const float* initial_state;    // may be NULL
     float* final_state;            // may be NULL
-    float* o;                      // may be NULL when y is given
+    float* o;                      // may be NULL when y or o16 is given
     void* workspace;
     size_t workspace_bytes;
     // fused gated output norm (producer / consumer kernel only): y = norm_w * o /
@@ -33,6 +33,7 @@ struct PrefillArgs {
     const float* norm_w = nullptr;
     float eps = 0.f;
     uint16_t* y = nullptr;
+    uint16_t* o16 = nullptr;       // o stored as bf16 instead of o (round to nearest even)
 };
 
 // the gated output norm fused into a decode step (y == NULL: none); norm_w is

@@ -257,6 +257,7 @@ struct ClParams {
     const float* norm_w;
     float eps;
     uint16_t* y;
+    uint16_t* o16;         // o as bf16 (instead of o)
 };
 
 struct Ctx {
@@ -584,6 +585,20 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
                         if (j < nvalid) ocol[j * o_stride] = ov[j];
+                }
+            } else if (p.o16) {
+                // bf16 o: lanes l and l ^ 1 hold rows v and v ^ 1; they swap one
+                // value per token pair so that each writes one 4-byte word of the
+                // two rows (even lanes the even tokens, odd lanes the odd ones)
+                const bool odd = lane & 1;
+                uint32_t* orow2 = reinterpret_cast<uint32_t*>(p.o16 + t0 * o_stride + x.h * kD + (v & ~1));
+                const int64_t wstride = o_stride / 2;
+#pragma unroll
+                for (int j = 0; j < 16; j += 2) {
+                    const float other = __shfl_xor_sync(0xffffffffu, odd ? ov[j] : ov[j + 1], 1);
+                    const int jt = odd ? j + 1 : j;
+                    const uint32_t w = odd ? pack_bf16x2(other, ov[j + 1]) : pack_bf16x2(ov[j], other);
+                    if (jt < nvalid) orow2[jt * wstride] = w;
                 }
             }
             Gam = resc ? 1.f : Gn;
@@ -1410,7 +1425,7 @@ cudaError_t launch_prefill_pc(const PrefillArgs& a, cudaStream_t stream) {
     ClParams p{a.a, a.b, a.A_log, a.dt_bias, a.cu_seqlens, a.T, a.Hqk, a.Hv, a.scale,
                a.initial_state, a.final_state, a.o,
                reinterpret_cast<uint32_t*>(ws + kWsErrorWordOffset), ring, flags, gate_tma, n_prod, 0,
-               a.z, a.norm_w, a.eps, a.y};
+               a.z, a.norm_w, a.eps, a.y, a.o16};
     // Units run in launches of at most per_launch units, in order; each launch
     // starts from cleared counters.  A unit's CTAs wait on one another, so each
     // launch is cooperative (all of its CTAs resident together).

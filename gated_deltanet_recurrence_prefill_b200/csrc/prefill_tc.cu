@@ -143,6 +143,7 @@ struct TcParams {
     float* o;
     uint32_t* err;
     int gate_tma;          // a, b staged by TMA (needs Hv % 4 == 0), else read directly
+    uint16_t* o16;         // o as bf16 (instead of o)
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -374,7 +375,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 // o_t = scale (O'_t + (Qh S^T)_t)
                 const int t = r;
                 const bool valid = tok0 + t < eos;
-                float* orow = p.o + ((tok0 + t) * p.Hv + h) * kD + v0;
+                const int64_t orow_off = ((tok0 + t) * p.Hv + h) * kD + v0;
                 for (int half = 0; half < 2; ++half) {
                     float op[32], qs[32];
                     tmem_ld32(tl + x2col + half * 32, op);
@@ -387,7 +388,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                             w.y = p.scale * (op[j + 1] + qs[j + 1]);
                             w.z = p.scale * (op[j + 2] + qs[j + 2]);
                             w.w = p.scale * (op[j + 3] + qs[j + 3]);
-                            *reinterpret_cast<float4*>(orow + half * 32 + j) = w;
+                            if (p.o16)
+                                *reinterpret_cast<uint2*>(p.o16 + orow_off + half * 32 + j) =
+                                    make_uint2(pack_bf16x2(w.x, w.y), pack_bf16x2(w.z, w.w));
+                            else
+                                *reinterpret_cast<float4*>(p.o + orow_off + half * 32 + j) = w;
                         }
                     }
                 }
@@ -776,7 +781,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t stream) {
     TcParams p{a.a, a.b, a.A_log, a.dt_bias, a.cu_seqlens, a.T, a.Hqk, a.Hv, a.scale,
                a.initial_state, a.final_state, a.o,
                reinterpret_cast<uint32_t*>(static_cast<char*>(a.workspace) + kWsErrorWordOffset),
-               gate_tma};
+               gate_tma, a.o16};
     const int64_t blocks = (int64_t)a.n_seq * a.Hv * (kD / kBV);
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     prefill_tc_kernel<<<(unsigned)blocks, kThreads, SMEM_ALLOC, stream>>>(mq, mk, mv, ma, mb, p);

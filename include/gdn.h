@@ -204,6 +204,25 @@ gdn_status gdn_prefill(const uint16_t* q, const uint16_t* k, const uint16_t* v, 
                        gdn_stream_t stream);
 
 /*
+ * gdn_prefill_bf16 -- gdn_prefill with the output o stored as bf16 (rounded to
+ * nearest even from the same float32 values) instead of float32: the bf16
+ * output variant.  The architecture page (section 2.2) puts the layer's state
+ * in float32 and gives a ~75 MB figure for the 48 layers' state at 2 bytes per
+ * element; o is the activation that leaves the recurrence, and halving its
+ * bytes cuts the prefill's algorithmic traffic from 45,440 to 33,152 bytes per
+ * token (16 / 48 heads, d = 128).  Arguments, layouts, ownership and errors as
+ * gdn_prefill, except
+ *  o  [T, Hv, d] bf16 (uint16 bits), written; 16-byte aligned.
+ * The state (initial_state, final_state) stays float32.
+ */
+gdn_status gdn_prefill_bf16(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* a,
+                            const float* b, const float* A_log, const float* dt_bias,
+                            const int32_t* cu_seqlens, int32_t n_seq, int64_t T, int32_t Hqk,
+                            int32_t Hv, int32_t d, float scale, const float* initial_state,
+                            float* final_state, uint16_t* o, void* workspace, size_t workspace_bytes,
+                            gdn_stream_t stream);
+
+/*
  * gdn_prefill_status -- waits for `stream`, then reads the error word that the
  * last gdn_prefill on this workspace left: GDN_OK, or GDN_ERR_TIMEOUT if a
  * bounded wait inside the kernel ran out (the outputs are then invalid).

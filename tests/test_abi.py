@@ -321,3 +321,18 @@ def test_check_async_rejects_bad_arguments(L):
     """gdn_check_async validates its output word before enqueueing anything."""
     assert L.gdn_check_async(_p(0x20000), None, None) == 1          # no status word
     assert L.gdn_check_async(_p(0x20000), _p(0x30002), None) == 3   # not 4-byte aligned
+
+
+def test_prefill_bf16_rejects_bad_arguments(L):
+    """gdn_prefill_bf16 checks its arguments as gdn_prefill does (no launch)."""
+    p = _p()
+    ws = _p(0x40000)
+    # no output
+    assert L.gdn_prefill_bf16(p, p, p, p, p, p, p, None, 1, 64, 16, 48, 128, 0.088, None, None, None,
+                              ws, 1 << 20, None) == 1
+    # unsupported head size
+    assert L.gdn_prefill_bf16(p, p, p, p, p, p, p, None, 1, 64, 16, 48, 64, 0.088, None, None, p,
+                              ws, 1 << 20, None) == 2
+    # misaligned output
+    assert L.gdn_prefill_bf16(p, p, p, p, p, p, p, None, 1, 64, 16, 48, 128, 0.088, None, None, _p(FAKE + 2),
+                              ws, 1 << 20, None) == 3
