@@ -894,6 +894,7 @@ def profile_case(args):
       decode16    gdn_decode_step, 16 sequences x 48 layers    (~2.4 GB of state)
       decode16bf  gdn_decode_step_bf16, the same units         (~1.2 GB of state)
       frontbw8k   gdn_conv1d_silu_backward, T=8192, history    (~1.3 GB)
+      bwc2k       gdn_prefill_backward_chunked, T=2048          (~0.6 GB with its workspace)
     """
     import numpy as np
     import torch
@@ -940,6 +941,16 @@ def profile_case(args):
         dv = torch.randn(T_MAIN, HV, D, generator=gen, device=dev)
         for _ in range(args.warmup + args.steps):
             gdn.conv1d_silu_backward(x, w, dq, dk, dv, HQK, HV, conv_state=cs)
+    elif args.profile_case == "bwc2k":
+        inp = synth.make_prefill([2048], 5, init_state=True)
+        d = [to16(inp.q), to16(inp.k), to16(inp.v), f32(inp.a), f32(inp.b), f32(inp.A_log), f32(inp.dt_bias)]
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(8)
+        d_o = torch.randn(2048, HV, D, generator=gen, device=dev)
+        d_fin = 0.1 * torch.randn(1, HV, D, D, generator=gen, device=dev)
+        s0 = f32(inp.initial_state)
+        for _ in range(args.warmup + args.steps):
+            gdn.prefill_backward_chunked(*d, d_o, d_final_state=d_fin, initial_state=s0)
     torch.cuda.synchronize()
     print(f"profile case {args.profile_case}: ok")
 
@@ -983,7 +994,7 @@ def main():
     ap.add_argument("--primary-only", action="store_true", help="skip the 262K and decode lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--profile-case", choices=["prefill8k", "frontend8k", "decode16", "decode16bf", "frontbw8k"],
+    ap.add_argument("--profile-case", choices=["prefill8k", "frontend8k", "decode16", "decode16bf", "frontbw8k", "bwc2k"],
                     help="run one kernel on a small case for an ncu capture; no timing")
     args = ap.parse_args()
     if args.warmup < 3:
