@@ -308,6 +308,7 @@ def bench_main(args, world, rank, local):
         extra["backward_T8192"] = bench_backward(args, dev, flush, peaks, world)
         extra["decode_128seq_48layers"] = bench_decode(args, dev, peaks, world)
         extra["decode_fused_128seq_48layers"] = bench_decode_fused(args, dev, peaks, world)
+        extra["decode_fused_bf16state_128seq_48layers"] = bench_decode_fused(args, dev, peaks, world, bf16_state=True)
         extra["decode_bf16state_128seq_48layers"] = bench_decode(args, dev, peaks, world, bf16_state=True)
         extra["decode_gated_128seq_48layers"] = bench_decode(args, dev, peaks, world, gated=True)
         if world == 1:
@@ -799,10 +800,10 @@ def bench_decode(args, dev, peaks, world, bf16_state=False, gated=False):
     return out
 
 
-def bench_decode_fused(args, dev, peaks, world):
+def bench_decode_fused(args, dev, peaks, world, bf16_state=False):
     """One fused decode step (front end + recurrence) for 128 sequences x 48
-    layers: 19.3 GB float32 state and 0.75 GB of convolution history in place
-    (inputs drawn on the device; far larger than L2)."""
+    layers: 19.3 GB float32 state (or 9.7 GB bf16 state) and 0.75 GB of
+    convolution history in place (inputs drawn on the device; far larger than L2)."""
     import torch
     import gated_deltanet_recurrence_prefill_b200 as gdn
     n_seq, L = 128, 48
@@ -818,7 +819,7 @@ def bench_decode_fused(args, dev, peaks, world):
     A_log = torch.log(torch.empty(L, HV, device=dev).uniform_(1, 16, generator=gen))
     dt = torch.exp(torch.empty(L, HV, device=dev).uniform_(-6.907755, -2.302585, generator=gen))
     dt_bias = torch.log(torch.expm1(dt))
-    state = torch.empty(U, HV, D, D, dtype=torch.float32, device=dev)
+    state = torch.empty(U, HV, D, D, dtype=torch.bfloat16 if bf16_state else torch.float32, device=dev)
     for i in range(0, U, 512):
         state[i:i + 512].normal_(0.0, 0.02, generator=gen)
     slot = torch.randperm(n_seq, generator=gen, device=dev).to(torch.int32)
@@ -837,11 +838,13 @@ def bench_decode_fused(args, dev, peaks, world):
     dummy = torch.empty(1, device=dev)
     times, _ = _time_steps(step, max(3, args.warmup), max(5, min(args.steps, 50)), dummy, mk, world)
     ms = _max_over_ranks(sum(times) / len(times), world)
-    bytes_step = (2 * U * STATE_BYTES + 2 * U * ctot * 3 * 4 + U * ctot * 2 + L * ctot * 16
+    state_bytes = STATE_BYTES // 2 if bf16_state else STATE_BYTES
+    bytes_step = (2 * U * state_bytes + 2 * U * ctot * 3 * 4 + U * ctot * 2 + L * ctot * 16
                   + U * HV * (2 * 4 + 4 * D))
     gbs = bytes_step / (ms * 1e-3) / 1e9
-    out = {"workload": "gdn_decode_step_fused 128 seq x 48 layers (front end fused), fp32 state "
-                       "19.33 GB + conv history 0.75 GB in place, shuffled slots",
+    wl = ("gdn_decode_step_fused_bf16 128 seq x 48 layers (front end fused), bf16 state 9.66 GB"
+          if bf16_state else "gdn_decode_step_fused 128 seq x 48 layers (front end fused), fp32 state 19.33 GB")
+    out = {"workload": wl + " + conv history 0.75 GB in place, shuffled slots",
            "ms": round(ms, 4), "GB_s": round(gbs, 1), "hbm_frac": round(gbs / peaks["hbm_gbs"], 4),
            "bytes_per_step": int(bytes_step), "launches_per_step": 1}
     del state, conv_state, qkv, o

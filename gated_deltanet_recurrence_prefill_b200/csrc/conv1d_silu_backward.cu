@@ -109,7 +109,9 @@ __global__ void __launch_bounds__(kWarpsF * 32) fbw_stream_kernel(Params p, int 
     float* dxp = p.dx + (t0 - 3) * Ctot + c0;       // d x of token t0 + tau - 3
     const uint16_t* xn = xs + kRingF * Ctot;          // the input kRingF tokens ahead
     const float* gn = gsrc + kRingF * dstride;
-#pragma unroll 1
+    // two tokens per iteration, so that the second token's forward overlaps the
+    // first one's reductions
+#pragma unroll 2
     for (int tau = 0; tau < kSpan; ++tau) {
         cp_wait<kRingF - 1>();
         const int slot = tau & (kRingF - 1);

@@ -237,17 +237,17 @@ BWC_FN void reduce_w_block(const Params& p, int64_t blk, int tid) {
     const int64_t Ctot = (int64_t)(2 * p.Hqk + p.Hv) * kD;
     const int64_t i = blk * kThreads + tid;
     if (i >= Ctot * 4) return;
-    // the partial sums are added in tile order; eight are loaded ahead of their
+    // the partial sums are added in tile order; 32 are loaded ahead of their
     // additions so that the loads overlap (the order of the additions, and so
     // the result, is the same)
     float s = 0.f;
     const float* src = p.dwp + i;
     const int64_t stride = Ctot * 4;
     int64_t tl = 0;
-    for (; tl + 8 <= p.n_tiles; tl += 8) {
-        float v[8];
-        for (int r = 0; r < 8; ++r) v[r] = src[(tl + r) * stride];
-        for (int r = 0; r < 8; ++r) s += v[r];
+    for (; tl + 32 <= p.n_tiles; tl += 32) {
+        float v[32];
+        for (int r = 0; r < 32; ++r) v[r] = src[(tl + r) * stride];
+        for (int r = 0; r < 32; ++r) s += v[r];
     }
     for (; tl < p.n_tiles; ++tl) s += src[tl * stride];
     p.dw[i] = s;

@@ -22,6 +22,7 @@
 #include "common.cuh"
 #include "decode_state.cuh"
 #include "kernels.h"
+#include "tc_util.cuh"
 
 namespace gdn {
 
@@ -68,7 +69,7 @@ decode_fused_kernel(const uint16_t* __restrict__ qkv, const float* __restrict__ 
                     const float* __restrict__ dt_bias, const int32_t* __restrict__ slot,
                     int32_t layers, int32_t Hqk, int32_t Hv, float scale, StateT* __restrict__ state,
                     float* __restrict__ o) {
-    __shared__ float qs[kD], ks[kD], vs[kD];
+    __shared__ __align__(16) float qs[kD], ks[kD], vs[kD];      // read as float4
     __shared__ float red[4];
     const int64_t ug = blockIdx.x;                 // unit * Hqk + key head
     const int64_t u = ug / Hqk;
@@ -161,6 +162,141 @@ decode_fused_kernel(const uint16_t* __restrict__ qkv, const float* __restrict__ 
     }
 }
 
+// bf16 state: the states of the key head's r value heads (r x 32 KiB, contiguous)
+// are brought into shared memory by one bulk copy issued first, so the copy
+// overlaps the front end's arithmetic and the bytes in flight come from shared
+// memory instead of registers; each value head's rows are then read from
+// shared memory and written back from registers.
+constexpr int kFusedBf16Rows = 8;
+constexpr uint64_t kFusedWaitLimitNs = 2000000000ull;      // 2 s
+
+__global__ void __launch_bounds__(kThreads, 2)
+decode_fused_bf16_smem_kernel(const uint16_t* __restrict__ qkv, const float* __restrict__ conv_w,
+                              float* __restrict__ conv_state, const float* __restrict__ a,
+                              const float* __restrict__ b, const float* __restrict__ A_log,
+                              const float* __restrict__ dt_bias, const int32_t* __restrict__ slot,
+                              int32_t layers, int32_t Hqk, int32_t Hv, float scale, uint16_t* __restrict__ state,
+                              float* __restrict__ o) {
+    extern __shared__ __align__(128) uint8_t tiles[];          // r states of 128 x 128 bf16
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ __align__(16) float qs[kD], ks[kD], vs[kD];      // read as float4
+    __shared__ float red[4];
+    __shared__ int abort_flag;
+    const int64_t ug = blockIdx.x;                 // unit * Hqk + key head
+    const int64_t u = ug / Hqk;
+    const int g = (int)(ug - u * Hqk);
+    const int64_t n = u / layers;
+    const int l = (int)(u - n * layers);
+    const int64_t su = (int64_t)(slot ? slot[n] : n) * layers + l;      // state unit of (slot, layer)
+    const int r = Hv / Hqk;                        // value heads per key head
+    const int64_t Ctot = (int64_t)(2 * Hqk + Hv) * kD;
+    const int t = threadIdx.x;
+    const int lane = t & 31, warp = t >> 5;
+    uint16_t* S0 = state + (su * Hv + (int64_t)g * r) * (int64_t)(kD * kD);
+    const uint32_t tile_bytes = (uint32_t)r * kD * kD * 2;
+    const uint32_t bar_a = tc::smem_u32(&bar);
+    if (t == 0) {
+        abort_flag = 0;
+        tc::mbar_init(bar_a, 1);
+        tc::fence_mbar_init();
+        tc::mbar_arrive_expect_tx(bar_a, tile_bytes);
+        tc::bulk_load(tc::smem_u32(tiles), S0, tile_bytes, bar_a);
+    }
+
+    const uint16_t* xrow = qkv + u * Ctot;
+    const float* wl = conv_w + (int64_t)l * Ctot * 4;
+    float* csu = conv_state + su * Ctot * 3;
+
+    // ---- q and k of key head g: channel t of each
+    {
+        const int64_t cq = (int64_t)g * kD + t, ck = (int64_t)(Hqk + g) * kD + t;
+        float csq[3], csk[3];
+        for (int j = 0; j < 3; ++j) { csq[j] = csu[cq * 3 + j]; csk[j] = csu[ck * 3 + j]; }
+        const float yq = conv_channel(bf16_to_f32(xrow[cq]), csq, wl + cq * 4);
+        const float yk = conv_channel(bf16_to_f32(xrow[ck]), csk, wl + ck * 4);
+        for (int j = 0; j < 3; ++j) { csu[cq * 3 + j] = csq[j]; csu[ck * 3 + j] = csk[j]; }
+        const float nq = block_sum(yq * yq, red);
+        const float nk = block_sum(yk * yk, red);
+        qs[t] = yq * rsqrtf(nq + 1e-6f);
+        ks[t] = yk * rsqrtf(nk + 1e-6f);
+    }
+    __syncthreads();
+    const float4 k4 = *reinterpret_cast<const float4*>(ks + lane * 4);
+    const float4 q4 = *reinterpret_cast<const float4*>(qs + lane * 4);
+    const float kq = warp_sum(k4.x * q4.x + k4.y * q4.y + k4.z * q4.z + k4.w * q4.w);
+    // the states have landed (bounded: on expiry the outputs of this key head's
+    // value heads become NaN, the states are left as they were, and the copy is
+    // waited for again, bounded, before the CTA exits)
+    const bool landed = tc::mbar_wait(bar_a, 0, &abort_flag, kFusedWaitLimitNs);
+
+    for (int j = 0; j < r; ++j) {
+        const int h = g * r + j;
+        // ---- v of value head h: channel t (the conv history advances either way)
+        {
+            const int64_t cv = (int64_t)(2 * Hqk + h) * kD + t;
+            float csv[3];
+            for (int m = 0; m < 3; ++m) csv[m] = csu[cv * 3 + m];
+            const float yv = conv_channel(bf16_to_f32(xrow[cv]), csv, wl + cv * 4);
+            for (int m = 0; m < 3; ++m) csu[cv * 3 + m] = csv[m];
+            __syncthreads();                       // the previous head's rows are done with vs
+            vs[t] = yv;
+            __syncthreads();
+        }
+        const int64_t uh = u * Hv + h;
+        float* oh = o + uh * kD;
+        if (!landed) {
+            oh[t] = __int_as_float(0x7fc00000);
+            continue;
+        }
+        const float alpha = expf(log_alpha_f32(a[uh], A_log[(int64_t)l * Hv + h], dt_bias[(int64_t)l * Hv + h]));
+        const float beta = sigmoid_f32(b[uh]);
+        uint16_t* S = S0 + (int64_t)j * (kD * kD);
+        const uint2* tile = reinterpret_cast<const uint2*>(tiles + (size_t)j * kD * kD * 2);
+#pragma unroll 1
+        for (int r0 = warp * 32; r0 < warp * 32 + 32; r0 += kFusedBf16Rows) {
+            float4 sr[kFusedBf16Rows];
+#pragma unroll
+            for (int i = 0; i < kFusedBf16Rows; ++i) {
+                const uint2 w2 = tile[(r0 + i) * (kD / 4) + lane];
+                const float2 x0 = bf16x2_to_f32x2(w2.x), x1 = bf16x2_to_f32x2(w2.y);
+                sr[i] = make_float4(x0.x, x0.y, x1.x, x1.y);
+            }
+            float xk[kFusedBf16Rows], xq[kFusedBf16Rows];
+#pragma unroll
+            for (int i = 0; i < kFusedBf16Rows; ++i) {
+                xk[i] = sr[i].x * k4.x + sr[i].y * k4.y + sr[i].z * k4.z + sr[i].w * k4.w;
+                xq[i] = sr[i].x * q4.x + sr[i].y * q4.y + sr[i].z * q4.z + sr[i].w * q4.w;
+            }
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) {
+#pragma unroll
+                for (int i = 0; i < kFusedBf16Rows; ++i) {
+                    xk[i] += __shfl_xor_sync(0xffffffffu, xk[i], m);
+                    xq[i] += __shfl_xor_sync(0xffffffffu, xq[i], m);
+                }
+            }
+            float orow = 0.f;
+#pragma unroll
+            for (int i = 0; i < kFusedBf16Rows; ++i) {
+                const float w = beta * (vs[r0 + i] - alpha * xk[i]);
+                float4 nv;
+                nv.x = fmaf(alpha, sr[i].x, w * k4.x);
+                nv.y = fmaf(alpha, sr[i].y, w * k4.y);
+                nv.z = fmaf(alpha, sr[i].z, w * k4.z);
+                nv.w = fmaf(alpha, sr[i].w, w * k4.w);
+                state_store4(S + (int64_t)(r0 + i) * kD, lane, nv);
+                const float oi = scale * fmaf(alpha, xq[i], w * kq);
+                if (lane == i) orow = oi;
+            }
+            if (lane < kFusedBf16Rows) oh[r0 + lane] = orow;
+        }
+    }
+    if (!landed) {
+        volatile int no_abort = 0;
+        tc::mbar_wait(bar_a, 0, &no_abort, kFusedWaitLimitNs);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_decode_fused(const uint16_t* qkv, const float* conv_w, float* conv_state,
@@ -184,7 +320,18 @@ cudaError_t launch_decode_fused_bf16(const uint16_t* qkv, const float* conv_w, f
     const int64_t blocks = (int64_t)n_seq * layers * Hqk;
     if (blocks == 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    decode_fused_kernel<uint16_t><<<(unsigned)blocks, kThreads, 0, stream>>>(
+    const int r = Hv / Hqk;
+    const size_t smem = (size_t)r * kD * kD * 2;
+    if (smem > 200 * 1024) {
+        // more value heads per key head than the staged kernel holds: the register kernel
+        decode_fused_kernel<uint16_t><<<(unsigned)blocks, kThreads, 0, stream>>>(
+            qkv, conv_w, conv_state, a, b, A_log, dt_bias, slot, layers, Hqk, Hv, scale, state, o);
+        return cudaGetLastError();
+    }
+    cudaError_t e = cudaFuncSetAttribute(decode_fused_bf16_smem_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    decode_fused_bf16_smem_kernel<<<(unsigned)blocks, kThreads, smem, stream>>>(
         qkv, conv_w, conv_state, a, b, A_log, dt_bias, slot, layers, Hqk, Hv, scale, state, o);
     return cudaGetLastError();
 }
