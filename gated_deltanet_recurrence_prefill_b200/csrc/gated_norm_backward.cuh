@@ -78,6 +78,33 @@ BWC_FN float bf16f(uint16_t h) {
 #endif
 }
 
+// four consecutive floats / bf16 values of a row (16- / 8-byte aligned): one
+// vector access on the GPU
+BWC_FN void ld4f(const float* src, float* v) {
+#ifdef __CUDA_ARCH__
+    const float4 t = *reinterpret_cast<const float4*>(src);
+    v[0] = t.x; v[1] = t.y; v[2] = t.z; v[3] = t.w;
+#else
+    memcpy(v, src, 4 * sizeof(float));
+#endif
+}
+BWC_FN void st4f(float* dst, const float* v) {
+#ifdef __CUDA_ARCH__
+    *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+#else
+    memcpy(dst, v, 4 * sizeof(float));
+#endif
+}
+BWC_FN void ld4bf(const uint16_t* src, float* v) {
+#ifdef __CUDA_ARCH__
+    const uint2 t = *reinterpret_cast<const uint2*>(src);
+    v[0] = __uint_as_float(t.x << 16); v[1] = __uint_as_float(t.x & 0xFFFF0000u);
+    v[2] = __uint_as_float(t.y << 16); v[3] = __uint_as_float(t.y & 0xFFFF0000u);
+#else
+    for (int i = 0; i < 4; ++i) v[i] = bf16f(src[i]);
+#endif
+}
+
 BWC_FN void rows_block(const Params& p, int64_t tile, int hg, int tid, float* sm) {
     float* red = sm;                  // [warp][token][element]: each warp's weight gradient
     const int warp = tid >> 5, lane = tid & 31;
@@ -88,6 +115,13 @@ BWC_FN void rows_block(const Params& p, int64_t tile, int hg, int tid, float* sm
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[j][i] = 0.f;
     if (h < p.Hv) {                                       // the same for every lane of the warp
+        // restrict-qualified copies: the stores of one token do not order the
+        // next token's loads behind them
+        const float* __restrict__ po = p.o;
+        const uint16_t* __restrict__ pz = p.z;
+        const float* __restrict__ pdy = p.dy;
+        float* __restrict__ pdo = p.d_o;
+        float* __restrict__ pdz = p.d_z;
 #pragma unroll
         for (int j = 0; j < kTok; ++j) {
             const int64_t t = tile * kTok + j;
@@ -96,11 +130,11 @@ BWC_FN void rows_block(const Params& p, int64_t tile, int hg, int tid, float* sm
             const float* wl = p.w + (int64_t)(t % p.layers) * kD + lane * 4;
             float o[4], z[4], dy[4], w[4], sg[4], u[4];
             float ss = 0.f, ou = 0.f;
+            ld4f(po + row, o);
+            ld4bf(pz + row, z);
+            ld4f(pdy + row, dy);
+            ld4f(wl, w);
             for (int i = 0; i < 4; ++i) {
-                o[i] = p.o[row + i];
-                z[i] = bf16f(p.z[row + i]);
-                dy[i] = p.dy[row + i];
-                w[i] = wl[i];
                 sg[i] = 1.f / (1.f + expf(-z[i]));
                 u[i] = w[i] * z[i] * sg[i] * dy[i];
                 ss = fmaf(o[i], o[i], ss);
@@ -111,11 +145,14 @@ BWC_FN void rows_block(const Params& p, int64_t tile, int hg, int tid, float* sm
                 ou += BWC_SHFL_XOR(ou, m);
             }
             const float r = 1.f / sqrtf(ss / kD + p.eps);
+            float dov[4], dzv[4];
             for (int i = 0; i < 4; ++i) {
-                p.d_o[row + i] = r * u[i] - r * r * r / kD * o[i] * ou;
-                p.d_z[row + i] = dy[i] * w[i] * r * o[i] * sg[i] * (1.f + z[i] * (1.f - sg[i]));
+                dov[i] = r * u[i] - r * r * r / kD * o[i] * ou;
+                dzv[i] = dy[i] * w[i] * r * o[i] * sg[i] * (1.f + z[i] * (1.f - sg[i]));
                 acc[j][i] = dy[i] * r * o[i] * (z[i] * sg[i]);
             }
+            st4f(pdo + row, dov);
+            st4f(pdz + row, dzv);
         }
     }
 #pragma unroll
