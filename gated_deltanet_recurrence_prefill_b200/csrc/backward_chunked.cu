@@ -6,10 +6,15 @@
 //   3. forward chain, kRowSplit CTAs per (sequence, value head): S_c;
 //   4. backward chain, likewise: dS_c and dL/dS_0;
 //   5. gradients, one CTA per (chunk, value head): dq, dk (per value head), dv,
-//      da, db and per-chunk sums for the gate parameters;
+//      da, db and per-chunk sums for the gate parameters -- on the tensor cores
+//      (backward_chunked_tc.cu) unless GDN_BACKWARD_GRAD=simt selects the
+//      float32 CUDA-core block function below;
 //   6. sums over each key head's value heads and over chunks.
 // Every CTA has 256 threads; 2, 3 and 5 take almost all of an SM's shared
 // memory, 4 about half.
+#include <stdlib.h>
+#include <string.h>
+
 #include "backward_chunked.cuh"
 #include "kernels.h"
 
@@ -59,7 +64,15 @@ cudaError_t launch_smem(K kernel, int64_t blocks, int floats, const Params& p, c
     return cudaGetLastError();
 }
 
+// GDN_BACKWARD_GRAD=simt: the float32 CUDA-core gradient kernel
+bool grad_on_cuda_cores() {
+    const char* env = getenv("GDN_BACKWARD_GRAD");
+    return env && strcmp(env, "simt") == 0;
+}
+
 }  // namespace
+
+cudaError_t launch_backward_grad_tc(const Params& p, int64_t jobs, cudaStream_t s);
 
 size_t backward_chunked_workspace_bytes(int32_t n_seq, int64_t T, int32_t Hv) {
     return make_plan(n_seq, T, Hv).bytes;
@@ -77,7 +90,8 @@ cudaError_t launch_backward_chunked(const BackwardArgs& a, cudaStream_t s) {
     bind_workspace(p, a.workspace, plan);
     const int64_t jobs = plan.n_slots * a.Hv;
     const int64_t chains = (int64_t)a.n_seq * a.Hv * kRowSplit;
-    cudaError_t e = cudaMemsetAsync(p.jobs, 0xFF, (size_t)plan.n_slots * 2 * sizeof(int32_t), s);
+    cudaError_t e = cudaMemsetAsync(p.err, 0, plan.jobs - plan.err, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(p.jobs, 0xFF, (size_t)plan.n_slots * 2 * sizeof(int32_t), s);
     if (e == cudaSuccess) {
         bwc_jobs_kernel<<<(unsigned)a.n_seq, kThreads, 0, s>>>(p);
         e = cudaGetLastError();
@@ -85,7 +99,9 @@ cudaError_t launch_backward_chunked(const BackwardArgs& a, cudaStream_t s) {
     if (e == cudaSuccess) e = launch_smem(bwc_prep_kernel, jobs, kPrepFloats, p, s);
     if (e == cudaSuccess) e = launch_smem(bwc_fwd_chain_kernel, chains, kChainFloats, p, s);
     if (e == cudaSuccess) e = launch_smem(bwc_bwd_chain_kernel, chains, kChainFloats, p, s);
-    if (e == cudaSuccess) e = launch_smem(bwc_grad_kernel, jobs, kGradFloats, p, s);
+    if (e == cudaSuccess)
+        e = grad_on_cuda_cores() ? launch_smem(bwc_grad_kernel, jobs, kGradFloats, p, s)
+                                 : launch_backward_grad_tc(p, jobs, s);
     const int64_t n = a.T * a.Hqk * kD;
     if (e == cudaSuccess && n > 0) {
         bwc_reduce_qk_kernel<<<(unsigned)((n + kThreads - 1) / kThreads), kThreads, 0, s>>>(p);

@@ -65,6 +65,8 @@ constexpr int kLt = kC + 4;
 constexpr int kLu = kRows + 4;
 
 // ---- workspace plan ----------------------------------------------------------------
+// A 256-byte header holding the error word (uint32 at offset 0, 0 = ok: the
+// tensor-core gradient kernel sets it when a bounded wait gives up).
 // Per (chunk slot, value head): W, U' [64 x 128], T [64 x 64], Y, S_c, dS_c
 // [128 x 128], kap and gam_{L-1} [65]; per token and value head: dq, dk before
 // the sum over each key head's value heads; per (slot, head) two gate sums.
@@ -72,7 +74,7 @@ constexpr int kLu = kRows + 4;
 // most T / 64 + n_seq + 1 slots).
 struct Plan {
     int64_t n_slots;
-    size_t jobs, W, Up, T, Y, S, dS, G, dqh, dkh, gpart, bytes;
+    size_t err, jobs, W, Up, T, Y, S, dS, G, dqh, dkh, gpart, bytes;
 };
 
 BWC_HD size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -82,6 +84,7 @@ BWC_HD Plan make_plan(int32_t n_seq, int64_t T, int32_t Hv) {
     p.n_slots = T / kC + n_seq + 1;
     const size_t sh = (size_t)p.n_slots * Hv;
     size_t off = 0;
+    p.err = off;  off = 256;
     p.jobs = off; off = align256(off + (size_t)p.n_slots * 2 * sizeof(int32_t));
     p.W = off;    off = align256(off + sh * kC * kD * sizeof(float));
     p.Up = off;   off = align256(off + sh * kC * kD * sizeof(float));
@@ -114,6 +117,7 @@ struct Params {
     int64_t T, n_slots;
     float scale;
     // workspace (see Plan)
+    uint32_t* err;              // error word (0 = ok)
     int32_t* jobs;              // per slot: sequence (-1: unused) and first token
     float *W, *Up, *Tm, *Y, *S, *dS, *G, *dqh, *dkh, *gpart;
     // outputs
@@ -124,6 +128,7 @@ struct Params {
 BWC_HD void bind_workspace(Params& p, void* ws, const Plan& plan) {
     char* base = static_cast<char*>(ws);
     p.n_slots = plan.n_slots;
+    p.err = reinterpret_cast<uint32_t*>(base + plan.err);
     p.jobs = reinterpret_cast<int32_t*>(base + plan.jobs);
     p.W = reinterpret_cast<float*>(base + plan.W);
     p.Up = reinterpret_cast<float*>(base + plan.Up);

@@ -440,7 +440,8 @@ gdn_status gdn_prefill_backward(const uint16_t* q, const uint16_t* k, const uint
 
 /*
  * gdn_prefill_backward_chunked_workspace_size -- bytes of device workspace
- * gdn_prefill_backward_chunked needs (a multiple of 256).  With
+ * gdn_prefill_backward_chunked needs (a multiple of 256).  A 256-byte header
+ * whose first word is the error word (as in the prefill's workspace); with
  * slots = T / 64 + n_seq + 1: per (slot, value head) W and U' (2 * 64 * d
  * floats), T (64 * 64), Y, the chunk-start state and the chunk-end gradient
  * (3 * d * d) and 65 decay floats; dq and dk per value head (2 * T * Hv * d
@@ -457,10 +458,19 @@ size_t gdn_prefill_backward_chunked_workspace_size(int32_t n_seq, int64_t T, int
  * instead of one over tokens: the chunk-start states, and the gradient at each
  * chunk end, dS_{c-1} = gam dS_c - (diag(kap) K dS_c^T)^T W + Y_c, whose
  * state-free term Y_c is computed for all chunks at once; everything else (dq,
- * dk, dv, the gates) is computed per (chunk, value head) in parallel.  Float32
- * arithmetic on CUDA cores, no atomics: the result is deterministic.
+ * dk, dv, the gates) is computed per (chunk, value head) in parallel.  The
+ * chains and the per-chunk preparation run in float32 on the CUDA cores; the
+ * per-chunk gradient step runs its products on the tensor cores (tcgen05, bf16
+ * operands, float32 accumulation; the bf16 tensor-core prefill's tolerance,
+ * 1e-2 relative to the largest reference element, applies), or in float32 on
+ * the CUDA cores when the environment variable GDN_BACKWARD_GRAD=simt is set
+ * (2e-3).  No atomics: the result is deterministic.
  * Arguments, layouts, outputs and errors as for gdn_prefill_backward, with the
- * workspace sized by gdn_prefill_backward_chunked_workspace_size().
+ * workspace sized by gdn_prefill_backward_chunked_workspace_size().  The
+ * tensor-core step waits (bounded, 2 s) for its products; if a wait gives up
+ * it sets the workspace's error word, which gdn_prefill_status and
+ * gdn_check_async read, and its outputs are not valid.  The call clears the
+ * word first.
  */
 gdn_status gdn_prefill_backward_chunked(const uint16_t* q, const uint16_t* k, const uint16_t* v, const float* a,
                                         const float* b, const float* A_log, const float* dt_bias,

@@ -230,13 +230,14 @@ def test_backward_rejects_bad_arguments(L):
 
 
 def test_chunked_backward_workspace_formula(L):
-    # gdn.h: per (slot, value head) W, U', T, Y, S, dS and the decays; dq, dk per
-    # value head; the chunk list and gate sums, each region rounded to 256 bytes
+    # gdn.h: a 256-byte header (the error word); per (slot, value head) W, U',
+    # T, Y, S, dS and the decays; dq, dk per value head; the chunk list and gate
+    # sums, each region rounded to 256 bytes
     r = lambda x: (x + 255) // 256 * 256
     for n, T, Hv in ((1, 8192, 48), (16, 241567, 48), (3, 100, 6)):
         d = 128
         sh = (T // 64 + n + 1) * Hv
-        want = (r((T // 64 + n + 1) * 2 * 4) + 2 * r(sh * 64 * d * 4) + r(sh * 64 * 64 * 4)
+        want = (256 + r((T // 64 + n + 1) * 2 * 4) + 2 * r(sh * 64 * d * 4) + r(sh * 64 * 64 * 4)
                 + 3 * r(sh * d * d * 4) + r(sh * 65 * 4) + 2 * r(T * Hv * d * 4) + r(sh * 2 * 4))
         assert L.gdn_prefill_backward_chunked_workspace_size(n, T, Hv, d) == want
 

@@ -1,6 +1,13 @@
 """gdn_prefill_backward_chunked against the fp64 oracle's gradient, on the
-shapes of the token-by-token backward's tests.  Float32 arithmetic as in the
-token-by-token kernel; max |x - x_ref| / max |x_ref| <= 2e-3.
+shapes of the token-by-token backward's tests, with each of its two gradient
+kernels:
+  * tc (the default): the per-chunk products on the tensor cores with bf16
+    operands and float32 accumulation; the tolerance of the bf16 tensor-core
+    prefill, max |x - x_ref| / max |x_ref| <= 1e-2 (a float32 model of the
+    chunked backward with every product operand rounded to bf16 stays at
+    ~5e-3 against the oracle, so 1e-2 holds with room);
+  * simt (GDN_BACKWARD_GRAD=simt): float32 on the CUDA cores, <= 2e-3 as for
+    the token-by-token kernel.
 
 (Its kernels' source is also run on the CPU under emulation by
 test_backward_chunked_emu; this file runs after every other GPU test.)"""
@@ -11,7 +18,16 @@ import synth
 from tests.helpers import dev_bf16, dev_f32, dev_i32, host, rel_err
 
 pytestmark = pytest.mark.gpu
-TOL = 2e-3
+TOLS = {"tc": 1e-2, "simt": 2e-3}
+
+
+@pytest.fixture(params=sorted(TOLS))
+def tol(request, monkeypatch):
+    if request.param == "simt":
+        monkeypatch.setenv("GDN_BACKWARD_GRAD", "simt")
+    else:
+        monkeypatch.delenv("GDN_BACKWARD_GRAD", raising=False)
+    return TOLS[request.param]
 
 
 def _grads_in(inp, seed):
@@ -32,35 +48,35 @@ def _run(inp, d_o, d_fin, with_s0=True, chunked=True):
               scale=inp.scale, initial_state=s0)
 
 
-def _compare(got, ref):
+def _compare(got, ref, tol):
     pairs = [("dq", "dq"), ("dk", "dk"), ("dv", "dv"), ("da", "da"), ("db", "db"), ("dA_log", "dA_log"),
              ("ddt_bias", "ddt_bias"), ("d_initial_state", "d_initial")]
     for gname, rname in pairs:
         if got[gname] is None:
             continue
         err = rel_err(host(got[gname]), ref[rname])
-        assert err <= TOL, f"{gname}: {err}"
+        assert err <= tol, f"{gname}: {err}"
 
 
 @pytest.mark.parametrize("Hqk,Hv", [(2, 6), (4, 12)])
-def test_chunked_backward_varlen(orc, Hqk, Hv):
+def test_chunked_backward_varlen(orc, tol, Hqk, Hv):
     lengths = [1, 63, 64, 0, 65, 130]
     inp = synth.make_prefill(lengths, seed=80, init_state=True, init_std=0.05, Hqk=Hqk, Hv=Hv)
     d_o, d_fin = _grads_in(inp, 1)
     ref = orc.prefill_backward(inp.q, inp.k, inp.v, inp.a, inp.b, inp.A_log, inp.dt_bias, d_o, d_final=d_fin,
                                cu_seqlens=inp.cu_seqlens, scale=inp.scale, initial_state=inp.initial_state)
-    _compare(_run(inp, d_o, d_fin), ref)
+    _compare(_run(inp, d_o, d_fin), ref, tol)
 
 
-def test_chunked_backward_no_state_gradients(orc):
+def test_chunked_backward_no_state_gradients(orc, tol):
     inp = synth.make_prefill([150, 20], seed=81, init_state=False, Hqk=2, Hv=6)
     d_o, _ = _grads_in(inp, 2)
     ref = orc.prefill_backward(inp.q, inp.k, inp.v, inp.a, inp.b, inp.A_log, inp.dt_bias, d_o,
                                cu_seqlens=inp.cu_seqlens, scale=inp.scale)
-    _compare(_run(inp, d_o, None, with_s0=False), ref)
+    _compare(_run(inp, d_o, None, with_s0=False), ref, tol)
 
 
-def test_chunked_backward_deterministic_and_equal_to_token_by_token():
+def test_chunked_backward_deterministic_and_equal_to_token_by_token(tol):
     import torch
     inp = synth.make_prefill([200, 37], seed=82, init_state=True, Hqk=2, Hv=6)
     d_o, d_fin = _grads_in(inp, 3)
@@ -70,10 +86,10 @@ def test_chunked_backward_deterministic_and_equal_to_token_by_token():
     g3 = _run(inp, d_o, d_fin, chunked=False)
     for name in g1:
         x, r = host(g1[name]), host(g3[name])
-        assert rel_err(x, r) <= TOL, name
+        assert rel_err(x, r) <= tol, name
 
 
-def test_chunked_backward_2k_full_heads_sampled(orc):
+def test_chunked_backward_2k_full_heads_sampled(orc, tol):
     # 2048 tokens with the full 16 / 48 heads in one call; two value heads (with
     # their key heads) against the oracle on those heads alone
     inp = synth.make_prefill([2048], seed=83, init_state=True)
@@ -91,10 +107,10 @@ def test_chunked_backward_2k_full_heads_sampled(orc):
         gk = h // 3
         ref = one_head(h)
         for gname, rname in (("dv", "dv"), ("da", "da"), ("db", "db"), ("d_initial_state", "d_initial")):
-            assert rel_err(got[gname][:, h:h + 1], ref[rname]) <= TOL, (h, gname)
+            assert rel_err(got[gname][:, h:h + 1], ref[rname]) <= tol, (h, gname)
         for gname in ("dA_log", "ddt_bias"):
-            assert rel_err(got[gname][h:h + 1], ref[gname]) <= TOL, (h, gname)
+            assert rel_err(got[gname][h:h + 1], ref[gname]) <= tol, (h, gname)
         # dq, dk of key head gk sum its three value heads
         refs = [ref if hh == h else one_head(hh) for hh in range(3 * gk, 3 * gk + 3)]
-        assert rel_err(got["dq"][:, gk:gk + 1], sum(r["dq"] for r in refs)) <= TOL, h
-        assert rel_err(got["dk"][:, gk:gk + 1], sum(r["dk"] for r in refs)) <= TOL, h
+        assert rel_err(got["dq"][:, gk:gk + 1], sum(r["dq"] for r in refs)) <= tol, h
+        assert rel_err(got["dk"][:, gk:gk + 1], sum(r["dk"] for r in refs)) <= tol, h
