@@ -77,7 +77,9 @@ enum : int {
     F_CSA = 1024,     // column sums of dA o beta A'
     F_RED = 1088,     // [256]    block reduction
     F_SS = 1344,      // <dS, S>
-    F_END = 1352
+    F_SIG = 1352,     // sigmoid(a + dt_bias) per row
+    F_XCH = 1416,     // [16] exchange between the two gate warps
+    F_END = 1432
 };
 constexpr uint32_t S_MISC = S_TILES;
 constexpr uint32_t S_BAR = S_MISC + F_END * 4;      // mbarrier (8), TMEM base (4), abort flag (4)
@@ -180,8 +182,38 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
         fence_mbar_init();
         *abort_flag = 0;
     }
-    // gates (ends with a barrier, which also publishes the TMEM base and the mbarrier)
-    chunk_gates(p, h, t0, L, tid, lg, be, G, gam, kap);
+    // gates (warps 0-1, one row each): log alpha, beta, G = running sum of log
+    // alpha (an inclusive scan; rows >= L add 0, so they carry G_{L-1}), gamma,
+    // kappa, and sigmoid(a + dt_bias) for d a
+    if (tid < kC) {
+        const int r = tid;
+        float la = 0.f, bb = 0.f, sg = 0.f;
+        if (r < L) {
+            const int64_t t = t0 + r;
+            const float av = p.a[t * p.Hv + h], dtb = p.dt_bias[h];
+            la = log_alpha(av, p.A_log[h], dtb);
+            bb = sigmoid(p.b[t * p.Hv + h]);
+            sg = sigmoid(av + dtb);
+        }
+        float run = la;
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) {
+            const float o = __shfl_up_sync(0xffffffffu, run, m);
+            if (lane >= m) run += o;
+        }
+        if (r == 31) F[F_XCH] = run;
+        named_bar_sync(1, kC);
+        if (r >= 32) run += F[F_XCH];
+        lg[r] = la;
+        be[r] = bb;
+        G[r] = run;
+        gam[r] = expf(run);
+        F[F_SIG + r] = sg;
+        named_bar_sync(1, kC);
+        kap[r] = r < L ? expf(G[L - 1] - run) : 0.f;
+    }
+    // (this barrier also publishes the TMEM base and the mbarrier)
+    __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_slot;
     const bool issuer = tid == 0;
@@ -647,40 +679,53 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
                 }
             }
         }
-        // the gates: per row, then the suffix sums over the chunk
-        float* dGv = F + F_RED;
-        float* dbe = F + F_RED + 64;
-        float* kdk = F + F_RED + 128;
-        if (tid < 64) {
+        // the gates (warps 0-1, one row each): dG per row, then
+        // d log alpha_m = sum_{i >= m} dG_i (a suffix scan), d a, d b, and the
+        // chunk's sums for dA_log and ddt_bias (fixed reduction order)
+        if (tid < kC) {
             const int r = tid;
             const float dkap = F[F_DKAP + r] + F[F_DKAP + 64 + r];
             const float sk = F[F_SKT + r];
             const float dgam = scale * (F[F_DGAM + r] + F[F_DGAM + 64 + r]) + be[r] * sk +
                                (r == L - 1 ? F[F_SS] : 0.f);
             const float rsa = F[F_RSA + r] + F[F_RSA + 64 + r];
-            dbe[r] = F[F_DBET + r] + gam[r] * sk + rsa;
-            dGv[r] = (F[F_RSM + r] + F[F_RSM + 64 + r] - F[F_CSM + r]) + (be[r] * rsa - F[F_CSA + r]) +
-                     gam[r] * dgam - kap[r] * dkap;
-            kdk[r] = kap[r] * dkap;
-        }
-        __syncthreads();
-        if (tid == 0) {
-            float ks = 0.f;
-            for (int r = 0; r < L; ++r) ks += kdk[r];
-            dGv[L - 1] += ks;
-            const float eA = expf(p.A_log[h]), dtb = p.dt_bias[h];
-            float suf = 0.f, gA = 0.f, gD = 0.f;
-            for (int m = L - 1; m >= 0; --m) {
-                suf += dGv[m];
-                const int64_t t = t0 + m;
-                const float dat = suf * (-eA * sigmoid(p.a[t * p.Hv + h] + dtb));
-                p.da[t * p.Hv + h] = dat;
-                p.db[t * p.Hv + h] = dbe[m] * be[m] * (1.f - be[m]);
-                gA = fmaf(suf, lg[m], gA);
-                gD += dat;
+            const float dbe = F[F_DBET + r] + gam[r] * sk + rsa;
+            float dG = (F[F_RSM + r] + F[F_RSM + 64 + r] - F[F_CSM + r]) + (be[r] * rsa - F[F_CSA + r]) +
+                       gam[r] * dgam - kap[r] * dkap;
+            // sum over the chunk of kappa dkappa (rows >= L have kappa = 0) joins dG_{L-1}
+            float kd = warp_sum(kap[r] * dkap);
+            if (lane == 0) F[F_XCH + 2 + (r >> 5)] = kd;
+            named_bar_sync(1, kC);
+            if (r == L - 1) dG += F[F_XCH + 2] + F[F_XCH + 3];
+            if (r >= L) dG = 0.f;
+            // suffix scan (rows 63 .. 0): within the warp, then warp 0 adds warp 1's total
+            float suf = dG;
+#pragma unroll
+            for (int m = 1; m < 32; m <<= 1) {
+                const float o = __shfl_down_sync(0xffffffffu, suf, m);
+                if (lane + m < 32) suf += o;
             }
-            p.gpart[sh * 2 + 0] = gA;
-            p.gpart[sh * 2 + 1] = gD;
+            if (r == 32) F[F_XCH + 4] = suf;
+            named_bar_sync(1, kC);
+            if (r < 32) suf += F[F_XCH + 4];
+            const float eA = expf(p.A_log[h]);
+            const float dat = r < L ? suf * (-eA * F[F_SIG + r]) : 0.f;
+            if (r < L) {
+                const int64_t t = t0 + r;
+                p.da[t * p.Hv + h] = dat;
+                p.db[t * p.Hv + h] = dbe * be[r] * (1.f - be[r]);
+            }
+            const float gA = warp_sum(r < L ? suf * lg[r] : 0.f);
+            const float gD = warp_sum(dat);
+            if (lane == 0) {
+                F[F_XCH + 5 + (r >> 5)] = gA;
+                F[F_XCH + 7 + (r >> 5)] = gD;
+            }
+            named_bar_sync(1, kC);
+            if (r == 0) {
+                p.gpart[sh * 2 + 0] = F[F_XCH + 5] + F[F_XCH + 6];
+                p.gpart[sh * 2 + 1] = F[F_XCH + 7] + F[F_XCH + 8];
+            }
         }
     } while (false);
 
