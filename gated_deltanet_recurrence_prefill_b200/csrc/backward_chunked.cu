@@ -2,13 +2,17 @@
 // (the algebra and the block functions are in backward_chunked.cuh).
 //
 //   1. chunk list: per slot the sequence and first token of its chunk;
-//   2. prep, one CTA per (chunk, value head): T, W, U', the decays, Y_c;
-//   3. forward chain, kRowSplit CTAs per (sequence, value head): S_c;
-//   4. backward chain, likewise: dS_c and dL/dS_0;
+//   2. prep, one CTA per (chunk, value head): T, W, U', the decays, Y_c (on the
+//      tensor cores, or in float32 with GDN_BACKWARD_GRAD=simt);
+//   3. forward chain: S_c;
+//   4. backward chain: dS_c and dL/dS_0 -- both on the tensor cores, one CTA per
+//      (sequence, value head) (backward_chunked_tc.cu), or with
+//      GDN_BACKWARD_GRAD=simt in float32 on the CUDA cores, kRowSplit CTAs per
+//      (sequence, value head);
 //   5. gradients, one CTA per (chunk, value head): dq, dk (per value head), dv,
 //      da, db and per-chunk sums for the gate parameters -- on the tensor cores
-//      (backward_chunked_tc.cu) unless GDN_BACKWARD_GRAD=simt selects the
-//      float32 CUDA-core block function below;
+//      (backward_chunked_tc.cu), or the float32 block function with
+//      GDN_BACKWARD_GRAD=simt;
 //   6. sums over each key head's value heads and over chunks.
 // Every CTA has 256 threads; 2, 3 and 5 take almost all of an SM's shared
 // memory, 4 about half.
@@ -64,7 +68,7 @@ cudaError_t launch_smem(K kernel, int64_t blocks, int floats, const Params& p, c
     return cudaGetLastError();
 }
 
-// GDN_BACKWARD_GRAD=simt: the float32 CUDA-core gradient kernel
+// GDN_BACKWARD_GRAD=simt: the float32 CUDA-core chains and gradient step
 bool grad_on_cuda_cores() {
     const char* env = getenv("GDN_BACKWARD_GRAD");
     return env && strcmp(env, "simt") == 0;
@@ -73,6 +77,8 @@ bool grad_on_cuda_cores() {
 }  // namespace
 
 cudaError_t launch_backward_grad_tc(const Params& p, int64_t jobs, cudaStream_t s);
+cudaError_t launch_backward_chains_tc(const Params& p, int64_t units, bool backward, cudaStream_t s);
+cudaError_t launch_backward_prep_tc(const Params& p, int64_t jobs, cudaStream_t s);
 
 size_t backward_chunked_workspace_bytes(int32_t n_seq, int64_t T, int32_t Hv) {
     return make_plan(n_seq, T, Hv).bytes;
@@ -96,12 +102,19 @@ cudaError_t launch_backward_chunked(const BackwardArgs& a, cudaStream_t s) {
         bwc_jobs_kernel<<<(unsigned)a.n_seq, kThreads, 0, s>>>(p);
         e = cudaGetLastError();
     }
-    if (e == cudaSuccess) e = launch_smem(bwc_prep_kernel, jobs, kPrepFloats, p, s);
-    if (e == cudaSuccess) e = launch_smem(bwc_fwd_chain_kernel, chains, kChainFloats, p, s);
-    if (e == cudaSuccess) e = launch_smem(bwc_bwd_chain_kernel, chains, kChainFloats, p, s);
-    if (e == cudaSuccess)
-        e = grad_on_cuda_cores() ? launch_smem(bwc_grad_kernel, jobs, kGradFloats, p, s)
-                                 : launch_backward_grad_tc(p, jobs, s);
+    const bool simt = grad_on_cuda_cores();
+    const int64_t units = (int64_t)a.n_seq * a.Hv;
+    if (simt) {
+        if (e == cudaSuccess) e = launch_smem(bwc_prep_kernel, jobs, kPrepFloats, p, s);
+        if (e == cudaSuccess) e = launch_smem(bwc_fwd_chain_kernel, chains, kChainFloats, p, s);
+        if (e == cudaSuccess) e = launch_smem(bwc_bwd_chain_kernel, chains, kChainFloats, p, s);
+        if (e == cudaSuccess) e = launch_smem(bwc_grad_kernel, jobs, kGradFloats, p, s);
+    } else {
+        if (e == cudaSuccess) e = launch_backward_prep_tc(p, jobs, s);
+        if (e == cudaSuccess) e = launch_backward_chains_tc(p, units, false, s);
+        if (e == cudaSuccess) e = launch_backward_chains_tc(p, units, true, s);
+        if (e == cudaSuccess) e = launch_backward_grad_tc(p, jobs, s);
+    }
     const int64_t n = a.T * a.Hqk * kD;
     if (e == cudaSuccess && n > 0) {
         bwc_reduce_qk_kernel<<<(unsigned)((n + kThreads - 1) / kThreads), kThreads, 0, s>>>(p);

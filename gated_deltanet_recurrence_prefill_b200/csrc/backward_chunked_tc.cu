@@ -747,6 +747,634 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
     }
 }
 
+// ---- the per-chunk preparation on the tensor cores ---------------------------------------
+// One CTA of 8 warps per (chunk, value head): the quantities the chains and the
+// gradient step read, as prep_block in backward_chunked.cuh computes them:
+//   round 1  D0 = [Q; K] K^T                 -> P = lower(Gamma o Q K^T) (bf16),
+//                                               A = diag(beta) strict_lower(Gamma o K K^T) (f32)
+//   solve    T = (I + A)^{-1}: 16 x 16 diagonal blocks by forward substitution,
+//            then 32 x 32 and 64 x 64 by T10 = -T11 A10 T00 (float32, CUDA cores)
+//   round 2  W = (T diag(beta)) (diag(gam) K), U' = (T diag(beta)) V, Z = P^T dO
+//   round 3  Y / scale = dO^T (diag(gam) Q) - Z^T W
+constexpr uint32_t R_QK = 0;                        // [Q; K]             128 x 128
+constexpr uint32_t R_V = R_QK + 2 * kPanel128;      // V                  64 x 128
+constexpr uint32_t R_DO = R_V + 2 * kPanel64;       // dO (bf16)          64 x 128
+constexpr uint32_t R_GK = R_DO + 2 * kPanel64;      // diag(gam) K        64 x 128
+constexpr uint32_t R_GQ = R_GK + 2 * kPanel64;      // diag(gam) Q        64 x 128
+constexpr uint32_t R_Z = R_GQ + 2 * kPanel64;       // Z                  64 x 128
+constexpr uint32_t R_NW = R_Z + 2 * kPanel64;       // -W                 64 x 128
+constexpr uint32_t R_P = R_NW + 2 * kPanel64;       // P                  64 x 64
+constexpr uint32_t R_TB = R_P + kPanel64;           // T diag(beta)       64 x 64
+constexpr uint32_t R_PAD = R_TB + kPanel64;         // (rows 64-127 of the M = 128 reads of T diag(beta))
+constexpr uint32_t R_AF = R_PAD + kPanel64;         // A, f32             64 x 65
+constexpr uint32_t R_TF = R_AF + 64 * 65 * 4;       // T, f32             64 x 65
+constexpr uint32_t R_XF = R_TF + 64 * 65 * 4;       // solve scratch, f32 64 x 65
+constexpr uint32_t R_MISC = R_XF + 64 * 65 * 4;     // gates, exchange
+constexpr uint32_t R_BAR = R_MISC + 400 * 4;
+constexpr uint32_t PREP_SMEM_ALLOC = R_BAR + 16 + 1024;
+static_assert(R_BAR % 8 == 0, "mbarrier alignment");
+static_assert(PREP_SMEM_ALLOC <= 232448, "shared memory budget of one CTA");
+constexpr uint32_t PT_D0 = 0, PT_W = 64, PT_U = 192, PT_Z = 320, PT_Y = 64;
+
+__global__ void __launch_bounds__(kGThreads, 1) bwc_prep_tc_kernel(Params p) {
+    extern __shared__ uint8_t bwt_prep_smem_raw[];
+    uint8_t* sm =
+        reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(bwt_prep_smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sb = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t slot = blockIdx.x / p.Hv;
+    const int h = blockIdx.x % p.Hv;
+    const size_t sh = sh_index(p, slot, h);
+    const int n = p.jobs[2 * slot];
+    if (n < 0) {
+        if (tid < 2) p.gpart[sh * 2 + tid] = 0.f;
+        return;
+    }
+    const int64_t t0 = p.jobs[2 * slot + 1];
+    int64_t bos, eos;
+    seq_bounds(p, n, bos, eos);
+    const int L = (int)((eos - t0) < kC ? (eos - t0) : kC);
+    const int g = h / (p.Hv / p.Hqk);
+
+    float* F = reinterpret_cast<float*>(sm + R_MISC);
+    float *be = F, *G = F + 64, *gam = F + 128, *kap = F + 192, *xch = F + 256;
+    float* Af = reinterpret_cast<float*>(sm + R_AF);
+    float* Tf = reinterpret_cast<float*>(sm + R_TF);
+    float* Xf = reinterpret_cast<float*>(sm + R_XF);
+    constexpr int kLf = 65;
+    const uint32_t bar = sb + R_BAR;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + R_BAR + 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + R_BAR + 12);
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+        tc_fence_before();
+    }
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        *abort_flag = 0;
+    }
+    // gates (warps 0-1): beta, G, gamma, kappa
+    if (tid < kC) {
+        const int r = tid;
+        float la = 0.f, bb = 0.f;
+        if (r < L) {
+            const int64_t t = t0 + r;
+            la = log_alpha(p.a[t * p.Hv + h], p.A_log[h], p.dt_bias[h]);
+            bb = sigmoid(p.b[t * p.Hv + h]);
+        }
+        float run = la;
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) {
+            const float o = __shfl_up_sync(0xffffffffu, run, m);
+            if (lane >= m) run += o;
+        }
+        if (r == 31) xch[0] = run;
+        named_bar_sync(1, kC);
+        if (r >= 32) run += xch[0];
+        be[r] = bb;
+        G[r] = run;
+        gam[r] = expf(run);
+        named_bar_sync(1, kC);
+        kap[r] = r < L ? expf(G[L - 1] - run) : 0.f;
+    }
+    // operands: [Q; K], V, dO (rows >= L zero)
+    {
+        uint4 kx[4], qx[4], vx[4];
+        float4 ox[4][2];
+        const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+        const float4 zf = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int it = tid + kGThreads * x, r = it >> 4, ch = it & 15;
+            const bool ok = r < L;
+            kx[x] = ok ? ldu4(p.k + ((size_t)(t0 + r) * p.Hqk + g) * kD + ch * 8) : z4;
+            qx[x] = ok ? ldu4(p.q + ((size_t)(t0 + r) * p.Hqk + g) * kD + ch * 8) : z4;
+            vx[x] = ok ? ldu4(p.v + ((size_t)(t0 + r) * p.Hv + h) * kD + ch * 8) : z4;
+            const float* op = p.d_o + ((size_t)(t0 + r) * p.Hv + h) * kD + ch * 8;
+            ox[x][0] = ok ? ldf4(op) : zf;
+            ox[x][1] = ok ? ldf4(op + 4) : zf;
+        }
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int it = tid + kGThreads * x, r = it >> 4, ch = it & 15;
+            st16(sm, R_QK, kPanel128, r, ch, qx[x]);
+            st16(sm, R_QK, kPanel128, 64 + r, ch, kx[x]);
+            st16(sm, R_V, kPanel64, r, ch, vx[x]);
+            st16(sm, R_DO, kPanel64, r, ch, pack8(ox[x][0], ox[x][1]));
+        }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const bool issuer = tid == 0;
+    const int q = warp & 3, hf = warp >> 2;
+    const uint32_t tl = tbase + ((uint32_t)(32 * q) << 16);
+    const bool lo = q < 2;
+    const int i = 32 * (q & 1) + lane;
+    int phase = 0;
+    auto products_done = [&]() -> bool {
+        mbar_wait(bar, (uint32_t)(phase & 1), abort_flag, kWaitLimitNs);
+        ++phase;
+        __syncthreads();
+        tc_fence_after();
+        return *abort_flag == 0;
+    };
+    auto publish = [&]() {
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+    };
+
+    do {
+        // ---- round 1: D0 = [Q; K] K^T (lanes 0-63 Q K^T, 64-127 K K^T)
+        if (issuer) {
+            tc_fence_after();
+            mma_run(tbase + PT_D0, sb + R_QK, kPanel128, false, sb + R_QK + 8192, kPanel128, false, ID_KK64, 8,
+                    false);
+            mma_commit(bar);
+        }
+        // meanwhile: T's scratch cleared (the solve reads its zero upper blocks);
+        // diag(gam) K and diag(gam) Q (from the staged tiles)
+        for (int x = tid; x < 64 * kLf; x += kGThreads) Tf[x] = 0.f;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int it = tid + kGThreads * x, r = it >> 4, ch = it & 15;
+            float kv[8], qv[8];
+            tile::ld_bf16x8(sm + R_QK + (ch >> 3) * kPanel128, 64 + r, ch & 7, kv);
+            tile::ld_bf16x8(sm + R_QK + (ch >> 3) * kPanel128, r, ch & 7, qv);
+            const float gr = gam[r];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                kv[e] *= gr;
+                qv[e] *= gr;
+            }
+            put8(sm, R_GK, kPanel64, r, ch, kv);
+            put8(sm, R_GQ, kPanel64, r, ch, qv);
+        }
+        if (!products_done()) break;
+        // ---- epilogue 1: P (lanes 0-63), A (lanes 64-127); each warp 32 columns
+        {
+            float d[32];
+            tmem_ld32(tl + PT_D0 + 32 * hf, d);
+            tmem_ld_wait();
+            const float Gi = G[i];
+            if (lo) {
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int j = 32 * hf + jj;
+                    d[jj] = (j <= i && i < L) ? d[jj] * expf(Gi - G[j]) : 0.f;
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) put8(sm, R_P, kPanel64, i, 4 * hf + c, d + 8 * c);
+            } else {
+                const float bi = be[i];
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    const int j = 32 * hf + jj;
+                    Af[i * kLf + j] = (j < i && i < L) ? bi * d[jj] * expf(Gi - G[j]) : 0.f;
+                }
+            }
+        }
+        __syncthreads();
+        // ---- T = (I + A)^{-1}, unit lower triangular
+        // 16 x 16 diagonal blocks: warp b, lane c < 16 holds column c
+        if (warp < 4) {
+            const int b0 = 16 * warp, c = lane & 15;
+            float xv[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float acc = 0.f;
+#pragma unroll
+                for (int m = 0; m < r; ++m) acc = fmaf(Af[(b0 + r) * kLf + b0 + m], xv[m], acc);
+                xv[r] = (r == c ? 1.f : 0.f) - acc;
+            }
+            if (lane < 16) {
+#pragma unroll
+                for (int r = 0; r < 16; ++r) Tf[(b0 + r) * kLf + b0 + c] = xv[r];
+            }
+        }
+        __syncthreads();
+        // 32 x 32 blocks (rows and columns 0-31, 32-63): T[R1][R0] = -T[R1][R1] A[R1][R0] T[R0][R0]
+        {
+            const int blk = tid >> 7, e = tid & 127;            // two elements of a 16 x 16 block each
+            const int R0 = 32 * blk, R1 = R0 + 16;
+            const int r = e >> 3, c0 = (e & 7) * 2;
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                const int c = c0 + x;
+                float acc = 0.f;
+#pragma unroll
+                for (int m = 0; m < 16; ++m) acc = fmaf(Af[(R1 + r) * kLf + R0 + m], Tf[(R0 + m) * kLf + R0 + c], acc);
+                Xf[(R1 + r) * kLf + R0 + c] = acc;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                const int c = c0 + x;
+                float acc = 0.f;
+#pragma unroll
+                for (int m = 0; m < 16; ++m) acc = fmaf(Tf[(R1 + r) * kLf + R1 + m], Xf[(R1 + m) * kLf + R0 + c], acc);
+                Tf[(R1 + r) * kLf + R0 + c] = -acc;
+            }
+        }
+        __syncthreads();
+        // 64 x 64: T[32:64][0:32] = -T[32:64][32:64] A[32:64][0:32] T[0:32][0:32]; four elements each
+        {
+            const int r = tid >> 3, c0 = (tid & 7) * 4;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+            for (int m = 0; m < 32; ++m) {
+                const float av = Af[(32 + r) * kLf + m];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) acc[x] = fmaf(av, Tf[m * kLf + c0 + x], acc[x]);
+            }
+#pragma unroll
+            for (int x = 0; x < 4; ++x) Xf[(32 + r) * kLf + c0 + x] = acc[x];
+            __syncthreads();
+#pragma unroll
+            for (int x = 0; x < 4; ++x) acc[x] = 0.f;
+#pragma unroll 8
+            for (int m = 0; m < 32; ++m) {
+                const float tv = Tf[(32 + r) * kLf + 32 + m];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) acc[x] = fmaf(tv, Xf[(32 + m) * kLf + c0 + x], acc[x]);
+            }
+#pragma unroll
+            for (int x = 0; x < 4; ++x) Tf[(32 + r) * kLf + c0 + x] = -acc[x];
+        }
+        __syncthreads();
+        // T out (f32, zeros above the diagonal) and T diag(beta) (bf16)
+        {
+            float* Tg = p.Tm + sh * kC * kC;
+#pragma unroll
+            for (int x = 0; x < 2; ++x) {
+                const int it = tid + kGThreads * x, r = it >> 3, ch = it & 7;
+                float tv[8], tb[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int c = 8 * ch + e;
+                    tv[e] = c <= r ? Tf[r * kLf + c] : 0.f;
+                    tb[e] = tv[e] * be[c];
+                }
+                stf4(Tg + r * kC + 8 * ch, tv[0], tv[1], tv[2], tv[3]);
+                stf4(Tg + r * kC + 8 * ch + 4, tv[4], tv[5], tv[6], tv[7]);
+                put8(sm, R_TB, kPanel64, r, ch, tb);
+            }
+            if (tid <= kC) p.G[sh * (kC + 1) + tid] = tid < kC ? kap[tid] : gam[L - 1];
+        }
+        publish();
+        // ---- round 2: W, U' (A = T diag(beta), K-major), Z = P^T dO (lanes 0-63)
+        if (issuer) {
+            tc_fence_after();
+            mma_run(tbase + PT_W, sb + R_TB, kPanel64, false, sb + R_GK, kPanel64, true, ID_KM128, 4, false);
+            mma_run(tbase + PT_U, sb + R_TB, kPanel64, false, sb + R_V, kPanel64, true, ID_KM128, 4, false);
+            mma_run(tbase + PT_Z, sb + R_P, kPanel64, true, sb + R_DO, kPanel64, true, ID_MM128, 4, false);
+            mma_commit(bar);
+        }
+        if (!products_done()) break;
+        // ---- epilogue 2 (lanes 0-63): W, U' out; -W and Z as bf16 operands
+        if (lo) {
+            float* Wg = p.W + sh * kC * kD + (size_t)i * kD;
+            float* Ug = p.Up + sh * kC * kD + (size_t)i * kD;
+#pragma unroll 1
+            for (int cb = 0; cb < 2; ++cb) {
+                const int c0 = 64 * hf + 32 * cb;
+                float w[32], u[32];
+                tmem_ld32x2(tl + PT_W + c0, tl + PT_U + c0, w, u);
+#pragma unroll
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    stf4(Wg + c0 + 4 * e4, w[4 * e4], w[4 * e4 + 1], w[4 * e4 + 2], w[4 * e4 + 3]);
+                    stf4(Ug + c0 + 4 * e4, u[4 * e4], u[4 * e4 + 1], u[4 * e4 + 2], u[4 * e4 + 3]);
+                }
+#pragma unroll
+                for (int e = 0; e < 32; ++e) w[e] = -w[e];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) put8(sm, R_NW, kPanel64, i, c0 / 8 + c, w + 8 * c);
+                float z[32];
+                tmem_ld32(tl + PT_Z + c0, z);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < 4; ++c) put8(sm, R_Z, kPanel64, i, c0 / 8 + c, z + 8 * c);
+            }
+        }
+        publish();
+        // ---- round 3: Y / scale = dO^T (diag(gam) Q) + Z^T (-W) (all 128 lanes: rows e)
+        if (issuer) {
+            tc_fence_after();
+            mma_run(tbase + PT_Y, sb + R_DO, kPanel64, true, sb + R_GQ, kPanel64, true, ID_MM128, 4, false);
+            mma_run(tbase + PT_Y, sb + R_Z, kPanel64, true, sb + R_NW, kPanel64, true, ID_MM128, 4, true);
+            mma_commit(bar);
+        }
+        if (!products_done()) break;
+        {
+            const int e = 32 * q + lane;
+            float* Yg = p.Y + sh * kD * kD + (size_t)e * kD;
+#pragma unroll 1
+            for (int cb = 0; cb < 2; ++cb) {
+                const int c0 = 64 * hf + 32 * cb;
+                float y[32];
+                tmem_ld32(tl + PT_Y + c0, y);
+                tmem_ld_wait();
+#pragma unroll
+                for (int f4 = 0; f4 < 8; ++f4)
+                    stf4(Yg + c0 + 4 * f4, p.scale * y[4 * f4], p.scale * y[4 * f4 + 1], p.scale * y[4 * f4 + 2],
+                         p.scale * y[4 * f4 + 3]);
+            }
+        }
+    } while (false);
+
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag) {
+        if (tid == 0) {
+            *reinterpret_cast<volatile uint32_t*>(p.err) = 1u;
+            volatile int no_abort = 0;
+            mma_commit(bar);
+            mbar_wait(bar, (uint32_t)(phase & 1), &no_abort, kWaitLimitNs);
+        }
+        __syncthreads();
+    }
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tbase, kTmemCols);
+    }
+}
+
+// ---- the two state chains on the tensor cores -------------------------------------------
+// One CTA of 8 warps per (sequence, value head).  The state (S forward, dS
+// backward; float32) stays in registers: thread (warp w, lane l) holds row
+// 32 (w % 4) + l, columns 64 (w / 4) .. + 64.  Per chunk, two products:
+//   forward   U^T = ...: X = W S^T (rows i; tokens), then
+//             U = kappa (U' - X) (bf16, rows i) and dS~ = U^T K;  S <- gamma_L S + dS~
+//   backward  X = K dS^T (rows i), X <- kappa X (bf16), dS~ = X^T W;
+//             dS <- gamma_L dS + Y - dS~
+// Both products use the bf16 state as the operand (the chain itself is carried
+// in float32).  The next chunk's K, W and U' (or Y) are fetched while the
+// current chunk's products run: K and U' / Y by cp.async straight into shared
+// memory, W through registers (converted to bf16).
+constexpr uint32_t C_ST = 0;                        // the state, bf16       128 x 128
+constexpr uint32_t C_WT = C_ST + 2 * kPanel128;     // W, bf16               64 x 128
+constexpr uint32_t C_KT = C_WT + 2 * kPanel64;      // K, bf16               64 x 128
+constexpr uint32_t C_XT = C_KT + 2 * kPanel64;      // kappa U or kappa X    64 x 128
+constexpr uint32_t C_BUF = C_XT + 2 * kPanel64;     // U' (64 rows) or Y (128 rows), f32
+constexpr int kBufLd = 132;                         // floats per row (16-byte rows, conflict-free float4 reads)
+constexpr uint32_t C_MISC = C_BUF + 128 * kBufLd * 4;   // kappa [64], gamma_L
+constexpr uint32_t C_BAR = C_MISC + 80 * 4;         // mbarrier (8), TMEM base (4), abort flag (4)
+constexpr uint32_t CH_SMEM_ALLOC = C_BAR + 16 + 1024;
+static_assert(C_BAR % 8 == 0, "mbarrier alignment");
+constexpr uint32_t CT_X = 0, CT_D = 128, kChainTmemCols = 256;
+
+TC_DEVICE void cp_async16z(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+TC_DEVICE void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+TC_DEVICE void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+template <bool kBwd>
+__global__ void __launch_bounds__(kGThreads, 1) bwc_chain_tc_kernel(Params p) {
+    extern __shared__ uint8_t bwt_chain_smem_raw[];
+    uint8_t* sm =
+        reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(bwt_chain_smem_raw) + 1023) & ~(uintptr_t)1023);
+    const uint32_t sb = smem_u32(sm);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n = blockIdx.x / p.Hv, h = blockIdx.x % p.Hv;
+    const int g = h / (p.Hv / p.Hqk);
+    int64_t bos, eos;
+    seq_bounds(p, n, bos, eos);
+    const int64_t nch = (eos - bos + kC - 1) / kC;
+    const int q = warp & 3, hf = warp >> 2;
+    const int row = 32 * q + lane;                   // state row (TMEM lane) of this thread
+    const size_t unit = ((size_t)n * p.Hv + h) * kD * kD + (size_t)row * kD + 64 * hf;
+    float st[64];
+    {
+        const float* init = kBwd ? p.d_fin : p.s0;
+#pragma unroll
+        for (int c4 = 0; c4 < 16; ++c4) {
+            const float4 v = init ? ldf4(init + unit + 4 * c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            st[4 * c4] = v.x; st[4 * c4 + 1] = v.y; st[4 * c4 + 2] = v.z; st[4 * c4 + 3] = v.w;
+        }
+    }
+    if (nch == 0) {
+        if (kBwd && p.d_init) {
+#pragma unroll
+            for (int c4 = 0; c4 < 16; ++c4) stf4(p.d_init + unit + 4 * c4, st[4 * c4], st[4 * c4 + 1], st[4 * c4 + 2], st[4 * c4 + 3]);
+        }
+        return;
+    }
+    float* kap = reinterpret_cast<float*>(sm + C_MISC);
+    const uint32_t bar = sb + C_BAR;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C_BAR + 8);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C_BAR + 12);
+    if (warp == 0) {
+        tmem_alloc(smem_u32(tmem_slot), kChainTmemCols);
+        tc_fence_before();
+    }
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+        *abort_flag = 0;
+    }
+
+    // chunk jj of the walk (backward: from the last)
+    auto chunk_t0 = [&](int64_t jj) -> int64_t { return bos + (kBwd ? nch - 1 - jj : jj) * kC; };
+    auto chunk_len = [&](int64_t t0) -> int { return (int)((eos - t0) < kC ? (eos - t0) : kC); };
+    auto fetch_k = [&](int64_t t0) {
+        const int Lc = chunk_len(t0);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int it = tid + kGThreads * x, r = it >> 4, ch = it & 15;
+            const bool ok = r < Lc;
+            const uint16_t* src = ok ? p.k + ((size_t)(t0 + r) * p.Hqk + g) * kD + ch * 8 : p.k;
+            cp_async16z(sb + C_KT + (uint32_t)(ch >> 3) * kPanel64 + sw128_off(r, ch & 7), src, ok ? 16u : 0u);
+        }
+    };
+    auto fetch_buf = [&](int64_t t0) {
+        const size_t sh = sh_index(p, t0 / kC + n, h);
+        const float* src = kBwd ? p.Y + sh * kD * kD : p.Up + sh * kC * kD;
+        constexpr int kItems = (kBwd ? 128 : 64) * 32 / kGThreads;
+#pragma unroll
+        for (int x = 0; x < kItems; ++x) {
+            const int it = tid + kGThreads * x, r = it >> 5, pc = it & 31;
+            cp_async16z(sb + C_BUF + (uint32_t)(r * kBufLd + 4 * pc) * 4u, src + (size_t)r * kD + 4 * pc, 16u);
+        }
+    };
+    float4 wr[4][2];
+    auto load_w = [&](int64_t t0) {
+        const float* src = p.W + sh_index(p, t0 / kC + n, h) * kC * kD;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int it = tid + kGThreads * x, r = it >> 4, ch = it & 15;
+            wr[x][0] = ldf4(src + (size_t)r * kD + ch * 8);
+            wr[x][1] = ldf4(src + (size_t)r * kD + ch * 8 + 4);
+        }
+    };
+    auto store_w = [&]() {
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int it = tid + kGThreads * x, r = it >> 4, ch = it & 15;
+            st16(sm, C_WT, kPanel64, r, ch, pack8(wr[x][0], wr[x][1]));
+        }
+    };
+    auto load_gates = [&](int64_t t0) {
+        const size_t sh = sh_index(p, t0 / kC + n, h);
+        if (tid <= kC) kap[tid] = p.G[sh * (kC + 1) + tid];     // kappa_0..63, then gamma_L at [64]
+    };
+
+    // prologue: chunk 0's operands
+    {
+        const int64_t t0 = chunk_t0(0);
+        fetch_k(t0);
+        fetch_buf(t0);
+        cp_async_commit();
+        load_w(t0);
+        store_w();
+        load_gates(t0);
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_slot;
+    const uint32_t tl = tbase + ((uint32_t)(32 * q) << 16);
+    int phase = 0;
+    auto products_done = [&]() -> bool {
+        mbar_wait(bar, (uint32_t)(phase & 1), abort_flag, kWaitLimitNs);
+        ++phase;
+        __syncthreads();
+        tc_fence_after();
+        return *abort_flag == 0;
+    };
+
+    for (int64_t jj = 0; jj < nch; ++jj) {
+        const int64_t t0 = chunk_t0(jj);
+        const size_t sh = sh_index(p, t0 / kC + n, h);
+        const bool more = jj + 1 < nch;
+        const int64_t t0n = more ? chunk_t0(jj + 1) : t0;
+        // the state at this chunk's start (forward) or end (backward), kept for
+        // the gradient step, and as the bf16 operand
+        {
+            float* dst = (kBwd ? p.dS : p.S) + sh * kD * kD + (size_t)row * kD + 64 * hf;
+#pragma unroll
+            for (int c4 = 0; c4 < 16; ++c4) stf4(dst + 4 * c4, st[4 * c4], st[4 * c4 + 1], st[4 * c4 + 2], st[4 * c4 + 3]);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) put8(sm, C_ST, kPanel128, row, 8 * hf + j, st + 8 * j);
+        }
+        cp_async_wait_all();
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            // X = W S^T (forward) or K dS^T (backward): rows i in TMEM lanes 0-63
+            mma_run(tbase + CT_X, sb + (kBwd ? C_KT : C_WT), kPanel64, false, sb + C_ST, kPanel128, false, ID_KK128,
+                    8, false);
+            mma_commit(bar);
+        }
+        if (more) load_w(t0n);
+        if (!products_done()) break;
+        if (q < 2) {
+            const int i = row;
+            const float ki = kap[i];
+#pragma unroll 1
+            for (int hb = 0; hb < 2; ++hb) {
+                const int c0 = 64 * hf + 32 * hb;
+                float x[32];
+                tmem_ld32(tl + CT_X + c0, x);
+                tmem_ld_wait();
+                if (!kBwd) {
+                    const float* up = reinterpret_cast<const float*>(sm + C_BUF) + i * kBufLd + c0;
+#pragma unroll
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const float4 u4 = ldf4(up + 4 * e4);
+                        x[4 * e4] = ki * (u4.x - x[4 * e4]);
+                        x[4 * e4 + 1] = ki * (u4.y - x[4 * e4 + 1]);
+                        x[4 * e4 + 2] = ki * (u4.z - x[4 * e4 + 2]);
+                        x[4 * e4 + 3] = ki * (u4.w - x[4 * e4 + 3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[e] *= ki;
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) put8(sm, C_XT, kPanel64, i, c0 / 8 + j, x + 8 * j);
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            // dS~ = (kappa U)^T K (forward) or (kappa X)^T W (backward): A and B
+            // MN-major (rows = tokens)
+            mma_run(tbase + CT_D, sb + C_XT, kPanel64, true, sb + (kBwd ? C_WT : C_KT), kPanel64, true, ID_MM128, 4,
+                    false);
+            mma_commit(bar);
+        }
+        // U' (forward) has been read; K (backward) is no longer read by the tensor core
+        if (more) {
+            if (kBwd) fetch_k(t0n);
+            else fetch_buf(t0n);
+            cp_async_commit();
+        }
+        if (!products_done()) break;
+        {
+            const float gL = kap[kC];
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb) {
+                float d[32];
+                tmem_ld32(tl + CT_D + 64 * hf + 32 * hb, d);
+                tmem_ld_wait();
+                float* s32 = st + 32 * hb;
+                if (!kBwd) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) s32[e] = fmaf(gL, s32[e], d[e]);
+                } else {
+                    const float* y = reinterpret_cast<const float*>(sm + C_BUF) + row * kBufLd + 64 * hf + 32 * hb;
+#pragma unroll
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const float4 y4 = ldf4(y + 4 * e4);
+                        s32[4 * e4] = fmaf(gL, s32[4 * e4], y4.x) - d[4 * e4];
+                        s32[4 * e4 + 1] = fmaf(gL, s32[4 * e4 + 1], y4.y) - d[4 * e4 + 1];
+                        s32[4 * e4 + 2] = fmaf(gL, s32[4 * e4 + 2], y4.z) - d[4 * e4 + 2];
+                        s32[4 * e4 + 3] = fmaf(gL, s32[4 * e4 + 3], y4.w) - d[4 * e4 + 3];
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        // every read of this chunk's operands is done: the next chunk's take their place
+        if (more) {
+            if (kBwd) fetch_buf(t0n);
+            else fetch_k(t0n);
+            cp_async_commit();
+            store_w();
+            load_gates(t0n);
+        }
+    }
+    if (kBwd && p.d_init && *abort_flag == 0) {
+#pragma unroll
+        for (int c4 = 0; c4 < 16; ++c4) stf4(p.d_init + unit + 4 * c4, st[4 * c4], st[4 * c4 + 1], st[4 * c4 + 2], st[4 * c4 + 3]);
+    }
+    cp_async_wait_all();
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag) {
+        if (tid == 0) {
+            *reinterpret_cast<volatile uint32_t*>(p.err) = 1u;
+            volatile int no_abort = 0;
+            mma_commit(bar);
+            mbar_wait(bar, (uint32_t)(phase & 1), &no_abort, kWaitLimitNs);
+        }
+        __syncthreads();
+    }
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tbase, kChainTmemCols);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_backward_grad_tc(const Params& p, int64_t jobs, cudaStream_t s) {
@@ -756,6 +1384,26 @@ cudaError_t launch_backward_grad_tc(const Params& p, int64_t jobs, cudaStream_t 
                                          (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     bwc_grad_tc_kernel<<<(unsigned)jobs, kGThreads, SMEM_ALLOC, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_backward_prep_tc(const Params& p, int64_t jobs, cudaStream_t s) {
+    if (jobs <= 0) return cudaSuccess;
+    if (jobs > 0x7fffffff) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(bwc_prep_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)PREP_SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    bwc_prep_tc_kernel<<<(unsigned)jobs, kGThreads, PREP_SMEM_ALLOC, s>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_backward_chains_tc(const Params& p, int64_t units, bool backward, cudaStream_t s) {
+    if (units <= 0) return cudaSuccess;
+    if (units > 0x7fffffff) return cudaErrorInvalidValue;
+    auto kernel = backward ? bwc_chain_tc_kernel<true> : bwc_chain_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CH_SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    kernel<<<(unsigned)units, kGThreads, CH_SMEM_ALLOC, s>>>(p);
     return cudaGetLastError();
 }
 
