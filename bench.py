@@ -644,11 +644,19 @@ def bench_backward(args, dev, flush, peaks, world, chunked=False):
                   "end": torch.cuda.Event(enable_timing=True)}
     times, _ = _time_steps(step, 3, 3, flush, mk, world)
     ms = _max_over_ranks(sum(times) / len(times), world)
-    how = ("CUDA cores, chunk-parallel prep and gradients, two state chains over chunks" if chunked
-           else "CUDA cores, one CTA per value head, token by token")
+    how = ("tensor cores (tcgen05): chunk-parallel preparation and gradient step, two state chains "
+           "over chunks" if chunked else "CUDA cores, one CTA per value head, token by token")
     out = {"workload": f"{entry} T={T} N=1 Hqk=16 Hv=48 d=128, S0 and dL/dS_T given ({how})",
            "ms": round(ms, 3), "tokens_per_s_layer": round(weak_scaling_rate(T, ms, world), 1),
            "launches_per_step": 7 if chunked else 3}
+    if chunked:
+        # useful products per (chunk, value head), bf16 operands: preparation
+        # 9.4 MFLOP, each chain 4.2 MFLOP, gradient step 25.2 MFLOP
+        flop = (T // 64) * HV * (9.44e6 + 2 * 4.19e6 + 25.17e6)
+        out["tensor_flop_per_step"] = flop
+        out["roofline"] = {"bound": "latency (serial chains, per-chunk phases)",
+                           "tensor_tflops": round(flop / (ms * 1e-3) / 1e12, 1),
+                           "tensor_frac": round(flop / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)}
     del q, k, v, d_o, ws
     torch.cuda.empty_cache()
     return out
