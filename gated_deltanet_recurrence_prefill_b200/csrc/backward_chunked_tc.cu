@@ -146,9 +146,29 @@ TC_DEVICE void stf4(float* p, float a, float b, float c, float d) {
     *reinterpret_cast<float4*>(p) = make_float4(a, b, c, d);
 }
 
+// 16-byte cp.async (src_bytes < 16 zero-fills the rest), its groups
+TC_DEVICE void cp_async16z(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+TC_DEVICE void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+TC_DEVICE void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // scratch: quantity 0 in columns 0-63, quantity 1 in 64-127, rotated by the row
 // (conflict-free both for a thread per row and for a thread per column)
 TC_DEVICE int scr_ix(int i, int j) { return i * 128 + ((j + i) & 127); }
+// column j of the scratch summed over its 64 rows (four partial sums, fixed order)
+TC_DEVICE float col_sum(const float* scr, int j) {
+    float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll 4
+    for (int r = 0; r < 64; r += 4) {
+        s0 += scr[scr_ix(r, j)];
+        s1 += scr[scr_ix(r + 1, j)];
+        s2 += scr[scr_ix(r + 2, j)];
+        s3 += scr[scr_ix(r + 3, j)];
+    }
+    return (s0 + s1) + (s2 + s3);
+}
 
 __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
     extern __shared__ uint8_t bwt_smem_raw[];
@@ -182,6 +202,73 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
         fence_mbar_init();
         *abort_flag = 0;
     }
+    // gate inputs (threads 0-63, one row each), requested before the operands
+    float g_a = 0.f, g_b = 0.f;
+    if (tid < kC && tid < L) {
+        const int64_t t = t0 + tid;
+        g_a = p.a[t * p.Hv + h];
+        g_b = p.b[t * p.Hv + h];
+    }
+
+    // ---- stage the operands -------------------------------------------------------------
+    // By cp.async straight into their tiles: K, Q, V (bf16 inputs; rows >= L
+    // zero-filled), and S, dS and W, which the chains and the preparation wrote
+    // as bf16 tiles in this very layout.  dO and T (float32) through registers.
+    {
+        const uint8_t* Sg = reinterpret_cast<const uint8_t*>(p.S + sh * kD * kD);
+        const uint8_t* dSg = reinterpret_cast<const uint8_t*>(p.dS + sh * kD * kD);
+        const uint8_t* Wg = reinterpret_cast<const uint8_t*>(p.W + sh * kC * kD);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int it = tid + kGThreads * x, r = it >> 4, ch = it & 15;
+            const bool ok = r < L;
+            const uint32_t z = ok ? 16u : 0u;
+            const size_t kq = ((size_t)(t0 + r) * p.Hqk + g) * kD + ch * 8;
+            const uint32_t off = (uint32_t)(ch >> 3) * kPanel192;
+            cp_async16z(sb + S_KQW + off + sw128_off(128 + r, ch & 7), ok ? p.k + kq : p.k, z);
+            cp_async16z(sb + S_KQW + off + sw128_off(64 + r, ch & 7), ok ? p.q + kq : p.q, z);
+            cp_async16z(sb + S_UV + (uint32_t)(ch >> 3) * kPanel128 + sw128_off(64 + r, ch & 7),
+                        ok ? p.v + ((size_t)(t0 + r) * p.Hv + h) * kD + ch * 8 : p.v, z);
+            // W rows 0-63: the tile's panels are 8 KB apart, the [W; Q; K] tile's 24 KB
+            cp_async16z(sb + S_KQW + off + sw128_off(r, ch & 7), Wg + (ch >> 3) * kPanel64 + sw128_off(r, ch & 7), 16u);
+        }
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+            const uint32_t o = (uint32_t)(tid + kGThreads * x) * 16u;
+            cp_async16z(sb + S_S + o, Sg + o, 16u);
+            cp_async16z(sb + S_DS + o, dSg + o, 16u);
+        }
+        cp_async_commit();
+    }
+    {
+        float4 ox[4][2], tx[2][2];
+        const float4 zf = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float* Tg = p.Tm + sh * kC * kC;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int it = tid + kGThreads * x, r = it >> 4, ch = it & 15;
+            const bool ok = r < L;
+            const float* op = p.d_o + ((size_t)(t0 + r) * p.Hv + h) * kD + ch * 8;
+            ox[x][0] = ok ? ldf4(op) : zf;
+            ox[x][1] = ok ? ldf4(op + 4) : zf;
+        }
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            const int it = tid + kGThreads * x, r = it >> 3, ch = it & 7;
+            tx[x][0] = ldf4(Tg + r * kC + ch * 8);
+            tx[x][1] = ldf4(Tg + r * kC + ch * 8 + 4);
+        }
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const int it = tid + kGThreads * x, r = it >> 4, ch = it & 15;
+            st16(sm, S_DUO, kPanel128, r, ch, pack8(ox[x][0], ox[x][1]));
+        }
+#pragma unroll
+        for (int x = 0; x < 2; ++x) {
+            const int it = tid + kGThreads * x, r = it >> 3, ch = it & 7;
+            st16(sm, S_T, kPanel64, r, ch, pack8(tx[x][0], tx[x][1]));
+        }
+    }
     // gates (warps 0-1, one row each): log alpha, beta, G = running sum of log
     // alpha (an inclusive scan; rows >= L add 0, so they carry G_{L-1}), gamma,
     // kappa, and sigmoid(a + dt_bias) for d a
@@ -189,11 +276,10 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
         const int r = tid;
         float la = 0.f, bb = 0.f, sg = 0.f;
         if (r < L) {
-            const int64_t t = t0 + r;
-            const float av = p.a[t * p.Hv + h], dtb = p.dt_bias[h];
-            la = log_alpha(av, p.A_log[h], dtb);
-            bb = sigmoid(p.b[t * p.Hv + h]);
-            sg = sigmoid(av + dtb);
+            const float dtb = p.dt_bias[h];
+            la = log_alpha(g_a, p.A_log[h], dtb);
+            bb = sigmoid(g_b);
+            sg = sigmoid(g_a + dtb);
         }
         float run = la;
 #pragma unroll
@@ -212,6 +298,27 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
         named_bar_sync(1, kC);
         kap[r] = r < L ? expf(G[L - 1] - run) : 0.f;
     }
+    cp_async_wait<0>();
+    // <dS, S> over the state (this thread's own 16-byte pieces of the two tiles)
+    {
+        float ss = 0.f;
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+            const uint32_t o = (uint32_t)(tid + kGThreads * x) * 16u;
+            const uint4 a4 = *reinterpret_cast<const uint4*>(sm + S_S + o);
+            const uint4 b4 = *reinterpret_cast<const uint4*>(sm + S_DS + o);
+            const uint32_t av[4] = {a4.x, a4.y, a4.z, a4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+            for (int y = 0; y < 4; ++y) {
+                const float2 sa = bf16x2_to_f32x2(av[y]), sd = bf16x2_to_f32x2(bv[y]);
+                ss = fmaf(sa.x, sd.x, fmaf(sa.y, sd.y, ss));
+            }
+        }
+        ss = warp_sum(ss);
+        if (lane == 0) F[F_RED + warp] = ss;
+    }
+    fence_async_smem();
+    tc_fence_before();
     // (this barrier also publishes the TMEM base and the mbarrier)
     __syncthreads();
     tc_fence_after();
@@ -222,95 +329,6 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
     const bool lo = q < 2;                           // TMEM lanes 0-63
     const int i = 32 * (q & 1) + lane;               // chunk row of this thread's TMEM lane
     const float scale = p.scale;
-
-    // ---- stage the operands -------------------------------------------------------------
-    {
-        uint4 kx[4], qx[4], vx[4];
-        float4 wx[4][2];
-        const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const int it = tid + kGThreads * x, r = it >> 4, ch = it & 15;
-            const bool ok = r < L;
-            kx[x] = ok ? ldu4(p.k + ((size_t)(t0 + r) * p.Hqk + g) * kD + ch * 8) : z4;
-            qx[x] = ok ? ldu4(p.q + ((size_t)(t0 + r) * p.Hqk + g) * kD + ch * 8) : z4;
-            vx[x] = ok ? ldu4(p.v + ((size_t)(t0 + r) * p.Hv + h) * kD + ch * 8) : z4;
-            const float* wp = p.W + sh * kC * kD + (size_t)r * kD + ch * 8;
-            wx[x][0] = ldf4(wp);
-            wx[x][1] = ldf4(wp + 4);
-        }
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const int it = tid + kGThreads * x, r = it >> 4, ch = it & 15;
-            st16(sm, S_KQW, kPanel192, r, ch, pack8(wx[x][0], wx[x][1]));
-            st16(sm, S_KQW, kPanel192, 64 + r, ch, qx[x]);
-            st16(sm, S_KQW, kPanel192, 128 + r, ch, kx[x]);
-            st16(sm, S_UV, kPanel128, 64 + r, ch, vx[x]);
-        }
-    }
-    float ss = 0.f;
-    {
-        const float* Sg = p.S + sh * kD * kD;
-        const float* dSg = p.dS + sh * kD * kD;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float4 sx[4][2], dx[4][2];
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const int it = tid + kGThreads * (4 * half + x), r = it >> 4, ch = it & 15;
-                sx[x][0] = ldf4(Sg + (size_t)r * kD + ch * 8);
-                sx[x][1] = ldf4(Sg + (size_t)r * kD + ch * 8 + 4);
-                dx[x][0] = ldf4(dSg + (size_t)r * kD + ch * 8);
-                dx[x][1] = ldf4(dSg + (size_t)r * kD + ch * 8 + 4);
-            }
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const int it = tid + kGThreads * (4 * half + x), r = it >> 4, ch = it & 15;
-                st16(sm, S_S, kPanel128, r, ch, pack8(sx[x][0], sx[x][1]));
-                st16(sm, S_DS, kPanel128, r, ch, pack8(dx[x][0], dx[x][1]));
-#pragma unroll
-                for (int y = 0; y < 2; ++y) {
-                    ss = fmaf(sx[x][y].x, dx[x][y].x, ss);
-                    ss = fmaf(sx[x][y].y, dx[x][y].y, ss);
-                    ss = fmaf(sx[x][y].z, dx[x][y].z, ss);
-                    ss = fmaf(sx[x][y].w, dx[x][y].w, ss);
-                }
-            }
-        }
-    }
-    {
-        float4 ox[4][2], tx[2][2];
-        const float4 zf = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const int it = tid + kGThreads * x, r = it >> 4, ch = it & 15;
-            const bool ok = r < L;
-            const float* op = p.d_o + ((size_t)(t0 + r) * p.Hv + h) * kD + ch * 8;
-            ox[x][0] = ok ? ldf4(op) : zf;
-            ox[x][1] = ok ? ldf4(op + 4) : zf;
-        }
-        const float* Tg = p.Tm + sh * kC * kC;
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-            const int it = tid + kGThreads * x, r = it >> 3, ch = it & 7;
-            tx[x][0] = ldf4(Tg + r * kC + ch * 8);
-            tx[x][1] = ldf4(Tg + r * kC + ch * 8 + 4);
-        }
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const int it = tid + kGThreads * x, r = it >> 4, ch = it & 15;
-            st16(sm, S_DUO, kPanel128, r, ch, pack8(ox[x][0], ox[x][1]));
-        }
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-            const int it = tid + kGThreads * x, r = it >> 3, ch = it & 7;
-            st16(sm, S_T, kPanel64, r, ch, pack8(tx[x][0], tx[x][1]));
-        }
-    }
-    F[F_RED + tid] = ss;
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
 
     int phase = 0;
     // all threads wait for the products issued last; false (uniformly) if a
@@ -345,8 +363,18 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
         }
         if (tid == 0) {
             float s = 0.f;
-            for (int x = 0; x < kGThreads; ++x) s += F[F_RED + x];
+            for (int x = 0; x < kGThreads / 32; ++x) s += F[F_RED + x];
             F[F_SS] = s;
+        }
+        // epilogue 1's rows from global memory, requested while the products run:
+        // U' (lanes 0-63) or dO (lanes 64-127), columns 64 hf .. + 64
+        float4 pre[16];
+        {
+            const bool ok = lo || i < L;
+            const float* src = lo ? p.Up + sh * kC * kD + (size_t)i * kD + 64 * hf
+                                  : p.d_o + ((size_t)(t0 + (ok ? i : 0)) * p.Hv + h) * kD + 64 * hf;
+#pragma unroll
+            for (int c4 = 0; c4 < 16; ++c4) pre[c4] = ok ? ldf4(src + 4 * c4) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
         if (!products_done()) break;
 
@@ -354,15 +382,14 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
         if (lo) {
             const float ki = kap[i];
             float r1 = 0.f;
-            const float* up = p.Up + sh * kC * kD + (size_t)i * kD;
-#pragma unroll 1
+#pragma unroll
             for (int cb = 0; cb < 2; ++cb) {
                 const int c0 = 64 * hf + 32 * cb;
                 float x1[32], kd[32];
                 tmem_ld32x2(tl + T_C1 + c0, tl + T_C2 + c0, x1, kd);
 #pragma unroll
                 for (int j8 = 0; j8 < 4; ++j8) {
-                    const float4 a = ldf4(up + c0 + 8 * j8), b = ldf4(up + c0 + 8 * j8 + 4);
+                    const float4 a = pre[8 * cb + 2 * j8], b = pre[8 * cb + 2 * j8 + 1];
                     const float upv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
                     float u[8], ku[8];
 #pragma unroll
@@ -389,22 +416,19 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
             for (int c = 0; c < 4; ++c) put8(sm, S_P, kPanel64, i, 4 * hf + c, qk + 8 * c);
         } else {
             float r2 = 0.f;
-#pragma unroll 1
+#pragma unroll
             for (int cb = 0; cb < 2; ++cb) {
                 const int c0 = 64 * hf + 32 * cb;
                 float qs[32];
                 tmem_ld32(tl + T_C1 + c0, qs);
                 tmem_ld_wait();
-                if (i < L) {
-                    const float* op = p.d_o + ((size_t)(t0 + i) * p.Hv + h) * kD + c0;
 #pragma unroll
-                    for (int e4 = 0; e4 < 8; ++e4) {
-                        const float4 o4 = ldf4(op + 4 * e4);
-                        r2 = fmaf(o4.x, qs[4 * e4], r2);
-                        r2 = fmaf(o4.y, qs[4 * e4 + 1], r2);
-                        r2 = fmaf(o4.z, qs[4 * e4 + 2], r2);
-                        r2 = fmaf(o4.w, qs[4 * e4 + 3], r2);
-                    }
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    const float4 o4 = pre[8 * cb + e4];
+                    r2 = fmaf(o4.x, qs[4 * e4], r2);
+                    r2 = fmaf(o4.y, qs[4 * e4 + 1], r2);
+                    r2 = fmaf(o4.z, qs[4 * e4 + 2], r2);
+                    r2 = fmaf(o4.w, qs[4 * e4 + 3], r2);
                 }
             }
             F[F_DGAM + 64 * hf + i] = r2;
@@ -532,11 +556,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
                     false);
             mma_commit(bar);
         }
-        if (tid < 64) {
-            float s = 0.f;
-            for (int r = 0; r < 64; ++r) s += scr[scr_ix(r, tid)];
-            F[F_CSM + tid] = s;
-        }
+        if (tid < 64) F[F_CSM + tid] = col_sum(scr, tid);
         if (!products_done()) break;
 
         // ---- epilogue 4: dT = lower(beta_j dU V^T + beta_j gam_j dW K^T) (lanes 64-127)
@@ -574,12 +594,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
             mma_run(tbase + T_C4, sb + S_T, kPanel64, true, sb + S_DT, kPanel64, true, ID_MM64, 4, false);
             mma_commit(bar);
         }
-        if (tid < 128) {
-            const int j = tid & 63, qn = tid >> 6;
-            float s = 0.f;
-            for (int r = 0; r < 64; ++r) s += scr[scr_ix(r, j + 64 * qn)];
-            F[(qn == 0 ? F_DBET : F_SKT) + j] = s;
-        }
+        if (tid < 128) F[(tid < 64 ? F_DBET : F_SKT) + (tid & 63)] = col_sum(scr, tid);
         if (!products_done()) break;
 
         // ---- epilogue 5: dv out; M2 into rows 64-127 of its tile (lanes 0-63)
@@ -655,11 +670,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
                     true);
             mma_commit(bar);
         }
-        if (tid < 64) {
-            float s = 0.f;
-            for (int r = 0; r < 64; ++r) s += scr[scr_ix(r, tid)];
-            F[F_CSA + tid] = s;
-        }
+        if (tid < 64) F[F_CSA + tid] = col_sum(scr, tid);
         if (!products_done()) break;
 
         // ---- epilogue 7: dq, dk of this value head (lanes 0-63)
@@ -761,9 +772,9 @@ constexpr uint32_t R_V = R_QK + 2 * kPanel128;      // V                  64 x 1
 constexpr uint32_t R_DO = R_V + 2 * kPanel64;       // dO (bf16)          64 x 128
 constexpr uint32_t R_GK = R_DO + 2 * kPanel64;      // diag(gam) K        64 x 128
 constexpr uint32_t R_GQ = R_GK + 2 * kPanel64;      // diag(gam) Q        64 x 128
-constexpr uint32_t R_Z = R_GQ + 2 * kPanel64;       // Z                  64 x 128
-constexpr uint32_t R_NW = R_Z + 2 * kPanel64;       // -W                 64 x 128
-constexpr uint32_t R_P = R_NW + 2 * kPanel64;       // P                  64 x 64
+constexpr uint32_t R_Z = R_GQ + 2 * kPanel64;       // -Z                 64 x 128
+constexpr uint32_t R_W = R_Z + 2 * kPanel64;        // W (also the workspace's copy) 64 x 128
+constexpr uint32_t R_P = R_W + 2 * kPanel64;        // P                  64 x 64
 constexpr uint32_t R_TB = R_P + kPanel64;           // T diag(beta)       64 x 64
 constexpr uint32_t R_PAD = R_TB + kPanel64;         // (rows 64-127 of the M = 128 reads of T diag(beta))
 constexpr uint32_t R_AF = R_PAD + kPanel64;         // A, f32             64 x 65
@@ -1035,9 +1046,9 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_prep_tc_kernel(Params p) {
             mma_commit(bar);
         }
         if (!products_done()) break;
-        // ---- epilogue 2 (lanes 0-63): W, U' out; -W and Z as bf16 operands
+        // ---- epilogue 2 (lanes 0-63): U' out (f32); W (bf16, the operand
+        //      layout the chains and the gradient step copy as is) and -Z
         if (lo) {
-            float* Wg = p.W + sh * kC * kD + (size_t)i * kD;
             float* Ug = p.Up + sh * kC * kD + (size_t)i * kD;
 #pragma unroll 1
             for (int cb = 0; cb < 2; ++cb) {
@@ -1045,28 +1056,29 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_prep_tc_kernel(Params p) {
                 float w[32], u[32];
                 tmem_ld32x2(tl + PT_W + c0, tl + PT_U + c0, w, u);
 #pragma unroll
-                for (int e4 = 0; e4 < 8; ++e4) {
-                    stf4(Wg + c0 + 4 * e4, w[4 * e4], w[4 * e4 + 1], w[4 * e4 + 2], w[4 * e4 + 3]);
+                for (int e4 = 0; e4 < 8; ++e4)
                     stf4(Ug + c0 + 4 * e4, u[4 * e4], u[4 * e4 + 1], u[4 * e4 + 2], u[4 * e4 + 3]);
-                }
 #pragma unroll
-                for (int e = 0; e < 32; ++e) w[e] = -w[e];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) put8(sm, R_NW, kPanel64, i, c0 / 8 + c, w + 8 * c);
+                for (int c = 0; c < 4; ++c) put8(sm, R_W, kPanel64, i, c0 / 8 + c, w + 8 * c);
                 float z[32];
                 tmem_ld32(tl + PT_Z + c0, z);
                 tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) z[e] = -z[e];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) put8(sm, R_Z, kPanel64, i, c0 / 8 + c, z + 8 * c);
             }
         }
         publish();
-        // ---- round 3: Y / scale = dO^T (diag(gam) Q) + Z^T (-W) (all 128 lanes: rows e)
+        // ---- round 3: Y / scale = dO^T (diag(gam) Q) + (-Z)^T W (all 128 lanes: rows e)
         if (issuer) {
             tc_fence_after();
             mma_run(tbase + PT_Y, sb + R_DO, kPanel64, true, sb + R_GQ, kPanel64, true, ID_MM128, 4, false);
-            mma_run(tbase + PT_Y, sb + R_Z, kPanel64, true, sb + R_NW, kPanel64, true, ID_MM128, 4, true);
+            mma_run(tbase + PT_Y, sb + R_Z, kPanel64, true, sb + R_W, kPanel64, true, ID_MM128, 4, true);
             mma_commit(bar);
+            // the W tile to the workspace (16 KB, read by the async proxy after the fence above)
+            bulk_store(p.W + sh * kC * kD, sb + R_W, 2 * kPanel64);
+            bulk_commit();
         }
         if (!products_done()) break;
         {
@@ -1086,6 +1098,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_prep_tc_kernel(Params p) {
         }
     } while (false);
 
+    if (tid == 0) bulk_wait();
     tc_fence_before();
     __syncthreads();
     if (*abort_flag) {
@@ -1107,31 +1120,30 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_prep_tc_kernel(Params p) {
 // One CTA of 8 warps per (sequence, value head).  The state (S forward, dS
 // backward; float32) stays in registers: thread (warp w, lane l) holds row
 // 32 (w % 4) + l, columns 64 (w / 4) .. + 64.  Per chunk, two products:
-//   forward   U^T = ...: X = W S^T (rows i; tokens), then
-//             U = kappa (U' - X) (bf16, rows i) and dS~ = U^T K;  S <- gamma_L S + dS~
+//   forward   X = W S^T (rows i = tokens), U = kappa (U' - X) (bf16),
+//             dS~ = U^T K;   S <- gamma_L S + dS~
 //   backward  X = K dS^T (rows i), X <- kappa X (bf16), dS~ = X^T W;
 //             dS <- gamma_L dS + Y - dS~
-// Both products use the bf16 state as the operand (the chain itself is carried
-// in float32).  The next chunk's K, W and U' (or Y) are fetched while the
-// current chunk's products run: K and U' / Y by cp.async straight into shared
-// memory, W through registers (converted to bf16).
+// Both products take the bf16 state as their operand; the chain itself is
+// carried in float32.  The chunk's state checkpoint is that bf16 operand tile,
+// written out by one bulk copy (the gradient step copies it back as is).  The
+// next chunk's operands are requested a whole chunk ahead: K, W (the
+// preparation's bf16 tile) and U' (forward) into the other half of double
+// buffers by cp.async, the decays through registers; Y (backward, 64 KB) by
+// cp.async at the start of the chunk that reads it at its end.
 constexpr uint32_t C_ST = 0;                        // the state, bf16       128 x 128
-constexpr uint32_t C_WT = C_ST + 2 * kPanel128;     // W, bf16               64 x 128
-constexpr uint32_t C_KT = C_WT + 2 * kPanel64;      // K, bf16               64 x 128
-constexpr uint32_t C_XT = C_KT + 2 * kPanel64;      // kappa U or kappa X    64 x 128
-constexpr uint32_t C_BUF = C_XT + 2 * kPanel64;     // U' (64 rows) or Y (128 rows), f32
+constexpr uint32_t C_WT = C_ST + 2 * kPanel128;     // W, bf16, 2 buffers    64 x 128
+constexpr uint32_t C_KT = C_WT + 4 * kPanel64;      // K, bf16, 2 buffers    64 x 128
+constexpr uint32_t C_XT = C_KT + 4 * kPanel64;      // kappa U or kappa X    64 x 128
+constexpr uint32_t C_BUF = C_XT + 2 * kPanel64;     // U' (2 buffers of 64 rows) or Y (128 rows), f32
 constexpr int kBufLd = 132;                         // floats per row (16-byte rows, conflict-free float4 reads)
-constexpr uint32_t C_MISC = C_BUF + 128 * kBufLd * 4;   // kappa [64], gamma_L
-constexpr uint32_t C_BAR = C_MISC + 80 * 4;         // mbarrier (8), TMEM base (4), abort flag (4)
+constexpr uint32_t kBufHalf = 64 * kBufLd * 4;
+constexpr uint32_t C_MISC = C_BUF + 2 * kBufHalf;   // kappa [64] and gamma_L, 2 buffers of 68
+constexpr uint32_t C_BAR = C_MISC + 2 * 68 * 4;     // mbarrier (8), TMEM base (4), abort flag (4)
 constexpr uint32_t CH_SMEM_ALLOC = C_BAR + 16 + 1024;
 static_assert(C_BAR % 8 == 0, "mbarrier alignment");
 constexpr uint32_t CT_X = 0, CT_D = 128, kChainTmemCols = 256;
 
-TC_DEVICE void cp_async16z(uint32_t dst, const void* src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-TC_DEVICE void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-TC_DEVICE void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 template <bool kBwd>
 __global__ void __launch_bounds__(kGThreads, 1) bwc_chain_tc_kernel(Params p) {
@@ -1160,11 +1172,12 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_chain_tc_kernel(Params p) {
     if (nch == 0) {
         if (kBwd && p.d_init) {
 #pragma unroll
-            for (int c4 = 0; c4 < 16; ++c4) stf4(p.d_init + unit + 4 * c4, st[4 * c4], st[4 * c4 + 1], st[4 * c4 + 2], st[4 * c4 + 3]);
+            for (int c4 = 0; c4 < 16; ++c4)
+                stf4(p.d_init + unit + 4 * c4, st[4 * c4], st[4 * c4 + 1], st[4 * c4 + 2], st[4 * c4 + 3]);
         }
         return;
     }
-    float* kap = reinterpret_cast<float*>(sm + C_MISC);
+    float* misc = reinterpret_cast<float*>(sm + C_MISC);
     const uint32_t bar = sb + C_BAR;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C_BAR + 8);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C_BAR + 12);
@@ -1180,58 +1193,51 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_chain_tc_kernel(Params p) {
 
     // chunk jj of the walk (backward: from the last)
     auto chunk_t0 = [&](int64_t jj) -> int64_t { return bos + (kBwd ? nch - 1 - jj : jj) * kC; };
-    auto chunk_len = [&](int64_t t0) -> int { return (int)((eos - t0) < kC ? (eos - t0) : kC); };
-    auto fetch_k = [&](int64_t t0) {
-        const int Lc = chunk_len(t0);
+    auto slot_of = [&](int64_t t0) -> size_t { return sh_index(p, t0 / kC + n, h); };
+    auto fetch_k = [&](int64_t t0, int b) {
+        const int Lc = (int)((eos - t0) < kC ? (eos - t0) : kC);
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
             const int it = tid + kGThreads * x, r = it >> 4, ch = it & 15;
             const bool ok = r < Lc;
             const uint16_t* src = ok ? p.k + ((size_t)(t0 + r) * p.Hqk + g) * kD + ch * 8 : p.k;
-            cp_async16z(sb + C_KT + (uint32_t)(ch >> 3) * kPanel64 + sw128_off(r, ch & 7), src, ok ? 16u : 0u);
+            cp_async16z(sb + C_KT + (uint32_t)b * 2 * kPanel64 + (uint32_t)(ch >> 3) * kPanel64 + sw128_off(r, ch & 7),
+                        src, ok ? 16u : 0u);
         }
     };
-    auto fetch_buf = [&](int64_t t0) {
-        const size_t sh = sh_index(p, t0 / kC + n, h);
+    // U' (forward, 64 rows, into buffer b) or Y (backward, 128 rows)
+    auto fetch_buf = [&](int64_t t0, int b) {
+        const size_t sh = slot_of(t0);
         const float* src = kBwd ? p.Y + sh * kD * kD : p.Up + sh * kC * kD;
+        const uint32_t base = sb + C_BUF + (kBwd ? 0u : (uint32_t)b * kBufHalf);
         constexpr int kItems = (kBwd ? 128 : 64) * 32 / kGThreads;
 #pragma unroll
         for (int x = 0; x < kItems; ++x) {
             const int it = tid + kGThreads * x, r = it >> 5, pc = it & 31;
-            cp_async16z(sb + C_BUF + (uint32_t)(r * kBufLd + 4 * pc) * 4u, src + (size_t)r * kD + 4 * pc, 16u);
+            cp_async16z(base + (uint32_t)(r * kBufLd + 4 * pc) * 4u, src + (size_t)r * kD + 4 * pc, 16u);
         }
     };
-    float4 wr[4][2];
-    auto load_w = [&](int64_t t0) {
-        const float* src = p.W + sh_index(p, t0 / kC + n, h) * kC * kD;
+    // W: the preparation's bf16 tile (16 KB, the shared-memory image) into buffer b
+    auto fetch_w = [&](int64_t t0, int b) {
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(p.W + slot_of(t0) * kC * kD);
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
-            const int it = tid + kGThreads * x, r = it >> 4, ch = it & 15;
-            wr[x][0] = ldf4(src + (size_t)r * kD + ch * 8);
-            wr[x][1] = ldf4(src + (size_t)r * kD + ch * 8 + 4);
+            const uint32_t off = (uint32_t)(tid + kGThreads * x) * 16u;
+            cp_async16z(sb + C_WT + (uint32_t)b * 2 * kPanel64 + off, src + off, 16u);
         }
     };
-    auto store_w = [&]() {
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const int it = tid + kGThreads * x, r = it >> 4, ch = it & 15;
-            st16(sm, C_WT, kPanel64, r, ch, pack8(wr[x][0], wr[x][1]));
-        }
-    };
-    auto load_gates = [&](int64_t t0) {
-        const size_t sh = sh_index(p, t0 / kC + n, h);
-        if (tid <= kC) kap[tid] = p.G[sh * (kC + 1) + tid];     // kappa_0..63, then gamma_L at [64]
-    };
+    // kappa_0..63 and gamma_L of a chunk (threads 0..64)
+    auto load_gate = [&](int64_t t0) -> float { return tid <= kC ? p.G[slot_of(t0) * (kC + 1) + tid] : 0.f; };
 
     // prologue: chunk 0's operands
     {
         const int64_t t0 = chunk_t0(0);
-        fetch_k(t0);
-        fetch_buf(t0);
+        fetch_k(t0, 0);
+        fetch_w(t0, 0);
+        if (!kBwd) fetch_buf(t0, 0);
         cp_async_commit();
-        load_w(t0);
-        store_w();
-        load_gates(t0);
+        const float gv = load_gate(t0);
+        if (tid <= kC) misc[tid] = gv;
     }
     __syncthreads();
     tc_fence_after();
@@ -1247,31 +1253,50 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_chain_tc_kernel(Params p) {
     };
 
     for (int64_t jj = 0; jj < nch; ++jj) {
+        const int b = (int)(jj & 1);
         const int64_t t0 = chunk_t0(jj);
-        const size_t sh = sh_index(p, t0 / kC + n, h);
+        const size_t sh = slot_of(t0);
         const bool more = jj + 1 < nch;
         const int64_t t0n = more ? chunk_t0(jj + 1) : t0;
-        // the state at this chunk's start (forward) or end (backward), kept for
-        // the gradient step, and as the bf16 operand
-        {
-            float* dst = (kBwd ? p.dS : p.S) + sh * kD * kD + (size_t)row * kD + 64 * hf;
-#pragma unroll
-            for (int c4 = 0; c4 < 16; ++c4) stf4(dst + 4 * c4, st[4 * c4], st[4 * c4 + 1], st[4 * c4 + 2], st[4 * c4 + 3]);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) put8(sm, C_ST, kPanel128, row, 8 * hf + j, st + 8 * j);
+        const float* kap = misc + 68 * b;
+        // requests for later: Y of this chunk (backward), the next chunk's K (and U')
+        if (kBwd) {
+            fetch_buf(t0, 0);
+            cp_async_commit();
         }
-        cp_async_wait_all();
+        if (more) {
+            fetch_k(t0n, b ^ 1);
+            fetch_w(t0n, b ^ 1);
+            if (!kBwd) fetch_buf(t0n, b ^ 1);
+            cp_async_commit();
+        }
+        const float gnext = more ? load_gate(t0n) : 0.f;
+        // the state at this chunk's start (forward) or end (backward) as the bf16
+        // operand (its previous bulk copy out has been read: see the end of the loop)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) put8(sm, C_ST, kPanel128, row, 8 * hf + j, st + 8 * j);
+        // this chunk's K (and U') have landed; the requests just made may be in flight
+        if (kBwd) {
+            if (more) cp_async_wait<2>();
+            else cp_async_wait<1>();
+        } else {
+            if (more) cp_async_wait<1>();
+            else cp_async_wait<0>();
+        }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
+        const uint32_t kt = sb + C_KT + (uint32_t)b * 2 * kPanel64;
+        const uint32_t wt = sb + C_WT + (uint32_t)b * 2 * kPanel64;
         if (tid == 0) {
             tc_fence_after();
             // X = W S^T (forward) or K dS^T (backward): rows i in TMEM lanes 0-63
-            mma_run(tbase + CT_X, sb + (kBwd ? C_KT : C_WT), kPanel64, false, sb + C_ST, kPanel128, false, ID_KK128,
-                    8, false);
+            mma_run(tbase + CT_X, kBwd ? kt : wt, kPanel64, false, sb + C_ST, kPanel128, false, ID_KK128, 8, false);
             mma_commit(bar);
+            // the state checkpoint: the bf16 operand tile (32 KB) to the workspace
+            bulk_store(kBwd ? p.dS + sh * kD * kD : p.S + sh * kD * kD, sb + C_ST, 2 * kPanel128);
+            bulk_commit();
         }
-        if (more) load_w(t0n);
         if (!products_done()) break;
         if (q < 2) {
             const int i = row;
@@ -1283,7 +1308,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_chain_tc_kernel(Params p) {
                 tmem_ld32(tl + CT_X + c0, x);
                 tmem_ld_wait();
                 if (!kBwd) {
-                    const float* up = reinterpret_cast<const float*>(sm + C_BUF) + i * kBufLd + c0;
+                    const float* up = reinterpret_cast<const float*>(sm + C_BUF + (uint32_t)b * kBufHalf) + i * kBufLd + c0;
 #pragma unroll
                     for (int e4 = 0; e4 < 8; ++e4) {
                         const float4 u4 = ldf4(up + 4 * e4);
@@ -1307,15 +1332,14 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_chain_tc_kernel(Params p) {
             tc_fence_after();
             // dS~ = (kappa U)^T K (forward) or (kappa X)^T W (backward): A and B
             // MN-major (rows = tokens)
-            mma_run(tbase + CT_D, sb + C_XT, kPanel64, true, sb + (kBwd ? C_WT : C_KT), kPanel64, true, ID_MM128, 4,
-                    false);
+            mma_run(tbase + CT_D, sb + C_XT, kPanel64, true, kBwd ? wt : kt, kPanel64, true, ID_MM128, 4, false);
             mma_commit(bar);
         }
-        // U' (forward) has been read; K (backward) is no longer read by the tensor core
-        if (more) {
-            if (kBwd) fetch_k(t0n);
-            else fetch_buf(t0n);
-            cp_async_commit();
+        if (kBwd) {
+            // this chunk's Y (the next chunk's K may still be in flight); the
+            // barrier in products_done makes every thread's part visible
+            if (more) cp_async_wait<1>();
+            else cp_async_wait<0>();
         }
         if (!products_done()) break;
         {
@@ -1342,22 +1366,20 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_chain_tc_kernel(Params p) {
                 }
             }
         }
+        // the state tile's copy out has been read before the next chunk rewrites it
+        if (tid == 0) bulk_wait_read();
         tc_fence_before();
         __syncthreads();
-        // every read of this chunk's operands is done: the next chunk's take their place
-        if (more) {
-            if (kBwd) fetch_buf(t0n);
-            else fetch_k(t0n);
-            cp_async_commit();
-            store_w();
-            load_gates(t0n);
-        }
+        // every read of this chunk's decays is done: the next chunk's take their place
+        if (more && tid <= kC) misc[68 * (b ^ 1) + tid] = gnext;
     }
     if (kBwd && p.d_init && *abort_flag == 0) {
 #pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) stf4(p.d_init + unit + 4 * c4, st[4 * c4], st[4 * c4 + 1], st[4 * c4 + 2], st[4 * c4 + 3]);
+        for (int c4 = 0; c4 < 16; ++c4)
+            stf4(p.d_init + unit + 4 * c4, st[4 * c4], st[4 * c4 + 1], st[4 * c4 + 2], st[4 * c4 + 3]);
     }
-    cp_async_wait_all();
+    cp_async_wait<0>();
+    if (tid == 0) bulk_wait();
     tc_fence_before();
     __syncthreads();
     if (*abort_flag) {
