@@ -16,6 +16,7 @@ from ._lib import (  # noqa: F401
     decode_step_gated,
     gated_norm,
     gated_norm_backward,
+    layer_prefill_host,
     lib,
     lib_path,
     prefill,

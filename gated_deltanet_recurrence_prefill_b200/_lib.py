@@ -34,6 +34,9 @@ SIGNATURES = {
     "gdn_prefill_bf16": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32, _i32,
                                    _f32, _vp, _vp, _vp, _vp, _sz, _vp]),
     "gdn_check_async": (C.c_int, [_vp, _vp, _vp]),
+    "gdn_layer_prefill_host_workspace_size": (_sz, [_i64, _i32, _i32, _i32, _i32]),
+    "gdn_layer_prefill_host": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i32, _i32, _i32, _f32,
+                                         _i32, _vp, _vp, _vp, _vp, _sz, _vp, _vp, _vp]),
     "gdn_prefill_noalloc": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i64, _i32, _i32,
                                       _i32, _f32, _vp, _vp, _vp, _vp]),
     "gdn_decode_step": (C.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
@@ -111,12 +114,14 @@ def _check(fn, status):
         raise GdnError(fn, status)
 
 
-def _need(t, dtype, shape, name):
+def _need(t, dtype, shape, name, device="cuda"):
     import torch
     if t is None:
         raise ValueError(f"{name} is required")
-    if not t.is_cuda:
+    if device == "cuda" and not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if device == "cpu" and t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
     if t.dtype != dtype:
         raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
     if tuple(t.shape) != tuple(shape):
@@ -280,6 +285,54 @@ def prefill(q, k, v, a, b, A_log, dt_bias, cu_seqlens=None, scale=None, initial_
             workspace.numel() * workspace.element_size(), _stream(stream))
     _check(name, st)
     return o, final_state
+
+
+_copy_streams = {}
+
+
+def layer_prefill_host(h_qkv, h_a, h_b, conv_w, A_log, dt_bias, Hqk, Hv, h_o=None, h_final_state=None,
+                       conv_state_in=None, initial_state=None, conv_state_out=None, n_blocks=8, scale=None,
+                       workspace=None, stream=None, copy_streams=None):
+    """gdn_layer_prefill_host: front end + prefill of one sequence from pinned
+    host tensors (h_qkv [T, (2Hqk+Hv)d] bf16, h_a, h_b [T, Hv] f32) to pinned
+    host tensors (h_o [T, Hv, d] f32, h_final_state [Hv, d, d] f32), the copies
+    overlapped with the compute over n_blocks token ranges.  conv_w, A_log,
+    dt_bias, conv_state_in / _out and initial_state are device tensors.
+    copy_streams: (upload, download) torch streams; by default two streams kept
+    per device.  Returns (h_o, h_final_state), ready once `stream` (default: the
+    current stream) reaches the point after the call."""
+    import torch
+    d = 128
+    T = h_qkv.shape[0]
+    dev = conv_w.device
+    _need(h_qkv, torch.bfloat16, (T, (2 * Hqk + Hv) * d), "h_qkv", device="cpu")
+    _need(h_a, torch.float32, (T, Hv), "h_a", device="cpu")
+    _need(h_b, torch.float32, (T, Hv), "h_b", device="cpu")
+    if h_o is None:
+        h_o = torch.empty(T, Hv, d, dtype=torch.float32).pin_memory()
+    if h_final_state is None:
+        h_final_state = torch.empty(Hv, d, d, dtype=torch.float32).pin_memory()
+    _need(h_o, torch.float32, (T, Hv, d), "h_o", device="cpu")
+    _need(h_final_state, torch.float32, (Hv, d, d), "h_final_state", device="cpu")
+    if scale is None:
+        scale = d ** -0.5
+    ws_bytes = lib().gdn_layer_prefill_host_workspace_size(T, Hqk, Hv, d, n_blocks)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    if copy_streams is None:
+        key = dev.index if dev.index is not None else torch.cuda.current_device()
+        if key not in _copy_streams:
+            _copy_streams[key] = (torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev))
+        copy_streams = _copy_streams[key]
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    st = lib().gdn_layer_prefill_host(
+        _ptr(h_qkv), _ptr(h_a), _ptr(h_b), _ptr(conv_w), _ptr(A_log), _ptr(dt_bias), _ptr(conv_state_in),
+        _ptr(initial_state), T, Hqk, Hv, d, float(scale), n_blocks, _ptr(h_o), _ptr(h_final_state),
+        _ptr(conv_state_out), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream),
+        _stream(copy_streams[0]), _stream(copy_streams[1]))
+    _check("gdn_layer_prefill_host", st)
+    return h_o, h_final_state
 
 
 def prefill_noalloc(q, k, v, a, b, A_log, dt_bias, cu_seqlens=None, scale=None,

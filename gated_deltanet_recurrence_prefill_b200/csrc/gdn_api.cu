@@ -54,6 +54,12 @@ PrefillKernel pick_prefill_kernel(size_t workspace_bytes) {
 }  // namespace
 
 namespace gdn {
+// for the entry points defined in other files
+gdn_status set_last_cuda_error(cudaError_t e) { return cuda_fail(e); }
+}  // namespace gdn
+
+
+namespace gdn {
 
 size_t prefill_min_workspace_bytes(int32_t n_seq, int32_t Hv) {
     const size_t n = n_seq > 0 ? (size_t)n_seq : 1;

@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/gdn.h"
+
 namespace gdn {
 
 struct PrefillArgs {
@@ -160,6 +162,8 @@ constexpr size_t kWsHeaderBytes = 256;
 // gdn_prefill_noalloc) on the current device, looked up once per device and
 // cached; null if the lookup fails.  Allocates nothing.
 void* noalloc_scratch();
+// records e for gdn_last_cuda_error and returns GDN_ERR_CUDA (gdn_api.cu)
+gdn_status set_last_cuda_error(cudaError_t e);
 size_t noalloc_scratch_bytes();
 
 }  // namespace gdn

@@ -29,6 +29,9 @@
  *    otherwise; the caller owns all memory.  The library never allocates,
  *    frees or synchronises, and enqueues all work on `stream` (NULL = the
  *    legacy default stream).  Results are ready when the stream reaches them.
+ *    (gdn_layer_prefill_host also uses two caller-given copy streams and
+ *    creates and releases CUDA events to order them; gdn_prefill_status waits
+ *    for its stream, as documented there.)
  *  - Types.  bf16 tensors are passed as uint16_t bit patterns.  Layouts are
  *    dense row-major in the order written; "[T, H, d]" means d is contiguous.
  *  - Alignment.  Every tensor pointer must be 16-byte aligned
@@ -221,6 +224,57 @@ gdn_status gdn_prefill_bf16(const uint16_t* q, const uint16_t* k, const uint16_t
                             int32_t Hv, int32_t d, float scale, const float* initial_state,
                             float* final_state, uint16_t* o, void* workspace, size_t workspace_bytes,
                             gdn_stream_t stream);
+
+/*
+ * gdn_layer_prefill_host_workspace_size -- bytes of device workspace that
+ * gdn_layer_prefill_host needs for T tokens cut into n_blocks ranges: a prefill
+ * workspace for one range (first, so that its error word is this workspace's
+ * first word), two input buffers of a range (qkv, a, b), q/k/v of a range, two
+ * output buffers of a range, two conv histories and two states.  0 for
+ * unsupported arguments.  Host-only.
+ */
+size_t gdn_layer_prefill_host_workspace_size(int64_t T, int32_t Hqk, int32_t Hv, int32_t d, int32_t n_blocks);
+
+/*
+ * gdn_layer_prefill_host -- gdn_conv1d_silu then gdn_prefill for one sequence,
+ * from HOST inputs to HOST outputs, with the host<->device copies overlapped
+ * with the compute (the operation is that of the two calls; architecture page
+ * sections 2.1 and 2.2).  The T tokens are cut into ranges of whole 64-token
+ * chunks (ceil(ceil(T / 64) / n_blocks) chunks each): range r's inputs are
+ * copied up on `upload_stream` into one of two device buffers; its front end
+ * (continuing range r-1's conv history) and prefill (continuing range r-1's
+ * state) run on `stream`; its output is copied down on `download_stream` from
+ * one of two output buffers.  Range r+1's upload and range r-1's download thus
+ * run while range r computes.  The result equals the two device calls on the
+ * whole sequence within the prefill's tolerance (the state is handed between
+ * ranges in float32; gdn_prefill's own chunking runs unchanged inside each).
+ *  h_qkv          [T, (2 Hqk + Hv) d] bf16, HOST (pinned: page-locked host
+ *                 memory is what lets the copies overlap)
+ *  h_a, h_b       [T, Hv] float32, HOST (pinned)
+ *  conv_w, A_log, dt_bias   device, as for gdn_conv1d_silu / gdn_prefill
+ *  conv_state_in  [(2 Hqk + Hv) d, 3] float32 device, or NULL (zero history)
+ *  initial_state  [Hv, d, d] float32 device, or NULL (zero state)
+ *  h_o            [T, Hv, d] float32, HOST (pinned), written
+ *  h_final_state  [Hv, d, d] float32, HOST (pinned), written
+ *  conv_state_out [(2 Hqk + Hv) d, 3] float32 device, or NULL
+ *  workspace      gdn_layer_prefill_host_workspace_size() bytes, 256-byte aligned
+ *  stream, upload_stream, download_stream: three distinct streams.
+ * The call only enqueues work and returns; everything it enqueues is ordered
+ * before work enqueued on `stream` afterwards (the host outputs are ready when
+ * `stream` reaches that point), and its device-side reads of the workspace wait
+ * for work enqueued on `stream` before the call.  It creates CUDA events for
+ * the ordering and releases them before returning (the driver keeps them until
+ * the work they mark completes); it allocates no memory.  n_blocks in
+ * [1, 4096].  Errors as for gdn_prefill; a timeout inside a range's prefill sets
+ * the workspace's error word (gdn_prefill_status / gdn_check_async on this
+ * workspace).  Supported: d = 128.
+ */
+gdn_status gdn_layer_prefill_host(const uint16_t* h_qkv, const float* h_a, const float* h_b, const float* conv_w,
+                                  const float* A_log, const float* dt_bias, const float* conv_state_in,
+                                  const float* initial_state, int64_t T, int32_t Hqk, int32_t Hv, int32_t d,
+                                  float scale, int32_t n_blocks, float* h_o, float* h_final_state,
+                                  float* conv_state_out, void* workspace, size_t workspace_bytes,
+                                  gdn_stream_t stream, gdn_stream_t upload_stream, gdn_stream_t download_stream);
 
 /*
  * gdn_prefill_status -- waits for `stream`, then reads the error word that the

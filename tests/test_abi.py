@@ -337,3 +337,30 @@ def test_prefill_bf16_rejects_bad_arguments(L):
     # misaligned output
     assert L.gdn_prefill_bf16(p, p, p, p, p, p, p, None, 1, 64, 16, 48, 128, 0.088, None, None, _p(FAKE + 2),
                               ws, 1 << 20, None) == 3
+
+
+def test_layer_prefill_host_rejects_bad_arguments_on_the_host(L):
+    """gdn_layer_prefill_host checks its arguments before touching CUDA."""
+    p = _p()
+    s0, s1, s2 = _p(0x1000), _p(0x2000), _p(0x3000)   # stand-in stream handles, never used
+
+    def call(qkv=p, T=256, d=128, nb=2, o=p, wsb=1 << 30, su=s1, sd=s2, ws=_p(0x40000)):
+        return L.gdn_layer_prefill_host(qkv, p, p, p, p, p, None, None, T, 2, 6, d, 0.088, nb, o, p, None,
+                                        ws, wsb, s0, su, sd)
+
+    assert call(d=64) == 2                  # unsupported head width
+    assert call(nb=0) == 1                  # no ranges
+    assert call(nb=5000) == 1               # too many ranges
+    assert call(qkv=None) == 1              # no input
+    assert call(o=None) == 1                # no output
+    assert call(su=s0) == 1                 # copy stream equal to the compute stream
+    assert call(sd=s1) == 1                 # the two copy streams equal
+    assert call(o=_p(FAKE + 4)) == 3        # misaligned
+    assert call(wsb=1024) == 6              # workspace too small
+    assert call(ws=_p(0x40010)) == 3        # workspace not 256-byte aligned
+    assert call(T=0) == 0                   # nothing to do
+    # the workspace formula: a prefill workspace of one range first, then the buffers
+    assert L.gdn_layer_prefill_host_workspace_size(256, 2, 6, 64, 2) == 0
+    n1 = L.gdn_layer_prefill_host_workspace_size(8192, 16, 48, 128, 8)
+    assert n1 > L.gdn_prefill_workspace_size(1, 1024, 16, 48, 128)
+    assert n1 % 256 == 0
