@@ -899,57 +899,68 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
         if (pw == 0 && lane == 0) TRACE_CLK(19, c);
         tc_fence_after();
         {
+            // eight columns at a time, the loop not unrolled (a smaller hot loop)
             const bool fast = gb.fast != 0;
-            float dv[32];
-            tmem_ld32(tl + PCOL_D0 + hh * 32, dv);
-            tmem_ld_wait();
             const int i_ = (q & 1) * 32 + lane;      // row within KK^T (q<2) or QK^T (q>=2)
             const float Gi = gb.G[i_];
             if (q < 2) {
                 // A_ij = beta_i 2^{G_i - G_j} (k_i . k_j), j < i
                 const float ci = fast ? gb.beta[i_] * gb.gamma[i_] : gb.beta[i_];
                 float* arow = Af + i_ * kLdF + hh * 32;
+#pragma unroll 1
+                for (int j8 = 0; j8 < 4; ++j8) {
+                    float dv[8];
+                    tmem_ld8(tl + PCOL_D0 + hh * 32 + j8 * 8, dv);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int j4 = 0; j4 < 32; j4 += 4) {
-                    const int j = hh * 32 + j4;
-                    float4 w;
-                    if (fast) {
-                        const float4 ig = *reinterpret_cast<const float4*>(&gb.igamma[j]);
-                        w.x = (j + 0 < i_) ? ci * dv[j4 + 0] * ig.x : 0.f;
-                        w.y = (j + 1 < i_) ? ci * dv[j4 + 1] * ig.y : 0.f;
-                        w.z = (j + 2 < i_) ? ci * dv[j4 + 2] * ig.z : 0.f;
-                        w.w = (j + 3 < i_) ? ci * dv[j4 + 3] * ig.w : 0.f;
-                    } else {
-                        const float4 gj = *reinterpret_cast<const float4*>(&gb.G[j]);
-                        w.x = (j + 0 < i_) ? ci * dv[j4 + 0] * exp2f(Gi - gj.x) : 0.f;
-                        w.y = (j + 1 < i_) ? ci * dv[j4 + 1] * exp2f(Gi - gj.y) : 0.f;
-                        w.z = (j + 2 < i_) ? ci * dv[j4 + 2] * exp2f(Gi - gj.z) : 0.f;
-                        w.w = (j + 3 < i_) ? ci * dv[j4 + 3] * exp2f(Gi - gj.w) : 0.f;
+                    for (int h4 = 0; h4 < 2; ++h4) {
+                        const int j4 = 4 * h4;
+                        const int j = hh * 32 + j8 * 8 + j4;
+                        float4 w;
+                        if (fast) {
+                            const float4 ig = *reinterpret_cast<const float4*>(&gb.igamma[j]);
+                            w.x = (j + 0 < i_) ? ci * dv[j4 + 0] * ig.x : 0.f;
+                            w.y = (j + 1 < i_) ? ci * dv[j4 + 1] * ig.y : 0.f;
+                            w.z = (j + 2 < i_) ? ci * dv[j4 + 2] * ig.z : 0.f;
+                            w.w = (j + 3 < i_) ? ci * dv[j4 + 3] * ig.w : 0.f;
+                        } else {
+                            const float4 gj = *reinterpret_cast<const float4*>(&gb.G[j]);
+                            w.x = (j + 0 < i_) ? ci * dv[j4 + 0] * exp2f(Gi - gj.x) : 0.f;
+                            w.y = (j + 1 < i_) ? ci * dv[j4 + 1] * exp2f(Gi - gj.y) : 0.f;
+                            w.z = (j + 2 < i_) ? ci * dv[j4 + 2] * exp2f(Gi - gj.z) : 0.f;
+                            w.w = (j + 3 < i_) ? ci * dv[j4 + 3] * exp2f(Gi - gj.w) : 0.f;
+                        }
+                        *reinterpret_cast<float4*>(arow + j8 * 8 + j4) = w;
                     }
-                    *reinterpret_cast<float4*>(arow + j4) = w;
                 }
             } else {
                 // P_ij = 2^{G_i - G_j} (q_i . k_j), j <= i
                 const float ci = fast ? gb.gamma[i_] : 1.f;
+#pragma unroll 1
+                for (int j8 = 0; j8 < 4; ++j8) {
+                    float dv[8];
+                    tmem_ld8(tl + PCOL_D0 + hh * 32 + j8 * 8, dv);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int j4 = 0; j4 < 32; j4 += 4) {
-                    const int j = hh * 32 + j4;
-                    if (fast) {
-                        const float4 ig = *reinterpret_cast<const float4*>(&gb.igamma[j]);
-                        dv[j4 + 0] = (j + 0 <= i_) ? ci * dv[j4 + 0] * ig.x : 0.f;
-                        dv[j4 + 1] = (j + 1 <= i_) ? ci * dv[j4 + 1] * ig.y : 0.f;
-                        dv[j4 + 2] = (j + 2 <= i_) ? ci * dv[j4 + 2] * ig.z : 0.f;
-                        dv[j4 + 3] = (j + 3 <= i_) ? ci * dv[j4 + 3] * ig.w : 0.f;
-                    } else {
-                        const float4 gj = *reinterpret_cast<const float4*>(&gb.G[j]);
-                        dv[j4 + 0] = (j + 0 <= i_) ? dv[j4 + 0] * exp2f(Gi - gj.x) : 0.f;
-                        dv[j4 + 1] = (j + 1 <= i_) ? dv[j4 + 1] * exp2f(Gi - gj.y) : 0.f;
-                        dv[j4 + 2] = (j + 2 <= i_) ? dv[j4 + 2] * exp2f(Gi - gj.z) : 0.f;
-                        dv[j4 + 3] = (j + 3 <= i_) ? dv[j4 + 3] * exp2f(Gi - gj.w) : 0.f;
+                    for (int h4 = 0; h4 < 2; ++h4) {
+                        const int j4 = 4 * h4;
+                        const int j = hh * 32 + j8 * 8 + j4;
+                        if (fast) {
+                            const float4 ig = *reinterpret_cast<const float4*>(&gb.igamma[j]);
+                            dv[j4 + 0] = (j + 0 <= i_) ? ci * dv[j4 + 0] * ig.x : 0.f;
+                            dv[j4 + 1] = (j + 1 <= i_) ? ci * dv[j4 + 1] * ig.y : 0.f;
+                            dv[j4 + 2] = (j + 2 <= i_) ? ci * dv[j4 + 2] * ig.z : 0.f;
+                            dv[j4 + 3] = (j + 3 <= i_) ? ci * dv[j4 + 3] * ig.w : 0.f;
+                        } else {
+                            const float4 gj = *reinterpret_cast<const float4*>(&gb.G[j]);
+                            dv[j4 + 0] = (j + 0 <= i_) ? dv[j4 + 0] * exp2f(Gi - gj.x) : 0.f;
+                            dv[j4 + 1] = (j + 1 <= i_) ? dv[j4 + 1] * exp2f(Gi - gj.y) : 0.f;
+                            dv[j4 + 2] = (j + 2 <= i_) ? dv[j4 + 2] * exp2f(Gi - gj.z) : 0.f;
+                            dv[j4 + 3] = (j + 3 <= i_) ? dv[j4 + 3] * exp2f(Gi - gj.w) : 0.f;
+                        }
                     }
+                    st_bf16x8(gbase + G_PT, i_, hh * 4 + j8, dv);
                 }
-#pragma unroll
-                for (int j = 0; j < 4; ++j) st_bf16x8(gbase + G_PT, i_, hh * 4 + j, dv + 8 * j);
             }
         }
         tc_fence_before();
@@ -1031,22 +1042,22 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
         tc_fence_after();
         {
             const int i_ = (q & 1) * 32 + lane;
-            float v[32];
-            if (q < 2) {
-                tmem_ld32(tl + PCOL_R + hh * 32, v);
-                tmem_ld_wait();
-            } else {
-#pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    const float4 t4 = *reinterpret_cast<const float4*>(Tf + i_ * kLdF + hh * 32 + j);
-                    v[j] = t4.x; v[j + 1] = t4.y; v[j + 2] = t4.z; v[j + 3] = t4.w;
-                }
-            }
             const int row = (q < 2 ? 0 : 64) + i_;     // [R bg; T bg]: R in rows 0-63
             const int row2 = (q < 2 ? 64 : 0) + i_;    // [T b; R b]: T in rows 0-63
-#pragma unroll
+            // eight columns at a time, the loop not unrolled (a smaller hot loop)
+#pragma unroll 1
             for (int j8 = 0; j8 < 4; ++j8) {
                 const int j0 = hh * 32 + j8 * 8;
+                float v8[8];
+                if (q < 2) {
+                    tmem_ld8(tl + PCOL_R + j0, v8);
+                    tmem_ld_wait();
+                } else {
+                    const float4 t0 = *reinterpret_cast<const float4*>(Tf + i_ * kLdF + j0);
+                    const float4 t1 = *reinterpret_cast<const float4*>(Tf + i_ * kLdF + j0 + 4);
+                    v8[0] = t0.x; v8[1] = t0.y; v8[2] = t0.z; v8[3] = t0.w;
+                    v8[4] = t1.x; v8[5] = t1.y; v8[6] = t1.z; v8[7] = t1.w;
+                }
                 const float4 b0 = *reinterpret_cast<const float4*>(&gb.beta[j0]);
                 const float4 b1 = *reinterpret_cast<const float4*>(&gb.beta[j0 + 4]);
                 const float4 g0 = *reinterpret_cast<const float4*>(&gb.gamma[j0]);
@@ -1056,7 +1067,7 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
                 float wb[8], wg[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    wb[e] = v[j8 * 8 + e] * bj[e];
+                    wb[e] = v8[e] * bj[e];
                     wg[e] = wb[e] * gj[e];
                 }
                 st_bf16x8(gbase + G_PT, row, hh * 4 + j8, wg);
@@ -1088,7 +1099,7 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
         {
             const int i_ = (q & 1) * 32 + lane;
             const float ga = gb.gamma[i_];
-#pragma unroll
+#pragma unroll 1
             for (int part = 0; part < 2; ++part) {
                 const int dcol = hh * 64 + part * 32;          // 32 of the 128 d columns
                 const int panel = dcol >> 6, ch0 = (dcol & 63) >> 3;
