@@ -77,3 +77,22 @@ def test_layer_prefill_host_rejects_bad_arguments():
     assert call(wsb=nbytes - 256) == 6           # workspace too small
     assert call(T=0) == 0                        # nothing to do
     assert L.gdn_layer_prefill_host_workspace_size(256, HQK, HV, 64, 2) == 0
+
+
+def test_layer_prefill_host_without_history_or_state(orc):
+    """No conv history in or out and no initial state: zero history, zero state."""
+    import torch
+    import gated_deltanet_recurrence_prefill_b200 as gdn
+    T = 700
+    fe = synth.make_frontend([T], seed=331, conv_state=False, init_state=False, Hqk=HQK, Hv=HV)
+    g = fe.gates
+    h_qkv = _host_bf16(fe.qkv)
+    h_a = torch.from_numpy(np.ascontiguousarray(g.a)).pin_memory()
+    h_b = torch.from_numpy(np.ascontiguousarray(g.b)).pin_memory()
+    h_o, h_fs = gdn.layer_prefill_host(h_qkv, h_a, h_b, dev_f32(fe.conv_w), dev_f32(g.A_log), dev_f32(g.dt_bias),
+                                       HQK, HV, n_blocks=3)
+    torch.cuda.synchronize()
+    rq, rk, rv, _ = orc.conv1d_silu(fe.qkv, fe.conv_w, None, HQK, HV, 128, None)
+    o_ref, s_ref = orc.prefill(rq, rk, rv, g.a, g.b, g.A_log, g.dt_bias, scale=g.scale)
+    assert rel_err(h_o.numpy(), o_ref) <= TOL
+    assert rel_err(h_fs.numpy(), s_ref[0]) <= TOL
