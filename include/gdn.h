@@ -513,12 +513,13 @@ size_t gdn_prefill_backward_chunked_workspace_size(int32_t n_seq, int64_t T, int
  * chunk end, dS_{c-1} = gam dS_c - (diag(kap) K dS_c^T)^T W + Y_c, whose
  * state-free term Y_c is computed for all chunks at once; everything else (dq,
  * dk, dv, the gates) is computed per (chunk, value head) in parallel.  The
- * chains and the per-chunk preparation run in float32 on the CUDA cores; the
- * per-chunk gradient step runs its products on the tensor cores (tcgen05, bf16
- * operands, float32 accumulation; the bf16 tensor-core prefill's tolerance,
- * 1e-2 relative to the largest reference element, applies), or in float32 on
- * the CUDA cores when the environment variable GDN_BACKWARD_GRAD=simt is set
- * (2e-3).  No atomics: the result is deterministic.
+ * per-chunk preparation, both chains and the per-chunk gradient step run their
+ * products on the tensor cores (tcgen05, bf16 operands, float32 accumulation;
+ * the chains carry the state in float32; the bf16 tensor-core prefill's
+ * tolerance, 1e-2 relative to the largest reference element, applies), or all
+ * in float32 on the CUDA cores when the environment variable
+ * GDN_BACKWARD_GRAD=simt is set (2e-3).  No atomics: the result is
+ * deterministic.
  * Arguments, layouts, outputs and errors as for gdn_prefill_backward, with the
  * workspace sized by gdn_prefill_backward_chunked_workspace_size().  The
  * tensor-core step waits (bounded, 2 s) for its products; if a wait gives up
