@@ -36,7 +36,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 T_MAIN = 8192
-E2E_BLOCKS = 4          # token ranges of the end-to-end call (2048 tokens each at T = 8192)
+E2E_BLOCKS = 6          # token ranges of the end-to-end call (448 tokens, then 1600 each, at T = 8192)
 T_LONG = 262144
 HQK, HV, D = 16, 48, 128
 # algorithmic work per token per layer (chunked form, C = 64): 48 value heads x

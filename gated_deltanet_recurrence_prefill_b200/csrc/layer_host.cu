@@ -2,7 +2,10 @@
 // layer from pinned host inputs to pinned host outputs, with the PCIe copies
 // overlapped with the compute.
 //
-// The tokens are cut into ranges of whole 64-token chunks.  Range r's inputs go
+// The tokens are cut into ranges of whole 64-token chunks, the first of them a
+// quarter as long as the others so that the first download starts early (the
+// downloads, 24.6 KB per token against 20.9 KB up, are the longer direction).
+// Range r's inputs go
 // up on the upload stream into one of two device buffers, its front end and
 // prefill run on the caller's stream (the front end continues range r-1's
 // conv history, the prefill range r-1's state: gdn_conv1d_silu's
@@ -22,17 +25,37 @@
 namespace {
 
 struct HostPlan {
-    int64_t Tb;                // tokens per range (a multiple of 64)
+    int64_t first;             // tokens of range 0 (a multiple of 64, or T)
+    int64_t Tb;                // tokens of each later range (a multiple of 64): the buffers' size
     size_t pws, qkv, ab, qk, v, o, cs, st, bytes;   // byte offsets into the workspace
 };
+
+// token range r of the plan: [*t0, *t0 + *len)
+void host_range(const HostPlan& p, int64_t T, int64_t r, int64_t* t0, int64_t* len) {
+    const int64_t s = r == 0 ? 0 : p.first + (r - 1) * p.Tb;
+    const int64_t n = r == 0 ? p.first : p.Tb;
+    *t0 = s;
+    *len = (T - s) < n ? (T - s) : n;
+}
 
 size_t up256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 bool make_host_plan(int64_t T, int32_t Hqk, int32_t Hv, int32_t d, int32_t n_blocks, HostPlan& p) {
     if (T <= 0 || n_blocks <= 0) return false;
     const int64_t chunks = (T + 63) / 64;
-    const int64_t per = (chunks + n_blocks - 1) / n_blocks;
-    p.Tb = per * 64;
+    if (n_blocks == 1 || chunks < 2) {
+        p.first = p.Tb = chunks * 64;
+    } else {
+        // range 0 takes a quarter share, the other n_blocks - 1 ranges the rest
+        const int64_t share = (4 * chunks + 4 * n_blocks - 3 - 1) / (4 * n_blocks - 3);   // ceil(chunks / (n - 3/4))
+        int64_t f = (share + 3) / 4;
+        if (f < 1) f = 1;
+        if (f > chunks - 1) f = chunks - 1;
+        const int64_t rest = chunks - f;
+        p.first = f * 64;
+        p.Tb = ((rest + n_blocks - 2) / (n_blocks - 1)) * 64;
+        if (p.Tb < p.first) p.Tb = p.first;
+    }
     const size_t C = (size_t)(2 * Hqk + Hv) * d;
     size_t off = 0;
     // the prefill's workspace first: its error word is the first word of this one
@@ -86,7 +109,7 @@ gdn_status gdn_layer_prefill_host(const uint16_t* h_qkv, const float* h_a, const
     cudaStream_t s0 = (cudaStream_t)stream, su = (cudaStream_t)upload_stream, sd = (cudaStream_t)download_stream;
     char* ws = static_cast<char*>(workspace);
     const size_t C = (size_t)(2 * Hqk + Hv) * d;
-    const int64_t nb = (T + pl.Tb - 1) / pl.Tb;
+    const int64_t nb = 1 + (T > pl.first ? (T - pl.first + pl.Tb - 1) / pl.Tb : 0);
     auto qkv_buf = [&](int b) { return reinterpret_cast<uint16_t*>(ws + pl.qkv + b * up256((size_t)pl.Tb * C * 2)); };
     auto ab_buf = [&](int i) { return reinterpret_cast<float*>(ws + pl.ab + i * up256((size_t)pl.Tb * Hv * 4)); };
     uint16_t* qb = reinterpret_cast<uint16_t*>(ws + pl.qk);
@@ -119,8 +142,8 @@ gdn_status gdn_layer_prefill_host(const uint16_t* h_qkv, const float* h_a, const
     if (e == cudaSuccess) e = cudaStreamWaitEvent(sd, ev_start, 0);
     for (int64_t r = 0; r < nb && e == cudaSuccess && status == GDN_OK; ++r) {
         const int b = (int)(r & 1);
-        const int64_t t0 = r * pl.Tb;
-        const int64_t L = (T - t0) < pl.Tb ? (T - t0) : pl.Tb;
+        int64_t t0, L;
+        host_range(pl, T, r, &t0, &L);
         // upload: buffer b is free once range r - 2 has been computed
         if (r >= 2) e = cudaStreamWaitEvent(su, ev_comp(r - 2), 0);
         if (e == cudaSuccess)

@@ -239,8 +239,9 @@ size_t gdn_layer_prefill_host_workspace_size(int64_t T, int32_t Hqk, int32_t Hv,
  * gdn_layer_prefill_host -- gdn_conv1d_silu then gdn_prefill for one sequence,
  * from HOST inputs to HOST outputs, with the host<->device copies overlapped
  * with the compute (the operation is that of the two calls; architecture page
- * sections 2.1 and 2.2).  The T tokens are cut into ranges of whole 64-token
- * chunks (ceil(ceil(T / 64) / n_blocks) chunks each): range r's inputs are
+ * sections 2.1 and 2.2).  The T tokens are cut into n_blocks ranges of whole
+ * 64-token chunks, the first a quarter as long as the others (so that the first
+ * download, the longer copy direction, starts early): range r's inputs are
  * copied up on `upload_stream` into one of two device buffers; its front end
  * (continuing range r-1's conv history) and prefill (continuing range r-1's
  * state) run on `stream`; its output is copied down on `download_stream` from
