@@ -8,7 +8,7 @@
 // shared memory with the 128-byte swizzle, float32 accumulators in TMEM), and
 // the element-wise parts between the products (causal masks, decays, the row
 // and column sums of the gate gradients) run on the CUDA cores.  One CTA of 8
-// warps per (chunk, value head); the products come in seven rounds, each issued
+// warps per (chunk, value head); the products come in seven phases, each issued
 // by one thread once the operands it needs are in shared memory:
 //
 //   1. D0 = [Q; K] K^T, [W; Q] S^T, K dS^T        -> P, U = U' - W S^T, kappa U,
@@ -348,7 +348,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
     };
 
     do {
-        // ---- round 1
+        // ---- phase 1
         if (issuer) {
             tc_fence_after();
             // D0 = [Q; K] K^T: lanes 0-63 Q K^T, 64-127 K K^T
@@ -435,7 +435,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
         }
         publish();
 
-        // ---- round 2: P^T dO (lanes 0-63)
+        // ---- phase 2: P^T dO (lanes 0-63)
         if (issuer) {
             tc_fence_after();
             mma_run(tbase + T_C3, sb + S_P, kPanel64, true, sb + S_DUO, kPanel128, true, ID_MM128, 4, false);
@@ -462,7 +462,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
         }
         publish();
 
-        // ---- round 3
+        // ---- phase 3
         if (issuer) {
             tc_fence_after();
             // [dO; dU] S: lanes 0-63 dO S, 64-127 dU S (= -dW)
@@ -522,7 +522,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
 #pragma unroll
                 for (int j8 = 0; j8 < 4; ++j8) put8(sm, S_DW, kPanel128, 64 + i, c0 / 8 + j8, v + 8 * j8);
             }
-            // T diag(beta) and T diag(beta gam) (over kappa U, read by round 3)
+            // T diag(beta) and T diag(beta gam) (over kappa U, read by phase 3)
             const int ht = 64 * hf + 32 * (q - 2) + lane;
             const float* Tg = p.Tm + sh * kC * kC;
 #pragma unroll
@@ -542,7 +542,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
         }
         publish();
 
-        // ---- round 4
+        // ---- phase 4
         if (issuer) {
             tc_fence_after();
             // dq += M1 K (lanes 0-63; lanes 64-127 held dU S, already read)
@@ -584,7 +584,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
         }
         publish();
 
-        // ---- round 5
+        // ---- phase 5
         if (issuer) {
             tc_fence_after();
             // dv = (T diag(beta))^T dU (lanes 0-63)
@@ -620,7 +620,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
         }
         publish();
 
-        // ---- round 6: M2 T^T (lanes 64-127)
+        // ---- phase 6: M2 T^T (lanes 64-127)
         if (issuer) {
             tc_fence_after();
             mma_run(tbase + T_C4, sb + S_M2, kPanel64, false, sb + S_T, kPanel64, false, ID_KK64, 4, false);
@@ -663,7 +663,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
         }
         publish();
 
-        // ---- round 7: dk += (E + E^T) K
+        // ---- phase 7: dk += (E + E^T) K
         if (issuer) {
             tc_fence_after();
             mma_run(tbase + T_C3, sb + S_ES, kPanel64, false, sb + S_KQW + 16384, kPanel192, true, ID_KM128, 4,
@@ -761,12 +761,12 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_grad_tc_kernel(Params p) {
 // ---- the per-chunk preparation on the tensor cores ---------------------------------------
 // One CTA of 8 warps per (chunk, value head): the quantities the chains and the
 // gradient step read, as prep_block in backward_chunked.cuh computes them:
-//   round 1  D0 = [Q; K] K^T                 -> P = lower(Gamma o Q K^T) (bf16),
+//   phase 1  D0 = [Q; K] K^T                 -> P = lower(Gamma o Q K^T) (bf16),
 //                                               A = diag(beta) strict_lower(Gamma o K K^T) (f32)
 //   solve    T = (I + A)^{-1}: 16 x 16 diagonal blocks by forward substitution,
 //            then 32 x 32 and 64 x 64 by T10 = -T11 A10 T00 (float32, CUDA cores)
-//   round 2  W = (T diag(beta)) (diag(gam) K), U' = (T diag(beta)) V, Z = P^T dO
-//   round 3  Y / scale = dO^T (diag(gam) Q) - Z^T W
+//   phase 2  W = (T diag(beta)) (diag(gam) K), U' = (T diag(beta)) V, Z = P^T dO
+//   phase 3  Y / scale = dO^T (diag(gam) Q) - Z^T W
 constexpr uint32_t R_QK = 0;                        // [Q; K]             128 x 128
 constexpr uint32_t R_V = R_QK + 2 * kPanel128;      // V                  64 x 128
 constexpr uint32_t R_DO = R_V + 2 * kPanel64;       // dO (bf16)          64 x 128
@@ -900,7 +900,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_prep_tc_kernel(Params p) {
     };
 
     do {
-        // ---- round 1: D0 = [Q; K] K^T (lanes 0-63 Q K^T, 64-127 K K^T)
+        // ---- phase 1: D0 = [Q; K] K^T (lanes 0-63 Q K^T, 64-127 K K^T)
         if (issuer) {
             tc_fence_after();
             mma_run(tbase + PT_D0, sb + R_QK, kPanel128, false, sb + R_QK + 8192, kPanel128, false, ID_KK64, 8,
@@ -1037,7 +1037,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_prep_tc_kernel(Params p) {
             if (tid <= kC) p.G[sh * (kC + 1) + tid] = tid < kC ? kap[tid] : gam[L - 1];
         }
         publish();
-        // ---- round 2: W, U' (A = T diag(beta), K-major), Z = P^T dO (lanes 0-63)
+        // ---- phase 2: W, U' (A = T diag(beta), K-major), Z = P^T dO (lanes 0-63)
         if (issuer) {
             tc_fence_after();
             mma_run(tbase + PT_W, sb + R_TB, kPanel64, false, sb + R_GK, kPanel64, true, ID_KM128, 4, false);
@@ -1070,7 +1070,7 @@ __global__ void __launch_bounds__(kGThreads, 1) bwc_prep_tc_kernel(Params p) {
             }
         }
         publish();
-        // ---- round 3: Y / scale = dO^T (diag(gam) Q) + (-Z)^T W (all 128 lanes: rows e)
+        // ---- phase 3: Y / scale = dO^T (diag(gam) Q) + (-Z)^T W (all 128 lanes: rows e)
         if (issuer) {
             tc_fence_after();
             mma_run(tbase + PT_Y, sb + R_DO, kPanel64, true, sb + R_GQ, kPanel64, true, ID_MM128, 4, false);
