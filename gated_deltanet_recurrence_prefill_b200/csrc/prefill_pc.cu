@@ -903,63 +903,91 @@ __device__ __forceinline__ void producer(const Ctx& x, int pidx, const CUtensorM
             const bool fast = gb.fast != 0;
             const int i_ = (q & 1) * 32 + lane;      // row within KK^T (q<2) or QK^T (q>=2)
             const float Gi = gb.G[i_];
+            // (the fast and the slow decay forms in separate loops, so that the loop that
+            // runs holds one of them)
             if (q < 2) {
                 // A_ij = beta_i 2^{G_i - G_j} (k_i . k_j), j < i
-                const float ci = fast ? gb.beta[i_] * gb.gamma[i_] : gb.beta[i_];
                 float* arow = Af + i_ * kLdF + hh * 32;
+                if (fast) {
+                    const float ci = gb.beta[i_] * gb.gamma[i_];
 #pragma unroll 1
-                for (int j8 = 0; j8 < 4; ++j8) {
-                    float dv[8];
-                    tmem_ld8(tl + PCOL_D0 + hh * 32 + j8 * 8, dv);
-                    tmem_ld_wait();
+                    for (int j8 = 0; j8 < 4; ++j8) {
+                        float dv[8];
+                        tmem_ld8(tl + PCOL_D0 + hh * 32 + j8 * 8, dv);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int h4 = 0; h4 < 2; ++h4) {
-                        const int j4 = 4 * h4;
-                        const int j = hh * 32 + j8 * 8 + j4;
-                        float4 w;
-                        if (fast) {
+                        for (int h4 = 0; h4 < 2; ++h4) {
+                            const int j4 = 4 * h4;
+                            const int j = hh * 32 + j8 * 8 + j4;
                             const float4 ig = *reinterpret_cast<const float4*>(&gb.igamma[j]);
+                            float4 w;
                             w.x = (j + 0 < i_) ? ci * dv[j4 + 0] * ig.x : 0.f;
                             w.y = (j + 1 < i_) ? ci * dv[j4 + 1] * ig.y : 0.f;
                             w.z = (j + 2 < i_) ? ci * dv[j4 + 2] * ig.z : 0.f;
                             w.w = (j + 3 < i_) ? ci * dv[j4 + 3] * ig.w : 0.f;
-                        } else {
+                            *reinterpret_cast<float4*>(arow + j8 * 8 + j4) = w;
+                        }
+                    }
+                } else {
+                    const float ci = gb.beta[i_];
+#pragma unroll 1
+                    for (int j8 = 0; j8 < 4; ++j8) {
+                        float dv[8];
+                        tmem_ld8(tl + PCOL_D0 + hh * 32 + j8 * 8, dv);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int h4 = 0; h4 < 2; ++h4) {
+                            const int j4 = 4 * h4;
+                            const int j = hh * 32 + j8 * 8 + j4;
                             const float4 gj = *reinterpret_cast<const float4*>(&gb.G[j]);
+                            float4 w;
                             w.x = (j + 0 < i_) ? ci * dv[j4 + 0] * exp2f(Gi - gj.x) : 0.f;
                             w.y = (j + 1 < i_) ? ci * dv[j4 + 1] * exp2f(Gi - gj.y) : 0.f;
                             w.z = (j + 2 < i_) ? ci * dv[j4 + 2] * exp2f(Gi - gj.z) : 0.f;
                             w.w = (j + 3 < i_) ? ci * dv[j4 + 3] * exp2f(Gi - gj.w) : 0.f;
+                            *reinterpret_cast<float4*>(arow + j8 * 8 + j4) = w;
                         }
-                        *reinterpret_cast<float4*>(arow + j8 * 8 + j4) = w;
                     }
                 }
             } else {
                 // P_ij = 2^{G_i - G_j} (q_i . k_j), j <= i
-                const float ci = fast ? gb.gamma[i_] : 1.f;
+                if (fast) {
+                    const float ci = gb.gamma[i_];
 #pragma unroll 1
-                for (int j8 = 0; j8 < 4; ++j8) {
-                    float dv[8];
-                    tmem_ld8(tl + PCOL_D0 + hh * 32 + j8 * 8, dv);
-                    tmem_ld_wait();
+                    for (int j8 = 0; j8 < 4; ++j8) {
+                        float dv[8];
+                        tmem_ld8(tl + PCOL_D0 + hh * 32 + j8 * 8, dv);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int h4 = 0; h4 < 2; ++h4) {
-                        const int j4 = 4 * h4;
-                        const int j = hh * 32 + j8 * 8 + j4;
-                        if (fast) {
+                        for (int h4 = 0; h4 < 2; ++h4) {
+                            const int j4 = 4 * h4;
+                            const int j = hh * 32 + j8 * 8 + j4;
                             const float4 ig = *reinterpret_cast<const float4*>(&gb.igamma[j]);
                             dv[j4 + 0] = (j + 0 <= i_) ? ci * dv[j4 + 0] * ig.x : 0.f;
                             dv[j4 + 1] = (j + 1 <= i_) ? ci * dv[j4 + 1] * ig.y : 0.f;
                             dv[j4 + 2] = (j + 2 <= i_) ? ci * dv[j4 + 2] * ig.z : 0.f;
                             dv[j4 + 3] = (j + 3 <= i_) ? ci * dv[j4 + 3] * ig.w : 0.f;
-                        } else {
+                        }
+                        st_bf16x8(gbase + G_PT, i_, hh * 4 + j8, dv);
+                    }
+                } else {
+#pragma unroll 1
+                    for (int j8 = 0; j8 < 4; ++j8) {
+                        float dv[8];
+                        tmem_ld8(tl + PCOL_D0 + hh * 32 + j8 * 8, dv);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int h4 = 0; h4 < 2; ++h4) {
+                            const int j4 = 4 * h4;
+                            const int j = hh * 32 + j8 * 8 + j4;
                             const float4 gj = *reinterpret_cast<const float4*>(&gb.G[j]);
                             dv[j4 + 0] = (j + 0 <= i_) ? dv[j4 + 0] * exp2f(Gi - gj.x) : 0.f;
                             dv[j4 + 1] = (j + 1 <= i_) ? dv[j4 + 1] * exp2f(Gi - gj.y) : 0.f;
                             dv[j4 + 2] = (j + 2 <= i_) ? dv[j4 + 2] * exp2f(Gi - gj.z) : 0.f;
                             dv[j4 + 3] = (j + 3 <= i_) ? dv[j4 + 3] * exp2f(Gi - gj.w) : 0.f;
                         }
+                        st_bf16x8(gbase + G_PT, i_, hh * 4 + j8, dv);
                     }
-                    st_bf16x8(gbase + G_PT, i_, hh * 4 + j8, dv);
                 }
             }
         }
