@@ -587,18 +587,19 @@ __device__ __forceinline__ void consumer(const Ctx& x, const CUtensorMap* tm_k, 
                         if (j < nvalid) ocol[j * o_stride] = ov[j];
                 }
             } else if (p.o16) {
-                // bf16 o: lanes l and l ^ 1 hold rows v and v ^ 1; they swap one
-                // value per token pair so that each writes one 4-byte word of the
-                // two rows (even lanes the even tokens, odd lanes the odd ones)
+                // bf16 o: each lane packs its tokens j, j + 1; lanes l and l ^ 1 (rows v and
+                // v ^ 1) swap the packed words, and each assembles one 4-byte word of
+                // the two rows (even lanes token j, odd lanes token j + 1)
                 const bool odd = lane & 1;
+                const uint32_t sel = odd ? 0x3276u : 0x5410u;
                 uint32_t* orow2 = reinterpret_cast<uint32_t*>(p.o16 + t0 * o_stride + x.h * kD + (v & ~1));
                 const int64_t wstride = o_stride / 2;
 #pragma unroll
                 for (int j = 0; j < 16; j += 2) {
-                    const float other = __shfl_xor_sync(0xffffffffu, odd ? ov[j] : ov[j + 1], 1);
+                    const uint32_t own = pack_bf16x2(ov[j], ov[j + 1]);
+                    const uint32_t other = __shfl_xor_sync(0xffffffffu, own, 1);
                     const int jt = odd ? j + 1 : j;
-                    const uint32_t w = odd ? pack_bf16x2(other, ov[j + 1]) : pack_bf16x2(ov[j], other);
-                    if (jt < nvalid) orow2[jt * wstride] = w;
+                    if (jt < nvalid) orow2[jt * wstride] = __byte_perm(own, other, sel);
                 }
             }
             Gam = resc ? 1.f : Gn;
